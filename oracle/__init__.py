@@ -1,0 +1,267 @@
+"""CPU oracle for the W4A8 Integer-Scale linear layer (TEST INFRASTRUCTURE).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never calls it and shares no code with it.
+
+The arithmetic lives in ``oracle.c`` (plain scalar C, int64 accumulation, fp64
+results); this module compiles it with gcc on first use (or ``build()``) and
+wraps each function with numpy marshalling.  Every function cites the passage
+it follows in the C source.  Two small steps are written here in numpy because
+they are plain definitions: the unquantized fp64 matmul ``x @ w`` used as the
+accuracy reference, and rounding an fp64 result to the output type.
+
+Parity status per function (what pins it, see tests/test_oracle_pins.py):
+  quantize_rows / quantize_groups  brute-force nearest-code search, tie cases,
+                                   round-trip error bound |x - s q| <= s/2,
+                                   error variance ~ s^2/12, hand-worked goldens
+  pack_int4 / unpack_int4          exhaustive nibble round trip, hand-packed bytes
+  amplifier_search                 postcondition (min scale * alpha >= 1 and
+                                   minimal), frexp closed form, hand-worked goldens
+  integer_scales                   |S - s*alpha| <= 1/2, exact at representable values
+  intscale_acc                     equals the expanded-W_int form, numpy int64
+                                   matmul when S is constant over groups, brute
+                                   fp64 dequantized matmul on tiny inputs, X=0,
+                                   one-hot columns
+  floatscale                       equals the per-channel outer-product dequant
+                                   when group = K; equals intscale when s_g*alpha
+                                   is an integer
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+INT8_QMAX = 127
+INT4_QMAX = 7
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so with plain IEEE floating point."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = [
+            "gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+            "-ffp-contract=off", "-o", _LIB, _SRC, "-lm",
+        ]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            I = ctypes.c_int64
+            I32 = ctypes.c_int32
+            sig = {
+                "oracle_quantize_rows": ([P, I, I, I32, P, P], None),
+                "oracle_quantize_groups": ([P, I, I, I, I32, P, P], None),
+                "oracle_pack_int4": ([P, I, I, P], None),
+                "oracle_unpack_int4": ([P, I, I, P], None),
+                "oracle_amplifier_search": ([P, I], I32),
+                "oracle_integer_scales": ([P, I, I32, P], None),
+                "oracle_intscale_acc": ([P, P, P, I, I, I, I, P], None),
+                "oracle_intscale_acc_expanded": ([P, P, P, I, I, I, I, P], None),
+                "oracle_intscale_acc_at": ([P, P, P, I, I, I, I, P, P, I, P], None),
+                "oracle_intscale_output": ([P, P, I32, I, I, P], None),
+                "oracle_floatscale": ([P, P, P, P, I, I, I, I, P], None),
+                "oracle_floatscale_at": ([P, P, P, P, I, I, I, I, P, P, I, P], None),
+                "oracle_scale_colsum_max": ([P, I, I], I),
+            }
+            for name, (args, res) in sig.items():
+                f = getattr(lib, name)
+                f.argtypes = args
+                f.restype = res
+            _lib = lib
+    return _lib
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# ---------------------------------------------------------------- quantizers
+
+def quantize_rows(x, qmax: int = INT8_QMAX):
+    """Per-row symmetric quantization: returns (q int8 [R,C], s float32 [R])."""
+    x = _c(x, np.float32)
+    R, C = x.shape
+    q = np.empty((R, C), np.int8)
+    s = np.empty(R, np.float32)
+    _load().oracle_quantize_rows(_p(x), R, C, qmax, _p(q), _p(s))
+    return q, s
+
+
+def quantize_act_per_token(x):
+    """Per-token int8 activation codes and scales (qmax = 127)."""
+    return quantize_rows(x, INT8_QMAX)
+
+
+def quantize_groups(w, group: int = 128, qmax: int = INT4_QMAX):
+    """Per-(group, column) symmetric quantization of w [K,N]: (q int8 [K,N], s_g float32 [K/group,N])."""
+    w = _c(w, np.float32)
+    K, N = w.shape
+    if K % group:
+        raise ValueError("K must be a multiple of group")
+    q = np.empty((K, N), np.int8)
+    s = np.empty((K // group, N), np.float32)
+    _load().oracle_quantize_groups(_p(w), K, N, group, qmax, _p(q), _p(s))
+    return q, s
+
+
+def pack_int4(q):
+    """Codes q [K,N] in [-8,7] -> packed uint8 [N, K/2]."""
+    q = _c(q, np.int8)
+    K, N = q.shape
+    out = np.empty((N, K // 2), np.uint8)
+    _load().oracle_pack_int4(_p(q), K, N, _p(out))
+    return out
+
+
+def unpack_int4(packed, K: int, N: int):
+    packed = _c(packed, np.uint8)
+    out = np.empty((K, N), np.int8)
+    _load().oracle_unpack_int4(_p(packed), K, N, _p(out))
+    return out
+
+
+def amplifier_search(scales) -> int:
+    s = _c(np.ravel(scales), np.float32)
+    return int(_load().oracle_amplifier_search(_p(s), s.size))
+
+
+def integer_scales(s_g, alpha: int):
+    s = _c(s_g, np.float32)
+    out = np.empty(s.shape, np.int32)
+    _load().oracle_integer_scales(_p(s), s.size, int(alpha), _p(out))
+    return out
+
+
+def scale_colsum_max(S) -> int:
+    S = _c(S, np.int32)
+    G, N = S.shape
+    return int(_load().oracle_scale_colsum_max(_p(S), G, N))
+
+
+# ---------------------------------------------------------------- GEMMs
+
+def intscale_acc(qx, qw, S, group: int = 128):
+    qx = _c(qx, np.int8)
+    qw = _c(qw, np.int8)
+    S = _c(S, np.int32)
+    M, K = qx.shape
+    N = qw.shape[1]
+    acc = np.empty((M, N), np.int64)
+    _load().oracle_intscale_acc(_p(qx), _p(qw), _p(S), M, N, K, group, _p(acc))
+    return acc
+
+
+def intscale_acc_expanded(qx, qw, S, group: int = 128):
+    qx = _c(qx, np.int8)
+    qw = _c(qw, np.int8)
+    S = _c(S, np.int32)
+    M, K = qx.shape
+    N = qw.shape[1]
+    acc = np.empty((M, N), np.int64)
+    _load().oracle_intscale_acc_expanded(_p(qx), _p(qw), _p(S), M, N, K, group, _p(acc))
+    return acc
+
+
+def intscale_acc_at(qx, qw, S, ms, ns, group: int = 128):
+    qx = _c(qx, np.int8)
+    qw = _c(qw, np.int8)
+    S = _c(S, np.int32)
+    ms = _c(ms, np.int64)
+    ns = _c(ns, np.int64)
+    M, K = qx.shape
+    N = qw.shape[1]
+    acc = np.empty(ms.size, np.int64)
+    _load().oracle_intscale_acc_at(_p(qx), _p(qw), _p(S), M, N, K, group, _p(ms), _p(ns), ms.size, _p(acc))
+    return acc
+
+
+def intscale_output(acc, s_a, alpha: int):
+    acc = _c(acc, np.int64)
+    s_a = _c(s_a, np.float32)
+    M, N = acc.shape
+    y = np.empty((M, N), np.float64)
+    _load().oracle_intscale_output(_p(acc), _p(s_a), int(alpha), M, N, _p(y))
+    return y
+
+
+def floatscale(qx, s_a, qw, s_g, group: int = 128):
+    qx = _c(qx, np.int8)
+    s_a = _c(s_a, np.float32)
+    qw = _c(qw, np.int8)
+    s_g = _c(s_g, np.float32)
+    M, K = qx.shape
+    N = qw.shape[1]
+    y = np.empty((M, N), np.float64)
+    _load().oracle_floatscale(_p(qx), _p(s_a), _p(qw), _p(s_g), M, N, K, group, _p(y))
+    return y
+
+
+def floatscale_at(qx, s_a, qw, s_g, ms, ns, group: int = 128):
+    qx = _c(qx, np.int8)
+    s_a = _c(s_a, np.float32)
+    qw = _c(qw, np.int8)
+    s_g = _c(s_g, np.float32)
+    ms = _c(ms, np.int64)
+    ns = _c(ns, np.int64)
+    M, K = qx.shape
+    N = qw.shape[1]
+    y = np.empty(ms.size, np.float64)
+    _load().oracle_floatscale_at(_p(qx), _p(s_a), _p(qw), _p(s_g), M, N, K, group, _p(ms), _p(ns), ms.size, _p(y))
+    return y
+
+
+def round_output(y, out: str):
+    """fp64 result -> the output type ('f32' or 'f16'), round to nearest even."""
+    if out == "f32":
+        return np.asarray(y, np.float64).astype(np.float32)
+    if out == "f16":
+        return np.asarray(y, np.float64).astype(np.float16)
+    raise ValueError(out)
+
+
+# ---------------------------------------------------------------- whole layer
+
+def linear_intscale(x, w, *, group: int = 128, alpha=1024, out: str = "f16"):
+    """The whole Integer-Scale path on the CPU.
+
+    alpha: an integer power of two, or None for the amplifier search.
+    Returns a dict with every intermediate (codes, scales, packed bytes,
+    integer scales, raw accumulators, fp64 and rounded outputs).
+    """
+    qx, s_a = quantize_act_per_token(x)
+    qw, s_g = quantize_groups(w, group)
+    a = amplifier_search(s_g) if alpha is None else int(alpha)
+    S = integer_scales(s_g, a)
+    acc = intscale_acc(qx, qw, S, group)
+    y64 = intscale_output(acc, s_a, a)
+    return dict(qx=qx, s_a=s_a, qw=qw, s_g=s_g, packed=pack_int4(qw), alpha=a, S=S, acc=acc,
+                y64=y64, y=round_output(y64, out))
+
+
+def linear_floatscale(x, w, *, group: int = 128, out: str = "f16"):
+    qx, s_a = quantize_act_per_token(x)
+    qw, s_g = quantize_groups(w, group)
+    y64 = floatscale(qx, s_a, qw, s_g, group)
+    return dict(qx=qx, s_a=s_a, qw=qw, s_g=s_g, y64=y64, y=round_output(y64, out))

@@ -1,0 +1,375 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself -- hand-worked values, closed forms, brute force, library routines on
+special cases, and the pages' error model -- chosen so that a dropped term, a
+wrong sign, index or transposed operand in the oracle fails at least one.
+
+No GPU is needed here."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from bit_gemm_quantize_b200 import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _bits(x):
+    return int(np.asarray(x, np.float32).view(np.uint32))
+
+
+def _nearest_code_bruteforce(x, s, qmax):
+    """Search every code for the one nearest to the fp32 quotient x/s, ties to
+    the even code.  Uses numpy's fp32 division, independent of the oracle."""
+    x = np.asarray(x, np.float32)
+    s = np.float32(s)
+    if s == 0:
+        return np.zeros(x.shape, np.int64)
+    t = (x / s).astype(np.float64)  # the quotient, rounded once to fp32
+    codes = np.arange(-qmax, qmax + 1, dtype=np.float64)
+    d = np.abs(t[..., None] - codes)
+    best = d.min(axis=-1, keepdims=True)
+    cand = np.where(d == best, codes, np.nan)
+    # among equally near codes take the even one
+    n_near = (d == best).sum(axis=-1)
+    lowest = np.nanmin(cand, axis=-1)
+    # a tie has exactly two candidates, one of them even
+    tie_pick = np.where(np.fmod(np.abs(lowest), 2) == 0, lowest, lowest + 1)
+    return np.where(n_near == 1, lowest, tie_pick).astype(np.int64)
+
+
+# ------------------------------------------------------------- quantize rows
+
+def test_quantize_golden_rows():
+    g = _golden("quantize_int8_symmetric.json")
+    for case in g["cases"]:
+        q, s = oracle.quantize_act_per_token(np.array([case["x"]], np.float32))
+        assert q[0].tolist() == case["q"], case["derivation"]
+        assert _bits(s[0]) == int(case["s_bits"], 16), case["derivation"]
+
+
+def test_quantize_rows_bruteforce_nearest_code():
+    rng = np.random.default_rng(1)
+    for qmax in (127, 7):
+        x = rng.standard_normal((64, 256)).astype(np.float32)
+        x[:, 3] *= 20
+        q, s = oracle.quantize_rows(x, qmax)
+        for m in range(x.shape[0]):
+            ref = _nearest_code_bruteforce(x[m], s[m], qmax)
+            assert np.array_equal(q[m].astype(np.int64), ref)
+
+
+def test_quantize_rows_absmax_maps_to_qmax_and_bound():
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal((32, 512)) * rng.uniform(0.01, 100, (32, 1))).astype(np.float32)
+    q, s = oracle.quantize_act_per_token(x)
+    am = np.abs(x).max(axis=1)
+    arg = np.abs(x).argmax(axis=1)
+    # the largest magnitude is the clip point: it lands on +-127
+    assert np.all(np.abs(q[np.arange(32), arg]) == 127)
+    assert np.all(np.sign(q[np.arange(32), arg]) == np.sign(x[np.arange(32), arg]))
+    # s * qmax reproduces the absmax to fp32 rounding
+    assert np.allclose(s.astype(np.float64) * 127, am, rtol=2e-7, atol=0)
+    # rounding error of a symmetric absmax quantizer: |x - s q| <= s/2 (no clipping)
+    err = np.abs(x.astype(np.float64) - s[:, None].astype(np.float64) * q)
+    assert np.all(err <= s[:, None] * (0.5 + 1e-5))
+    # -128 is never produced
+    assert q.min() >= -127 and q.max() <= 127
+
+
+def test_quantize_rows_error_variance_s2_over_12():
+    """Rounding error of a uniform quantizer has variance ~ s^2/12
+    (探秘Transformer系列之（34）量化基礎, 量化誤差)."""
+    w = workloads.make_linear(64, 4096, 8, x_dtype="f32", seed=3)
+    x = w.x
+    q, s = oracle.quantize_act_per_token(x)
+    mask = np.ones(x.shape[1], bool)
+    mask[w.outlier_cols] = False
+    e = (x.astype(np.float64) - s[:, None] * q.astype(np.float64))[:, mask]
+    ratio = np.mean(e ** 2 / (s[:, None].astype(np.float64) ** 2 / 12.0))
+    assert e.size >= 1e5
+    assert 0.9 <= ratio <= 1.1, ratio
+
+
+def test_quantize_zero_row_and_sign_symmetry():
+    x = np.array([[0, 0, 0, 0], [1.0, -2.0, 3.0, -4.0]], np.float32)
+    q, s = oracle.quantize_act_per_token(x)
+    assert s[0] == 0 and not q[0].any()
+    qn, sn = oracle.quantize_act_per_token(-x)
+    assert np.array_equal(qn, -q) and np.array_equal(sn, s)
+
+
+# ------------------------------------------------------------- group quantize
+
+def test_quantize_groups_bruteforce_and_layout():
+    rng = np.random.default_rng(4)
+    K, N, g = 384, 24, 128
+    w = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    q, s = oracle.quantize_groups(w, g)
+    assert q.shape == (K, N) and s.shape == (K // g, N)
+    for gi in range(K // g):
+        blk = w[gi * g:(gi + 1) * g]
+        # the scale belongs to (group, column): absmax over the group's k only
+        assert np.allclose(s[gi].astype(np.float64) * 7, np.abs(blk).max(axis=0), rtol=2e-7)
+        for n in range(N):
+            ref = _nearest_code_bruteforce(blk[:, n], s[gi, n], 7)
+            assert np.array_equal(q[gi * g:(gi + 1) * g, n].astype(np.int64), ref)
+    assert q.min() >= -7 and q.max() <= 7
+
+
+def test_quantize_groups_locality():
+    """Changing one weight moves only its own (group, column) scale and codes."""
+    rng = np.random.default_rng(5)
+    K, N, g = 256, 8, 128
+    w = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    q0, s0 = oracle.quantize_groups(w, g)
+    w2 = w.copy()
+    w2[200, 5] = 1.0
+    q1, s1 = oracle.quantize_groups(w2, g)
+    diff_s = np.argwhere(s0 != s1)
+    assert diff_s.tolist() == [[1, 5]]
+    changed = np.argwhere(q0 != q1)
+    assert all(128 <= k < 256 and n == 5 for k, n in changed)
+
+
+def test_quantize_groups_per_channel_equals_rows_of_transpose():
+    """group = K is per-channel quantization: the same as per-row of W^T."""
+    rng = np.random.default_rng(6)
+    w = (rng.standard_normal((256, 16)) * 0.02).astype(np.float32)
+    q, s = oracle.quantize_groups(w, 256)
+    qt, st = oracle.quantize_rows(w.T.copy(), 7)
+    assert np.array_equal(q, qt.T) and np.array_equal(s[0], st)
+
+
+# ------------------------------------------------------------- packing
+
+def test_pack_golden():
+    g = _golden("pack_int4.json")
+    q = np.array(g["q_KxN"], np.int8)
+    p = oracle.pack_int4(q)
+    assert p.tolist() == g["packed_NxK2"], g["derivation"]
+
+
+def test_pack_exhaustive_nibble_roundtrip():
+    vals = np.arange(-8, 8, dtype=np.int8)
+    lo, hi = np.meshgrid(vals, vals, indexing="ij")
+    q = np.stack([lo.ravel(), hi.ravel()])  # K=2, N=256
+    p = oracle.pack_int4(q)
+    assert p.shape == (256, 1)
+    assert sorted(p.ravel().tolist()) == list(range(256))  # a bijection onto bytes
+    assert np.array_equal(oracle.unpack_int4(p, 2, 256), q)
+    # nibble semantics: low nibble is the even k, both two's complement
+    b = p[:, 0].astype(np.int64)
+    assert np.array_equal(((b & 0xF) ^ 8) - 8, lo.ravel())
+    assert np.array_equal((((b >> 4) & 0xF) ^ 8) - 8, hi.ravel())
+
+
+# ------------------------------------------------------------- amplifier
+
+def test_amplifier_golden():
+    for case in _golden("amplifier_search.json")["cases"]:
+        assert oracle.amplifier_search(np.array(case["scales"], np.float32)) == case["alpha"], case
+
+
+def _alpha_closed_form(smin):
+    f, e = math.frexp(smin)  # smin = f * 2^e, f in [0.5, 1)
+    j = max(0, 1 - e)
+    return 1 << j
+
+
+def test_amplifier_postcondition_and_closed_form():
+    rng = np.random.default_rng(7)
+    for _ in range(500):
+        scales = (10.0 ** rng.uniform(-8, 1, rng.integers(1, 50))).astype(np.float32)
+        a = oracle.amplifier_search(scales)
+        smin = float(scales.min())
+        assert a == _alpha_closed_form(smin)
+        assert a >= 1 and (a & (a - 1)) == 0
+        assert np.all(scales.astype(np.float64) * a >= 1)
+        assert a == 1 or smin * a / 2 < 1
+
+
+# ------------------------------------------------------------- integer scales
+
+def test_integer_scales_rounding():
+    s = np.array([0.0078125, 7.5 / 1024, 8.5 / 1024, 0.0077, 0.005, 0.0], np.float32)
+    S = oracle.integer_scales(s, 1024)
+    assert S.tolist() == [8, 8, 8, 8, 5, 0]
+    rng = np.random.default_rng(8)
+    s = rng.uniform(0, 0.05, 10000).astype(np.float32)
+    for a in (1, 128, 1024, 4096):
+        S = oracle.integer_scales(s, a)
+        assert np.all(np.abs(S - s.astype(np.float64) * a) <= 0.5)
+
+
+# ------------------------------------------------------------- GEMMs
+
+def _rand_codes(rng, M, N, K):
+    qx = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    qw = rng.integers(-7, 8, (K, N)).astype(np.int8)
+    return qx, qw
+
+
+def test_tiny_linear_golden():
+    g = _golden("tiny_linear.json")
+    x = np.zeros((1, 256), np.float32)
+    w = np.zeros((256, 1), np.float32)
+    for k, v in g["x_nonzero"].items():
+        x[0, int(k)] = v
+    for k, v in g["w_nonzero"].items():
+        w[int(k), 0] = v
+    r = oracle.linear_intscale(x, w, alpha=1024, out="f32")
+    assert r["s_a"].tolist() == [g["s_a"]]
+    assert r["s_g"][:, 0].tolist() == g["s_g"]
+    assert {str(k): int(r["qx"][0, k]) for k in np.flatnonzero(r["qx"][0])} == g["qx_nonzero"]
+    assert {str(k): int(r["qw"][k, 0]) for k in np.flatnonzero(r["qw"][:, 0])} == g["qw_nonzero"]
+    assert r["S"][:, 0].tolist() == g["S_alpha1024"]
+    assert int(r["acc"][0, 0]) == g["acc_alpha1024"]
+    assert r["y64"][0, 0] == g["y"]
+    r2 = oracle.linear_intscale(x, w, alpha=None, out="f32")
+    assert r2["alpha"] == g["search_alpha"]
+    assert r2["S"][:, 0].tolist() == g["S_search"] and int(r2["acc"][0, 0]) == g["acc_search"]
+    assert r2["y64"][0, 0] == g["y"]
+    f = oracle.linear_floatscale(x, w, out="f32")
+    assert f["y64"][0, 0] == g["y"]
+    assert float((x.astype(np.float64) @ w.astype(np.float64))[0, 0]) == g["y"]
+
+
+def test_intscale_groupwise_equals_expanded_weight():
+    rng = np.random.default_rng(9)
+    for (M, N, K, g) in [(3, 5, 256, 128), (1, 17, 384, 128), (4, 8, 128, 32), (2, 3, 512, 256)]:
+        qx, qw = _rand_codes(rng, M, N, K)
+        S = rng.integers(-3000, 30000, (K // g, N)).astype(np.int32)
+        a = oracle.intscale_acc(qx, qw, S, g)
+        b = oracle.intscale_acc_expanded(qx, qw, S, g)
+        assert np.array_equal(a, b)
+        # and the sampled variant agrees at arbitrary positions
+        ms = rng.integers(0, M, 20)
+        ns = rng.integers(0, N, 20)
+        assert np.array_equal(oracle.intscale_acc_at(qx, qw, S, ms, ns, g), a[ms, ns])
+
+
+def test_intscale_constant_scale_is_plain_integer_matmul():
+    rng = np.random.default_rng(10)
+    M, N, K = 6, 11, 512
+    qx, qw = _rand_codes(rng, M, N, K)
+    Sn = rng.integers(1, 40, N).astype(np.int32)
+    S = np.tile(Sn, (K // 128, 1))
+    acc = oracle.intscale_acc(qx, qw, S)
+    ref = (qx.astype(np.int64) @ qw.astype(np.int64)) * Sn.astype(np.int64)
+    assert np.array_equal(acc, ref)
+
+
+def test_intscale_bruteforce_dequantized_fp64():
+    """acc * s_a / alpha equals the fp64 matmul of the dequantized operands
+    (s_a q_x) and (S/alpha q_w) on tiny inputs."""
+    rng = np.random.default_rng(11)
+    for seed in range(300):
+        M = int(rng.integers(1, 5))
+        N = int(rng.integers(1, 9))
+        K = int(rng.choice([128, 256]))
+        x = rng.standard_normal((M, K)).astype(np.float32)
+        w = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+        alpha = int(rng.choice([1024, 256]))
+        r = oracle.linear_intscale(x, w, alpha=alpha, out="f32")
+        xh = r["s_a"][:, None].astype(np.float64) * r["qx"]
+        G = K // 128
+        Sfull = np.repeat(r["S"], 128, axis=0).astype(np.float64)
+        wh = Sfull / alpha * r["qw"]
+        ref = xh @ wh
+        assert np.allclose(r["y64"], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_intscale_zero_input_and_one_hot_column():
+    rng = np.random.default_rng(12)
+    M, K, N = 3, 256, 4
+    w = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    r0 = oracle.linear_intscale(np.zeros((M, K), np.float32), w, out="f32")
+    assert not r0["acc"].any() and not r0["y64"].any()
+    # one-hot weight column: only k* = 150 (group 1) is non-zero in column 2
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    w[:, 2] = 0
+    w[150, 2] = -0.03
+    r = oracle.linear_intscale(x, w, alpha=1024, out="f32")
+    S = r["S"][1, 2]
+    assert r["qw"][150, 2] == -7 and r["S"][0, 2] == 0
+    expect = r["s_a"].astype(np.float64) * S / 1024 * (-7) * r["qx"][:, 150]
+    assert np.allclose(r["y64"][:, 2], expect, rtol=1e-15)
+
+
+def test_floatscale_equals_intscale_when_scales_are_exact():
+    """With s_g = S/alpha exactly, the float-scale path must give the
+    integer-scale result (two different summations)."""
+    rng = np.random.default_rng(13)
+    M, N, K = 5, 9, 384
+    qx, qw = _rand_codes(rng, M, N, K)
+    S = rng.integers(1, 20, (K // 128, N)).astype(np.int32)
+    s_a = rng.uniform(0.01, 0.1, M).astype(np.float32)
+    s_g = (S / 1024.0).astype(np.float32)
+    yf = oracle.floatscale(qx, s_a, qw, s_g)
+    yi = oracle.intscale_output(oracle.intscale_acc(qx, qw, S), s_a, 1024)
+    assert np.allclose(yf, yi, rtol=1e-12, atol=1e-12)
+    ms = np.array([0, 4, 2])
+    ns = np.array([8, 0, 3])
+    assert np.allclose(oracle.floatscale_at(qx, s_a, qw, s_g, ms, ns), yf[ms, ns], rtol=1e-15)
+
+
+def test_floatscale_per_channel_is_outer_product_dequant():
+    """group = K: y = (s_a s_w^T) o (q_x q_w), the token x channel outer-product
+    dequantization (探秘Transformer系列之（34）, 逐通道量化 & 逐token量化)."""
+    rng = np.random.default_rng(14)
+    M, N, K = 4, 6, 256
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    w = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    qx, s_a = oracle.quantize_act_per_token(x)
+    qw, s_w = oracle.quantize_groups(w, K)
+    y = oracle.floatscale(qx, s_a, qw, s_w, K)
+    ref = np.outer(s_a.astype(np.float64), s_w[0].astype(np.float64)) * (qx.astype(np.int64) @ qw.astype(np.int64))
+    assert np.allclose(y, ref, rtol=1e-14)
+
+
+def test_intscale_error_bound_against_unquantized():
+    """Per element: |y_IS - x w| <= sum_k |x_hat| (s_g/2 + 3.5/alpha) + (s_a/2)|w|,
+    from |x - x_hat| <= s_a/2 and |w - (S/alpha) q_w| <= s_g/2 + 7/(2 alpha)."""
+    for cfg_seed, (M, K, N) in enumerate([(16, 1024, 64), (4, 512, 96)]):
+        wl = workloads.make_linear(M, K, N, x_dtype="f32", seed=cfg_seed, outlier_scale=20.0)
+        for alpha in (1024, None):
+            r = oracle.linear_intscale(wl.x, wl.w, alpha=alpha, out="f32")
+            a = r["alpha"]
+            xh = np.abs(r["s_a"][:, None].astype(np.float64) * r["qx"])
+            sg = np.repeat(r["s_g"], 128, axis=0).astype(np.float64)
+            bound = xh @ (sg / 2 + 3.5 / a) + (r["s_a"][:, None].astype(np.float64) / 2) @ np.ones((1, K)) @ np.abs(wl.w.astype(np.float64))
+            y_true = wl.x.astype(np.float64) @ wl.w.astype(np.float64)
+            err = np.abs(r["y64"] - y_true)
+            assert np.all(err <= bound * (1 + 1e-9) + 1e-12)
+
+
+def test_int32_bound_and_colsum():
+    rng = np.random.default_rng(15)
+    K, N = 512, 10
+    qx = np.full((2, K), 127, np.int8)
+    qw = np.full((K, N), 7, np.int8)
+    qx[1] = -127
+    S = rng.integers(0, 50, (K // 128, N)).astype(np.int32)
+    acc = oracle.intscale_acc(qx, qw, S)
+    colsum = oracle.scale_colsum_max(S)
+    assert colsum == int(np.abs(S).sum(axis=0).max())
+    # extreme codes reach the bound exactly at the column with the largest sum
+    assert int(np.abs(acc).max()) == 127 * 7 * 128 * colsum
+
+
+def test_workload_bound_holds_for_default_amplifier():
+    """The generator's weights keep the worst-case accumulator inside int32."""
+    wl = workloads.make_linear(1, 4096, 512, seed=0)
+    qw, s_g = oracle.quantize_groups(wl.w, 128)
+    S = oracle.integer_scales(s_g, 1024)
+    assert S.max() <= 32767
+    assert 127 * 7 * 128 * oracle.scale_colsum_max(S) < 2 ** 31
