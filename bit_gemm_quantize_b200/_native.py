@@ -1,0 +1,251 @@
+"""ctypes binding of the C ABI in include/w4a8_intscale.h.
+
+Argument marshalling only: torch tensors are checked for device, dtype,
+shape and contiguity, and their data pointers and the current CUDA stream are
+handed to the library, which does every step of the computation in its own
+kernels.  There is no CPU path: a missing library or a CPU tensor raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libw4a8_intscale.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "w4a8_intscale.h")
+
+# w4a8_dtype
+F32, F16, BF16, I32 = 0, 1, 2, 3
+PACK_WORKSPACE_BYTES = 1 << 20
+
+STATUS = {
+    0: "W4A8_OK",
+    1: "W4A8_ERR_INVALID_ARG",
+    2: "W4A8_ERR_SHAPE",
+    3: "W4A8_ERR_ALIGN",
+    4: "W4A8_ERR_DTYPE",
+    5: "W4A8_ERR_OVERFLOW_BOUND",
+    6: "W4A8_ERR_SCALE_RANGE",
+    7: "W4A8_ERR_CUDA",
+    8: "W4A8_ERR_TIMEOUT",
+    9: "W4A8_ERR_WORKSPACE",
+}
+
+
+class W4A8Error(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def declared_symbols():
+    """Names of the functions the public header declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return re.findall(r"W4A8_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def load(path: str = LIB_PATH):
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"CUDA library not found at {path}; build it with `python -m bit_gemm_quantize_b200.build`"
+            )
+        lib = ctypes.CDLL(path)
+        P, I64, I32_ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+        sigs = {
+            "w4a8_status_string": ([I32_], ctypes.c_char_p),
+            "quantize_act_per_token": ([P, I32_, I64, I64, I64, P, P, P], I32_),
+            "w4a8_amplifier_search": ([P, I64, P, P, P], I32_),
+            "pack_w4_groupwise": ([P, I64, I64, I32_, I32_, P, P, P, P, P, P, P], I32_),
+            "w4a8_gemm_workspace_size": ([I64, I64, I64, I32_, I32_], I64),
+            "w4a8_gemm_intscale": ([P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
+            "w4a8_gemm_floatscale": ([P, P, P, P, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
+            "w4a8_device_status": ([P, I32_], I32_),
+        }
+        for name, (args, res) in sigs.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+        return lib
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise W4A8Error(fn, code)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(name, t, dtype=None, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ------------------------------------------------------------------ workspace
+
+_ws_cache = {}
+
+
+def gemm_workspace(M: int, N: int, K: int, group: int, path: int, device) -> torch.Tensor | None:
+    """A zero-filled workspace big enough for the call, reused across calls on
+    the device (the kernels leave it zeroed after a successful call)."""
+    lib = load()
+    with torch.cuda.device(device):
+        need = int(lib.w4a8_gemm_workspace_size(M, N, K, group, path))
+    if need < 0:
+        raise RuntimeError("w4a8_gemm_workspace_size: no CUDA device")
+    if need == 0:
+        return None
+    key = torch.device(device).index
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+# ------------------------------------------------------------------ operations
+
+def quantize_act_per_token(x: torch.Tensor, q_x: torch.Tensor | None = None, s_a: torch.Tensor | None = None):
+    """Per-token int8 codes and fp32 scales of x [M, K] (fp32 or bf16)."""
+    _need_cuda("x", x, ndim=2)
+    if x.dtype == torch.float32:
+        dt = F32
+    elif x.dtype == torch.bfloat16:
+        dt = BF16
+    else:
+        raise ValueError("x must be float32 or bfloat16")
+    M, K = x.shape
+    if q_x is None:
+        q_x = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if s_a is None:
+        s_a = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _need_cuda("q_x", q_x, torch.int8, 2)
+    _need_cuda("s_a", s_a, torch.float32, 1)
+    code = load().quantize_act_per_token(_ptr(x), dt, M, K, K, _ptr(q_x), _ptr(s_a), _stream(x.device))
+    _check("quantize_act_per_token", code)
+    return q_x, s_a
+
+
+def w4a8_amplifier_search(scales: torch.Tensor) -> int:
+    _need_cuda("scales", scales, torch.float32)
+    ws = torch.empty(PACK_WORKSPACE_BYTES, dtype=torch.uint8, device=scales.device)
+    alpha = ctypes.c_int32(0)
+    code = load().w4a8_amplifier_search(_ptr(scales), scales.numel(), _ptr(ws), ctypes.byref(alpha),
+                                        _stream(scales.device))
+    _check("w4a8_amplifier_search", code)
+    return int(alpha.value)
+
+
+def pack_w4_groupwise(w: torch.Tensor, group: int = 128, alpha: int | None = 1024, scales_only: bool = False):
+    """Quantize and pack fp32 weights w [K, N].  alpha=None runs the search.
+
+    Returns dict(packed [N, K/2] uint8, s_g [K/group, N] f32, S [K/group, N]
+    int16, alpha, colsum_max), or dict(s_g) when scales_only."""
+    _need_cuda("w", w, torch.float32, 2)
+    K, N = w.shape
+    dev = w.device
+    s_g = torch.empty((K // group, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(PACK_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
+    lib = load()
+    if scales_only:
+        code = lib.pack_w4_groupwise(_ptr(w), K, N, group, 0, None, _ptr(s_g), None, None, None, _ptr(ws),
+                                     _stream(dev))
+        _check("pack_w4_groupwise", code)
+        return dict(s_g=s_g)
+    packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    S = torch.empty((K // group, N), dtype=torch.int16, device=dev)
+    a_out = ctypes.c_int32(0)
+    colsum = ctypes.c_int64(0)
+    code = lib.pack_w4_groupwise(_ptr(w), K, N, group, 0 if alpha is None else int(alpha), _ptr(packed),
+                                 _ptr(s_g), _ptr(S), ctypes.byref(a_out), ctypes.byref(colsum), _ptr(ws),
+                                 _stream(dev))
+    _check("pack_w4_groupwise", code)
+    return dict(packed=packed, s_g=s_g, S=S, alpha=int(a_out.value), colsum_max=int(colsum.value))
+
+
+_OUT = {"f32": (F32, torch.float32), "f16": (F16, torch.float16), "i32": (I32, torch.int32)}
+
+
+def _gemm_args(q_x, s_a, packed, N, K, group):
+    _need_cuda("q_x", q_x, torch.int8, 2)
+    _need_cuda("s_a", s_a, torch.float32, 1)
+    _need_cuda("w_packed", packed, torch.uint8, 2)
+    M = q_x.shape[0]
+    if q_x.shape[1] != K or packed.shape != (N, K // 2) or s_a.shape[0] != M:
+        raise ValueError("inconsistent GEMM operand shapes")
+    return M
+
+
+def w4a8_gemm_intscale(q_x, s_a, w_packed, S, alpha: int, *, group: int = 128, out: str = "f16",
+                       y: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """y [M, N] = integer-scale W4A8 GEMM (out: 'f16', 'f32' or 'i32' raw accumulators)."""
+    N, K2 = w_packed.shape
+    K = 2 * K2
+    M = _gemm_args(q_x, s_a, w_packed, N, K, group)
+    _need_cuda("S", S, torch.int16, 2)
+    dt, tdt = _OUT[out]
+    if y is None:
+        y = torch.empty((M, N), dtype=tdt, device=q_x.device)
+    _need_cuda("y", y, tdt, 2)
+    if workspace is None:
+        workspace = gemm_workspace(M, N, K, group, 0, q_x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = load().w4a8_gemm_intscale(_ptr(q_x), _ptr(s_a), _ptr(w_packed), _ptr(S), int(alpha), M, N, K, group,
+                                     _ptr(y), dt, _ptr(workspace), ws_bytes, _stream(q_x.device))
+    _check("w4a8_gemm_intscale", code)
+    return y
+
+
+def w4a8_gemm_floatscale(q_x, s_a, w_packed, s_g, *, group: int = 128, out: str = "f16",
+                         y: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """y [M, N] = float-scale W4A8 GEMM (the comparison path; out 'f16' or 'f32')."""
+    N, K2 = w_packed.shape
+    K = 2 * K2
+    M = _gemm_args(q_x, s_a, w_packed, N, K, group)
+    _need_cuda("s_g", s_g, torch.float32, 2)
+    if out not in ("f16", "f32"):
+        raise ValueError("float-scale output must be f16 or f32")
+    dt, tdt = _OUT[out]
+    if y is None:
+        y = torch.empty((M, N), dtype=tdt, device=q_x.device)
+    _need_cuda("y", y, tdt, 2)
+    if workspace is None:
+        workspace = gemm_workspace(M, N, K, group, 1, q_x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = load().w4a8_gemm_floatscale(_ptr(q_x), _ptr(s_a), _ptr(w_packed), _ptr(s_g), M, N, K, group, _ptr(y),
+                                       dt, _ptr(workspace), ws_bytes, _stream(q_x.device))
+    _check("w4a8_gemm_floatscale", code)
+    return y
+
+
+def device_status(clear: bool = True) -> int:
+    v = ctypes.c_int32(0)
+    _check("w4a8_device_status", load().w4a8_device_status(ctypes.byref(v), 1 if clear else 0))
+    return int(v.value)

@@ -1,0 +1,290 @@
+// C ABI of the library: argument checks on the host, tensor maps, launches.
+// The operations and their sources are documented in include/w4a8_intscale.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/w4a8_intscale.h"
+#include "gemm_w4a8.h"
+#include "kernels.h"
+
+namespace {
+
+// One status word per device that loads the library; bounded waits that run
+// out write W4A8_ERR_TIMEOUT into it.
+__device__ int g_status_word;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    int* status = nullptr;
+};
+
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_devices_mutex;
+
+w4a8_status current_device(DeviceInfo& out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W4A8_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_devices_mutex);
+    DeviceInfo& d = g_devices[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return W4A8_ERR_CUDA;
+        if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_status_word) != cudaSuccess)
+            return W4A8_ERR_CUDA;
+        d.ready = true;
+    }
+    out = d;
+    return W4A8_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D uint8 tensor map: [rows][cols] bytes with row pitch `pitch`.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch, uint32_t box_cols,
+                 uint32_t box_rows, CUtensorMapSwizzle swz) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {pitch};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Whether the stream-K partition of `pl` cuts any tile (then a workspace is needed).
+bool plan_splits_tiles(const w4a8::gemm::Plan& pl) {
+    for (int64_t b = 1; b < pl.grid; ++b)
+        if ((b * pl.W / pl.grid) % pl.G != 0) return true;
+    return false;
+}
+
+w4a8_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int32_t group) {
+    if (M < 0 || N <= 0 || K <= 0 || group <= 0) return W4A8_ERR_SHAPE;
+    if (N % 8 != 0 || K % 128 != 0 || group % 128 != 0 || K % group != 0) return W4A8_ERR_SHAPE;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return W4A8_ERR_SHAPE;
+    return W4A8_OK;
+}
+
+w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_t* w_packed, const int16_t* S,
+                     const float* s_g, int32_t alpha, int64_t M, int64_t N, int64_t K, int32_t group, void* y,
+                     int32_t y_dtype, void* workspace, int64_t workspace_bytes, void* stream) {
+    w4a8_status st = check_gemm_shape(M, N, K, group);
+    if (st != W4A8_OK) return st;
+    if (path == w4a8::gemm::kIntScale) {
+        if (y_dtype != W4A8_F16 && y_dtype != W4A8_F32 && y_dtype != W4A8_I32) return W4A8_ERR_DTYPE;
+        if (!is_pow2(alpha) || alpha > (1 << 30)) return W4A8_ERR_INVALID_ARG;
+    } else {
+        if (y_dtype != W4A8_F16 && y_dtype != W4A8_F32) return W4A8_ERR_DTYPE;
+    }
+    if (M == 0) return W4A8_OK;
+    if (!q_x || !s_a || !w_packed || !y || (path == w4a8::gemm::kIntScale ? !S : !s_g)) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(q_x) || !aligned16(w_packed) || !aligned16(y) || !aligned16(s_a) ||
+        !aligned16(path == w4a8::gemm::kIntScale ? static_cast<const void*>(S) : static_cast<const void*>(s_g)))
+        return W4A8_ERR_ALIGN;
+
+    DeviceInfo dev;
+    if ((st = current_device(dev)) != W4A8_OK) return st;
+    const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms);
+    int32_t* ws_count = nullptr;
+    int32_t* ws_part = nullptr;
+    if (plan_splits_tiles(pl)) {
+        if (!workspace || workspace_bytes < pl.ws_bytes) return W4A8_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return W4A8_ERR_ALIGN;
+        ws_count = static_cast<int32_t*>(workspace);
+        ws_part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + pl.count_bytes);
+    }
+
+    CUtensorMap tm_w, tm_x;
+    if (!make_map_u8(&tm_w, w_packed, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+        return W4A8_ERR_CUDA;
+    if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(M), uint64_t(K), 128, uint32_t(pl.BT),
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return W4A8_ERR_CUDA;
+
+    w4a8::gemm::Params p{};
+    p.s_a = s_a;
+    p.S = S;
+    p.s_g = s_g;
+    p.y = y;
+    p.ws_part = ws_part;
+    p.ws_count = ws_count;
+    p.status = dev.status;
+    p.M = M;
+    p.N = N;
+    p.G = pl.G;
+    p.kb_per_group = group / 128;
+    p.m_tiles = pl.m_tiles;
+    p.W = pl.W;
+    p.grid = pl.grid;
+    p.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
+    p.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
+                                    : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
+    if (w4a8::gemm::launch(tm_w, tm_x, p, pl.BT, path, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return W4A8_ERR_CUDA;
+    return W4A8_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* w4a8_status_string(int32_t status) {
+    switch (status) {
+        case W4A8_OK: return "ok";
+        case W4A8_ERR_INVALID_ARG: return "invalid argument";
+        case W4A8_ERR_SHAPE: return "unsupported shape";
+        case W4A8_ERR_ALIGN: return "misaligned pointer or leading dimension";
+        case W4A8_ERR_DTYPE: return "unsupported dtype";
+        case W4A8_ERR_OVERFLOW_BOUND: return "worst-case int32 accumulator bound exceeded";
+        case W4A8_ERR_SCALE_RANGE: return "integer scale or amplifier out of range";
+        case W4A8_ERR_CUDA: return "CUDA runtime error";
+        case W4A8_ERR_TIMEOUT: return "kernel wait timed out";
+        case W4A8_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+w4a8_status quantize_act_per_token(const void* x, int32_t x_dtype, int64_t M, int64_t K, int64_t ldx,
+                                   int8_t* q_x, float* s_a, void* stream) {
+    if (x_dtype != W4A8_F32 && x_dtype != W4A8_BF16) return W4A8_ERR_DTYPE;
+    if (M < 0 || K <= 0 || K % 16 != 0 || ldx < K) return W4A8_ERR_SHAPE;
+    if (M == 0) return W4A8_OK;
+    if (!x || !q_x || !s_a) return W4A8_ERR_INVALID_ARG;
+    const int64_t esz = x_dtype == W4A8_BF16 ? 2 : 4;
+    if (!aligned16(x) || !aligned16(q_x) || (ldx * esz) % 16 != 0) return W4A8_ERR_ALIGN;
+    DeviceInfo dev;
+    w4a8_status st = current_device(dev);
+    if (st != W4A8_OK) return st;
+    if (w4a8::quant::launch(x, x_dtype == W4A8_BF16, M, K, ldx, q_x, s_a, dev.status,
+                            static_cast<cudaStream_t>(stream), dev.sms) != cudaSuccess)
+        return W4A8_ERR_CUDA;
+    return W4A8_OK;
+}
+
+w4a8_status w4a8_amplifier_search(const float* scales, int64_t count, void* workspace, int32_t* alpha_host,
+                                  void* stream) {
+    if (!scales || !workspace || !alpha_host) return W4A8_ERR_INVALID_ARG;
+    if (count <= 0) return W4A8_ERR_SHAPE;
+    if (!aligned16(workspace)) return W4A8_ERR_ALIGN;
+    DeviceInfo dev;
+    w4a8_status st = current_device(dev);
+    if (st != W4A8_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (w4a8::pack::amplifier(scales, count, 0, workspace, s, dev.sms) != cudaSuccess) return W4A8_ERR_CUDA;
+    w4a8::pack::Results r;
+    if (cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s) != cudaSuccess) return W4A8_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return W4A8_ERR_CUDA;
+    if (r.error) return W4A8_ERR_SCALE_RANGE;
+    *alpha_host = r.alpha;
+    return W4A8_OK;
+}
+
+w4a8_status pack_w4_groupwise(const float* w, int64_t K, int64_t N, int32_t group, int32_t alpha_in,
+                              uint8_t* w_packed, float* s_g, int16_t* S, int32_t* alpha_out_host,
+                              int64_t* colsum_max_host, void* workspace, void* stream) {
+    if (K <= 0 || N <= 0 || group <= 0 || group % 32 != 0 || K % group != 0 || N % 8 != 0) return W4A8_ERR_SHAPE;
+    if (K > INT32_MAX || N > INT32_MAX || K / group > 65535 || K / 32 > 65535) return W4A8_ERR_SHAPE;
+    if (!w || !s_g) return W4A8_ERR_INVALID_ARG;
+    const bool scales_only = (w_packed == nullptr && S == nullptr);
+    if (!scales_only && (!w_packed || !S || !alpha_out_host || !workspace)) return W4A8_ERR_INVALID_ARG;
+    if (alpha_in < 0 || (alpha_in > 0 && (!is_pow2(alpha_in) || alpha_in > (1 << 30)))) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(s_g) || (w_packed && !aligned16(w_packed)) || (S && !aligned16(S)) ||
+        (workspace && !aligned16(workspace)))
+        return W4A8_ERR_ALIGN;
+    DeviceInfo dev;
+    w4a8_status st = current_device(dev);
+    if (st != W4A8_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (w4a8::pack::group_scales(w, K, N, group, s_g, s) != cudaSuccess) return W4A8_ERR_CUDA;
+    if (scales_only) return cudaStreamSynchronize(s) == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+
+    const int64_t G = K / group;
+    if (w4a8::pack::amplifier(s_g, G * N, alpha_in, workspace, s, dev.sms) != cudaSuccess) return W4A8_ERR_CUDA;
+    w4a8::pack::Results r;
+    if (cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s) != cudaSuccess) return W4A8_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return W4A8_ERR_CUDA;
+    if (r.error) return W4A8_ERR_SCALE_RANGE;
+    // the largest integer scale is round(s_max * alpha)
+    if (std::nearbyint(double(r.s_max) * double(r.alpha)) > 32767.0) {
+        *alpha_out_host = r.alpha;
+        return W4A8_ERR_SCALE_RANGE;
+    }
+    if (w4a8::pack::quantize_pack(w, s_g, r.alpha, K, N, group, w_packed, S, workspace, s) != cudaSuccess)
+        return W4A8_ERR_CUDA;
+    if (cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s) != cudaSuccess) return W4A8_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return W4A8_ERR_CUDA;
+    *alpha_out_host = r.alpha;
+    if (colsum_max_host) *colsum_max_host = int64_t(r.colsum_max);
+    const double bound = 127.0 * 7.0 * double(group) * double(r.colsum_max);
+    if (bound >= 2147483648.0) return W4A8_ERR_OVERFLOW_BOUND;
+    return W4A8_OK;
+}
+
+int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group, int32_t path) {
+    (void)path;
+    if (check_gemm_shape(M, N, K, group) != W4A8_OK || M == 0) return 0;
+    DeviceInfo dev;
+    if (current_device(dev) != W4A8_OK) return -1;
+    const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms);
+    return plan_splits_tiles(pl) ? pl.ws_bytes : 0;
+}
+
+w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, const uint8_t* w_packed, const int16_t* S,
+                               int32_t alpha, int64_t M, int64_t N, int64_t K, int32_t group, void* y,
+                               int32_t y_dtype, void* workspace, int64_t workspace_bytes, void* stream) {
+    return run_gemm(w4a8::gemm::kIntScale, q_x, s_a, w_packed, S, nullptr, alpha, M, N, K, group, y, y_dtype,
+                    workspace, workspace_bytes, stream);
+}
+
+w4a8_status w4a8_gemm_floatscale(const int8_t* q_x, const float* s_a, const uint8_t* w_packed, const float* s_g,
+                                 int64_t M, int64_t N, int64_t K, int32_t group, void* y, int32_t y_dtype,
+                                 void* workspace, int64_t workspace_bytes, void* stream) {
+    return run_gemm(w4a8::gemm::kFloatScale, q_x, s_a, w_packed, nullptr, s_g, 1, M, N, K, group, y, y_dtype,
+                    workspace, workspace_bytes, stream);
+}
+
+w4a8_status w4a8_device_status(int32_t* code_host, int32_t clear) {
+    if (!code_host) return W4A8_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    w4a8_status st = current_device(dev);
+    if (st != W4A8_OK) return st;
+    int v = 0;
+    if (cudaMemcpy(&v, dev.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return W4A8_ERR_CUDA;
+    *code_host = v;
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpy(dev.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return W4A8_ERR_CUDA;
+    }
+    return W4A8_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,48 @@
+// Host/device interface of the W4A8 GEMM kernels (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace w4a8 {
+namespace gemm {
+
+enum Path { kIntScale = 0, kFloatScale = 1 };
+enum OutType { kOutF32 = 0, kOutF16 = 1, kOutI32 = 3 };
+
+struct Params {
+    const float* s_a;    // [M] token scales
+    const int16_t* S;    // [G, N] integer group scales (integer-scale path)
+    const float* s_g;    // [G, N] float group scales (float-scale path)
+    void* y;             // [M, N] output
+    int32_t* ws_part;    // [grid][2][128 * BT] partial sums of split tiles
+    int32_t* ws_count;   // [tiles] arrival counters, zero between calls
+    int* status;         // device status word for timeouts
+    int64_t M, N;
+    int64_t G;           // groups along K
+    int32_t kb_per_group;  // 128-wide K blocks per group
+    int64_t m_tiles;
+    int64_t W;           // total (tile, group) steps
+    int64_t grid;        // CTAs
+    float inv_alpha;     // 1 / alpha (exact, alpha is a power of two)
+    int32_t y_dtype;     // OutType
+};
+
+struct Plan {
+    int BT;              // tokens per tile (MMA N)
+    int64_t n_tiles, m_tiles, tiles, G, W, grid;
+    int64_t count_bytes;  // bytes of per-tile counters at the start of the workspace
+    int64_t ws_bytes;     // total workspace bytes
+};
+
+Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms);
+
+cudaError_t launch(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const Params& p, int BT, int path,
+                   cudaStream_t stream);
+
+int token_tile_rows();
+
+}  // namespace gemm
+}  // namespace w4a8

@@ -1,0 +1,35 @@
+// Internal launch entry points of the library's kernels (host side).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace w4a8 {
+
+namespace quant {
+cudaError_t launch(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a,
+                   int* status, cudaStream_t stream, int num_sms);
+}
+
+namespace pack {
+// Layout of the pack workspace (device bytes).
+struct Results {
+    int32_t alpha;         // chosen amplifier
+    int32_t error;         // nonzero: no power of two up to 2^30 suffices
+    float s_min_pos;       // smallest positive scale (+inf when none)
+    float s_max;           // largest scale
+    unsigned long long colsum_max;  // max_n sum_g |S[g,n]|
+};
+constexpr int64_t kPartialsOffset = 256;  // per-block (min, max) pairs start here
+constexpr int kMaxPartialBlocks = 4096;
+
+cudaError_t group_scales(const float* w, int64_t K, int64_t N, int32_t group, float* s_g, cudaStream_t stream);
+// min / max reduction + amplifier search (alpha_in > 0: fixed amplifier)
+cudaError_t amplifier(const float* scales, int64_t count, int32_t alpha_in, void* workspace,
+                      cudaStream_t stream, int num_sms);
+cudaError_t quantize_pack(const float* w, const float* s_g, int32_t alpha, int64_t K, int64_t N, int32_t group,
+                          uint8_t* packed, int16_t* S, void* workspace, cudaStream_t stream);
+}  // namespace pack
+
+}  // namespace w4a8

@@ -1,0 +1,229 @@
+// Per-token symmetric int8 activation quantization for sm_100a.
+//
+// "Quantization" notes, Symmetric Quantization: s = max|x| / 127, z = 0,
+// q = clip(round(x / s), -127, 127); 探秘Transformer系列之（34）量化基礎
+// §2.3.3 (one scale per token row).  round() is half to even and x / s is one
+// IEEE fp32 division, so codes match a plain CPU evaluation bit for bit.
+//
+// HBM-bound: every input byte is read once and every code written once.
+// A persistent grid (SMs x resident CTAs) walks the rows; each CTA stages one
+// row in shared memory with a bulk async copy while it quantizes the previous
+// row (two buffers), reduces |x| with warp shuffles, and writes the codes with
+// 16-byte stores.  Rows too long for two shared-memory buffers take a second
+// kernel that re-reads the row (from L2) instead of staging it.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace w4a8 {
+namespace quant {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+// 16 consecutive elements of a row as fp32.
+template <typename T>
+__device__ __forceinline__ void load16(const T* src, float (&v)[16]);
+
+template <>
+__device__ __forceinline__ void load16<float>(const float* src, float (&v)[16]) {
+    const float4* s = reinterpret_cast<const float4*>(src);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 f = s[i];
+        v[4 * i + 0] = f.x;
+        v[4 * i + 1] = f.y;
+        v[4 * i + 2] = f.z;
+        v[4 * i + 3] = f.w;
+    }
+}
+
+template <>
+__device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16* src, float (&v)[16]) {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const uint4 u = s[i];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {  // bf16 -> fp32 is a 16-bit shift
+            v[8 * i + 2 * j + 0] = __uint_as_float(w[j] << 16);
+            v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+}
+
+// Code for one element: rne(fl32(x / s)) clamped to [-127, 127].
+// Fast path: x * fl32(1/s) is within 2^-23 |x/s| <= 1.6e-5 of x/s, and the
+// correctly rounded quotient within 3.9e-6, so when the product is farther
+// than 2^-14 from a half-integer both round to the same integer.  Otherwise
+// (or for tiny s, whose reciprocal would overflow) take the IEEE division.
+__device__ __forceinline__ int code_i8(float x, float s, float rcp, bool exact_only) {
+    float t = __fmul_rn(x, rcp);
+    float r = rintf(t);
+    if (exact_only || fabsf(t - r) > 0.49993896484375f) {
+        t = __fdiv_rn(x, s);
+        r = rintf(t);
+    }
+    r = fminf(fmaxf(r, -127.0f), 127.0f);
+    return int(r);
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) red[warp] = v;
+    __syncthreads();
+    float r = red[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) r = fmaxf(r, red[w]);
+    return r;
+}
+
+template <typename T>
+__device__ __forceinline__ void quantize_row(const T* row, int64_t K, float s, int8_t* qrow) {
+    const bool zero = (s == 0.0f);
+    const bool exact_only = s < 1e-30f;
+    const float rcp = zero ? 0.0f : __frcp_rn(s);
+    for (int64_t c = threadIdx.x; c < K / 16; c += kThreads) {
+        uint32_t packed[4] = {0u, 0u, 0u, 0u};
+        if (!zero) {
+            float v[16];
+            load16<T>(row + c * 16, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                packed[i >> 2] |= (uint32_t(code_i8(v[i], s, rcp, exact_only)) & 0xFFu) << (8 * (i & 3));
+        }
+        *reinterpret_cast<uint4*>(qrow + c * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ float row_absmax(const T* row, int64_t K, float* red) {
+    float a = 0.0f;
+    for (int64_t c = threadIdx.x; c < K / 16; c += kThreads) {
+        float v[16];
+        load16<T>(row + c * 16, v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
+    }
+    return block_max(a, red);
+}
+
+// Row staged in shared memory by a bulk async copy; two buffers.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) quant_rows_staged(const T* __restrict__ x, int64_t M, int64_t K,
+                                                              int64_t ldx, int8_t* __restrict__ q,
+                                                              float* __restrict__ s_a, int* status) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const uint32_t row_bytes = uint32_t(K * sizeof(T));
+    const uint32_t buf_bytes = (row_bytes + 127u) & ~127u;
+    T* buf[2] = {reinterpret_cast<T*>(smem), reinterpret_cast<T*>(smem + buf_bytes)};
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * buf_bytes);
+    float* red = reinterpret_cast<float*>(bars + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(red + kWarps);
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    int64_t row = blockIdx.x;
+    bool inflight[2] = {false, false};  // meaningful in thread 0, which issues the copies
+    if (threadIdx.x == 0 && row < M) {
+        mbar_arrive_expect_tx(&bars[0], row_bytes);
+        bulk_load(buf[0], x + row * ldx, row_bytes, &bars[0]);
+        inflight[0] = true;
+    }
+    uint32_t phase[2] = {0u, 0u};
+    int st = 0;
+    for (; row < M; row += gridDim.x) {
+        const int64_t next = row + gridDim.x;
+        if (threadIdx.x == 0 && next < M) {  // prefetch the next row into the other buffer
+            mbar_arrive_expect_tx(&bars[st ^ 1], row_bytes);
+            bulk_load(buf[st ^ 1], x + next * ldx, row_bytes, &bars[st ^ 1]);
+            inflight[st ^ 1] = true;
+        }
+        if (!mbar_wait(&bars[st], phase[st], abort_flag, status)) break;
+        inflight[st] = false;
+        phase[st] ^= 1u;
+        const float a = row_absmax<T>(buf[st], K, red);
+        const float s = (a == 0.0f) ? 0.0f : __fdiv_rn(a, 127.0f);
+        if (threadIdx.x == 0) s_a[row] = s;
+        quantize_row<T>(buf[st], K, s, q + row * K);
+        __syncthreads();  // buffer and reduction scratch are free again
+        st ^= 1;
+    }
+    // after a timeout, let copies in flight land before leaving
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < 2; ++b) {
+            if (!inflight[b]) continue;
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&bars[b], phase[b]) && globaltimer_ns() - t0 < 1000000000ull) {
+            }
+        }
+    }
+}
+
+// Long rows: read the row twice from global memory (the second pass hits L2).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) quant_rows_direct(const T* __restrict__ x, int64_t M, int64_t K,
+                                                              int64_t ldx, int8_t* __restrict__ q,
+                                                              float* __restrict__ s_a) {
+    __shared__ float red[kWarps];
+    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+        const T* r = x + row * ldx;
+        const float a = row_absmax<T>(r, K, red);
+        const float s = (a == 0.0f) ? 0.0f : __fdiv_rn(a, 127.0f);
+        if (threadIdx.x == 0) s_a[row] = s;
+        quantize_row<T>(r, K, s, q + row * K);
+        __syncthreads();
+    }
+}
+
+template <typename T>
+static cudaError_t launch_t(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a, int* status,
+                            cudaStream_t stream, int num_sms) {
+    const uint32_t row_bytes = uint32_t(K * sizeof(T));
+    const uint32_t buf_bytes = (row_bytes + 127u) & ~127u;
+    const size_t smem = 2 * size_t(buf_bytes) + 2 * sizeof(uint64_t) + kWarps * sizeof(float) + 16;
+    if (smem <= 200 * 1024) {
+        auto kern = quant_rows_staged<T>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+        if (e != cudaSuccess) return e;
+        if (per_sm < 1) per_sm = 1;
+        const int64_t grid = M < int64_t(num_sms) * per_sm ? M : int64_t(num_sms) * per_sm;
+        kern<<<unsigned(grid), kThreads, smem, stream>>>(x, M, K, ldx, q, s_a, status);
+        return cudaGetLastError();
+    }
+    auto kern = quant_rows_direct<T>;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    const int64_t grid = M < int64_t(num_sms) * per_sm ? M : int64_t(num_sms) * per_sm;
+    kern<<<unsigned(grid), kThreads, 0, stream>>>(x, M, K, ldx, q, s_a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a,
+                   int* status, cudaStream_t stream, int num_sms) {
+    if (bf16)
+        return launch_t<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), M, K, ldx, q, s_a, status, stream,
+                                       num_sms);
+    return launch_t<float>(static_cast<const float*>(x), M, K, ldx, q, s_a, status, stream, num_sms);
+}
+
+}  // namespace quant
+}  // namespace w4a8

@@ -1,0 +1,188 @@
+/*
+ * w4a8_intscale.h -- C ABI of the B200 (sm_100a) W4A8 Integer-Scale library.
+ *
+ * Fine-grained W4A8 linear-layer compute:
+ *   y[m,n] = s_a[m]/alpha * sum_g S[g,n] * sum_{k in g} q_x[m,k] q_w[k,n]
+ * with per-token symmetric int8 activations (q_x, s_a), per-group symmetric
+ * int4 weights (q_w, float group scales s_g), and integer group scales
+ * S = round(s_g * alpha) for a power-of-two amplifier alpha.
+ *
+ * Sources, by page and section:
+ *  - "Quantization" notes, 量化公式 / Symmetric Quantization: q = clip(round(x/s)
+ *    + z, qmin, qmax), s = max|x| / qmax, z = 0, int8 range [-127, 127];
+ *    矩阵乘法中的量化计算: with z = 0 the integer part of a quantized matmul is
+ *    q_W q_X alone.
+ *  - 探秘Transformer系列之（34）量化基礎 §2.3.3: per-token activation scales,
+ *    per-group weight scales (逐组量化).
+ *  - "Integer Scale: A Free Lunch for Faster Fine-grained Quantization of LLMs"
+ *    (summary): Fig. 3(a) shapes X [M,K], W [K,N]; §3.2 / Fig. 3(b) float-scale
+ *    path (one I32->F32 conversion and float multiply per group result);
+ *    §4 / Fig. 3(c) integer scales, integer accumulation, one rescale by
+ *    s_a/alpha; §4 amplifier search; §5.1 Table 1 group 128, symmetric,
+ *    amplifier 1024.
+ *  - 极致量化, 数据打包: several int4 values stored in one byte.
+ *
+ * Conventions for every entry point:
+ *  - Device pointers are caller-owned (any allocator); the library allocates
+ *    no device memory.  Host pointers are named *_host.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Calls are asynchronous on it unless stated "synchronous".
+ *  - Arguments are validated on the host before any launch; an error return
+ *    means nothing was launched.  No C++ exception crosses the ABI.
+ *  - Kernels bound every wait; a wait that runs out (about one second) makes
+ *    the kernel return early and records W4A8_ERR_TIMEOUT in a device status
+ *    word that w4a8_device_status() reads.
+ *  - Layouts are row-major.  All device pointers must be 16-byte aligned.
+ *  - Readings where the pages are silent: round() is round half to even;
+ *    an all-zero row or group gets scale 0 and codes 0; int4 codes are
+ *    symmetric in [-7, 7]; inputs must be finite.
+ */
+#ifndef W4A8_INTSCALE_H
+#define W4A8_INTSCALE_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define W4A8_API __attribute__((visibility("default")))
+#else
+#define W4A8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W4A8_OK = 0,
+    W4A8_ERR_INVALID_ARG = 1,    /* null pointer, bad enum, alpha not a power of two */
+    W4A8_ERR_SHAPE = 2,          /* M/N/K/group outside what the kernels accept */
+    W4A8_ERR_ALIGN = 3,          /* pointer or leading dimension not 16-byte aligned */
+    W4A8_ERR_DTYPE = 4,          /* dtype not supported for this argument */
+    W4A8_ERR_OVERFLOW_BOUND = 5, /* 127*7*group*max_n sum_g|S[g,n]| >= 2^31 */
+    W4A8_ERR_SCALE_RANGE = 6,    /* S would exceed int16, or alpha > 2^30 needed */
+    W4A8_ERR_CUDA = 7,           /* a CUDA runtime call failed */
+    W4A8_ERR_TIMEOUT = 8,        /* a kernel wait ran out (device status only) */
+    W4A8_ERR_WORKSPACE = 9       /* workspace missing or too small */
+} w4a8_status;
+
+typedef enum {
+    W4A8_F32 = 0,
+    W4A8_F16 = 1,
+    W4A8_BF16 = 2,
+    W4A8_I32 = 3 /* raw int32 accumulators (integer-scale GEMM only) */
+} w4a8_dtype;
+
+/* Human-readable name of a status code (static string). */
+W4A8_API const char* w4a8_status_string(int32_t status);
+
+/*
+ * Per-token symmetric int8 activation quantization.
+ * ("Quantization" notes, Symmetric Quantization; 探秘Transformer系列之（34）
+ *  §2.3.3 逐token量化; Integer Scale summary §5.4 per-token 8-bit activations.)
+ *   s_a[m] = fl32(max_k |x[m,k]| / 127)
+ *   q_x[m,k] = clamp(rne(fl32(x[m,k] / s_a[m])), -127, 127)   (0 when s_a[m] = 0)
+ * x       device, [M, ldx] of x_dtype (W4A8_F32 or W4A8_BF16); row m starts at x + m*ldx
+ * M, K    M >= 0 (M = 0 is a no-op), K > 0 and K % 16 == 0; ldx >= K, ldx*sizeof(x) % 16 == 0
+ * q_x     device, [M, K] int8, written
+ * s_a     device, [M] float32, written
+ */
+W4A8_API w4a8_status quantize_act_per_token(const void* x, int32_t x_dtype, int64_t M, int64_t K, int64_t ldx,
+                                   int8_t* q_x, float* s_a, void* stream);
+
+/*
+ * Amplifier search over a set of float group scales (synchronous).
+ * (Integer Scale summary §4 heuristic search.)  alpha is the smallest power
+ * of two 2^j, j >= 0, with s_min * alpha >= 1, s_min the smallest POSITIVE
+ * scale; 1 when no scale is positive or s_min >= 1.
+ * scales     device, [count] float32
+ * workspace  device, >= W4A8_PACK_WORKSPACE_BYTES bytes, contents scratch
+ * alpha_host host, written
+ * Returns W4A8_ERR_SCALE_RANGE when alpha would exceed 2^30.
+ */
+#define W4A8_PACK_WORKSPACE_BYTES (1 << 20)
+W4A8_API w4a8_status w4a8_amplifier_search(const float* scales, int64_t count, void* workspace,
+                                  int32_t* alpha_host, void* stream);
+
+/*
+ * Per-group symmetric int4 weight quantization, nibble packing, amplifier and
+ * integer scales (synchronous: it waits for the stream once or twice).
+ * (探秘Transformer系列之（34）§2.3.3 逐组量化; Integer Scale summary Fig. 3(a),
+ *  §4; 极致量化 数据打包.)
+ *   s_g[g,n]  = fl32(max_{k in g} |w[k,n]| / 7)
+ *   q_w[k,n]  = clamp(rne(fl32(w[k,n] / s_g[g(k),n])), -7, 7)
+ *   w_packed[n, k/2] = (q_w[k,n] & 0xF) | (q_w[k+1,n] & 0xF) << 4   (k even)
+ *   alpha     = alpha_in if alpha_in > 0 (must be a power of two <= 2^30),
+ *               else the amplifier search over this layer's s_g
+ *   S[g,n]    = rne(s_g[g,n] * alpha)
+ * w          device, [K, N] float32
+ * K, N       K % group == 0, N % 8 == 0, N > 0
+ * group      even, group % 32 == 0 (128 in the method)
+ * w_packed   device, [N, K/2] uint8, written; may be NULL together with S to
+ *            compute s_g only (alpha_out and colsum_max_host are then untouched)
+ * s_g        device, [K/group, N] float32, written
+ * S          device, [K/group, N] int16, written (or NULL, see w_packed)
+ * alpha_out_host      host int32, written: the alpha used
+ * colsum_max_host     host int64, written (may be NULL): max_n sum_g |S[g,n]|
+ * workspace  device, >= W4A8_PACK_WORKSPACE_BYTES bytes, contents scratch
+ * Errors: W4A8_ERR_SCALE_RANGE if max S > 32767; W4A8_ERR_OVERFLOW_BOUND if
+ * 127*7*group*colsum_max >= 2^31 (outputs are written in both cases).
+ */
+W4A8_API w4a8_status pack_w4_groupwise(const float* w, int64_t K, int64_t N, int32_t group, int32_t alpha_in,
+                              uint8_t* w_packed, float* s_g, int16_t* S, int32_t* alpha_out_host,
+                              int64_t* colsum_max_host, void* workspace, void* stream);
+
+/*
+ * Bytes of workspace the GEMMs below need for (M, N, K, group) on the current
+ * device (0 when they need none).  path: 0 integer scale, 1 float scale.
+ * The workspace must be zero-filled before its first use; the GEMMs leave it
+ * zero-filled again on success, so one allocation serves any number of calls
+ * that run one after another (calls that overlap on the GPU need one each).
+ * After an error or a timeout, zero it again.
+ */
+W4A8_API int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group, int32_t path);
+
+/*
+ * W4A8 GEMM with integer group scales (the Integer-Scale scheme).
+ * (Integer Scale summary §4 / Fig. 3(c); "Quantization" notes 矩阵乘法中的量化计算.)
+ *   P_g[m,n] = sum_{k in g} q_x[m,k] q_w[k,n]            (int8 x int4 -> int32, tensor cores)
+ *   acc[m,n] = sum_g S[g,n] * P_g[m,n]                    (int32, exact)
+ *   y[m,n]   = fl_out(fl32(acc) * fl32(s_a[m] / alpha))   (one conversion per output)
+ * q_x, s_a   device, [M, K] int8 and [M] float32 (from quantize_act_per_token)
+ * w_packed   device, [N, K/2] uint8; S device [K/group, N] int16 (from pack_w4_groupwise)
+ * alpha      power of two, 1 <= alpha <= 2^30
+ * M >= 0 (0 is a no-op), N % 8 == 0, K % 128 == 0, group % 128 == 0, K % group == 0
+ * y          device, [M, N] of y_dtype: W4A8_F16, W4A8_F32, or W4A8_I32 (acc itself)
+ * workspace  device, >= w4a8_gemm_workspace_size(M, N, K, group, 0) bytes (may be
+ *            NULL when that size is 0), zero-filled, see above
+ * Precondition (established by pack_w4_groupwise): the worst-case accumulator
+ * 127*7*group*max_n sum_g |S[g,n]| stays below 2^31.
+ */
+W4A8_API w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, const uint8_t* w_packed,
+                               const int16_t* S, int32_t alpha, int64_t M, int64_t N, int64_t K,
+                               int32_t group, void* y, int32_t y_dtype, void* workspace,
+                               int64_t workspace_bytes, void* stream);
+
+/*
+ * W4A8 GEMM with float group scales, the comparison path.
+ * (Integer Scale summary §3.2 / Fig. 3(b): every group's int32 result is
+ *  converted to fp32 and multiplied by its float scale.)
+ *   y[m,n] = fl_out(s_a[m] * sum_g s_g[g,n] * float(P_g[m,n]))   (fp32, group order)
+ * Arguments as w4a8_gemm_intscale with float s_g [K/group, N] in place of S and
+ * alpha; y_dtype W4A8_F16 or W4A8_F32; workspace size from path 1.
+ */
+W4A8_API w4a8_status w4a8_gemm_floatscale(const int8_t* q_x, const float* s_a, const uint8_t* w_packed,
+                                 const float* s_g, int64_t M, int64_t N, int64_t K, int32_t group,
+                                 void* y, int32_t y_dtype, void* workspace, int64_t workspace_bytes,
+                                 void* stream);
+
+/*
+ * Reads (and with clear != 0 resets) the device status word of the current
+ * device that bounded waits write on a timeout.  Synchronous.  0 = no timeout.
+ */
+W4A8_API w4a8_status w4a8_device_status(int32_t* code_host, int32_t clear);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A8_INTSCALE_H */
