@@ -1,0 +1,423 @@
+"""Benchmark of the W4A8 Integer-Scale hot path on B200.
+
+Workload (default): the FFN up-projection batch sweep at the kernel shape of
+the Integer Scale summary's kernel comparison (§5.2, Fig. 5a / Fig. 6):
+K = 4096, N = 22016, group 128, alpha = 1024, bf16 activations,
+M in {1, 8, 32, 128, 512, 1024}, fp16 output.  One step = for every M:
+per-token int8 quantization of X [M, K] and the integer-scale W4A8 GEMM.
+The float-scale GEMM (the comparison path) is timed beside it per M.
+
+Weights are packed once before timing (offline step).  Six packed copies are
+rotated, one per M, so every GEMM streams weights that the previous five
+GEMMs (>= 225 MB) have evicted from the 126 MB L2.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bit_gemm_quantize_b200 import workloads  # noqa: E402
+
+K_DIM, N_DIM, GROUP, ALPHA = 4096, 22016, 128, 1024
+SWEEP = workloads.SWEEP_M
+METRIC = "W4A8-IntScale GEMM TOPS and HBM GB/s vs M (1-4096); % of roofline on 1 B200"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+# nominal dense int8 : bf16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s)
+INT8_PER_BF16 = 2.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def config_dict():
+    return {
+        "workload": "ffn_up_sweep",
+        "K": K_DIM,
+        "N": N_DIM,
+        "M": list(SWEEP),
+        "group": GROUP,
+        "alpha": ALPHA,
+        "x_dtype": "bf16",
+        "out": "f16",
+        "l2": "inputs larger than L2: 6 packed weight copies (271 MB) rotated, one per M",
+        "timing": "CUDA events between CUDA-graph replays, one graph per kernel launch",
+    }
+
+
+def alg_bytes(M, path="is"):
+    """Bytes the method must move for one GEMM: int4 W, group scales, int8 codes,
+    token scales, fp16 output."""
+    G = K_DIM // GROUP
+    scale_bytes = (2 if path == "is" else 4) * G * N_DIM
+    return N_DIM * K_DIM // 2 + scale_bytes + M * K_DIM + 4 * M + 2 * M * N_DIM
+
+
+def alg_ops(M):
+    return 2 * M * N_DIM * K_DIM
+
+
+def quant_bytes(M):
+    return 2 * M * K_DIM + M * K_DIM + 4 * M
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active," \
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown," \
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+
+class OracleLeg:
+    """The oracle, as it stands, on bounded samples of the workload: token rows
+    of the batch through per-token quantize + group-wise integer GEMM + rescale
+    over the full K x N layer.  The weights are quantized once beforehand
+    (the offline step, untimed)."""
+
+    def __init__(self, seed: int = 1):
+        import oracle
+
+        self.oracle = oracle
+        wl = workloads.make_linear(1, K_DIM, N_DIM, x_dtype="bf16", seed=seed)
+        self.qw, sg = oracle.quantize_groups(wl.w, GROUP)
+        self.S = oracle.integer_scales(sg, ALPHA)
+
+    def run(self, rows: int, seed: int):
+        o = self.oracle
+        x = workloads.make_linear(rows, K_DIM, 8, x_dtype="bf16", seed=seed).x
+        t0 = time.perf_counter()
+        qx, sa = o.quantize_act_per_token(x)
+        acc = o.intscale_acc(qx, self.qw, self.S, GROUP)
+        y = o.round_output(o.intscale_output(acc, sa, ALPHA), "f16")
+        dt = time.perf_counter() - t0
+        assert y.shape == (rows, N_DIM)
+        return dt
+
+
+def cpu_oracle_sample(rows: int = 32, seed: int = 1):
+    leg = OracleLeg(seed)
+    dt = leg.run(rows, seed + 1)
+    return {"value": alg_ops(rows) / dt / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} token rows x full K={K_DIM}, N={N_DIM} layer: per-token quantize + "
+                      f"group-wise integer GEMM + rescale, single-threaded C, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    rows = 2
+    leg = OracleLeg(1)
+    total_t = 0.0
+    for i in range(args.warmup + args.steps):
+        dt = leg.run(rows, 10 + i)
+        if i >= args.warmup:
+            total_t += dt
+    v = alg_ops(rows) * args.steps / total_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8xi4->i64",
+        "data": "synthetic", "config": config_dict(),
+        "cpu_baseline": {"value": v, "unit": "TOPS", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: {rows} token rows x full K={K_DIM}, N={N_DIM} layer through the "
+                                   "oracle (quantize + group-wise integer GEMM + rescale), single-threaded C"},
+        "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import bit_gemm_quantize_b200 as bgq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    hbm_peak, bf16_peak, peak_src = load_peaks()
+    int8_peak = bf16_peak * INT8_PER_BF16
+
+    # ---- inputs (per rank: an independent layer; weak scaling)
+    wl = workloads.make_linear(1, K_DIM, N_DIM, x_dtype="bf16", seed=1000 + rank)
+    w_dev = torch.from_numpy(wl.w).to(dev)
+    pk = bgq.pack_w4_groupwise(w_dev, group=GROUP, alpha=ALPHA)
+    del w_dev
+    copies = [pk] + [{k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in pk.items()}
+                     for _ in range(len(SWEEP) - 1)]
+    xs, qs, ss, ys, yfs = [], [], [], [], []
+    for i, M in enumerate(SWEEP):
+        x = workloads.make_linear(M, K_DIM, 8, x_dtype="bf16", seed=2000 + 10 * rank + i).x
+        xs.append(torch.from_numpy(x).to(dev).to(torch.bfloat16))
+        qs.append(torch.empty((M, K_DIM), dtype=torch.int8, device=dev))
+        ss.append(torch.empty((M,), dtype=torch.float32, device=dev))
+        ys.append(torch.empty((M, N_DIM), dtype=torch.float16, device=dev))
+        yfs.append(torch.empty((M, N_DIM), dtype=torch.float16, device=dev))
+    ws = {M: bgq.gemm_workspace(M, N_DIM, K_DIM, GROUP, 0, dev) for M in SWEEP}
+    wsf = {M: bgq.gemm_workspace(M, N_DIM, K_DIM, GROUP, 1, dev) for M in SWEEP}
+    # one workspace serves all sequential calls: keep the largest
+    ws_all = max([w for w in list(ws.values()) + list(wsf.values()) if w is not None],
+                 key=lambda t: t.numel(), default=None)
+    stream = torch.cuda.current_stream(dev)
+
+    def quant(i):
+        bgq.quantize_act_per_token(xs[i], qs[i], ss[i])
+
+    def gemm_is(i):
+        c = copies[i]
+        bgq.w4a8_gemm_intscale(qs[i], ss[i], c["packed"], c["S"], ALPHA, group=GROUP, out="f16", y=ys[i],
+                               workspace=ws_all)
+
+    def gemm_fs(i):
+        c = copies[i]
+        bgq.w4a8_gemm_floatscale(qs[i], ss[i], c["packed"], c["s_g"], group=GROUP, out="f16", y=yfs[i],
+                                 workspace=ws_all)
+
+    # warm-up through direct calls, then capture one CUDA graph per (M, kernel)
+    # so that the timed steps replay kernels without host launch overhead
+    for _ in range(max(3, args.warmup)):
+        for i in range(len(SWEEP)):
+            quant(i)
+            gemm_is(i)
+            gemm_fs(i)
+    torch.cuda.synchronize(dev)
+    graphs = []
+    for i in range(len(SWEEP)):
+        row = []
+        for fn in (quant, gemm_is, gemm_fs):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn(i)
+            row.append(g)
+        graphs.append(row)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        for gq, gi, gf in graphs:
+            gq.replay()
+            gi.replay()
+            gf.replay()
+    torch.cuda.synchronize(dev)
+
+    # ---- timed region: K steps of the hot path (quantize + integer-scale GEMM per M)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in SWEEP] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for k in range(args.steps):
+        for i, (gq, gi, _) in enumerate(graphs):
+            evs[k][i][0].record(stream)
+            gq.replay()
+            evs[k][i][1].record(stream)
+            gi.replay()
+            evs[k][i][2].record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = start.elapsed_time(stop)
+    q_ms = np.array([[evs[k][i][0].elapsed_time(evs[k][i][1]) for i in range(len(SWEEP))] for k in range(args.steps)])
+    g_ms = np.array([[evs[k][i][1].elapsed_time(evs[k][i][2]) for i in range(len(SWEEP))] for k in range(args.steps)])
+
+    # float-scale comparison, same rotation, timed separately
+    fevs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in SWEEP] for _ in range(args.steps)]
+    for k in range(args.steps):
+        for i, (_, _, gf) in enumerate(graphs):
+            fevs[k][i][0].record(stream)
+            gf.replay()
+            fevs[k][i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    f_ms = np.array([[fevs[k][i][0].elapsed_time(fevs[k][i][1]) for i in range(len(SWEEP))] for k in range(args.steps)])
+
+    # ---- end to end through the public API with host buffers
+    xh = [x.cpu().pin_memory() for x in xs]
+    yh = [torch.empty((M, N_DIM), dtype=torch.float16).pin_memory() for M in SWEEP]
+    xd = [torch.empty_like(x) for x in xs]
+
+    def e2e_step():
+        # the call a user makes: public API, host input in, host output back
+        for i, M in enumerate(SWEEP):
+            c = copies[i]
+            xd[i].copy_(xh[i], non_blocking=True)
+            bgq.quantize_act_per_token(xd[i], qs[i], ss[i])
+            bgq.w4a8_gemm_intscale(qs[i], ss[i], c["packed"], c["S"], ALPHA, group=GROUP, out="f16", y=ys[i],
+                                   workspace=ws_all)
+            yh[i].copy_(ys[i], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = sum(M * K_DIM * 2 for M in SWEEP)
+    d2h = sum(M * N_DIM * 2 for M in SWEEP)
+
+    # ---- aggregate over ranks: max time
+    vals = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(vals[0]), float(vals[1])
+    ops_step = sum(alg_ops(M) for M in SWEEP)
+    value = world * ops_step * args.steps / (total_ms * 1e-3) / 1e12
+    e2e_value = world * ops_step * args.steps / (e2e_ms * 1e-3) / 1e12
+
+    sweep = []
+    for i, M in enumerate(SWEEP):
+        g = float(np.mean(g_ms[:, i])) * 1e3  # us
+        f = float(np.mean(f_ms[:, i])) * 1e3
+        q = float(np.mean(q_ms[:, i])) * 1e3
+        b_is = alg_bytes(M, "is")
+        t_hbm = b_is / (hbm_peak * 1e9)
+        t_tc = alg_ops(M) / (int8_peak * 1e12)
+        bound = "hbm" if t_hbm >= t_tc else "tensor"
+        ach_gbs = b_is / (g * 1e-6) / 1e9
+        ach_tops = alg_ops(M) / (g * 1e-6) / 1e12
+        sweep.append({
+            "M": M, "is_us": round(g, 2), "fs_us": round(f, 2), "quant_us": round(q, 2),
+            "is_tops": round(ach_tops, 2), "is_gbs": round(ach_gbs, 1),
+            "fs_tops": round(alg_ops(M) / (f * 1e-6) / 1e12, 2),
+            "bound": bound,
+            "frac_hbm": round(ach_gbs / hbm_peak, 4), "frac_int8": round(ach_tops / int8_peak, 4),
+            "is_faster_than_fs": g < f,
+        })
+    shares = g_ms.mean(axis=0)
+    dom = int(np.argmax(shares))
+    Md = SWEEP[dom]
+    gd = float(np.mean(g_ms[:, dom])) * 1e-3  # s
+    if sweep[dom]["bound"] == "hbm":
+        roof = {"bound": "hbm", "achieved": alg_bytes(Md) / gd / 1e9, "peak": hbm_peak, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": alg_ops(Md) / gd / 1e12, "peak": int8_peak, "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = f"w4a8_gemm_kernel (integer scale), M={Md} launch"
+    roof["peak_source"] = (f"{peak_src}: HBM copy {hbm_peak} GB/s; int8 = bf16 {bf16_peak} TFLOP/s x "
+                           f"{INT8_PER_BF16} (nominal int8:bf16 ratio)")
+
+    del graphs
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8xi4->i32", "data": "synthetic",
+        "config": config_dict(), "roofline": roof, "sweep": sweep, "clocks": clocks,
+        "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * len(SWEEP) * args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

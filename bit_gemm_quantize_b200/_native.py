@@ -37,9 +37,9 @@ STATUS = {
 
 
 class W4A8Error(RuntimeError):
-    def __init__(self, fn: str, code: int):
+    def __init__(self, fn: str, code: int, detail: str = ""):
         self.code = code
-        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}{detail}")
 
 
 _lock = threading.Lock()
@@ -74,6 +74,8 @@ def load(path: str = LIB_PATH):
             "w4a8_gemm_intscale": ([P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
             "w4a8_gemm_floatscale": ([P, P, P, P, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
             "w4a8_device_status": ([P, I32_], I32_),
+            "w4a8_last_cuda_error": ([I32_], I32_),
+            "w4a8_cuda_error_string": ([I32_], ctypes.c_char_p),
         }
         for name, (args, res) in sigs.items():
             fn = getattr(lib, name)
@@ -85,7 +87,12 @@ def load(path: str = LIB_PATH):
 
 def _check(fn: str, code: int):
     if code != 0:
-        raise W4A8Error(fn, code)
+        detail = ""
+        if code == 7:  # W4A8_ERR_CUDA: name the runtime error behind it
+            lib = load()
+            e = int(lib.w4a8_last_cuda_error(1))
+            detail = f" ({lib.w4a8_cuda_error_string(e).decode()})"
+        raise W4A8Error(fn, code, detail)
 
 
 def _ptr(t):

@@ -8,7 +8,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/w4a8_intscale.h"
+#include "w4a8_intscale.h"
 #include "gemm_w4a8.h"
 #include "kernels.h"
 
@@ -29,15 +29,29 @@ struct DeviceInfo {
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_devices_mutex;
 
+// Last CUDA runtime error seen by this thread's library calls.
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+w4a8_status cuda_fail(cudaError_t e) {
+    t_last_cuda_error = e;
+    return W4A8_ERR_CUDA;
+}
+
+#define W4A8_CUDA_TRY(expr)                           \
+    do {                                              \
+        const cudaError_t w4a8_e_ = (expr);           \
+        if (w4a8_e_ != cudaSuccess) return cuda_fail(w4a8_e_); \
+    } while (0)
+
 w4a8_status current_device(DeviceInfo& out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return W4A8_ERR_CUDA;
+    W4A8_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return W4A8_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_devices_mutex);
     DeviceInfo& d = g_devices[dev];
     if (!d.ready) {
-        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return W4A8_ERR_CUDA;
-        if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_status_word) != cudaSuccess)
-            return W4A8_ERR_CUDA;
+        W4A8_CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+        W4A8_CUDA_TRY(cudaGetSymbolAddress(reinterpret_cast<void**>(&d.status), g_status_word));
         d.ready = true;
     }
     out = d;
@@ -123,8 +137,9 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     }
 
     CUtensorMap tm_w, tm_x;
-    if (!make_map_u8(&tm_w, w_packed, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 64, 128,
-                     CU_TENSOR_MAP_SWIZZLE_NONE))
+    // packed weights: one box = 128 columns x 128 bytes (two 128-wide K blocks), 128-byte swizzle
+    if (!make_map_u8(&tm_w, w_packed, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2),
+                     uint32_t(w4a8::gemm::weight_box_bytes()), 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return W4A8_ERR_CUDA;
     if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(M), uint64_t(K), 128, uint32_t(pl.BT),
                      CU_TENSOR_MAP_SWIZZLE_128B))
@@ -148,8 +163,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     p.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
     p.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
                                     : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
-    if (w4a8::gemm::launch(tm_w, tm_x, p, pl.BT, path, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-        return W4A8_ERR_CUDA;
+    W4A8_CUDA_TRY(w4a8::gemm::launch(tm_w, tm_x, p, pl.BT, path, static_cast<cudaStream_t>(stream)));
     return W4A8_OK;
 }
 
@@ -184,9 +198,8 @@ w4a8_status quantize_act_per_token(const void* x, int32_t x_dtype, int64_t M, in
     DeviceInfo dev;
     w4a8_status st = current_device(dev);
     if (st != W4A8_OK) return st;
-    if (w4a8::quant::launch(x, x_dtype == W4A8_BF16, M, K, ldx, q_x, s_a, dev.status,
-                            static_cast<cudaStream_t>(stream), dev.sms) != cudaSuccess)
-        return W4A8_ERR_CUDA;
+    W4A8_CUDA_TRY(w4a8::quant::launch(x, x_dtype == W4A8_BF16, M, K, ldx, q_x, s_a, dev.status,
+                                      static_cast<cudaStream_t>(stream), dev.sms));
     return W4A8_OK;
 }
 
@@ -199,10 +212,10 @@ w4a8_status w4a8_amplifier_search(const float* scales, int64_t count, void* work
     w4a8_status st = current_device(dev);
     if (st != W4A8_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (w4a8::pack::amplifier(scales, count, 0, workspace, s, dev.sms) != cudaSuccess) return W4A8_ERR_CUDA;
+    W4A8_CUDA_TRY(w4a8::pack::amplifier(scales, count, 0, workspace, s, dev.sms));
     w4a8::pack::Results r;
-    if (cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s) != cudaSuccess) return W4A8_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return W4A8_ERR_CUDA;
+    W4A8_CUDA_TRY(cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s));
+    W4A8_CUDA_TRY(cudaStreamSynchronize(s));
     if (r.error) return W4A8_ERR_SCALE_RANGE;
     *alpha_host = r.alpha;
     return W4A8_OK;
@@ -224,24 +237,26 @@ w4a8_status pack_w4_groupwise(const float* w, int64_t K, int64_t N, int32_t grou
     w4a8_status st = current_device(dev);
     if (st != W4A8_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (w4a8::pack::group_scales(w, K, N, group, s_g, s) != cudaSuccess) return W4A8_ERR_CUDA;
-    if (scales_only) return cudaStreamSynchronize(s) == cudaSuccess ? W4A8_OK : W4A8_ERR_CUDA;
+    W4A8_CUDA_TRY(w4a8::pack::group_scales(w, K, N, group, s_g, s));
+    if (scales_only) {
+        W4A8_CUDA_TRY(cudaStreamSynchronize(s));
+        return W4A8_OK;
+    }
 
     const int64_t G = K / group;
-    if (w4a8::pack::amplifier(s_g, G * N, alpha_in, workspace, s, dev.sms) != cudaSuccess) return W4A8_ERR_CUDA;
+    W4A8_CUDA_TRY(w4a8::pack::amplifier(s_g, G * N, alpha_in, workspace, s, dev.sms));
     w4a8::pack::Results r;
-    if (cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s) != cudaSuccess) return W4A8_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return W4A8_ERR_CUDA;
+    W4A8_CUDA_TRY(cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s));
+    W4A8_CUDA_TRY(cudaStreamSynchronize(s));
     if (r.error) return W4A8_ERR_SCALE_RANGE;
     // the largest integer scale is round(s_max * alpha)
     if (std::nearbyint(double(r.s_max) * double(r.alpha)) > 32767.0) {
         *alpha_out_host = r.alpha;
         return W4A8_ERR_SCALE_RANGE;
     }
-    if (w4a8::pack::quantize_pack(w, s_g, r.alpha, K, N, group, w_packed, S, workspace, s) != cudaSuccess)
-        return W4A8_ERR_CUDA;
-    if (cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s) != cudaSuccess) return W4A8_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return W4A8_ERR_CUDA;
+    W4A8_CUDA_TRY(w4a8::pack::quantize_pack(w, s_g, r.alpha, K, N, group, w_packed, S, workspace, s));
+    W4A8_CUDA_TRY(cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s));
+    W4A8_CUDA_TRY(cudaStreamSynchronize(s));
     *alpha_out_host = r.alpha;
     if (colsum_max_host) *colsum_max_host = int64_t(r.colsum_max);
     const double bound = 127.0 * 7.0 * double(group) * double(r.colsum_max);
@@ -272,17 +287,25 @@ w4a8_status w4a8_gemm_floatscale(const int8_t* q_x, const float* s_a, const uint
                     workspace, workspace_bytes, stream);
 }
 
+int32_t w4a8_last_cuda_error(int32_t clear) {
+    const int32_t e = int32_t(t_last_cuda_error);
+    if (clear) t_last_cuda_error = cudaSuccess;
+    return e;
+}
+
+const char* w4a8_cuda_error_string(int32_t code) { return cudaGetErrorString(cudaError_t(code)); }
+
 w4a8_status w4a8_device_status(int32_t* code_host, int32_t clear) {
     if (!code_host) return W4A8_ERR_INVALID_ARG;
     DeviceInfo dev;
     w4a8_status st = current_device(dev);
     if (st != W4A8_OK) return st;
     int v = 0;
-    if (cudaMemcpy(&v, dev.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return W4A8_ERR_CUDA;
+    W4A8_CUDA_TRY(cudaMemcpy(&v, dev.status, sizeof(int), cudaMemcpyDeviceToHost));
     *code_host = v;
     if (clear) {
         const int zero = 0;
-        if (cudaMemcpy(dev.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return W4A8_ERR_CUDA;
+        W4A8_CUDA_TRY(cudaMemcpy(dev.status, &zero, sizeof(int), cudaMemcpyHostToDevice));
     }
     return W4A8_OK;
 }

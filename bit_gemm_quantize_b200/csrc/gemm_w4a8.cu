@@ -12,19 +12,28 @@
 // lane therefore owns one output column n, so the group scale S[g,n] is a
 // per-thread scalar in the per-group drain.
 //
-//   HBM --TMA--> packed int4 tile [128 n][64 B]  --unpack warps-->
-//   int8 tile [128 n][128 k] (128-byte swizzle, K-major) = MMA operand A
-//   HBM --TMA--> token codes [BT m][128 k] (128-byte swizzle) = MMA operand B
-//   tcgen05.mma.kind::i8 x4 (K = 32 each) -> TMEM int32 P_g [128 lanes][BT cols]
-//   epilogue warps: tcgen05.ld P_g, acc += S[g,n] * P_g (or accf += s_g * float(P_g))
-//   after the last group: y = acc * s_a[m] / alpha  (or accf * s_a[m])
+// Data flow per pipeline stage (256 consecutive K):
+//   HBM --TMA--> packed int4 box [128 n][128 B] (128-byte swizzle)      (W ring)
+//   HBM --TMA--> token codes [BT m][128 k] x2 (128-byte swizzle)        (X ring)
+//   unpack warps: packed W -> int8 [128 n][128 k] x2, K-major, 128-byte
+//   swizzle = MMA operand A                                             (A ring)
+//   tcgen05.mma.kind::i8, K = 32 each, accumulating one group's P_g in a
+//   TMEM buffer [128 lanes][BT columns]                                 (TMEM ring)
+//   epilogue warps per group: tcgen05.ld P_g, acc += S[g,n] * P_g (or
+//   accf += s_g * float(P_g)); after the last group y = acc * s_a[m] / alpha
+//   (or accf * s_a[m]).
+// The W ring is released by the unpack warps as soon as they have read a
+// stage (plain mbarrier arrivals), so the HBM stream only waits on the unpack;
+// the X and A rings are released by tcgen05.commit after the MMAs.
 //
 // Work partition: the (tile, group) steps of the whole problem are split into
 // one contiguous range per CTA of a persistent grid (stream-K).  A tile whose
 // groups fall into several CTAs' ranges is combined through a workspace: each
-// contributor stores its partial, the last one to arrive (per-tile counter)
-// sums the partials in CTA order and writes y.  Integer partials are exact;
-// float partials are summed in a fixed order, so results are deterministic.
+// contributor stores its partial, the last one to arrive (an arrival counter
+// per split tile, indexed by the tile's first contributing CTA, which is the
+// first contributor of no other split tile) sums the partials in CTA order
+// and writes y.  Integer partials are exact; float partials are summed in a
+// fixed order, so results are deterministic.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -38,35 +47,50 @@ namespace w4a8 {
 namespace gemm {
 
 constexpr int kTileN = 128;   // weight columns per tile (MMA M)
-constexpr int kBlockK = 128;  // K per pipeline stage
-constexpr int kUnpackWarps = 4;
+constexpr int kBlockK = 128;  // K per MMA block (one 128-byte swizzle row of int8)
+constexpr int kStageK = 256;  // K per pipeline stage (one 128-byte row of packed int4)
 constexpr int kEpiWarps = 8;
-constexpr int kNumWarps = 2 + kUnpackWarps + kEpiWarps;
-constexpr int kThreads = kNumWarps * 32;
+constexpr int64_t kCounterBytes = 4096;  // one int32 arrival counter per CTA, fixed region
+constexpr int64_t kMaxGrid = kCounterBytes / 4;
 
-template <int BT>
+template <int BT, int PATH>
 struct Cfg {
-    static constexpr int kA = kTileN * kBlockK;       // unpacked weights, bytes
-    static constexpr int kB = BT * kBlockK;           // token codes, bytes
-    static constexpr int kWp = kTileN * kBlockK / 2;  // packed weights, bytes
-    static constexpr int kStageBytes = kA + kB + kWp;
-    static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
-    static constexpr int offA = 0;
-    static constexpr int offB = offA + kStages * kA;
-    static constexpr int offWp = offB + kStages * kB;
-    static constexpr int offBar = offWp + kStages * kWp;
-    static constexpr int kBars = 3 * kStages + 5;  // full, wready, empty, tfull x2, tempty x2, mma_done
+    // int4 -> int8 unpack warps: more of them for small token tiles, where the
+    // unpack is on the HBM critical path and the epilogue needs few registers.
+    static constexpr int kUnpackWarps = BT <= 32 ? 8 : 4;
+    static constexpr int kThreads = 32 * (2 + kUnpackWarps + kEpiWarps);
+    // TMEM accumulator buffers: the MMA may run kAcc - 1 groups ahead of the
+    // per-group drain, so the drain's latency is hidden.
+    static constexpr int kAcc = BT == 128 ? 4 : 8;
+    // Unpack to 16*q (nibble into the high half of each byte, 5 integer ops per
+    // 8 weights) instead of q (9 ops).  The float-scale path folds the 1/16 into
+    // s_g for free; the integer-scale path pays one shift per output per group,
+    // worth it only while the unpack dominates (small token tiles).
+    static constexpr bool kX16 = (PATH == kFloatScale) || BT <= 32;
+    static constexpr int kWBytes = kTileN * kStageK / 2;  // packed weights per stage: 16 KB
+    static constexpr int kXBytes = BT * kStageK;          // token codes per stage
+    static constexpr int kABytes = kTileN * kStageK;      // unpacked weights per stage: 32 KB
+    static constexpr int kSA = 2;
+    static constexpr int kSW = BT <= 32 ? 7 : (BT == 64 ? 6 : 3);
+    static constexpr int kSX = BT == 16 ? 8 : (BT == 32 ? 4 : 3);
+    static constexpr int offW = 0;
+    static constexpr int offX = offW + kSW * kWBytes;
+    static constexpr int offA = offX + kSX * kXBytes;
+    static constexpr int offBar = offA + kSA * kABytes;
+    static constexpr int kBars = 2 * kSW + 2 * kSX + 2 * kSA + 2 * kAcc + 1;
     static constexpr int offMisc = offBar + kBars * 8;
     static constexpr int kSmemBytes = offMisc + 64 + 1024;  // + slack to align the base to 1024
-    static constexpr uint32_t kTmemCols = (2 * BT) < 32 ? 32u : uint32_t(2 * BT);
-    static_assert(kB % 1024 == 0, "token tile must hold whole 8-row swizzle atoms");
-    static_assert(kStages >= 2, "pipeline too shallow");
+    static constexpr uint32_t kTmemCols = (kAcc * BT) < 32 ? 32u : uint32_t(kAcc * BT);
+    static_assert(kAcc * BT <= 512 && (kTmemCols & (kTmemCols - 1)) == 0, "TMEM allocation");
+    static_assert(kXBytes % 2048 == 0, "token stage must hold whole 8-row swizzle atoms per k-block");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
 // One contiguous run of groups [g0, g1) of one tile inside a CTA's range.
 struct Segment {
     int64_t tile;
-    int g0, g1;
+    int32_t n_tile, m_tile;
+    int32_t g0, g1;
     int64_t first;  // flattened index of the segment's first step
 };
 
@@ -77,36 +101,104 @@ __device__ __forceinline__ int64_t range_owner(int64_t i, int64_t W, int64_t gri
     return ((i + 1) * grid - 1) / W;
 }
 
-// Iterates the segments of CTA `b`.
+// Iterates the segments of CTA `b`.  The divisions happen once, at the start
+// of the range; afterwards the tile coordinates advance incrementally (64-bit
+// division is a long software sequence on the GPU).
 struct SegmentIter {
-    int64_t i, end, G;
+    int64_t i, end, tile;
+    int32_t G, g, n_tile, m_tile, m_tiles;
     __device__ SegmentIter(const Params& p, int64_t b) {
-        G = p.G;
+        G = int32_t(p.G);
+        m_tiles = int32_t(p.m_tiles);
         i = range_start(b, p.W, p.grid);
         end = range_start(b + 1, p.W, p.grid);
+        tile = i / G;
+        g = int32_t(i - tile * G);
+        n_tile = int32_t(tile / m_tiles);
+        m_tile = int32_t(tile - int64_t(n_tile) * m_tiles);
     }
     __device__ bool next(Segment& s) {
         if (i >= end) return false;
-        s.tile = i / G;
-        s.g0 = int(i - s.tile * G);
-        int64_t stop = (s.tile + 1) * G < end ? (s.tile + 1) * G : end;
-        s.g1 = int(stop - s.tile * G);
+        s.tile = tile;
+        s.n_tile = n_tile;
+        s.m_tile = m_tile;
+        s.g0 = g;
+        const int64_t left = end - i;
+        s.g1 = (left >= int64_t(G - g)) ? G : g + int32_t(left);
         s.first = i;
-        i = stop;
+        i += s.g1 - s.g0;
+        if (s.g1 == G) {
+            g = 0;
+            ++tile;
+            if (++m_tile == m_tiles) {
+                m_tile = 0;
+                ++n_tile;
+            }
+        } else {
+            g = s.g1;
+        }
+        return true;
+    }
+};
+
+// One pipeline stage: up to two consecutive 128-wide K blocks of one segment.
+struct Stage {
+    int32_t n_tile, m_tile;
+    int32_t kb;   // first K block (global index along K)
+    int32_t nkb;  // 1 or 2
+};
+
+struct StageIter {
+    SegmentIter seg;
+    int32_t kbpg;
+    int32_t n_tile = 0, m_tile = 0;
+    int32_t kb = 0, kb_end = 0;
+    __device__ StageIter(const Params& p, int64_t b) : seg(p, b), kbpg(p.kb_per_group) {}
+    __device__ bool next(Stage& st) {
+        while (kb >= kb_end) {
+            Segment s;
+            if (!seg.next(s)) return false;
+            n_tile = s.n_tile;
+            m_tile = s.m_tile;
+            kb = s.g0 * kbpg;
+            kb_end = s.g1 * kbpg;
+        }
+        st.n_tile = n_tile;
+        st.m_tile = m_tile;
+        st.kb = kb;
+        st.nkb = (kb_end - kb) >= 2 ? 2 : 1;
+        kb += st.nkb;
         return true;
     }
 };
 
 // int4 two's-complement nibbles -> int8, 8 values per 32-bit word.  Input byte
 // j holds k = 2j (low nibble) and k = 2j+1 (high nibble); output words hold
-// k = 0..3 and k = 4..7 in byte order.  Per byte: ((v ^ 8) + 0x78) ^ 0x80
-// maps nibble v to its sign-extended byte without carries between bytes.
+// k = 0..3 and k = 4..7 in byte order.
+// Exact: per byte ((v ^ 8) + 0x78) ^ 0x80 maps nibble v to its sign-extended
+// byte without carries between bytes.
 __device__ __forceinline__ uint2 unpack_int4x8(uint32_t w) {
     uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
     uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
     lo = (lo + 0x78787878u) ^ 0x80808080u;
     hi = (hi + 0x78787878u) ^ 0x80808080u;
     return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+}
+
+// Scaled: each nibble lands in the high half of its byte, which read as int8
+// is 16 * q exactly.
+__device__ __forceinline__ uint2 unpack_int4x8_x16(uint32_t w) {
+    const uint32_t lo = (w << 4) & 0xF0F0F0F0u;
+    const uint32_t hi = w & 0xF0F0F0F0u;
+    return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+}
+
+template <bool X16>
+__device__ __forceinline__ uint2 unpack8(uint32_t w) {
+    if constexpr (X16)
+        return unpack_int4x8_x16(w);
+    else
+        return unpack_int4x8(w);
 }
 
 __device__ __forceinline__ void epi_bar_sync() {
@@ -152,22 +244,38 @@ __device__ __forceinline__ void store_output(const Params& p, int64_t m, int64_t
         static_cast<float*>(p.y)[idx] = vf;
 }
 
+struct Ring {
+    int idx = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void advance(int n) {
+        if (++idx == n) {
+            idx = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
 template <int BT, int PATH>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                      const Params p) {
-    using C = Cfg<BT>;
-    constexpr int S = C::kStages;
+    using C = Cfg<BT, PATH>;
+    constexpr int kAcc = C::kAcc;
+    constexpr int kU = C::kUnpackWarps;
+    constexpr int SW = C::kSW, SX = C::kSX, SA = C::kSA;
     constexpr int HC = BT / 2;  // columns per epilogue thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::offBar);
-    uint64_t* full = bars;
-    uint64_t* wready = bars + S;
-    uint64_t* empty = bars + 2 * S;
-    uint64_t* tfull = bars + 3 * S;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* mma_done = tempty + 2;
+    uint64_t* full_w = bars;              // W box landed (TMA transaction count)
+    uint64_t* empty_w = full_w + SW;      // unpack warps have read the W box
+    uint64_t* full_x = empty_w + SW;      // token codes landed
+    uint64_t* empty_x = full_x + SX;      // MMAs have read the token codes
+    uint64_t* full_a = empty_x + SX;      // unpacked operand written
+    uint64_t* empty_a = full_a + SA;      // MMAs have read the unpacked operand
+    uint64_t* tfull = empty_a + SA;       // P_g complete in a TMEM buffer
+    uint64_t* tempty = tfull + kAcc;      // epilogue has read a TMEM buffer
+    uint64_t* mma_done = tempty + kAcc;
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::offMisc);  // [0] tmem base [1] abort [2] last
     volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
@@ -175,14 +283,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&wready[s], kUnpackWarps);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < SW; ++s) {
+            mbar_init(&full_w[s], 1);
+            mbar_init(&empty_w[s], kU);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], kEpiWarps);
+        for (int s = 0; s < SX; ++s) {
+            mbar_init(&full_x[s], 1);
+            mbar_init(&empty_x[s], 1);
+        }
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(&full_a[s], kU);
+            mbar_init(&empty_a[s], 1);
+        }
+        for (int s = 0; s < kAcc; ++s) {
+            mbar_init(&tfull[s], 1);
+            mbar_init(&tempty[s], kEpiWarps);
         }
         mbar_init(mma_done, 1);
         misc[1] = 0;
@@ -200,139 +315,170 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int issued_parity[S];
-            for (int s = 0; s < S; ++s) issued_parity[s] = -1;
-            SegmentIter it(p, b);
-            Segment sg;
-            bool ok = true;
-            while (ok && it.next(sg)) {
-                const int32_t n0 = int32_t((sg.tile / p.m_tiles) * kTileN);
-                const int32_t m0 = int32_t((sg.tile % p.m_tiles) * BT);
-                for (int g = sg.g0; ok && g < sg.g1; ++g) {
-                    for (int kb = 0; kb < p.kb_per_group; ++kb) {
-                        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) {
-                            ok = false;
-                            break;
-                        }
-                        const int32_t kblk = g * p.kb_per_group + kb;
-                        mbar_arrive_expect_tx(&full[stage], C::kWp + C::kB);
-                        tma_load_2d(smem + C::offWp + stage * C::kWp, &tm_w, kblk * (kBlockK / 2), n0, &full[stage]);
-                        tma_load_2d(smem + C::offB + stage * C::kB, &tm_x, kblk * kBlockK, m0, &full[stage]);
-                        issued_parity[stage] = int(phase);
-                        if (++stage == S) {
-                            stage = 0;
-                            phase ^= 1u;
-                        }
-                    }
-                }
+        // The whole warp walks the loop (so it never diverges around the block
+        // barriers); lane 0 issues the copies.
+        const bool leader = (lane == 0);
+        Ring rw, rx;
+        uint32_t w_issued = 0u, w_par = 0u, x_issued = 0u, x_par = 0u;  // per slot: copy issued / its parity
+        StageIter it(p, b);
+        Stage st;
+        bool ok = true;
+        while (ok && it.next(st)) {
+            const int32_t n0 = st.n_tile * kTileN;
+            const int32_t m0 = st.m_tile * BT;
+            if (!mbar_wait_warp(&empty_w[rw.idx], rw.phase ^ 1u, abort_flag, p.status)) {
+                ok = false;
+                break;
             }
-            if (!ok) {  // let copies in flight land before the CTA leaves
-                for (int s = 0; s < S; ++s)
-                    if (issued_parity[s] >= 0) drain_wait(&full[s], uint32_t(issued_parity[s]));
+            if (leader) {
+                // one 128 x 128 B box = two K blocks (a lone last block over-reads 64 B per row: harmless)
+                mbar_arrive_expect_tx(&full_w[rw.idx], C::kWBytes);
+                tma_load_2d(smem + C::offW + rw.idx * C::kWBytes, &tm_w, st.kb * (kBlockK / 2), n0,
+                            &full_w[rw.idx]);
             }
+            w_issued |= 1u << rw.idx;
+            w_par = (w_par & ~(1u << rw.idx)) | (rw.phase << rw.idx);
+            rw.advance(SW);
+            if (!mbar_wait_warp(&empty_x[rx.idx], rx.phase ^ 1u, abort_flag, p.status)) {
+                ok = false;
+                break;
+            }
+            if (leader) {
+                mbar_arrive_expect_tx(&full_x[rx.idx], uint32_t(st.nkb * BT * kBlockK));
+                for (int j = 0; j < st.nkb; ++j)
+                    tma_load_2d(smem + C::offX + rx.idx * C::kXBytes + j * BT * kBlockK, &tm_x,
+                                (st.kb + j) * kBlockK, m0, &full_x[rx.idx]);
+            }
+            x_issued |= 1u << rx.idx;
+            x_par = (x_par & ~(1u << rx.idx)) | (rx.phase << rx.idx);
+            rx.advance(SX);
         }
+        if (!ok && leader) {  // let copies in flight land before the CTA leaves
+            for (int s = 0; s < SW; ++s)
+                if (w_issued & (1u << s)) drain_wait(&full_w[s], (w_par >> s) & 1u);
+            for (int s = 0; s < SX; ++s)
+                if (x_issued & (1u << s)) drain_wait(&full_x[s], (x_par >> s) & 1u);
+        }
+        __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_i8(kTileN, BT);
-            int stage = 0;
-            uint32_t phase = 0;
-            int ab = 0;
-            uint32_t aphase = 0;
-            SegmentIter it(p, b);
-            Segment sg;
-            bool ok = true;
-            while (ok && it.next(sg)) {
-                for (int g = sg.g0; ok && g < sg.g1; ++g) {
-                    if (!mbar_wait(&tempty[ab], aphase ^ 1u, abort_flag, p.status)) {
+        // The whole warp walks the loop; lane 0 issues the MMAs and the commits
+        // (a commit tracks the MMAs of the thread that issues it).
+        const bool leader = (lane == 0);
+        constexpr uint32_t idesc = idesc_i8(kTileN, BT);
+        Ring rx, ra, rt;
+        StageIter it(p, b);
+        Stage st;
+        bool ok = true;
+        int32_t kin = 0;  // position of the next K block inside its group (segments start on group boundaries)
+        while (ok && it.next(st)) {
+            if (!mbar_wait_warp(&full_a[ra.idx], ra.phase, abort_flag, p.status) ||
+                !mbar_wait_warp(&full_x[rx.idx], rx.phase, abort_flag, p.status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t a_base = smem_u32(smem + C::offA + ra.idx * C::kABytes);
+            const uint32_t x_base = smem_u32(smem + C::offX + rx.idx * C::kXBytes);
+            for (int j = 0; j < st.nkb; ++j) {
+                const bool first = (kin == 0);
+                const bool last = (kin == p.kb_per_group - 1);
+                kin = last ? 0 : kin + 1;
+                if (first) {
+                    if (!mbar_wait_warp(&tempty[rt.idx], rt.phase ^ 1u, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t d = tmem_base + uint32_t(ab * BT);
-                    for (int kb = 0; kb < p.kb_per_group; ++kb) {
-                        if (!mbar_wait(&wready[stage], phase, abort_flag, p.status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t a_addr = smem_u32(smem + C::offA + stage * C::kA);
-                        const uint32_t b_addr = smem_u32(smem + C::offB + stage * C::kB);
-#pragma unroll
-                        for (int k = 0; k < kBlockK / 32; ++k)
-                            mma_i8(d, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(b_addr + k * 32), idesc,
-                                   uint32_t(kb | k));
-                        mma_commit(&empty[stage]);
-                        if (++stage == S) {
-                            stage = 0;
-                            phase ^= 1u;
-                        }
-                    }
-                    if (!ok) break;
-                    mma_commit(&tfull[ab]);
-                    ab ^= 1;
-                    if (ab == 0) aphase ^= 1u;
                 }
+                if (leader) {
+                    const uint32_t d = tmem_base + uint32_t(rt.idx * BT);
+                    const uint32_t a_addr = a_base + uint32_t(j * kTileN * kBlockK);
+                    const uint32_t x_addr = x_base + uint32_t(j * BT * kBlockK);
+#pragma unroll
+                    for (int k = 0; k < kBlockK / 32; ++k)
+                        mma_i8(d, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(x_addr + k * 32), idesc,
+                               (first && k == 0) ? 0u : 1u);
+                    if (last) mma_commit(&tfull[rt.idx]);
+                }
+                if (last) rt.advance(kAcc);
+                __syncwarp();
             }
-            // every MMA this thread issued has finished before TMEM is released
+            if (!ok) break;
+            if (leader) {
+                mma_commit(&empty_a[ra.idx]);
+                mma_commit(&empty_x[rx.idx]);
+            }
+            __syncwarp();
+            ra.advance(SA);
+            rx.advance(SX);
+        }
+        // every MMA this warp issued has finished before TMEM is released
+        if (leader) {
             mma_commit(mma_done);
             drain_wait(mma_done, 0);
         }
-    } else if (warp < 2 + kUnpackWarps) {
+        __syncwarp();
+    } else if (warp < 2 + kU) {
         // ---------------------------------------------------------- int4 -> int8 unpack
+        // Thread -> (row, 16-byte packed chunk): a quarter warp covers two rows x
+        // four chunks, which with the 128-byte swizzle of both tiles keeps the
+        // shared-memory reads and writes free of bank conflicts.
         const int uw = warp - 2;
-        int stage = 0;
-        uint32_t phase = 0;
-        SegmentIter it(p, b);
-        Segment sg;
+        constexpr int kRowsPerWarp = kTileN / kU;
+        Ring rw, ra;
+        StageIter it(p, b);
+        Stage st;
         bool ok = true;
-        while (ok && it.next(sg)) {
-            const int steps = (sg.g1 - sg.g0) * p.kb_per_group;
-            for (int st = 0; st < steps; ++st) {
-                if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) {
-                    ok = false;
-                    break;
-                }
-                const uint8_t* wp = smem + C::offWp + stage * C::kWp;
-                uint8_t* a = smem + C::offA + stage * C::kA;
+        while (ok && it.next(st)) {
+            if (!mbar_wait_warp(&full_w[rw.idx], rw.phase, abort_flag, p.status) ||
+                !mbar_wait_warp(&empty_a[ra.idx], ra.phase ^ 1u, abort_flag, p.status)) {
+                ok = false;
+                break;
+            }
+            const uint8_t* wsrc = smem + C::offW + rw.idx * C::kWBytes;
+            uint8_t* adst = smem + C::offA + ra.idx * C::kABytes;
+            const int c = lane & 3;
 #pragma unroll
-                for (int itr = 0; itr < kTileN / (8 * kUnpackWarps); ++itr) {
-                    const int r = uw * (kTileN / kUnpackWarps) + itr * 8 + (lane >> 2);
-                    const int c = lane & 3;
-                    const uint4 v = *reinterpret_cast<const uint4*>(wp + r * (kBlockK / 2) + c * 16);
-                    const uint2 o0 = unpack_int4x8(v.x), o1 = unpack_int4x8(v.y);
-                    const uint2 o2 = unpack_int4x8(v.z), o3 = unpack_int4x8(v.w);
-                    uint8_t* row = a + r * kBlockK;
-                    const int sw = r & 7;
-                    *reinterpret_cast<uint4*>(row + (((2 * c) ^ sw) << 4)) = make_uint4(o0.x, o0.y, o1.x, o1.y);
-                    *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ sw) << 4)) = make_uint4(o2.x, o2.y, o3.x, o3.y);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&wready[stage]);
-                if (++stage == S) {
-                    stage = 0;
-                    phase ^= 1u;
+            for (int itr = 0; itr < kRowsPerWarp / 8; ++itr) {
+                const int r = uw * kRowsPerWarp + itr * 8 + (lane >> 2);
+                const int sw = r & 7;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    if (j < st.nkb) {
+                        const uint4 v =
+                            *reinterpret_cast<const uint4*>(wsrc + r * (kStageK / 2) + (((j * 4 + c) ^ sw) << 4));
+                        const uint2 o0 = unpack8<C::kX16>(v.x), o1 = unpack8<C::kX16>(v.y);
+                        const uint2 o2 = unpack8<C::kX16>(v.z), o3 = unpack8<C::kX16>(v.w);
+                        uint8_t* row = adst + j * (kTileN * kBlockK) + r * kBlockK;
+                        *reinterpret_cast<uint4*>(row + (((2 * c) ^ sw) << 4)) = make_uint4(o0.x, o0.y, o1.x, o1.y);
+                        *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ sw) << 4)) =
+                            make_uint4(o2.x, o2.y, o3.x, o3.y);
+                    }
                 }
             }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&full_a[ra.idx]);
+                mbar_arrive(&empty_w[rw.idx]);
+            }
+            rw.advance(SW);
+            ra.advance(SA);
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        const int ew = warp - (2 + kUnpackWarps);
+        const int ew = warp - (2 + kU);
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int half = ew >> 2;      // which half of the BT columns
         const int r = quarter * 32 + lane;
-        int ab = 0;
-        uint32_t aphase = 0;
+        Ring rt;
         SegmentIter it(p, b);
         Segment sg;
         bool ok = true;
         while (ok && it.next(sg)) {
-            const int64_t n0 = (sg.tile / p.m_tiles) * kTileN;
-            const int64_t m0 = (sg.tile % p.m_tiles) * BT + half * HC;
+            const int64_t n0 = int64_t(sg.n_tile) * kTileN;
+            const int64_t m0 = int64_t(sg.m_tile) * BT + half * HC;
             const int64_t n = n0 + r;
             const bool nvalid = n < p.N;
             int32_t acc[HC];
@@ -352,19 +498,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int g = sg.g0; g < sg.g1; ++g) {
                 const int32_t s_cur = s_next;
-                const float f_cur = f_next;
+                const float f_cur = C::kX16 ? __fmul_rn(f_next, 0.0625f) : f_next;  // P_g was computed as 16 P_g
                 if (nvalid && g + 1 < sg.g1) {
                     if (PATH == kIntScale)
                         s_next = p.S[int64_t(g + 1) * p.N + n];
                     else
                         f_next = p.s_g[int64_t(g + 1) * p.N + n];
                 }
-                if (!mbar_wait(&tfull[ab], aphase, abort_flag, p.status)) {
+                if (!mbar_wait_warp(&tfull[rt.idx], rt.phase, abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(ab * BT + half * HC);
+                const uint32_t taddr =
+                    tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(rt.idx * BT + half * HC);
                 constexpr int CH = HC < 32 ? HC : 32;
 #pragma unroll
                 for (int c0 = 0; c0 < HC; c0 += CH) {
@@ -373,17 +520,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < CH; ++j) {
-                        if (PATH == kIntScale)
-                            acc[c0 + j] += s_cur * int32_t(v[j]);
-                        else
+                        if (PATH == kIntScale) {
+                            const int32_t pg = C::kX16 ? (int32_t(v[j]) >> 4) : int32_t(v[j]);  // exact
+                            acc[c0 + j] += s_cur * pg;
+                        } else {
                             accf[c0 + j] = __fmaf_rn(f_cur, __int2float_rn(int32_t(v[j])), accf[c0 + j]);
+                        }
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[ab]);
-                ab ^= 1;
-                if (ab == 0) aphase ^= 1u;
+                if (lane == 0) mbar_arrive(&tempty[rt.idx]);
+                rt.advance(kAcc);
             }
             if (!ok) break;
 
@@ -414,7 +562,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int64_t b_first = range_owner(t0, p.W, p.grid);
             const int64_t b_last = range_owner(t0 + p.G - 1, p.W, p.grid);
             if (ew == 0 && lane == 0) {
-                const int old = atomicAdd(&p.ws_count[sg.tile], 1);
+                // one counter per CTA: a CTA is the first contributor of at most one split tile
+                const int old = atomicAdd(&p.ws_count[b_first], 1);
                 misc[2] = (old == int(b_last - b_first)) ? 1u : 0u;
             }
             epi_bar_sync();
@@ -442,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < HC; ++j)
                         if (m0 + j < p.M) store_output<PATH>(p, m0 + j, n, accf[j], acc[j]);
                 }
-                if (ew == 0 && lane == 0) p.ws_count[sg.tile] = 0;
+                if (ew == 0 && lane == 0) p.ws_count[b_first] = 0;
             }
             epi_bar_sync();
         }
@@ -474,19 +623,33 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms) {
     pl.tiles = pl.n_tiles * pl.m_tiles;
     pl.W = pl.tiles * pl.G;
     pl.grid = pl.W < num_sms ? pl.W : num_sms;
+    if (pl.grid > kMaxGrid) pl.grid = kMaxGrid;
     const int64_t slot_bytes = int64_t(kTileN) * pl.BT * 4;
-    pl.count_bytes = ((pl.tiles * 4 + 255) / 256) * 256;
+    pl.count_bytes = kCounterBytes;
     pl.ws_bytes = pl.count_bytes + pl.grid * 2 * slot_bytes;
     return pl;
 }
 
 template <int BT, int PATH>
 static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, cudaStream_t stream) {
+    using C = Cfg<BT, PATH>;
     auto kern = w4a8_gemm_kernel<BT, PATH>;
-    const int smem = Cfg<BT>::kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = C::kSmemBytes;
+    // the shared-memory opt-in is a per-device function attribute: set it once
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    kern<<<dim3(unsigned(p.grid)), dim3(kThreads), smem, stream>>>(tw, tx, p);
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        int resident = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, C::kThreads, smem);
+        if (e != cudaSuccess) return e;
+        if (resident < 1) return cudaErrorLaunchOutOfResources;
+        if (dev >= 0 && dev < 64) configured[dev] = true;
+    }
+    kern<<<dim3(unsigned(p.grid)), dim3(C::kThreads), smem, stream>>>(tw, tx, p);
     return cudaGetLastError();
 }
 
@@ -509,6 +672,8 @@ cudaError_t launch(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p
 }
 
 int token_tile_rows() { return kTileN; }
+
+int weight_box_bytes() { return kStageK / 2; }
 
 }  // namespace gemm
 }  // namespace w4a8

@@ -18,7 +18,7 @@ struct Params {
     const float* s_g;    // [G, N] float group scales (float-scale path)
     void* y;             // [M, N] output
     int32_t* ws_part;    // [grid][2][128 * BT] partial sums of split tiles
-    int32_t* ws_count;   // [tiles] arrival counters, zero between calls
+    int32_t* ws_count;   // [grid] arrival counters (index: first contributing CTA), zero between calls
     int* status;         // device status word for timeouts
     int64_t M, N;
     int64_t G;           // groups along K
@@ -33,7 +33,7 @@ struct Params {
 struct Plan {
     int BT;              // tokens per tile (MMA N)
     int64_t n_tiles, m_tiles, tiles, G, W, grid;
-    int64_t count_bytes;  // bytes of per-tile counters at the start of the workspace
+    int64_t count_bytes;  // bytes of the fixed counter region at the start of the workspace
     int64_t ws_bytes;     // total workspace bytes
 };
 
@@ -43,6 +43,9 @@ cudaError_t launch(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const Param
                    cudaStream_t stream);
 
 int token_tile_rows();
+
+// Bytes per row of one packed-weight TMA box (one pipeline stage of K).
+int weight_box_bytes();
 
 }  // namespace gemm
 }  // namespace w4a8

@@ -15,6 +15,8 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
+#include <vector>
 
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -189,20 +191,54 @@ __global__ void __launch_bounds__(kThreads) quant_rows_direct(const T* __restric
     }
 }
 
+constexpr size_t kMaxStagedSmem = 200 * 1024;
+
+// Resident CTAs per SM of the staged kernel for a given shared-memory size,
+// with the shared-memory opt-in set once per device and kernel; cached.
+template <typename K>
+static cudaError_t staged_blocks_per_sm(K kern, size_t smem, int* per_sm) {
+    struct Entry {
+        int dev;
+        size_t smem;
+        int blocks;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> cache;
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& c : cache)
+        if (c.dev == dev && c.smem == smem) {
+            *per_sm = c.blocks;
+            return cudaSuccess;
+        }
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kMaxStagedSmem + 1024));
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev] = true;
+    }
+    int blocks = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (blocks < 1) blocks = 1;
+    if (cache.size() < 256) cache.push_back({dev, smem, blocks});
+    *per_sm = blocks;
+    return cudaSuccess;
+}
+
 template <typename T>
 static cudaError_t launch_t(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a, int* status,
                             cudaStream_t stream, int num_sms) {
     const uint32_t row_bytes = uint32_t(K * sizeof(T));
     const uint32_t buf_bytes = (row_bytes + 127u) & ~127u;
     const size_t smem = 2 * size_t(buf_bytes) + 2 * sizeof(uint64_t) + kWarps * sizeof(float) + 16;
-    if (smem <= 200 * 1024) {
+    if (smem <= kMaxStagedSmem) {
         auto kern = quant_rows_staged<T>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-        if (e != cudaSuccess) return e;
         int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+        cudaError_t e = staged_blocks_per_sm(kern, smem, &per_sm);
         if (e != cudaSuccess) return e;
-        if (per_sm < 1) per_sm = 1;
         const int64_t grid = M < int64_t(num_sms) * per_sm ? M : int64_t(num_sms) * per_sm;
         kern<<<unsigned(grid), kThreads, smem, stream>>>(x, M, K, ldx, q, s_a, status);
         return cudaGetLastError();

@@ -52,6 +52,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the warp sleeps until the phase
+// completes or about `hint_ns` pass, instead of spinning on the barrier.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete, for at most about
 // one second.  On a timeout: record it in the device status word `status`,
 // set the CTA-wide abort flag and return false.  Every role checks the flag
@@ -60,18 +74,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           int* status) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    uint32_t spins = 0;
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((++spins & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > 1000000000ull) {
-                *abort_flag = 1;
-                atomicExch(status, kStatusTimeout);
-                return false;
-            }
+        if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > 1000000000ull) {
+            *abort_flag = 1;
+            atomicExch(status, kStatusTimeout);
+            return false;
         }
     }
+}
+
+// Warp-wide form: every lane waits, and the result is made uniform across the
+// warp so that a timeout never splits a warp between loop iterations.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               int* status) {
+    const bool r = mbar_wait(bar, parity, abort_flag, status);
+    return __all_sync(0xffffffffu, r) != 0;
 }
 
 // ---------------------------------------------------------------- async proxy

@@ -134,10 +134,12 @@ W4A8_API w4a8_status pack_w4_groupwise(const float* w, int64_t K, int64_t N, int
 /*
  * Bytes of workspace the GEMMs below need for (M, N, K, group) on the current
  * device (0 when they need none).  path: 0 integer scale, 1 float scale.
- * The workspace must be zero-filled before its first use; the GEMMs leave it
- * zero-filled again on success, so one allocation serves any number of calls
- * that run one after another (calls that overlap on the GPU need one each).
- * After an error or a timeout, zero it again.
+ * The workspace must be zero-filled before its first use.  Its first 4096
+ * bytes hold arrival counters that every successful call leaves at zero
+ * again (the rest is scratch), so one allocation of the largest size needed
+ * serves any sequence of calls that run one after another; calls that
+ * overlap on the GPU need one workspace each.  After an error or a timeout,
+ * zero it again.
  */
 W4A8_API int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group, int32_t path);
 
@@ -174,6 +176,14 @@ W4A8_API w4a8_status w4a8_gemm_floatscale(const int8_t* q_x, const float* s_a, c
                                  const float* s_g, int64_t M, int64_t N, int64_t K, int32_t group,
                                  void* y, int32_t y_dtype, void* workspace, int64_t workspace_bytes,
                                  void* stream);
+
+/*
+ * The CUDA runtime error code (cudaError_t) behind the last W4A8_ERR_CUDA that
+ * a call of this library returned on the calling thread (0 if none); with
+ * clear != 0 the record is reset.  w4a8_cuda_error_string names a code.
+ */
+W4A8_API int32_t w4a8_last_cuda_error(int32_t clear);
+W4A8_API const char* w4a8_cuda_error_string(int32_t code);
 
 /*
  * Reads (and with clear != 0 resets) the device status word of the current
