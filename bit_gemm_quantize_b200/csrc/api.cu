@@ -79,18 +79,22 @@ EncodeTiledFn encode_tiled() {
     return fn;
 }
 
-// 2-D uint8 tensor map: [rows][cols] bytes with row pitch `pitch`.
-bool make_map_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch, uint32_t box_cols,
-                 uint32_t box_rows, CUtensorMapSwizzle swz) {
+// 2-D tensor map: [rows][cols] elements of `type` with row pitch `pitch` bytes.
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType type, const void* base, uint64_t cols, uint64_t rows,
+                 uint64_t pitch, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return false;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {pitch};
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return enc(m, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch, uint32_t box_cols,
+                 uint32_t box_rows, CUtensorMapSwizzle swz) {
+    return make_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, cols, rows, pitch, box_cols, box_rows, swz);
 }
 
 // Whether the stream-K partition of `pl` cuts any tile (then a workspace is needed).
@@ -136,13 +140,19 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
         ws_part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + pl.count_bytes);
     }
 
-    CUtensorMap tm_w, tm_x;
+    CUtensorMap tm_w, tm_x, tm_s;
     // packed weights: one box = 128 columns x 128 bytes (two 128-wide K blocks), 128-byte swizzle
     if (!make_map_u8(&tm_w, w_packed, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2),
                      uint32_t(w4a8::gemm::weight_box_bytes()), 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return W4A8_ERR_CUDA;
     if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(M), uint64_t(K), 128, uint32_t(pl.BT),
                      CU_TENSOR_MAP_SWIZZLE_128B))
+        return W4A8_ERR_CUDA;
+    // group scales [G][N]: one box = 128 columns x 2 groups (rows past G read as zero)
+    const bool is = (path == w4a8::gemm::kIntScale);
+    if (!make_map_2d(&tm_s, is ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                     is ? static_cast<const void*>(S) : static_cast<const void*>(s_g), uint64_t(N), uint64_t(pl.G),
+                     uint64_t(N) * (is ? 2u : 4u), 128, 2, CU_TENSOR_MAP_SWIZZLE_NONE))
         return W4A8_ERR_CUDA;
 
     w4a8::gemm::Params p{};
@@ -163,7 +173,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     p.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
     p.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
                                     : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
-    W4A8_CUDA_TRY(w4a8::gemm::launch(tm_w, tm_x, p, pl.BT, path, static_cast<cudaStream_t>(stream)));
+    W4A8_CUDA_TRY(w4a8::gemm::launch(tm_w, tm_x, tm_s, p, pl.BT, path, static_cast<cudaStream_t>(stream)));
     return W4A8_OK;
 }
 

@@ -49,7 +49,6 @@ namespace gemm {
 constexpr int kTileN = 128;   // weight columns per tile (MMA M)
 constexpr int kBlockK = 128;  // K per MMA block (one 128-byte swizzle row of int8)
 constexpr int kStageK = 256;  // K per pipeline stage (one 128-byte row of packed int4)
-constexpr int kEpiWarps = 8;
 constexpr int64_t kCounterBytes = 4096;  // one int32 arrival counter per CTA, fixed region
 constexpr int64_t kMaxGrid = kCounterBytes / 4;
 
@@ -57,8 +56,15 @@ template <int BT, int PATH>
 struct Cfg {
     // int4 -> int8 unpack warps: more of them for small token tiles, where the
     // unpack is on the HBM critical path and the epilogue needs few registers.
-    static constexpr int kUnpackWarps = BT <= 32 ? 8 : 4;
-    static constexpr int kThreads = 32 * (2 + kUnpackWarps + kEpiWarps);
+    static constexpr int kUnpackWarps = 4;
+    // epilogue warps: one warpgroup covers the 128 TMEM lanes; a second one
+    // splits the columns of wide token tiles
+    static constexpr int kEpiWarps = BT <= 32 ? 4 : 8;
+    // warp roles: 0 TMA producer, 1-2 MMA issuers, then unpack, then epilogue
+    static constexpr int kMmaWarps = 2;
+    static constexpr int kFirstUnpackWarp = 1 + kMmaWarps;
+    static constexpr int kFirstEpiWarp = kFirstUnpackWarp + kUnpackWarps;
+    static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
     // TMEM accumulator buffers: the MMA may run kAcc - 1 groups ahead of the
     // per-group drain, so the drain's latency is hidden.
     static constexpr int kAcc = BT == 128 ? 4 : 8;
@@ -70,14 +76,22 @@ struct Cfg {
     static constexpr int kWBytes = kTileN * kStageK / 2;  // packed weights per stage: 16 KB
     static constexpr int kXBytes = BT * kStageK;          // token codes per stage
     static constexpr int kABytes = kTileN * kStageK;      // unpacked weights per stage: 32 KB
-    static constexpr int kSA = 2;
-    static constexpr int kSW = BT <= 32 ? 7 : (BT == 64 ? 6 : 3);
-    static constexpr int kSX = BT == 16 ? 8 : (BT == 32 ? 4 : 3);
+    static constexpr int kSA = BT <= 32 ? 3 : 2;
+    static constexpr int kSW = BT <= 32 ? 5 : (BT == 64 ? 6 : 3);
+    static constexpr int kSX = BT <= 32 ? 4 : 3;
+    // stage-done ring: one tcgen05.commit per stage (a commit costs about as
+    // much issue time as two small MMAs), read by every role that recycles a
+    // resource of that stage; the group scales of a stage travel in a slot of
+    // this ring too (TMA box: 2 groups x 128 columns)
+    static constexpr int kSD = 16;
+    static_assert(kSD >= kSX && kSD >= kSA, "stage-done ring shallower than a ring it releases");
+    static constexpr int kSBytes = 2 * kTileN * (PATH == kIntScale ? 2 : 4);
     static constexpr int offW = 0;
     static constexpr int offX = offW + kSW * kWBytes;
     static constexpr int offA = offX + kSX * kXBytes;
-    static constexpr int offBar = offA + kSA * kABytes;
-    static constexpr int kBars = 2 * kSW + 2 * kSX + 2 * kSA + 2 * kAcc + 1;
+    static constexpr int offS = offA + kSA * kABytes;
+    static constexpr int offBar = offS + kSD * kSBytes;
+    static constexpr int kBars = 2 * kSW + kSX + kSA + 3 * kSD + kAcc + kMmaWarps;
     static constexpr int offMisc = offBar + kBars * 8;
     static constexpr int kSmemBytes = offMisc + 64 + 1024;  // + slack to align the base to 1024
     static constexpr uint32_t kTmemCols = (kAcc * BT) < 32 ? 32u : uint32_t(kAcc * BT);
@@ -146,6 +160,7 @@ struct Stage {
     int32_t n_tile, m_tile;
     int32_t kb;   // first K block (global index along K)
     int32_t nkb;  // 1 or 2
+    int32_t g;    // group of the first K block; the groups that end in the stage are g and g + 1
 };
 
 struct StageIter {
@@ -153,6 +168,7 @@ struct StageIter {
     int32_t kbpg;
     int32_t n_tile = 0, m_tile = 0;
     int32_t kb = 0, kb_end = 0;
+    int32_t g = 0, kin = 0;  // group of the next K block and its position in the group
     __device__ StageIter(const Params& p, int64_t b) : seg(p, b), kbpg(p.kb_per_group) {}
     __device__ bool next(Stage& st) {
         while (kb >= kb_end) {
@@ -162,12 +178,21 @@ struct StageIter {
             m_tile = s.m_tile;
             kb = s.g0 * kbpg;
             kb_end = s.g1 * kbpg;
+            g = s.g0;
+            kin = 0;
         }
         st.n_tile = n_tile;
         st.m_tile = m_tile;
         st.kb = kb;
         st.nkb = (kb_end - kb) >= 2 ? 2 : 1;
+        st.g = g;
         kb += st.nkb;
+        for (int j = 0; j < st.nkb; ++j) {
+            if (++kin == kbpg) {
+                kin = 0;
+                ++g;
+            }
+        }
         return true;
     }
 };
@@ -201,8 +226,8 @@ __device__ __forceinline__ uint2 unpack8(uint32_t w) {
         return unpack_int4x8(w);
 }
 
-__device__ __forceinline__ void epi_bar_sync() {
-    asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32) : "memory");
+__device__ __forceinline__ void epi_bar_sync(int threads) {
+    asm volatile("bar.sync 1, %0;" ::"r"(threads) : "memory");
 }
 
 template <int N>
@@ -219,9 +244,9 @@ __device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t (&r)[N]) {
 
 // Bounded wait without the abort short-cut, for draining copies in flight.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    const uint64_t t0 = globaltimer_ns();
+    const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > 1000000000ull) break;
+        if (clock64() - t0 > kWaitLimitCycles) break;
     }
 }
 
@@ -258,23 +283,24 @@ struct Ring {
 template <int BT, int PATH>
 __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-                     const Params p) {
+                     const __grid_constant__ CUtensorMap tm_s, const Params p) {
     using C = Cfg<BT, PATH>;
     constexpr int kAcc = C::kAcc;
     constexpr int kU = C::kUnpackWarps;
-    constexpr int SW = C::kSW, SX = C::kSX, SA = C::kSA;
-    constexpr int HC = BT / 2;  // columns per epilogue thread
+    constexpr int SW = C::kSW, SX = C::kSX, SA = C::kSA, SD = C::kSD;
+    constexpr int kEpiWarps = C::kEpiWarps;
+    constexpr int HC = BT / (kEpiWarps / 4);  // columns per epilogue thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::offBar);
     uint64_t* full_w = bars;              // W box landed (TMA transaction count)
     uint64_t* empty_w = full_w + SW;      // unpack warps have read the W box
     uint64_t* full_x = empty_w + SW;      // token codes landed
-    uint64_t* empty_x = full_x + SX;      // MMAs have read the token codes
-    uint64_t* full_a = empty_x + SX;      // unpacked operand written
-    uint64_t* empty_a = full_a + SA;      // MMAs have read the unpacked operand
-    uint64_t* tfull = empty_a + SA;       // P_g complete in a TMEM buffer
-    uint64_t* tempty = tfull + kAcc;      // epilogue has read a TMEM buffer
+    uint64_t* full_a = full_x + SX;       // unpacked operand written
+    uint64_t* sdone = full_a + SA;        // all MMAs of a stage complete (one commit per stage)
+    uint64_t* sfree = sdone + SD;         // epilogue has seen a stage-done phase (slot may be committed again)
+    uint64_t* full_s = sfree + SD;        // a stage's group scales landed
+    uint64_t* tempty = full_s + SD;       // epilogue has read a TMEM accumulator buffer
     uint64_t* mma_done = tempty + kAcc;
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::offMisc);  // [0] tmem base [1] abort [2] last
     volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
@@ -287,24 +313,21 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
             mbar_init(&full_w[s], 1);
             mbar_init(&empty_w[s], kU);
         }
-        for (int s = 0; s < SX; ++s) {
-            mbar_init(&full_x[s], 1);
-            mbar_init(&empty_x[s], 1);
+        for (int s = 0; s < SX; ++s) mbar_init(&full_x[s], 1);
+        for (int s = 0; s < SA; ++s) mbar_init(&full_a[s], kU);
+        for (int s = 0; s < SD; ++s) {
+            mbar_init(&sdone[s], 1);
+            mbar_init(&sfree[s], kEpiWarps);
+            mbar_init(&full_s[s], 1);
         }
-        for (int s = 0; s < SA; ++s) {
-            mbar_init(&full_a[s], kU);
-            mbar_init(&empty_a[s], 1);
-        }
-        for (int s = 0; s < kAcc; ++s) {
-            mbar_init(&tfull[s], 1);
-            mbar_init(&tempty[s], kEpiWarps);
-        }
-        mbar_init(mma_done, 1);
+        for (int s = 0; s < kAcc; ++s) mbar_init(&tempty[s], kEpiWarps);
+        for (int s = 0; s < C::kMmaWarps; ++s) mbar_init(&mma_done[s], 1);
         misc[1] = 0;
         misc[2] = 0;
         fence_mbar_init();
         prefetch_tensormap(&tm_w);
         prefetch_tensormap(&tm_x);
+        prefetch_tensormap(&tm_s);
     }
     if (warp == 1) tmem_alloc(&misc[0], C::kTmemCols);
     tc_fence_before();
@@ -319,7 +342,11 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
         // barriers); lane 0 issues the copies.
         const bool leader = (lane == 0);
         Ring rw, rx;
+        Ring rxd;          // stage-done slot of the stage whose token slot is reused (SX stages back)
+        Ring rs;           // scale slot (same index as the stage-done ring)
+        int32_t pst = 0;   // stages issued so far
         uint32_t w_issued = 0u, w_par = 0u, x_issued = 0u, x_par = 0u;  // per slot: copy issued / its parity
+        uint32_t s_issued = 0u, s_par = 0u;
         StageIter it(p, b);
         Stage st;
         bool ok = true;
@@ -339,9 +366,12 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
             w_issued |= 1u << rw.idx;
             w_par = (w_par & ~(1u << rw.idx)) | (rw.phase << rw.idx);
             rw.advance(SW);
-            if (!mbar_wait_warp(&empty_x[rx.idx], rx.phase ^ 1u, abort_flag, p.status)) {
-                ok = false;
-                break;
+            if (pst >= SX) {  // the MMAs of stage pst - SX have read this token slot
+                if (!mbar_wait_warp(&sdone[rxd.idx], rxd.phase, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                rxd.advance(SD);
             }
             if (leader) {
                 mbar_arrive_expect_tx(&full_x[rx.idx], uint32_t(st.nkb * BT * kBlockK));
@@ -352,90 +382,143 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
             x_issued |= 1u << rx.idx;
             x_par = (x_par & ~(1u << rx.idx)) | (rx.phase << rx.idx);
             rx.advance(SX);
+            // the stage's group scales (rows g, g+1; rows past the last group read as zero)
+            if (!mbar_wait_warp(&sfree[rs.idx], rs.phase ^ 1u, abort_flag, p.status)) {
+                ok = false;
+                break;
+            }
+            if (leader) {
+                mbar_arrive_expect_tx(&full_s[rs.idx], C::kSBytes);
+                tma_load_2d(smem + C::offS + rs.idx * C::kSBytes, &tm_s, n0, st.g, &full_s[rs.idx]);
+            }
+            s_issued |= 1u << rs.idx;
+            s_par = (s_par & ~(1u << rs.idx)) | (rs.phase << rs.idx);
+            rs.advance(SD);
+            ++pst;
         }
         if (!ok && leader) {  // let copies in flight land before the CTA leaves
             for (int s = 0; s < SW; ++s)
                 if (w_issued & (1u << s)) drain_wait(&full_w[s], (w_par >> s) & 1u);
             for (int s = 0; s < SX; ++s)
                 if (x_issued & (1u << s)) drain_wait(&full_x[s], (x_par >> s) & 1u);
+            for (int s = 0; s < SD; ++s)
+                if (s_issued & (1u << s)) drain_wait(&full_s[s], (s_par >> s) & 1u);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ---------------------------------------------------------- MMA issuer
-        // The whole warp walks the loop; lane 0 issues the MMAs and the commits
-        // (a commit tracks the MMAs of the thread that issues it).
+    } else if (warp < C::kFirstUnpackWarp) {
+        // ---------------------------------------------------------- MMA issuers
+        // The issue of one tcgen05.mma, a barrier poll or a commit occupies the
+        // issuing thread for tens to hundreds of cycles, and one thread's issues
+        // do not overlap, while the tensor core accepts small MMAs about twice
+        // as fast as one thread issues them.  So two warps issue alternate
+        // stages.  When a group spans more than two K blocks, consecutive stages
+        // accumulate into one TMEM buffer and must stay in one warp's order, so
+        // the first warp then issues every stage.
+        // Each warp walks every stage (so the ring, buffer and group
+        // bookkeeping stays identical in both) and issues its own; lane 0 issues
+        // the MMAs and the commit (a commit tracks the MMAs of its thread).
+        // One commit per stage, to the stage-done ring; before a stage-done slot
+        // is committed again the epilogue must have seen its previous phase.
+        const int mw = warp - 1;
+        const int nmma = (p.kb_per_group <= 2) ? C::kMmaWarps : 1;
         const bool leader = (lane == 0);
         constexpr uint32_t idesc = idesc_i8(kTileN, BT);
-        Ring rx, ra, rt;
-        StageIter it(p, b);
-        Stage st;
-        bool ok = true;
-        int32_t kin = 0;  // position of the next K block inside its group (segments start on group boundaries)
-        while (ok && it.next(st)) {
-            if (!mbar_wait_warp(&full_a[ra.idx], ra.phase, abort_flag, p.status) ||
-                !mbar_wait_warp(&full_x[rx.idx], rx.phase, abort_flag, p.status)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t a_base = smem_u32(smem + C::offA + ra.idx * C::kABytes);
-            const uint32_t x_base = smem_u32(smem + C::offX + rx.idx * C::kXBytes);
-            for (int j = 0; j < st.nkb; ++j) {
-                const bool first = (kin == 0);
-                const bool last = (kin == p.kb_per_group - 1);
-                kin = last ? 0 : kin + 1;
-                if (first) {
-                    if (!mbar_wait_warp(&tempty[rt.idx], rt.phase ^ 1u, abort_flag, p.status)) {
+        if (mw < nmma) {
+            Ring rx, ra, rt, rd;
+            StageIter it(p, b);
+            Stage st;
+            bool ok = true;
+            int32_t si = 0;   // stage index within this CTA
+            int32_t kin = 0;  // position of the next K block inside its group (segments start on group boundaries)
+            // descriptor low words of slot 0; slots and K steps are plain offsets from here
+            const uint32_t a_lo0 = smem_desc_sw128_lo(smem_u32(smem + C::offA));
+            const uint32_t x_lo0 = smem_desc_sw128_lo(smem_u32(smem + C::offX));
+            while (ok && it.next(st)) {
+                if ((si % nmma) != mw) {  // another warp's stage: only keep the bookkeeping in step
+                    for (int j = 0; j < st.nkb; ++j) {
+                        const bool last = (kin == p.kb_per_group - 1);
+                        kin = last ? 0 : kin + 1;
+                        if (last) rt.advance(kAcc);
+                    }
+                } else {
+                    if (!mbar_wait_warp(&full_a[ra.idx], ra.phase, abort_flag, p.status) ||
+                        !mbar_wait_warp(&full_x[rx.idx], rx.phase, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                }
-                if (leader) {
-                    const uint32_t d = tmem_base + uint32_t(rt.idx * BT);
-                    const uint32_t a_addr = a_base + uint32_t(j * kTileN * kBlockK);
-                    const uint32_t x_addr = x_base + uint32_t(j * BT * kBlockK);
+                    const uint32_t a_lo = a_lo0 + uint32_t(ra.idx) * uint32_t(C::kABytes >> 4);
+                    const uint32_t x_lo = x_lo0 + uint32_t(rx.idx) * uint32_t(C::kXBytes >> 4);
 #pragma unroll
-                    for (int k = 0; k < kBlockK / 32; ++k)
-                        mma_i8(d, smem_desc_sw128(a_addr + k * 32), smem_desc_sw128(x_addr + k * 32), idesc,
-                               (first && k == 0) ? 0u : 1u);
-                    if (last) mma_commit(&tfull[rt.idx]);
+                    for (int j = 0; j < 2; ++j) {
+                        if (j >= st.nkb) break;
+                        const bool first = (kin == 0);
+                        const bool last = (kin == p.kb_per_group - 1);
+                        kin = last ? 0 : kin + 1;
+                        if (first) {
+                            if (!mbar_wait_warp(&tempty[rt.idx], rt.phase ^ 1u, abort_flag, p.status)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                        }
+                        if (leader) {
+                            const uint32_t d = tmem_base + uint32_t(rt.idx * BT);
+                            const uint32_t aj = a_lo + uint32_t(j * ((kTileN * kBlockK) >> 4));
+                            const uint32_t xj = x_lo + uint32_t(j * ((BT * kBlockK) >> 4));
+#pragma unroll
+                            for (int k = 0; k < kBlockK / 32; ++k)  // 32 bytes of K per MMA = 2 descriptor units
+                                mma_i8(d, smem_desc_from_lo(aj + 2u * k), smem_desc_from_lo(xj + 2u * k), idesc,
+                                       (first && k == 0) ? 0u : 1u);
+                        }
+                        if (last) rt.advance(kAcc);
+                    }
+                    if (!ok) break;
+                    if (!mbar_wait_warp(&sfree[rd.idx], rd.phase ^ 1u, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) mma_commit(&sdone[rd.idx]);
+                    __syncwarp();
                 }
-                if (last) rt.advance(kAcc);
-                __syncwarp();
+                ra.advance(SA);
+                rx.advance(SX);
+                rd.advance(SD);
+                ++si;
             }
-            if (!ok) break;
+            // every MMA this warp issued has finished before TMEM is released
             if (leader) {
-                mma_commit(&empty_a[ra.idx]);
-                mma_commit(&empty_x[rx.idx]);
+                mma_commit(&mma_done[mw]);
+                drain_wait(&mma_done[mw], 0);
             }
             __syncwarp();
-            ra.advance(SA);
-            rx.advance(SX);
         }
-        // every MMA this warp issued has finished before TMEM is released
-        if (leader) {
-            mma_commit(mma_done);
-            drain_wait(mma_done, 0);
-        }
-        __syncwarp();
-    } else if (warp < 2 + kU) {
+    } else if (warp < C::kFirstEpiWarp) {
         // ---------------------------------------------------------- int4 -> int8 unpack
         // Thread -> (row, 16-byte packed chunk): a quarter warp covers two rows x
         // four chunks, which with the 128-byte swizzle of both tiles keeps the
         // shared-memory reads and writes free of bank conflicts.
-        const int uw = warp - 2;
+        const int uw = warp - C::kFirstUnpackWarp;
         constexpr int kRowsPerWarp = kTileN / kU;
         Ring rw, ra;
+        Ring rad;          // stage-done slot of the stage whose operand slot is reused (SA stages back)
+        int32_t ust = 0;   // stages unpacked so far
         StageIter it(p, b);
         Stage st;
         bool ok = true;
         while (ok && it.next(st)) {
-            if (!mbar_wait_warp(&full_w[rw.idx], rw.phase, abort_flag, p.status) ||
-                !mbar_wait_warp(&empty_a[ra.idx], ra.phase ^ 1u, abort_flag, p.status)) {
+            if (!mbar_wait_warp(&full_w[rw.idx], rw.phase, abort_flag, p.status)) {
                 ok = false;
                 break;
             }
+            if (ust >= SA) {  // the MMAs of stage ust - SA have read this operand slot
+                if (!mbar_wait_warp(&sdone[rad.idx], rad.phase, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                rad.advance(SD);
+            }
+            ++ust;
             const uint8_t* wsrc = smem + C::offW + rw.idx * C::kWBytes;
             uint8_t* adst = smem + C::offA + ra.idx * C::kABytes;
             const int c = lane & 3;
@@ -468,11 +551,11 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        const int ew = warp - (2 + kU);
+        const int ew = warp - C::kFirstEpiWarp;
         const int quarter = warp & 3;  // TMEM lanes this warp may access
-        const int half = ew >> 2;      // which half of the BT columns
+        const int half = ew >> 2;      // which part of the BT columns
         const int r = quarter * 32 + lane;
-        Ring rt;
+        Ring rt, rd;
         SegmentIter it(p, b);
         Segment sg;
         bool ok = true;
@@ -488,50 +571,103 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 acc[j] = 0;
                 accf[j] = 0.0f;
             }
-            int32_t s_next = 0;
-            float f_next = 0.0f;
-            if (nvalid) {
-                if (PATH == kIntScale)
-                    s_next = p.S[int64_t(sg.g0) * p.N + n];
-                else
-                    f_next = p.s_g[int64_t(sg.g0) * p.N + n];
-            }
-            for (int g = sg.g0; g < sg.g1; ++g) {
-                const int32_t s_cur = s_next;
-                const float f_cur = C::kX16 ? __fmul_rn(f_next, 0.0625f) : f_next;  // P_g was computed as 16 P_g
-                if (nvalid && g + 1 < sg.g1) {
-                    if (PATH == kIntScale)
-                        s_next = p.S[int64_t(g + 1) * p.N + n];
-                    else
-                        f_next = p.s_g[int64_t(g + 1) * p.N + n];
-                }
-                if (!mbar_wait_warp(&tfull[rt.idx], rt.phase, abort_flag, p.status)) {
+            // Walk the segment's stages in the order the MMA warp commits them:
+            // wait for each stage's done phase, tell the MMA warp it was seen,
+            // then drain every group whose last K block was in that stage.
+            int32_t g = sg.g0;  // next group to drain
+            int32_t kin = 0;    // position of the next K block inside its group
+            int32_t kb = sg.g0 * p.kb_per_group;
+            const int32_t kb_end = sg.g1 * p.kb_per_group;
+            while (kb < kb_end) {
+                const int32_t nkb = (kb_end - kb) >= 2 ? 2 : 1;
+                kb += nkb;
+                if (!mbar_wait_warp(&sdone[rd.idx], rd.phase, abort_flag, p.status) ||
+                    !mbar_wait_warp(&full_s[rd.idx], rd.phase, abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t taddr =
-                    tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(rt.idx * BT + half * HC);
-                constexpr int CH = HC < 32 ? HC : 32;
+                // this column's scales of the stage's groups g and g + 1 (raw 32 bits)
+                uint32_t sc0, sc1;
+                {
+                    const uint8_t* sbuf = smem + C::offS + rd.idx * C::kSBytes;
+                    if (PATH == kIntScale) {
+                        const int16_t* s16 = reinterpret_cast<const int16_t*>(sbuf);
+                        sc0 = uint32_t(int32_t(s16[r]));
+                        sc1 = uint32_t(int32_t(s16[kTileN + r]));
+                    } else {
+                        const uint32_t* s32 = reinterpret_cast<const uint32_t*>(sbuf);
+                        sc0 = s32[r];
+                        sc1 = s32[kTileN + r];
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfree[rd.idx]);  // the scale slot may be refilled
+                rd.advance(SD);
+                // groups whose last K block is in this stage (at most two)
+                int ng = 0;
+                uint32_t gb0 = 0u, gb1 = 0u;  // their TMEM buffers
+                for (int j = 0; j < nkb; ++j) {
+                    const bool last = (kin == p.kb_per_group - 1);
+                    kin = last ? 0 : kin + 1;
+                    if (last) {
+                        if (ng == 0)
+                            gb0 = uint32_t(rt.idx);
+                        else
+                            gb1 = uint32_t(rt.idx);
+                        ++ng;
+                        rt.advance(kAcc);
+                    }
+                }
+                if (ng == 0) continue;
+                // Segments start on group boundaries and stages cover consecutive K
+                // blocks, so the groups ending in a stage are the stage's first group
+                // (row 0 of the scale box) and possibly the next one (row 1).
+                int taken = 0;
+                auto take_scale = [&]() -> uint32_t { return (taken++ == 0) ? sc0 : sc1; };
+                auto accumulate = [&](const uint32_t* v, int c0, int cnt, uint32_t sraw) {
+                    const int32_t s_cur = int32_t(sraw);
+                    const float f_cur = C::kX16 ? __fmul_rn(__uint_as_float(sraw), 0.0625f)  // P_g was 16 P_g
+                                                : __uint_as_float(sraw);
 #pragma unroll
-                for (int c0 = 0; c0 < HC; c0 += CH) {
-                    uint32_t v[CH];
-                    tmem_load<CH>(taddr + uint32_t(c0), v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < CH; ++j) {
+                    for (int q = 0; q < cnt; ++q) {
                         if (PATH == kIntScale) {
-                            const int32_t pg = C::kX16 ? (int32_t(v[j]) >> 4) : int32_t(v[j]);  // exact
-                            acc[c0 + j] += s_cur * pg;
+                            const int32_t pg = C::kX16 ? (int32_t(v[q]) >> 4) : int32_t(v[q]);  // exact
+                            acc[c0 + q] += s_cur * pg;
                         } else {
-                            accf[c0 + j] = __fmaf_rn(f_cur, __int2float_rn(int32_t(v[j])), accf[c0 + j]);
+                            accf[c0 + q] = __fmaf_rn(f_cur, __int2float_rn(int32_t(v[q])), accf[c0 + q]);
+                        }
+                    }
+                };
+                const uint32_t lane_cols = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(half * HC);
+                if constexpr (HC <= 16) {
+                    // small tiles: both groups' loads in flight before one wait
+                    uint32_t v0[HC], v1[HC];
+                    tmem_load<HC>(lane_cols + gb0 * uint32_t(BT), v0);
+                    if (ng == 2) tmem_load<HC>(lane_cols + gb1 * uint32_t(BT), v1);
+                    tmem_wait_ld();
+                    accumulate(v0, 0, HC, take_scale());
+                    if (ng == 2) accumulate(v1, 0, HC, take_scale());
+                } else {
+                    constexpr int CH = 32;
+                    for (int gi = 0; gi < ng; ++gi) {
+                        const uint32_t sraw = take_scale();
+#pragma unroll
+                        for (int c0 = 0; c0 < HC; c0 += CH) {
+                            uint32_t v[CH];
+                            tmem_load<CH>(lane_cols + (gi == 0 ? gb0 : gb1) * uint32_t(BT) + uint32_t(c0), v);
+                            tmem_wait_ld();
+                            accumulate(v, c0, CH, sraw);
                         }
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty[rt.idx]);
-                rt.advance(kAcc);
+                if (lane == 0) {
+                    mbar_arrive(&tempty[gb0]);
+                    if (ng == 2) mbar_arrive(&tempty[gb1]);
+                }
+                g += ng;
             }
             if (!ok) break;
 
@@ -557,7 +693,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                     part[e] = __float_as_int(accf[j]);
             }
             __threadfence();
-            epi_bar_sync();
+            epi_bar_sync(kEpiWarps * 32);
             const int64_t t0 = sg.tile * p.G;
             const int64_t b_first = range_owner(t0, p.W, p.grid);
             const int64_t b_last = range_owner(t0 + p.G - 1, p.W, p.grid);
@@ -566,7 +702,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 const int old = atomicAdd(&p.ws_count[b_first], 1);
                 misc[2] = (old == int(b_last - b_first)) ? 1u : 0u;
             }
-            epi_bar_sync();
+            epi_bar_sync(kEpiWarps * 32);
             if (misc[2]) {
                 __threadfence();
 #pragma unroll
@@ -593,7 +729,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 }
                 if (ew == 0 && lane == 0) p.ws_count[b_first] = 0;
             }
-            epi_bar_sync();
+            epi_bar_sync(kEpiWarps * 32);
         }
     }
 
@@ -631,7 +767,8 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms) {
 }
 
 template <int BT, int PATH>
-static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, cudaStream_t stream) {
+static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts, const Params& p,
+                             cudaStream_t stream) {
     using C = Cfg<BT, PATH>;
     auto kern = w4a8_gemm_kernel<BT, PATH>;
     const int smem = C::kSmemBytes;
@@ -649,25 +786,25 @@ static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const
         if (resident < 1) return cudaErrorLaunchOutOfResources;
         if (dev >= 0 && dev < 64) configured[dev] = true;
     }
-    kern<<<dim3(unsigned(p.grid)), dim3(C::kThreads), smem, stream>>>(tw, tx, p);
+    kern<<<dim3(unsigned(p.grid)), dim3(C::kThreads), smem, stream>>>(tw, tx, ts, p);
     return cudaGetLastError();
 }
 
-cudaError_t launch(const CUtensorMap& tw, const CUtensorMap& tx, const Params& p, int BT, int path,
+cudaError_t launch(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts, const Params& p, int BT, int path,
                    cudaStream_t stream) {
     if (path == kIntScale) {
         switch (BT) {
-            case 16: return launch_bt<16, kIntScale>(tw, tx, p, stream);
-            case 32: return launch_bt<32, kIntScale>(tw, tx, p, stream);
-            case 64: return launch_bt<64, kIntScale>(tw, tx, p, stream);
-            default: return launch_bt<128, kIntScale>(tw, tx, p, stream);
+            case 16: return launch_bt<16, kIntScale>(tw, tx, ts, p, stream);
+            case 32: return launch_bt<32, kIntScale>(tw, tx, ts, p, stream);
+            case 64: return launch_bt<64, kIntScale>(tw, tx, ts, p, stream);
+            default: return launch_bt<128, kIntScale>(tw, tx, ts, p, stream);
         }
     }
     switch (BT) {
-        case 16: return launch_bt<16, kFloatScale>(tw, tx, p, stream);
-        case 32: return launch_bt<32, kFloatScale>(tw, tx, p, stream);
-        case 64: return launch_bt<64, kFloatScale>(tw, tx, p, stream);
-        default: return launch_bt<128, kFloatScale>(tw, tx, p, stream);
+        case 16: return launch_bt<16, kFloatScale>(tw, tx, ts, p, stream);
+        case 32: return launch_bt<32, kFloatScale>(tw, tx, ts, p, stream);
+        case 64: return launch_bt<64, kFloatScale>(tw, tx, ts, p, stream);
+        default: return launch_bt<128, kFloatScale>(tw, tx, ts, p, stream);
     }
 }
 

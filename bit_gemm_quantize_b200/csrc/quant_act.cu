@@ -168,8 +168,8 @@ __global__ void __launch_bounds__(kThreads) quant_rows_staged(const T* __restric
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
             if (!inflight[b]) continue;
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&bars[b], phase[b]) && globaltimer_ns() - t0 < 1000000000ull) {
+            const long long t0 = clock64();
+            while (!mbar_try_wait(&bars[b], phase[b]) && clock64() - t0 < kWaitLimitCycles) {
             }
         }
     }

@@ -67,17 +67,20 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 }
 
 // Wait for the phase with the given parity to complete, for at most about
-// one second.  On a timeout: record it in the device status word `status`,
+// one second (2^31 SM cycles; the cycle counter is cheap to read, unlike the
+// global timer).  On a timeout: record it in the device status word `status`,
 // set the CTA-wide abort flag and return false.  Every role checks the flag
 // so that the whole CTA leaves its loops and reaches the teardown.
+constexpr long long kWaitLimitCycles = 1ll << 31;
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int* status) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
         if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > 1000000000ull) {
+        if (clock64() - t0 > kWaitLimitCycles) {
             *abort_flag = 1;
             atomicExch(status, kStatusTimeout);
             return false;
@@ -85,12 +88,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-// Warp-wide form: every lane waits, and the result is made uniform across the
-// warp so that a timeout never splits a warp between loop iterations.
+// Warp-wide form: lane 0 polls the barrier (one barrier operation per poll
+// instead of 32) and the result is broadcast, so the warp leaves together and
+// a timeout never splits it.  The shuffle is a warp-level synchronisation, so
+// the other lanes' later accesses are ordered after lane 0's acquire.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                                int* status) {
-    const bool r = mbar_wait(bar, parity, abort_flag, status);
-    return __all_sync(0xffffffffu, r) != 0;
+    int r = 1;
+    if ((threadIdx.x & 31) == 0) r = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, r, 0) != 0;
 }
 
 // ---------------------------------------------------------------- async proxy
@@ -203,6 +209,21 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
     d |= static_cast<uint64_t>(1u) << 46;                       // descriptor version for tcgen05
     d |= static_cast<uint64_t>(2u) << 61;                       // 128-byte swizzle
     return d;
+}
+
+// The same descriptor split in two 32-bit words: the low word carries the
+// start address (bits 0-13, in 16-byte units) and the leading byte offset;
+// the high word is the same for every tile of this layout.  Advancing a
+// descriptor by a byte offset inside shared memory is then one 32-bit add of
+// offset / 16 to the low word (addresses stay below 2^18, so no carry).
+constexpr uint32_t kDescSw128Hi = (1024u >> 4) | (1u << 14) | (2u << 29);
+
+__device__ __forceinline__ uint32_t smem_desc_sw128_lo(uint32_t saddr) {
+    return ((saddr >> 4) & 0x3FFFu) | (1u << 16);
+}
+
+__device__ __forceinline__ uint64_t smem_desc_from_lo(uint32_t lo) {
+    return (static_cast<uint64_t>(kDescSw128Hi) << 32) | lo;
 }
 
 // Instruction descriptor: kind::i8, signed A and B, int32 accumulator,
