@@ -13,18 +13,25 @@
 // per-thread scalar in the per-group drain.
 //
 // Data flow per pipeline stage (256 consecutive K):
-//   HBM --TMA--> packed int4 box [128 n][128 B] (128-byte swizzle)      (W ring)
-//   HBM --TMA--> token codes [BT m][128 k] x2 (128-byte swizzle)        (X ring)
-//   unpack warps: packed W -> int8 [128 n][128 k] x2, K-major, 128-byte
-//   swizzle = MMA operand A                                             (A ring)
-//   tcgen05.mma.kind::i8, K = 32 each, accumulating one group's P_g in a
-//   TMEM buffer [128 lanes][BT columns]                                 (TMEM ring)
+//   HBM --TMA--> packed int4 box [128 n][128 B] (128-byte swizzle)      (W ring, smem)
+//   HBM --TMA--> token codes [BT m][128 k] x2 (128-byte swizzle)        (X ring, smem)
+//   HBM --TMA--> group scales [2 g][128 n]                              (S ring, smem)
+//   unpack warps (one thread per weight row = TMEM lane): packed int4 ->
+//   int8, written with tcgen05.st as the MMA's A operand, 64 TMEM columns
+//   of 4 K values each                                                  (A ring, TMEM)
+//   tcgen05.mma.kind::i8, A from TMEM, B = token codes from smem, K = 32
+//   each, accumulating one group's P_g in a TMEM buffer [128][BT]       (acc ring, TMEM)
 //   epilogue warps per group: tcgen05.ld P_g, acc += S[g,n] * P_g (or
 //   accf += s_g * float(P_g)); after the last group y = acc * s_a[m] / alpha
 //   (or accf * s_a[m]).
+// Keeping the unpacked operand in TMEM instead of shared memory saves two of
+// its passes through the shared-memory port (the unpack's store and the MMA's
+// read, 64 KB per stage), which bound small-token-tile MMAs at about 40
+// cycles each; read from TMEM they take 16 (N = 16) to 64 (N = 128, the full
+// int8 rate) cycles.
 // The W ring is released by the unpack warps as soon as they have read a
-// stage (plain mbarrier arrivals), so the HBM stream only waits on the unpack;
-// the X and A rings are released by tcgen05.commit after the MMAs.
+// stage, so the HBM stream only waits on the unpack; the X ring and the A
+// ring are released by one tcgen05.commit per stage, after its MMAs.
 //
 // Work partition: the (tile, group) steps of the whole problem are split into
 // one contiguous range per CTA of a persistent grid (stream-K).  A tile whose
@@ -47,27 +54,31 @@ namespace w4a8 {
 namespace gemm {
 
 constexpr int kTileN = 128;   // weight columns per tile (MMA M)
-constexpr int kBlockK = 128;  // K per MMA block (one 128-byte swizzle row of int8)
+constexpr int kBlockK = 128;  // K per MMA block (one 128-byte swizzle row of int8 token codes)
 constexpr int kStageK = 256;  // K per pipeline stage (one 128-byte row of packed int4)
+constexpr int kStageCols = kStageK / 4;  // TMEM columns of one stage's A operand (4 int8 per column)
 constexpr int64_t kCounterBytes = 4096;  // one int32 arrival counter per CTA, fixed region
 constexpr int64_t kMaxGrid = kCounterBytes / 4;
 
 template <int BT, int PATH>
 struct Cfg {
-    // int4 -> int8 unpack warps: more of them for small token tiles, where the
-    // unpack is on the HBM critical path and the epilogue needs few registers.
+    // warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-5 unpack
+    // (four consecutive warps cover the four TMEM lane quarters), then the
+    // epilogue: one warpgroup covers the 128 lanes, a second one splits the
+    // columns of wide token tiles
     static constexpr int kUnpackWarps = 4;
-    // epilogue warps: one warpgroup covers the 128 TMEM lanes; a second one
-    // splits the columns of wide token tiles
-    static constexpr int kEpiWarps = BT <= 32 ? 4 : 8;
-    // warp roles: 0 TMA producer, 1-2 MMA issuers, then unpack, then epilogue
-    static constexpr int kMmaWarps = 2;
-    static constexpr int kFirstUnpackWarp = 1 + kMmaWarps;
+    static constexpr int kFirstUnpackWarp = 2;
     static constexpr int kFirstEpiWarp = kFirstUnpackWarp + kUnpackWarps;
+    static constexpr int kEpiWarps = BT <= 32 ? 4 : 8;
     static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
-    // TMEM accumulator buffers: the MMA may run kAcc - 1 groups ahead of the
-    // per-group drain, so the drain's latency is hidden.
-    static constexpr int kAcc = BT == 128 ? 4 : 8;
+    // TMEM (512 columns): kSA unpacked-operand slots of 64 columns, then kAcc
+    // accumulator buffers of BT columns.  The MMA may run kAcc - 1 groups
+    // ahead of the per-group drain.
+    static constexpr int kAcc = BT == 128 ? 3 : (BT == 64 ? 4 : 8);
+    static constexpr int kSA = (512 - kAcc * BT) / kStageCols > 6 ? 6 : (512 - kAcc * BT) / kStageCols;
+    static constexpr uint32_t kAccCol0 = uint32_t(kSA * kStageCols);
+    static constexpr uint32_t kTmemCols = 512;
+    static_assert(kSA >= 2 && kSA * kStageCols + kAcc * BT <= 512, "TMEM budget");
     // Unpack to 16*q (nibble into the high half of each byte, 5 integer ops per
     // 8 weights) instead of q (9 ops).  The float-scale path folds the 1/16 into
     // s_g for free; the integer-scale path pays one shift per output per group,
@@ -75,27 +86,21 @@ struct Cfg {
     static constexpr bool kX16 = (PATH == kFloatScale) || BT <= 32;
     static constexpr int kWBytes = kTileN * kStageK / 2;  // packed weights per stage: 16 KB
     static constexpr int kXBytes = BT * kStageK;          // token codes per stage
-    static constexpr int kABytes = kTileN * kStageK;      // unpacked weights per stage: 32 KB
-    static constexpr int kSA = BT <= 32 ? 3 : 2;
-    static constexpr int kSW = BT <= 32 ? 5 : (BT == 64 ? 6 : 3);
-    static constexpr int kSX = BT <= 32 ? 4 : 3;
-    // stage-done ring: one tcgen05.commit per stage (a commit costs about as
-    // much issue time as two small MMAs), read by every role that recycles a
-    // resource of that stage; the group scales of a stage travel in a slot of
-    // this ring too (TMA box: 2 groups x 128 columns)
+    static constexpr int kSW = BT <= 32 ? 8 : (BT == 64 ? 6 : 4);
+    static constexpr int kSX = BT <= 32 ? 6 : (BT == 64 ? 4 : 3);
+    // stage-done ring: one tcgen05.commit per stage, read by every role that
+    // recycles a resource of that stage; the group scales of a stage travel in
+    // a slot of this ring too (TMA box: 2 groups x 128 columns)
     static constexpr int kSD = 16;
     static_assert(kSD >= kSX && kSD >= kSA, "stage-done ring shallower than a ring it releases");
     static constexpr int kSBytes = 2 * kTileN * (PATH == kIntScale ? 2 : 4);
     static constexpr int offW = 0;
     static constexpr int offX = offW + kSW * kWBytes;
-    static constexpr int offA = offX + kSX * kXBytes;
-    static constexpr int offS = offA + kSA * kABytes;
+    static constexpr int offS = offX + kSX * kXBytes;
     static constexpr int offBar = offS + kSD * kSBytes;
-    static constexpr int kBars = 2 * kSW + kSX + kSA + 3 * kSD + kAcc + kMmaWarps;
+    static constexpr int kBars = 2 * kSW + kSX + kSA + 3 * kSD + kAcc + 1;
     static constexpr int offMisc = offBar + kBars * 8;
     static constexpr int kSmemBytes = offMisc + 64 + 1024;  // + slack to align the base to 1024
-    static constexpr uint32_t kTmemCols = (kAcc * BT) < 32 ? 32u : uint32_t(kAcc * BT);
-    static_assert(kAcc * BT <= 512 && (kTmemCols & (kTmemCols - 1)) == 0, "TMEM allocation");
     static_assert(kXBytes % 2048 == 0, "token stage must hold whole 8-row swizzle atoms per k-block");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -296,7 +301,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
     uint64_t* full_w = bars;              // W box landed (TMA transaction count)
     uint64_t* empty_w = full_w + SW;      // unpack warps have read the W box
     uint64_t* full_x = empty_w + SW;      // token codes landed
-    uint64_t* full_a = full_x + SX;       // unpacked operand written
+    uint64_t* full_a = full_x + SX;       // unpacked operand written to its TMEM slot
     uint64_t* sdone = full_a + SA;        // all MMAs of a stage complete (one commit per stage)
     uint64_t* sfree = sdone + SD;         // epilogue has seen a stage-done phase (slot may be committed again)
     uint64_t* full_s = sfree + SD;        // a stage's group scales landed
@@ -321,7 +326,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
             mbar_init(&full_s[s], 1);
         }
         for (int s = 0; s < kAcc; ++s) mbar_init(&tempty[s], kEpiWarps);
-        for (int s = 0; s < C::kMmaWarps; ++s) mbar_init(&mma_done[s], 1);
+        mbar_init(&mma_done[0], 1);
         misc[1] = 0;
         misc[2] = 0;
         fence_mbar_init();
@@ -338,9 +343,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
-        // The whole warp walks the loop (so it never diverges around the block
-        // barriers); lane 0 issues the copies.
-        const bool leader = (lane == 0);
+        // The whole warp walks the loop; one elected lane issues the copies.
         Ring rw, rx;
         Ring rxd;          // stage-done slot of the stage whose token slot is reused (SX stages back)
         Ring rs;           // scale slot (same index as the stage-done ring)
@@ -357,12 +360,9 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 ok = false;
                 break;
             }
-            if (leader) {
-                // one 128 x 128 B box = two K blocks (a lone last block over-reads 64 B per row: harmless)
-                mbar_arrive_expect_tx(&full_w[rw.idx], C::kWBytes);
-                tma_load_2d(smem + C::offW + rw.idx * C::kWBytes, &tm_w, st.kb * (kBlockK / 2), n0,
-                            &full_w[rw.idx]);
-            }
+            // one 128 x 128 B box = two K blocks (a lone last block over-reads 64 B per row: harmless)
+            mbar_arrive_expect_tx_one(&full_w[rw.idx], C::kWBytes);
+            tma_load_2d_one(smem + C::offW + rw.idx * C::kWBytes, &tm_w, st.kb * (kBlockK / 2), n0, &full_w[rw.idx]);
             w_issued |= 1u << rw.idx;
             w_par = (w_par & ~(1u << rw.idx)) | (rw.phase << rw.idx);
             rw.advance(SW);
@@ -373,12 +373,11 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 }
                 rxd.advance(SD);
             }
-            if (leader) {
-                mbar_arrive_expect_tx(&full_x[rx.idx], uint32_t(st.nkb * BT * kBlockK));
-                for (int j = 0; j < st.nkb; ++j)
-                    tma_load_2d(smem + C::offX + rx.idx * C::kXBytes + j * BT * kBlockK, &tm_x,
-                                (st.kb + j) * kBlockK, m0, &full_x[rx.idx]);
-            }
+            mbar_arrive_expect_tx_one(&full_x[rx.idx], uint32_t(st.nkb * BT * kBlockK));
+            tma_load_2d_one(smem + C::offX + rx.idx * C::kXBytes, &tm_x, st.kb * kBlockK, m0, &full_x[rx.idx]);
+            if (st.nkb == 2)
+                tma_load_2d_one(smem + C::offX + rx.idx * C::kXBytes + BT * kBlockK, &tm_x, (st.kb + 1) * kBlockK,
+                                m0, &full_x[rx.idx]);
             x_issued |= 1u << rx.idx;
             x_par = (x_par & ~(1u << rx.idx)) | (rx.phase << rx.idx);
             rx.advance(SX);
@@ -387,16 +386,14 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 ok = false;
                 break;
             }
-            if (leader) {
-                mbar_arrive_expect_tx(&full_s[rs.idx], C::kSBytes);
-                tma_load_2d(smem + C::offS + rs.idx * C::kSBytes, &tm_s, n0, st.g, &full_s[rs.idx]);
-            }
+            mbar_arrive_expect_tx_one(&full_s[rs.idx], C::kSBytes);
+            tma_load_2d_one(smem + C::offS + rs.idx * C::kSBytes, &tm_s, n0, st.g, &full_s[rs.idx]);
             s_issued |= 1u << rs.idx;
             s_par = (s_par & ~(1u << rs.idx)) | (rs.phase << rs.idx);
             rs.advance(SD);
             ++pst;
         }
-        if (!ok && leader) {  // let copies in flight land before the CTA leaves
+        if (!ok && lane == 0) {  // let copies in flight land before the CTA leaves
             for (int s = 0; s < SW; ++s)
                 if (w_issued & (1u << s)) drain_wait(&full_w[s], (w_par >> s) & 1u);
             for (int s = 0; s < SX; ++s)
@@ -405,147 +402,134 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 if (s_issued & (1u << s)) drain_wait(&full_s[s], (s_par >> s) & 1u);
         }
         __syncwarp();
-    } else if (warp < C::kFirstUnpackWarp) {
-        // ---------------------------------------------------------- MMA issuers
-        // The issue of one tcgen05.mma, a barrier poll or a commit occupies the
-        // issuing thread for tens to hundreds of cycles, and one thread's issues
-        // do not overlap, while the tensor core accepts small MMAs about twice
-        // as fast as one thread issues them.  So two warps issue alternate
-        // stages.  When a group spans more than two K blocks, consecutive stages
-        // accumulate into one TMEM buffer and must stay in one warp's order, so
-        // the first warp then issues every stage.
-        // Each warp walks every stage (so the ring, buffer and group
-        // bookkeeping stays identical in both) and issues its own; lane 0 issues
-        // the MMAs and the commit (a commit tracks the MMAs of its thread).
-        // One commit per stage, to the stage-done ring; before a stage-done slot
-        // is committed again the epilogue must have seen its previous phase.
-        const int mw = warp - 1;
-        const int nmma = (p.kb_per_group <= 2) ? C::kMmaWarps : 1;
-        const bool leader = (lane == 0);
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        // One converged warp; each MMA and the per-stage commit are issued by
+        // one elected lane.  Per stage: wait for the unpacked operand (TMEM
+        // slot) and the token codes, issue up to 8 MMAs (4 per K block) into
+        // the accumulator buffer of the current group, and commit once to the
+        // stage-done ring, which frees the operand slot, the token slot and,
+        // for the epilogue, marks the groups that ended in the stage.  Before a
+        // stage-done slot is committed again the epilogue must have seen its
+        // previous phase.
         constexpr uint32_t idesc = idesc_i8(kTileN, BT);
-        if (mw < nmma) {
-            Ring rx, ra, rt, rd;
-            StageIter it(p, b);
-            Stage st;
-            bool ok = true;
-            int32_t si = 0;   // stage index within this CTA
-            int32_t kin = 0;  // position of the next K block inside its group (segments start on group boundaries)
-            // descriptor low words of slot 0; slots and K steps are plain offsets from here
-            const uint32_t a_lo0 = smem_desc_sw128_lo(smem_u32(smem + C::offA));
-            const uint32_t x_lo0 = smem_desc_sw128_lo(smem_u32(smem + C::offX));
-            while (ok && it.next(st)) {
-                if ((si % nmma) != mw) {  // another warp's stage: only keep the bookkeeping in step
-                    for (int j = 0; j < st.nkb; ++j) {
-                        const bool last = (kin == p.kb_per_group - 1);
-                        kin = last ? 0 : kin + 1;
-                        if (last) rt.advance(kAcc);
-                    }
-                } else {
-                    if (!mbar_wait_warp(&full_a[ra.idx], ra.phase, abort_flag, p.status) ||
-                        !mbar_wait_warp(&full_x[rx.idx], rx.phase, abort_flag, p.status)) {
+        Ring rx, ra, rt, rd;
+        StageIter it(p, b);
+        Stage st;
+        bool ok = true;
+        int32_t kin = 0;  // position of the next K block inside its group (segments start on group boundaries)
+        const uint32_t x_lo0 = smem_desc_sw128_lo(smem_u32(smem + C::offX));
+        while (ok && it.next(st)) {
+            if (!mbar_wait_warp(&full_a[ra.idx], ra.phase, abort_flag, p.status) ||
+                !mbar_wait_warp(&full_x[rx.idx], rx.phase, abort_flag, p.status)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t a_col = tmem_base + uint32_t(ra.idx * kStageCols);
+            const uint32_t x_lo = x_lo0 + uint32_t(rx.idx) * uint32_t(C::kXBytes >> 4);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                if (j >= st.nkb) break;
+                const bool first = (kin == 0);
+                const bool last = (kin == p.kb_per_group - 1);
+                kin = last ? 0 : kin + 1;
+                if (first) {
+                    if (!mbar_wait_warp(&tempty[rt.idx], rt.phase ^ 1u, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_lo = a_lo0 + uint32_t(ra.idx) * uint32_t(C::kABytes >> 4);
-                    const uint32_t x_lo = x_lo0 + uint32_t(rx.idx) * uint32_t(C::kXBytes >> 4);
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        if (j >= st.nkb) break;
-                        const bool first = (kin == 0);
-                        const bool last = (kin == p.kb_per_group - 1);
-                        kin = last ? 0 : kin + 1;
-                        if (first) {
-                            if (!mbar_wait_warp(&tempty[rt.idx], rt.phase ^ 1u, abort_flag, p.status)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                        }
-                        if (leader) {
-                            const uint32_t d = tmem_base + uint32_t(rt.idx * BT);
-                            const uint32_t aj = a_lo + uint32_t(j * ((kTileN * kBlockK) >> 4));
-                            const uint32_t xj = x_lo + uint32_t(j * ((BT * kBlockK) >> 4));
-#pragma unroll
-                            for (int k = 0; k < kBlockK / 32; ++k)  // 32 bytes of K per MMA = 2 descriptor units
-                                mma_i8(d, smem_desc_from_lo(aj + 2u * k), smem_desc_from_lo(xj + 2u * k), idesc,
-                                       (first && k == 0) ? 0u : 1u);
-                        }
-                        if (last) rt.advance(kAcc);
-                    }
-                    if (!ok) break;
-                    if (!mbar_wait_warp(&sfree[rd.idx], rd.phase ^ 1u, abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    if (leader) mma_commit(&sdone[rd.idx]);
-                    __syncwarp();
                 }
-                ra.advance(SA);
-                rx.advance(SX);
-                rd.advance(SD);
-                ++si;
+                const uint32_t d = tmem_base + C::kAccCol0 + uint32_t(rt.idx * BT);
+                const uint32_t aj = a_col + uint32_t(j * (kBlockK / 4));
+                const uint32_t xj = x_lo + uint32_t(j * ((BT * kBlockK) >> 4));
+#pragma unroll
+                for (int k = 0; k < kBlockK / 32; ++k)  // 32 K per MMA: 8 TMEM columns of A, 2 descriptor units of B
+                    mma_i8_tmem_a_one(d, aj + uint32_t(8 * k), smem_desc_from_lo(xj + 2u * k), idesc,
+                                      (first && k == 0) ? 0u : 1u);
+                if (last) rt.advance(kAcc);
             }
-            // every MMA this warp issued has finished before TMEM is released
-            if (leader) {
-                mma_commit(&mma_done[mw]);
-                drain_wait(&mma_done[mw], 0);
+            if (!ok) break;
+            if (!mbar_wait_warp(&sfree[rd.idx], rd.phase ^ 1u, abort_flag, p.status)) {
+                ok = false;
+                break;
             }
-            __syncwarp();
+            mma_commit_one(&sdone[rd.idx]);
+            ra.advance(SA);
+            rx.advance(SX);
+            rd.advance(SD);
         }
+        // every MMA issued has finished before TMEM is released
+        mma_commit_one(&mma_done[0]);
+        if (lane == 0) drain_wait(&mma_done[0], 0);
+        __syncwarp();
     } else if (warp < C::kFirstEpiWarp) {
         // ---------------------------------------------------------- int4 -> int8 unpack
-        // Thread -> (row, 16-byte packed chunk): a quarter warp covers two rows x
-        // four chunks, which with the 128-byte swizzle of both tiles keeps the
-        // shared-memory reads and writes free of bank conflicts.
-        const int uw = warp - C::kFirstUnpackWarp;
-        constexpr int kRowsPerWarp = kTileN / kU;
+        // Thread = weight row r of the tile = TMEM lane r.  Per stage it reads
+        // its row's 128 packed bytes (eight 16-byte chunks; with the 128-byte
+        // swizzle the warp's 32 rows spread each chunk over all banks), turns
+        // every chunk into 32 int8 values = 8 TMEM columns, and stores the
+        // stage's 64 columns to its lane of the operand slot.
+        const int quarter = warp & 3;  // TMEM lanes this warp may access
+        const int r = quarter * 32 + lane;
+        const int sw = r & 7;
         Ring rw, ra;
         Ring rad;          // stage-done slot of the stage whose operand slot is reused (SA stages back)
         int32_t ust = 0;   // stages unpacked so far
         StageIter it(p, b);
         Stage st;
         bool ok = true;
+        const uint32_t lane_base = tmem_base + (uint32_t(quarter * 32) << 16);
         while (ok && it.next(st)) {
             if (!mbar_wait_warp(&full_w[rw.idx], rw.phase, abort_flag, p.status)) {
                 ok = false;
                 break;
             }
+            const uint8_t* wrow = smem + C::offW + rw.idx * C::kWBytes + r * (kStageK / 2);
+            uint4 v[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                if (c < 4 * st.nkb) v[c] = *reinterpret_cast<const uint4*>(wrow + ((c ^ sw) << 4));
+            // the packed box may be refilled once every warp has read it (the
+            // arrive releases this thread's loads above)
+            __syncwarp();
+            mbar_arrive_one(&empty_w[rw.idx]);
             if (ust >= SA) {  // the MMAs of stage ust - SA have read this operand slot
                 if (!mbar_wait_warp(&sdone[rad.idx], rad.phase, abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
                 rad.advance(SD);
+                tc_fence_after();
             }
             ++ust;
-            const uint8_t* wsrc = smem + C::offW + rw.idx * C::kWBytes;
-            uint8_t* adst = smem + C::offA + ra.idx * C::kABytes;
-            const int c = lane & 3;
+            const uint32_t slot = lane_base + uint32_t(ra.idx * kStageCols);
 #pragma unroll
-            for (int itr = 0; itr < kRowsPerWarp / 8; ++itr) {
-                const int r = uw * kRowsPerWarp + itr * 8 + (lane >> 2);
-                const int sw = r & 7;
+            for (int j = 0; j < 2; ++j) {
+                if (j < st.nkb) {
+                    uint32_t o[32];
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    if (j < st.nkb) {
-                        const uint4 v =
-                            *reinterpret_cast<const uint4*>(wsrc + r * (kStageK / 2) + (((j * 4 + c) ^ sw) << 4));
-                        const uint2 o0 = unpack8<C::kX16>(v.x), o1 = unpack8<C::kX16>(v.y);
-                        const uint2 o2 = unpack8<C::kX16>(v.z), o3 = unpack8<C::kX16>(v.w);
-                        uint8_t* row = adst + j * (kTileN * kBlockK) + r * kBlockK;
-                        *reinterpret_cast<uint4*>(row + (((2 * c) ^ sw) << 4)) = make_uint4(o0.x, o0.y, o1.x, o1.y);
-                        *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ sw) << 4)) =
-                            make_uint4(o2.x, o2.y, o3.x, o3.y);
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 w = v[4 * j + c];
+                        const uint2 o0 = unpack8<C::kX16>(w.x), o1 = unpack8<C::kX16>(w.y);
+                        const uint2 o2 = unpack8<C::kX16>(w.z), o3 = unpack8<C::kX16>(w.w);
+                        o[8 * c + 0] = o0.x;
+                        o[8 * c + 1] = o0.y;
+                        o[8 * c + 2] = o1.x;
+                        o[8 * c + 3] = o1.y;
+                        o[8 * c + 4] = o2.x;
+                        o[8 * c + 5] = o2.y;
+                        o[8 * c + 6] = o3.x;
+                        o[8 * c + 7] = o3.y;
                     }
+                    tmem_st32(slot + uint32_t(j * (kBlockK / 4)), o);
                 }
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&full_a[ra.idx]);
-                mbar_arrive(&empty_w[rw.idx]);
-            }
+            mbar_arrive_one(&full_a[ra.idx]);
             rw.advance(SW);
             ra.advance(SA);
         }
@@ -602,7 +586,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sfree[rd.idx]);  // the scale slot may be refilled
+                mbar_arrive_one(&sfree[rd.idx]);  // the scale slot may be refilled
                 rd.advance(SD);
                 // groups whose last K block is in this stage (at most two)
                 int ng = 0;
@@ -639,7 +623,8 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                         }
                     }
                 };
-                const uint32_t lane_cols = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(half * HC);
+                const uint32_t lane_cols =
+                    tmem_base + (uint32_t(quarter * 32) << 16) + C::kAccCol0 + uint32_t(half * HC);
                 if constexpr (HC <= 16) {
                     // small tiles: both groups' loads in flight before one wait
                     uint32_t v0[HC], v1[HC];
@@ -663,10 +648,8 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&tempty[gb0]);
-                    if (ng == 2) mbar_arrive(&tempty[gb1]);
-                }
+                mbar_arrive_one(&tempty[gb0]);
+                if (ng == 2) mbar_arrive_one(&tempty[gb1]);
                 g += ng;
             }
             if (!ok) break;
