@@ -131,6 +131,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     DeviceInfo dev;
     if ((st = current_device(dev)) != W4A8_OK) return st;
     const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms);
+    if (pl.W >= (int64_t(1) << 31)) return W4A8_ERR_SHAPE;  // the kernel indexes (tile, group) steps in 32 bits
     int32_t* ws_count = nullptr;
     int32_t* ws_part = nullptr;
     if (plan_splits_tiles(pl)) {
@@ -170,6 +171,8 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     p.m_tiles = pl.m_tiles;
     p.W = pl.W;
     p.grid = pl.grid;
+    p.w_q = uint32_t(pl.W / pl.grid);
+    p.w_r = uint32_t(pl.W % pl.grid);
     p.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
     p.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
                                     : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);

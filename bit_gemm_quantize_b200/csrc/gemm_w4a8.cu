@@ -48,6 +48,7 @@
 #include <cstdint>
 
 #include "gemm_w4a8.h"
+#include "kernels.h"
 #include "sm100_ptx.cuh"
 
 namespace w4a8 {
@@ -106,35 +107,45 @@ struct Cfg {
 };
 
 // One contiguous run of groups [g0, g1) of one tile inside a CTA's range.
+// Step counts stay below 2^31 (checked on the host), so all index arithmetic
+// is 32-bit: a 64-bit division is a long software sequence on the GPU.
 struct Segment {
-    int64_t tile;
+    uint32_t tile;
     int32_t n_tile, m_tile;
     int32_t g0, g1;
-    int64_t first;  // flattened index of the segment's first step
+    uint32_t first;  // flattened index of the segment's first step
 };
 
-__device__ __forceinline__ int64_t range_start(int64_t b, int64_t W, int64_t grid) { return b * W / grid; }
+// First step of CTA b's range: floor(b * W / grid) = b * (W / grid) + floor(b * (W % grid) / grid).
+__device__ __forceinline__ uint32_t range_start(uint32_t b, const Params& p) {
+    return b * p.w_q + (b * p.w_r) / uint32_t(p.grid);
+}
 
-// CTA whose range holds flattened step i.
-__device__ __forceinline__ int64_t range_owner(int64_t i, int64_t W, int64_t grid) {
-    return ((i + 1) * grid - 1) / W;
+// CTA whose range holds step i: the largest b with range_start(b) <= i, from
+// a floating-point estimate corrected with exact starts.
+__device__ __forceinline__ uint32_t range_owner(uint32_t i, const Params& p) {
+    const uint32_t grid = uint32_t(p.grid);
+    uint32_t o = uint32_t((double(i) + 1.0) * double(grid) / double(p.W));
+    if (o >= grid) o = grid - 1;
+    while (o > 0 && range_start(o, p) > i) --o;
+    while (o + 1 < grid && range_start(o + 1, p) <= i) ++o;
+    return o;
 }
 
 // Iterates the segments of CTA `b`.  The divisions happen once, at the start
-// of the range; afterwards the tile coordinates advance incrementally (64-bit
-// division is a long software sequence on the GPU).
+// of the range; afterwards the tile coordinates advance incrementally.
 struct SegmentIter {
-    int64_t i, end, tile;
+    uint32_t i, end, tile;
     int32_t G, g, n_tile, m_tile, m_tiles;
-    __device__ SegmentIter(const Params& p, int64_t b) {
+    __device__ SegmentIter(const Params& p, uint32_t b) {
         G = int32_t(p.G);
         m_tiles = int32_t(p.m_tiles);
-        i = range_start(b, p.W, p.grid);
-        end = range_start(b + 1, p.W, p.grid);
-        tile = i / G;
-        g = int32_t(i - tile * G);
-        n_tile = int32_t(tile / m_tiles);
-        m_tile = int32_t(tile - int64_t(n_tile) * m_tiles);
+        i = range_start(b, p);
+        end = range_start(b + 1, p);
+        tile = i / uint32_t(G);
+        g = int32_t(i - tile * uint32_t(G));
+        n_tile = int32_t(tile / uint32_t(m_tiles));
+        m_tile = int32_t(tile - uint32_t(n_tile) * uint32_t(m_tiles));
     }
     __device__ bool next(Segment& s) {
         if (i >= end) return false;
@@ -142,8 +153,8 @@ struct SegmentIter {
         s.n_tile = n_tile;
         s.m_tile = m_tile;
         s.g0 = g;
-        const int64_t left = end - i;
-        s.g1 = (left >= int64_t(G - g)) ? G : g + int32_t(left);
+        const uint32_t left = end - i;
+        s.g1 = (left >= uint32_t(G - g)) ? G : g + int32_t(left);
         s.first = i;
         i += s.g1 - s.g0;
         if (s.g1 == G) {
@@ -174,7 +185,7 @@ struct StageIter {
     int32_t n_tile = 0, m_tile = 0;
     int32_t kb = 0, kb_end = 0;
     int32_t g = 0, kin = 0;  // group of the next K block and its position in the group
-    __device__ StageIter(const Params& p, int64_t b) : seg(p, b), kbpg(p.kb_per_group) {}
+    __device__ StageIter(const Params& p, uint32_t b) : seg(p, b), kbpg(p.kb_per_group) {}
     __device__ bool next(Stage& st) {
         while (kb >= kb_end) {
             Segment s;
@@ -339,7 +350,10 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = misc[0];
-    const int64_t b = blockIdx.x;
+    const uint32_t b = blockIdx.x;
+    // The next kernel in the stream may be scheduled now; it cannot share an
+    // SM with this CTA (shared memory), so its CTAs start where ours finish.
+    if (threadIdx.x == 0) griddep_launch_dependents();
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
@@ -350,6 +364,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
         int32_t pst = 0;   // stages issued so far
         uint32_t w_issued = 0u, w_par = 0u, x_issued = 0u, x_par = 0u;  // per slot: copy issued / its parity
         uint32_t s_issued = 0u, s_par = 0u;
+        griddep_wait();  // the token codes may be the previous kernel's output
         StageIter it(p, b);
         Stage st;
         bool ok = true;
@@ -535,6 +550,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------- epilogue
+        griddep_wait();  // s_a, y and the workspace may be in use by the previous kernel
         const int ew = warp - C::kFirstEpiWarp;
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int half = ew >> 2;      // which part of the BT columns
@@ -664,9 +680,9 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 continue;
             }
             // ---- split tile: store this CTA's partial, the last contributor combines
-            const int slot = (sg.first == range_start(b, p.W, p.grid)) ? 0 : 1;
+            const int slot = (sg.first == range_start(b, p)) ? 0 : 1;
             const int64_t slot_elems = int64_t(kTileN) * BT;
-            int32_t* part = p.ws_part + (b * 2 + slot) * slot_elems;
+            int32_t* part = p.ws_part + (int64_t(b) * 2 + slot) * slot_elems;
 #pragma unroll
             for (int j = 0; j < HC; ++j) {
                 const int64_t e = int64_t(half * HC + j) * kTileN + r;
@@ -677,9 +693,9 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
             }
             __threadfence();
             epi_bar_sync(kEpiWarps * 32);
-            const int64_t t0 = sg.tile * p.G;
-            const int64_t b_first = range_owner(t0, p.W, p.grid);
-            const int64_t b_last = range_owner(t0 + p.G - 1, p.W, p.grid);
+            const uint32_t t0 = sg.tile * uint32_t(p.G);
+            const uint32_t b_first = range_owner(t0, p);
+            const uint32_t b_last = range_owner(t0 + uint32_t(p.G) - 1u, p);
             if (ew == 0 && lane == 0) {
                 // one counter per CTA: a CTA is the first contributor of at most one split tile
                 const int old = atomicAdd(&p.ws_count[b_first], 1);
@@ -693,9 +709,9 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                     acc[j] = 0;
                     accf[j] = 0.0f;
                 }
-                for (int64_t c = b_first; c <= b_last; ++c) {
-                    const int cslot = (range_start(c, p.W, p.grid) >= t0) ? 0 : 1;
-                    const int32_t* cp = p.ws_part + (c * 2 + cslot) * slot_elems;
+                for (uint32_t c = b_first; c <= b_last; ++c) {
+                    const int cslot = (range_start(c, p) >= t0) ? 0 : 1;
+                    const int32_t* cp = p.ws_part + (int64_t(c) * 2 + cslot) * slot_elems;
 #pragma unroll
                     for (int j = 0; j < HC; ++j) {
                         const int32_t v = __ldcg(cp + int64_t(half * HC + j) * kTileN + r);
@@ -769,8 +785,8 @@ static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const
         if (resident < 1) return cudaErrorLaunchOutOfResources;
         if (dev >= 0 && dev < 64) configured[dev] = true;
     }
-    kern<<<dim3(unsigned(p.grid)), dim3(C::kThreads), smem, stream>>>(tw, tx, ts, p);
-    return cudaGetLastError();
+    const LaunchPdl lc(unsigned(p.grid), C::kThreads, size_t(smem), stream);
+    return cudaLaunchKernelEx(&lc.cfg, kern, tw, tx, ts, p);
 }
 
 cudaError_t launch(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts, const Params& p, int BT, int path,

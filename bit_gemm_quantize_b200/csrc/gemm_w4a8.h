@@ -24,8 +24,9 @@ struct Params {
     int64_t G;           // groups along K
     int32_t kb_per_group;  // 128-wide K blocks per group
     int64_t m_tiles;
-    int64_t W;           // total (tile, group) steps
+    int64_t W;           // total (tile, group) steps, < 2^31
     int64_t grid;        // CTAs
+    uint32_t w_q, w_r;   // W / grid, W % grid
     float inv_alpha;     // 1 / alpha (exact, alpha is a power of two)
     int32_t y_dtype;     // OutType
 };

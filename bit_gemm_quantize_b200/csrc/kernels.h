@@ -7,6 +7,26 @@
 
 namespace w4a8 {
 
+// Launch configuration with programmatic stream serialization: the kernel
+// may start while the previous kernel in the stream is still running; it
+// orders its own accesses with griddepcontrol.wait (see sm100_ptx.cuh).
+struct LaunchPdl {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1]{};
+    LaunchPdl(unsigned grid, unsigned threads, size_t smem, cudaStream_t stream) {
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(threads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    LaunchPdl(const LaunchPdl&) = delete;
+    LaunchPdl& operator=(const LaunchPdl&) = delete;
+};
+
 namespace quant {
 cudaError_t launch(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a,
                    int* status, cudaStream_t stream, int num_sms);

@@ -135,7 +135,10 @@ __global__ void __launch_bounds__(kThreads) quant_rows_staged(const T* __restric
         mbar_init(&bars[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
+        griddep_launch_dependents();
     }
+    // x may be the previous kernel's output, q and s_a its input
+    griddep_wait();
     __syncthreads();
 
     int64_t row = blockIdx.x;
@@ -181,6 +184,8 @@ __global__ void __launch_bounds__(kThreads) quant_rows_direct(const T* __restric
                                                               int64_t ldx, int8_t* __restrict__ q,
                                                               float* __restrict__ s_a) {
     __shared__ float red[kWarps];
+    if (threadIdx.x == 0) griddep_launch_dependents();
+    griddep_wait();  // x may be the previous kernel's output, q and s_a its input
     for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
         const T* r = x + row * ldx;
         const float a = row_absmax<T>(r, K, red);
@@ -240,8 +245,8 @@ static cudaError_t launch_t(const T* x, int64_t M, int64_t K, int64_t ldx, int8_
         cudaError_t e = staged_blocks_per_sm(kern, smem, &per_sm);
         if (e != cudaSuccess) return e;
         const int64_t grid = M < int64_t(num_sms) * per_sm ? M : int64_t(num_sms) * per_sm;
-        kern<<<unsigned(grid), kThreads, smem, stream>>>(x, M, K, ldx, q, s_a, status);
-        return cudaGetLastError();
+        const LaunchPdl lc(unsigned(grid), kThreads, smem, stream);
+        return cudaLaunchKernelEx(&lc.cfg, kern, x, M, K, ldx, q, s_a, status);
     }
     auto kern = quant_rows_direct<T>;
     int per_sm = 0;
@@ -249,8 +254,8 @@ static cudaError_t launch_t(const T* x, int64_t M, int64_t K, int64_t ldx, int8_
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
     const int64_t grid = M < int64_t(num_sms) * per_sm ? M : int64_t(num_sms) * per_sm;
-    kern<<<unsigned(grid), kThreads, 0, stream>>>(x, M, K, ldx, q, s_a);
-    return cudaGetLastError();
+    const LaunchPdl lc(unsigned(grid), kThreads, 0, stream);
+    return cudaLaunchKernelEx(&lc.cfg, kern, x, M, K, ldx, q, s_a);
 }
 
 cudaError_t launch(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a,

@@ -82,13 +82,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-// Warp-wide form: every lane polls (one warp instruction per poll, no
-// divergence around the caller's loop) and the lanes vote, so the warp leaves
-// together and a timeout never splits it.
+// Warp-wide form.  Every lane polls (one warp instruction per poll) and the
+// lanes vote, so the warp stays converged, leaves together and a timeout
+// never splits it.  The common case, a phase that has already completed,
+// costs one poll and one vote; the blocking loop is out of line so that it
+// adds neither instructions nor registers to the caller's fast path.
+static __device__ __noinline__ bool mbar_wait_warp_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                 int* status) {
+    const long long t0 = clock64();
+    while (true) {
+        const bool ok = mbar_try_wait_sleep(bar, parity, 200000u);
+        if (__all_sync(0xffffffffu, ok)) return true;
+        int fail = 0;
+        if ((threadIdx.x & 31) == 0) {
+            if (*abort_flag) {
+                fail = 1;
+            } else if (clock64() - t0 > kWaitLimitCycles) {
+                *abort_flag = 1;
+                atomicExch(status, kStatusTimeout);
+                fail = 1;
+            }
+        }
+        if (__shfl_sync(0xffffffffu, fail, 0)) return false;
+    }
+}
+
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                                int* status) {
-    const bool ok = mbar_wait(bar, parity, abort_flag, status);
-    return __all_sync(0xffffffffu, ok) != 0;
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    return mbar_wait_warp_slow(bar, parity, abort_flag, status);
 }
 
 // ---------------------------------------------------------------- one-lane operations of a converged warp
@@ -111,6 +133,20 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_one(uint64_t* bar, uint32_
         "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
         "r"(bytes)
         : "memory");
+}
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while
+// the previous kernel in the stream is still running.  griddep_wait() blocks
+// the calling thread until that kernel has completed and its memory
+// operations are visible; every thread that reads what the previous kernel
+// may have written, or writes what it may still read, calls it first.
+// griddep_launch_dependents() lets the next kernel start once every CTA of
+// this one has called it or exited (a no-op without the launch attribute).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- async proxy

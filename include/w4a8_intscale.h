@@ -152,7 +152,10 @@ W4A8_API int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32
  * q_x, s_a   device, [M, K] int8 and [M] float32 (from quantize_act_per_token)
  * w_packed   device, [N, K/2] uint8; S device [K/group, N] int16 (from pack_w4_groupwise)
  * alpha      power of two, 1 <= alpha <= 2^30
- * M >= 0 (0 is a no-op), N % 8 == 0, K % 128 == 0, group % 128 == 0, K % group == 0
+ * M >= 0 (0 is a no-op), N % 8 == 0, K % 128 == 0, group % 128 == 0, K % group == 0,
+ *            and ceil(N/128) * ceil(M/BT) * (K/group) < 2^31 with BT the token tile
+ *            (16, 32, 64 or 128, the smallest that holds M, capped at 128);
+ *            otherwise W4A8_ERR_SHAPE
  * y          device, [M, N] of y_dtype: W4A8_F16, W4A8_F32, or W4A8_I32 (acc itself)
  * workspace  device, >= w4a8_gemm_workspace_size(M, N, K, group, 0) bytes (may be
  *            NULL when that size is 0), zero-filled, see above
