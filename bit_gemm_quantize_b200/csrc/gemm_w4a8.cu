@@ -61,6 +61,14 @@ constexpr int kStageCols = kStageK / 4;  // TMEM columns of one stage's A operan
 constexpr int64_t kCounterBytes = 4096;  // one int32 arrival counter per CTA, fixed region
 constexpr int64_t kMaxGrid = kCounterBytes / 4;
 
+// Ring depths (stages) of the packed weights and the token codes.
+#ifndef W4A8_SW
+#define W4A8_SW(BT) ((BT) <= 32 ? 8 : ((BT) == 64 ? 6 : 4))
+#endif
+#ifndef W4A8_SX
+#define W4A8_SX(BT) ((BT) <= 32 ? 6 : ((BT) == 64 ? 4 : 3))
+#endif
+
 template <int BT, int PATH>
 struct Cfg {
     // warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-5 unpack
@@ -87,8 +95,8 @@ struct Cfg {
     static constexpr bool kX16 = (PATH == kFloatScale) || BT <= 32;
     static constexpr int kWBytes = kTileN * kStageK / 2;  // packed weights per stage: 16 KB
     static constexpr int kXBytes = BT * kStageK;          // token codes per stage
-    static constexpr int kSW = BT <= 32 ? 8 : (BT == 64 ? 6 : 4);
-    static constexpr int kSX = BT <= 32 ? 6 : (BT == 64 ? 4 : 3);
+    static constexpr int kSW = W4A8_SW(BT);
+    static constexpr int kSX = W4A8_SX(BT);
     // stage-done ring: one tcgen05.commit per stage, read by every role that
     // recycles a resource of that stage; the group scales of a stage travel in
     // a slot of this ring too (TMA box: 2 groups x 128 columns)
@@ -358,28 +366,50 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         // The whole warp walks the loop; one elected lane issues the copies.
+        // The packed weights of the first SW stages are requested before
+        // waiting for the previous kernel in the stream (this kernel may start
+        // early under programmatic dependent launch; packed weights are never
+        // written by a kernel that lets its successor start early), so the
+        // weight stream is under way by the time the token codes, which that
+        // kernel may still be writing, can be read.
         Ring rw, rx;
         Ring rxd;          // stage-done slot of the stage whose token slot is reused (SX stages back)
         Ring rs;           // scale slot (same index as the stage-done ring)
         int32_t pst = 0;   // stages issued so far
         uint32_t w_issued = 0u, w_par = 0u, x_issued = 0u, x_par = 0u;  // per slot: copy issued / its parity
         uint32_t s_issued = 0u, s_par = 0u;
+        auto issue_w = [&](const Stage& st, const Ring& slot) {
+            // one 128 x 128 B box = two K blocks (a lone last block over-reads 64 B per row: harmless)
+            mbar_arrive_expect_tx_one(&full_w[slot.idx], C::kWBytes);
+            tma_load_2d_one(smem + C::offW + slot.idx * C::kWBytes, &tm_w, st.kb * (kBlockK / 2),
+                            st.n_tile * kTileN, &full_w[slot.idx]);
+            w_issued |= 1u << slot.idx;
+            w_par = (w_par & ~(1u << slot.idx)) | (slot.phase << slot.idx);
+        };
+        int32_t prefetched = 0;  // leading stages whose weights were requested before the wait
+        {
+            StageIter it(p, b);
+            Stage st;
+            while (prefetched < SW && it.next(st)) {
+                issue_w(st, rw);  // fresh ring: every slot is free
+                rw.advance(SW);
+                ++prefetched;
+            }
+        }
+        rw = Ring{};
         griddep_wait();  // the token codes may be the previous kernel's output
         StageIter it(p, b);
         Stage st;
         bool ok = true;
         while (ok && it.next(st)) {
-            const int32_t n0 = st.n_tile * kTileN;
             const int32_t m0 = st.m_tile * BT;
-            if (!mbar_wait_warp(&empty_w[rw.idx], rw.phase ^ 1u, abort_flag, p.status)) {
-                ok = false;
-                break;
+            if (pst >= prefetched) {
+                if (!mbar_wait_warp(&empty_w[rw.idx], rw.phase ^ 1u, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                issue_w(st, rw);
             }
-            // one 128 x 128 B box = two K blocks (a lone last block over-reads 64 B per row: harmless)
-            mbar_arrive_expect_tx_one(&full_w[rw.idx], C::kWBytes);
-            tma_load_2d_one(smem + C::offW + rw.idx * C::kWBytes, &tm_w, st.kb * (kBlockK / 2), n0, &full_w[rw.idx]);
-            w_issued |= 1u << rw.idx;
-            w_par = (w_par & ~(1u << rw.idx)) | (rw.phase << rw.idx);
             rw.advance(SW);
             if (pst >= SX) {  // the MMAs of stage pst - SX have read this token slot
                 if (!mbar_wait_warp(&sdone[rxd.idx], rxd.phase, abort_flag, p.status)) {
@@ -402,7 +432,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 break;
             }
             mbar_arrive_expect_tx_one(&full_s[rs.idx], C::kSBytes);
-            tma_load_2d_one(smem + C::offS + rs.idx * C::kSBytes, &tm_s, n0, st.g, &full_s[rs.idx]);
+            tma_load_2d_one(smem + C::offS + rs.idx * C::kSBytes, &tm_s, st.n_tile * kTileN, st.g, &full_s[rs.idx]);
             s_issued |= 1u << rs.idx;
             s_par = (s_par & ~(1u << rs.idx)) | (rs.phase << rs.idx);
             rs.advance(SD);
