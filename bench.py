@@ -17,6 +17,7 @@ bounded sample of the same workload instead.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -397,7 +398,7 @@ def run_ours(args):
     else:
         roof = {"bound": "tensor", "achieved": alg_ops(Md) / gd / 1e12, "peak": int8_peak, "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = measured_traffic(Md)
     roof["kernel"] = f"w4a8_gemm_kernel (integer scale), M={Md} launch"
     roof["peak_source"] = (f"{peak_src}: HBM copy {hbm_peak} GB/s; int8 = bf16 {bf16_peak} TFLOP/s x "
                            f"{INT8_PER_BF16} (nominal int8:bf16 ratio)")
@@ -417,6 +418,25 @@ def run_ours(args):
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+# DRAM bytes (read + write) per launch of the integer-scale GEMM, from one
+# ncu capture (profiles/gemm_intscale_bt128_m1024_k4096_n22016.md), valid for
+# the kernel source it was taken with (first 16 hex digits of its SHA-256).
+MEASURED_TRAFFIC = {1024: (57.799936e6 + 24.859136e6, "17a547ba26bc1abf")}
+
+
+def measured_traffic(M):
+    rec = MEASURED_TRAFFIC.get(M)
+    if rec is None:
+        return None
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "bit_gemm_quantize_b200", "csrc", "gemm_w4a8.cu")
+    try:
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return rec[0] if digest == rec[1] else None
 
 
 def main():
