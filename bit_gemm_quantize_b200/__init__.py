@@ -14,6 +14,7 @@ from ._native import (  # noqa: F401
     w4a8_amplifier_search,
     w4a8_gemm_floatscale,
     w4a8_gemm_intscale,
+    w4a8_gemm_intscale_static_ws,
 )
 
 __all__ = [
@@ -26,4 +27,5 @@ __all__ = [
     "w4a8_amplifier_search",
     "w4a8_gemm_floatscale",
     "w4a8_gemm_intscale",
+    "w4a8_gemm_intscale_static_ws",
 ]

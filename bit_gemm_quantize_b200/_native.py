@@ -72,6 +72,7 @@ def load(path: str = LIB_PATH):
             "pack_w4_groupwise": ([P, I64, I64, I32_, I32_, P, P, P, P, P, P, P], I32_),
             "w4a8_gemm_workspace_size": ([I64, I64, I64, I32_, I32_], I64),
             "w4a8_gemm_intscale": ([P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
+            "w4a8_gemm_intscale_static_ws": ([P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P], I32_),
             "w4a8_gemm_floatscale": ([P, P, P, P, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
             "w4a8_device_status": ([P, I32_], I32_),
             "w4a8_last_cuda_error": ([I32_], I32_),
@@ -227,6 +228,23 @@ def w4a8_gemm_intscale(q_x, s_a, w_packed, S, alpha: int, *, group: int = 128, o
     code = load().w4a8_gemm_intscale(_ptr(q_x), _ptr(s_a), _ptr(w_packed), _ptr(S), int(alpha), M, N, K, group,
                                      _ptr(y), dt, _ptr(workspace), ws_bytes, _stream(q_x.device))
     _check("w4a8_gemm_intscale", code)
+    return y
+
+
+def w4a8_gemm_intscale_static_ws(q_x, s_a, w_packed, S, alpha: int, *, group: int = 128, out: str = "f16",
+                                 y: torch.Tensor | None = None):
+    """w4a8_gemm_intscale with the library's fixed per-device workspace (no workspace argument)."""
+    N, K2 = w_packed.shape
+    K = 2 * K2
+    M = _gemm_args(q_x, s_a, w_packed, N, K, group)
+    _need_cuda("S", S, torch.int16, 2)
+    dt, tdt = _OUT[out]
+    if y is None:
+        y = torch.empty((M, N), dtype=tdt, device=q_x.device)
+    _need_cuda("y", y, tdt, 2)
+    code = load().w4a8_gemm_intscale_static_ws(_ptr(q_x), _ptr(s_a), _ptr(w_packed), _ptr(S), int(alpha), M, N, K,
+                                               group, _ptr(y), dt, _stream(q_x.device))
+    _check("w4a8_gemm_intscale_static_ws", code)
     return y
 
 

@@ -29,6 +29,25 @@ struct DeviceInfo {
 DeviceInfo g_devices[kMaxDevices];
 std::mutex g_devices_mutex;
 
+// Workspace of w4a8_gemm_intscale_static_ws: one fixed array per device,
+// shared by every call of that entry point on the device.  Its first 4096
+// bytes are the split-tile arrival counters, zero at module load (device
+// globals without an initializer are zero-filled) and left zero by every
+// call that completes; the rest holds partial sums and needs no clearing.
+__device__ __align__(256) uint8_t g_static_workspace[W4A8_STATIC_WORKSPACE_BYTES];
+
+struct StaticWorkspace {
+    bool ready = false;
+    void* ptr = nullptr;
+};
+
+StaticWorkspace g_static_ws[kMaxDevices];
+std::mutex g_static_ws_mutex;
+
+// Device address of the current device's static workspace, looked up once per
+// device (the first call on a device does this set-up).
+w4a8_status static_workspace(void** out);
+
 // Last CUDA runtime error seen by this thread's library calls.
 thread_local cudaError_t t_last_cuda_error = cudaSuccess;
 
@@ -42,6 +61,20 @@ w4a8_status cuda_fail(cudaError_t e) {
         const cudaError_t w4a8_e_ = (expr);           \
         if (w4a8_e_ != cudaSuccess) return cuda_fail(w4a8_e_); \
     } while (0)
+
+w4a8_status static_workspace(void** out) {
+    int dev = 0;
+    W4A8_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return W4A8_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+    StaticWorkspace& w = g_static_ws[dev];
+    if (!w.ready) {
+        W4A8_CUDA_TRY(cudaGetSymbolAddress(&w.ptr, g_static_workspace));
+        w.ready = true;
+    }
+    *out = w.ptr;
+    return W4A8_OK;
+}
 
 w4a8_status current_device(DeviceInfo& out) {
     int dev = 0;
@@ -291,6 +324,21 @@ w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, const uint8_
                                int32_t y_dtype, void* workspace, int64_t workspace_bytes, void* stream) {
     return run_gemm(w4a8::gemm::kIntScale, q_x, s_a, w_packed, S, nullptr, alpha, M, N, K, group, y, y_dtype,
                     workspace, workspace_bytes, stream);
+}
+
+w4a8_status w4a8_gemm_intscale_static_ws(const int8_t* q_x, const float* s_a, const uint8_t* w_packed,
+                                         const int16_t* S, int32_t alpha, int64_t M, int64_t N, int64_t K,
+                                         int32_t group, void* y, int32_t y_dtype, void* stream) {
+    const w4a8_status st = check_gemm_shape(M, N, K, group);
+    if (st != W4A8_OK) return st;
+    const int64_t need = w4a8_gemm_workspace_size(M, N, K, group, 0);
+    if (need < 0) return W4A8_ERR_CUDA;
+    if (need > int64_t(W4A8_STATIC_WORKSPACE_BYTES)) return W4A8_ERR_WORKSPACE;
+    void* ws = nullptr;
+    const w4a8_status sw = static_workspace(&ws);
+    if (sw != W4A8_OK) return sw;
+    return run_gemm(w4a8::gemm::kIntScale, q_x, s_a, w_packed, S, nullptr, alpha, M, N, K, group, y, y_dtype, ws,
+                    int64_t(W4A8_STATIC_WORKSPACE_BYTES), stream);
 }
 
 w4a8_status w4a8_gemm_floatscale(const int8_t* q_x, const float* s_a, const uint8_t* w_packed, const float* s_g,

@@ -168,6 +168,30 @@ W4A8_API w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, con
                                int64_t workspace_bytes, void* stream);
 
 /*
+ * The integer-scale GEMM above with its workspace in a fixed device array of
+ * the library instead of a caller buffer, so that a call allocates nothing.
+ * The paper has no counterpart: it is a deployment convenience of this
+ * library, the computation is w4a8_gemm_intscale's.
+ * Arguments as w4a8_gemm_intscale without workspace and workspace_bytes.
+ * Limit: calls whose w4a8_gemm_workspace_size(M, N, K, group, 0) exceeds
+ * W4A8_STATIC_WORKSPACE_BYTES (8 MiB: every plan with token tiles up to 32,
+ * i.e. M <= 32, and any plan that splits no tile) are refused with
+ * W4A8_ERR_WORKSPACE before anything is launched.
+ * The array is one per device and shared by every call of this entry point
+ * on that device: calls whose kernels overlap on the GPU (different streams
+ * without ordering) race on it and must not be issued.  Its first 4096 bytes
+ * are arrival counters that start at zero (at library load) and that every
+ * completed call leaves at zero; the rest needs no clearing.
+ * The first call on a device looks the array's address up (a CUDA runtime
+ * call that must not run inside a stream capture), so make one call on each
+ * device before capturing any.
+ */
+#define W4A8_STATIC_WORKSPACE_BYTES (8 << 20)
+W4A8_API w4a8_status w4a8_gemm_intscale_static_ws(const int8_t* q_x, const float* s_a, const uint8_t* w_packed,
+                                                 const int16_t* S, int32_t alpha, int64_t M, int64_t N, int64_t K,
+                                                 int32_t group, void* y, int32_t y_dtype, void* stream);
+
+/*
  * W4A8 GEMM with float group scales, the comparison path.
  * (Integer Scale summary §3.2 / Fig. 3(b): every group's int32 result is
  *  converted to fp32 and multiplied by its float scale.)
