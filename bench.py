@@ -204,6 +204,31 @@ def run_reference(args):
     return 0
 
 
+# ---------------------------------------------------------------- rank aggregation
+
+def max_over_ranks(times_ms, world, device):
+    """Element-wise maximum over all ranks of this rank's device times (ms).
+
+    Every rank calls it in the same order (one collective); with world == 1
+    it returns the times unchanged.
+    """
+    import torch
+    import torch.distributed as dist
+
+    vals = torch.tensor([float(t) for t in times_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    return [float(v) for v in vals]
+
+
+def whole_job_tops(world, ops_per_step_per_rank, steps, max_ms):
+    """Whole-job throughput: the work of all ranks over the slowest rank's time.
+
+    Each rank processes its own, equally sized layer (weak scaling).
+    """
+    return world * ops_per_step_per_rank * steps / (max_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- GPU leg
 
 def run_ours(args):
@@ -362,13 +387,10 @@ def run_ours(args):
     d2h = sum(M * N_DIM * 2 for M in SWEEP)
 
     # ---- aggregate over ranks: max time
-    vals = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(vals[0]), float(vals[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, dev)
     ops_step = sum(alg_ops(M) for M in SWEEP)
-    value = world * ops_step * args.steps / (total_ms * 1e-3) / 1e12
-    e2e_value = world * ops_step * args.steps / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_tops(world, ops_step, args.steps, total_ms)
+    e2e_value = whole_job_tops(world, ops_step, args.steps, e2e_ms)
 
     sweep = []
     for i, M in enumerate(SWEEP):
