@@ -61,6 +61,18 @@ constexpr int kStageCols = kStageK / 4;  // TMEM columns of one stage's A operan
 constexpr int64_t kCounterBytes = 4096;  // one int32 arrival counter per CTA, fixed region
 constexpr int64_t kMaxGrid = kCounterBytes / 4;
 
+// Epilogue warps (multiples of 4) and TMEM columns per drain load.
+#ifndef W4A8_EPI_WARPS
+#define W4A8_EPI_WARPS(BT) ((BT) <= 32 ? 4 : ((BT) == 64 ? 8 : 16))
+#endif
+#ifndef W4A8_DRAIN_CH
+#define W4A8_DRAIN_CH 16
+#endif
+// Token tiles up to which the integer-scale path unpacks to 16*q.
+#ifndef W4A8_X16_IS_MAX_BT
+#define W4A8_X16_IS_MAX_BT 128
+#endif
+
 // Ring depths (stages) of the packed weights and the token codes.
 #ifndef W4A8_SW
 #define W4A8_SW(BT) ((BT) <= 32 ? 8 : ((BT) == 64 ? 6 : 4))
@@ -73,12 +85,13 @@ template <int BT, int PATH>
 struct Cfg {
     // warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-5 unpack
     // (four consecutive warps cover the four TMEM lane quarters), then the
-    // epilogue: one warpgroup covers the 128 lanes, a second one splits the
-    // columns of wide token tiles
+    // epilogue: each warpgroup covers the 128 lanes for its share of the BT
+    // columns (1, 2 or 4 warpgroups: wide tiles split the per-group drain so
+    // that each thread keeps fewer running sums and more drains overlap)
     static constexpr int kUnpackWarps = 4;
     static constexpr int kFirstUnpackWarp = 2;
     static constexpr int kFirstEpiWarp = kFirstUnpackWarp + kUnpackWarps;
-    static constexpr int kEpiWarps = BT <= 32 ? 4 : 8;
+    static constexpr int kEpiWarps = W4A8_EPI_WARPS(BT);
     static constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
     // TMEM (512 columns): kSA unpacked-operand slots of 64 columns, then kAcc
     // accumulator buffers of BT columns.  The MMA may run kAcc - 1 groups
@@ -90,9 +103,10 @@ struct Cfg {
     static_assert(kSA >= 2 && kSA * kStageCols + kAcc * BT <= 512, "TMEM budget");
     // Unpack to 16*q (nibble into the high half of each byte, 5 integer ops per
     // 8 weights) instead of q (9 ops).  The float-scale path folds the 1/16 into
-    // s_g for free; the integer-scale path pays one shift per output per group,
-    // worth it only while the unpack dominates (small token tiles).
-    static constexpr bool kX16 = (PATH == kFloatScale) || BT <= 32;
+    // s_g for free; the integer-scale path pays one shift per output per group
+    // (P_g is 16 times the group product exactly), which measured faster than
+    // the exact unpack for every token tile.
+    static constexpr bool kX16 = (PATH == kFloatScale) || BT <= W4A8_X16_IS_MAX_BT;
     static constexpr int kWBytes = kTileN * kStageK / 2;  // packed weights per stage: 16 KB
     static constexpr int kXBytes = BT * kStageK;          // token codes per stage
     static constexpr int kSW = W4A8_SW(BT);
@@ -680,7 +694,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                     accumulate(v0, 0, HC, take_scale());
                     if (ng == 2) accumulate(v1, 0, HC, take_scale());
                 } else {
-                    constexpr int CH = 32;
+                    constexpr int CH = W4A8_DRAIN_CH < HC ? W4A8_DRAIN_CH : HC;
                     for (int gi = 0; gi < ng; ++gi) {
                         const uint32_t sraw = take_scale();
 #pragma unroll
