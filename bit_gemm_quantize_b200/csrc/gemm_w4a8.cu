@@ -35,12 +35,14 @@
 //
 // Work partition: the (tile, group) steps of the whole problem are split into
 // one contiguous range per CTA of a persistent grid (stream-K).  A tile whose
-// groups fall into several CTAs' ranges is combined through a workspace: each
-// contributor stores its partial, the last one to arrive (an arrival counter
-// per split tile, indexed by the tile's first contributing CTA, which is the
-// first contributor of no other split tile) sums the partials in CTA order
-// and writes y.  Integer partials are exact; float partials are summed in a
-// fixed order, so results are deterministic.
+// groups fall into several CTAs' ranges is combined through a workspace: its
+// first contributor covers the tile's first groups at the end of its own
+// range, so it finishes its share last; every other contributor stores its
+// partial and signals an arrival counter (indexed by the first contributor,
+// which is the first contributor of no other split tile); the first
+// contributor waits for them, adds the partials to its own in CTA order and
+// writes y.  Integer partials are exact; float partials are summed in a fixed
+// order, so results are deterministic.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -288,23 +290,37 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// Output scale of token m: s_a[m] / alpha (exact: 1/alpha is a power of two)
+// for the integer-scale path, s_a[m] for the float-scale path.
 template <int PATH>
-__device__ __forceinline__ void store_output(const Params& p, int64_t m, int64_t n, float vf, int32_t vi) {
+__device__ __forceinline__ float output_scale(const Params& p, int64_t m) {
+    return PATH == kIntScale ? __fmul_rn(p.s_a[m], p.inv_alpha) : p.s_a[m];
+}
+
+template <int PATH>
+__device__ __forceinline__ void store_output(const Params& p, int64_t m, int64_t n, float vf, int32_t vi,
+                                             float scale) {
     const int64_t idx = m * p.N + n;
     if (PATH == kIntScale) {
         if (p.y_dtype == kOutI32) {
             static_cast<int32_t*>(p.y)[idx] = vi;
             return;
         }
-        const float scale = __fmul_rn(p.s_a[m], p.inv_alpha);  // exact: inv_alpha is a power of two
         vf = __fmul_rn(__int2float_rn(vi), scale);
     } else {
-        vf = __fmul_rn(vf, p.s_a[m]);
+        vf = __fmul_rn(vf, scale);
     }
     if (p.y_dtype == kOutF16)
         static_cast<__half*>(p.y)[idx] = __float2half_rn(vf);
     else
         static_cast<float*>(p.y)[idx] = vf;
+}
+
+// Acquire load at GPU scope (the arrival counter of a split tile).
+__device__ __forceinline__ int ld_acquire_gpu(const int* addr) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+    return v;
 }
 
 struct Ring {
@@ -714,50 +730,86 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
             }
             if (!ok) break;
 
+            // valid token columns of this thread's share; with narrow tiles their
+            // output scales are requested first so that they arrive during the
+            // rest of the tail (wide tiles have no registers to spare for them)
+            const int nv = p.M - m0 >= HC ? HC : (p.M - m0 > 0 ? int(p.M - m0) : 0);
+            constexpr bool kEarlyScale = HC <= 16;
+            float osc[kEarlyScale ? HC : 1];
+            if constexpr (kEarlyScale) {
+#pragma unroll
+                for (int j = 0; j < HC; ++j) osc[j] = j < nv ? output_scale<PATH>(p, m0 + j) : 0.0f;
+            }
+            auto out_scale = [&](int j) -> float {
+                if constexpr (kEarlyScale)
+                    return osc[j];
+                else
+                    return output_scale<PATH>(p, m0 + j);
+            };
             const bool whole = (sg.g0 == 0 && sg.g1 == p.G);
             if (whole) {
                 if (nvalid) {
 #pragma unroll
                     for (int j = 0; j < HC; ++j)
-                        if (m0 + j < p.M) store_output<PATH>(p, m0 + j, n, accf[j], acc[j]);
+                        if (j < nv) store_output<PATH>(p, m0 + j, n, accf[j], acc[j], out_scale(j));
                 }
                 continue;
             }
-            // ---- split tile: store this CTA's partial, the last contributor combines
-            const int slot = (sg.first == range_start(b, p)) ? 0 : 1;
-            const int64_t slot_elems = int64_t(kTileN) * BT;
-            int32_t* part = p.ws_part + (int64_t(b) * 2 + slot) * slot_elems;
-#pragma unroll
-            for (int j = 0; j < HC; ++j) {
-                const int64_t e = int64_t(half * HC + j) * kTileN + r;
-                if (PATH == kIntScale)
-                    part[e] = acc[j];
-                else
-                    part[e] = __float_as_int(accf[j]);
-            }
-            __threadfence();
-            epi_bar_sync(kEpiWarps * 32);
+            // ---- split tile.  The tile's first contributor b_first covers the
+            // tile's first groups at the end of its own range, so it finishes its
+            // share last: it combines.  Every other contributor stores its partial
+            // (valid columns only, in the slot of its CTA: a CTA contributes a
+            // partial to at most one tile, the one whose last groups open its range)
+            // and signals an arrival counter indexed by b_first (the first
+            // contributor of no other tile).  b_first waits (bounded) for all
+            // arrivals, adds the partials to its own, which never leave registers,
+            // writes y and re-zeroes the counter.
             const uint32_t t0 = sg.tile * uint32_t(p.G);
             const uint32_t b_first = range_owner(t0, p);
             const uint32_t b_last = range_owner(t0 + uint32_t(p.G) - 1u, p);
-            if (ew == 0 && lane == 0) {
-                // one counter per CTA: a CTA is the first contributor of at most one split tile
-                const int old = atomicAdd(&p.ws_count[b_first], 1);
-                misc[2] = (old == int(b_last - b_first)) ? 1u : 0u;
-            }
-            epi_bar_sync(kEpiWarps * 32);
-            if (misc[2]) {
-                __threadfence();
+            const int64_t slot_elems = int64_t(kTileN) * BT;
+            if (b != b_first) {
+                int32_t* part = p.ws_part + int64_t(b) * slot_elems;
 #pragma unroll
                 for (int j = 0; j < HC; ++j) {
-                    acc[j] = 0;
-                    accf[j] = 0.0f;
+                    if (j < nv) {
+                        const int64_t e = int64_t(half * HC + j) * kTileN + r;
+                        part[e] = PATH == kIntScale ? acc[j] : __float_as_int(accf[j]);
+                    }
                 }
-                for (uint32_t c = b_first; c <= b_last; ++c) {
-                    const int cslot = (range_start(c, p) >= t0) ? 0 : 1;
-                    const int32_t* cp = p.ws_part + (int64_t(c) * 2 + cslot) * slot_elems;
+                epi_bar_sync(kEpiWarps * 32);
+                if (ew == 0 && lane == 0) {
+                    __threadfence();  // the CTA's partial stores (ordered by the barrier) before the arrival
+                    atomicAdd(&p.ws_count[b_first], 1);
+                }
+                continue;
+            }
+            if (ew == 0 && lane == 0) {
+                const int expect = int(b_last - b_first);
+                const long long w0 = clock64();
+                int ok_wait = 1;
+                while (ld_acquire_gpu(&p.ws_count[b_first]) < expect) {
+                    if (*abort_flag || clock64() - w0 > kWaitLimitCycles) {
+                        *abort_flag = 1;
+                        atomicExch(p.status, kStatusTimeout);
+                        ok_wait = 0;
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+                misc[2] = uint32_t(ok_wait);
+                __threadfence();
+            }
+            epi_bar_sync(kEpiWarps * 32);
+            if (!misc[2]) {
+                ok = false;
+                break;
+            }
+            for (uint32_t c = b_first + 1; c <= b_last; ++c) {
+                const int32_t* cp = p.ws_part + int64_t(c) * slot_elems;
 #pragma unroll
-                    for (int j = 0; j < HC; ++j) {
+                for (int j = 0; j < HC; ++j) {
+                    if (j < nv) {
                         const int32_t v = __ldcg(cp + int64_t(half * HC + j) * kTileN + r);
                         if (PATH == kIntScale)
                             acc[j] += v;
@@ -765,13 +817,14 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                             accf[j] = __fadd_rn(accf[j], __int_as_float(v));
                     }
                 }
-                if (nvalid) {
-#pragma unroll
-                    for (int j = 0; j < HC; ++j)
-                        if (m0 + j < p.M) store_output<PATH>(p, m0 + j, n, accf[j], acc[j]);
-                }
-                if (ew == 0 && lane == 0) p.ws_count[b_first] = 0;
             }
+            if (nvalid) {
+#pragma unroll
+                for (int j = 0; j < HC; ++j)
+                    if (j < nv) store_output<PATH>(p, m0 + j, n, accf[j], acc[j], out_scale(j));
+            }
+            epi_bar_sync(kEpiWarps * 32);  // every thread has read the partials before the counter is reused
+            if (ew == 0 && lane == 0) p.ws_count[b_first] = 0;
             epi_bar_sync(kEpiWarps * 32);
         }
     }
@@ -805,7 +858,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms) {
     if (pl.grid > kMaxGrid) pl.grid = kMaxGrid;
     const int64_t slot_bytes = int64_t(kTileN) * pl.BT * 4;
     pl.count_bytes = kCounterBytes;
-    pl.ws_bytes = pl.count_bytes + pl.grid * 2 * slot_bytes;
+    pl.ws_bytes = pl.count_bytes + pl.grid * slot_bytes;  // a CTA stores the partial of at most one tile
     return pl;
 }
 

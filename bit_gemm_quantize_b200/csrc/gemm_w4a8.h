@@ -17,7 +17,7 @@ struct Params {
     const int16_t* S;    // [G, N] integer group scales (integer-scale path)
     const float* s_g;    // [G, N] float group scales (float-scale path)
     void* y;             // [M, N] output
-    int32_t* ws_part;    // [grid][2][128 * BT] partial sums of split tiles
+    int32_t* ws_part;    // [grid][128 * BT] partial sums of split tiles (one per contributing CTA)
     int32_t* ws_count;   // [grid] arrival counters (index: first contributing CTA), zero between calls
     int* status;         // device status word for timeouts
     int64_t M, N;

@@ -174,8 +174,8 @@ W4A8_API w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, con
  * library, the computation is w4a8_gemm_intscale's.
  * Arguments as w4a8_gemm_intscale without workspace and workspace_bytes.
  * Limit: calls whose w4a8_gemm_workspace_size(M, N, K, group, 0) exceeds
- * W4A8_STATIC_WORKSPACE_BYTES (8 MiB: every plan with token tiles up to 32,
- * i.e. M <= 32, and any plan that splits no tile) are refused with
+ * W4A8_STATIC_WORKSPACE_BYTES (8 MiB: every plan with token tiles up to 64,
+ * i.e. M <= 64, and any plan that splits no tile) are refused with
  * W4A8_ERR_WORKSPACE before anything is launched.
  * The array is one per device and shared by every call of this entry point
  * on that device: calls whose kernels overlap on the GPU (different streams
