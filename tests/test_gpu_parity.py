@@ -7,6 +7,8 @@ must match bit for bit.  Floating-point outputs must satisfy
 rtol = 1e-3 for fp32 output and 4e-3 for fp16 output: y_ref is the oracle's
 fp64 result, the GPU rounds twice in fp32 before the output rounding.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -216,6 +218,31 @@ def test_gemm_search_alpha_and_tiny_config():
         assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
         y = bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], pk["alpha"], out="f32")
         _assert_close(y.cpu().numpy(), ref["y64"], "f32")
+
+
+@pytest.mark.parametrize("M,K,N", [(8, 4096, 1024), (200, 1024, 512)])
+def test_gemm_intscale_rows_beyond_the_shift_free_bound(M, K, N):
+    """Output columns whose sum_g |S[g,n]| is too large for accumulating 16 P_g
+    without overflow (here columns 64..127 and 300.., weights scaled up) take the
+    shifted drain, the others the shift-free one, inside the same tiles and the
+    same split tiles: raw accumulators bit-exact either way."""
+    dev = _dev()
+    wl = workloads.make_linear(M, K, N, x_dtype="bf16", seed=77 + M)
+    w = wl.w.copy()
+    big = 6.0 if K >= 4096 else 30.0  # enough groups x scale to pass the bound
+    w[:, 64:128] *= big
+    w[:, 300:] *= big
+    wl = dataclasses.replace(wl, w=w)
+    q, s, pk = _gpu_layer(wl, dev, 128, 1024)
+    colsum = pk["S"].abs().to(torch.int64).sum(0).cpu().numpy()
+    limit = (1 << 31) // (128 * 127 * 128)
+    assert (colsum[64:128] > limit).all() and (colsum[:64] <= limit).all()  # both drains are exercised
+    ref = oracle.linear_intscale(wl.x, wl.w, group=128, alpha=1024, out="f32")
+    acc = bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], pk["alpha"], group=128, out="i32")
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+    y = bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], pk["alpha"], group=128, out="f16")
+    _assert_close(y.float().cpu().numpy(), ref["y64"], "f16")
+    assert bgq.device_status() == 0
 
 
 def test_gemm_zero_input_and_empty():
