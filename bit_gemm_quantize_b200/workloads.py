@@ -31,6 +31,7 @@ __all__ = [
     "MoEWorkload",
     "make_linear",
     "make_moe",
+    "route_rows",
     "to_bf16_bits",
     "bf16_bits_to_f32",
     "SWEEP_M",
@@ -141,6 +142,24 @@ def make_moe(
     x = bf16_bits_to_f32(to_bf16_bits(x))
     route = np.stack([rng.choice(experts, size=topk, replace=False) for _ in range(tokens)]).astype(np.int64)
     return MoEWorkload(x=x, w=ws, experts=route, outlier_cols=cols.astype(np.int64), seed=seed)
+
+
+def route_rows(experts: np.ndarray, n_experts: int):
+    """Layout of the routed rows of a top-k routing [T, topk]: rows grouped by
+    expert (expert 0 first), tokens ascending within an expert.
+
+    Returns (row_index int32 [R]: the token of each routed row,
+    offsets int64 [E+1]: the rows of expert e are offsets[e] .. offsets[e+1]-1).
+    """
+    experts = np.asarray(experts, np.int64)
+    T, topk = experts.shape
+    token = np.repeat(np.arange(T, dtype=np.int64), topk)
+    expert = experts.reshape(-1)
+    order = np.lexsort((token, expert))  # by expert, then token
+    row_index = token[order].astype(np.int32)
+    counts = np.bincount(expert, minlength=n_experts).astype(np.int64)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+    return row_index, offsets
 
 
 # The five workloads, by what they are.  Each entry: dict of keyword arguments.

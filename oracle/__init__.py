@@ -26,6 +26,10 @@ Parity status per function (what pins it, see tests/test_oracle_pins.py):
   floatscale                       equals the per-channel outer-product dequant
                                    when group = K; equals intscale when s_g*alpha
                                    is an integer
+  moe_intscale                     one expert with every token routed to it is the
+                                   dense layer; identical experts repeat the dense
+                                   rows; the shared amplifier's postcondition over
+                                   all experts; rows depend only on (token, expert)
 """
 from __future__ import annotations
 
@@ -265,3 +269,42 @@ def linear_floatscale(x, w, *, group: int = 128, out: str = "f16"):
     qw, s_g = quantize_groups(w, group)
     y64 = floatscale(qx, s_a, qw, s_g, group)
     return dict(qx=qx, s_a=s_a, qw=qw, s_g=s_g, y64=y64, y=round_output(y64, out))
+
+
+# ---------------------------------------------------------------- mixture of experts
+
+def moe_intscale(x, ws, row_index, offsets, *, group: int = 128, alpha=1024, out: str = "f16"):
+    """A mixture-of-experts layer through the Integer-Scale path (the Integer
+    Scale summary, the Mixtral results of §5.3: per-expert fine-grained W4A8
+    GEMMs).  Every token is quantized once (its scale does not depend on the
+    expert); the amplifier is one per layer (the search of §3.3 run over the
+    group scales of all experts: the layer spans all of them, a reading); the
+    routed rows of expert e, row_index[offsets[e]:offsets[e+1]], go through
+    expert e's integer-scale GEMM.
+
+    Returns the routed rows' raw accumulators acc [R, N], fp64 outputs y64,
+    the rounded outputs, the shared alpha and every expert's codes, scales,
+    packed bytes and integer scales.
+    """
+    qx, s_a = quantize_act_per_token(x)
+    qws, sgs = [], []
+    for w in ws:
+        qw, sg = quantize_groups(w, group)
+        qws.append(qw)
+        sgs.append(sg)
+    a = amplifier_search(np.concatenate([sg.reshape(-1) for sg in sgs])) if alpha is None else int(alpha)
+    Ss = [integer_scales(sg, a) for sg in sgs]
+    row_index = np.asarray(row_index, np.int64)
+    N = ws[0].shape[1]
+    acc = np.zeros((row_index.shape[0], N), np.int64)
+    y64 = np.zeros((row_index.shape[0], N), np.float64)
+    for e in range(len(ws)):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi == lo:
+            continue
+        toks = row_index[lo:hi]
+        acc[lo:hi] = intscale_acc(qx[toks], qws[e], Ss[e], group)
+        y64[lo:hi] = intscale_output(acc[lo:hi], s_a[toks], a)
+    return dict(qx=qx, s_a=s_a, qw=qws, s_g=sgs, S=Ss, packed=[pack_int4(q) for q in qws], alpha=a, acc=acc,
+                y64=y64, y=round_output(y64, out))
+

@@ -373,3 +373,69 @@ def test_workload_bound_holds_for_default_amplifier():
     S = oracle.integer_scales(s_g, 1024)
     assert S.max() <= 32767
     assert 127 * 7 * 128 * oracle.scale_colsum_max(S) < 2 ** 31
+
+
+# ------------------------------------------------------------ mixture of experts (the Mixtral results)
+
+def test_route_rows_layout():
+    """Rows grouped by expert, tokens ascending inside an expert, every
+    (token, expert) pair of the routing exactly once; offsets = histogram."""
+    wl = workloads.make_moe(50, 128, 8, 6, topk=2, seed=3)
+    ri, off = workloads.route_rows(wl.experts, 6)
+    assert off[0] == 0 and off[-1] == 100
+    assert np.array_equal(np.diff(off), np.bincount(wl.experts.reshape(-1), minlength=6))
+    pairs = sorted((int(e), int(t)) for t in range(50) for e in wl.experts[t])
+    got = [(e, int(ri[i])) for e in range(6) for i in range(off[e], off[e + 1])]
+    assert got == pairs
+
+
+def test_moe_single_expert_is_the_dense_layer():
+    """E = 1 with every token routed to it: the dense Integer-Scale layer."""
+    wl = workloads.make_linear(24, 512, 136, x_dtype="bf16", seed=11)
+    ri, off = workloads.route_rows(np.zeros((24, 1), np.int64), 1)
+    for alpha in (1024, None):
+        moe = oracle.moe_intscale(wl.x, [wl.w], ri, off, alpha=alpha, out="f32")
+        dense = oracle.linear_intscale(wl.x, wl.w, alpha=alpha, out="f32")
+        assert moe["alpha"] == dense["alpha"]
+        assert np.array_equal(moe["acc"], dense["acc"])
+        assert np.array_equal(moe["y"], dense["y"])
+
+
+def test_moe_identical_experts_repeat_the_dense_rows():
+    """All experts equal: both routed rows of a token equal its dense row."""
+    wl = workloads.make_linear(20, 256, 64, x_dtype="bf16", seed=12)
+    route = np.array([[t % 3, (t + 1) % 3] for t in range(20)], np.int64)
+    ri, off = workloads.route_rows(route, 3)
+    moe = oracle.moe_intscale(wl.x, [wl.w] * 3, ri, off, alpha=1024, out="f32")
+    dense = oracle.linear_intscale(wl.x, wl.w, alpha=1024, out="f32")
+    assert np.array_equal(moe["acc"], dense["acc"][ri.astype(np.int64)])
+
+
+def test_moe_shared_amplifier_postcondition():
+    """One amplifier for the layer: the smallest power of two that lifts every
+    positive group scale of every expert to at least 1."""
+    wl = workloads.make_moe(8, 256, 32, 4, seed=5)
+    wl.w[2] *= np.float32(0.05)  # one expert with much smaller scales sets the amplifier
+    ri, off = workloads.route_rows(wl.experts, 4)
+    moe = oracle.moe_intscale(wl.x, wl.w, ri, off, alpha=None)
+    a = moe["alpha"]
+    allpos = np.concatenate([sg[sg > 0].reshape(-1) for sg in moe["s_g"]]).astype(np.float64)
+    assert (allpos * a >= 1.0).all()
+    assert a == 1 or (allpos * (a // 2) < 1.0).any()
+    assert a >= max(oracle.amplifier_search(sg) for sg in moe["s_g"])
+
+
+def test_moe_rows_follow_their_token_and_expert():
+    """Permuting the tokens moves rows, not values: the row of (token, expert)
+    is a function of that pair only."""
+    wl = workloads.make_moe(12, 256, 40, 3, seed=6)
+    ri, off = workloads.route_rows(wl.experts, 3)
+    base = oracle.moe_intscale(wl.x, wl.w, ri, off, alpha=1024)
+    perm = np.random.default_rng(0).permutation(12)
+    ri2, off2 = workloads.route_rows(wl.experts[perm], 3)
+    other = oracle.moe_intscale(wl.x[perm], wl.w, ri2, off2, alpha=1024)
+    assert np.array_equal(off, off2)
+    for e in range(3):
+        a = {int(t): base["acc"][i] for t, i in zip(ri[off[e]:off[e + 1]], range(off[e], off[e + 1]))}
+        for i in range(off2[e], off2[e + 1]):
+            assert np.array_equal(other["acc"][i], a[int(perm[ri2[i]])])
