@@ -9,12 +9,15 @@ from ._native import (  # noqa: F401
     device_status,
     gemm_workspace,
     load,
+    moe_workspace,
+    pack_moe_experts,
     pack_w4_groupwise,
     quantize_act_per_token,
     w4a8_amplifier_search,
     w4a8_gemm_floatscale,
     w4a8_gemm_intscale,
     w4a8_gemm_intscale_static_ws,
+    w4a8_moe_gemm_intscale,
 )
 
 __all__ = [
@@ -22,10 +25,13 @@ __all__ = [
     "device_status",
     "gemm_workspace",
     "load",
+    "moe_workspace",
+    "pack_moe_experts",
     "pack_w4_groupwise",
     "quantize_act_per_token",
     "w4a8_amplifier_search",
     "w4a8_gemm_floatscale",
     "w4a8_gemm_intscale",
     "w4a8_gemm_intscale_static_ws",
+    "w4a8_moe_gemm_intscale",
 ]

@@ -12,6 +12,7 @@ import os
 import re
 import threading
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -75,6 +76,9 @@ def load(path: str = LIB_PATH):
             "w4a8_gemm_intscale_static_ws": ([P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P], I32_),
             "w4a8_gemm_floatscale": ([P, P, P, P, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
             "w4a8_device_status": ([P, I32_], I32_),
+            "w4a8_moe_workspace_size": ([I32_, P, I64, I64, I32_], I64),
+            "w4a8_moe_gemm_intscale": ([P, P, I64, P, P, P, P, I32_, I32_, I64, I64, I32_, P, I32_, P, I64, P],
+                                       I32_),
             "w4a8_last_cuda_error": ([I32_], I32_),
             "w4a8_cuda_error_string": ([I32_], ctypes.c_char_p),
         }
@@ -267,6 +271,62 @@ def w4a8_gemm_floatscale(q_x, s_a, w_packed, s_g, *, group: int = 128, out: str 
     code = load().w4a8_gemm_floatscale(_ptr(q_x), _ptr(s_a), _ptr(w_packed), _ptr(s_g), M, N, K, group, _ptr(y),
                                        dt, _ptr(workspace), ws_bytes, _stream(q_x.device))
     _check("w4a8_gemm_floatscale", code)
+    return y
+
+
+def pack_moe_experts(ws, group: int = 128, alpha: int | None = None):
+    """Pack every expert's fp32 weights [K, N] with one amplifier for the layer:
+    the search over all experts' group scales (alpha=None) or the given one.
+
+    Returns dict(packed=[...], S=[...], s_g=[...], alpha)."""
+    if alpha is None:
+        sgs = [pack_w4_groupwise(w, group=group, scales_only=True)["s_g"] for w in ws]
+        alpha = w4a8_amplifier_search(torch.cat([s.reshape(-1) for s in sgs]))
+    pks = [pack_w4_groupwise(w, group=group, alpha=alpha) for w in ws]
+    return dict(packed=[p["packed"] for p in pks], S=[p["S"] for p in pks], s_g=[p["s_g"] for p in pks],
+                alpha=int(alpha))
+
+
+def moe_workspace(offsets, N: int, K: int, group: int, device) -> torch.Tensor:
+    """A zero-filled workspace for w4a8_moe_gemm_intscale with these row offsets."""
+    off = np.ascontiguousarray(np.asarray(offsets, np.int64))
+    with torch.cuda.device(device):
+        need = load().w4a8_moe_workspace_size(len(off) - 1, off.ctypes.data_as(ctypes.c_void_p), N, K, group)
+    if need < 0:
+        raise W4A8Error("w4a8_moe_workspace_size", 1, " (invalid offsets or shape)")
+    return torch.zeros(max(int(need), 16), dtype=torch.uint8, device=device)
+
+
+def w4a8_moe_gemm_intscale(q_x, s_a, row_index, offsets, packed, S, alpha: int, *, group: int = 128,
+                           out: str = "f16", y: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None, N: int | None = None):
+    """y [R, N]: expert e's integer-scale GEMM over its routed rows
+    row_index[offsets[e]:offsets[e+1]] (offsets: host, E+1 values).  N is taken
+    from the packed weights unless given (needed when every expert is empty)."""
+    _need_cuda("q_x", q_x, torch.int8, 2)
+    _need_cuda("s_a", s_a, torch.float32, 1)
+    _need_cuda("row_index", row_index, torch.int32, 1)
+    off = np.ascontiguousarray(np.asarray(offsets, np.int64))
+    E = len(off) - 1
+    if len(packed) != E or len(S) != E:
+        raise ValueError("one packed weight and one integer-scale tensor per expert")
+    T, K = q_x.shape
+    if N is None:
+        N = int(next((p.shape[0] for p in packed if p is not None), 0))
+    R = int(off[-1])
+    dt, tdt = _OUT[out]
+    if y is None:
+        y = torch.empty((R, N), dtype=tdt, device=q_x.device)
+    _need_cuda("y", y, tdt, 2)
+    if workspace is None:
+        workspace = moe_workspace(off, N, K, group, q_x.device)
+    wp = (ctypes.c_void_p * E)(*[p.data_ptr() if p is not None else 0 for p in packed])
+    sp = (ctypes.c_void_p * E)(*[s.data_ptr() if s is not None else 0 for s in S])
+    code = load().w4a8_moe_gemm_intscale(_ptr(q_x), _ptr(s_a), T, _ptr(row_index),
+                                         off.ctypes.data_as(ctypes.c_void_p), ctypes.cast(wp, ctypes.c_void_p),
+                                         ctypes.cast(sp, ctypes.c_void_p), int(alpha), E, N, K, group, _ptr(y), dt,
+                                         _ptr(workspace), workspace.numel(), _stream(q_x.device))
+    _check("w4a8_moe_gemm_intscale", code)
     return y
 
 

@@ -213,6 +213,43 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     return W4A8_OK;
 }
 
+// Layout of the mixture-of-experts workspace for host row offsets off[0..E]:
+// [GEMM workspace (counters first)] [gathered codes R x K] [gathered scales,
+// each expert's 16-byte aligned], every part 256-byte aligned.
+struct MoeLayout {
+    int64_t R = 0, max_rows = 0;
+    int64_t gemm_bytes = 0, x_off = 0, s_off = 0, total = 0;
+    int32_t sbase[w4a8::moe::kMaxExperts] = {};
+};
+
+int64_t align256(int64_t v) { return (v + 255) & ~int64_t(255); }
+
+w4a8_status moe_layout(int32_t E, const int64_t* off, int64_t N, int64_t K, int32_t group, const DeviceInfo& dev,
+                       MoeLayout& L) {
+    if (E < 1 || E > w4a8::moe::kMaxExperts || !off) return W4A8_ERR_INVALID_ARG;
+    if (off[0] != 0) return W4A8_ERR_INVALID_ARG;
+    int64_t sfloats = 0;
+    for (int32_t e = 0; e < E; ++e) {
+        const int64_t m = off[e + 1] - off[e];
+        if (m < 0) return W4A8_ERR_INVALID_ARG;
+        L.sbase[e] = int32_t(sfloats);
+        sfloats += (m + 3) & ~int64_t(3);
+        if (m > L.max_rows) L.max_rows = m;
+        if (m > 0) {
+            const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(m, N, K, group, dev.sms);
+            if (pl.W >= (int64_t(1) << 31)) return W4A8_ERR_SHAPE;
+            const int64_t need = plan_splits_tiles(pl) ? pl.ws_bytes : 0;
+            if (need > L.gemm_bytes) L.gemm_bytes = need;
+        }
+    }
+    L.R = off[E];
+    if (L.R > INT32_MAX || sfloats > INT32_MAX) return W4A8_ERR_SHAPE;
+    L.x_off = align256(L.gemm_bytes);
+    L.s_off = L.x_off + align256(L.R * K);
+    L.total = L.s_off + align256(sfloats * 4);
+    return W4A8_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -339,6 +376,70 @@ w4a8_status w4a8_gemm_intscale_static_ws(const int8_t* q_x, const float* s_a, co
     if (sw != W4A8_OK) return sw;
     return run_gemm(w4a8::gemm::kIntScale, q_x, s_a, w_packed, S, nullptr, alpha, M, N, K, group, y, y_dtype, ws,
                     int64_t(W4A8_STATIC_WORKSPACE_BYTES), stream);
+}
+
+int64_t w4a8_moe_workspace_size(int32_t E, const int64_t* expert_offsets_host, int64_t N, int64_t K,
+                                int32_t group) {
+    if (check_gemm_shape(1, N, K, group) != W4A8_OK) return -1;
+    DeviceInfo dev;
+    if (current_device(dev) != W4A8_OK) return -1;
+    MoeLayout L;
+    if (moe_layout(E, expert_offsets_host, N, K, group, dev, L) != W4A8_OK) return -1;
+    return L.total;
+}
+
+w4a8_status w4a8_moe_gemm_intscale(const int8_t* q_x, const float* s_a, int64_t T, const int32_t* row_index,
+                                   const int64_t* expert_offsets_host, const uint8_t* const* w_packed_host,
+                                   const int16_t* const* S_host, int32_t alpha, int32_t E, int64_t N, int64_t K,
+                                   int32_t group, void* y, int32_t y_dtype, void* workspace,
+                                   int64_t workspace_bytes, void* stream) {
+    w4a8_status st = check_gemm_shape(1, N, K, group);
+    if (st != W4A8_OK) return st;
+    if (T < 0 || T > INT32_MAX) return W4A8_ERR_SHAPE;
+    if (y_dtype != W4A8_F16 && y_dtype != W4A8_F32 && y_dtype != W4A8_I32) return W4A8_ERR_DTYPE;
+    if (!is_pow2(alpha) || alpha > (1 << 30)) return W4A8_ERR_INVALID_ARG;
+    if (!expert_offsets_host || !w_packed_host || !S_host) return W4A8_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if ((st = current_device(dev)) != W4A8_OK) return st;
+    MoeLayout L;
+    if ((st = moe_layout(E, expert_offsets_host, N, K, group, dev, L)) != W4A8_OK) return st;
+    if (L.R == 0) return W4A8_OK;
+    if (!q_x || !s_a || !row_index || !y || T == 0) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(q_x) || !aligned16(y) || !aligned16(s_a) || !aligned16(row_index)) return W4A8_ERR_ALIGN;
+    for (int32_t e = 0; e < E; ++e) {
+        if (expert_offsets_host[e + 1] == expert_offsets_host[e]) continue;
+        if (!w_packed_host[e] || !S_host[e]) return W4A8_ERR_INVALID_ARG;
+        if (!aligned16(w_packed_host[e]) || !aligned16(S_host[e])) return W4A8_ERR_ALIGN;
+    }
+    if (!workspace || workspace_bytes < L.total) return W4A8_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return W4A8_ERR_ALIGN;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+    w4a8::moe::GatherParams gp{};
+    gp.q_x = q_x;
+    gp.s_a = s_a;
+    gp.T = T;
+    gp.K = K;
+    gp.row_index = row_index;
+    gp.xg = reinterpret_cast<int8_t*>(ws + L.x_off);
+    gp.sg = reinterpret_cast<float*>(ws + L.s_off);
+    gp.status = dev.status;
+    gp.E = E;
+    for (int32_t e = 0; e <= E; ++e) gp.off[e] = int32_t(expert_offsets_host[e]);
+    for (int32_t e = 0; e < E; ++e) gp.sbase[e] = L.sbase[e];
+    W4A8_CUDA_TRY(w4a8::moe::gather(gp, int(L.max_rows), cs));
+
+    const int64_t ysz = y_dtype == W4A8_F16 ? 2 : 4;
+    for (int32_t e = 0; e < E; ++e) {
+        const int64_t lo = expert_offsets_host[e], m = expert_offsets_host[e + 1] - lo;
+        if (m == 0) continue;
+        st = run_gemm(w4a8::gemm::kIntScale, gp.xg + lo * K, gp.sg + L.sbase[e], w_packed_host[e], S_host[e],
+                      nullptr, alpha, m, N, K, group, static_cast<uint8_t*>(y) + lo * N * ysz, y_dtype,
+                      L.gemm_bytes ? ws : nullptr, L.gemm_bytes, stream);
+        if (st != W4A8_OK) return st;
+    }
+    return W4A8_OK;
 }
 
 w4a8_status w4a8_gemm_floatscale(const int8_t* q_x, const float* s_a, const uint8_t* w_packed, const float* s_g,

@@ -192,6 +192,45 @@ W4A8_API w4a8_status w4a8_gemm_intscale_static_ws(const int8_t* q_x, const float
                                                  int32_t group, void* y, int32_t y_dtype, void* stream);
 
 /*
+ * Mixture-of-experts layer: one integer-scale W4A8 GEMM per expert over the
+ * rows routed to it.  (Integer Scale summary §5.3: the method applied to
+ * Mixtral 8x7B; every expert's linear layer is a fine-grained W4A8 GEMM and
+ * the amplifier is one per layer, shared by all experts.)
+ *   for every routed row i of expert e (offsets[e] <= i < offsets[e+1]):
+ *     y[i, :] = w4a8_gemm_intscale row of token row_index[i] with expert e's
+ *               w_packed[e], S[e] and the shared alpha
+ * q_x, s_a   device, [T, K] int8 and [T] float32: every token quantized once
+ *            (quantize_act_per_token); T >= 1 when any row is routed
+ * row_index  device, [R] int32: the token of each routed row, rows grouped by
+ *            expert (expert 0 first); a token index outside [0, T) makes that
+ *            row's output zero and sets the device status word to
+ *            W4A8_ERR_INVALID_ARG (read with w4a8_device_status)
+ * expert_offsets_host  HOST, [E+1] int64: offsets[0] = 0, non-decreasing,
+ *            R = offsets[E] < 2^31; they size the per-expert launches
+ * w_packed_host, S_host  HOST arrays of E device pointers: expert e's packed
+ *            weights [N, K/2] and integer scales [K/group, N], all packed with
+ *            the same alpha (pack each expert's s_g with S = NULL, run
+ *            w4a8_amplifier_search over all of them, pack every expert with it);
+ *            pointers of experts with no rows may be NULL
+ * 1 <= E <= 256; N, K, group as for w4a8_gemm_intscale
+ * y          device, [R, N] of y_dtype (W4A8_F16, W4A8_F32, W4A8_I32)
+ * workspace  device, >= w4a8_moe_workspace_size(E, offsets, N, K, group) bytes,
+ *            zero-filled before its first use; its first 4096 bytes are
+ *            counters that every completed call leaves at zero, the rest holds
+ *            the gathered rows and partial sums
+ * Launches a gather kernel and one GEMM per expert with rows, asynchronously
+ * on `stream`.
+ */
+W4A8_API int64_t w4a8_moe_workspace_size(int32_t E, const int64_t* expert_offsets_host, int64_t N, int64_t K,
+                                         int32_t group);
+W4A8_API w4a8_status w4a8_moe_gemm_intscale(const int8_t* q_x, const float* s_a, int64_t T,
+                                           const int32_t* row_index, const int64_t* expert_offsets_host,
+                                           const uint8_t* const* w_packed_host, const int16_t* const* S_host,
+                                           int32_t alpha, int32_t E, int64_t N, int64_t K, int32_t group,
+                                           void* y, int32_t y_dtype, void* workspace, int64_t workspace_bytes,
+                                           void* stream);
+
+/*
  * W4A8 GEMM with float group scales, the comparison path.
  * (Integer Scale summary §3.2 / Fig. 3(b): every group's int32 result is
  *  converted to fp32 and multiplied by its float scale.)
@@ -214,7 +253,9 @@ W4A8_API const char* w4a8_cuda_error_string(int32_t code);
 
 /*
  * Reads (and with clear != 0 resets) the device status word of the current
- * device that bounded waits write on a timeout.  Synchronous.  0 = no timeout.
+ * device: 0, or the last device-side error: W4A8_ERR_TIMEOUT (a bounded wait
+ * ran out) or W4A8_ERR_INVALID_ARG (a routed row's token index out of range in
+ * w4a8_moe_gemm_intscale).  Synchronous.
  */
 W4A8_API w4a8_status w4a8_device_status(int32_t* code_host, int32_t clear);
 

@@ -1,0 +1,109 @@
+"""Mixture-of-experts path on the GPU against the oracle: routed-row gather and
+one integer-scale GEMM per expert with a shared amplifier (the Integer Scale
+summary's Mixtral results)."""
+import numpy as np
+import pytest
+import torch
+
+import bit_gemm_quantize_b200 as bgq
+import oracle
+from bit_gemm_quantize_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def _close(y, y_ref, out):
+    ref = np.asarray(y_ref, np.float64)
+    tau = 1e-2 * np.sqrt(np.mean(ref * ref)) if ref.size else 0.0
+    rtol = 1e-3 if out == "f32" else 4e-3
+    err = np.abs(np.asarray(y, np.float64) - ref)
+    assert np.all(err <= rtol * np.maximum(np.abs(ref), tau))
+
+
+def _run(wl, E, alpha, out="i32", route=None):
+    dev = torch.device("cuda:0")
+    route = wl.experts if route is None else route
+    ri, off = workloads.route_rows(route, E)
+    x = torch.from_numpy(wl.x).to(dev).to(torch.bfloat16)
+    q, s = bgq.quantize_act_per_token(x)
+    pk = bgq.pack_moe_experts([torch.from_numpy(w).to(dev) for w in wl.w], alpha=alpha)
+    y = bgq.w4a8_moe_gemm_intscale(q, s, torch.from_numpy(ri).to(dev), off, pk["packed"], pk["S"], pk["alpha"],
+                                   out=out)
+    torch.cuda.synchronize()
+    return ri, off, pk, y
+
+
+@pytest.mark.parametrize("T,K,N,E,topk", [(64, 512, 256, 4, 2), (37, 256, 136, 8, 2), (200, 1024, 520, 3, 1)])
+@pytest.mark.parametrize("alpha", [1024, None])
+def test_moe_parity(T, K, N, E, topk, alpha):
+    wl = workloads.make_moe(T, K, N, E, topk=topk, seed=T + E)
+    ri, off, pk, acc = _run(wl, E, alpha, "i32")
+    ref = oracle.moe_intscale(wl.x, wl.w, ri, off, alpha=alpha, out="f32")
+    assert pk["alpha"] == ref["alpha"]
+    for e in range(E):
+        assert np.array_equal(pk["packed"][e].cpu().numpy(), ref["packed"][e])
+        assert np.array_equal(pk["S"][e].cpu().numpy(), ref["S"][e])
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+    for out in ("f32", "f16"):
+        _, _, _, y = _run(wl, E, alpha, out)
+        _close(y.float().cpu().numpy(), ref["y64"], out)
+    assert bgq.device_status() == 0
+
+
+def test_moe_empty_experts_and_single_expert():
+    wl = workloads.make_moe(48, 512, 256, 5, topk=1, seed=9)
+    route = np.full((48, 1), 3, np.int64)  # every token to expert 3, experts 0, 1, 2, 4 empty
+    ri, off, pk, acc = _run(wl, 5, 1024, "i32", route)
+    ref = oracle.moe_intscale(wl.x, wl.w, ri, off, alpha=1024)
+    assert list(np.diff(off)) == [0, 0, 0, 48, 0]
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+    # no routed rows at all: nothing to do
+    dev = torch.device("cuda:0")
+    q = torch.zeros((4, 512), dtype=torch.int8, device=dev)
+    s = torch.ones((4,), dtype=torch.float32, device=dev)
+    y = bgq.w4a8_moe_gemm_intscale(q, s, torch.zeros((0,), dtype=torch.int32, device=dev), [0, 0, 0],
+                                   [None, None], [None, None], 1024, N=256)
+    assert y.shape == (0, 256)
+
+
+def test_moe_out_of_range_token_index_is_reported():
+    """A routed row naming a token outside [0, T) is written as zeros and the
+    device status word reports W4A8_ERR_INVALID_ARG (1); the other rows are right."""
+    dev = torch.device("cuda:0")
+    wl = workloads.make_moe(16, 256, 128, 2, topk=1, seed=4)
+    ri, off = workloads.route_rows(wl.experts, 2)
+    ri_bad = ri.copy()
+    ri_bad[0] = 1000
+    x = torch.from_numpy(wl.x).to(dev).to(torch.bfloat16)
+    q, s = bgq.quantize_act_per_token(x)
+    pk = bgq.pack_moe_experts([torch.from_numpy(w).to(dev) for w in wl.w], alpha=1024)
+    bgq.device_status(clear=True)
+    acc = bgq.w4a8_moe_gemm_intscale(q, s, torch.from_numpy(ri_bad).to(dev), off, pk["packed"], pk["S"], 1024,
+                                     out="i32")
+    torch.cuda.synchronize()
+    assert bgq.device_status(clear=True) == 1
+    ref = oracle.moe_intscale(wl.x, wl.w, ri, off, alpha=1024)
+    a = acc.cpu().numpy().astype(np.int64)
+    assert np.all(a[0] == 0)
+    assert np.array_equal(a[1:], ref["acc"][1:])
+
+
+def test_moe_mixtral_shaped_sampled():
+    """A Mixtral-shaped layer slice (K = 4096, 8 experts, top-2, 256 tokens,
+    N = 2048): raw accumulators at sampled (row, column) positions."""
+    T, K, N, E = 256, 4096, 2048, 8
+    wl = workloads.make_moe(T, K, N, E, topk=2, seed=21)
+    ri, off, pk, acc = _run(wl, E, None, "i32")
+    qx, s_a = oracle.quantize_act_per_token(wl.x)
+    rng = np.random.default_rng(5)
+    a = acc.cpu().numpy().astype(np.int64)
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        qw, sg = oracle.quantize_groups(wl.w[e], 128)
+        S = oracle.integer_scales(sg, pk["alpha"])
+        ms = rng.integers(0, hi - lo, 40)
+        ns = rng.integers(0, N, 40)
+        want = oracle.intscale_acc_at(qx[ri[lo:hi].astype(np.int64)], qw, S, ms, ns)
+        assert np.array_equal(a[lo + ms, ns], want)
