@@ -174,7 +174,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
         ws_part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + pl.count_bytes);
     }
 
-    CUtensorMap tm_w, tm_x, tm_s;
+    CUtensorMap tm_w, tm_x, tm_y;
     // packed weights: one box = 128 columns x 128 bytes (two 128-wide K blocks), 128-byte swizzle
     if (!make_map_u8(&tm_w, w_packed, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2),
                      uint32_t(w4a8::gemm::weight_box_bytes()), 128, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -182,12 +182,16 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(M), uint64_t(K), 128, uint32_t(pl.BT),
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return W4A8_ERR_CUDA;
-    // group scales [G][N]: one box = 128 columns x 2 groups (rows past G read as zero)
-    const bool is = (path == w4a8::gemm::kIntScale);
-    if (!make_map_2d(&tm_s, is ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                     is ? static_cast<const void*>(S) : static_cast<const void*>(s_g), uint64_t(N), uint64_t(pl.G),
-                     uint64_t(N) * (is ? 2u : 4u), 128, 2, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return W4A8_ERR_CUDA;
+    // output: one box = 128 columns x BT rows, stored from the CTA's staging tile
+    {
+        const bool f16 = (y_dtype == W4A8_F16);
+        const CUtensorMapDataType t = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                          : (y_dtype == W4A8_I32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                                                 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+        if (!make_map_2d(&tm_y, t, y, uint64_t(N), uint64_t(M), uint64_t(N) * (f16 ? 2u : 4u), 128,
+                         uint32_t(pl.BT), CU_TENSOR_MAP_SWIZZLE_NONE))
+            return W4A8_ERR_CUDA;
+    }
 
     w4a8::gemm::Params p{};
     p.s_a = s_a;
@@ -209,7 +213,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     p.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
     p.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
                                     : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
-    W4A8_CUDA_TRY(w4a8::gemm::launch(tm_w, tm_x, tm_s, p, pl.BT, path, static_cast<cudaStream_t>(stream)));
+    W4A8_CUDA_TRY(w4a8::gemm::launch(tm_w, tm_x, tm_y, p, pl.BT, path, static_cast<cudaStream_t>(stream)));
     return W4A8_OK;
 }
 

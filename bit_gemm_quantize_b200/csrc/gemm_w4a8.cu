@@ -83,6 +83,10 @@ constexpr int64_t kMaxGrid = kCounterBytes / 4;
 #define W4A8_PREFETCH(SW) ((SW) < 2 ? (SW) : 2)
 #endif
 
+#ifndef W4A8_GROUP_COMMIT_MIN_BT
+#define W4A8_GROUP_COMMIT_MIN_BT 64
+#endif
+
 // Ring depths (stages) of the packed weights and the token codes.
 #ifndef W4A8_SW
 #define W4A8_SW(BT) ((BT) <= 32 ? 8 : ((BT) == 64 ? 6 : 4))
@@ -119,22 +123,29 @@ struct Cfg {
     static constexpr bool kX16 = (PATH == kFloatScale) || BT <= W4A8_X16_IS_MAX_BT;
     static constexpr int kWBytes = kTileN * kStageK / 2;  // packed weights per stage: 16 KB
     static constexpr int kXBytes = BT * kStageK;          // token codes per stage
+    // Wide token tiles commit every group to its accumulator buffer, so the
+    // epilogue drains a group while the MMAs of the next one run; narrow tiles
+    // commit once per stage (their drains are short, the extra commits are not).
+    static constexpr bool kGroupCommit = BT >= W4A8_GROUP_COMMIT_MIN_BT;
     static constexpr int kSW = W4A8_SW(BT);
     static constexpr int kSX = W4A8_SX(BT);
     // stage-done ring: one tcgen05.commit per stage, read by every role that
-    // recycles a resource of that stage; the group scales of a stage travel in
-    // a slot of this ring too (TMA box: 2 groups x 128 columns)
+    // recycles a resource of that stage
     static constexpr int kSD = 16;
     static_assert(kSD >= kSX && kSD >= kSA, "stage-done ring shallower than a ring it releases");
-    static constexpr int kSBytes = 2 * kTileN * (PATH == kIntScale ? 2 : 4);
+    // output staging tile [BT tokens][128 columns] (elements of at most 4
+    // bytes) and the tile's output scales, for the TMA store of the tail
+    static constexpr int kYBytes = BT * kTileN * 4;
     static constexpr int offW = 0;
     static constexpr int offX = offW + kSW * kWBytes;
-    static constexpr int offS = offX + kSX * kXBytes;
-    static constexpr int offBar = offS + kSD * kSBytes;
-    static constexpr int kBars = 2 * kSW + kSX + kSA + 3 * kSD + kAcc + 1;
+    static constexpr int offY = offX + kSX * kXBytes;
+    static constexpr int offSA = offY + kYBytes;
+    static constexpr int offBar = offSA + BT * 4;
+    static constexpr int kBars = 2 * kSW + kSX + kSA + 2 * kSD + 2 * kAcc + 1;
     static constexpr int offMisc = offBar + kBars * 8;
     static constexpr int kSmemBytes = offMisc + 64 + 1024;  // + slack to align the base to 1024
     static_assert(kXBytes % 2048 == 0, "token stage must hold whole 8-row swizzle atoms per k-block");
+    static_assert(offY % 128 == 0, "TMA store source alignment");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -305,25 +316,6 @@ __device__ __forceinline__ float output_scale(const Params& p, int64_t m) {
     return PATH == kIntScale ? __fmul_rn(p.s_a[m], p.inv_alpha) : p.s_a[m];
 }
 
-template <int PATH>
-__device__ __forceinline__ void store_output(const Params& p, int64_t m, int64_t n, float vf, int32_t vi,
-                                             float scale) {
-    const int64_t idx = m * p.N + n;
-    if (PATH == kIntScale) {
-        if (p.y_dtype == kOutI32) {
-            static_cast<int32_t*>(p.y)[idx] = vi;
-            return;
-        }
-        vf = __fmul_rn(__int2float_rn(vi), scale);
-    } else {
-        vf = __fmul_rn(vf, scale);
-    }
-    if (p.y_dtype == kOutF16)
-        static_cast<__half*>(p.y)[idx] = __float2half_rn(vf);
-    else
-        static_cast<float*>(p.y)[idx] = vf;
-}
-
 // Acquire load at GPU scope (the arrival counter of a split tile).
 __device__ __forceinline__ int ld_acquire_gpu(const int* addr) {
     int v;
@@ -345,7 +337,7 @@ struct Ring {
 template <int BT, int PATH>
 __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-                     const __grid_constant__ CUtensorMap tm_s, const Params p) {
+                     const __grid_constant__ CUtensorMap tm_y, const Params p) {
     using C = Cfg<BT, PATH>;
     constexpr int kAcc = C::kAcc;
     constexpr int kU = C::kUnpackWarps;
@@ -360,10 +352,10 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
     uint64_t* full_x = empty_w + SW;      // token codes landed
     uint64_t* full_a = full_x + SX;       // unpacked operand written to its TMEM slot
     uint64_t* sdone = full_a + SA;        // all MMAs of a stage complete (one commit per stage)
-    uint64_t* sfree = sdone + SD;         // epilogue has seen a stage-done phase (slot may be committed again)
-    uint64_t* full_s = sfree + SD;        // a stage's group scales landed
-    uint64_t* tempty = full_s + SD;       // epilogue has read a TMEM accumulator buffer
-    uint64_t* mma_done = tempty + kAcc;
+    uint64_t* sseen = sdone + SD;         // per-stage commits: the epilogue has seen a stage-done phase
+    uint64_t* tempty = sseen + SD;        // epilogue has read a TMEM accumulator buffer
+    uint64_t* afull = tempty + kAcc;      // a group's MMAs into an accumulator buffer are complete
+    uint64_t* mma_done = afull + kAcc;
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::offMisc);  // [0] tmem base [1] abort [2] last
     volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
@@ -379,17 +371,19 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
         for (int s = 0; s < SA; ++s) mbar_init(&full_a[s], kU);
         for (int s = 0; s < SD; ++s) {
             mbar_init(&sdone[s], 1);
-            mbar_init(&sfree[s], kEpiWarps);
-            mbar_init(&full_s[s], 1);
+            mbar_init(&sseen[s], kEpiWarps);
         }
-        for (int s = 0; s < kAcc; ++s) mbar_init(&tempty[s], kEpiWarps);
+        for (int s = 0; s < kAcc; ++s) {
+            mbar_init(&tempty[s], kEpiWarps);
+            mbar_init(&afull[s], 1);
+        }
         mbar_init(&mma_done[0], 1);
         misc[1] = 0;
         misc[2] = 0;
         fence_mbar_init();
         prefetch_tensormap(&tm_w);
         prefetch_tensormap(&tm_x);
-        prefetch_tensormap(&tm_s);
+        prefetch_tensormap(&tm_y);
     }
     if (warp == 1) tmem_alloc(&misc[0], C::kTmemCols);
     tc_fence_before();
@@ -412,10 +406,8 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
         // kernel may still be writing, can be read.
         Ring rw, rx;
         Ring rxd;          // stage-done slot of the stage whose token slot is reused (SX stages back)
-        Ring rs;           // scale slot (same index as the stage-done ring)
         int32_t pst = 0;   // stages issued so far
         uint32_t w_issued = 0u, w_par = 0u, x_issued = 0u, x_par = 0u;  // per slot: copy issued / its parity
-        uint32_t s_issued = 0u, s_par = 0u;
         auto issue_w = [&](const Stage& st, const Ring& slot) {
             // one 128 x 128 B box = two K blocks (a lone last block over-reads 64 B per row: harmless)
             mbar_arrive_expect_tx_one(&full_w[slot.idx], C::kWBytes);
@@ -464,16 +456,6 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
             x_issued |= 1u << rx.idx;
             x_par = (x_par & ~(1u << rx.idx)) | (rx.phase << rx.idx);
             rx.advance(SX);
-            // the stage's group scales (rows g, g+1; rows past the last group read as zero)
-            if (!mbar_wait_warp(&sfree[rs.idx], rs.phase ^ 1u, abort_flag, p.status)) {
-                ok = false;
-                break;
-            }
-            mbar_arrive_expect_tx_one(&full_s[rs.idx], C::kSBytes);
-            tma_load_2d_one(smem + C::offS + rs.idx * C::kSBytes, &tm_s, st.n_tile * kTileN, st.g, &full_s[rs.idx]);
-            s_issued |= 1u << rs.idx;
-            s_par = (s_par & ~(1u << rs.idx)) | (rs.phase << rs.idx);
-            rs.advance(SD);
             ++pst;
         }
         if (!ok && lane == 0) {  // let copies in flight land before the CTA leaves
@@ -481,20 +463,17 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 if (w_issued & (1u << s)) drain_wait(&full_w[s], (w_par >> s) & 1u);
             for (int s = 0; s < SX; ++s)
                 if (x_issued & (1u << s)) drain_wait(&full_x[s], (x_par >> s) & 1u);
-            for (int s = 0; s < SD; ++s)
-                if (s_issued & (1u << s)) drain_wait(&full_s[s], (s_par >> s) & 1u);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        // One converged warp; each MMA and the per-stage commit are issued by
-        // one elected lane.  Per stage: wait for the unpacked operand (TMEM
-        // slot) and the token codes, issue up to 8 MMAs (4 per K block) into
-        // the accumulator buffer of the current group, and commit once to the
-        // stage-done ring, which frees the operand slot, the token slot and,
-        // for the epilogue, marks the groups that ended in the stage.  Before a
-        // stage-done slot is committed again the epilogue must have seen its
-        // previous phase.
+        // One converged warp; each MMA and commit is issued by one elected
+        // lane.  Per stage: wait for the unpacked operand (TMEM slot) and the
+        // token codes, issue up to 8 MMAs (4 per K block) into the accumulator
+        // buffer of the current group, commit each group that ends to its
+        // buffer's full barrier (the epilogue drains it as soon as its MMAs
+        // are done, while the next group's run), and commit the stage to the
+        // stage-done ring, which frees the operand slot and the token slot.
         constexpr uint32_t idesc = idesc_i8(kTileN, BT);
         Ring rx, ra, rt, rd;
         StageIter it(p, b);
@@ -531,12 +510,19 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 for (int k = 0; k < kBlockK / 32; ++k)  // 32 K per MMA: 8 TMEM columns of A, 2 descriptor units of B
                     mma_i8_tmem_a_one(d, aj + uint32_t(8 * k), smem_desc_from_lo(xj + 2u * k), idesc,
                                       (first && k == 0) ? 0u : 1u);
-                if (last) rt.advance(kAcc);
+                if (last) {
+                    if constexpr (C::kGroupCommit) mma_commit_one(&afull[rt.idx]);
+                    rt.advance(kAcc);
+                }
             }
             if (!ok) break;
-            if (!mbar_wait_warp(&sfree[rd.idx], rd.phase ^ 1u, abort_flag, p.status)) {
-                ok = false;
-                break;
+            if constexpr (!C::kGroupCommit) {
+                // the epilogue waits on stage-done phases: it must have seen the
+                // previous phase of this slot before it is committed again
+                if (!mbar_wait_warp(&sseen[rd.idx], rd.phase ^ 1u, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
             }
             mma_commit_one(&sdone[rd.idx]);
             ra.advance(SA);
@@ -627,11 +613,21 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
         SegmentIter it(p, b);
         Segment sg;
         bool ok = true;
+        const int32_t kbpg = p.kb_per_group;
+        const int32_t G = int32_t(p.G);
         while (ok && it.next(sg)) {
             const int64_t n0 = int64_t(sg.n_tile) * kTileN;
             const int64_t m0 = int64_t(sg.m_tile) * BT + half * HC;
             const int64_t n = n0 + r;
             const bool nvalid = n < p.N;
+            // output scale of token (tile start + this thread's index among the
+            // epilogue threads), handed to the tail through shared memory
+            float sa_pref = 0.0f;
+            {
+                const int te = ew * 32 + lane;
+                const int64_t mt = int64_t(sg.m_tile) * BT + te;
+                if (te < BT && mt < p.M) sa_pref = output_scale<PATH>(p, mt);
+            }
             int32_t acc[HC];
             float accf[HC];
 #pragma unroll
@@ -639,202 +635,255 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 acc[j] = 0;
                 accf[j] = 0.0f;
             }
-            // Walk the segment's stages in the order the MMA warp commits them:
-            // wait for each stage's done phase, tell the MMA warp it was seen,
-            // then drain every group whose last K block was in that stage.
-            int32_t g = sg.g0;  // next group to drain
+            // This column's scales (raw 32 bits) of group g, read straight from
+            // global memory two stages before they are used, so that no wait
+            // or shared-memory round trip sits between two drains.  Rows past
+            // the last group and columns past N read as zero.
+            auto load_scale = [&](int32_t g) -> uint32_t {
+                if (g >= G || !nvalid) return 0u;
+                const int64_t idx = int64_t(g) * p.N + n;
+                if constexpr (PATH == kIntScale)
+                    return uint32_t(int32_t(__ldg(p.S + idx)));
+                else
+                    return __float_as_uint(__ldg(p.s_g + idx));
+            };
+            // the groups ending in a stage are the stage's first group and the next one
+            auto stage_group = [&](int32_t kb_first) -> int32_t {
+                return kbpg == 1 ? kb_first : int32_t(uint32_t(kb_first) / uint32_t(kbpg));
+            };
+            // Walk the segment's stages in the order the MMA warp issues them and
+            // drain every group whose last K block was in that stage, each as
+            // soon as its MMAs are complete, handing its accumulator buffer back
+            // to the MMA warp.
             int32_t kin = 0;    // position of the next K block inside its group
-            int32_t kb = sg.g0 * p.kb_per_group;
-            const int32_t kb_end = sg.g1 * p.kb_per_group;
+            int32_t kb = sg.g0 * kbpg;
+            const int32_t kb_end = sg.g1 * kbpg;
+            uint32_t sc0 = 0u, sc1 = 0u, nx0 = 0u, nx1 = 0u;  // scales of this stage and of the next
+            {
+                const int32_t g0 = stage_group(kb);
+                sc0 = load_scale(g0);
+                sc1 = load_scale(g0 + 1);
+                if (kb + 2 < kb_end) {
+                    const int32_t g1 = stage_group(kb + 2);
+                    nx0 = load_scale(g1);
+                    nx1 = load_scale(g1 + 1);
+                }
+            }
             while (kb < kb_end) {
                 const int32_t nkb = (kb_end - kb) >= 2 ? 2 : 1;
+                const uint32_t s0 = sc0, s1 = sc1;
+                sc0 = nx0;
+                sc1 = nx1;
+                if (kb + 4 < kb_end) {  // the stage after next
+                    const int32_t g2 = stage_group(kb + 4);
+                    nx0 = load_scale(g2);
+                    nx1 = load_scale(g2 + 1);
+                }
                 kb += nkb;
-                if (!mbar_wait_warp(&sdone[rd.idx], rd.phase, abort_flag, p.status) ||
-                    !mbar_wait_warp(&full_s[rd.idx], rd.phase, abort_flag, p.status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                // this column's scales of the stage's groups g and g + 1 (raw 32 bits)
-                uint32_t sc0, sc1;
-                {
-                    const uint8_t* sbuf = smem + C::offS + rd.idx * C::kSBytes;
-                    if (PATH == kIntScale) {
-                        const int16_t* s16 = reinterpret_cast<const int16_t*>(sbuf);
-                        sc0 = uint32_t(int32_t(s16[r]));
-                        sc1 = uint32_t(int32_t(s16[kTileN + r]));
-                    } else {
-                        const uint32_t* s32 = reinterpret_cast<const uint32_t*>(sbuf);
-                        sc0 = s32[r];
-                        sc1 = s32[kTileN + r];
+                if constexpr (!C::kGroupCommit) {
+                    // Per-stage commits: wait for the stage, then tell the MMA
+                    // warp its phase was seen (it waits for that before it
+                    // commits the slot again).
+                    if (!mbar_wait_warp(&sdone[rd.idx], rd.phase, abort_flag, p.status)) {
+                        ok = false;
+                        break;
                     }
+                    tc_fence_after();
+                    __syncwarp();
+                    mbar_arrive_one(&sseen[rd.idx]);
+                    rd.advance(SD);
                 }
-                __syncwarp();
-                mbar_arrive_one(&sfree[rd.idx]);  // the scale slot may be refilled
-                rd.advance(SD);
                 // groups whose last K block is in this stage (at most two)
                 int ng = 0;
                 uint32_t gb0 = 0u, gb1 = 0u;  // their TMEM buffers
+                uint32_t ph0 = 0u, ph1 = 0u;  // and the phases of the buffers' full barriers
                 for (int j = 0; j < nkb; ++j) {
-                    const bool last = (kin == p.kb_per_group - 1);
+                    const bool last = (kin == kbpg - 1);
                     kin = last ? 0 : kin + 1;
                     if (last) {
-                        if (ng == 0)
+                        if (ng == 0) {
                             gb0 = uint32_t(rt.idx);
-                        else
+                            ph0 = rt.phase;
+                        } else {
                             gb1 = uint32_t(rt.idx);
+                            ph1 = rt.phase;
+                        }
                         ++ng;
                         rt.advance(kAcc);
                     }
                 }
                 if (ng == 0) continue;
-                // Segments start on group boundaries and stages cover consecutive K
-                // blocks, so the groups ending in a stage are the stage's first group
-                // (row 0 of the scale box) and possibly the next one (row 1).
-                int taken = 0;
-                auto take_scale = [&]() -> uint32_t { return (taken++ == 0) ? sc0 : sc1; };
-                auto accumulate = [&](const uint32_t* v, int c0, int cnt, uint32_t sraw) {
-                    const int32_t s_cur = int32_t(sraw);
-                    const float f_cur = C::kX16 ? __fmul_rn(__uint_as_float(sraw), 0.0625f)  // P_g was 16 P_g
-                                                : __uint_as_float(sraw);
-#pragma unroll
-                    for (int q = 0; q < cnt; ++q) {
-                        if (PATH == kIntScale) {
-                            const int32_t pg = C::kX16 ? (int32_t(v[q]) >> 4) : int32_t(v[q]);  // exact
-                            acc[c0 + q] += s_cur * pg;
-                        } else {
-                            accf[c0 + q] = __fmaf_rn(f_cur, __int2float_rn(int32_t(v[q])), accf[c0 + q]);
-                        }
-                    }
-                };
                 const uint32_t lane_cols =
                     tmem_base + (uint32_t(quarter * 32) << 16) + C::kAccCol0 + uint32_t(half * HC);
+                auto accumulate = [&](const uint32_t* v, int c0, int cnt, uint32_t sraw) {
+                    if constexpr (PATH == kIntScale) {
+                        const int32_t s_cur = int32_t(sraw);
+#pragma unroll
+                        for (int q = 0; q < cnt; ++q) {
+                            const int32_t pg = C::kX16 ? (int32_t(v[q]) >> 4) : int32_t(v[q]);  // exact
+                            acc[c0 + q] += s_cur * pg;
+                        }
+                    } else {
+                        const float f_cur = C::kX16 ? __fmul_rn(__uint_as_float(sraw), 0.0625f)  // P_g was 16 P_g
+                                                    : __uint_as_float(sraw);
+#pragma unroll
+                        for (int q = 0; q < cnt; ++q)
+                            accf[c0 + q] = __fmaf_rn(f_cur, __int2float_rn(int32_t(v[q])), accf[c0 + q]);
+                    }
+                };
                 if constexpr (HC <= 16) {
                     // small tiles: both groups' loads in flight before one wait
+                    if constexpr (C::kGroupCommit) {
+                        if (!mbar_wait_warp(&afull[gb0], ph0, abort_flag, p.status) ||
+                            (ng == 2 && !mbar_wait_warp(&afull[gb1], ph1, abort_flag, p.status))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
                     uint32_t v0[HC], v1[HC];
                     tmem_load<HC>(lane_cols + gb0 * uint32_t(BT), v0);
                     if (ng == 2) tmem_load<HC>(lane_cols + gb1 * uint32_t(BT), v1);
                     tmem_wait_ld();
-                    accumulate(v0, 0, HC, take_scale());
-                    if (ng == 2) accumulate(v1, 0, HC, take_scale());
+                    accumulate(v0, 0, HC, s0);
+                    if (ng == 2) accumulate(v1, 0, HC, s1);
+                    tc_fence_before();
+                    __syncwarp();
+                    mbar_arrive_one(&tempty[gb0]);
+                    if (ng == 2) mbar_arrive_one(&tempty[gb1]);
                 } else {
+                    // wide tiles: each group's buffer goes back to the MMA warp
+                    // as soon as it is drained
                     constexpr int CH = W4A8_DRAIN_CH < HC ? W4A8_DRAIN_CH : HC;
                     for (int gi = 0; gi < ng; ++gi) {
-                        const uint32_t sraw = take_scale();
+                        const uint32_t gb = gi == 0 ? gb0 : gb1;
+                        if constexpr (C::kGroupCommit) {
+                            if (!mbar_wait_warp(&afull[gb], gi == 0 ? ph0 : ph1, abort_flag, p.status)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                        }
+                        const uint32_t sraw = gi == 0 ? s0 : s1;
 #pragma unroll
                         for (int c0 = 0; c0 < HC; c0 += CH) {
                             uint32_t v[CH];
-                            tmem_load<CH>(lane_cols + (gi == 0 ? gb0 : gb1) * uint32_t(BT) + uint32_t(c0), v);
+                            tmem_load<CH>(lane_cols + gb * uint32_t(BT) + uint32_t(c0), v);
                             tmem_wait_ld();
                             accumulate(v, c0, CH, sraw);
                         }
+                        tc_fence_before();
+                        __syncwarp();
+                        mbar_arrive_one(&tempty[gb]);
                     }
+                    if (!ok) break;
                 }
-                tc_fence_before();
-                __syncwarp();
-                mbar_arrive_one(&tempty[gb0]);
-                if (ng == 2) mbar_arrive_one(&tempty[gb1]);
-                g += ng;
             }
             if (!ok) break;
 
-            // valid token columns of this thread's share; with narrow tiles their
-            // output scales are requested first so that they arrive during the
-            // rest of the tail (wide tiles have no registers to spare for them)
+            // valid token columns of this thread's share (split-tile partials)
             const int nv = p.M - m0 >= HC ? HC : (p.M - m0 > 0 ? int(p.M - m0) : 0);
-            constexpr bool kEarlyScale = HC <= 16;
-            float osc[kEarlyScale ? HC : 1];
-            if constexpr (kEarlyScale) {
-#pragma unroll
-                for (int j = 0; j < HC; ++j) osc[j] = j < nv ? output_scale<PATH>(p, m0 + j) : 0.0f;
-            }
-            auto out_scale = [&](int j) -> float {
-                if constexpr (kEarlyScale)
-                    return osc[j];
-                else
-                    return output_scale<PATH>(p, m0 + j);
-            };
             const bool whole = (sg.g0 == 0 && sg.g1 == p.G);
-            if (whole) {
-                if (nvalid) {
+            if (!whole) {
+                // ---- split tile.  The tile's first contributor b_first covers the
+                // tile's first groups at the end of its own range, so it finishes its
+                // share last: it combines.  Every other contributor stores its partial
+                // (valid columns only, in the slot of its CTA: a CTA contributes a
+                // partial to at most one tile, the one whose last groups open its range)
+                // and signals an arrival counter indexed by b_first (the first
+                // contributor of no other tile).  b_first waits (bounded) for all
+                // arrivals, adds the partials to its own, which never leave registers,
+                // writes y and re-zeroes the counter.
+                const uint32_t t0 = sg.tile * uint32_t(p.G);
+                const uint32_t b_first = range_owner(t0, p);
+                const uint32_t b_last = range_owner(t0 + uint32_t(p.G) - 1u, p);
+                const int64_t slot_elems = int64_t(kTileN) * BT;
+                if (b != b_first) {
+                    int32_t* part = p.ws_part + int64_t(b) * slot_elems + int64_t(half * HC) * kTileN + r;
 #pragma unroll
                     for (int j = 0; j < HC; ++j)
-                        if (j < nv) store_output<PATH>(p, m0 + j, n, accf[j], acc[j], out_scale(j));
-                }
-                continue;
-            }
-            // ---- split tile.  The tile's first contributor b_first covers the
-            // tile's first groups at the end of its own range, so it finishes its
-            // share last: it combines.  Every other contributor stores its partial
-            // (valid columns only, in the slot of its CTA: a CTA contributes a
-            // partial to at most one tile, the one whose last groups open its range)
-            // and signals an arrival counter indexed by b_first (the first
-            // contributor of no other tile).  b_first waits (bounded) for all
-            // arrivals, adds the partials to its own, which never leave registers,
-            // writes y and re-zeroes the counter.
-            const uint32_t t0 = sg.tile * uint32_t(p.G);
-            const uint32_t b_first = range_owner(t0, p);
-            const uint32_t b_last = range_owner(t0 + uint32_t(p.G) - 1u, p);
-            const int64_t slot_elems = int64_t(kTileN) * BT;
-            if (b != b_first) {
-                int32_t* part = p.ws_part + int64_t(b) * slot_elems;
-#pragma unroll
-                for (int j = 0; j < HC; ++j) {
-                    if (j < nv) {
-                        const int64_t e = int64_t(half * HC + j) * kTileN + r;
-                        part[e] = PATH == kIntScale ? acc[j] : __float_as_int(accf[j]);
+                        if (j < nv) part[j * kTileN] = PATH == kIntScale ? acc[j] : __float_as_int(accf[j]);
+                    epi_bar_sync(kEpiWarps * 32);
+                    if (ew == 0 && lane == 0) {
+                        __threadfence();  // the CTA's partial stores (ordered by the barrier) before the arrival
+                        atomicAdd(&p.ws_count[b_first], 1);
                     }
+                    continue;
+                }
+                if (ew == 0 && lane == 0) {
+                    const int expect = int(b_last - b_first);
+                    const long long w0 = clock64();
+                    int ok_wait = 1;
+                    while (ld_acquire_gpu(&p.ws_count[b_first]) < expect) {
+                        if (*abort_flag || clock64() - w0 > kWaitLimitCycles) {
+                            *abort_flag = 1;
+                            atomicExch(p.status, kStatusTimeout);
+                            ok_wait = 0;
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                    misc[2] = uint32_t(ok_wait);
+                    __threadfence();
                 }
                 epi_bar_sync(kEpiWarps * 32);
-                if (ew == 0 && lane == 0) {
-                    __threadfence();  // the CTA's partial stores (ordered by the barrier) before the arrival
-                    atomicAdd(&p.ws_count[b_first], 1);
+                if (!misc[2]) {
+                    ok = false;
+                    break;
                 }
-                continue;
-            }
-            if (ew == 0 && lane == 0) {
-                const int expect = int(b_last - b_first);
-                const long long w0 = clock64();
-                int ok_wait = 1;
-                while (ld_acquire_gpu(&p.ws_count[b_first]) < expect) {
-                    if (*abort_flag || clock64() - w0 > kWaitLimitCycles) {
-                        *abort_flag = 1;
-                        atomicExch(p.status, kStatusTimeout);
-                        ok_wait = 0;
-                        break;
-                    }
-                    __nanosleep(64);
-                }
-                misc[2] = uint32_t(ok_wait);
-                __threadfence();
-            }
-            epi_bar_sync(kEpiWarps * 32);
-            if (!misc[2]) {
-                ok = false;
-                break;
-            }
-            for (uint32_t c = b_first + 1; c <= b_last; ++c) {
-                const int32_t* cp = p.ws_part + int64_t(c) * slot_elems;
+                for (uint32_t c = b_first + 1; c <= b_last; ++c) {
+                    const int32_t* cp = p.ws_part + int64_t(c) * slot_elems + int64_t(half * HC) * kTileN + r;
 #pragma unroll
-                for (int j = 0; j < HC; ++j) {
-                    if (j < nv) {
-                        const int32_t v = __ldcg(cp + int64_t(half * HC + j) * kTileN + r);
-                        if (PATH == kIntScale)
-                            acc[j] += v;
-                        else
-                            accf[j] = __fadd_rn(accf[j], __int_as_float(v));
+                    for (int j = 0; j < HC; ++j) {
+                        if (j < nv) {
+                            const int32_t v = __ldcg(cp + j * kTileN);
+                            if (PATH == kIntScale)
+                                acc[j] += v;
+                            else
+                                accf[j] = __fadd_rn(accf[j], __int_as_float(v));
+                        }
                     }
                 }
+                epi_bar_sync(kEpiWarps * 32);  // every thread has read the partials before the counter is reused
+                if (ew == 0 && lane == 0) p.ws_count[b_first] = 0;
             }
-            if (nvalid) {
-#pragma unroll
-                for (int j = 0; j < HC; ++j)
-                    if (j < nv) store_output<PATH>(p, m0 + j, n, accf[j], acc[j], out_scale(j));
-            }
-            epi_bar_sync(kEpiWarps * 32);  // every thread has read the partials before the counter is reused
-            if (ew == 0 && lane == 0) p.ws_count[b_first] = 0;
+            // ---- the tile's outputs: converted in registers, staged in shared
+            // memory as [BT tokens][128 columns], stored by one TMA tensor store
+            // (which leaves out rows past M and columns past N).
+            const bool leader = (ew == 0 && lane == 0);
+            if (leader) bulk_wait_read_all();  // the previous tile's store has read the staging buffer
             epi_bar_sync(kEpiWarps * 32);
+            float* sa_tile = reinterpret_cast<float*>(smem + C::offSA);
+            if (ew * 32 + lane < BT) sa_tile[ew * 32 + lane] = sa_pref;
+            epi_bar_sync(kEpiWarps * 32);
+            {
+                const int base = half * HC * kTileN + r;  // element index of (token half*HC, column r)
+                const float* sa = sa_tile + half * HC;
+                if (p.y_dtype == kOutI32) {
+                    int32_t* yo = reinterpret_cast<int32_t*>(smem + C::offY) + base;
+#pragma unroll
+                    for (int j = 0; j < HC; ++j) yo[j * kTileN] = acc[j];
+                } else if (p.y_dtype == kOutF16) {
+                    __half* yo = reinterpret_cast<__half*>(smem + C::offY) + base;
+#pragma unroll
+                    for (int j = 0; j < HC; ++j)
+                        yo[j * kTileN] = __float2half_rn(
+                            __fmul_rn(PATH == kIntScale ? __int2float_rn(acc[j]) : accf[j], sa[j]));
+                } else {
+                    float* yo = reinterpret_cast<float*>(smem + C::offY) + base;
+#pragma unroll
+                    for (int j = 0; j < HC; ++j)
+                        yo[j * kTileN] = __fmul_rn(PATH == kIntScale ? __int2float_rn(acc[j]) : accf[j], sa[j]);
+                }
+            }
+            fence_proxy_async_smem();  // the staged outputs, visible to the TMA unit
+            epi_bar_sync(kEpiWarps * 32);
+            if (leader) {
+                tma_store_2d(&tm_y, smem + C::offY, int32_t(n0), sg.m_tile * BT);
+                bulk_commit_group();
+            }
         }
+        if (ew == 0 && lane == 0) bulk_wait_all();  // every output store has completed
     }
 
     tc_fence_before();
@@ -871,7 +920,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms) {
 }
 
 template <int BT, int PATH>
-static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts, const Params& p,
+static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty, const Params& p,
                              cudaStream_t stream) {
     using C = Cfg<BT, PATH>;
     auto kern = w4a8_gemm_kernel<BT, PATH>;
@@ -891,24 +940,24 @@ static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const
         if (dev >= 0 && dev < 64) configured[dev] = true;
     }
     const LaunchPdl lc(unsigned(p.grid), C::kThreads, size_t(smem), stream);
-    return cudaLaunchKernelEx(&lc.cfg, kern, tw, tx, ts, p);
+    return cudaLaunchKernelEx(&lc.cfg, kern, tw, tx, ty, p);
 }
 
-cudaError_t launch(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ts, const Params& p, int BT, int path,
+cudaError_t launch(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty, const Params& p, int BT, int path,
                    cudaStream_t stream) {
     if (path == kIntScale) {
         switch (BT) {
-            case 16: return launch_bt<16, kIntScale>(tw, tx, ts, p, stream);
-            case 32: return launch_bt<32, kIntScale>(tw, tx, ts, p, stream);
-            case 64: return launch_bt<64, kIntScale>(tw, tx, ts, p, stream);
-            default: return launch_bt<128, kIntScale>(tw, tx, ts, p, stream);
+            case 16: return launch_bt<16, kIntScale>(tw, tx, ty, p, stream);
+            case 32: return launch_bt<32, kIntScale>(tw, tx, ty, p, stream);
+            case 64: return launch_bt<64, kIntScale>(tw, tx, ty, p, stream);
+            default: return launch_bt<128, kIntScale>(tw, tx, ty, p, stream);
         }
     }
     switch (BT) {
-        case 16: return launch_bt<16, kFloatScale>(tw, tx, ts, p, stream);
-        case 32: return launch_bt<32, kFloatScale>(tw, tx, ts, p, stream);
-        case 64: return launch_bt<64, kFloatScale>(tw, tx, ts, p, stream);
-        default: return launch_bt<128, kFloatScale>(tw, tx, ts, p, stream);
+        case 16: return launch_bt<16, kFloatScale>(tw, tx, ty, p, stream);
+        case 32: return launch_bt<32, kFloatScale>(tw, tx, ty, p, stream);
+        case 64: return launch_bt<64, kFloatScale>(tw, tx, ty, p, stream);
+        default: return launch_bt<128, kFloatScale>(tw, tx, ty, p, stream);
     }
 }
 

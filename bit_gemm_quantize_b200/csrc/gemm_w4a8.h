@@ -42,8 +42,9 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms);
 
 // tm_w: packed weights [N][K/2] u8, box 128 B x 128 rows, 128-byte swizzle
 // tm_x: token codes [M][K] u8, box 128 B x BT rows, 128-byte swizzle
-// tm_s: group scales [K/group][N] (int16 or fp32), box 128 columns x 2 groups
-cudaError_t launch(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap& tm_s, const Params& p, int BT,
+// tm_y: output y [M][N] (f16, f32 or i32 as Params::y_dtype), box 128 columns x BT rows
+// The group scales are read through Params::S / Params::s_g.
+cudaError_t launch(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap& tm_y, const Params& p, int BT,
                    int path, cudaStream_t stream);
 
 int token_tile_rows();
