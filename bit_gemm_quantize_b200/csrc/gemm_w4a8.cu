@@ -127,6 +127,9 @@ struct Cfg {
     // epilogue drains a group while the MMAs of the next one run; narrow tiles
     // commit once per stage (their drains are short, the extra commits are not).
     static constexpr bool kGroupCommit = BT >= W4A8_GROUP_COMMIT_MIN_BT;
+    // Narrow tiles read a split tile's single other partial when their
+    // segment starts (registers to spare for it).
+    static constexpr bool kEarlyCombine = BT <= 32;
     static constexpr int kSW = W4A8_SW(BT);
     static constexpr int kSX = W4A8_SX(BT);
     // stage-done ring: one tcgen05.commit per stage, read by every role that
@@ -321,6 +324,12 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* addr) {
     int v;
     asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
     return v;
+}
+
+// Release add at GPU scope: the CTA's writes ordered before it (by a CTA
+// barrier) become visible to a thread that acquires the counter.
+__device__ __forceinline__ void red_release_gpu_add(int* addr, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
 }
 
 struct Ring {
@@ -635,6 +644,30 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 acc[j] = 0;
                 accf[j] = 0.0f;
             }
+            // A split tile's first contributor (its segment opens the tile) finishes
+            // its share last; the other contributors did theirs at the start of
+            // their ranges.  With narrow tiles and one other contributor, that
+            // partial is usually complete already: read it now, while this
+            // segment's groups are drained, instead of at the end.
+            int32_t pacc[C::kEarlyCombine ? HC : 1];
+            bool early = false;
+            if constexpr (C::kEarlyCombine) {
+                if (sg.g0 == 0 && sg.g1 < int32_t(p.G)) {
+                    const uint32_t t0 = sg.tile * uint32_t(p.G);
+                    const uint32_t b_last = range_owner(t0 + uint32_t(p.G) - 1u, p);
+                    if (ew == 0 && lane == 0)
+                        misc[3] = (b_last == b + 1 && ld_acquire_gpu(&p.ws_count[b]) >= 1) ? 1u : 0u;
+                    epi_bar_sync(kEpiWarps * 32);
+                    early = misc[3] != 0u;  // the same for every epilogue thread
+                    if (early) {
+                        const int nv = p.M - m0 >= HC ? HC : (p.M - m0 > 0 ? int(p.M - m0) : 0);
+                        const int32_t* cp = p.ws_part + int64_t(b + 1) * (int64_t(kTileN) * BT) +
+                                            int64_t(half * HC) * kTileN + r;
+#pragma unroll
+                        for (int j = 0; j < HC; ++j) pacc[j] = j < nv ? __ldcg(cp + j * kTileN) : 0;
+                    }
+                }
+            }
             // This column's scales (raw 32 bits) of group g, read straight from
             // global memory two stages before they are used, so that no wait
             // or shared-memory round trip sits between two drains.  Rows past
@@ -803,14 +836,23 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < HC; ++j)
                         if (j < nv) part[j * kTileN] = PATH == kIntScale ? acc[j] : __float_as_int(accf[j]);
-                    epi_bar_sync(kEpiWarps * 32);
-                    if (ew == 0 && lane == 0) {
-                        __threadfence();  // the CTA's partial stores (ordered by the barrier) before the arrival
-                        atomicAdd(&p.ws_count[b_first], 1);
-                    }
+                    epi_bar_sync(kEpiWarps * 32);  // the CTA's partial stores, before the arrival
+                    if (ew == 0 && lane == 0) red_release_gpu_add(&p.ws_count[b_first], 1);
                     continue;
                 }
-                if (ew == 0 && lane == 0) {
+                if (early) {
+                    // one other contributor, read at the start of the segment (the
+                    // same sum, in the same order, as below)
+#pragma unroll
+                    for (int j = 0; j < HC; ++j) {
+                        if constexpr (C::kEarlyCombine) {
+                            if (PATH == kIntScale)
+                                acc[j] += pacc[j];
+                            else
+                                accf[j] = __fadd_rn(accf[j], __int_as_float(pacc[j]));
+                        }
+                    }
+                } else if (ew == 0 && lane == 0) {
                     const int expect = int(b_last - b_first);
                     const long long w0 = clock64();
                     int ok_wait = 1;
@@ -824,14 +866,15 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                         __nanosleep(64);
                     }
                     misc[2] = uint32_t(ok_wait);
-                    __threadfence();
                 }
-                epi_bar_sync(kEpiWarps * 32);
-                if (!misc[2]) {
-                    ok = false;
-                    break;
+                if (!early) {
+                    epi_bar_sync(kEpiWarps * 32);
+                    if (!misc[2]) {
+                        ok = false;
+                        break;
+                    }
                 }
-                for (uint32_t c = b_first + 1; c <= b_last; ++c) {
+                for (uint32_t c = early ? b_last + 1 : b_first + 1; c <= b_last; ++c) {
                     const int32_t* cp = p.ws_part + int64_t(c) * slot_elems + int64_t(half * HC) * kTileN + r;
 #pragma unroll
                     for (int j = 0; j < HC; ++j) {
@@ -883,7 +926,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 bulk_commit_group();
             }
         }
-        if (ew == 0 && lane == 0) bulk_wait_all();  // every output store has completed
+        if (ew == 0 && lane == 0) bulk_wait_read_all();  // shared memory stays until the stores have read it
     }
 
     tc_fence_before();
