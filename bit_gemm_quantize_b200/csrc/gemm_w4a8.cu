@@ -72,7 +72,7 @@ constexpr int64_t kMaxGrid = kCounterBytes / 4;
 #endif
 // Token tiles up to which the integer-scale path unpacks to 16*q.
 #ifndef W4A8_X16_IS_MAX_BT
-#define W4A8_X16_IS_MAX_BT 128
+#define W4A8_X16_IS_MAX_BT 64
 #endif
 
 // Leading stages whose packed weights are requested before waiting on the
@@ -118,8 +118,9 @@ struct Cfg {
     // Unpack to 16*q (nibble into the high half of each byte, 5 integer ops per
     // 8 weights) instead of q (9 ops).  The float-scale path folds the 1/16 into
     // s_g for free; the integer-scale path pays one shift per output per group
-    // (P_g is 16 times the group product exactly), which measured faster than
-    // the exact unpack for every token tile.
+    // (P_g is 16 times the group product exactly).  With 128-token tiles the
+    // drain's shifts (32 per 8 weights unpacked) outweigh the cheaper unpack,
+    // so the integer path unpacks q exactly there (measured: 3% faster).
     static constexpr bool kX16 = (PATH == kFloatScale) || BT <= W4A8_X16_IS_MAX_BT;
     static constexpr int kWBytes = kTileN * kStageK / 2;  // packed weights per stage: 16 KB
     static constexpr int kXBytes = BT * kStageK;          // token codes per stage
