@@ -223,7 +223,6 @@ struct Stage {
     int32_t n_tile, m_tile;
     int32_t kb;   // first K block (global index along K)
     int32_t nkb;  // 1 or 2
-    int32_t g;    // group of the first K block; the groups that end in the stage are g and g + 1
 };
 
 struct StageIter {
@@ -231,7 +230,6 @@ struct StageIter {
     int32_t kbpg;
     int32_t n_tile = 0, m_tile = 0;
     int32_t kb = 0, kb_end = 0;
-    int32_t g = 0, kin = 0;  // group of the next K block and its position in the group
     __device__ StageIter(const Params& p, uint32_t b) : seg(p, b), kbpg(p.kb_per_group) {}
     __device__ bool next(Stage& st) {
         while (kb >= kb_end) {
@@ -241,21 +239,12 @@ struct StageIter {
             m_tile = s.m_tile;
             kb = s.g0 * kbpg;
             kb_end = s.g1 * kbpg;
-            g = s.g0;
-            kin = 0;
         }
         st.n_tile = n_tile;
         st.m_tile = m_tile;
         st.kb = kb;
         st.nkb = (kb_end - kb) >= 2 ? 2 : 1;
-        st.g = g;
         kb += st.nkb;
-        for (int j = 0; j < st.nkb; ++j) {
-            if (++kin == kbpg) {
-                kin = 0;
-                ++g;
-            }
-        }
         return true;
     }
 };
@@ -675,7 +664,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
             // the last group and columns past N read as zero.
             auto load_scale = [&](int32_t g) -> uint32_t {
                 if (g >= G || !nvalid) return 0u;
-                const int64_t idx = int64_t(g) * p.N + n;
+                const int64_t idx = int64_t(g) * int32_t(p.N) + n;  // N < 2^31 (checked on the host)
                 if constexpr (PATH == kIntScale)
                     return uint32_t(int32_t(__ldg(p.S + idx)));
                 else
@@ -731,19 +720,31 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
                 int ng = 0;
                 uint32_t gb0 = 0u, gb1 = 0u;  // their TMEM buffers
                 uint32_t ph0 = 0u, ph1 = 0u;  // and the phases of the buffers' full barriers
-                for (int j = 0; j < nkb; ++j) {
-                    const bool last = (kin == kbpg - 1);
-                    kin = last ? 0 : kin + 1;
-                    if (last) {
-                        if (ng == 0) {
-                            gb0 = uint32_t(rt.idx);
-                            ph0 = rt.phase;
-                        } else {
-                            gb1 = uint32_t(rt.idx);
-                            ph1 = rt.phase;
-                        }
-                        ++ng;
+                if (kbpg == 1) {  // 128-wide groups: every K block ends one
+                    ng = nkb;
+                    gb0 = uint32_t(rt.idx);
+                    ph0 = rt.phase;
+                    rt.advance(kAcc);
+                    if (nkb == 2) {
+                        gb1 = uint32_t(rt.idx);
+                        ph1 = rt.phase;
                         rt.advance(kAcc);
+                    }
+                } else {
+                    for (int j = 0; j < nkb; ++j) {
+                        const bool last = (kin == kbpg - 1);
+                        kin = last ? 0 : kin + 1;
+                        if (last) {
+                            if (ng == 0) {
+                                gb0 = uint32_t(rt.idx);
+                                ph0 = rt.phase;
+                            } else {
+                                gb1 = uint32_t(rt.idx);
+                                ph1 = rt.phase;
+                            }
+                            ++ng;
+                            rt.advance(kAcc);
+                        }
                     }
                 }
                 if (ng == 0) continue;
