@@ -115,12 +115,12 @@ struct Cfg {
     static constexpr uint32_t kAccCol0 = uint32_t(kSA * kStageCols);
     static constexpr uint32_t kTmemCols = 512;
     static_assert(kSA >= 2 && kSA * kStageCols + kAcc * BT <= 512, "TMEM budget");
-    // Unpack to 16*q (nibble into the high half of each byte, 5 integer ops per
-    // 8 weights) instead of q (9 ops).  The float-scale path folds the 1/16 into
+    // Unpack to 16*q (nibble into the high half of each byte, 3 integer ops per
+    // 8 weights) instead of q (7 ops).  The float-scale path folds the 1/16 into
     // s_g for free; the integer-scale path pays one shift per output per group
     // (P_g is 16 times the group product exactly).  With 128-token tiles the
     // drain's shifts (32 per 8 weights unpacked) outweigh the cheaper unpack,
-    // so the integer path unpacks q exactly there (measured: 3% faster).
+    // so the integer path unpacks q exactly there.
     static constexpr bool kX16 = (PATH == kFloatScale) || BT <= W4A8_X16_IS_MAX_BT;
     static constexpr int kWBytes = kTileN * kStageK / 2;  // packed weights per stage: 16 KB
     static constexpr int kXBytes = BT * kStageK;          // token codes per stage
@@ -249,9 +249,10 @@ struct StageIter {
     }
 };
 
-// int4 two's-complement nibbles -> int8, 8 values per 32-bit word.  Input byte
-// j holds k = 2j (low nibble) and k = 2j+1 (high nibble); output words hold
-// k = 0..3 and k = 4..7 in byte order.
+// int4 two's-complement nibbles -> int8, 8 values per 32-bit word.  Byte j
+// of the word holds K position j (low nibble) and j + 4 (high nibble), so the
+// low nibbles give output word 0 (K 0..3) and the high nibbles word 1 (K 4..7)
+// in MMA order with no byte permute.
 // Exact: per byte ((v ^ 8) + 0x78) ^ 0x80 maps nibble v to its sign-extended
 // byte without carries between bytes.
 __device__ __forceinline__ uint2 unpack_int4x8(uint32_t w) {
@@ -259,15 +260,13 @@ __device__ __forceinline__ uint2 unpack_int4x8(uint32_t w) {
     uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
     lo = (lo + 0x78787878u) ^ 0x80808080u;
     hi = (hi + 0x78787878u) ^ 0x80808080u;
-    return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+    return make_uint2(lo, hi);
 }
 
 // Scaled: each nibble lands in the high half of its byte, which read as int8
 // is 16 * q exactly.
 __device__ __forceinline__ uint2 unpack_int4x8_x16(uint32_t w) {
-    const uint32_t lo = (w << 4) & 0xF0F0F0F0u;
-    const uint32_t hi = w & 0xF0F0F0F0u;
-    return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+    return make_uint2((w << 4) & 0xF0F0F0F0u, w & 0xF0F0F0F0u);
 }
 
 template <bool X16>

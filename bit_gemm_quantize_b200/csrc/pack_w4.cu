@@ -120,7 +120,8 @@ __global__ void __launch_bounds__(kThreads) quantize_pack_kernel(const float* __
             const float t = __fdiv_rn(w[(k0 + i) * N + n], s);
             const float r = fminf(fmaxf(rintf(t), -7.0f), 7.0f);
             const uint32_t nib = uint32_t(int(r)) & 0xFu;
-            words[i >> 3] |= nib << (4 * (i & 7));
+            // code j = i mod 8 of its word: byte j mod 4, high nibble for j >= 4
+            words[i >> 3] |= nib << (8 * (i & 3) + 4 * ((i >> 2) & 1));
         }
     }
     *reinterpret_cast<uint4*>(packed + n * (K / 2) + k0 / 2) = make_uint4(words[0], words[1], words[2], words[3]);

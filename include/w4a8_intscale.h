@@ -110,7 +110,9 @@ W4A8_API w4a8_status w4a8_amplifier_search(const float* scales, int64_t count, v
  *  §4; 极致量化 数据打包.)
  *   s_g[g,n]  = fl32(max_{k in g} |w[k,n]| / 7)
  *   q_w[k,n]  = clamp(rne(fl32(w[k,n] / s_g[g(k),n])), -7, 7)
- *   w_packed[n, k/2] = (q_w[k,n] & 0xF) | (q_w[k+1,n] & 0xF) << 4   (k even)
+ *   w_packed[n, 4b + i] = (q_w[8b+i,n] & 0xF) | (q_w[8b+4+i,n] & 0xF) << 4   (i = 0..3):
+ *               each 32-bit word holds 8 consecutive codes along K, code j in
+ *               byte j mod 4, low nibble for j < 4, high nibble for j >= 4
  *   alpha     = alpha_in if alpha_in > 0 (must be a power of two <= 2^30),
  *               else the amplifier search over this layer's s_g
  *   S[g,n]    = rne(s_g[g,n] * alpha)

@@ -131,15 +131,19 @@ def quantize_groups(w, group: int = 128, qmax: int = INT4_QMAX):
 
 
 def pack_int4(q):
-    """Codes q [K,N] in [-8,7] -> packed uint8 [N, K/2]."""
+    """Codes q [K,N] in [-8,7] -> packed uint8 [N, K/2] (K a multiple of 8)."""
     q = _c(q, np.int8)
     K, N = q.shape
+    if K % 8:
+        raise ValueError(f"K must be a multiple of 8, got {K}")
     out = np.empty((N, K // 2), np.uint8)
     _load().oracle_pack_int4(_p(q), K, N, _p(out))
     return out
 
 
 def unpack_int4(packed, K: int, N: int):
+    if K % 8:
+        raise ValueError(f"K must be a multiple of 8, got {K}")
     packed = _c(packed, np.uint8)
     out = np.empty((K, N), np.int8)
     _load().oracle_unpack_int4(_p(packed), K, N, _p(out))

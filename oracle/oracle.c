@@ -100,13 +100,22 @@ void oracle_quantize_groups(const float* w, int64_t K, int64_t N, int64_t group,
 
 /* ---- [X4] nibble packing -------------------------------------------------- */
 
+/* Layout (a reading: the pages only say that several low-bit values share one
+ * standard integer).  Along K, every 8 codes fill one 32-bit word, 4 bytes:
+ * code i of the 8 (k = 8b + i) sits in byte 4b + (i mod 4), in the low nibble
+ * for i < 4 and the high nibble for i >= 4, as a two's-complement nibble.
+ * K must be a multiple of 8. */
+static int64_t packed_byte(int64_t k) { return (k >> 3) * 4 + (k & 3); }
+static int packed_shift(int64_t k) { return (int)((k >> 2) & 1) * 4; }
+
 void oracle_pack_int4(const int8_t* q, int64_t K, int64_t N, uint8_t* packed) {
-    for (int64_t n = 0; n < N; ++n)
-        for (int64_t k = 0; k < K; k += 2) {
-            unsigned lo = (unsigned)(uint8_t)q[k * N + n] & 0xFu;
-            unsigned hi = (unsigned)(uint8_t)q[(k + 1) * N + n] & 0xFu;
-            packed[n * (K / 2) + k / 2] = (uint8_t)(lo | (hi << 4));
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t j = 0; j < K / 2; ++j) packed[n * (K / 2) + j] = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            unsigned nib = (unsigned)(uint8_t)q[k * N + n] & 0xFu;
+            packed[n * (K / 2) + packed_byte(k)] |= (uint8_t)(nib << packed_shift(k));
         }
+    }
 }
 
 /* Two's-complement nibble back to a signed value. */
@@ -114,10 +123,9 @@ static int32_t nibble_value(unsigned nib) { return (nib & 0x8u) ? (int32_t)nib -
 
 void oracle_unpack_int4(const uint8_t* packed, int64_t K, int64_t N, int8_t* q) {
     for (int64_t n = 0; n < N; ++n)
-        for (int64_t k = 0; k < K; k += 2) {
-            uint8_t b = packed[n * (K / 2) + k / 2];
-            q[k * N + n] = (int8_t)nibble_value(b & 0xFu);
-            q[(k + 1) * N + n] = (int8_t)nibble_value((b >> 4) & 0xFu);
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t b = packed[n * (K / 2) + packed_byte(k)];
+            q[k * N + n] = (int8_t)nibble_value((b >> packed_shift(k)) & 0xFu);
         }
 }
 

@@ -161,15 +161,23 @@ def test_pack_golden():
 def test_pack_exhaustive_nibble_roundtrip():
     vals = np.arange(-8, 8, dtype=np.int8)
     lo, hi = np.meshgrid(vals, vals, indexing="ij")
-    q = np.stack([lo.ravel(), hi.ravel()])  # K=2, N=256
+    rng = np.random.default_rng(11)
+    # K=8, N=256: every (code 0, code 4) pair once, the other six codes random
+    q = rng.integers(-8, 8, size=(8, 256)).astype(np.int8)
+    q[0], q[4] = lo.ravel(), hi.ravel()
     p = oracle.pack_int4(q)
-    assert p.shape == (256, 1)
-    assert sorted(p.ravel().tolist()) == list(range(256))  # a bijection onto bytes
-    assert np.array_equal(oracle.unpack_int4(p, 2, 256), q)
-    # nibble semantics: low nibble is the even k, both two's complement
-    b = p[:, 0].astype(np.int64)
-    assert np.array_equal(((b & 0xF) ^ 8) - 8, lo.ravel())
-    assert np.array_equal((((b >> 4) & 0xF) ^ 8) - 8, hi.ravel())
+    assert p.shape == (256, 4)
+    assert sorted(p[:, 0].tolist()) == list(range(256))  # byte 0 is a bijection of (code 0, code 4)
+    assert np.array_equal(oracle.unpack_int4(p, 8, 256), q)
+    # nibble semantics: byte j holds code j (low) and code j + 4 (high), two's complement
+    for j in range(4):
+        b = p[:, j].astype(np.int64)
+        assert np.array_equal(((b & 0xF) ^ 8) - 8, q[j])
+        assert np.array_equal((((b >> 4) & 0xF) ^ 8) - 8, q[j + 4])
+    # the next 8 codes go to the next 4 bytes
+    q2 = np.zeros((16, 1), np.int8)
+    q2[8:, 0] = np.arange(1, 9)
+    assert oracle.pack_int4(q2)[0].tolist() == [0, 0, 0, 0, 0x51, 0x62, 0x73, 0x84]
 
 
 # ------------------------------------------------------------- amplifier
