@@ -273,6 +273,78 @@ def measure_moe(dev, rank, world, int8_peak, reps=10):
             "timing": "CUDA events over graph replays of quantize + gather + per-expert GEMMs; weights > L2"}
 
 
+PREFILL = dict(M=4096, shapes=[(4096, 11008), (11008, 4096)])  # (K, N) of the two layers
+
+
+def measure_prefill(dev, rank, world, int8_peak, reps=10):
+    """The prefill-shaped layers (4096 tokens; K=4096, N=11008 and K=11008,
+    N=4096): per-token quantize of bf16 tokens with outlier channels, then the
+    integer-scale GEMM with fp16 output.  Inputs are drawn on the device
+    (seeded Philox: weights ~ N(0, 0.02), tokens ~ N(0, 1) with 0.5% of the
+    channels scaled by 30), alpha = 1024.  The two layers are replayed one
+    after the other; together they hold about 300 MB, more than the L2."""
+    import torch
+
+    import bit_gemm_quantize_b200 as bgq
+
+    M = PREFILL["M"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(4000 + rank)
+    layers = []
+    for K, N in PREFILL["shapes"]:
+        w = torch.randn((K, N), generator=g, device=dev)
+        w.mul_(0.02)
+        pk = bgq.pack_w4_groupwise(w, group=GROUP, alpha=1024)
+        del w
+        x = torch.randn((M, K), generator=g, device=dev)
+        cols = torch.randperm(K, generator=g, device=dev)[: max(1, K // 200)]
+        x[:, cols] *= 30.0
+        x = x.to(torch.bfloat16)
+        q = torch.empty((M, K), dtype=torch.int8, device=dev)
+        s = torch.empty((M,), dtype=torch.float32, device=dev)
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        wsp = bgq.gemm_workspace(M, N, K, GROUP, 0, dev)
+        layers.append((K, N, x, q, s, pk, y, wsp))
+    torch.cuda.empty_cache()
+
+    def run(layer):
+        K, N, x, q, s, pk, y, wsp = layer
+        bgq.quantize_act_per_token(x, q, s)
+        bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], pk["alpha"], group=GROUP, out="f16", y=y, workspace=wsp)
+
+    graphs = []
+    for layer in layers:
+        for _ in range(3):
+            run(layer)
+        torch.cuda.synchronize(dev)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            run(layer)
+        gr.replay()
+        graphs.append(gr)
+    stream = torch.cuda.current_stream(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in graphs]
+    tot = [0.0 for _ in graphs]
+    torch.cuda.synchronize(dev)
+    for _ in range(reps):
+        for i, gr in enumerate(graphs):
+            ev[i][0].record(stream)
+            gr.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        for i in range(len(graphs)):
+            tot[i] += ev[i][0].elapsed_time(ev[i][1])
+    ms = max_over_ranks([t / reps for t in tot], world, dev)
+    del graphs
+    out = []
+    for (K, N, *_), t in zip(layers, ms):
+        tops = 2.0 * M * N * K / (t * 1e-3) / 1e12
+        out.append({"M": M, "K": K, "N": N, "us_quantize_plus_gemm": round(t * 1e3, 2), "tops": round(tops, 2),
+                    "frac_int8": round(tops / int8_peak, 4)})
+    return {"workload": "prefill_4096", "group": GROUP, "alpha": 1024, "layers": out,
+            "timing": "CUDA events around graph replays of quantize + integer-scale GEMM, the two layers alternating"}
+
+
 # ---------------------------------------------------------------- rank aggregation
 
 def max_over_ranks(times_ms, world, device):
@@ -495,6 +567,7 @@ def run_ours(args):
                            f"{INT8_PER_BF16} (nominal int8:bf16 ratio)")
 
     moe = measure_moe(dev, rank, world, int8_peak)
+    prefill = measure_prefill(dev, rank, world, int8_peak)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
@@ -504,6 +577,7 @@ def run_ours(args):
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * len(SWEEP) * args.steps,
         "moe": moe,
+        "prefill": prefill,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample()
