@@ -502,15 +502,32 @@ def run_ours(args):
     yh = [torch.empty((M, N_DIM), dtype=torch.float16).pin_memory() for M in SWEEP]
     xd = [torch.empty_like(x) for x in xs]
 
+    # The calls a user makes (public API, host input in, host output back),
+    # pipelined the way a serving loop would run them: uploads on one stream,
+    # quantize + GEMM on the main stream, downloads on a third, so a layer's
+    # download overlaps the next layers' uploads and compute (PCIe carries
+    # both directions at once).
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
     def e2e_step():
-        # the call a user makes: public API, host input in, host output back
+        up.wait_stream(stream)  # the previous step's compute has read the device inputs
+        ev_in = []
+        with torch.cuda.stream(up):
+            for i in range(len(SWEEP)):
+                xd[i].copy_(xh[i], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(up)
+                ev_in.append(ev)
         for i, M in enumerate(SWEEP):
             c = copies[i]
-            xd[i].copy_(xh[i], non_blocking=True)
+            stream.wait_event(ev_in[i])
             bgq.quantize_act_per_token(xd[i], qs[i], ss[i])
             bgq.w4a8_gemm_intscale(qs[i], ss[i], c["packed"], c["S"], ALPHA, group=GROUP, out="f16", y=ys[i],
                                    workspace=ws_all)
-            yh[i].copy_(ys[i], non_blocking=True)
+            down.wait_stream(stream)
+            with torch.cuda.stream(down):
+                yh[i].copy_(ys[i], non_blocking=True)
+        stream.wait_stream(down)  # the step ends when every output is on the host
 
     for _ in range(3):
         e2e_step()
