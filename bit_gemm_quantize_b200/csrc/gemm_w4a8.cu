@@ -15,15 +15,16 @@
 // Data flow per pipeline stage (256 consecutive K):
 //   HBM --TMA--> packed int4 box [128 n][128 B] (128-byte swizzle)      (W ring, smem)
 //   HBM --TMA--> token codes [BT m][128 k] x2 (128-byte swizzle)        (X ring, smem)
-//   HBM --TMA--> group scales [2 g][128 n]                              (S ring, smem)
 //   unpack warps (one thread per weight row = TMEM lane): packed int4 ->
 //   int8, written with tcgen05.st as the MMA's A operand, 64 TMEM columns
 //   of 4 K values each                                                  (A ring, TMEM)
 //   tcgen05.mma.kind::i8, A from TMEM, B = token codes from smem, K = 32
 //   each, accumulating one group's P_g in a TMEM buffer [128][BT]       (acc ring, TMEM)
-//   epilogue warps per group: tcgen05.ld P_g, acc += S[g,n] * P_g (or
-//   accf += s_g * float(P_g)); after the last group y = acc * s_a[m] / alpha
-//   (or accf * s_a[m]).
+//   epilogue warps per group: this column's S[g,n] (or s_g), loaded from
+//   global memory two stages ahead; tcgen05.ld P_g, acc += S[g,n] * P_g (or
+//   accf += s_g * float(P_g)); after the tile's last group y = acc * s_a[m]
+//   / alpha (or accf * s_a[m]), staged in shared memory and written by one
+//   TMA tensor store.
 // Keeping the unpacked operand in TMEM instead of shared memory saves two of
 // its passes through the shared-memory port (the unpack's store and the MMA's
 // read, 64 KB per stage), which bound small-token-tile MMAs at about 40
