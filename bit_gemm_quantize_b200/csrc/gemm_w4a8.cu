@@ -88,12 +88,19 @@ constexpr int64_t kMaxGrid = kCounterBytes / 4;
 #define W4A8_GROUP_COMMIT_MIN_BT 64
 #endif
 
-// Ring depths (stages) of the packed weights and the token codes.
+// CTAs per SM: decode-shaped calls (16-token tiles) run two CTAs per SM,
+// each with half of the TMEM and shared memory, so that the two pipelines'
+// chains of dependent waits and copies overlap.
+#ifndef W4A8_CTAS_PER_SM
+#define W4A8_CTAS_PER_SM(BT) ((BT) == 16 ? 2 : 1)
+#endif
+
+// Ring depths (stages) of the packed weights and the token codes (per CTA).
 #ifndef W4A8_SW
-#define W4A8_SW(BT) ((BT) <= 32 ? 8 : ((BT) == 64 ? 6 : 4))
+#define W4A8_SW(BT) (W4A8_CTAS_PER_SM(BT) == 2 ? 4 : ((BT) <= 32 ? 8 : ((BT) == 64 ? 6 : 4)))
 #endif
 #ifndef W4A8_SX
-#define W4A8_SX(BT) ((BT) <= 32 ? 6 : ((BT) == 64 ? 4 : 3))
+#define W4A8_SX(BT) (W4A8_CTAS_PER_SM(BT) == 2 ? 3 : ((BT) <= 32 ? 6 : ((BT) == 64 ? 4 : 3)))
 #endif
 
 template <int BT, int PATH>
@@ -111,11 +118,12 @@ struct Cfg {
     // TMEM (512 columns): kSA unpacked-operand slots of 64 columns, then kAcc
     // accumulator buffers of BT columns.  The MMA may run kAcc - 1 groups
     // ahead of the per-group drain.
+    static constexpr int kCtasPerSm = W4A8_CTAS_PER_SM(BT);
+    static constexpr uint32_t kTmemCols = 512u / uint32_t(kCtasPerSm);  // TMEM columns of this CTA
     static constexpr int kAcc = BT == 128 ? 3 : (BT == 64 ? 4 : 8);
-    static constexpr int kSA = (512 - kAcc * BT) / kStageCols > 6 ? 6 : (512 - kAcc * BT) / kStageCols;
+    static constexpr int kSA = (int(kTmemCols) - kAcc * BT) / kStageCols > 6 ? 6 : (int(kTmemCols) - kAcc * BT) / kStageCols;
     static constexpr uint32_t kAccCol0 = uint32_t(kSA * kStageCols);
-    static constexpr uint32_t kTmemCols = 512;
-    static_assert(kSA >= 2 && kSA * kStageCols + kAcc * BT <= 512, "TMEM budget");
+    static_assert(kSA >= 2 && kSA * kStageCols + kAcc * BT <= int(kTmemCols), "TMEM budget");
     // Unpack to 16*q (nibble into the high half of each byte, 3 integer ops per
     // 8 weights) instead of q (7 ops).  The float-scale path folds the 1/16 into
     // s_g for free; the integer-scale path pays one shift per output per group
@@ -152,6 +160,7 @@ struct Cfg {
     static_assert(kXBytes % 2048 == 0, "token stage must hold whole 8-row swizzle atoms per k-block");
     static_assert(offY % 128 == 0, "TMA store source alignment");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+    static_assert(kCtasPerSm == 1 || kSmemBytes * kCtasPerSm <= 227 * 1024, "shared memory for two CTAs per SM");
 };
 
 // One contiguous run of groups [g0, g1) of one tile inside a CTA's range.
@@ -334,7 +343,7 @@ struct Ring {
 };
 
 template <int BT, int PATH>
-__global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, 1)
+__global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, Cfg<BT, PATH>::kCtasPerSm)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_y, const Params p) {
     using C = Cfg<BT, PATH>;
@@ -956,7 +965,8 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms) {
     pl.G = K / group;
     pl.tiles = pl.n_tiles * pl.m_tiles;
     pl.W = pl.tiles * pl.G;
-    pl.grid = pl.W < num_sms ? pl.W : num_sms;
+    const int64_t slots = int64_t(num_sms) * W4A8_CTAS_PER_SM(pl.BT);  // resident CTAs
+    pl.grid = pl.W < slots ? pl.W : slots;
     if (pl.grid > kMaxGrid) pl.grid = kMaxGrid;
     const int64_t slot_bytes = int64_t(kTileN) * pl.BT * 4;
     pl.count_bytes = kCounterBytes;
