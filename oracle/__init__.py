@@ -19,6 +19,9 @@ Parity status per function (what pins it, see tests/test_oracle_pins.py):
   amplifier_search                 postcondition (min scale * alpha >= 1 and
                                    minimal), frexp closed form, hand-worked goldens
   integer_scales                   |S - s*alpha| <= 1/2, exact at representable values
+  alpha_sweep                      MSE <= mean(q^2) / (4 alpha^2), zero when every
+                                   s_g * alpha is an integer, a hand-worked case,
+                                   bit counts at powers of two
   intscale_acc                     equals the expanded-W_int form, numpy int64
                                    matmul when S is constant over groups, brute
                                    fp64 dequantized matmul on tiny inputs, X=0,
@@ -74,6 +77,7 @@ def _load():
                 "oracle_quantize_rows": ([P, I, I, I32, P, P], None),
                 "oracle_quantize_groups": ([P, I, I, I, I32, P, P], None),
                 "oracle_pack_int4": ([P, I, I, P], None),
+                "oracle_alpha_sweep": ([P, P, I, I, I, P, I, P, P], None),
                 "oracle_unpack_int4": ([P, I, I, P], None),
                 "oracle_amplifier_search": ([P, I], I32),
                 "oracle_integer_scales": ([P, I, I32, P], None),
@@ -160,6 +164,21 @@ def integer_scales(s_g, alpha: int):
     out = np.empty(s.shape, np.int32)
     _load().oracle_integer_scales(_p(s), s.size, int(alpha), _p(out))
     return out
+
+
+def alpha_sweep(qw, s_g, alphas, group: int = 128):
+    """Amplifier analysis (Integer Scale summary §4, Fig. 4(a)/(c)): for each
+    alpha, the weight MSE between integer-scale (S / alpha) and float-scale
+    (s_g) dequantization of the codes qw [K,N], and the bits of the largest
+    S = rne(s_g * alpha).  Returns (mse [n] float64, bits [n] int32)."""
+    qw = _c(qw, np.int8)
+    s_g = _c(s_g, np.float32)
+    a = _c(np.ravel(alphas), np.int32)
+    K, N = qw.shape
+    mse = np.empty(a.size, np.float64)
+    bits = np.empty(a.size, np.int32)
+    _load().oracle_alpha_sweep(_p(qw), _p(s_g), K, N, group, _p(a), a.size, _p(mse), _p(bits))
+    return mse, bits
 
 
 def scale_colsum_max(S) -> int:

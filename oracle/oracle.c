@@ -263,6 +263,36 @@ void oracle_floatscale_at(const int8_t* qx, const float* s_a, const int8_t* qw, 
     }
 }
 
+/* ---- [IS] §4, Fig. 4(a)/(c): amplifier analysis ------------------------- */
+
+/* For each amplifier alphas[i]: the mean squared difference between the
+ * weights dequantized with the integer scales and with the float scales,
+ * mean over (k, n) of (q[k,n] * (S[g,n] / alpha - s_g[g,n]))^2 with
+ * S = rne(s_g * alpha) as in oracle_integer_scales (Fig. 4(c)), and the bits
+ * the largest S needs as an unsigned integer (Fig. 4(a)).  fp64 throughout. */
+void oracle_alpha_sweep(const int8_t* q, const float* s_g, int64_t K, int64_t N, int64_t group,
+                        const int32_t* alphas, int64_t n_alpha, double* mse, int32_t* max_bits) {
+    int64_t G = K / group;
+    for (int64_t i = 0; i < n_alpha; ++i) {
+        double a = (double)alphas[i], sum = 0.0, smax = 0.0;
+        for (int64_t g = 0; g < G; ++g)
+            for (int64_t n = 0; n < N; ++n) {
+                double sf = (double)s_g[g * N + n];
+                double S = rint(sf * a);
+                double d = S / a - sf;
+                if (S > smax) smax = S;
+                for (int64_t k = g * group; k < (g + 1) * group; ++k) {
+                    double e = (double)q[k * N + n] * d;
+                    sum += e * e;
+                }
+            }
+        mse[i] = sum / ((double)K * (double)N);
+        int32_t bits = 0;
+        while (bits < 62 && (double)((int64_t)1 << bits) <= smax) ++bits;  /* smallest b with smax < 2^b */
+        max_bits[i] = bits;
+    }
+}
+
 /* ---- worst-case int32 bound ----------------------------------------------- */
 
 /* max over columns n of sum_g |S[g,n]|, the factor that multiplies

@@ -447,3 +447,46 @@ def test_moe_rows_follow_their_token_and_expert():
         a = {int(t): base["acc"][i] for t, i in zip(ri[off[e]:off[e + 1]], range(off[e], off[e + 1]))}
         for i in range(off2[e], off2[e + 1]):
             assert np.array_equal(other["acc"][i], a[int(perm[ri2[i]])])
+
+
+# ------------------------------------------------------------- amplifier analysis (Fig. 4)
+
+def test_alpha_sweep_hand_case():
+    # one group of two codes, s = 0.3: S = rne(0.3 alpha) = 0, 1, 1 for alpha = 1, 2, 4;
+    # MSE = mean((q (S/alpha - 0.3))^2) = (49 + 9) d^2 / 2 with d = -0.3, 0.2, -0.05
+    q = np.array([[7], [-3]], np.int8)
+    s = np.array([[0.3]], np.float32)
+    mse, bits = oracle.alpha_sweep(q, s, [1, 2, 4], group=2)
+    np.testing.assert_allclose(mse, [2.61, 1.16, 0.0725], rtol=1e-6)
+    assert bits.tolist() == [0, 1, 1]
+
+
+def test_alpha_sweep_rounding_bound():
+    # |S/alpha - s| <= 1/(2 alpha) per group, so MSE <= mean(q^2) / (4 alpha^2)
+    rng = np.random.default_rng(21)
+    w = (rng.standard_normal((512, 64)) * 0.02).astype(np.float32)
+    q, s = oracle.quantize_groups(w, 128)
+    alphas = [1 << j for j in range(15)]
+    mse, bits = oracle.alpha_sweep(q, s, alphas, group=128)
+    bound = np.mean(q.astype(np.float64) ** 2) / (4.0 * np.array(alphas, np.float64) ** 2)
+    assert np.all(mse <= bound * (1 + 1e-12))
+    assert np.all(np.diff(bits) >= 0) and bits[-1] > bits[0]
+
+
+def test_alpha_sweep_exact_when_scales_are_multiples():
+    # s_g = j / 1024 exactly: integer scales reproduce the float scales at alpha >= 1024
+    q = np.array([[7, -5], [3, 2], [-7, 1], [0, -3]], np.int8)
+    s = np.array([[37 / 1024, 5 / 1024]], np.float32)
+    mse, _ = oracle.alpha_sweep(q, s, [256, 1024, 4096], group=4)
+    assert mse[1] == 0.0 and mse[2] == 0.0 and mse[0] > 0.0
+
+
+def test_alpha_sweep_bit_counts():
+    # the largest S as an unsigned integer: 255 needs 8 bits, 256 needs 9
+    q = np.ones((2, 2), np.int8)
+    s = np.array([[255.0, 1.0]], np.float32)
+    _, bits = oracle.alpha_sweep(q, s, [1], group=2)
+    assert bits.tolist() == [8]
+    s = np.array([[256.0, 3.0]], np.float32)
+    _, bits = oracle.alpha_sweep(q, s, [1], group=2)
+    assert bits.tolist() == [9]
