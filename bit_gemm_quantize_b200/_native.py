@@ -71,6 +71,7 @@ def load(path: str = LIB_PATH):
             "quantize_act_per_token": ([P, I32_, I64, I64, I64, P, P, P], I32_),
             "w4a8_amplifier_search": ([P, I64, P, P, P], I32_),
             "pack_w4_groupwise": ([P, I64, I64, I32_, I32_, P, P, P, P, P, P, P], I32_),
+            "pack_w4_groupwise_range": ([P, I64, I64, I32_, I32_, I32_, P, P, P, P, P, P, P], I32_),
             "w4a8_gemm_workspace_size": ([I64, I64, I64, I32_, I32_], I64),
             "w4a8_gemm_intscale": ([P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
             "w4a8_gemm_intscale_static_ws": ([P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P], I32_),
@@ -175,8 +176,11 @@ def w4a8_amplifier_search(scales: torch.Tensor) -> int:
     return int(alpha.value)
 
 
-def pack_w4_groupwise(w: torch.Tensor, group: int = 128, alpha: int | None = 1024, scales_only: bool = False):
+def pack_w4_groupwise(w: torch.Tensor, group: int = 128, alpha: int | None = 1024, scales_only: bool = False,
+                      qmin: int = -7):
     """Quantize and pack fp32 weights w [K, N].  alpha=None runs the search.
+    qmin=-7: codes in [-7, 7], s_g = max|w| / 7; qmin=-8: the full int4
+    range [-8, 7], s_g = max|w| / 8.
 
     Returns dict(packed [N, K/2] uint8, s_g [K/group, N] f32, S [K/group, N]
     int16, alpha, colsum_max), or dict(s_g) when scales_only."""
@@ -187,18 +191,18 @@ def pack_w4_groupwise(w: torch.Tensor, group: int = 128, alpha: int | None = 102
     ws = torch.empty(PACK_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
     lib = load()
     if scales_only:
-        code = lib.pack_w4_groupwise(_ptr(w), K, N, group, 0, None, _ptr(s_g), None, None, None, _ptr(ws),
-                                     _stream(dev))
-        _check("pack_w4_groupwise", code)
+        code = lib.pack_w4_groupwise_range(_ptr(w), K, N, group, 0, int(qmin), None, _ptr(s_g), None, None, None,
+                                           _ptr(ws), _stream(dev))
+        _check("pack_w4_groupwise_range", code)
         return dict(s_g=s_g)
     packed = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
     S = torch.empty((K // group, N), dtype=torch.int16, device=dev)
     a_out = ctypes.c_int32(0)
     colsum = ctypes.c_int64(0)
-    code = lib.pack_w4_groupwise(_ptr(w), K, N, group, 0 if alpha is None else int(alpha), _ptr(packed),
-                                 _ptr(s_g), _ptr(S), ctypes.byref(a_out), ctypes.byref(colsum), _ptr(ws),
-                                 _stream(dev))
-    _check("pack_w4_groupwise", code)
+    code = lib.pack_w4_groupwise_range(_ptr(w), K, N, group, 0 if alpha is None else int(alpha), int(qmin),
+                                       _ptr(packed), _ptr(s_g), _ptr(S), ctypes.byref(a_out), ctypes.byref(colsum),
+                                       _ptr(ws), _stream(dev))
+    _check("pack_w4_groupwise_range", code)
     return dict(packed=packed, s_g=s_g, S=S, alpha=int(a_out.value), colsum_max=int(colsum.value))
 
 

@@ -308,9 +308,10 @@ w4a8_status w4a8_amplifier_search(const float* scales, int64_t count, void* work
     return W4A8_OK;
 }
 
-w4a8_status pack_w4_groupwise(const float* w, int64_t K, int64_t N, int32_t group, int32_t alpha_in,
-                              uint8_t* w_packed, float* s_g, int16_t* S, int32_t* alpha_out_host,
-                              int64_t* colsum_max_host, void* workspace, void* stream) {
+w4a8_status pack_w4_groupwise_range(const float* w, int64_t K, int64_t N, int32_t group, int32_t alpha_in,
+                                    int32_t qmin, uint8_t* w_packed, float* s_g, int16_t* S, int32_t* alpha_out_host,
+                                    int64_t* colsum_max_host, void* workspace, void* stream) {
+    if (qmin != -7 && qmin != -8) return W4A8_ERR_INVALID_ARG;
     if (K <= 0 || N <= 0 || group <= 0 || group % 32 != 0 || K % group != 0 || N % 8 != 0) return W4A8_ERR_SHAPE;
     if (K > INT32_MAX || N > INT32_MAX || K / group > 65535 || K / 32 > 65535) return W4A8_ERR_SHAPE;
     if (!w || !s_g) return W4A8_ERR_INVALID_ARG;
@@ -324,7 +325,7 @@ w4a8_status pack_w4_groupwise(const float* w, int64_t K, int64_t N, int32_t grou
     w4a8_status st = current_device(dev);
     if (st != W4A8_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    W4A8_CUDA_TRY(w4a8::pack::group_scales(w, K, N, group, s_g, s));
+    W4A8_CUDA_TRY(w4a8::pack::group_scales(w, K, N, group, qmin, s_g, s));
     if (scales_only) {
         W4A8_CUDA_TRY(cudaStreamSynchronize(s));
         return W4A8_OK;
@@ -341,14 +342,21 @@ w4a8_status pack_w4_groupwise(const float* w, int64_t K, int64_t N, int32_t grou
         *alpha_out_host = r.alpha;
         return W4A8_ERR_SCALE_RANGE;
     }
-    W4A8_CUDA_TRY(w4a8::pack::quantize_pack(w, s_g, r.alpha, K, N, group, w_packed, S, workspace, s));
+    W4A8_CUDA_TRY(w4a8::pack::quantize_pack(w, s_g, r.alpha, K, N, group, qmin, w_packed, S, workspace, s));
     W4A8_CUDA_TRY(cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s));
     W4A8_CUDA_TRY(cudaStreamSynchronize(s));
     *alpha_out_host = r.alpha;
     if (colsum_max_host) *colsum_max_host = int64_t(r.colsum_max);
-    const double bound = 127.0 * 7.0 * double(group) * double(r.colsum_max);
+    const double bound = 127.0 * double(-qmin) * double(group) * double(r.colsum_max);
     if (bound >= 2147483648.0) return W4A8_ERR_OVERFLOW_BOUND;
     return W4A8_OK;
+}
+
+w4a8_status pack_w4_groupwise(const float* w, int64_t K, int64_t N, int32_t group, int32_t alpha_in,
+                              uint8_t* w_packed, float* s_g, int16_t* S, int32_t* alpha_out_host,
+                              int64_t* colsum_max_host, void* workspace, void* stream) {
+    return pack_w4_groupwise_range(w, K, N, group, alpha_in, -7, w_packed, s_g, S, alpha_out_host, colsum_max_host,
+                                   workspace, stream);
 }
 
 int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group, int32_t path) {

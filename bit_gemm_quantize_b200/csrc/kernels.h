@@ -63,12 +63,15 @@ struct Results {
 constexpr int64_t kPartialsOffset = 256;  // per-block (min, max) pairs start here
 constexpr int kMaxPartialBlocks = 4096;
 
-cudaError_t group_scales(const float* w, int64_t K, int64_t N, int32_t group, float* s_g, cudaStream_t stream);
+// qmin: the lowest code, -7 (codes [-7, 7], s = max|w| / 7) or -8 (codes
+// [-8, 7], s = max|w| / 8)
+cudaError_t group_scales(const float* w, int64_t K, int64_t N, int32_t group, int32_t qmin, float* s_g,
+                         cudaStream_t stream);
 // min / max reduction + amplifier search (alpha_in > 0: fixed amplifier)
 cudaError_t amplifier(const float* scales, int64_t count, int32_t alpha_in, void* workspace,
                       cudaStream_t stream, int num_sms);
 cudaError_t quantize_pack(const float* w, const float* s_g, int32_t alpha, int64_t K, int64_t N, int32_t group,
-                          uint8_t* packed, int16_t* S, void* workspace, cudaStream_t stream);
+                          int32_t qmin, uint8_t* packed, int16_t* S, void* workspace, cudaStream_t stream);
 }  // namespace pack
 
 }  // namespace w4a8

@@ -3,7 +3,9 @@
 //
 // 探秘Transformer系列之（34）量化基礎 §2.3.3 逐组量化 (one scale per group of
 // consecutive K entries of a weight column); "Quantization" notes, Symmetric
-// Quantization (s = max|w| / qmax, z = 0), here with qmax = 7; Integer Scale
+// Quantization (s = max|w| / qmax, z = 0), here with qmax = 7 (codes [-7, 7]),
+// or the full signed 4-bit range [-8, 7] of 极致量化 其他子4位整数格式 with
+// s = max|w| / 8; Integer Scale
 // summary §4 (amplifier search, S = round(s_g * alpha)); 极致量化 数据打包.
 #include <cuda_runtime.h>
 
@@ -19,17 +21,18 @@ constexpr int kThreads = 256;
 
 __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); }
 
-// s_g[g, n] = fl32(max_{k in g} |w[k, n]| / 7).  One thread per column n and
-// group g; threads of a warp read consecutive columns of one row.
+// s_g[g, n] = fl32(max_{k in g} |w[k, n]| / qdiv), qdiv = 7 for codes in
+// [-7, 7] or 8 for the full two's-complement range [-8, 7].  One thread per
+// column n and group g; threads of a warp read consecutive columns of one row.
 __global__ void __launch_bounds__(kThreads) group_scales_kernel(const float* __restrict__ w, int64_t K, int64_t N,
-                                                                int32_t group, float* __restrict__ s_g) {
+                                                                int32_t group, float qdiv, float* __restrict__ s_g) {
     const int64_t n = int64_t(blockIdx.x) * kThreads + threadIdx.x;
     const int64_t g = blockIdx.y;
     if (n >= N) return;
     const float* col = w + g * group * N + n;
     float a = 0.0f;
     for (int32_t k = 0; k < group; ++k) a = fmaxf(a, fabsf(col[int64_t(k) * N]));
-    s_g[g * N + n] = (a == 0.0f) ? 0.0f : __fdiv_rn(a, 7.0f);
+    s_g[g * N + n] = (a == 0.0f) ? 0.0f : __fdiv_rn(a, qdiv);
 }
 
 // Per-block smallest positive and largest scale.
@@ -105,7 +108,7 @@ __global__ void amplifier_kernel(const float2* __restrict__ partial, int nblocks
 // consecutive n) and writes 16 packed bytes packed[n, k0/2 ..].
 __global__ void __launch_bounds__(kThreads) quantize_pack_kernel(const float* __restrict__ w,
                                                                  const float* __restrict__ s_g, int32_t alpha,
-                                                                 int64_t K, int64_t N, int32_t group,
+                                                                 int64_t K, int64_t N, int32_t group, float qmin,
                                                                  uint8_t* __restrict__ packed,
                                                                  int16_t* __restrict__ S) {
     const int64_t n = int64_t(blockIdx.x) * kThreads + threadIdx.x;
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(kThreads) quantize_pack_kernel(const float* __
 #pragma unroll 8
         for (int i = 0; i < 32; ++i) {
             const float t = __fdiv_rn(w[(k0 + i) * N + n], s);
-            const float r = fminf(fmaxf(rintf(t), -7.0f), 7.0f);
+            const float r = fminf(fmaxf(rintf(t), qmin), 7.0f);  // qmin: -7 or -8
             const uint32_t nib = uint32_t(int(r)) & 0xFu;
             // code j = i mod 8 of its word: byte j mod 4, high nibble for j >= 4
             words[i >> 3] |= nib << (8 * (i & 3) + 4 * ((i >> 2) & 1));
@@ -146,9 +149,10 @@ __global__ void __launch_bounds__(kThreads) colsum_kernel(const int16_t* __restr
     if ((threadIdx.x & 31) == 0) atomicMax(out, t);
 }
 
-cudaError_t group_scales(const float* w, int64_t K, int64_t N, int32_t group, float* s_g, cudaStream_t stream) {
+cudaError_t group_scales(const float* w, int64_t K, int64_t N, int32_t group, int32_t qmin, float* s_g,
+                         cudaStream_t stream) {
     dim3 grid(unsigned((N + kThreads - 1) / kThreads), unsigned(K / group));
-    group_scales_kernel<<<grid, kThreads, 0, stream>>>(w, K, N, group, s_g);
+    group_scales_kernel<<<grid, kThreads, 0, stream>>>(w, K, N, group, qmin == -8 ? 8.0f : 7.0f, s_g);
     return cudaGetLastError();
 }
 
@@ -168,9 +172,9 @@ cudaError_t amplifier(const float* scales, int64_t count, int32_t alpha_in, void
 }
 
 cudaError_t quantize_pack(const float* w, const float* s_g, int32_t alpha, int64_t K, int64_t N, int32_t group,
-                          uint8_t* packed, int16_t* S, void* workspace, cudaStream_t stream) {
+                          int32_t qmin, uint8_t* packed, int16_t* S, void* workspace, cudaStream_t stream) {
     dim3 grid(unsigned((N + kThreads - 1) / kThreads), unsigned(K / 32));
-    quantize_pack_kernel<<<grid, kThreads, 0, stream>>>(w, s_g, alpha, K, N, group, packed, S);
+    quantize_pack_kernel<<<grid, kThreads, 0, stream>>>(w, s_g, alpha, K, N, group, float(qmin), packed, S);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || S == nullptr) return e;
     auto* res = static_cast<Results*>(workspace);

@@ -134,6 +134,22 @@ W4A8_API w4a8_status pack_w4_groupwise(const float* w, int64_t K, int64_t N, int
                               int64_t* colsum_max_host, void* workspace, void* stream);
 
 /*
+ * pack_w4_groupwise with a choice of code range (极致量化 其他子4位整数格式:
+ * a signed N-bit integer holds [-2^(N-1), 2^(N-1) - 1]).
+ *   qmin = -7: s_g = max|w| / 7, codes clamp(rne(w / s_g), -7, 7)
+ *              (what pack_w4_groupwise does);
+ *   qmin = -8: s_g = max|w| / 8, codes clamp(rne(w / s_g), -8, 7): the full
+ *              two's-complement range; a group's positive extreme clips to 7.
+ * The overflow bound is then 127*8*group*colsum_max < 2^31.  The packed
+ * layout, alpha and S are as above; the GEMMs accept either range.
+ * Errors: as pack_w4_groupwise; W4A8_ERR_INVALID_ARG for any other qmin.
+ */
+W4A8_API w4a8_status pack_w4_groupwise_range(const float* w, int64_t K, int64_t N, int32_t group, int32_t alpha_in,
+                                    int32_t qmin, uint8_t* w_packed, float* s_g, int16_t* S,
+                                    int32_t* alpha_out_host, int64_t* colsum_max_host, void* workspace,
+                                    void* stream);
+
+/*
  * Bytes of workspace the GEMMs below need for (M, N, K, group) on the current
  * device (0 when they need none).  path: 0 integer scale, 1 float scale.
  * The workspace must be zero-filled before its first use.  Its first 4096

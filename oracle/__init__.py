@@ -12,6 +12,8 @@ they are plain definitions: the unquantized fp64 matmul ``x @ w`` used as the
 accuracy reference, and rounding an fp64 result to the output type.
 
 Parity status per function (what pins it, see tests/test_oracle_pins.py):
+  quantize_groups(qmin=-8)         brute-force nearest code in [-8, 7], the negative
+                                   extreme at -8, positive clipping, error bounds
   quantize_rows / quantize_groups  brute-force nearest-code search, tie cases,
                                    round-trip error bound |x - s q| <= s/2,
                                    error variance ~ s^2/12, hand-worked goldens
@@ -76,6 +78,7 @@ def _load():
             sig = {
                 "oracle_quantize_rows": ([P, I, I, I32, P, P], None),
                 "oracle_quantize_groups": ([P, I, I, I, I32, P, P], None),
+                "oracle_quantize_groups_full_range": ([P, I, I, I, P, P], None),
                 "oracle_pack_int4": ([P, I, I, P], None),
                 "oracle_alpha_sweep": ([P, P, I, I, I, P, I, P, P], None),
                 "oracle_unpack_int4": ([P, I, I, P], None),
@@ -122,15 +125,22 @@ def quantize_act_per_token(x):
     return quantize_rows(x, INT8_QMAX)
 
 
-def quantize_groups(w, group: int = 128, qmax: int = INT4_QMAX):
-    """Per-(group, column) symmetric quantization of w [K,N]: (q int8 [K,N], s_g float32 [K/group,N])."""
+def quantize_groups(w, group: int = 128, qmax: int = INT4_QMAX, qmin: int | None = None):
+    """Per-(group, column) symmetric quantization of w [K,N]: (q int8 [K,N], s_g float32 [K/group,N]).
+    qmin=None: codes in [-qmax, qmax], s = max|w| / qmax.  qmin=-8 (with qmax 7):
+    the full int4 range [-8, 7], s = max|w| / 8."""
     w = _c(w, np.float32)
     K, N = w.shape
     if K % group:
         raise ValueError("K must be a multiple of group")
     q = np.empty((K, N), np.int8)
     s = np.empty((K // group, N), np.float32)
-    _load().oracle_quantize_groups(_p(w), K, N, group, qmax, _p(q), _p(s))
+    if qmin is None or qmin == -qmax:
+        _load().oracle_quantize_groups(_p(w), K, N, group, qmax, _p(q), _p(s))
+    elif qmin == -8 and qmax == 7:
+        _load().oracle_quantize_groups_full_range(_p(w), K, N, group, _p(q), _p(s))
+    else:
+        raise ValueError(f"unsupported code range [{qmin}, {qmax}]")
     return q, s
 
 
@@ -270,15 +280,16 @@ def round_output(y, out: str):
 
 # ---------------------------------------------------------------- whole layer
 
-def linear_intscale(x, w, *, group: int = 128, alpha=1024, out: str = "f16"):
+def linear_intscale(x, w, *, group: int = 128, alpha=1024, out: str = "f16", qmin: int | None = None):
     """The whole Integer-Scale path on the CPU.
 
     alpha: an integer power of two, or None for the amplifier search.
+    qmin: None for weight codes in [-7, 7], -8 for the full int4 range.
     Returns a dict with every intermediate (codes, scales, packed bytes,
     integer scales, raw accumulators, fp64 and rounded outputs).
     """
     qx, s_a = quantize_act_per_token(x)
-    qw, s_g = quantize_groups(w, group)
+    qw, s_g = quantize_groups(w, group, qmin=qmin)
     a = amplifier_search(s_g) if alpha is None else int(alpha)
     S = integer_scales(s_g, a)
     acc = intscale_acc(qx, qw, S, group)

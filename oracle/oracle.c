@@ -98,6 +98,38 @@ void oracle_quantize_groups(const float* w, int64_t K, int64_t N, int64_t group,
     }
 }
 
+/* Per-group quantization over the full signed 4-bit range [-8, 7] ([X4]
+ * 其他子4位整数格式: a signed N-bit integer holds [-2^(N-1), 2^(N-1) - 1]).
+ * Reading: the scale divides the group's max |w| by 8, so the group's most
+ * negative extreme is code -8 and a positive extreme clips to 7:
+ * s_g = fl32(max|w| / 8), q = clip(rne(fl32(w / s_g)), -8, 7). */
+void oracle_quantize_groups_full_range(const float* w, int64_t K, int64_t N, int64_t group, int8_t* q,
+                                       float* s_g) {
+    int64_t G = K / group;
+    for (int64_t g = 0; g < G; ++g) {
+        for (int64_t n = 0; n < N; ++n) {
+            float a = 0.0f;
+            for (int64_t k = g * group; k < (g + 1) * group; ++k) {
+                float v = fabsf(w[k * N + n]);
+                if (v > a) a = v;
+            }
+            float sg = (a == 0.0f) ? 0.0f : symmetric_scale(a, 8);
+            s_g[g * N + n] = sg;
+            for (int64_t k = g * group; k < (g + 1) * group; ++k) {
+                int32_t c = 0;
+                if (sg != 0.0f) {
+                    volatile float t = w[k * N + n] / sg; /* one IEEE fp32 division */
+                    double r = rint((double)t);          /* round half to even */
+                    if (r > 7) r = 7;
+                    if (r < -8) r = -8;
+                    c = (int32_t)r;
+                }
+                q[k * N + n] = (int8_t)c;
+            }
+        }
+    }
+}
+
 /* ---- [X4] nibble packing -------------------------------------------------- */
 
 /* Layout (a reading: the pages only say that several low-bit values share one

@@ -116,6 +116,40 @@ def test_pack_bitexact(K, N, group, alpha):
     assert pk["colsum_max"] == oracle.scale_colsum_max(S)
 
 
+@pytest.mark.parametrize("K,N,group,alpha", [(1024, 1024, 128, 1024), (512, 264, 256, None)])
+def test_pack_full_range_bitexact(K, N, group, alpha):
+    """Weight codes over the full int4 range [-8, 7] (s_g = max|w| / 8)."""
+    dev = _dev()
+    wl = workloads.make_linear(1, K, N, seed=5 * K + N)
+    pk = bgq.pack_w4_groupwise(torch.from_numpy(wl.w).to(dev), group=group, alpha=alpha, qmin=-8)
+    qw, sg = oracle.quantize_groups(wl.w, group, qmin=-8)
+    assert qw.min() == -8  # the negative extremes use the extra code
+    a = oracle.amplifier_search(sg) if alpha is None else alpha
+    S = oracle.integer_scales(sg, a)
+    assert pk["alpha"] == a
+    assert np.array_equal(_bits(pk["s_g"].cpu().numpy()), _bits(sg))
+    assert np.array_equal(pk["packed"].cpu().numpy(), oracle.pack_int4(qw))
+    assert np.array_equal(pk["S"].cpu().numpy().astype(np.int32), S)
+
+
+@pytest.mark.parametrize("M,K,N", [(5, 512, 264), (130, 1024, 392)])
+def test_gemm_full_range_parity(M, K, N):
+    """The GEMMs with weight codes in [-8, 7]: raw accumulators bit-exact."""
+    dev = _dev()
+    wl = workloads.make_linear(M, K, N, x_dtype="bf16", seed=7 * M + K)
+    x = _to_dev_x(wl.x, wl.x_dtype, dev)
+    q, s = bgq.quantize_act_per_token(x)
+    pk = bgq.pack_w4_groupwise(torch.from_numpy(wl.w).to(dev), group=128, alpha=1024, qmin=-8)
+    ref = oracle.linear_intscale(wl.x, wl.w, group=128, alpha=1024, out="f32", qmin=-8)
+    acc = bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], pk["alpha"], group=128, out="i32")
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+    y = bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], pk["alpha"], group=128, out="f16")
+    _assert_close(y.float().cpu().numpy(), ref["y64"], "f16")
+    yf = bgq.w4a8_gemm_floatscale(q, s, pk["packed"], pk["s_g"], group=128, out="f32").cpu().numpy()
+    _assert_close(yf, oracle.floatscale(ref["qx"], ref["s_a"], ref["qw"], ref["s_g"], 128), "f32")
+    assert bgq.device_status() == 0
+
+
 def test_amplifier_search_device():
     dev = _dev()
     rng = np.random.default_rng(0)

@@ -490,3 +490,46 @@ def test_alpha_sweep_bit_counts():
     s = np.array([[256.0, 3.0]], np.float32)
     _, bits = oracle.alpha_sweep(q, s, [1], group=2)
     assert bits.tolist() == [9]
+
+
+# ------------------------------------------------------------- full int4 range [-8, 7]
+
+def _nearest_code_brute(t, lo, hi):
+    """Nearest integer code in [lo, hi] to t, ties to the even code."""
+    codes = np.arange(lo, hi + 1, dtype=np.int64)
+    d = np.abs(t[..., None].astype(np.float64) - codes)
+    nearest = d == d.min(axis=-1, keepdims=True)
+    nearest_even = nearest & (codes % 2 == 0)
+    idx = np.where(nearest_even.any(axis=-1), nearest_even.argmax(axis=-1), nearest.argmax(axis=-1))
+    return codes[idx]
+
+
+def test_full_range_codes_brute_force():
+    rng = np.random.default_rng(31)
+    w = (rng.standard_normal((256, 40)) * 0.02).astype(np.float32)
+    q, s = oracle.quantize_groups(w, 128, qmin=-8)
+    sg = np.repeat(s, 128, axis=0)
+    # the scale: one fp32 division of the group's max |w| by 8
+    amax = np.abs(w).reshape(2, 128, 40).max(axis=1).astype(np.float32)
+    assert np.array_equal(s, (amax / np.float32(8)).astype(np.float32))
+    t = (w / sg).astype(np.float32)
+    assert np.array_equal(q.astype(np.int64), _nearest_code_brute(t, -8, 7))
+    assert q.min() >= -8 and q.max() <= 7
+
+
+def test_full_range_extremes():
+    # group 0's extreme is negative: it maps to -8 exactly; group 1's is positive: it clips to 7
+    w = np.zeros((16, 1), np.float32)
+    w[:8, 0] = [0.1, -0.8, 0.3, 0.05, -0.2, 0.7, 0.0, 0.35]
+    w[8:, 0] = [0.8, -0.1, 0.3, 0.75, -0.7, 0.2, 0.0, -0.35]
+    q, s = oracle.quantize_groups(w, 8, qmin=-8)
+    assert s[0, 0] == np.float32(0.8) / np.float32(8) and s[1, 0] == np.float32(0.8) / np.float32(8)
+    assert q[1, 0] == -8 and q[8, 0] == 7 and q[11, 0] == 7  # 0.75 / 0.1 = 7.5 rounds to 8, clips to 7
+    err = np.abs(w[:, 0].astype(np.float64) - q[:, 0] * np.repeat(s[:, 0], 8).astype(np.float64))
+    sg = np.repeat(s[:, 0], 8).astype(np.float64)
+    inside = np.abs(w[:, 0] / np.repeat(s[:, 0], 8)) <= 7.5
+    assert np.all(err[inside] <= sg[inside] / 2 * (1 + 1e-6))
+    assert np.all(err[~inside] <= sg[~inside] * (1 + 1e-6))
+    # the default range never uses -8
+    q7, _ = oracle.quantize_groups(w, 8)
+    assert q7.min() >= -7
