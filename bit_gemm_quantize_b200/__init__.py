@@ -12,12 +12,14 @@ from ._native import (  # noqa: F401
     moe_workspace,
     pack_moe_experts,
     pack_w4_groupwise,
+    pack_w8_groupwise,
     quantize_act_per_token,
     w4a8_amplifier_search,
     w4a8_gemm_floatscale,
     w4a8_gemm_intscale,
     w4a8_gemm_intscale_static_ws,
     w4a8_moe_gemm_intscale,
+    w8a8_gemm_intscale,
 )
 
 __all__ = [
@@ -28,10 +30,12 @@ __all__ = [
     "moe_workspace",
     "pack_moe_experts",
     "pack_w4_groupwise",
+    "pack_w8_groupwise",
     "quantize_act_per_token",
     "w4a8_amplifier_search",
     "w4a8_gemm_floatscale",
     "w4a8_gemm_intscale",
     "w4a8_gemm_intscale_static_ws",
     "w4a8_moe_gemm_intscale",
+    "w8a8_gemm_intscale",
 ]

@@ -72,6 +72,8 @@ def load(path: str = LIB_PATH):
             "w4a8_amplifier_search": ([P, I64, P, P, P], I32_),
             "pack_w4_groupwise": ([P, I64, I64, I32_, I32_, P, P, P, P, P, P, P], I32_),
             "pack_w4_groupwise_range": ([P, I64, I64, I32_, I32_, I32_, P, P, P, P, P, P, P], I32_),
+            "pack_w8_groupwise": ([P, I64, I64, I32_, I32_, P, P, P, P, P, P, P], I32_),
+            "w8a8_gemm_intscale": ([P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
             "w4a8_gemm_workspace_size": ([I64, I64, I64, I32_, I32_], I64),
             "w4a8_gemm_intscale": ([P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
             "w4a8_gemm_intscale_static_ws": ([P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P], I32_),
@@ -206,6 +208,25 @@ def pack_w4_groupwise(w: torch.Tensor, group: int = 128, alpha: int | None = 102
     return dict(packed=packed, s_g=s_g, S=S, alpha=int(a_out.value), colsum_max=int(colsum.value))
 
 
+def pack_w8_groupwise(w: torch.Tensor, group: int = 128, alpha: int | None = None):
+    """Quantize fp32 weights w [K, N] to per-group 8-bit codes (W8A8).
+    alpha=None runs the search.  Returns dict(w8 [N, K] int8, s_g [K/group, N]
+    f32, S [K/group, N] int16, alpha, colsum_max)."""
+    _need_cuda("w", w, torch.float32, 2)
+    K, N = w.shape
+    dev = w.device
+    w8 = torch.empty((N, K), dtype=torch.int8, device=dev)
+    s_g = torch.empty((K // group, N), dtype=torch.float32, device=dev)
+    S = torch.empty((K // group, N), dtype=torch.int16, device=dev)
+    ws = torch.empty(PACK_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
+    a_out = ctypes.c_int32(0)
+    colsum = ctypes.c_int64(0)
+    code = load().pack_w8_groupwise(_ptr(w), K, N, group, 0 if alpha is None else int(alpha), _ptr(w8), _ptr(s_g),
+                                    _ptr(S), ctypes.byref(a_out), ctypes.byref(colsum), _ptr(ws), _stream(dev))
+    _check("pack_w8_groupwise", code)
+    return dict(w8=w8, s_g=s_g, S=S, alpha=int(a_out.value), colsum_max=int(colsum.value))
+
+
 _OUT = {"f32": (F32, torch.float32), "f16": (F16, torch.float16), "i32": (I32, torch.int32)}
 
 
@@ -236,6 +257,31 @@ def w4a8_gemm_intscale(q_x, s_a, w_packed, S, alpha: int, *, group: int = 128, o
     code = load().w4a8_gemm_intscale(_ptr(q_x), _ptr(s_a), _ptr(w_packed), _ptr(S), int(alpha), M, N, K, group,
                                      _ptr(y), dt, _ptr(workspace), ws_bytes, _stream(q_x.device))
     _check("w4a8_gemm_intscale", code)
+    return y
+
+
+def w8a8_gemm_intscale(q_x, s_a, w8, S, alpha: int, *, group: int = 128, out: str = "f16",
+                       y: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """y [M, N] = integer-scale W8A8 GEMM with 8-bit weight codes w8 [N, K]
+    (out: 'f16', 'f32' or 'i32' raw accumulators)."""
+    _need_cuda("q_x", q_x, torch.int8, 2)
+    _need_cuda("s_a", s_a, torch.float32, 1)
+    _need_cuda("w8", w8, torch.int8, 2)
+    N, K = w8.shape
+    M = q_x.shape[0]
+    if q_x.shape[1] != K or s_a.shape[0] != M:
+        raise ValueError("inconsistent GEMM operand shapes")
+    _need_cuda("S", S, torch.int16, 2)
+    dt, tdt = _OUT[out]
+    if y is None:
+        y = torch.empty((M, N), dtype=tdt, device=q_x.device)
+    _need_cuda("y", y, tdt, 2)
+    if workspace is None:
+        workspace = gemm_workspace(M, N, K, group, 2, q_x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = load().w8a8_gemm_intscale(_ptr(q_x), _ptr(s_a), _ptr(w8), _ptr(S), int(alpha), M, N, K, group, _ptr(y),
+                                     dt, _ptr(workspace), ws_bytes, _stream(q_x.device))
+    _check("w8a8_gemm_intscale", code)
     return y
 
 

@@ -146,7 +146,7 @@ w4a8_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int32_t group) {
 
 w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_t* w_packed, const int16_t* S,
                      const float* s_g, int32_t alpha, int64_t M, int64_t N, int64_t K, int32_t group, void* y,
-                     int32_t y_dtype, void* workspace, int64_t workspace_bytes, void* stream) {
+                     int32_t y_dtype, void* workspace, int64_t workspace_bytes, void* stream, bool w8 = false) {
     w4a8_status st = check_gemm_shape(M, N, K, group);
     if (st != W4A8_OK) return st;
     if (path == w4a8::gemm::kIntScale) {
@@ -163,7 +163,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
 
     DeviceInfo dev;
     if ((st = current_device(dev)) != W4A8_OK) return st;
-    const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms);
+    const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms, w8);
     if (pl.W >= (int64_t(1) << 31)) return W4A8_ERR_SHAPE;  // the kernel indexes (tile, group) steps in 32 bits
     int32_t* ws_count = nullptr;
     int32_t* ws_part = nullptr;
@@ -175,8 +175,9 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     }
 
     CUtensorMap tm_w, tm_x, tm_y;
-    // packed weights: one box = 128 columns x 128 bytes (two 128-wide K blocks), 128-byte swizzle
-    if (!make_map_u8(&tm_w, w_packed, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2),
+    // packed weights: one box = 128 columns x 128 bytes (two 128-wide K blocks), 128-byte swizzle;
+    // int8 weights: one box = 128 columns x 128 bytes (one K block)
+    if (!make_map_u8(&tm_w, w_packed, uint64_t(w8 ? K : K / 2), uint64_t(N), uint64_t(w8 ? K : K / 2),
                      uint32_t(w4a8::gemm::weight_box_bytes()), 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return W4A8_ERR_CUDA;
     if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(M), uint64_t(K), 128, uint32_t(pl.BT),
@@ -213,7 +214,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     p.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
     p.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
                                     : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
-    W4A8_CUDA_TRY(w4a8::gemm::launch(tm_w, tm_x, tm_y, p, pl.BT, path, static_cast<cudaStream_t>(stream)));
+    W4A8_CUDA_TRY(w4a8::gemm::launch(tm_w, tm_x, tm_y, p, pl.BT, path, static_cast<cudaStream_t>(stream), w8));
     return W4A8_OK;
 }
 
@@ -352,6 +353,40 @@ w4a8_status pack_w4_groupwise_range(const float* w, int64_t K, int64_t N, int32_
     return W4A8_OK;
 }
 
+w4a8_status pack_w8_groupwise(const float* w, int64_t K, int64_t N, int32_t group, int32_t alpha_in, int8_t* w8,
+                              float* s_g, int16_t* S, int32_t* alpha_out_host, int64_t* colsum_max_host,
+                              void* workspace, void* stream) {
+    if (K <= 0 || N <= 0 || group <= 0 || group % 32 != 0 || K % group != 0 || N % 8 != 0) return W4A8_ERR_SHAPE;
+    if (K > INT32_MAX || N > INT32_MAX || K / group > 65535 || K / 32 > 65535) return W4A8_ERR_SHAPE;
+    if (!w || !s_g || !w8 || !S || !alpha_out_host || !workspace) return W4A8_ERR_INVALID_ARG;
+    if (alpha_in < 0 || (alpha_in > 0 && (!is_pow2(alpha_in) || alpha_in > (1 << 30)))) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(s_g) || !aligned16(w8) || !aligned16(S) || !aligned16(workspace))
+        return W4A8_ERR_ALIGN;
+    DeviceInfo dev;
+    w4a8_status st = current_device(dev);
+    if (st != W4A8_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    W4A8_CUDA_TRY(w4a8::pack::group_scales_div(w, K, N, group, 127.0f, s_g, s));
+    const int64_t G = K / group;
+    W4A8_CUDA_TRY(w4a8::pack::amplifier(s_g, G * N, alpha_in, workspace, s, dev.sms));
+    w4a8::pack::Results r;
+    W4A8_CUDA_TRY(cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s));
+    W4A8_CUDA_TRY(cudaStreamSynchronize(s));
+    if (r.error) return W4A8_ERR_SCALE_RANGE;
+    if (std::nearbyint(double(r.s_max) * double(r.alpha)) > 32767.0) {
+        *alpha_out_host = r.alpha;
+        return W4A8_ERR_SCALE_RANGE;
+    }
+    W4A8_CUDA_TRY(w4a8::pack::quantize_w8(w, s_g, r.alpha, K, N, group, w8, S, workspace, s));
+    W4A8_CUDA_TRY(cudaMemcpyAsync(&r, workspace, sizeof(r), cudaMemcpyDeviceToHost, s));
+    W4A8_CUDA_TRY(cudaStreamSynchronize(s));
+    *alpha_out_host = r.alpha;
+    if (colsum_max_host) *colsum_max_host = int64_t(r.colsum_max);
+    const double bound = 127.0 * 127.0 * double(group) * double(r.colsum_max);
+    if (bound >= 2147483648.0) return W4A8_ERR_OVERFLOW_BOUND;
+    return W4A8_OK;
+}
+
 w4a8_status pack_w4_groupwise(const float* w, int64_t K, int64_t N, int32_t group, int32_t alpha_in,
                               uint8_t* w_packed, float* s_g, int16_t* S, int32_t* alpha_out_host,
                               int64_t* colsum_max_host, void* workspace, void* stream) {
@@ -360,11 +395,10 @@ w4a8_status pack_w4_groupwise(const float* w, int64_t K, int64_t N, int32_t grou
 }
 
 int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group, int32_t path) {
-    (void)path;
     if (check_gemm_shape(M, N, K, group) != W4A8_OK || M == 0) return 0;
     DeviceInfo dev;
     if (current_device(dev) != W4A8_OK) return -1;
-    const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms);
+    const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms, path == 2);
     return plan_splits_tiles(pl) ? pl.ws_bytes : 0;
 }
 
@@ -373,6 +407,13 @@ w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, const uint8_
                                int32_t y_dtype, void* workspace, int64_t workspace_bytes, void* stream) {
     return run_gemm(w4a8::gemm::kIntScale, q_x, s_a, w_packed, S, nullptr, alpha, M, N, K, group, y, y_dtype,
                     workspace, workspace_bytes, stream);
+}
+
+w4a8_status w8a8_gemm_intscale(const int8_t* q_x, const float* s_a, const int8_t* w8, const int16_t* S, int32_t alpha,
+                               int64_t M, int64_t N, int64_t K, int32_t group, void* y, int32_t y_dtype,
+                               void* workspace, int64_t workspace_bytes, void* stream) {
+    return run_gemm(w4a8::gemm::kIntScale, q_x, s_a, reinterpret_cast<const uint8_t*>(w8), S, nullptr, alpha, M, N,
+                    K, group, y, y_dtype, workspace, workspace_bytes, stream, true);
 }
 
 w4a8_status w4a8_gemm_intscale_static_ws(const int8_t* q_x, const float* s_a, const uint8_t* w_packed,

@@ -104,7 +104,11 @@ constexpr int64_t kMaxGrid = kCounterBytes / 4;
 #define W4A8_SX(BT) (W4A8_CTAS_PER_SM(BT) == 2 ? 3 : ((BT) <= 32 ? 6 : ((BT) == 64 ? 4 : 3)))
 #endif
 
-template <int BT, int PATH>
+// W8: 8-bit weight codes w8 [N, K] (the W8A8 variant).  The weight box then
+// is the MMA's A operand as it stands (read from shared memory through a
+// descriptor, like the token codes): no unpack, no TMEM operand slots, and
+// the weight slot is released by the stage's MMA commit.
+template <int BT, int PATH, bool W8 = false>
 struct Cfg {
     // warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-5 unpack
     // (four consecutive warps cover the four TMEM lane quarters), then the
@@ -119,20 +123,23 @@ struct Cfg {
     // TMEM (512 columns): kSA unpacked-operand slots of 64 columns, then kAcc
     // accumulator buffers of BT columns.  The MMA may run kAcc - 1 groups
     // ahead of the per-group drain.
-    static constexpr int kCtasPerSm = W4A8_CTAS_PER_SM(BT);
+    static constexpr bool kW8 = W8;
+    static constexpr int kCtasPerSm = W8 ? 1 : W4A8_CTAS_PER_SM(BT);
     static constexpr uint32_t kTmemCols = 512u / uint32_t(kCtasPerSm);  // TMEM columns of this CTA
-    static constexpr int kAcc = BT == 128 ? 3 : (BT == 64 ? 4 : 8);
-    static constexpr int kSA = (int(kTmemCols) - kAcc * BT) / kStageCols > 6 ? 6 : (int(kTmemCols) - kAcc * BT) / kStageCols;
+    static constexpr int kAcc = W8 ? (BT == 128 ? 4 : 8) : (BT == 128 ? 3 : (BT == 64 ? 4 : 8));
+    static constexpr int kSA = W8 ? 0
+                                  : ((int(kTmemCols) - kAcc * BT) / kStageCols > 6 ? 6
+                                                                                    : (int(kTmemCols) - kAcc * BT) / kStageCols);
     static constexpr uint32_t kAccCol0 = uint32_t(kSA * kStageCols);
-    static_assert(kSA >= 2 && kSA * kStageCols + kAcc * BT <= int(kTmemCols), "TMEM budget");
+    static_assert((W8 || kSA >= 2) && kSA * kStageCols + kAcc * BT <= int(kTmemCols), "TMEM budget");
     // Unpack to 16*q (nibble into the high half of each byte, 3 integer ops per
     // 8 weights) instead of q (7 ops).  The float-scale path folds the 1/16 into
     // s_g for free; the integer-scale path pays one shift per output per group
     // (P_g is 16 times the group product exactly).  With 128-token tiles the
     // drain's shifts (32 per 8 weights unpacked) outweigh the cheaper unpack,
     // so the integer path unpacks q exactly there.
-    static constexpr bool kX16 = (PATH == kFloatScale) || BT <= W4A8_X16_IS_MAX_BT;
-    static constexpr int kWBytes = kTileN * kStageK / 2;  // packed weights per stage: 16 KB
+    static constexpr bool kX16 = !W8 && ((PATH == kFloatScale) || BT <= W4A8_X16_IS_MAX_BT);
+    static constexpr int kWBytes = kTileN * kStageK / (W8 ? 1 : 2);  // weights per stage: 16 KB packed, 32 KB int8
     static constexpr int kXBytes = BT * kStageK;          // token codes per stage
     // Wide token tiles commit every group to its accumulator buffer, so the
     // epilogue drains a group while the MMAs of the next one run; narrow tiles
@@ -141,8 +148,8 @@ struct Cfg {
     // Narrow tiles read a split tile's single other partial when their
     // segment starts (registers to spare for it).
     static constexpr bool kEarlyCombine = BT <= 32;
-    static constexpr int kSW = W4A8_SW(BT);
-    static constexpr int kSX = W4A8_SX(BT);
+    static constexpr int kSW = W8 ? (BT == 128 ? 2 : (BT == 16 ? 6 : 4)) : W4A8_SW(BT);
+    static constexpr int kSX = W8 ? (BT <= 32 ? 6 : (BT == 64 ? 4 : 3)) : W4A8_SX(BT);
     // stage-done ring: one tcgen05.commit per stage, read by every role that
     // recycles a resource of that stage
     static constexpr int kSD = 16;
@@ -343,11 +350,11 @@ struct Ring {
     }
 };
 
-template <int BT, int PATH>
-__global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, Cfg<BT, PATH>::kCtasPerSm)
+template <int BT, int PATH, bool W8>
+__global__ void __launch_bounds__(Cfg<BT, PATH, W8>::kThreads, Cfg<BT, PATH, W8>::kCtasPerSm)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_y, const Params p) {
-    using C = Cfg<BT, PATH>;
+    using C = Cfg<BT, PATH, W8>;
     constexpr int kAcc = C::kAcc;
     constexpr int kU = C::kUnpackWarps;
     constexpr int SW = C::kSW, SX = C::kSX, SA = C::kSA, SD = C::kSD;
@@ -415,13 +422,24 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, Cfg<BT, PATH>::kCtasP
         // kernel may still be writing, can be read.
         Ring rw, rx;
         Ring rxd;          // stage-done slot of the stage whose token slot is reused (SX stages back)
+        Ring rwd;          // int8 weights: stage-done slot of the stage whose weight slot is reused (SW back)
         int32_t pst = 0;   // stages issued so far
         uint32_t w_issued = 0u, w_par = 0u, x_issued = 0u, x_par = 0u;  // per slot: copy issued / its parity
         auto issue_w = [&](const Stage& st, const Ring& slot) {
-            // one 128 x 128 B box = two K blocks (a lone last block over-reads 64 B per row: harmless)
-            mbar_arrive_expect_tx_one(&full_w[slot.idx], C::kWBytes);
-            tma_load_2d_one(smem + C::offW + slot.idx * C::kWBytes, &tm_w, st.kb * (kBlockK / 2),
-                            st.n_tile * kTileN, &full_w[slot.idx]);
+            if constexpr (C::kW8) {
+                // int8 weights: one 128-row x 128 B box per K block
+                uint8_t* dst = smem + C::offW + slot.idx * C::kWBytes;
+                mbar_arrive_expect_tx_one(&full_w[slot.idx], uint32_t(st.nkb * kTileN * kBlockK));
+                tma_load_2d_one(dst, &tm_w, st.kb * kBlockK, st.n_tile * kTileN, &full_w[slot.idx]);
+                if (st.nkb == 2)
+                    tma_load_2d_one(dst + kTileN * kBlockK, &tm_w, (st.kb + 1) * kBlockK, st.n_tile * kTileN,
+                                    &full_w[slot.idx]);
+            } else {
+                // one 128 x 128 B box = two K blocks (a lone last block over-reads 64 B per row: harmless)
+                mbar_arrive_expect_tx_one(&full_w[slot.idx], C::kWBytes);
+                tma_load_2d_one(smem + C::offW + slot.idx * C::kWBytes, &tm_w, st.kb * (kBlockK / 2),
+                                st.n_tile * kTileN, &full_w[slot.idx]);
+            }
             w_issued |= 1u << slot.idx;
             w_par = (w_par & ~(1u << slot.idx)) | (slot.phase << slot.idx);
         };
@@ -444,7 +462,15 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, Cfg<BT, PATH>::kCtasP
         while (ok && it.next(st)) {
             const int32_t m0 = st.m_tile * BT;
             if (pst >= prefetched) {
-                if (!mbar_wait_warp(&empty_w[rw.idx], rw.phase ^ 1u, abort_flag, p.status)) {
+                bool free_slot;
+                if constexpr (C::kW8) {
+                    // the MMAs of stage pst - SW have read this weight slot
+                    free_slot = pst < SW || mbar_wait_warp(&sdone[rwd.idx], rwd.phase, abort_flag, p.status);
+                    if (pst >= SW) rwd.advance(SD);
+                } else {
+                    free_slot = mbar_wait_warp(&empty_w[rw.idx], rw.phase ^ 1u, abort_flag, p.status);
+                }
+                if (!free_slot) {
                     ok = false;
                     break;
                 }
@@ -486,19 +512,24 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, Cfg<BT, PATH>::kCtasP
         // stage-done ring, which frees the operand slot and the token slot.
         constexpr uint32_t idesc = idesc_i8(kTileN, BT);
         Ring rx, ra, rt, rd;
+        Ring rw;  // int8 weights: the weight slot (the MMA's A operand in shared memory)
         StageIter it(p, b);
         Stage st;
         bool ok = true;
         int32_t kin = 0;  // position of the next K block inside its group (segments start on group boundaries)
         const uint32_t x_lo0 = smem_desc_sw128_lo(smem_u32(smem + C::offX));
+        const uint32_t w_lo0 = smem_desc_sw128_lo(smem_u32(smem + C::offW));
         while (ok && it.next(st)) {
-            if (!mbar_wait_warp(&full_a[ra.idx], ra.phase, abort_flag, p.status) ||
-                !mbar_wait_warp(&full_x[rx.idx], rx.phase, abort_flag, p.status)) {
+            // the A operand: the unpacked slot in TMEM, or the int8 weight box itself
+            const bool a_ready = C::kW8 ? mbar_wait_warp(&full_w[rw.idx], rw.phase, abort_flag, p.status)
+                                        : mbar_wait_warp(&full_a[ra.idx], ra.phase, abort_flag, p.status);
+            if (!a_ready || !mbar_wait_warp(&full_x[rx.idx], rx.phase, abort_flag, p.status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const uint32_t a_col = tmem_base + uint32_t(ra.idx * kStageCols);
+            const uint32_t w_lo = w_lo0 + uint32_t(rw.idx) * uint32_t(C::kWBytes >> 4);
             const uint32_t x_lo = x_lo0 + uint32_t(rx.idx) * uint32_t(C::kXBytes >> 4);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -514,12 +545,20 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, Cfg<BT, PATH>::kCtasP
                     tc_fence_after();
                 }
                 const uint32_t d = tmem_base + C::kAccCol0 + uint32_t(rt.idx * BT);
-                const uint32_t aj = a_col + uint32_t(j * (kBlockK / 4));
                 const uint32_t xj = x_lo + uint32_t(j * ((BT * kBlockK) >> 4));
+                if constexpr (C::kW8) {
+                    const uint32_t wj = w_lo + uint32_t(j * ((kTileN * kBlockK) >> 4));
 #pragma unroll
-                for (int k = 0; k < kBlockK / 32; ++k)  // 32 K per MMA: 8 TMEM columns of A, 2 descriptor units of B
-                    mma_i8_tmem_a_one(d, aj + uint32_t(8 * k), smem_desc_from_lo(xj + 2u * k), idesc,
+                    for (int k = 0; k < kBlockK / 32; ++k)  // 32 K per MMA: 2 descriptor units of A and of B
+                        mma_i8_ss_one(d, smem_desc_from_lo(wj + 2u * k), smem_desc_from_lo(xj + 2u * k), idesc,
                                       (first && k == 0) ? 0u : 1u);
+                } else {
+                    const uint32_t aj = a_col + uint32_t(j * (kBlockK / 4));
+#pragma unroll
+                    for (int k = 0; k < kBlockK / 32; ++k)  // 32 K per MMA: 8 TMEM columns of A, 2 descriptor units of B
+                        mma_i8_tmem_a_one(d, aj + uint32_t(8 * k), smem_desc_from_lo(xj + 2u * k), idesc,
+                                          (first && k == 0) ? 0u : 1u);
+                }
                 if (last) {
                     if constexpr (C::kGroupCommit) mma_commit_one(&afull[rt.idx]);
                     rt.advance(kAcc);
@@ -535,7 +574,10 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, Cfg<BT, PATH>::kCtasP
                 }
             }
             mma_commit_one(&sdone[rd.idx]);
-            ra.advance(SA);
+            if constexpr (C::kW8)
+                rw.advance(SW);
+            else
+                ra.advance(SA);
             rx.advance(SX);
             rd.advance(SD);
         }
@@ -544,6 +586,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, Cfg<BT, PATH>::kCtasP
         if (lane == 0) drain_wait(&mma_done[0], 0);
         __syncwarp();
     } else if (warp < C::kFirstEpiWarp) {
+      if constexpr (!C::kW8) {  // int8 weights need no unpack
         // ---------------------------------------------------------- int4 -> int8 unpack
         // Thread = weight row r of the tile = TMEM lane r.  Per stage it reads
         // its row's 128 packed bytes (eight 16-byte chunks; with the 128-byte
@@ -612,6 +655,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH>::kThreads, Cfg<BT, PATH>::kCtasP
             rw.advance(SW);
             ra.advance(SA);
         }
+      }
     } else {
         // ---------------------------------------------------------- epilogue
         griddep_wait();  // s_a, y and the workspace may be in use by the previous kernel
@@ -959,7 +1003,7 @@ static int token_tile_for(int64_t M) {
     return 128;
 }
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms) {
+Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool w8) {
     Plan pl{};
     pl.BT = token_tile_for(M);
     pl.n_tiles = (N + kTileN - 1) / kTileN;
@@ -967,7 +1011,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms) {
     pl.G = K / group;
     pl.tiles = pl.n_tiles * pl.m_tiles;
     pl.W = pl.tiles * pl.G;
-    const int64_t slots = int64_t(num_sms) * W4A8_CTAS_PER_SM(pl.BT);  // resident CTAs
+    const int64_t slots = int64_t(num_sms) * (w8 ? 1 : W4A8_CTAS_PER_SM(pl.BT));  // resident CTAs
     pl.grid = pl.W < slots ? pl.W : slots;
     if (pl.grid > kMaxGrid) pl.grid = kMaxGrid;
     const int64_t slot_bytes = int64_t(kTileN) * pl.BT * 4;
@@ -976,11 +1020,11 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms) {
     return pl;
 }
 
-template <int BT, int PATH>
+template <int BT, int PATH, bool W8 = false>
 static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty, const Params& p,
                              cudaStream_t stream) {
-    using C = Cfg<BT, PATH>;
-    auto kern = w4a8_gemm_kernel<BT, PATH>;
+    using C = Cfg<BT, PATH, W8>;
+    auto kern = w4a8_gemm_kernel<BT, PATH, W8>;
     const int smem = C::kSmemBytes;
     // the shared-memory opt-in is a per-device function attribute: set it once
     static bool configured[64] = {};
@@ -1001,7 +1045,15 @@ static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const
 }
 
 cudaError_t launch(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty, const Params& p, int BT, int path,
-                   cudaStream_t stream) {
+                   cudaStream_t stream, bool w8) {
+    if (w8) {  // int8 weights: the integer-scale path
+        switch (BT) {
+            case 16: return launch_bt<16, kIntScale, true>(tw, tx, ty, p, stream);
+            case 32: return launch_bt<32, kIntScale, true>(tw, tx, ty, p, stream);
+            case 64: return launch_bt<64, kIntScale, true>(tw, tx, ty, p, stream);
+            default: return launch_bt<128, kIntScale, true>(tw, tx, ty, p, stream);
+        }
+    }
     if (path == kIntScale) {
         switch (BT) {
             case 16: return launch_bt<16, kIntScale>(tw, tx, ty, p, stream);

@@ -38,14 +38,16 @@ struct Plan {
     int64_t ws_bytes;     // total workspace bytes
 };
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms);
+// w8: int8 weight codes (the W8A8 variant); its CTAs run one per SM
+Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool w8 = false);
 
 // tm_w: packed weights [N][K/2] u8, box 128 B x 128 rows, 128-byte swizzle
 // tm_x: token codes [M][K] u8, box 128 B x BT rows, 128-byte swizzle
 // tm_y: output y [M][N] (f16, f32 or i32 as Params::y_dtype), box 128 columns x BT rows
 // The group scales are read through Params::S / Params::s_g.
+// w8: tm_w covers int8 weights w8 [N][K] (box 128 B x 128 rows, 128-byte swizzle); integer-scale path only
 cudaError_t launch(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap& tm_y, const Params& p, int BT,
-                   int path, cudaStream_t stream);
+                   int path, cudaStream_t stream, bool w8 = false);
 
 int token_tile_rows();
 

@@ -67,11 +67,17 @@ constexpr int kMaxPartialBlocks = 4096;
 // [-8, 7], s = max|w| / 8)
 cudaError_t group_scales(const float* w, int64_t K, int64_t N, int32_t group, int32_t qmin, float* s_g,
                          cudaStream_t stream);
+// s_g = fl32(max|w| / qdiv) for any divisor (127 for 8-bit weight codes)
+cudaError_t group_scales_div(const float* w, int64_t K, int64_t N, int32_t group, float qdiv, float* s_g,
+                             cudaStream_t stream);
 // min / max reduction + amplifier search (alpha_in > 0: fixed amplifier)
 cudaError_t amplifier(const float* scales, int64_t count, int32_t alpha_in, void* workspace,
                       cudaStream_t stream, int num_sms);
 cudaError_t quantize_pack(const float* w, const float* s_g, int32_t alpha, int64_t K, int64_t N, int32_t group,
                           int32_t qmin, uint8_t* packed, int16_t* S, void* workspace, cudaStream_t stream);
+// 8-bit codes clip(rne(w / s_g), -127, 127) stored as w8 [N, K] int8, and S
+cudaError_t quantize_w8(const float* w, const float* s_g, int32_t alpha, int64_t K, int64_t N, int32_t group,
+                        int8_t* w8, int16_t* S, void* workspace, cudaStream_t stream);
 }  // namespace pack
 
 }  // namespace w4a8

@@ -131,6 +131,33 @@ __global__ void __launch_bounds__(kThreads) quantize_pack_kernel(const float* __
     if (S != nullptr && (k0 % group) == 0) S[g * N + n] = int16_t(rintf(s * float(alpha)));  // s * alpha exact
 }
 
+// 8-bit weight codes (the W8A8 variant): q = clip(rne(fl32(w / s_g)), -127, 127)
+// with s_g = max|w| / 127, stored K-contiguous per column, w8[n, k].  One
+// thread per column n and 32-wide K chunk, 32 bytes written per thread.
+__global__ void __launch_bounds__(kThreads) quantize_w8_kernel(const float* __restrict__ w,
+                                                               const float* __restrict__ s_g, int32_t alpha,
+                                                               int64_t K, int64_t N, int32_t group,
+                                                               int8_t* __restrict__ w8, int16_t* __restrict__ S) {
+    const int64_t n = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    const int64_t k0 = int64_t(blockIdx.y) * 32;
+    if (n >= N) return;
+    const int64_t g = k0 / group;
+    const float s = s_g[g * N + n];
+    uint32_t words[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    if (s != 0.0f) {
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) {
+            const float t = __fdiv_rn(w[(k0 + i) * N + n], s);
+            const float r = fminf(fmaxf(rintf(t), -127.0f), 127.0f);
+            words[i >> 2] |= (uint32_t(int(r)) & 0xFFu) << (8 * (i & 3));
+        }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(w8 + n * K + k0);
+    dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+    dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+    if (S != nullptr && (k0 % group) == 0) S[g * N + n] = int16_t(rintf(s * float(alpha)));  // s * alpha exact
+}
+
 // max over columns of sum_g |S[g, n]|.
 __global__ void __launch_bounds__(kThreads) colsum_kernel(const int16_t* __restrict__ S, int64_t G, int64_t N,
                                                           unsigned long long* __restrict__ out) {
@@ -151,8 +178,13 @@ __global__ void __launch_bounds__(kThreads) colsum_kernel(const int16_t* __restr
 
 cudaError_t group_scales(const float* w, int64_t K, int64_t N, int32_t group, int32_t qmin, float* s_g,
                          cudaStream_t stream) {
+    return group_scales_div(w, K, N, group, qmin == -8 ? 8.0f : 7.0f, s_g, stream);
+}
+
+cudaError_t group_scales_div(const float* w, int64_t K, int64_t N, int32_t group, float qdiv, float* s_g,
+                             cudaStream_t stream) {
     dim3 grid(unsigned((N + kThreads - 1) / kThreads), unsigned(K / group));
-    group_scales_kernel<<<grid, kThreads, 0, stream>>>(w, K, N, group, qmin == -8 ? 8.0f : 7.0f, s_g);
+    group_scales_kernel<<<grid, kThreads, 0, stream>>>(w, K, N, group, qdiv, s_g);
     return cudaGetLastError();
 }
 
@@ -168,6 +200,18 @@ cudaError_t amplifier(const float* scales, int64_t count, int32_t alpha_in, void
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     amplifier_kernel<<<1, 32, 0, stream>>>(partial, int(blocks), alpha_in, res);
+    return cudaGetLastError();
+}
+
+cudaError_t quantize_w8(const float* w, const float* s_g, int32_t alpha, int64_t K, int64_t N, int32_t group,
+                       int8_t* w8, int16_t* S, void* workspace, cudaStream_t stream) {
+    dim3 grid(unsigned((N + kThreads - 1) / kThreads), unsigned(K / 32));
+    quantize_w8_kernel<<<grid, kThreads, 0, stream>>>(w, s_g, alpha, K, N, group, w8, S);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || S == nullptr) return e;
+    auto* res = static_cast<Results*>(workspace);
+    colsum_kernel<<<unsigned((N + kThreads - 1) / kThreads), kThreads, 0, stream>>>(S, K / group, N,
+                                                                                   &res->colsum_max);
     return cudaGetLastError();
 }
 

@@ -150,8 +150,31 @@ W4A8_API w4a8_status pack_w4_groupwise_range(const float* w, int64_t K, int64_t 
                                     void* stream);
 
 /*
+ * Fine-grained W8A8 weights (the pages' W8A8 configurations, Integer Scale
+ * summary §5, with the same integer group scales): per-group symmetric 8-bit
+ * weight codes, amplifier and integer scales (synchronous like
+ * pack_w4_groupwise).
+ *   s_g[g,n]  = fl32(max_{k in g} |w[k,n]| / 127)
+ *   q_w[k,n]  = clamp(rne(fl32(w[k,n] / s_g[g(k),n])), -127, 127)
+ *   w8[n, k]  = q_w[k,n]        (int8, K-contiguous per output column)
+ *   alpha, S  as in pack_w4_groupwise
+ * w          device, [K, N] float32
+ * K, N       K % group == 0, N % 8 == 0, N > 0; group % 32 == 0
+ * w8         device, [N, K] int8, written
+ * s_g        device, [K/group, N] float32, written
+ * S          device, [K/group, N] int16, written
+ * alpha_out_host, colsum_max_host, workspace: as in pack_w4_groupwise
+ * Errors: W4A8_ERR_SCALE_RANGE if max S > 32767; W4A8_ERR_OVERFLOW_BOUND if
+ * 127*127*group*colsum_max >= 2^31 (outputs are written in both cases).
+ */
+W4A8_API w4a8_status pack_w8_groupwise(const float* w, int64_t K, int64_t N, int32_t group, int32_t alpha_in,
+                              int8_t* w8, float* s_g, int16_t* S, int32_t* alpha_out_host,
+                              int64_t* colsum_max_host, void* workspace, void* stream);
+
+/*
  * Bytes of workspace the GEMMs below need for (M, N, K, group) on the current
- * device (0 when they need none).  path: 0 integer scale, 1 float scale.
+ * device (0 when they need none).  path: 0 integer scale, 1 float scale,
+ * 2 the W8A8 integer-scale GEMM.
  * The workspace must be zero-filled before its first use.  Its first 4096
  * bytes hold arrival counters that every successful call leaves at zero
  * again (the rest is scratch), so one allocation of the largest size needed
@@ -184,6 +207,19 @@ W4A8_API w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, con
                                const int16_t* S, int32_t alpha, int64_t M, int64_t N, int64_t K,
                                int32_t group, void* y, int32_t y_dtype, void* workspace,
                                int64_t workspace_bytes, void* stream);
+
+/*
+ * W8A8 GEMM with integer group scales: the integer-scale GEMM above with
+ * 8-bit weight codes w8 [N, K] int8 (from pack_w8_groupwise) instead of packed
+ * int4.  acc[m,n] = sum_g S[g,n] * P_g[m,n] in int32 with
+ * P_g[m,n] = sum_{k in g} q_x[m,k] * w8[n,k]; y = acc * s_a[m] / alpha.
+ * Arguments, precondition (now 127*127*group*max_n sum_g |S[g,n]| < 2^31),
+ * workspace (w4a8_gemm_workspace_size with path 2), output and errors as in
+ * w4a8_gemm_intscale.
+ */
+W4A8_API w4a8_status w8a8_gemm_intscale(const int8_t* q_x, const float* s_a, const int8_t* w8, const int16_t* S,
+                               int32_t alpha, int64_t M, int64_t N, int64_t K, int32_t group, void* y,
+                               int32_t y_dtype, void* workspace, int64_t workspace_bytes, void* stream);
 
 /*
  * The integer-scale GEMM above with its workspace in a fixed device array of

@@ -280,21 +280,28 @@ def round_output(y, out: str):
 
 # ---------------------------------------------------------------- whole layer
 
-def linear_intscale(x, w, *, group: int = 128, alpha=1024, out: str = "f16", qmin: int | None = None):
+def linear_intscale(x, w, *, group: int = 128, alpha=1024, out: str = "f16", qmin: int | None = None,
+                    wbits: int = 4):
     """The whole Integer-Scale path on the CPU.
 
     alpha: an integer power of two, or None for the amplifier search.
     qmin: None for weight codes in [-7, 7], -8 for the full int4 range.
+    wbits: 4 (int4 codes, nibble-packed) or 8 (W8A8: codes in [-127, 127],
+    s_g = max|w| / 127, 'packed' is then the int8 layout w8 [N, K]).
     Returns a dict with every intermediate (codes, scales, packed bytes,
     integer scales, raw accumulators, fp64 and rounded outputs).
     """
     qx, s_a = quantize_act_per_token(x)
-    qw, s_g = quantize_groups(w, group, qmin=qmin)
+    if wbits == 8:
+        qw, s_g = quantize_groups(w, group, qmax=INT8_QMAX)
+    else:
+        qw, s_g = quantize_groups(w, group, qmin=qmin)
     a = amplifier_search(s_g) if alpha is None else int(alpha)
     S = integer_scales(s_g, a)
     acc = intscale_acc(qx, qw, S, group)
     y64 = intscale_output(acc, s_a, a)
-    return dict(qx=qx, s_a=s_a, qw=qw, s_g=s_g, packed=pack_int4(qw), alpha=a, S=S, acc=acc,
+    packed = np.ascontiguousarray(qw.T) if wbits == 8 else pack_int4(qw)
+    return dict(qx=qx, s_a=s_a, qw=qw, s_g=s_g, packed=packed, alpha=a, S=S, acc=acc,
                 y64=y64, y=round_output(y64, out))
 
 

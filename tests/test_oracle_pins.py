@@ -533,3 +533,29 @@ def test_full_range_extremes():
     # the default range never uses -8
     q7, _ = oracle.quantize_groups(w, 8)
     assert q7.min() >= -7
+
+
+# ------------------------------------------------------------- 8-bit weight codes (W8A8)
+
+def test_groups_qmax127_brute_force():
+    rng = np.random.default_rng(41)
+    w = (rng.standard_normal((256, 24)) * 0.02).astype(np.float32)
+    q, s = oracle.quantize_groups(w, 128, qmax=127)
+    amax = np.abs(w).reshape(2, 128, 24).max(axis=1).astype(np.float32)
+    assert np.array_equal(s, (amax / np.float32(127)).astype(np.float32))
+    t = (w / np.repeat(s, 128, axis=0)).astype(np.float32)
+    assert np.array_equal(q.astype(np.int64), _nearest_code_brute(t, -127, 127))
+    # every group's extreme reaches +-127
+    assert np.array_equal(np.abs(q).reshape(2, 128, 24).max(axis=1), np.full((2, 24), 127))
+
+
+def test_linear_w8a8_layout_and_accumulators():
+    rng = np.random.default_rng(42)
+    x = rng.standard_normal((3, 256)).astype(np.float32)
+    w = (rng.standard_normal((256, 16)) * 0.02).astype(np.float32)
+    r = oracle.linear_intscale(x, w, group=128, alpha=4096, wbits=8, out="f32")
+    assert r["packed"].shape == (16, 256) and r["packed"].dtype == np.int8
+    assert np.array_equal(r["packed"], r["qw"].T)
+    # the accumulators equal the dense int64 product with the integer weights W_int = S * q
+    Wint = np.repeat(r["S"].astype(np.int64), 128, axis=0) * r["qw"].astype(np.int64)
+    assert np.array_equal(r["acc"], r["qx"].astype(np.int64) @ Wint)
