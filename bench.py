@@ -345,6 +345,66 @@ def measure_prefill(dev, rank, world, int8_peak, reps=10):
             "timing": "CUDA events around graph replays of quantize + integer-scale GEMM, the two layers alternating"}
 
 
+W8A8 = dict(K=4096, N=22016, M=[1, 32, 1024])
+
+
+def measure_w8a8(dev, rank, world, hbm_peak, int8_peak, reps=7):
+    """The W8A8 variant on the FFN up-projection shape: 8-bit weight codes with
+    integer group scales (alpha from the search), per-launch time of the GEMM
+    from graphs of six launches alternating two weight copies (90 MB each, so
+    every launch streams its weights from HBM).  Inputs drawn on the device."""
+    import torch
+
+    import bit_gemm_quantize_b200 as bgq
+
+    K, N = W8A8["K"], W8A8["N"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(5000 + rank)
+    w = torch.randn((K, N), generator=g, device=dev)
+    w.mul_(0.02)
+    pk = bgq.pack_w8_groupwise(w, group=GROUP, alpha=None)
+    del w
+    copies = [pk["w8"], pk["w8"].clone()]
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    for M in W8A8["M"]:
+        x = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
+        q, s = bgq.quantize_act_per_token(x)
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        wsp = bgq.gemm_workspace(M, N, K, GROUP, 2, dev)
+
+        def call(i):
+            bgq.w8a8_gemm_intscale(q, s, copies[i % 2], pk["S"], pk["alpha"], group=GROUP, out="f16", y=y,
+                                   workspace=wsp)
+
+        for i in range(3):
+            call(i)
+        torch.cuda.synchronize(dev)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            for i in range(6):
+                call(i)
+        gr.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(reps):
+            gr.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = max_over_ranks([e0.elapsed_time(e1) / (6 * reps)], world, dev)[0]
+        del gr
+        bytes_ = N * K + 2 * (K // GROUP) * N + M * K + 4 * M + 2 * M * N
+        ops = 2.0 * M * N * K
+        t = ms * 1e-3
+        gbs, tops = bytes_ / t / 1e9, ops / t / 1e12
+        bound = "hbm" if bytes_ / (hbm_peak * 1e9) >= ops / (int8_peak * 1e12) else "tensor"
+        rows.append({"M": M, "us": round(ms * 1e3, 2), "tops": round(tops, 2), "gbs": round(gbs, 1), "bound": bound,
+                     "frac": round(gbs / hbm_peak if bound == "hbm" else tops / int8_peak, 4)})
+    return {"workload": "w8a8_ffn_up", "K": K, "N": N, "group": GROUP, "alpha": pk["alpha"], "rows": rows,
+            "timing": "CUDA events over graphs of six launches alternating two 90 MB weight copies"}
+
+
 # ---------------------------------------------------------------- rank aggregation
 
 def max_over_ranks(times_ms, world, device):
@@ -585,6 +645,7 @@ def run_ours(args):
 
     moe = measure_moe(dev, rank, world, int8_peak)
     prefill = measure_prefill(dev, rank, world, int8_peak)
+    w8a8 = measure_w8a8(dev, rank, world, hbm_peak, int8_peak)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
@@ -595,6 +656,7 @@ def run_ours(args):
         "gpu_launches": 2 * len(SWEEP) * args.steps,
         "moe": moe,
         "prefill": prefill,
+        "w8a8": w8a8,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample()
