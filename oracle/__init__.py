@@ -12,6 +12,13 @@ they are plain definitions: the unquantized fp64 matmul ``x @ w`` used as the
 accuracy reference, and rounding an fp64 result to the output type.
 
 Parity status per function (what pins it, see tests/test_oracle_pins.py):
+  quantize_rows_asym               hand-worked golden row, brute-force nearest code on
+                                   the grid s (q - z), zero exactly representable,
+                                   |x - s (q - z)| <= s/2 on rows spanning zero, the
+                                   range ends at the extreme codes, constant rows
+  intscale_acc_asym                equals intscale_acc when z = 0; equals the expanded
+                                   form q_W q_X - Z_X q_W (numpy int64); brute fp64
+                                   dequantized matmul on tiny inputs
   quantize_groups(qmin=-8)         brute-force nearest code in [-8, 7], the negative
                                    extreme at -8, positive clipping, error bounds
   quantize_rows / quantize_groups  brute-force nearest-code search, tie cases,
@@ -53,6 +60,8 @@ _lib = None
 
 INT8_QMAX = 127
 INT4_QMAX = 7
+INT8_ASYM_QMIN = -128
+INT8_ASYM_QMAX = 127
 
 
 def build(force: bool = False) -> str:
@@ -77,6 +86,7 @@ def _load():
             I32 = ctypes.c_int32
             sig = {
                 "oracle_quantize_rows": ([P, I, I, I32, P, P], None),
+                "oracle_quantize_rows_asym": ([P, I, I, I32, I32, P, P, P], None),
                 "oracle_quantize_groups": ([P, I, I, I, I32, P, P], None),
                 "oracle_quantize_groups_full_range": ([P, I, I, I, P, P], None),
                 "oracle_pack_int4": ([P, I, I, P], None),
@@ -87,6 +97,7 @@ def _load():
                 "oracle_intscale_acc": ([P, P, P, I, I, I, I, P], None),
                 "oracle_intscale_acc_expanded": ([P, P, P, I, I, I, I, P], None),
                 "oracle_intscale_acc_at": ([P, P, P, I, I, I, I, P, P, I, P], None),
+                "oracle_intscale_acc_asym": ([P, P, P, P, I, I, I, I, P], None),
                 "oracle_intscale_output": ([P, P, I32, I, I, P], None),
                 "oracle_floatscale": ([P, P, P, P, I, I, I, I, P], None),
                 "oracle_floatscale_at": ([P, P, P, P, I, I, I, I, P, P, I, P], None),
@@ -123,6 +134,22 @@ def quantize_rows(x, qmax: int = INT8_QMAX):
 def quantize_act_per_token(x):
     """Per-token int8 activation codes and scales (qmax = 127)."""
     return quantize_rows(x, INT8_QMAX)
+
+
+def quantize_rows_asym(x, qmin: int = INT8_ASYM_QMIN, qmax: int = INT8_ASYM_QMAX):
+    """Per-row asymmetric quantization: returns (q int8 [R,C], s float32 [R], z int32 [R])."""
+    x = _c(x, np.float32)
+    R, C = x.shape
+    q = np.empty((R, C), np.int8)
+    s = np.empty(R, np.float32)
+    z = np.empty(R, np.int32)
+    _load().oracle_quantize_rows_asym(_p(x), R, C, int(qmin), int(qmax), _p(q), _p(s), _p(z))
+    return q, s, z
+
+
+def quantize_act_per_token_asym(x):
+    """Per-token asymmetric int8 activation codes in [-128, 127], scales and zero points."""
+    return quantize_rows_asym(x, INT8_ASYM_QMIN, INT8_ASYM_QMAX)
 
 
 def quantize_groups(w, group: int = 128, qmax: int = INT4_QMAX, qmin: int | None = None):
@@ -234,6 +261,18 @@ def intscale_acc_at(qx, qw, S, ms, ns, group: int = 128):
     return acc
 
 
+def intscale_acc_asym(qx, z, qw, S, group: int = 128):
+    qx = _c(qx, np.int8)
+    z = _c(z, np.int32)
+    qw = _c(qw, np.int8)
+    S = _c(S, np.int32)
+    M, K = qx.shape
+    N = qw.shape[1]
+    acc = np.empty((M, N), np.int64)
+    _load().oracle_intscale_acc_asym(_p(qx), _p(z), _p(qw), _p(S), M, N, K, group, _p(acc))
+    return acc
+
+
 def intscale_output(acc, s_a, alpha: int):
     acc = _c(acc, np.int64)
     s_a = _c(s_a, np.float32)
@@ -281,27 +320,33 @@ def round_output(y, out: str):
 # ---------------------------------------------------------------- whole layer
 
 def linear_intscale(x, w, *, group: int = 128, alpha=1024, out: str = "f16", qmin: int | None = None,
-                    wbits: int = 4):
+                    wbits: int = 4, asym: bool = False):
     """The whole Integer-Scale path on the CPU.
 
     alpha: an integer power of two, or None for the amplifier search.
     qmin: None for weight codes in [-7, 7], -8 for the full int4 range.
     wbits: 4 (int4 codes, nibble-packed) or 8 (W8A8: codes in [-127, 127],
     s_g = max|w| / 127, 'packed' is then the int8 layout w8 [N, K]).
-    Returns a dict with every intermediate (codes, scales, packed bytes,
-    integer scales, raw accumulators, fp64 and rounded outputs).
+    asym: asymmetric per-token activations (codes in [-128, 127] with a zero
+    point z per token; the accumulator is then sum_g S sum_k (qx - z) qw).
+    Returns a dict with every intermediate (codes, scales, zero points, packed
+    bytes, integer scales, raw accumulators, fp64 and rounded outputs).
     """
-    qx, s_a = quantize_act_per_token(x)
+    if asym:
+        qx, s_a, z = quantize_act_per_token_asym(x)
+    else:
+        qx, s_a = quantize_act_per_token(x)
+        z = np.zeros(qx.shape[0], np.int32)
     if wbits == 8:
         qw, s_g = quantize_groups(w, group, qmax=INT8_QMAX)
     else:
         qw, s_g = quantize_groups(w, group, qmin=qmin)
     a = amplifier_search(s_g) if alpha is None else int(alpha)
     S = integer_scales(s_g, a)
-    acc = intscale_acc(qx, qw, S, group)
+    acc = intscale_acc_asym(qx, z, qw, S, group) if asym else intscale_acc(qx, qw, S, group)
     y64 = intscale_output(acc, s_a, a)
     packed = np.ascontiguousarray(qw.T) if wbits == 8 else pack_int4(qw)
-    return dict(qx=qx, s_a=s_a, qw=qw, s_g=s_g, packed=packed, alpha=a, S=S, acc=acc,
+    return dict(qx=qx, s_a=s_a, z=z, qw=qw, s_g=s_g, packed=packed, alpha=a, S=S, acc=acc,
                 y64=y64, y=round_output(y64, out))
 
 

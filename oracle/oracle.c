@@ -13,8 +13,12 @@
  *  [Q]  "Quantization" notes, sections "量化公式" and "Symmetric Quantization":
  *       q = clip(round(x/s) + z, qmin, qmax); x_hat = s (q - z); symmetric:
  *       alpha = max|x|, s = alpha / qmax, z = 0, q in [-qmax, qmax], int8 qmax = 127.
+ *  [Q-asym] same notes, "Asymmetric Quantization": the range [x_min, x_max]
+ *       maps onto [qmin, qmax], s = (x_max - x_min) / (qmax - qmin),
+ *       z = clip(round(qmin - x_min / s), qmin, qmax), q = clip(round(x / s) + z).
  *  [Q-mm] same notes, "矩阵乘法中的量化计算": with z = 0 on both operands the
- *       integer part of a quantized matmul is q_W q_X alone.
+ *       integer part of a quantized matmul is q_W q_X alone; with Z_W = 0 and an
+ *       activation zero point it is (q_X - Z_X) q_W.
  *  [T34] "探秘Transformer系列之（34）量化基礎", §2.2.1 eqs. (1)-(2) and "Scale
  *       Quantization" (int8 symmetric range [-127, 127]); §2.3.3 "逐组量化"
  *       (one scale per group of K consecutive inputs of a weight column) and
@@ -73,6 +77,53 @@ void oracle_quantize_rows(const float* x, int64_t rows, int64_t cols, int32_t qm
         float sm = (a == 0.0f) ? 0.0f : symmetric_scale(a, qmax);
         s[m] = sm;
         for (int64_t k = 0; k < cols; ++k) q[m * cols + k] = (int8_t)symmetric_code(xr[k], sm, qmax);
+    }
+}
+
+/* Per-row asymmetric quantization of x [rows, cols] ([Q-asym]; one scale and
+ * one zero point per token row as in [T34] 逐token量化).  Each step is one IEEE
+ * fp32 operation: d = x_max - x_min, s = d / (qmax - qmin), t = x_min / s,
+ * u = qmin - t, z = clip(rint(u)), and per element q = clip(rint(x / s) + z).
+ * Readings where the notes are silent: round() is half to even; a constant
+ * row (x_max = x_min) has an empty range, which is widened to include zero
+ * (so a constant c is reconstructed to within the rounding of s); a row whose
+ * scale is 0 (all zeros, or a range too small for an fp32 scale) gets z = 0
+ * and codes 0.  The clip of z acts only when the range excludes zero. */
+void oracle_quantize_rows_asym(const float* x, int64_t rows, int64_t cols, int32_t qmin, int32_t qmax,
+                               int8_t* q, float* s, int32_t* z) {
+    for (int64_t m = 0; m < rows; ++m) {
+        const float* xr = x + m * cols;
+        float lo = xr[0], hi = xr[0];
+        for (int64_t k = 1; k < cols; ++k) {
+            if (xr[k] < lo) lo = xr[k];
+            if (xr[k] > hi) hi = xr[k];
+        }
+        if (hi == lo) {
+            if (lo > 0.0f) lo = 0.0f;
+            if (hi < 0.0f) hi = 0.0f;
+        }
+        volatile float d = hi - lo;
+        volatile float sm = d / (float)(qmax - qmin);
+        s[m] = sm;
+        if (sm == 0.0f) {
+            z[m] = 0;
+            for (int64_t k = 0; k < cols; ++k) q[m * cols + k] = 0;
+            continue;
+        }
+        volatile float t = lo / sm;
+        volatile float u = (float)qmin - t;
+        double zr = rint((double)u);
+        if (zr < qmin) zr = qmin;
+        if (zr > qmax) zr = qmax;
+        const int32_t zm = (int32_t)zr;
+        z[m] = zm;
+        for (int64_t k = 0; k < cols; ++k) {
+            volatile float v = xr[k] / sm;
+            double r = rint((double)v) + (double)zm;
+            if (r < qmin) r = qmin;
+            if (r > qmax) r = qmax;
+            q[m * cols + k] = (int8_t)r;
+        }
     }
 }
 
@@ -248,6 +299,26 @@ void oracle_intscale_acc_at(const int8_t* qx, const int8_t* qw, const int32_t* S
         }
         acc[i] = total;
     }
+}
+
+/* Integer-scale accumulation with an asymmetric activation ([Q-mm] with
+ * Z_W = 0 and Z_X = z[m]; [IS] §4 integer group scales):
+ * acc[m,n] = sum_g S[g,n] * sum_{k in g} (qx[m,k] - z[m]) * qw[k,n].
+ * The final rescale is the same as the symmetric one, acc * s_a[m] / alpha. */
+void oracle_intscale_acc_asym(const int8_t* qx, const int32_t* z, const int8_t* qw, const int32_t* S,
+                              int64_t M, int64_t N, int64_t K, int64_t group, int64_t* acc) {
+    int64_t G = K / group;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t total = 0;
+            for (int64_t g = 0; g < G; ++g) {
+                int64_t p = 0;
+                for (int64_t k = g * group; k < (g + 1) * group; ++k)
+                    p += ((int64_t)qx[m * K + k] - (int64_t)z[m]) * (int64_t)qw[k * N + n];
+                total += (int64_t)S[g * N + n] * p;
+            }
+            acc[m * N + n] = total;
+        }
 }
 
 /* Final rescale, once per output: y = acc * s_a[m] / alpha, in fp64 ([IS] §4). */

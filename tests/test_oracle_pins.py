@@ -559,3 +559,125 @@ def test_linear_w8a8_layout_and_accumulators():
     # the accumulators equal the dense int64 product with the integer weights W_int = S * q
     Wint = np.repeat(r["S"].astype(np.int64), 128, axis=0) * r["qw"].astype(np.int64)
     assert np.array_equal(r["acc"], r["qx"].astype(np.int64) @ Wint)
+
+
+# ------------------------------------------------------------- asymmetric activations
+
+def test_asym_golden_rows():
+    g = _golden("quantize_int8_asymmetric.json")
+    for case in g["cases"]:
+        q, s, z = oracle.quantize_act_per_token_asym(np.array([case["x"]], np.float32))
+        assert q[0].tolist() == case["q"], case["derivation"]
+        assert _bits(s[0]) == int(case["s_bits"], 16), case["derivation"]
+        assert int(z[0]) == case["z"], case["derivation"]
+
+
+def _skewed_rows(rng, R, C, shift):
+    x = rng.standard_normal((R, C)).astype(np.float32) + np.float32(shift)
+    x[:, rng.choice(C, 3, replace=False)] *= np.float32(20)
+    x[:, 0] = 0.0  # every row spans zero
+    x[:, 1] = -abs(x[:, 1]) - 0.1
+    return x
+
+
+def test_asym_codes_are_the_nearest_grid_points():
+    """Each code is the nearest integer of x/s + z in [-128, 127] (ties to
+    even), searched by brute force; the scale is the range over 255 to within
+    the one fp32 rounding of each step, and z is within 1/2 of the real-valued
+    zero point -128 - x_min / s."""
+    rng = np.random.default_rng(51)
+    x = _skewed_rows(rng, 12, 384, 1.5)
+    q, s, z = oracle.quantize_act_per_token_asym(x)
+    lo = x.min(axis=1).astype(np.float64)
+    hi = x.max(axis=1).astype(np.float64)
+    assert np.all(np.abs(s - (hi - lo) / 255) <= 2 * np.spacing(s))
+    zr = -128 - lo / s.astype(np.float64)
+    assert np.all(np.abs(z - zr) <= 0.5 + 1e-4)
+    t = (x / s[:, None]).astype(np.float32).astype(np.float64) + z[:, None]
+    assert np.array_equal(q.astype(np.int64), _nearest_code_brute(t, -128, 127))
+
+
+def test_asym_zero_exact_extremes_and_error_bound():
+    rng = np.random.default_rng(52)
+    x = _skewed_rows(rng, 16, 256, 2.0)
+    q, s, z = oracle.quantize_act_per_token_asym(x)
+    # zero is exactly representable: x = 0 gets code z, x_hat = 0
+    assert np.array_equal(q[:, 0].astype(np.int64), z.astype(np.int64))
+    # the range ends land on the extreme codes (to within one rounding step)
+    rows = np.arange(x.shape[0])
+    assert np.all(q[rows, x.argmin(axis=1)] <= -127)
+    assert np.all(q[rows, x.argmax(axis=1)] >= 126)
+    # every value lies in the grid's range, so |x - s (q - z)| <= s/2
+    xh = s[:, None].astype(np.float64) * (q.astype(np.float64) - z[:, None])
+    err = np.abs(x - xh)
+    assert np.all(err <= s[:, None] * (0.5 + 1e-4))
+    # round-to-nearest error has variance about s^2 / 12
+    var = np.mean((err / s[:, None]) ** 2)
+    assert abs(var - 1 / 12) < 0.01
+
+
+def test_asym_constant_rows_and_scale_zero():
+    x = np.array([[3.0] * 8, [-0.75] * 8, [0.0] * 8], np.float32)
+    q, s, z = oracle.quantize_act_per_token_asym(x)
+    xh = s[:, None].astype(np.float64) * (q.astype(np.float64) - z[:, None])
+    assert np.allclose(xh[:2], x[:2], rtol=1e-6)
+    assert s[2] == 0 and z[2] == 0 and not q[2].any()
+
+
+def test_asym_beats_symmetric_on_one_sided_rows():
+    """The notes recommend asymmetric codes for activations that are not
+    centred on zero: on a shifted distribution its reconstruction error is
+    smaller than the symmetric one's."""
+    rng = np.random.default_rng(53)
+    x = np.abs(rng.standard_normal((8, 512))).astype(np.float32)
+    x[:, 0] = 0.0
+    qa, sa, za = oracle.quantize_act_per_token_asym(x)
+    qs, ss = oracle.quantize_act_per_token(x)
+    ea = np.mean((x - sa[:, None] * (qa.astype(np.float64) - za[:, None])) ** 2)
+    es = np.mean((x - ss[:, None] * qs.astype(np.float64)) ** 2)
+    assert ea < 0.5 * es
+
+
+def test_intscale_acc_asym_reduces_to_symmetric_when_z_is_zero():
+    rng = np.random.default_rng(54)
+    qx = rng.integers(-128, 128, (3, 256)).astype(np.int8)
+    qw = rng.integers(-7, 8, (256, 10)).astype(np.int8)
+    S = rng.integers(1, 300, (2, 10)).astype(np.int32)
+    assert np.array_equal(oracle.intscale_acc_asym(qx, np.zeros(3, np.int32), qw, S),
+                          oracle.intscale_acc(qx, qw, S))
+
+
+def test_intscale_acc_asym_equals_the_expanded_zero_point_form():
+    """(q_X - Z_X) q_W expands to q_W q_X - Z_X q_W: the second term is z[m]
+    times the column sum of the integer weights S * q_W, precomputable per
+    column; checked with numpy int64 matmuls."""
+    rng = np.random.default_rng(55)
+    M, K, N = 5, 384, 12
+    qx = rng.integers(-128, 128, (M, K)).astype(np.int8)
+    z = rng.integers(-128, 128, M).astype(np.int32)
+    qw = rng.integers(-8, 8, (K, N)).astype(np.int8)
+    S = rng.integers(1, 2000, (K // 128, N)).astype(np.int32)
+    Wint = np.repeat(S.astype(np.int64), 128, axis=0) * qw.astype(np.int64)
+    expanded = qx.astype(np.int64) @ Wint - z.astype(np.int64)[:, None] * Wint.sum(axis=0)[None, :]
+    assert np.array_equal(oracle.intscale_acc_asym(qx, z, qw, S), expanded)
+
+
+def test_linear_asym_bruteforce_dequantized_fp64():
+    """acc * s_a / alpha equals the fp64 matmul of the dequantized operands
+    s_a (q_x - z) and S / alpha q_w on tiny inputs."""
+    rng = np.random.default_rng(56)
+    for _ in range(150):
+        M = int(rng.integers(1, 5))
+        N = int(rng.integers(1, 9))
+        K = int(rng.choice([128, 256]))
+        x = (rng.standard_normal((M, K)) + rng.uniform(-2, 2)).astype(np.float32)
+        w = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+        alpha = int(rng.choice([1024, 256]))
+        r = oracle.linear_intscale(x, w, alpha=alpha, out="f32", asym=True)
+        xh = r["s_a"][:, None].astype(np.float64) * (r["qx"].astype(np.float64) - r["z"][:, None])
+        wh = np.repeat(r["S"], 128, axis=0).astype(np.float64) / alpha * r["qw"]
+        ref = xh @ wh
+        assert np.allclose(r["y64"], ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+        # on rows that span zero the activation side is within half a step of x
+        span = (x.min(axis=1) < 0) & (x.max(axis=1) > 0)
+        assert np.all(np.abs(x - xh)[span] <= (r["s_a"][:, None] * (0.5 + 1e-4) + 0 * xh)[span])
