@@ -14,9 +14,12 @@ from ._native import (  # noqa: F401
     pack_w4_groupwise,
     pack_w8_groupwise,
     quantize_act_per_token,
+    quantize_act_per_token_asym,
+    w4_zero_point_term,
     w4a8_amplifier_search,
     w4a8_gemm_floatscale,
     w4a8_gemm_intscale,
+    w4a8_gemm_intscale_asym,
     w4a8_gemm_intscale_static_ws,
     w4a8_moe_gemm_intscale,
     w8a8_gemm_intscale,
@@ -32,9 +35,12 @@ __all__ = [
     "pack_w4_groupwise",
     "pack_w8_groupwise",
     "quantize_act_per_token",
+    "quantize_act_per_token_asym",
+    "w4_zero_point_term",
     "w4a8_amplifier_search",
     "w4a8_gemm_floatscale",
     "w4a8_gemm_intscale",
+    "w4a8_gemm_intscale_asym",
     "w4a8_gemm_intscale_static_ws",
     "w4a8_moe_gemm_intscale",
     "w8a8_gemm_intscale",

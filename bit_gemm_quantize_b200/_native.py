@@ -69,6 +69,9 @@ def load(path: str = LIB_PATH):
         sigs = {
             "w4a8_status_string": ([I32_], ctypes.c_char_p),
             "quantize_act_per_token": ([P, I32_, I64, I64, I64, P, P, P], I32_),
+            "quantize_act_per_token_asym": ([P, I32_, I64, I64, I64, P, P, P, P], I32_),
+            "w4_zero_point_term": ([P, P, I64, I64, I32_, P, P], I32_),
+            "w4a8_gemm_intscale_asym": ([P, P, P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
             "w4a8_amplifier_search": ([P, I64, P, P, P], I32_),
             "pack_w4_groupwise": ([P, I64, I64, I32_, I32_, P, P, P, P, P, P, P], I32_),
             "pack_w4_groupwise_range": ([P, I64, I64, I32_, I32_, I32_, P, P, P, P, P, P, P], I32_),
@@ -230,6 +233,48 @@ def pack_w8_groupwise(w: torch.Tensor, group: int = 128, alpha: int | None = Non
 _OUT = {"f32": (F32, torch.float32), "f16": (F16, torch.float16), "i32": (I32, torch.int32)}
 
 
+def quantize_act_per_token_asym(x: torch.Tensor, q_x: torch.Tensor | None = None,
+                                s_a: torch.Tensor | None = None, z_a: torch.Tensor | None = None):
+    """Per-token asymmetric int8 codes in [-128, 127], fp32 scales and int32
+    zero points of x [M, K] (fp32 or bf16)."""
+    _need_cuda("x", x, ndim=2)
+    if x.dtype == torch.float32:
+        dt = F32
+    elif x.dtype == torch.bfloat16:
+        dt = BF16
+    else:
+        raise ValueError("x must be float32 or bfloat16")
+    M, K = x.shape
+    if q_x is None:
+        q_x = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if s_a is None:
+        s_a = torch.empty((M,), dtype=torch.float32, device=x.device)
+    if z_a is None:
+        z_a = torch.empty((M,), dtype=torch.int32, device=x.device)
+    _need_cuda("q_x", q_x, torch.int8, 2)
+    _need_cuda("s_a", s_a, torch.float32, 1)
+    _need_cuda("z_a", z_a, torch.int32, 1)
+    code = load().quantize_act_per_token_asym(_ptr(x), dt, M, K, K, _ptr(q_x), _ptr(s_a), _ptr(z_a),
+                                              _stream(x.device))
+    _check("quantize_act_per_token_asym", code)
+    return q_x, s_a, z_a
+
+
+def w4_zero_point_term(w_packed: torch.Tensor, S: torch.Tensor, group: int = 128) -> torch.Tensor:
+    """zc [N] int32 = sum_g S[g, n] * sum_{k in g} q[k, n] from the packed codes
+    (the weight-side term of an asymmetric activation's zero point)."""
+    _need_cuda("w_packed", w_packed, torch.uint8, 2)
+    _need_cuda("S", S, torch.int16, 2)
+    N, K2 = w_packed.shape
+    K = 2 * K2
+    if S.shape != (K // group, N):
+        raise ValueError("S must be [K / group, N]")
+    zc = torch.empty((N,), dtype=torch.int32, device=w_packed.device)
+    code = load().w4_zero_point_term(_ptr(w_packed), _ptr(S), K, N, group, _ptr(zc), _stream(w_packed.device))
+    _check("w4_zero_point_term", code)
+    return zc
+
+
 def _gemm_args(q_x, s_a, packed, N, K, group):
     _need_cuda("q_x", q_x, torch.int8, 2)
     _need_cuda("s_a", s_a, torch.float32, 1)
@@ -257,6 +302,33 @@ def w4a8_gemm_intscale(q_x, s_a, w_packed, S, alpha: int, *, group: int = 128, o
     code = load().w4a8_gemm_intscale(_ptr(q_x), _ptr(s_a), _ptr(w_packed), _ptr(S), int(alpha), M, N, K, group,
                                      _ptr(y), dt, _ptr(workspace), ws_bytes, _stream(q_x.device))
     _check("w4a8_gemm_intscale", code)
+    return y
+
+
+def w4a8_gemm_intscale_asym(q_x, s_a, z_a, w_packed, S, zc, alpha: int, *, group: int = 128, out: str = "f16",
+                            y: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """y [M, N] = integer-scale W4A8 GEMM of asymmetric token codes: the
+    accumulator is sum_g S sum_k (q_x - z_a) q, computed as the symmetric one
+    minus z_a[m] * zc[n] (out: 'f16', 'f32' or 'i32' for that accumulator)."""
+    N, K2 = w_packed.shape
+    K = 2 * K2
+    M = _gemm_args(q_x, s_a, w_packed, N, K, group)
+    _need_cuda("S", S, torch.int16, 2)
+    _need_cuda("z_a", z_a, torch.int32, 1)
+    _need_cuda("zc", zc, torch.int32, 1)
+    if z_a.shape[0] != M or zc.shape[0] != N:
+        raise ValueError("z_a must be [M] and zc [N]")
+    dt, tdt = _OUT[out]
+    if y is None:
+        y = torch.empty((M, N), dtype=tdt, device=q_x.device)
+    _need_cuda("y", y, tdt, 2)
+    if workspace is None:
+        workspace = gemm_workspace(M, N, K, group, 0, q_x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    code = load().w4a8_gemm_intscale_asym(_ptr(q_x), _ptr(s_a), _ptr(z_a), _ptr(w_packed), _ptr(S), _ptr(zc),
+                                          int(alpha), M, N, K, group, _ptr(y), dt, _ptr(workspace), ws_bytes,
+                                          _stream(q_x.device))
+    _check("w4a8_gemm_intscale_asym", code)
     return y
 
 

@@ -146,7 +146,8 @@ w4a8_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int32_t group) {
 
 w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_t* w_packed, const int16_t* S,
                      const float* s_g, int32_t alpha, int64_t M, int64_t N, int64_t K, int32_t group, void* y,
-                     int32_t y_dtype, void* workspace, int64_t workspace_bytes, void* stream, bool w8 = false) {
+                     int32_t y_dtype, void* workspace, int64_t workspace_bytes, void* stream, bool w8 = false,
+                     const int32_t* z_a = nullptr, const int32_t* zc = nullptr, bool zp = false) {
     w4a8_status st = check_gemm_shape(M, N, K, group);
     if (st != W4A8_OK) return st;
     if (path == w4a8::gemm::kIntScale) {
@@ -157,6 +158,8 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     }
     if (M == 0) return W4A8_OK;
     if (!q_x || !s_a || !w_packed || !y || (path == w4a8::gemm::kIntScale ? !S : !s_g)) return W4A8_ERR_INVALID_ARG;
+    if (zp && (!z_a || !zc)) return W4A8_ERR_INVALID_ARG;
+    if (zp && ((reinterpret_cast<uintptr_t>(z_a) | reinterpret_cast<uintptr_t>(zc)) & 3u) != 0) return W4A8_ERR_ALIGN;
     if (!aligned16(q_x) || !aligned16(w_packed) || !aligned16(y) || !aligned16(s_a) ||
         !aligned16(path == w4a8::gemm::kIntScale ? static_cast<const void*>(S) : static_cast<const void*>(s_g)))
         return W4A8_ERR_ALIGN;
@@ -214,6 +217,14 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     p.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
     p.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
                                     : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
+    if (zp) {
+        w4a8::gemm::ParamsZp pz{};
+        static_cast<w4a8::gemm::Params&>(pz) = p;
+        pz.z_a = z_a;
+        pz.zc = zc;
+        W4A8_CUDA_TRY(w4a8::gemm::launch_zp(tm_w, tm_x, tm_y, pz, pl.BT, static_cast<cudaStream_t>(stream)));
+        return W4A8_OK;
+    }
     W4A8_CUDA_TRY(w4a8::gemm::launch(tm_w, tm_x, tm_y, p, pl.BT, path, static_cast<cudaStream_t>(stream), w8));
     return W4A8_OK;
 }
@@ -288,6 +299,36 @@ w4a8_status quantize_act_per_token(const void* x, int32_t x_dtype, int64_t M, in
     if (st != W4A8_OK) return st;
     W4A8_CUDA_TRY(w4a8::quant::launch(x, x_dtype == W4A8_BF16, M, K, ldx, q_x, s_a, dev.status,
                                       static_cast<cudaStream_t>(stream), dev.sms));
+    return W4A8_OK;
+}
+
+w4a8_status quantize_act_per_token_asym(const void* x, int32_t x_dtype, int64_t M, int64_t K, int64_t ldx,
+                                        int8_t* q_x, float* s_a, int32_t* z_a, void* stream) {
+    if (x_dtype != W4A8_F32 && x_dtype != W4A8_BF16) return W4A8_ERR_DTYPE;
+    if (M < 0 || K <= 0 || K % 16 != 0 || ldx < K) return W4A8_ERR_SHAPE;
+    if (M == 0) return W4A8_OK;
+    if (!x || !q_x || !s_a || !z_a) return W4A8_ERR_INVALID_ARG;
+    const int64_t esz = x_dtype == W4A8_BF16 ? 2 : 4;
+    if (!aligned16(x) || !aligned16(q_x) || (ldx * esz) % 16 != 0) return W4A8_ERR_ALIGN;
+    DeviceInfo dev;
+    w4a8_status st = current_device(dev);
+    if (st != W4A8_OK) return st;
+    W4A8_CUDA_TRY(w4a8::quant::launch_asym(x, x_dtype == W4A8_BF16, M, K, ldx, q_x, s_a, z_a,
+                                           static_cast<cudaStream_t>(stream), dev.sms));
+    return W4A8_OK;
+}
+
+w4a8_status w4_zero_point_term(const uint8_t* w_packed, const int16_t* S, int64_t K, int64_t N, int32_t group,
+                               int32_t* zc, void* stream) {
+    if (K <= 0 || N <= 0 || group <= 0 || group % 32 != 0 || K % group != 0) return W4A8_ERR_SHAPE;
+    if (K > INT32_MAX || N > INT32_MAX) return W4A8_ERR_SHAPE;
+    if (!w_packed || !S || !zc) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(w_packed)) return W4A8_ERR_ALIGN;
+    DeviceInfo dev;
+    w4a8_status st = current_device(dev);
+    if (st != W4A8_OK) return st;
+    W4A8_CUDA_TRY(w4a8::pack::zero_point_term(w_packed, S, K, N, group, zc, static_cast<cudaStream_t>(stream),
+                                              dev.sms));
     return W4A8_OK;
 }
 
@@ -407,6 +448,14 @@ w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, const uint8_
                                int32_t y_dtype, void* workspace, int64_t workspace_bytes, void* stream) {
     return run_gemm(w4a8::gemm::kIntScale, q_x, s_a, w_packed, S, nullptr, alpha, M, N, K, group, y, y_dtype,
                     workspace, workspace_bytes, stream);
+}
+
+w4a8_status w4a8_gemm_intscale_asym(const int8_t* q_x, const float* s_a, const int32_t* z_a,
+                                    const uint8_t* w_packed, const int16_t* S, const int32_t* zc, int32_t alpha,
+                                    int64_t M, int64_t N, int64_t K, int32_t group, void* y, int32_t y_dtype,
+                                    void* workspace, int64_t workspace_bytes, void* stream) {
+    return run_gemm(w4a8::gemm::kIntScale, q_x, s_a, w_packed, S, nullptr, alpha, M, N, K, group, y, y_dtype,
+                    workspace, workspace_bytes, stream, false, z_a, zc, true);
 }
 
 w4a8_status w8a8_gemm_intscale(const int8_t* q_x, const float* s_a, const int8_t* w8, const int16_t* S, int32_t alpha,

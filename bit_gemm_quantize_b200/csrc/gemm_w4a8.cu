@@ -49,6 +49,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "gemm_w4a8.h"
 #include "kernels.h"
@@ -108,7 +109,11 @@ constexpr int64_t kMaxGrid = kCounterBytes / 4;
 // is the MMA's A operand as it stands (read from shared memory through a
 // descriptor, like the token codes): no unpack, no TMEM operand slots, and
 // the weight slot is released by the stage's MMA commit.
-template <int BT, int PATH, bool W8 = false>
+// ZP: asymmetric token codes with a zero point z[m] per token (integer-scale
+// path only).  The tile's tail subtracts z[m] * c[n] from the accumulator
+// before the rescale, c[n] = sum_g S[g,n] * sum_{k in g} q[k,n] precomputed
+// per weight column; nothing else changes.
+template <int BT, int PATH, bool W8 = false, bool ZP = false>
 struct Cfg {
     // warp roles: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-5 unpack
     // (four consecutive warps cover the four TMEM lane quarters), then the
@@ -161,7 +166,9 @@ struct Cfg {
     static constexpr int offX = offW + kSW * kWBytes;
     static constexpr int offY = offX + kSX * kXBytes;
     static constexpr int offSA = offY + kYBytes;
-    static constexpr int offBar = offSA + BT * 4;
+    static constexpr int offZ = offSA + BT * 4;                     // the tile's zero points (ZP)
+    static constexpr int offBar = offZ + (ZP ? BT * 4 : 0);
+    static_assert(!ZP || PATH == kIntScale, "zero points are applied on the integer-scale path");
     static constexpr int kBars = 2 * kSW + kSX + kSA + 2 * kSD + 2 * kAcc + 1;
     static constexpr int offMisc = offBar + kBars * 8;
     static constexpr int kSmemBytes = offMisc + 64 + 1024;  // + slack to align the base to 1024
@@ -350,11 +357,11 @@ struct Ring {
     }
 };
 
-template <int BT, int PATH, bool W8>
-__global__ void __launch_bounds__(Cfg<BT, PATH, W8>::kThreads, Cfg<BT, PATH, W8>::kCtasPerSm)
+template <int BT, int PATH, bool W8, bool ZP>
+__global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH, W8, ZP>::kCtasPerSm)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-                     const __grid_constant__ CUtensorMap tm_y, const Params p) {
-    using C = Cfg<BT, PATH, W8>;
+                     const __grid_constant__ CUtensorMap tm_y, const std::conditional_t<ZP, ParamsZp, Params> p) {
+    using C = Cfg<BT, PATH, W8, ZP>;
     constexpr int kAcc = C::kAcc;
     constexpr int kU = C::kUnpackWarps;
     constexpr int SW = C::kSW, SX = C::kSX, SA = C::kSA, SD = C::kSD;
@@ -677,10 +684,16 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8>::kThreads, Cfg<BT, PATH, W8>
             // output scale of token (tile start + this thread's index among the
             // epilogue threads), handed to the tail through shared memory
             float sa_pref = 0.0f;
+            int32_t z_pref = 0;   // zero point of the same token (ZP)
+            int32_t zc_n = 0;     // zero-point term of this thread's column (ZP)
             {
                 const int te = ew * 32 + lane;
                 const int64_t mt = int64_t(sg.m_tile) * BT + te;
                 if (te < BT && mt < p.M) sa_pref = output_scale<PATH>(p, mt);
+                if constexpr (ZP) {
+                    if (te < BT && mt < p.M) z_pref = p.z_a[mt];
+                    if (nvalid) zc_n = p.zc[n];
+                }
             }
             int32_t acc[HC];
             float accf[HC];
@@ -955,7 +968,19 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8>::kThreads, Cfg<BT, PATH, W8>
             epi_bar_sync(kEpiWarps * 32);
             float* sa_tile = reinterpret_cast<float*>(smem + C::offSA);
             if (ew * 32 + lane < BT) sa_tile[ew * 32 + lane] = sa_pref;
+            if constexpr (ZP) {
+                int32_t* z_tile = reinterpret_cast<int32_t*>(smem + C::offZ);
+                if (ew * 32 + lane < BT) z_tile[ew * 32 + lane] = z_pref;
+            }
             epi_bar_sync(kEpiWarps * 32);
+            if constexpr (ZP) {
+                // acc - z[m] * c[n], in two's-complement arithmetic: the terms may
+                // wrap, the difference (the true accumulator) fits in 32 bits
+                const int32_t* zt = reinterpret_cast<const int32_t*>(smem + C::offZ) + half * HC;
+#pragma unroll
+                for (int j = 0; j < HC; ++j)
+                    acc[j] = int32_t(uint32_t(acc[j]) - uint32_t(zt[j]) * uint32_t(zc_n));
+            }
             {
                 const int base = half * HC * kTileN + r;  // element index of (token half*HC, column r)
                 const float* sa = sa_tile + half * HC;
@@ -1020,11 +1045,11 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool
     return pl;
 }
 
-template <int BT, int PATH, bool W8 = false>
-static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty, const Params& p,
-                             cudaStream_t stream) {
-    using C = Cfg<BT, PATH, W8>;
-    auto kern = w4a8_gemm_kernel<BT, PATH, W8>;
+template <int BT, int PATH, bool W8 = false, bool ZP = false>
+static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty,
+                             const std::conditional_t<ZP, ParamsZp, Params>& p, cudaStream_t stream) {
+    using C = Cfg<BT, PATH, W8, ZP>;
+    auto kern = w4a8_gemm_kernel<BT, PATH, W8, ZP>;
     const int smem = C::kSmemBytes;
     // the shared-memory opt-in is a per-device function attribute: set it once
     static bool configured[64] = {};
@@ -1067,6 +1092,16 @@ cudaError_t launch(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorM
         case 32: return launch_bt<32, kFloatScale>(tw, tx, ty, p, stream);
         case 64: return launch_bt<64, kFloatScale>(tw, tx, ty, p, stream);
         default: return launch_bt<128, kFloatScale>(tw, tx, ty, p, stream);
+    }
+}
+
+cudaError_t launch_zp(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty, const ParamsZp& p, int BT,
+                      cudaStream_t stream) {
+    switch (BT) {
+        case 16: return launch_bt<16, kIntScale, false, true>(tw, tx, ty, p, stream);
+        case 32: return launch_bt<32, kIntScale, false, true>(tw, tx, ty, p, stream);
+        case 64: return launch_bt<64, kIntScale, false, true>(tw, tx, ty, p, stream);
+        default: return launch_bt<128, kIntScale, false, true>(tw, tx, ty, p, stream);
     }
 }
 

@@ -31,6 +31,13 @@ struct Params {
     int32_t y_dtype;     // OutType
 };
 
+// Parameters of the kernels for asymmetric token codes (a separate type, so
+// that the other kernels' parameter block stays as it is)
+struct ParamsZp : Params {
+    const int32_t* z_a;  // [M] token zero points
+    const int32_t* zc;   // [N] zero-point term zc[n] = sum_g S[g,n] sum_{k in g} q[k,n]
+};
+
 struct Plan {
     int BT;              // tokens per tile (MMA N)
     int64_t n_tiles, m_tiles, tiles, G, W, grid;
@@ -48,6 +55,10 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool
 // w8: tm_w covers int8 weights w8 [N][K] (box 128 B x 128 rows, 128-byte swizzle); integer-scale path only
 cudaError_t launch(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap& tm_y, const Params& p, int BT,
                    int path, cudaStream_t stream, bool w8 = false);
+// asymmetric token codes (zero points p.z_a, weight-side term p.zc): the
+// integer-scale path with int4 weights
+cudaError_t launch_zp(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap& tm_y, const ParamsZp& p,
+                      int BT, cudaStream_t stream);
 
 int token_tile_rows();
 

@@ -30,6 +30,9 @@ struct LaunchPdl {
 namespace quant {
 cudaError_t launch(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a,
                    int* status, cudaStream_t stream, int num_sms);
+// asymmetric codes in [-128, 127] with a zero point z_a[m] per row
+cudaError_t launch_asym(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a,
+                        int32_t* z_a, cudaStream_t stream, int num_sms);
 }
 
 namespace moe {
@@ -78,6 +81,10 @@ cudaError_t quantize_pack(const float* w, const float* s_g, int32_t alpha, int64
 // 8-bit codes clip(rne(w / s_g), -127, 127) stored as w8 [N, K] int8, and S
 cudaError_t quantize_w8(const float* w, const float* s_g, int32_t alpha, int64_t K, int64_t N, int32_t group,
                         int8_t* w8, int16_t* S, void* workspace, cudaStream_t stream);
+// zc[n] = sum_g S[g,n] * sum_{k in g} q[k,n] from the packed int4 codes (the
+// weight-side zero-point term of an asymmetric activation)
+cudaError_t zero_point_term(const uint8_t* packed, const int16_t* S, int64_t K, int64_t N, int32_t group,
+                            int32_t* zc, cudaStream_t stream, int num_sms);
 }  // namespace pack
 
 }  // namespace w4a8

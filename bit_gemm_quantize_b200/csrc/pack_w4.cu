@@ -176,6 +176,50 @@ __global__ void __launch_bounds__(kThreads) colsum_kernel(const int16_t* __restr
     if ((threadIdx.x & 31) == 0) atomicMax(out, t);
 }
 
+// Weight-side zero-point term of an asymmetric activation ("Quantization"
+// notes, quantized matmul expansion: with Z_W = 0 the term Z_X q_W depends on
+// the weights alone and is precomputed; with integer group scales it is
+// zc[n] = sum_g S[g, n] * sum_{k in g} q[k, n]).  One warp per column; each
+// lane sums whole 16-byte chunks of the packed row, 32 codes of one group (the
+// order of the nibbles inside a chunk does not matter to a sum).  Sums wrap in
+// 32 bits like the GEMM's accumulator, which subtracts z[m] * zc[n].
+__global__ void __launch_bounds__(kThreads) zero_point_term_kernel(const uint8_t* __restrict__ packed,
+                                                                   const int16_t* __restrict__ S, int64_t K,
+                                                                   int64_t N, int32_t group,
+                                                                   int32_t* __restrict__ zc) {
+    constexpr int kWarps = kThreads / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t chunks = K / 32;
+    const int64_t chunks_per_group = group / 32;
+    const int64_t stride = int64_t(gridDim.x) * kWarps;
+    for (int64_t n = int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5); n < N; n += stride) {
+        const uint4* row = reinterpret_cast<const uint4*>(packed + n * (K / 2));
+        uint32_t t = 0u;
+        for (int64_t c = lane; c < chunks; c += 32) {
+            const uint4 v = row[c];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            int32_t sum = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) sum += int32_t(w[i] << (28 - 4 * j)) >> 28;  // nibble j, sign-extended
+            t += uint32_t(int32_t(S[(c / chunks_per_group) * N + n])) * uint32_t(sum);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (lane == 0) zc[n] = int32_t(t);
+    }
+}
+
+cudaError_t zero_point_term(const uint8_t* packed, const int16_t* S, int64_t K, int64_t N, int32_t group,
+                            int32_t* zc, cudaStream_t stream, int num_sms) {
+    const int64_t per_block = kThreads / 32;
+    int64_t blocks = (N + per_block - 1) / per_block;
+    if (blocks > int64_t(num_sms) * 8) blocks = int64_t(num_sms) * 8;
+    zero_point_term_kernel<<<unsigned(blocks), kThreads, 0, stream>>>(packed, S, K, N, group, zc);
+    return cudaGetLastError();
+}
+
 cudaError_t group_scales(const float* w, int64_t K, int64_t N, int32_t group, int32_t qmin, float* s_g,
                          cudaStream_t stream) {
     return group_scales_div(w, K, N, group, qmin == -8 ? 8.0f : 7.0f, s_g, stream);

@@ -196,6 +196,86 @@ __global__ void __launch_bounds__(kThreads) quant_rows_direct(const T* __restric
     }
 }
 
+// ---- asymmetric codes ("Quantization" notes, Asymmetric Quantization): the
+// row's range [x_min, x_max] maps onto the int8 codes [-128, 127]:
+// s = (x_max - x_min) / 255, z = clip(rne(-128 - x_min / s), -128, 127),
+// q = clip(rne(x / s) + z, -128, 127).  Each step is one IEEE fp32 operation
+// (true division), so the codes match a plain CPU evaluation bit for bit.  A
+// constant row's empty range is widened to include zero; a row whose scale is
+// 0 gets z = 0 and codes 0.  Inputs are finite.  Two passes over the row (the
+// second from L2): the min / max reduction, then the codes.
+
+__device__ __forceinline__ void block_minmax(float& lo, float& hi, float* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) {
+        red[warp] = lo;
+        red[kWarps + warp] = hi;
+    }
+    __syncthreads();
+    lo = red[0];
+    hi = red[kWarps];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) {
+        lo = fminf(lo, red[w]);
+        hi = fmaxf(hi, red[kWarps + w]);
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) quant_rows_asym(const T* __restrict__ x, int64_t M, int64_t K,
+                                                            int64_t ldx, int8_t* __restrict__ q,
+                                                            float* __restrict__ s_a, int32_t* __restrict__ z_a) {
+    __shared__ float red[2 * kWarps];
+    if (threadIdx.x == 0) griddep_launch_dependents();
+    griddep_wait();  // x may be the previous kernel's output, q, s_a and z_a its input
+    for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
+        const T* r = x + row * ldx;
+        float lo = INFINITY, hi = -INFINITY;
+        for (int64_t c = threadIdx.x; c < K / 16; c += kThreads) {
+            float v[16];
+            load16<T>(r + c * 16, v);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                lo = fminf(lo, v[i]);
+                hi = fmaxf(hi, v[i]);
+            }
+        }
+        block_minmax(lo, hi, red);
+        if (hi == lo) {  // empty range: widen it to include zero
+            lo = fminf(lo, 0.0f);
+            hi = fmaxf(hi, 0.0f);
+        }
+        const float s = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
+        const bool zero = (s == 0.0f);
+        const float zf = zero ? 0.0f : fminf(fmaxf(rintf(__fsub_rn(-128.0f, __fdiv_rn(lo, s))), -128.0f), 127.0f);
+        if (threadIdx.x == 0) {
+            s_a[row] = s;
+            z_a[row] = int32_t(zf);
+        }
+        int8_t* qrow = q + row * K;
+        for (int64_t c = threadIdx.x; c < K / 16; c += kThreads) {
+            uint32_t packed[4] = {0u, 0u, 0u, 0u};
+            if (!zero) {
+                float v[16];
+                load16<T>(r + c * 16, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    // rne(x / s) + z is exact below 2^24; above it the clip decides alone
+                    const float t = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(v[i], s)), zf), -128.0f), 127.0f);
+                    packed[i >> 2] |= (uint32_t(int(t)) & 0xFFu) << (8 * (i & 3));
+                }
+            }
+            *reinterpret_cast<uint4*>(qrow + c * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        }
+        __syncthreads();  // the reduction scratch is free again
+    }
+}
+
 constexpr size_t kMaxStagedSmem = 200 * 1024;
 
 // Resident CTAs per SM of the staged kernel for a given shared-memory size,
@@ -264,6 +344,22 @@ cudaError_t launch(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, 
         return launch_t<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), M, K, ldx, q, s_a, status, stream,
                                        num_sms);
     return launch_t<float>(static_cast<const float*>(x), M, K, ldx, q, s_a, status, stream, num_sms);
+}
+
+cudaError_t launch_asym(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a,
+                        int32_t* z_a, cudaStream_t stream, int num_sms) {
+    int per_sm = 0;
+    cudaError_t e = bf16 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_rows_asym<__nv_bfloat16>,
+                                                                         kThreads, 0)
+                         : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, quant_rows_asym<float>, kThreads, 0);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    const int64_t grid = M < int64_t(num_sms) * per_sm ? M : int64_t(num_sms) * per_sm;
+    const LaunchPdl lc(unsigned(grid), kThreads, 0, stream);
+    if (bf16)
+        return cudaLaunchKernelEx(&lc.cfg, quant_rows_asym<__nv_bfloat16>, static_cast<const __nv_bfloat16*>(x), M,
+                                  K, ldx, q, s_a, z_a);
+    return cudaLaunchKernelEx(&lc.cfg, quant_rows_asym<float>, static_cast<const float*>(x), M, K, ldx, q, s_a, z_a);
 }
 
 }  // namespace quant

@@ -90,6 +90,26 @@ W4A8_API w4a8_status quantize_act_per_token(const void* x, int32_t x_dtype, int6
                                    int8_t* q_x, float* s_a, void* stream);
 
 /*
+ * Per-token asymmetric int8 activation quantization.
+ * ("Quantization" notes, Asymmetric Quantization: the range [x_min, x_max]
+ *  maps onto [q_min, q_max] = [-128, 127]; 探秘Transformer系列之（34）§2.3.3
+ *  逐token量化.)  Every step is one IEEE fp32 operation:
+ *   lo, hi  = min_k x[m,k], max_k x[m,k]; if lo == hi the range is widened to
+ *             include zero (lo = min(lo, 0), hi = max(hi, 0))
+ *   s_a[m]  = fl32(fl32(hi - lo) / 255)
+ *   z_a[m]  = clamp(rne(fl32(-128 - fl32(lo / s_a[m]))), -128, 127)
+ *   q_x[m,k] = clamp(rne(fl32(x[m,k] / s_a[m])) + z_a[m], -128, 127)
+ *   (s_a[m] = 0: z_a[m] = 0 and the row's codes are 0)
+ *   dequantized: x[m,k] ~ s_a[m] * (q_x[m,k] - z_a[m])
+ * x, M, K, ldx as quantize_act_per_token (finite values)
+ * q_x     device, [M, K] int8, written
+ * s_a     device, [M] float32, written
+ * z_a     device, [M] int32, written
+ */
+W4A8_API w4a8_status quantize_act_per_token_asym(const void* x, int32_t x_dtype, int64_t M, int64_t K, int64_t ldx,
+                                                 int8_t* q_x, float* s_a, int32_t* z_a, void* stream);
+
+/*
  * Amplifier search over a set of float group scales (synchronous).
  * (Integer Scale summary §4 heuristic search.)  alpha is the smallest power
  * of two 2^j, j >= 0, with s_min * alpha >= 1, s_min the smallest POSITIVE
@@ -207,6 +227,43 @@ W4A8_API w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, con
                                const int16_t* S, int32_t alpha, int64_t M, int64_t N, int64_t K,
                                int32_t group, void* y, int32_t y_dtype, void* workspace,
                                int64_t workspace_bytes, void* stream);
+
+/*
+ * Weight-side zero-point term for asymmetric activations.
+ * ("Quantization" notes, 矩阵乘法中的量化计算: with Z_W = 0 the integer part of
+ *  the product is q_W q_X - Z_X q_W, and the weight-dependent correction can
+ *  be precomputed; with integer group scales it is one int32 per column.)
+ *   zc[n] = sum_g S[g,n] * sum_{k in g} q_w[k,n]    (two's-complement int32)
+ * w_packed  device, [N, K/2] uint8, 16-byte aligned; S device [K/group, N] int16
+ *           (from pack_w4_groupwise or pack_w4_groupwise_range)
+ * K, N      K % group == 0, group % 32 == 0; otherwise W4A8_ERR_SHAPE
+ * zc        device, [N] int32, written
+ */
+W4A8_API w4a8_status w4_zero_point_term(const uint8_t* w_packed, const int16_t* S, int64_t K, int64_t N,
+                                        int32_t group, int32_t* zc, void* stream);
+
+/*
+ * W4A8 integer-scale GEMM of asymmetric token codes (from
+ * quantize_act_per_token_asym).  ("Quantization" notes, 矩阵乘法中的量化计算,
+ *  with Z_W = 0 and Z_X = z_a[m]; Integer Scale summary §4.)
+ *   acc[m,n] = sum_g S[g,n] * sum_{k in g} (q_x[m,k] - z_a[m]) q_w[k,n]
+ *            = (the w4a8_gemm_intscale accumulator) - z_a[m] * zc[n]
+ *   y[m,n]   = fl_out(fl32(acc) * fl32(s_a[m] / alpha))
+ * The subtraction happens once per output, in the tile's final pass, in
+ * two's-complement int32 arithmetic: the intermediate terms may wrap, the
+ * result is exact when acc itself fits in int32, which holds when
+ * 255*qw*group*max_n sum_g |S[g,n]| < 2^31 (255 = the widest |q_x - z_a|;
+ * qw = 7, or 8 for codes in the full range [-8, 7]).
+ * z_a        device, [M] int32 (4-byte aligned)
+ * zc         device, [N] int32 from w4_zero_point_term (4-byte aligned)
+ * Other arguments, workspace (path 0), output (W4A8_I32: acc itself) and
+ * errors as in w4a8_gemm_intscale.
+ */
+W4A8_API w4a8_status w4a8_gemm_intscale_asym(const int8_t* q_x, const float* s_a, const int32_t* z_a,
+                                             const uint8_t* w_packed, const int16_t* S, const int32_t* zc,
+                                             int32_t alpha, int64_t M, int64_t N, int64_t K, int32_t group,
+                                             void* y, int32_t y_dtype, void* workspace, int64_t workspace_bytes,
+                                             void* stream);
 
 /*
  * W8A8 GEMM with integer group scales: the integer-scale GEMM above with
