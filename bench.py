@@ -405,6 +405,69 @@ def measure_w8a8(dev, rank, world, hbm_peak, int8_peak, reps=7):
             "timing": "CUDA events over graphs of six launches alternating two 90 MB weight copies"}
 
 
+ASYM = dict(K=4096, N=22016, M=[1, 32, 1024])
+
+
+def measure_asym(dev, rank, world, reps=7):
+    """Asymmetric per-token activations (a zero point per token) against the
+    symmetric ones on the FFN up-projection shape: per-launch time of the
+    quantize kernels and of the two GEMMs (integer scale, alpha = 1024), from
+    graphs of six launches rotating over four packed weight copies (180 MB, so
+    every launch streams its weights from HBM).  Inputs drawn on the device,
+    moved off zero as after a one-sided activation function."""
+    import torch
+
+    import bit_gemm_quantize_b200 as bgq
+
+    K, N = ASYM["K"], ASYM["N"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(7000 + rank)
+    w = torch.randn((K, N), generator=g, device=dev)
+    w.mul_(0.02)
+    pk = bgq.pack_w4_groupwise(w, group=GROUP, alpha=ALPHA)
+    del w
+    zc = bgq.w4_zero_point_term(pk["packed"], pk["S"], group=GROUP)
+    copies = [pk["packed"]] + [pk["packed"].clone() for _ in range(3)]
+    stream = torch.cuda.current_stream(dev)
+
+    def per_launch_ms(call):
+        for i in range(3):
+            call(i)
+        torch.cuda.synchronize(dev)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            for i in range(6):
+                call(i)
+        gr.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(reps):
+            gr.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        del gr
+        return max_over_ranks([e0.elapsed_time(e1) / (6 * reps)], world, dev)[0]
+
+    rows = []
+    for M in ASYM["M"]:
+        x = torch.randn((M, K), generator=g, device=dev).add_(1.0).to(torch.bfloat16)
+        qa, sa, za = bgq.quantize_act_per_token_asym(x)
+        qs, ss = bgq.quantize_act_per_token(x)
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        wsp = bgq.gemm_workspace(M, N, K, GROUP, 0, dev)
+        t_qa = per_launch_ms(lambda i: bgq.quantize_act_per_token_asym(x, qa, sa, za))
+        t_qs = per_launch_ms(lambda i: bgq.quantize_act_per_token(x, qs, ss))
+        t_ga = per_launch_ms(lambda i: bgq.w4a8_gemm_intscale_asym(
+            qa, sa, za, copies[i % 4], pk["S"], zc, ALPHA, group=GROUP, out="f16", y=y, workspace=wsp))
+        t_gs = per_launch_ms(lambda i: bgq.w4a8_gemm_intscale(
+            qs, ss, copies[i % 4], pk["S"], ALPHA, group=GROUP, out="f16", y=y, workspace=wsp))
+        rows.append({"M": M, "quant_asym_us": round(t_qa * 1e3, 2), "quant_sym_us": round(t_qs * 1e3, 2),
+                     "gemm_asym_us": round(t_ga * 1e3, 2), "gemm_sym_us": round(t_gs * 1e3, 2)})
+    return {"workload": "asym_act_ffn_up", "K": K, "N": N, "group": GROUP, "alpha": ALPHA, "rows": rows,
+            "timing": "CUDA events over graphs of six launches rotating four 45 MB weight copies"}
+
+
 # ---------------------------------------------------------------- rank aggregation
 
 def max_over_ranks(times_ms, world, device):
@@ -646,6 +709,7 @@ def run_ours(args):
     moe = measure_moe(dev, rank, world, int8_peak)
     prefill = measure_prefill(dev, rank, world, int8_peak)
     w8a8 = measure_w8a8(dev, rank, world, hbm_peak, int8_peak)
+    asym = measure_asym(dev, rank, world)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
@@ -657,6 +721,7 @@ def run_ours(args):
         "moe": moe,
         "prefill": prefill,
         "w8a8": w8a8,
+        "asym": asym,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample()
@@ -670,7 +735,7 @@ def run_ours(args):
 # DRAM bytes (read + write) per launch of the integer-scale GEMM, from one
 # ncu capture (profiles/gemm_intscale_bt128_m1024_k4096_n22016.md), valid for
 # the kernel source it was taken with (first 16 hex digits of its SHA-256).
-MEASURED_TRAFFIC = {1024: (56.348672e6 + 20.430848e6, "a7dc0b0564b15adc")}
+MEASURED_TRAFFIC = {1024: (56.385536e6 + 19.70176e6, "e11cabb5d4346aad")}
 
 
 def measured_traffic(M):
