@@ -141,3 +141,68 @@ def test_binding_fails_loudly_without_library(tmp_path):
             _native.load(str(tmp_path / "missing.so"))
         finally:
             _native._lib = saved
+
+
+def test_range_and_w8_pack_argument_checks(lib):
+    a_out = ctypes.c_int32(0)
+    c_out = ctypes.c_int64(0)
+
+    def pr(qmin=-8, K=256, group=128):
+        return lib.pack_w4_groupwise_range(ctypes.c_void_p(A), K, 128, group, 1024, qmin, ctypes.c_void_p(A),
+                                           ctypes.c_void_p(A), ctypes.c_void_p(A), ctypes.byref(a_out),
+                                           ctypes.byref(c_out), ctypes.c_void_p(A), None)
+
+    assert pr(qmin=-6) == INVALID
+    assert pr(qmin=-9) == INVALID
+    assert pr(K=200) == SHAPE
+
+    def p8(w8=A, K=256, group=128, alpha=0):
+        return lib.pack_w8_groupwise(ctypes.c_void_p(A), K, 128, group, alpha, ctypes.c_void_p(w8), ctypes.c_void_p(A),
+                                     ctypes.c_void_p(A), ctypes.byref(a_out), ctypes.byref(c_out), ctypes.c_void_p(A),
+                                     None)
+
+    assert p8(K=200) == SHAPE
+    assert p8(group=48) == SHAPE
+    assert p8(w8=0) == INVALID
+    assert p8(alpha=6) == INVALID
+    assert p8(w8=U) == ALIGN
+
+    def g8(M=16, K=256, dt=_native.F16, S=A):
+        return lib.w8a8_gemm_intscale(ctypes.c_void_p(A), ctypes.c_void_p(A), ctypes.c_void_p(A), ctypes.c_void_p(S),
+                                      1024, M, 128, K, 128, ctypes.c_void_p(A), dt, None, 0, None)
+
+    assert g8(K=200) == SHAPE
+    assert g8(dt=_native.BF16) == DTYPE
+    assert g8(S=0) == INVALID
+    assert g8(M=0) == OK
+
+
+def test_asymmetric_argument_checks(lib):
+    def qa(x=A, dt=_native.BF16, K=256, z=A):
+        return lib.quantize_act_per_token_asym(ctypes.c_void_p(x), dt, 4, K, K, ctypes.c_void_p(A),
+                                               ctypes.c_void_p(A), ctypes.c_void_p(z), None)
+
+    assert qa(dt=_native.F16) == DTYPE
+    assert qa(K=100) == SHAPE
+    assert qa(z=0) == INVALID
+    assert qa(x=U) == ALIGN
+
+    def zt(wp=A, K=256, group=128, zc=A):
+        return lib.w4_zero_point_term(ctypes.c_void_p(wp), ctypes.c_void_p(A), K, 128, group, ctypes.c_void_p(zc), None)
+
+    assert zt(K=200) == SHAPE
+    assert zt(group=48) == SHAPE
+    assert zt(zc=0) == INVALID
+    assert zt(wp=U) == ALIGN
+
+    def ga(z=A, zc=A, M=16, dt=_native.F16, alpha=1024):
+        return lib.w4a8_gemm_intscale_asym(ctypes.c_void_p(A), ctypes.c_void_p(A), ctypes.c_void_p(z),
+                                           ctypes.c_void_p(A), ctypes.c_void_p(A), ctypes.c_void_p(zc), alpha, M, 128,
+                                           256, 128, ctypes.c_void_p(A), dt, None, 0, None)
+
+    assert ga(z=0) == INVALID
+    assert ga(zc=0) == INVALID
+    assert ga(z=A + 2) == ALIGN  # zero points are int32: 4-byte aligned
+    assert ga(dt=_native.BF16) == DTYPE
+    assert ga(alpha=48) == INVALID
+    assert ga(M=0) == OK
