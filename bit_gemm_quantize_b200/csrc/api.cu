@@ -92,6 +92,7 @@ w4a8_status current_device(DeviceInfo& out) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -294,6 +295,7 @@ w4a8_status quantize_act_per_token(const void* x, int32_t x_dtype, int64_t M, in
     if (!x || !q_x || !s_a) return W4A8_ERR_INVALID_ARG;
     const int64_t esz = x_dtype == W4A8_BF16 ? 2 : 4;
     if (!aligned16(x) || !aligned16(q_x) || (ldx * esz) % 16 != 0) return W4A8_ERR_ALIGN;
+    if (!aligned4(s_a)) return W4A8_ERR_ALIGN;
     DeviceInfo dev;
     w4a8_status st = current_device(dev);
     if (st != W4A8_OK) return st;
@@ -310,6 +312,7 @@ w4a8_status quantize_act_per_token_asym(const void* x, int32_t x_dtype, int64_t 
     if (!x || !q_x || !s_a || !z_a) return W4A8_ERR_INVALID_ARG;
     const int64_t esz = x_dtype == W4A8_BF16 ? 2 : 4;
     if (!aligned16(x) || !aligned16(q_x) || (ldx * esz) % 16 != 0) return W4A8_ERR_ALIGN;
+    if (!aligned4(s_a) || !aligned4(z_a)) return W4A8_ERR_ALIGN;
     DeviceInfo dev;
     w4a8_status st = current_device(dev);
     if (st != W4A8_OK) return st;
@@ -323,7 +326,7 @@ w4a8_status w4_zero_point_term(const uint8_t* w_packed, const int16_t* S, int64_
     if (K <= 0 || N <= 0 || group <= 0 || group % 32 != 0 || K % group != 0) return W4A8_ERR_SHAPE;
     if (K > INT32_MAX || N > INT32_MAX) return W4A8_ERR_SHAPE;
     if (!w_packed || !S || !zc) return W4A8_ERR_INVALID_ARG;
-    if (!aligned16(w_packed)) return W4A8_ERR_ALIGN;
+    if (!aligned16(w_packed) || (reinterpret_cast<uintptr_t>(S) & 1u) != 0 || !aligned4(zc)) return W4A8_ERR_ALIGN;
     DeviceInfo dev;
     w4a8_status st = current_device(dev);
     if (st != W4A8_OK) return st;

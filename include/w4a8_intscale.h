@@ -85,6 +85,8 @@ W4A8_API const char* w4a8_status_string(int32_t status);
  * M, K    M >= 0 (M = 0 is a no-op), K > 0 and K % 16 == 0; ldx >= K, ldx*sizeof(x) % 16 == 0
  * q_x     device, [M, K] int8, written
  * s_a     device, [M] float32, written
+ * Errors: W4A8_ERR_DTYPE, W4A8_ERR_SHAPE as above; W4A8_ERR_INVALID_ARG for a NULL
+ * pointer; W4A8_ERR_ALIGN unless x and q_x are 16-byte and s_a 4-byte aligned.
  */
 W4A8_API w4a8_status quantize_act_per_token(const void* x, int32_t x_dtype, int64_t M, int64_t K, int64_t ldx,
                                    int8_t* q_x, float* s_a, void* stream);
@@ -105,6 +107,7 @@ W4A8_API w4a8_status quantize_act_per_token(const void* x, int32_t x_dtype, int6
  * q_x     device, [M, K] int8, written
  * s_a     device, [M] float32, written
  * z_a     device, [M] int32, written
+ * Errors as quantize_act_per_token; z_a must be 4-byte aligned (W4A8_ERR_ALIGN).
  */
 W4A8_API w4a8_status quantize_act_per_token_asym(const void* x, int32_t x_dtype, int64_t M, int64_t K, int64_t ldx,
                                                  int8_t* q_x, float* s_a, int32_t* z_a, void* stream);
@@ -238,6 +241,8 @@ W4A8_API w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, con
  *           (from pack_w4_groupwise or pack_w4_groupwise_range)
  * K, N      K % group == 0, group % 32 == 0; otherwise W4A8_ERR_SHAPE
  * zc        device, [N] int32, written
+ * Errors: W4A8_ERR_INVALID_ARG for a NULL pointer; W4A8_ERR_ALIGN unless w_packed is
+ * 16-byte, S 2-byte and zc 4-byte aligned.
  */
 W4A8_API w4a8_status w4_zero_point_term(const uint8_t* w_packed, const int16_t* S, int64_t K, int64_t N,
                                         int32_t group, int32_t* zc, void* stream);

@@ -54,6 +54,7 @@ def test_quantize_argument_checks(lib):
     assert _q(lib, x=U) == ALIGN
     assert _q(lib, q=U) == ALIGN
     assert _q(lib, ldx=260) == ALIGN  # bf16 rows 520 bytes apart: not 16-byte aligned
+    assert _q(lib, s=A + 2) == ALIGN  # fp32 scales: 4-byte aligned
 
 
 def _is(lib, qx=A, sa=A, wp=A, S=A, alpha=1024, M=16, N=128, K=256, group=128, y=A, dt=_native.F16, ws=0, wsb=0):
@@ -186,6 +187,7 @@ def test_asymmetric_argument_checks(lib):
     assert qa(K=100) == SHAPE
     assert qa(z=0) == INVALID
     assert qa(x=U) == ALIGN
+    assert qa(z=A + 2) == ALIGN
 
     def zt(wp=A, K=256, group=128, zc=A):
         return lib.w4_zero_point_term(ctypes.c_void_p(wp), ctypes.c_void_p(A), K, 128, group, ctypes.c_void_p(zc), None)
@@ -194,6 +196,7 @@ def test_asymmetric_argument_checks(lib):
     assert zt(group=48) == SHAPE
     assert zt(zc=0) == INVALID
     assert zt(wp=U) == ALIGN
+    assert zt(zc=A + 2) == ALIGN
 
     def ga(z=A, zc=A, M=16, dt=_native.F16, alpha=1024):
         return lib.w4a8_gemm_intscale_asym(ctypes.c_void_p(A), ctypes.c_void_p(A), ctypes.c_void_p(z),
