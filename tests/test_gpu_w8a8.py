@@ -89,3 +89,31 @@ def test_w8a8_matches_dense_integer_product():
     acc = bgq.w8a8_gemm_intscale(q, s, pk["w8"], pk["S"], pk["alpha"], group=128, out="i32").cpu().numpy()
     Wint = np.repeat(pk["S"].cpu().numpy().astype(np.int64), 128, axis=0) * pk["w8"].cpu().numpy().T.astype(np.int64)
     assert np.array_equal(acc.astype(np.int64), q.cpu().numpy().astype(np.int64) @ Wint)
+
+
+@pytest.mark.parametrize("M", [1, 32, 1024])
+def test_w8a8_ffn_up_full_size_sampled(M):
+    # the FFN up-projection shape the benchmark times (K = 4096, N = 22016), sampled outputs
+    dev = _dev()
+    K, N = 4096, 22016
+    wl = workloads.make_linear(M, K, N, x_dtype="bf16", seed=400 + M)
+    x = torch.from_numpy(np.ascontiguousarray(wl.x)).to(dev).to(torch.bfloat16)
+    q, s = bgq.quantize_act_per_token(x)
+    pk = bgq.pack_w8_groupwise(torch.from_numpy(wl.w).to(dev), group=128, alpha=None)
+    qx, sa = oracle.quantize_act_per_token(wl.x)
+    qw, sg = oracle.quantize_groups(wl.w, 128, qmax=127)
+    alpha = oracle.amplifier_search(sg)
+    S = oracle.integer_scales(sg, alpha)
+    assert pk["alpha"] == alpha
+    assert np.array_equal(q.cpu().numpy(), qx)
+    assert np.array_equal(pk["S"].cpu().numpy().astype(np.int32), S)
+    rng = np.random.default_rng(M)
+    ms = np.concatenate([rng.integers(0, M, 600), [0, M - 1]])
+    ns = np.concatenate([rng.integers(0, N, 600), [0, N - 1]])
+    acc = bgq.w8a8_gemm_intscale(q, s, pk["w8"], pk["S"], alpha, group=128, out="i32").cpu().numpy()
+    acc_ref = oracle.intscale_acc_at(qx, qw, S, ms, ns)
+    assert np.array_equal(acc[ms, ns].astype(np.int64), acc_ref)
+    y = bgq.w8a8_gemm_intscale(q, s, pk["w8"], pk["S"], alpha, group=128, out="f16").float().cpu().numpy()
+    y_ref = acc_ref.astype(np.float64) * sa[ms].astype(np.float64) / alpha
+    _assert_close_f16(y[ms, ns], y_ref)
+    assert bgq.device_status() == 0
