@@ -98,6 +98,8 @@ def load(path: str = LIB_PATH):
 
 def _check(fn: str, code: int):
     if code != 0:
+        if "gemm" in fn and code in (7, 8):  # a launch failed: its workspace may hold counts
+            _reset_workspaces()
         detail = ""
         if code == 7:  # W4A8_ERR_CUDA: name the runtime error behind it
             lib = load()
@@ -130,9 +132,21 @@ def _need_cuda(name, t, dtype=None, ndim=None):
 _ws_cache = {}
 
 
+def _reset_workspaces():
+    """Zero every cached GEMM workspace: after a failed launch or a kernel
+    timeout the split-tile arrival counters may be left nonzero."""
+    for ws in _ws_cache.values():
+        try:
+            ws.zero_()
+        except Exception:  # a lost context: nothing more to clean
+            pass
+
+
 def gemm_workspace(M: int, N: int, K: int, group: int, path: int, device) -> torch.Tensor | None:
     """A zero-filled workspace big enough for the call, reused across calls on
-    the device (the kernels leave it zeroed after a successful call)."""
+    the device (the kernels leave it zeroed after a successful call).  Calls
+    that may overlap on the GPU (different streams without ordering) must
+    each pass a workspace of their own."""
     lib = load()
     with torch.cuda.device(device):
         need = int(lib.w4a8_gemm_workspace_size(M, N, K, group, path))
@@ -453,6 +467,10 @@ def w4a8_moe_gemm_intscale(q_x, s_a, row_index, offsets, packed, S, alpha: int, 
 
 
 def device_status(clear: bool = True) -> int:
+    """The device status word (0, or the code of a kernel wait that timed
+    out); a nonzero status also re-zeroes the cached GEMM workspaces."""
     v = ctypes.c_int32(0)
     _check("w4a8_device_status", load().w4a8_device_status(ctypes.byref(v), 1 if clear else 0))
+    if v.value != 0:
+        _reset_workspaces()
     return int(v.value)

@@ -209,3 +209,27 @@ def test_asymmetric_argument_checks(lib):
     assert ga(dt=_native.BF16) == DTYPE
     assert ga(alpha=48) == INVALID
     assert ga(M=0) == OK
+
+
+def test_failed_gemm_rezeroes_cached_workspaces(lib):
+    # host logic: a GEMM that failed or timed out may leave split-tile counts in
+    # the cached workspace, so the binding zeroes every cached workspace
+    class FakeWs:
+        zeroed = 0
+
+        def zero_(self):
+            FakeWs.zeroed += 1
+
+    saved = dict(_native._ws_cache)
+    try:
+        _native._ws_cache.clear()
+        _native._ws_cache[0] = FakeWs()
+        with pytest.raises(_native.W4A8Error):
+            _native._check("w4a8_gemm_intscale", 8)  # W4A8_ERR_TIMEOUT
+        assert FakeWs.zeroed == 1
+        with pytest.raises(_native.W4A8Error):
+            _native._check("w4a8_gemm_intscale", 2)  # a shape error launches nothing
+        assert FakeWs.zeroed == 1
+    finally:
+        _native._ws_cache.clear()
+        _native._ws_cache.update(saved)
