@@ -573,6 +573,18 @@ w4a8_status w4a8_device_status(int32_t* code_host, int32_t clear) {
     if (clear) {
         const int zero = 0;
         W4A8_CUDA_TRY(cudaMemcpy(dev.status, &zero, sizeof(int), cudaMemcpyHostToDevice));
+        if (v == W4A8_ERR_TIMEOUT) {
+            // a timed-out GEMM may have left split-tile arrival counts in the
+            // library's own workspace: zero its counter region (4096 bytes)
+            int d = 0;
+            W4A8_CUDA_TRY(cudaGetDevice(&d));
+            void* ws = nullptr;
+            {
+                std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+                if (d >= 0 && d < kMaxDevices && g_static_ws[d].ready) ws = g_static_ws[d].ptr;
+            }
+            if (ws) W4A8_CUDA_TRY(cudaMemset(ws, 0, 4096));
+        }
     }
     return W4A8_OK;
 }

@@ -371,7 +371,10 @@ W4A8_API const char* w4a8_cuda_error_string(int32_t code);
  * Reads (and with clear != 0 resets) the device status word of the current
  * device: 0, or the last device-side error: W4A8_ERR_TIMEOUT (a bounded wait
  * ran out) or W4A8_ERR_INVALID_ARG (a routed row's token index out of range in
- * w4a8_moe_gemm_intscale).  Synchronous.
+ * w4a8_moe_gemm_intscale).  Synchronous.  Clearing a W4A8_ERR_TIMEOUT also
+ * zeroes the arrival counters of the library's own workspace
+ * (w4a8_gemm_intscale_static_ws); caller workspaces must be zeroed by the
+ * caller.
  */
 W4A8_API w4a8_status w4a8_device_status(int32_t* code_host, int32_t clear);
 
