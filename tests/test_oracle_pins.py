@@ -681,3 +681,20 @@ def test_linear_asym_bruteforce_dequantized_fp64():
         # on rows that span zero the activation side is within half a step of x
         span = (x.min(axis=1) < 0) & (x.max(axis=1) > 0)
         assert np.all(np.abs(x - xh)[span] <= (r["s_a"][:, None] * (0.5 + 1e-4) + 0 * xh)[span])
+
+
+def test_asym_error_analysis_trend():
+    """The oracle-side analysis (oracle/asym_error.py) on a small layer: while
+    the rows span zero (offsets up to 2 here), the asymmetric codes' error is
+    below the symmetric one's and the gap grows with the offset.  Further off
+    zero a row's range excludes zero, the printed clip of z acts and the
+    asymmetric codes lose the row's far end (the notes' formulas as printed)."""
+    from oracle import asym_error
+
+    rows = {r["offset"]: r for r in asym_error.analyse(M=8, K=512, N=64, outliers=False)}
+    for off in (0.0, 0.5, 1.0, 2.0):
+        assert rows[off]["act_mse_asym"] < rows[off]["act_mse_sym"]
+        assert rows[off]["out_rel_rms_err_act_only_asym"] < rows[off]["out_rel_rms_err_act_only_sym"]
+    gap = [rows[o]["out_rel_rms_err_act_only_sym"] - rows[o]["out_rel_rms_err_act_only_asym"] for o in (0.5, 1.0, 2.0)]
+    assert gap[0] < gap[1] < gap[2]
+    assert rows[4.0]["act_mse_asym"] > rows[4.0]["act_mse_sym"]
