@@ -43,6 +43,7 @@ struct StaticWorkspace {
 
 StaticWorkspace g_static_ws[kMaxDevices];
 std::mutex g_static_ws_mutex;
+std::mutex g_gemm_launch_mutex;
 
 // Device address of the current device's static workspace, looked up once per
 // device (the first call on a device does this set-up).
@@ -218,6 +219,9 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     p.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
     p.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
                                     : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
+    // The launchers set each kernel's shared-memory limit once per device,
+    // which is not safe to race: launches from several host threads take turns.
+    std::lock_guard<std::mutex> lock(g_gemm_launch_mutex);
     if (zp) {
         w4a8::gemm::ParamsZp pz{};
         static_cast<w4a8::gemm::Params&>(pz) = p;
