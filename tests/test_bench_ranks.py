@@ -62,3 +62,25 @@ def test_single_rank_is_identity():
     bench = _bench()
     assert bench.max_over_ranks([3.0, 4.0], 1, "cpu") == [3.0, 4.0]
     assert bench.whole_job_tops(1, 2e12, 10, 20.0) == pytest.approx(2e12 * 10 / 20e-3 / 1e12)
+
+
+def test_reference_arm_prints_the_contract_line():
+    # the reference arm (the oracle on the host cores) needs no GPU: one short
+    # run must print one JSON line with the keys the benchmark contract names
+    import json
+    import subprocess
+    import sys
+
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in line, k
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["config"]["workload"] == "ffn_up_sweep"
+    for k in ("value", "unit", "cores", "kind", "sample"):
+        assert k in line["cpu_baseline"], k
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
