@@ -42,6 +42,9 @@ PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 INT8_PER_BF16 = 2.0
 
 
+CASE_OPS = ["quant", "gemm_is", "gemm_fs", "gemm_w8", "gemm_asym"]
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -49,7 +52,72 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    # one kernel configuration, launched --reps times (for profilers and quick
+    # timing; prints a one-line summary, not the benchmark's JSON line)
+    ap.add_argument("--case", choices=CASE_OPS, default=None,
+                    help="quant | gemm_is | gemm_fs | gemm_w8 (8-bit weight codes) | gemm_asym (asymmetric tokens)")
+    ap.add_argument("--M", type=int, default=1024)
+    ap.add_argument("--K", type=int, default=K_DIM)
+    ap.add_argument("--N", type=int, default=N_DIM)
+    ap.add_argument("--group", type=int, default=GROUP)
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--out", default="f16", choices=["f16", "f32", "i32"])
     return ap.parse_args()
+
+
+def run_case(a):
+    """One kernel configuration, --reps launches back to back on the current
+    stream.  Inputs come from the seeded workload generator (tokens moved off
+    zero by +1 for gemm_asym); weights are packed once before the launches.
+    Prints the mean CUDA-event time per launch and the device status."""
+    import torch
+
+    import bit_gemm_quantize_b200 as bgq
+
+    dev = torch.device("cuda:0")
+    wl = workloads.make_linear(a.M, a.K, a.N if a.case != "quant" else 8, x_dtype="bf16", seed=7,
+                               group=a.group)
+    xs = wl.x + 1.0 if a.case == "gemm_asym" else wl.x
+    x = torch.from_numpy(xs).to(dev).to(torch.bfloat16)
+    if a.case == "gemm_asym":
+        q, s, z = bgq.quantize_act_per_token_asym(x)
+    else:
+        q, s = bgq.quantize_act_per_token(x)
+    if a.case == "gemm_w8":
+        pk = bgq.pack_w8_groupwise(torch.from_numpy(wl.w).to(dev), group=a.group, alpha=None)
+    elif a.case != "quant":
+        pk = bgq.pack_w4_groupwise(torch.from_numpy(wl.w).to(dev), group=a.group, alpha=ALPHA)
+    if a.case == "gemm_asym":
+        zc = bgq.w4_zero_point_term(pk["packed"], pk["S"], group=a.group, colsum_max=pk["colsum_max"])
+    if a.case != "quant":
+        path = {"gemm_is": 0, "gemm_asym": 0, "gemm_fs": 1, "gemm_w8": 2}[a.case]
+        ws = bgq.gemm_workspace(a.M, a.N, a.K, a.group, path, dev)
+
+    def once():
+        if a.case == "quant":
+            bgq.quantize_act_per_token(x, q, s)
+        elif a.case == "gemm_is":
+            bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], pk["alpha"], group=a.group, out=a.out, workspace=ws)
+        elif a.case == "gemm_w8":
+            bgq.w8a8_gemm_intscale(q, s, pk["w8"], pk["S"], pk["alpha"], group=a.group, out=a.out, workspace=ws)
+        elif a.case == "gemm_asym":
+            bgq.w4a8_gemm_intscale_asym(q, s, z, pk["packed"], pk["S"], zc, pk["alpha"], group=a.group, out=a.out,
+                                        workspace=ws)
+        else:
+            bgq.w4a8_gemm_floatscale(q, s, pk["packed"], pk["s_g"], group=a.group,
+                                     out="f16" if a.out == "i32" else a.out, workspace=ws)
+
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.reps):
+        once()
+    e1.record()
+    torch.cuda.synchronize()
+    st = bgq.device_status()
+    print(f"{a.case} M={a.M} K={a.K} N={a.N}: {e0.elapsed_time(e1) / a.reps * 1e3:.2f} us per launch "
+          f"(device status {st})")
+    return 0 if st == 0 else 1
 
 
 def config_dict():
@@ -431,7 +499,7 @@ def measure_asym(dev, rank, world, reps=7):
     w.mul_(0.02)
     pk = bgq.pack_w4_groupwise(w, group=GROUP, alpha=ALPHA)
     del w
-    zc = bgq.w4_zero_point_term(pk["packed"], pk["S"], group=GROUP)
+    zc = bgq.w4_zero_point_term(pk["packed"], pk["S"], group=GROUP, colsum_max=pk["colsum_max"])
     copies = [pk["packed"]] + [pk["packed"].clone() for _ in range(3)]
     stream = torch.cuda.current_stream(dev)
 
@@ -754,8 +822,8 @@ def run_ours(args):
 
 
 # DRAM bytes (read + write) per launch of the integer-scale GEMM, from one
-# ncu capture (profiles/gemm_intscale_bt128_m1024_k4096_n22016.md), valid for
-# the kernel source it was taken with (first 16 hex digits of its SHA-256).
+# ncu capture of `bench.py --case gemm_is --M <M>`, valid for the kernel source
+# it was taken with (first 16 hex digits of its SHA-256).
 MEASURED_TRAFFIC = {1024: (56.385536e6 + 19.70176e6, "e11cabb5d4346aad")}
 
 
@@ -774,6 +842,8 @@ def measured_traffic(M):
 
 def main():
     args = parse()
+    if args.case is not None:
+        return run_case(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

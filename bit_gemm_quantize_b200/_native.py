@@ -70,7 +70,8 @@ def load(path: str = LIB_PATH):
             "w4a8_status_string": ([I32_], ctypes.c_char_p),
             "quantize_act_per_token": ([P, I32_, I64, I64, I64, P, P, P], I32_),
             "quantize_act_per_token_asym": ([P, I32_, I64, I64, I64, P, P, P, P], I32_),
-            "w4_zero_point_term": ([P, P, I64, I64, I32_, P, P], I32_),
+            "w4_zero_point_term": ([P, P, I64, I64, I32_, I32_, I64, P, P], I32_),
+            "w4a8_static_workspace_reset": ([], I32_),
             "w4a8_gemm_intscale_asym": ([P, P, P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
             "w4a8_amplifier_search": ([P, I64, P, P, P], I32_),
             "pack_w4_groupwise": ([P, I64, I64, I32_, I32_, P, P, P, P, P, P, P], I32_),
@@ -132,13 +133,23 @@ def _need_cuda(name, t, dtype=None, ndim=None):
 _ws_cache = {}
 
 
+_static_ws_devices = set()  # devices on which the library's own workspace has been used
+
+
 def _reset_workspaces():
-    """Zero every cached GEMM workspace: after a failed launch or a kernel
-    timeout the split-tile arrival counters may be left nonzero."""
+    """Zero every cached GEMM workspace and the library's own (static)
+    workspace counters: after a failed launch or a device-side error the
+    split-tile arrival counters may be left nonzero."""
     for ws in _ws_cache.values():
         try:
             ws.zero_()
         except Exception:  # a lost context: nothing more to clean
+            pass
+    for d in list(_static_ws_devices):
+        try:
+            with torch.cuda.device(d):
+                load().w4a8_static_workspace_reset()
+        except Exception:
             pass
 
 
@@ -274,17 +285,24 @@ def quantize_act_per_token_asym(x: torch.Tensor, q_x: torch.Tensor | None = None
     return q_x, s_a, z_a
 
 
-def w4_zero_point_term(w_packed: torch.Tensor, S: torch.Tensor, group: int = 128) -> torch.Tensor:
+def w4_zero_point_term(w_packed: torch.Tensor, S: torch.Tensor, group: int = 128, *, colsum_max: int | None = None,
+                       qmin: int = -7) -> torch.Tensor:
     """zc [N] int32 = sum_g S[g, n] * sum_{k in g} q[k, n] from the packed codes
-    (the weight-side term of an asymmetric activation's zero point)."""
+    (the weight-side term of an asymmetric activation's zero point).
+    colsum_max: max_n sum_g |S[g, n]| as the pack reported it (taken from S
+    when not given); the library refuses weights whose asymmetric accumulator
+    could leave int32 (W4A8_ERR_OVERFLOW_BOUND)."""
     _need_cuda("w_packed", w_packed, torch.uint8, 2)
     _need_cuda("S", S, torch.int16, 2)
     N, K2 = w_packed.shape
     K = 2 * K2
     if S.shape != (K // group, N):
         raise ValueError("S must be [K / group, N]")
+    if colsum_max is None:
+        colsum_max = int(S.abs().to(torch.int64).sum(0).max().item())
     zc = torch.empty((N,), dtype=torch.int32, device=w_packed.device)
-    code = load().w4_zero_point_term(_ptr(w_packed), _ptr(S), K, N, group, _ptr(zc), _stream(w_packed.device))
+    code = load().w4_zero_point_term(_ptr(w_packed), _ptr(S), K, N, group, int(qmin), int(colsum_max), _ptr(zc),
+                                     _stream(w_packed.device))
     _check("w4_zero_point_term", code)
     return zc
 
@@ -382,6 +400,7 @@ def w4a8_gemm_intscale_static_ws(q_x, s_a, w_packed, S, alpha: int, *, group: in
     if y is None:
         y = torch.empty((M, N), dtype=tdt, device=q_x.device)
     _need_cuda("y", y, tdt, 2)
+    _static_ws_devices.add(torch.device(q_x.device).index)
     code = load().w4a8_gemm_intscale_static_ws(_ptr(q_x), _ptr(s_a), _ptr(w_packed), _ptr(S), int(alpha), M, N, K,
                                                group, _ptr(y), dt, _stream(q_x.device))
     _check("w4a8_gemm_intscale_static_ws", code)

@@ -43,7 +43,6 @@ struct StaticWorkspace {
 
 StaticWorkspace g_static_ws[kMaxDevices];
 std::mutex g_static_ws_mutex;
-std::mutex g_gemm_launch_mutex;
 
 // Device address of the current device's static workspace, looked up once per
 // device (the first call on a device does this set-up).
@@ -219,9 +218,6 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     p.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
     p.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
                                     : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
-    // The launchers set each kernel's shared-memory limit once per device,
-    // which is not safe to race: launches from several host threads take turns.
-    std::lock_guard<std::mutex> lock(g_gemm_launch_mutex);
     if (zp) {
         w4a8::gemm::ParamsZp pz{};
         static_cast<w4a8::gemm::Params&>(pz) = p;
@@ -326,9 +322,14 @@ w4a8_status quantize_act_per_token_asym(const void* x, int32_t x_dtype, int64_t 
 }
 
 w4a8_status w4_zero_point_term(const uint8_t* w_packed, const int16_t* S, int64_t K, int64_t N, int32_t group,
-                               int32_t* zc, void* stream) {
+                               int32_t qmin, int64_t colsum_max, int32_t* zc, void* stream) {
     if (K <= 0 || N <= 0 || group <= 0 || group % 32 != 0 || K % group != 0) return W4A8_ERR_SHAPE;
     if (K > INT32_MAX || N > INT32_MAX) return W4A8_ERR_SHAPE;
+    if (qmin != -7 && qmin != -8) return W4A8_ERR_INVALID_ARG;
+    if (colsum_max < 0) return W4A8_ERR_INVALID_ARG;
+    // asymmetric token codes span 255 values: the accumulator of the
+    // asymmetric GEMM stays exact only while 255 * |qmin| * group * colsum < 2^31
+    if (255.0 * double(-qmin) * double(group) * double(colsum_max) >= 2147483648.0) return W4A8_ERR_OVERFLOW_BOUND;
     if (!w_packed || !S || !zc) return W4A8_ERR_INVALID_ARG;
     if (!aligned16(w_packed) || (reinterpret_cast<uintptr_t>(S) & 1u) != 0 || !aligned4(zc)) return W4A8_ERR_ALIGN;
     DeviceInfo dev;
@@ -577,18 +578,29 @@ w4a8_status w4a8_device_status(int32_t* code_host, int32_t clear) {
     if (clear) {
         const int zero = 0;
         W4A8_CUDA_TRY(cudaMemcpy(dev.status, &zero, sizeof(int), cudaMemcpyHostToDevice));
-        if (v == W4A8_ERR_TIMEOUT) {
-            // a timed-out GEMM may have left split-tile arrival counts in the
-            // library's own workspace: zero its counter region (4096 bytes)
-            int d = 0;
-            W4A8_CUDA_TRY(cudaGetDevice(&d));
-            void* ws = nullptr;
-            {
-                std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-                if (d >= 0 && d < kMaxDevices && g_static_ws[d].ready) ws = g_static_ws[d].ptr;
-            }
-            if (ws) W4A8_CUDA_TRY(cudaMemset(ws, 0, 4096));
+        // Any device-side error may have cut a GEMM short (the word keeps only
+        // the last error, so a timeout can hide behind a later code): the
+        // split-tile arrival counts of the library's own workspace may be
+        // stale, so zero them whenever a nonzero status is cleared.
+        if (v != 0) {
+            const w4a8_status r = w4a8_static_workspace_reset();
+            if (r != W4A8_OK) return r;
         }
+    }
+    return W4A8_OK;
+}
+
+w4a8_status w4a8_static_workspace_reset(void) {
+    int d = 0;
+    W4A8_CUDA_TRY(cudaGetDevice(&d));
+    void* ws = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+        if (d >= 0 && d < kMaxDevices && g_static_ws[d].ready) ws = g_static_ws[d].ptr;
+    }
+    if (ws) {  // the arrival counters: the first 4096 bytes of the array
+        W4A8_CUDA_TRY(cudaMemset(ws, 0, 4096));
+        W4A8_CUDA_TRY(cudaDeviceSynchronize());
     }
     return W4A8_OK;
 }

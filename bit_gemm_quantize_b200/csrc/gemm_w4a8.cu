@@ -1051,20 +1051,8 @@ static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const
     using C = Cfg<BT, PATH, W8, ZP>;
     auto kern = w4a8_gemm_kernel<BT, PATH, W8, ZP>;
     const int smem = C::kSmemBytes;
-    // the shared-memory opt-in is a per-device function attribute: set it once
-    static bool configured[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    const cudaError_t e = configure_once(kern, C::kThreads, smem);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        int resident = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, C::kThreads, smem);
-        if (e != cudaSuccess) return e;
-        if (resident < 1) return cudaErrorLaunchOutOfResources;
-        if (dev >= 0 && dev < 64) configured[dev] = true;
-    }
     const LaunchPdl lc(unsigned(p.grid), C::kThreads, size_t(smem), stream);
     return cudaLaunchKernelEx(&lc.cfg, kern, tw, tx, ty, p);
 }

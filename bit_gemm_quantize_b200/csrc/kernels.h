@@ -4,8 +4,32 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 namespace w4a8 {
+
+// The dynamic shared-memory opt-in of a kernel is a per-device function
+// attribute: set it (and check that one CTA fits) once per (kernel, device),
+// the first time the kernel is launched on the device.  Thread-safe; later
+// launches only read the recorded result.
+template <typename Kernel>
+cudaError_t configure_once(Kernel kern, int threads, int smem) {
+    constexpr int kDevs = 64;
+    static std::once_flag once[kDevs];
+    static cudaError_t result[kDevs];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kDevs) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [&] {
+        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        int resident = 0;
+        if (r == cudaSuccess) r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&resident, kern, threads, smem);
+        if (r == cudaSuccess && resident < 1) r = cudaErrorLaunchOutOfResources;
+        result[dev] = r;
+    });
+    return result[dev];
+}
 
 // Launch configuration with programmatic stream serialization: the kernel
 // may start while the previous kernel in the stream is still running; it

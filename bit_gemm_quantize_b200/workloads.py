@@ -18,6 +18,14 @@ and weights are not available, so:
 
 Draw order from one ``numpy.random.Generator(PCG64(seed))``: X, then W, then
 the outlier channel indices, then the routing.
+
+Every layer drawn here is checked against the int32 accumulator bound before
+it is returned (``assert_int32_bound``): the kernels and the oracle both
+accumulate sum_g S[g,n] * P_g[m,n] in 32 bits, so a generated weight matrix
+whose integer scales could push that sum past 2^31 for some input is refused
+with ``ValueError``.  The check is a conservative upper bound computed from
+the raw weights (largest |w| per group, never a quantized code or scale), so
+it feeds no value to either side.
 """
 from __future__ import annotations
 
@@ -36,6 +44,8 @@ __all__ = [
     "bf16_bits_to_f32",
     "SWEEP_M",
     "CONFIGS",
+    "int32_bound_upper",
+    "assert_int32_bound",
 ]
 
 # FFN up-projection batch sweep of the pages' kernel comparison (K=4096, N=22016).
@@ -85,6 +95,42 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
+def int32_bound_upper(w: np.ndarray, group: int = 128, alpha: Optional[int] = 1024, qmax_w: int = 7,
+                      qmax_x: int = 127) -> float:
+    """An upper bound on qmax_x * qmax_w * group * max_n sum_g |S[g,n]| for the
+    integer scales S = round(s_g * alpha), s_g = max_{k in g}|w[k,n]| / qmax_w,
+    derived from the raw weights alone (fp64): each S is at most
+    amax * alpha / qmax_w inflated by 2^-20 (fp32 rounding of the scale) plus
+    1/2 (rounding to an integer).  alpha=None bounds the searched amplifier
+    (the smallest power of two lifting the smallest positive scale to 1) by
+    the next power of two above the reciprocal of a deflated smallest scale."""
+    w = np.asarray(w)
+    K, N = w.shape
+    if K % group:
+        raise ValueError("K must be a multiple of group")
+    # largest |w| per (group, column): exact in the input precision, widened after
+    amax = np.abs(w.reshape(K // group, group, N)).max(axis=1).astype(np.float64)  # [G, N]
+    if alpha is None:
+        pos = amax[amax > 0]
+        if pos.size == 0:
+            return 0.0
+        s_lo = pos.min() / qmax_w * (1.0 - 2.0 ** -20)
+        alpha = 1.0 if s_lo >= 1.0 else 2.0 ** np.ceil(np.log2(1.0 / s_lo))
+    s_up = amax * float(alpha) / qmax_w * (1.0 + 2.0 ** -20) + 0.5
+    s_up[amax == 0] = 0.0
+    return float(qmax_x) * qmax_w * group * float(s_up.sum(axis=0).max(initial=0.0))
+
+
+def assert_int32_bound(w: np.ndarray, group: int = 128, alpha: Optional[int] = 1024, qmax_w: int = 7,
+                       qmax_x: int = 127) -> None:
+    """Refuse (ValueError) weights whose integer-scale accumulators could leave
+    int32 for some input (the worst case of int32_bound_upper)."""
+    b = int32_bound_upper(w, group, alpha, qmax_w, qmax_x)
+    if b >= 2.0 ** 31:
+        raise ValueError(f"weights break the int32 accumulator bound: worst case {b:.3e} >= 2^31 "
+                         f"(group {group}, alpha {alpha})")
+
+
 def _outlier_count(K: int, frac: float) -> int:
     return int(round(frac * K))
 
@@ -100,8 +146,13 @@ def make_linear(
     n_outliers: Optional[int] = None,
     outlier_scale: float = 30.0,
     w_std: float = 0.02,
+    group: int = 128,
+    alpha: Optional[int] = 1024,
+    check_bound: bool = True,
 ) -> LinearWorkload:
-    """One linear layer's synthetic activations and weights."""
+    """One linear layer's synthetic activations and weights.  The weights are
+    checked against the int32 accumulator bound for (group, alpha) unless
+    check_bound is False (alpha=None: the searched amplifier)."""
     if x_dtype not in ("f32", "bf16"):
         raise ValueError(f"x_dtype must be 'f32' or 'bf16', got {x_dtype!r}")
     rng = np.random.Generator(np.random.PCG64(seed))
@@ -113,6 +164,8 @@ def make_linear(
         x[:, cols] *= np.float32(outlier_scale)
     if x_dtype == "bf16":
         x = bf16_bits_to_f32(to_bf16_bits(x))
+    if check_bound and K % group == 0:
+        assert_int32_bound(w, group, alpha)
     return LinearWorkload(x=x, w=w, x_dtype=x_dtype, outlier_cols=cols.astype(np.int64), seed=seed)
 
 
@@ -127,8 +180,13 @@ def make_moe(
     outlier_frac: float = 0.005,
     outlier_scale: float = 30.0,
     w_std: float = 0.02,
+    group: int = 128,
+    alpha: Optional[int] = None,
 ) -> MoEWorkload:
-    """A mixture-of-experts layer: per-expert weights plus top-k routing."""
+    """A mixture-of-experts layer: per-expert weights plus top-k routing.  The
+    amplifier is one per layer (alpha=None: searched over every expert's
+    scales), so the int32 bound is checked for each expert with the bound on
+    the layer's amplifier."""
     rng = np.random.Generator(np.random.PCG64(seed))
     x = rng.standard_normal((tokens, K), dtype=np.float32)
     ws = [
@@ -141,7 +199,28 @@ def make_moe(
         x[:, cols] *= np.float32(outlier_scale)
     x = bf16_bits_to_f32(to_bf16_bits(x))
     route = np.stack([rng.choice(experts, size=topk, replace=False) for _ in range(tokens)]).astype(np.int64)
+    if K % group == 0:
+        a_layer = alpha
+        if alpha is None:  # one amplifier bound for the whole layer: from all experts' weights
+            a_layer = _searched_alpha_upper(ws, group)
+        for w in ws:
+            assert_int32_bound(w, group, a_layer)
     return MoEWorkload(x=x, w=ws, experts=route, outlier_cols=cols.astype(np.int64), seed=seed)
+
+
+def _searched_alpha_upper(ws, group: int, qmax_w: int = 7) -> int:
+    """Upper bound on the amplifier searched over several weight matrices."""
+    lo = np.inf
+    for w in ws:
+        w = np.asarray(w)
+        K, N = w.shape
+        amax = np.abs(w.reshape(K // group, group, N)).max(axis=1).astype(np.float64)
+        pos = amax[amax > 0]
+        if pos.size:
+            lo = min(lo, pos.min() / qmax_w * (1.0 - 2.0 ** -20))
+    if not np.isfinite(lo) or lo >= 1.0:
+        return 1
+    return int(2.0 ** np.ceil(np.log2(1.0 / lo)))
 
 
 def route_rows(experts: np.ndarray, n_experts: int):

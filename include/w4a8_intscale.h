@@ -32,6 +32,13 @@
  *  - Kernels bound every wait; a wait that runs out (about one second) makes
  *    the kernel return early and records W4A8_ERR_TIMEOUT in a device status
  *    word that w4a8_device_status() reads.
+ *  - The GEMMs run a persistent grid of at most one CTA per resident slot
+ *    (SMs x CTAs per SM) and split the (tile, group) steps into one range per
+ *    CTA.  A tile cut by two ranges is finished by one of its CTAs, which
+ *    waits for the others' partial sums: this assumes that every CTA of the
+ *    grid becomes resident.  A kernel on another stream that holds SMs for
+ *    long can delay a call by up to the wait limit, after which it fails with
+ *    W4A8_ERR_TIMEOUT instead of waiting forever.
  *  - Layouts are row-major.  All device pointers must be 16-byte aligned.
  *  - Readings where the pages are silent: round() is round half to even;
  *    an all-zero row or group gets scale 0 and codes 0; int4 codes are
@@ -240,12 +247,19 @@ W4A8_API w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, con
  * w_packed  device, [N, K/2] uint8, 16-byte aligned; S device [K/group, N] int16
  *           (from pack_w4_groupwise or pack_w4_groupwise_range)
  * K, N      K % group == 0, group % 32 == 0; otherwise W4A8_ERR_SHAPE
+ * qmin      the code range the weights were packed with: -7 ([-7, 7]) or -8 ([-8, 7])
+ * colsum_max  max_n sum_g |S[g,n]| as the pack call reported it (colsum_max_host)
  * zc        device, [N] int32, written
- * Errors: W4A8_ERR_INVALID_ARG for a NULL pointer; W4A8_ERR_ALIGN unless w_packed is
- * 16-byte, S 2-byte and zc 4-byte aligned.
+ * Errors: W4A8_ERR_OVERFLOW_BOUND, before anything is launched, when
+ * 255 * |qmin| * group * colsum_max >= 2^31: the asymmetric GEMM's accumulator
+ * would not be exact in int32 for every input (codes minus zero points span
+ * 255 values); W4A8_ERR_INVALID_ARG for a NULL pointer, another qmin or a
+ * negative colsum_max; W4A8_ERR_ALIGN unless w_packed is 16-byte, S 2-byte
+ * and zc 4-byte aligned.
  */
 W4A8_API w4a8_status w4_zero_point_term(const uint8_t* w_packed, const int16_t* S, int64_t K, int64_t N,
-                                        int32_t group, int32_t* zc, void* stream);
+                                        int32_t group, int32_t qmin, int64_t colsum_max, int32_t* zc,
+                                        void* stream);
 
 /*
  * W4A8 integer-scale GEMM of asymmetric token codes (from
@@ -258,7 +272,8 @@ W4A8_API w4a8_status w4_zero_point_term(const uint8_t* w_packed, const int16_t* 
  * two's-complement int32 arithmetic: the intermediate terms may wrap, the
  * result is exact when acc itself fits in int32, which holds when
  * 255*qw*group*max_n sum_g |S[g,n]| < 2^31 (255 = the widest |q_x - z_a|;
- * qw = 7, or 8 for codes in the full range [-8, 7]).
+ * qw = 7, or 8 for codes in the full range [-8, 7]); w4_zero_point_term
+ * refuses weights that break this bound, so a zc it wrote meets it.
  * z_a        device, [M] int32 (4-byte aligned)
  * zc         device, [N] int32 from w4_zero_point_term (4-byte aligned)
  * Other arguments, workspace (path 0), output (W4A8_I32: acc itself) and
@@ -371,12 +386,20 @@ W4A8_API const char* w4a8_cuda_error_string(int32_t code);
  * Reads (and with clear != 0 resets) the device status word of the current
  * device: 0, or the last device-side error: W4A8_ERR_TIMEOUT (a bounded wait
  * ran out) or W4A8_ERR_INVALID_ARG (a routed row's token index out of range in
- * w4a8_moe_gemm_intscale).  Synchronous.  Clearing a W4A8_ERR_TIMEOUT also
- * zeroes the arrival counters of the library's own workspace
- * (w4a8_gemm_intscale_static_ws); caller workspaces must be zeroed by the
- * caller.
+ * w4a8_moe_gemm_intscale).  Synchronous.  The word keeps only the last error,
+ * so clearing any nonzero status also zeroes the arrival counters of the
+ * library's own workspace (w4a8_static_workspace_reset); caller workspaces
+ * must be zeroed by the caller.
  */
 W4A8_API w4a8_status w4a8_device_status(int32_t* code_host, int32_t clear);
+
+/*
+ * Zeroes the split-tile arrival counters of the library's own workspace (the
+ * one w4a8_gemm_intscale_static_ws uses) on the current device, if that
+ * workspace has been set up there; synchronous.  Needed after a call that
+ * failed or timed out, which may leave counts behind.  Allocates nothing.
+ */
+W4A8_API w4a8_status w4a8_static_workspace_reset(void);
 
 #ifdef __cplusplus
 }

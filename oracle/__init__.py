@@ -94,10 +94,10 @@ def _load():
                 "oracle_unpack_int4": ([P, I, I, P], None),
                 "oracle_amplifier_search": ([P, I], I32),
                 "oracle_integer_scales": ([P, I, I32, P], None),
-                "oracle_intscale_acc": ([P, P, P, I, I, I, I, P], None),
+                "oracle_intscale_acc": ([P, P, P, I, I, I, I, P], I),
                 "oracle_intscale_acc_expanded": ([P, P, P, I, I, I, I, P], None),
-                "oracle_intscale_acc_at": ([P, P, P, I, I, I, I, P, P, I, P], None),
-                "oracle_intscale_acc_asym": ([P, P, P, P, I, I, I, I, P], None),
+                "oracle_intscale_acc_at": ([P, P, P, I, I, I, I, P, P, I, P], I),
+                "oracle_intscale_acc_asym": ([P, P, P, P, I, I, I, I, P], I),
                 "oracle_intscale_output": ([P, P, I32, I, I, P], None),
                 "oracle_floatscale": ([P, P, P, P, I, I, I, I, P], None),
                 "oracle_floatscale_at": ([P, P, P, P, I, I, I, I, P, P, I, P], None),
@@ -226,14 +226,35 @@ def scale_colsum_max(S) -> int:
 
 # ---------------------------------------------------------------- GEMMs
 
+class Int32BoundError(ValueError):
+    """An integer accumulator of the layer does not fit the int32 range the
+    kernels accumulate in (the Integer Scale summary, §4: the amplifier stays
+    at 1024 so that integer accumulation does not overflow)."""
+
+
+def _int32_checked(bad: int, what: str):
+    if bad:
+        raise Int32BoundError(f"{what}: {bad} accumulator(s) outside the int32 range")
+
+
+def check_worst_case(S, group: int, qx_max: int = INT8_QMAX, qw_max: int = INT4_QMAX):
+    """Raise Int32BoundError unless qx_max * qw_max * group * max_n sum_g |S[g,n]|
+    < 2^31: then no input whatever can push an accumulator out of int32."""
+    worst = int(qx_max) * int(qw_max) * int(group) * scale_colsum_max(S)
+    if worst >= 1 << 31:
+        raise Int32BoundError(f"worst-case accumulator {worst} >= 2^31")
+
+
 def intscale_acc(qx, qw, S, group: int = 128):
+    """Raw integer-scale accumulators acc [M, N] (int64); raises
+    Int32BoundError when any of them lies outside (-2^31, 2^31)."""
     qx = _c(qx, np.int8)
     qw = _c(qw, np.int8)
     S = _c(S, np.int32)
     M, K = qx.shape
     N = qw.shape[1]
     acc = np.empty((M, N), np.int64)
-    _load().oracle_intscale_acc(_p(qx), _p(qw), _p(S), M, N, K, group, _p(acc))
+    _int32_checked(_load().oracle_intscale_acc(_p(qx), _p(qw), _p(S), M, N, K, group, _p(acc)), "intscale_acc")
     return acc
 
 
@@ -257,7 +278,8 @@ def intscale_acc_at(qx, qw, S, ms, ns, group: int = 128):
     M, K = qx.shape
     N = qw.shape[1]
     acc = np.empty(ms.size, np.int64)
-    _load().oracle_intscale_acc_at(_p(qx), _p(qw), _p(S), M, N, K, group, _p(ms), _p(ns), ms.size, _p(acc))
+    _int32_checked(_load().oracle_intscale_acc_at(_p(qx), _p(qw), _p(S), M, N, K, group, _p(ms), _p(ns), ms.size,
+                                                  _p(acc)), "intscale_acc_at")
     return acc
 
 
@@ -269,7 +291,8 @@ def intscale_acc_asym(qx, z, qw, S, group: int = 128):
     M, K = qx.shape
     N = qw.shape[1]
     acc = np.empty((M, N), np.int64)
-    _load().oracle_intscale_acc_asym(_p(qx), _p(z), _p(qw), _p(S), M, N, K, group, _p(acc))
+    _int32_checked(_load().oracle_intscale_acc_asym(_p(qx), _p(z), _p(qw), _p(S), M, N, K, group, _p(acc)),
+                   "intscale_acc_asym")
     return acc
 
 
@@ -343,6 +366,12 @@ def linear_intscale(x, w, *, group: int = 128, alpha=1024, out: str = "f16", qmi
         qw, s_g = quantize_groups(w, group, qmin=qmin)
     a = amplifier_search(s_g) if alpha is None else int(alpha)
     S = integer_scales(s_g, a)
+    # the worst case over every input the layer may see must fit in int32
+    # (the column bound the pack step checks): widest |code| of each operand
+    # times group times the largest column sum of |S|
+    qx_max = 255 if asym else INT8_QMAX
+    qw_max = INT8_QMAX if wbits == 8 else (8 if qmin == -8 else INT4_QMAX)
+    check_worst_case(S, group, qx_max, qw_max)
     acc = intscale_acc_asym(qx, z, qw, S, group) if asym else intscale_acc(qx, qw, S, group)
     y64 = intscale_output(acc, s_a, a)
     packed = np.ascontiguousarray(qw.T) if wbits == 8 else pack_int4(qw)
@@ -380,6 +409,8 @@ def moe_intscale(x, ws, row_index, offsets, *, group: int = 128, alpha=1024, out
         sgs.append(sg)
     a = amplifier_search(np.concatenate([sg.reshape(-1) for sg in sgs])) if alpha is None else int(alpha)
     Ss = [integer_scales(sg, a) for sg in sgs]
+    for S in Ss:
+        check_worst_case(S, group)
     row_index = np.asarray(row_index, np.int64)
     N = ws[0].shape[1]
     acc = np.zeros((row_index.shape[0], N), np.int64)

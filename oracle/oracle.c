@@ -36,8 +36,11 @@
  *  - round() is round-half-to-even (C rint() in the default rounding mode);
  *  - an all-zero row or group gets scale 0 and codes 0;
  *  - int4 weights are symmetric with qmax = 7 (range [-7, 7]);
- *  - nibble packing: byte n*(K/2) + k/2 holds q[k] in its low nibble and
- *    q[k+1] in its high nibble (two's complement), K-contiguous per column n;
+ *  - nibble packing, K-contiguous per column n: every 8 codes along K fill
+ *    one 32-bit word (4 bytes); code i of the 8 sits in byte i mod 4, in the
+ *    low nibble for i < 4 and the high nibble for i >= 4 (two's complement);
+ *  - the GEMM accumulates in int32: every accumulator of a call must lie in
+ *    (-2^31, 2^31); the accumulating functions count those that do not;
  *  - the amplifier search ignores zero scales, and returns 1 when the
  *    smallest scale is already >= 1.
  */
@@ -249,11 +252,16 @@ void oracle_integer_scales(const float* s_g, int64_t count, int32_t alpha, int32
 
 /* ---- [IS] Fig. 3(c): group integer GEMM + integer-scale accumulation ------ */
 
+/* 1 when an accumulator leaves the int32 range the GPU accumulates in
+ * ([IS] §4: the amplifier is kept at 1024 to stay clear of overflow). */
+static int32_t outside_int32(int64_t v) { return v >= ((int64_t)1 << 31) || v <= -((int64_t)1 << 31); }
+
 /* acc[m,n] = sum_g S[g,n] * P_g[m,n],  P_g[m,n] = sum_{k in g} qx[m,k] qw[k,n]
- * qx [M,K], qw [K,N] codes, S [G,N]; everything in int64. */
-void oracle_intscale_acc(const int8_t* qx, const int8_t* qw, const int32_t* S, int64_t M,
-                         int64_t N, int64_t K, int64_t group, int64_t* acc) {
-    int64_t G = K / group;
+ * qx [M,K], qw [K,N] codes, S [G,N]; everything in int64.  Returns how many
+ * accumulators lie outside int32 (0 for a valid input). */
+int64_t oracle_intscale_acc(const int8_t* qx, const int8_t* qw, const int32_t* S, int64_t M,
+                            int64_t N, int64_t K, int64_t group, int64_t* acc) {
+    int64_t G = K / group, bad = 0;
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
             int64_t total = 0;
@@ -264,7 +272,9 @@ void oracle_intscale_acc(const int8_t* qx, const int8_t* qw, const int32_t* S, i
                 total += (int64_t)S[g * N + n] * p;
             }
             acc[m * N + n] = total;
+            bad += outside_int32(total);
         }
+    return bad;
 }
 
 /* The same integer reached the other way round: first the integer weight
@@ -283,11 +293,11 @@ void oracle_intscale_acc_expanded(const int8_t* qx, const int8_t* qw, const int3
 }
 
 /* Group-wise accumulators at selected output positions (m_i, n_i) only. */
-void oracle_intscale_acc_at(const int8_t* qx, const int8_t* qw, const int32_t* S, int64_t M,
-                            int64_t N, int64_t K, int64_t group, const int64_t* ms,
-                            const int64_t* ns, int64_t count, int64_t* acc) {
+int64_t oracle_intscale_acc_at(const int8_t* qx, const int8_t* qw, const int32_t* S, int64_t M,
+                               int64_t N, int64_t K, int64_t group, const int64_t* ms,
+                               const int64_t* ns, int64_t count, int64_t* acc) {
     (void)M;
-    int64_t G = K / group;
+    int64_t G = K / group, bad = 0;
     for (int64_t i = 0; i < count; ++i) {
         int64_t m = ms[i], n = ns[i];
         int64_t total = 0;
@@ -298,16 +308,18 @@ void oracle_intscale_acc_at(const int8_t* qx, const int8_t* qw, const int32_t* S
             total += (int64_t)S[g * N + n] * p;
         }
         acc[i] = total;
+        bad += outside_int32(total);
     }
+    return bad;
 }
 
 /* Integer-scale accumulation with an asymmetric activation ([Q-mm] with
  * Z_W = 0 and Z_X = z[m]; [IS] §4 integer group scales):
  * acc[m,n] = sum_g S[g,n] * sum_{k in g} (qx[m,k] - z[m]) * qw[k,n].
  * The final rescale is the same as the symmetric one, acc * s_a[m] / alpha. */
-void oracle_intscale_acc_asym(const int8_t* qx, const int32_t* z, const int8_t* qw, const int32_t* S,
-                              int64_t M, int64_t N, int64_t K, int64_t group, int64_t* acc) {
-    int64_t G = K / group;
+int64_t oracle_intscale_acc_asym(const int8_t* qx, const int32_t* z, const int8_t* qw, const int32_t* S,
+                                 int64_t M, int64_t N, int64_t K, int64_t group, int64_t* acc) {
+    int64_t G = K / group, bad = 0;
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
             int64_t total = 0;
@@ -318,7 +330,9 @@ void oracle_intscale_acc_asym(const int8_t* qx, const int32_t* z, const int8_t* 
                 total += (int64_t)S[g * N + n] * p;
             }
             acc[m * N + n] = total;
+            bad += outside_int32(total);
         }
+    return bad;
 }
 
 /* Final rescale, once per output: y = acc * s_a[m] / alpha, in fp64 ([IS] §4). */

@@ -189,14 +189,22 @@ def test_asymmetric_argument_checks(lib):
     assert qa(x=U) == ALIGN
     assert qa(z=A + 2) == ALIGN
 
-    def zt(wp=A, K=256, group=128, zc=A):
-        return lib.w4_zero_point_term(ctypes.c_void_p(wp), ctypes.c_void_p(A), K, 128, group, ctypes.c_void_p(zc), None)
+    def zt(wp=A, K=256, group=128, zc=A, qmin=-7, colsum=16):
+        return lib.w4_zero_point_term(ctypes.c_void_p(wp), ctypes.c_void_p(A), K, 128, group, qmin, colsum,
+                                      ctypes.c_void_p(zc), None)
 
     assert zt(K=200) == SHAPE
     assert zt(group=48) == SHAPE
     assert zt(zc=0) == INVALID
     assert zt(wp=U) == ALIGN
     assert zt(zc=A + 2) == ALIGN
+    assert zt(qmin=-6) == INVALID
+    assert zt(colsum=-1) == INVALID
+    # the asymmetric accumulator's worst case, 255 * |qmin| * group * colsum, must stay below 2^31
+    OVERFLOW = 5
+    assert zt(colsum=(1 << 31) // (255 * 7 * 128) + 1) == OVERFLOW
+    assert zt(colsum=(1 << 31) // (255 * 8 * 128) + 1, qmin=-8) == OVERFLOW
+    assert zt(colsum=(1 << 31) // (255 * 8 * 128) + 1, qmin=-8, zc=0) == OVERFLOW  # refused before anything else
 
     def ga(z=A, zc=A, M=16, dt=_native.F16, alpha=1024):
         return lib.w4a8_gemm_intscale_asym(ctypes.c_void_p(A), ctypes.c_void_p(A), ctypes.c_void_p(z),

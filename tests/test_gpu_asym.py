@@ -82,7 +82,8 @@ def test_zero_point_term_bitexact(K, N, qmin):
     dev = _dev()
     wl = workloads.make_linear(1, K, N, seed=K + N)
     pk = bgq.pack_w4_groupwise(torch.from_numpy(wl.w).to(dev), group=128, alpha=None, qmin=qmin)
-    zc = bgq.w4_zero_point_term(pk["packed"], pk["S"], group=128).cpu().numpy()
+    zc = bgq.w4_zero_point_term(pk["packed"], pk["S"], group=128, colsum_max=pk["colsum_max"],
+                                qmin=qmin).cpu().numpy()
     qw, sg = oracle.quantize_groups(wl.w, 128, qmin=None if qmin == -7 else qmin)
     S = oracle.integer_scales(sg, oracle.amplifier_search(sg))
     want = (np.repeat(S.astype(np.int64), 128, axis=0) * qw.astype(np.int64)).sum(axis=0)
@@ -100,6 +101,18 @@ ASYM_CASES = [
     (130, 768, 1032, 1.25),
     (300, 1024, 256, 3.0),
 ]
+
+
+def test_zero_point_term_refuses_weights_beyond_the_asymmetric_bound():
+    """Integer scales whose column sums are too large for 255-wide token codes
+    are refused before anything is launched."""
+    dev = _dev()
+    w = torch.full((128 * 64, 8), 0.51, device=dev)  # s_g = 0.51/7; S = 149 at alpha 2^11
+    pk = bgq.pack_w4_groupwise(w, alpha=1 << 11)  # 127 * 7 * 128 * 64 * 149 = 1.09e9: the symmetric bound holds
+    assert pk["colsum_max"] == 64 * 149
+    with pytest.raises(bgq.W4A8Error) as e:  # 255 * 7 * 128 * 64 * 149 = 2.18e9 >= 2^31
+        bgq.w4_zero_point_term(pk["packed"], pk["S"], group=128, colsum_max=pk["colsum_max"])
+    assert e.value.code == 5
 
 
 @pytest.mark.parametrize("M,K,N,offset", ASYM_CASES)

@@ -107,3 +107,50 @@ def test_moe_mixtral_shaped_sampled():
         ns = rng.integers(0, N, 40)
         want = oracle.intscale_acc_at(qx[ri[lo:hi].astype(np.int64)], qw, S, ms, ns)
         assert np.array_equal(a[lo + ms, ns], want)
+
+
+def test_moe_mixtral_full_layer_sampled():
+    """The whole Mixtral-shaped layer the benchmark times: 2048 tokens, 8
+    experts of W [4096, 14336], top-2 routing, one amplifier searched over all
+    experts' group scales.  Codes, token scales, the amplifier and every
+    expert's packed weights and integer scales bit-exact in full; raw
+    accumulators and fp16 outputs at samples spread over every expert and
+    every 128-column tile."""
+    T, K, N, E = 2048, 4096, 14336, 8
+    wl = workloads.make_moe(T, K, N, E, topk=2, seed=21)
+    ri, off = workloads.route_rows(wl.experts, E)
+    dev = torch.device("cuda:0")
+    x = torch.from_numpy(wl.x).to(dev).to(torch.bfloat16)
+    q, s = bgq.quantize_act_per_token(x)
+    pk = bgq.pack_moe_experts([torch.from_numpy(w).to(dev) for w in wl.w], alpha=None)
+    ri_d = torch.from_numpy(ri).to(dev)
+    acc = bgq.w4a8_moe_gemm_intscale(q, s, ri_d, off, pk["packed"], pk["S"], pk["alpha"], out="i32")
+    y = bgq.w4a8_moe_gemm_intscale(q, s, ri_d, off, pk["packed"], pk["S"], pk["alpha"], out="f16")
+    torch.cuda.synchronize()
+    assert bgq.device_status() == 0
+
+    qx, s_a = oracle.quantize_act_per_token(wl.x)
+    assert np.array_equal(q.cpu().numpy(), qx)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_a.view(np.uint32))
+    qws, sgs = zip(*[oracle.quantize_groups(w, 128) for w in wl.w])
+    alpha = oracle.amplifier_search(np.concatenate([sg.reshape(-1) for sg in sgs]))
+    assert pk["alpha"] == alpha
+    a = acc.cpu().numpy().astype(np.int64)
+    yh = y.float().cpu().numpy()
+    rng = np.random.default_rng(17)
+    for e in range(E):
+        S = oracle.integer_scales(sgs[e], alpha)
+        oracle.check_worst_case(S, 128)
+        assert np.array_equal(pk["S"][e].cpu().numpy().astype(np.int32), S)
+        assert np.array_equal(pk["packed"][e].cpu().numpy(), oracle.pack_int4(qws[e]))
+        lo, hi = int(off[e]), int(off[e + 1])
+        assert hi > lo
+        tiles = np.repeat(np.arange(N // 128), 2)  # two samples in every column tile
+        ns = tiles * 128 + rng.integers(0, 128, tiles.size)
+        ms = rng.integers(0, hi - lo, tiles.size)
+        ms[:2] = [0, hi - lo - 1]  # the expert's first and last rows
+        toks = ri[lo:hi].astype(np.int64)
+        want = oracle.intscale_acc_at(qx[toks], qws[e], S, ms, ns)
+        assert np.array_equal(a[lo + ms, ns], want)
+        y_ref = want.astype(np.float64) * s_a[toks[ms]].astype(np.float64) / alpha
+        _close(yh[lo + ms, ns], y_ref, "f16")

@@ -334,12 +334,55 @@ def _sampled_check(M, K, N, dev, seed, n_samples=1500):
     _assert_close(yf[ms, ns], yf_ref, "f16")
 
 
+def _rows_parallel(fn, M):
+    """fn(lo, hi) -> the oracle's rows lo..hi-1, run over row blocks on host
+    threads (the C oracle releases the interpreter lock while it runs) and
+    stacked: the same arithmetic, row by row, in less wall time."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    blocks = [(lo, min(M, lo + 2)) for lo in range(0, M, 2)]
+    with ThreadPoolExecutor(max_workers=min(16, len(blocks))) as ex:
+        parts = list(ex.map(lambda b: fn(*b), blocks))
+    return np.concatenate(parts, axis=0)
+
+
+def _full_check(M, K, N, dev, seed):
+    """Every element of the layer against the oracle, at the launch
+    configuration the benchmark uses: codes, token-scale bits, packed bytes,
+    integer scales, all M x N raw accumulators bit-exact; the integer-scale
+    and float-scale fp16 outputs within tolerance."""
+    wl = workloads.make_linear(M, K, N, x_dtype="bf16", seed=seed)
+    q, s, pk = _gpu_layer(wl, dev, 128, 1024)
+    qx, sa = oracle.quantize_act_per_token(wl.x)
+    qw, sg = oracle.quantize_groups(wl.w, 128)
+    S = oracle.integer_scales(sg, 1024)
+    oracle.check_worst_case(S, 128)
+    assert np.array_equal(q.cpu().numpy(), qx)
+    assert np.array_equal(_bits(s.cpu().numpy()), _bits(sa))
+    assert np.array_equal(pk["packed"].cpu().numpy(), oracle.pack_int4(qw))
+    assert np.array_equal(pk["S"].cpu().numpy().astype(np.int32), S)
+    acc_ref = _rows_parallel(lambda lo, hi: oracle.intscale_acc(qx[lo:hi], qw, S, 128), M)
+    acc = bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], 1024, out="i32").cpu().numpy()
+    assert np.array_equal(acc.astype(np.int64), acc_ref)
+    y = bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], 1024, out="f16").float().cpu().numpy()
+    _assert_close(y, oracle.intscale_output(acc_ref, sa, 1024), "f16")
+    yf_ref = _rows_parallel(lambda lo, hi: oracle.floatscale(qx[lo:hi], sa[lo:hi], qw, sg, 128), M)
+    yf = bgq.w4a8_gemm_floatscale(q, s, pk["packed"], pk["s_g"], out="f16").float().cpu().numpy()
+    _assert_close(yf, yf_ref, "f16")
+    assert bgq.device_status() == 0
+
+
 @pytest.mark.parametrize("M", [1, 4, 16])
-def test_decode_full_size_sampled(M):
-    _sampled_check(M, 4096, 4096, _dev(), seed=100 + M)
+def test_decode_full_size_every_element(M):
+    _full_check(M, 4096, 4096, _dev(), seed=100 + M)
 
 
-@pytest.mark.parametrize("M", workloads.SWEEP_M)
+@pytest.mark.parametrize("M", [m for m in workloads.SWEEP_M if m <= 32])
+def test_ffn_sweep_full_size_every_element(M):
+    _full_check(M, 4096, 22016, _dev(), seed=200 + M)
+
+
+@pytest.mark.parametrize("M", [m for m in workloads.SWEEP_M if m > 32])
 def test_ffn_sweep_full_size_sampled(M):
     _sampled_check(M, 4096, 22016, _dev(), seed=200 + M, n_samples=800)
 

@@ -383,6 +383,44 @@ def test_workload_bound_holds_for_default_amplifier():
     assert 127 * 7 * 128 * oracle.scale_colsum_max(S) < 2 ** 31
 
 
+def test_oracle_refuses_accumulators_outside_int32():
+    """Extreme codes with scales large enough to pass 2^31: the oracle raises
+    instead of returning an accumulator the int32 GPU path cannot hold."""
+    K, N = 1024, 4
+    qx = np.full((1, K), 127, np.int8)
+    qw = np.full((K, N), 7, np.int8)
+    S = np.full((K // 128, N), 2400, np.int32)  # 127 * 7 * 128 * 8 * 2400 = 2.18e9 > 2^31
+    with pytest.raises(oracle.Int32BoundError):
+        oracle.intscale_acc(qx, qw, S)
+    with pytest.raises(oracle.Int32BoundError):
+        oracle.intscale_acc_at(qx, qw, S, [0], [1])
+    with pytest.raises(oracle.Int32BoundError):
+        oracle.check_worst_case(S, 128)
+    S[:] = 2300  # 2.09e9 < 2^31: fine
+    acc = oracle.intscale_acc(qx, qw, S)
+    assert int(acc.max()) == 127 * 7 * 128 * 8 * 2300
+    oracle.check_worst_case(S, 128)
+
+
+def test_generator_refuses_weights_beyond_the_int32_bound():
+    """The seeded generator checks every layer it returns against the worst-case
+    accumulator bound (a conservative upper bound from the raw weights)."""
+    with pytest.raises(ValueError):
+        workloads.make_linear(1, 4096, 64, w_std=2.0, seed=1)  # S ~ 1000 over 32 groups
+    with pytest.raises(ValueError):
+        workloads.make_moe(4, 4096, 64, 2, w_std=2.0, alpha=1024, seed=1)
+    wl = workloads.make_linear(1, 4096, 64, w_std=2.0, seed=1, alpha=None)  # searched amplifier: fine
+    # the generator's bound is an upper bound of the exact worst case the oracle computes
+    for alpha in (1024, None):
+        wl = workloads.make_linear(2, 2048, 96, seed=5, alpha=alpha)
+        qw, s_g = oracle.quantize_groups(wl.w, 128)
+        a = oracle.amplifier_search(s_g) if alpha is None else alpha
+        S = oracle.integer_scales(s_g, a)
+        exact = 127 * 7 * 128 * oracle.scale_colsum_max(S)
+        upper = workloads.int32_bound_upper(wl.w, 128, alpha)
+        assert exact <= upper <= exact * 1.2 + 127 * 7 * 128 * 16
+
+
 # ------------------------------------------------------------ mixture of experts (the Mixtral results)
 
 def test_route_rows_layout():

@@ -23,11 +23,15 @@ def _inputs(M, K, N, seed):
     return q, s, pk
 
 
-# token tiles 16 and 32, with stream-K partitions that cut tiles (so the
-# workspace is used) and one that does not
-@pytest.mark.parametrize("M,K,N", [(1, 4096, 2048), (8, 2048, 1024), (32, 4096, 2048), (16, 128, 256)])
+# token tiles 16, 32 and 64, with stream-K partitions that cut tiles (so the
+# workspace is used; M = 48 takes the 64-token tile, the widest whose plans fit
+# the 8 MiB array) and one that cuts none
+@pytest.mark.parametrize("M,K,N,cuts", [(1, 4096, 2048, True), (8, 2048, 1024, True), (32, 4096, 2048, True),
+                                        (48, 4096, 2048, True), (16, 128, 256, False)])
 @pytest.mark.parametrize("out", ["i32", "f16"])
-def test_static_workspace_matches_caller_workspace(M, K, N, out):
+def test_static_workspace_matches_caller_workspace(M, K, N, cuts, out):
+    need = bgq.load().w4a8_gemm_workspace_size(M, N, K, 128, 0)
+    assert (need > 0) == cuts and need <= (8 << 20)
     q, s, pk = _inputs(M, K, N, seed=101 + M)
     ref = bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], pk["alpha"], group=128, out=out)
     for _ in range(2):  # two calls in a row: the counters must come back to zero
