@@ -231,35 +231,63 @@ class OracleLeg:
         self.qw, sg = oracle.quantize_groups(wl.w, GROUP)
         self.S = oracle.integer_scales(sg, ALPHA)
 
-    def run(self, rows: int, seed: int):
+    def run(self, rows: int, seed: int, threads: int = 1):
+        """Time `rows` token rows through the oracle.  threads > 1 splits the
+        rows over host threads, one oracle call per row (the C oracle releases
+        the interpreter lock while it runs, so the calls use separate cores)."""
         o = self.oracle
-        x = workloads.make_linear(rows, K_DIM, 8, x_dtype="bf16", seed=seed).x
+        x = workloads.make_linear(rows, K_DIM, 8, x_dtype="bf16", seed=seed, check_bound=False).x
+
+        def one(lo, hi):
+            qx, sa = o.quantize_act_per_token(x[lo:hi])
+            acc = o.intscale_acc(qx, self.qw, self.S, GROUP)
+            return o.round_output(o.intscale_output(acc, sa, ALPHA), "f16")
+
         t0 = time.perf_counter()
-        qx, sa = o.quantize_act_per_token(x)
-        acc = o.intscale_acc(qx, self.qw, self.S, GROUP)
-        y = o.round_output(o.intscale_output(acc, sa, ALPHA), "f16")
+        if threads <= 1:
+            y = one(0, rows)
+        else:
+            from concurrent.futures import ThreadPoolExecutor
+
+            with ThreadPoolExecutor(max_workers=threads) as ex:
+                y = np.concatenate(list(ex.map(lambda m: one(m, m + 1), range(rows))))
         dt = time.perf_counter() - t0
         assert y.shape == (rows, N_DIM)
         return dt
 
 
-def cpu_oracle_sample(rows: int = 32, seed: int = 1):
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_sample(seed: int = 1):
+    """The oracle on the host cores: single-threaded on 8 token rows, and on
+    every core on as many rows as there are cores (x2, at least 16)."""
     leg = OracleLeg(seed)
-    dt = leg.run(rows, seed + 1)
-    return {"value": alg_ops(rows) / dt / 1e12, "unit": "TOPS", "cores": 1, "kind": "oracle",
-            "sample": f"{rows} token rows x full K={K_DIM}, N={N_DIM} layer: per-token quantize + "
-                      f"group-wise integer GEMM + rescale, single-threaded C, {dt:.1f} s"}
+    dt1 = leg.run(8, seed + 1)
+    cores = host_cores()
+    rows_n = max(16, 2 * cores)
+    dtn = leg.run(rows_n, seed + 2, threads=cores)
+    return {"value": alg_ops(rows_n) / dtn / 1e12, "unit": "TOPS", "cores": cores, "kind": "oracle",
+            "single_core_value": alg_ops(8) / dt1 / 1e12,
+            "sample": f"{rows_n} token rows x full K={K_DIM}, N={N_DIM} layer on {cores} threads ({dtn:.1f} s); "
+                      f"single core: 8 rows ({dt1:.1f} s); per-token quantize + group-wise integer GEMM + "
+                      "rescale"}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    rows = 2
+    cores = host_cores()
+    rows = cores  # one row per core per step
     leg = OracleLeg(1)
     total_t = 0.0
     for i in range(args.warmup + args.steps):
-        dt = leg.run(rows, 10 + i)
+        dt = leg.run(rows, 10 + i, threads=cores)
         if i >= args.warmup:
             total_t += dt
     v = alg_ops(rows) * args.steps / total_t / 1e12
@@ -268,13 +296,113 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8xi4->i64",
         "data": "synthetic", "config": config_dict(),
-        "cpu_baseline": {"value": v, "unit": "TOPS", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": v, "unit": "TOPS", "cores": cores, "kind": "oracle",
                          "sample": f"each step: {rows} token rows x full K={K_DIM}, N={N_DIM} layer through the "
-                                   "oracle (quantize + group-wise integer GEMM + rescale), single-threaded C"},
+                                   f"oracle (quantize + group-wise integer GEMM + rescale), one row per host "
+                                   f"thread on {cores} threads"},
         "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ---------------------------------------------------------------- int8 tensor peak
+
+def measure_int8_peak(dev, world, iters=20000, reps=5):
+    """The int8 tensor-core rate of this GPU, measured: back-to-back
+    tcgen05.mma.kind::i8 (128 x 256 x 32, operands in shared memory, one CTA
+    per SM, no loads or epilogue), CUDA events around `reps` launches.  Also
+    the 128 x 128 shape with the weight operand in TMEM, as the GEMM issues it."""
+    import torch
+
+    import bit_gemm_quantize_b200 as bgq
+
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for key, n, a_tmem in (("ss_n256", 256, False), ("ts_n128", 128, True)):
+        for _ in range(2):
+            bgq.tensor_i8_peak_probe(iters, n, a_tmem, device=dev)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            ops = bgq.tensor_i8_peak_probe(iters, n, a_tmem, device=dev)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = max_over_ranks([e0.elapsed_time(e1) / reps], world, dev)[0]
+        out[key] = ops / (ms * 1e-3) / 1e12
+    assert bgq.device_status() == 0
+    return out
+
+
+DECODE = dict(K=4096, N=4096, M=[1, 4, 16])
+
+
+def measure_decode(dev, rank, world, hbm_peak, reps=7):
+    """The decode-shaped layer (K = N = 4096, M in {1, 4, 16}): per-launch time
+    of the quantize kernel and of the integer- and float-scale GEMMs, from
+    graphs of back-to-back launches that rotate over 36 packed weight copies
+    (300 MB, more than twice the L2), so every launch streams its weights from
+    HBM.  Inputs drawn on the device: weights ~ N(0, 0.02), tokens ~ N(0, 1)
+    with 0.5% of the channels x30, alpha = 1024, fp16 output."""
+    import torch
+
+    import bit_gemm_quantize_b200 as bgq
+
+    K, N = DECODE["K"], DECODE["N"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(6000 + rank)
+    w = torch.randn((K, N), generator=g, device=dev)
+    w.mul_(0.02)
+    pk = bgq.pack_w4_groupwise(w, group=GROUP, alpha=ALPHA)
+    del w
+    R = 36
+    copies = [pk["packed"]] + [pk["packed"].clone() for _ in range(R - 1)]
+    stream = torch.cuda.current_stream(dev)
+
+    def per_launch_ms(call):
+        for i in range(3):
+            call(i)
+        torch.cuda.synchronize(dev)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            for i in range(R):
+                call(i)
+        gr.replay()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            gr.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1) / R)
+        del gr
+        return max_over_ranks([float(np.median(ts))], world, dev)[0]
+
+    row = {}
+    for M in DECODE["M"]:
+        x = torch.randn((M, K), generator=g, device=dev)
+        cols = torch.randperm(K, generator=g, device=dev)[: max(1, K // 200)]
+        x[:, cols] *= 30.0
+        x = x.to(torch.bfloat16)
+        q, s = bgq.quantize_act_per_token(x)
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        ws = bgq.gemm_workspace(M, N, K, GROUP, 0, dev)
+        wsf = bgq.gemm_workspace(M, N, K, GROUP, 1, dev)
+        t_q = per_launch_ms(lambda i: bgq.quantize_act_per_token(x, q, s))
+        t_is = per_launch_ms(lambda i: bgq.w4a8_gemm_intscale(q, s, copies[i], pk["S"], ALPHA, group=GROUP, out="f16",
+                                                              y=y, workspace=ws))
+        t_fs = per_launch_ms(lambda i: bgq.w4a8_gemm_floatscale(q, s, copies[i], pk["s_g"], group=GROUP, out="f16",
+                                                                y=y, workspace=wsf))
+        b = N * K // 2 + 2 * (K // GROUP) * N + M * K + 4 * M + 2 * M * N
+        row[f"is_us_M{M}"] = round(t_is * 1e3, 2)
+        row[f"fs_us_M{M}"] = round(t_fs * 1e3, 2)
+        row[f"quant_us_M{M}"] = round(t_q * 1e3, 2)
+        row[f"frac_hbm_M{M}"] = round(b / (t_is * 1e-3) / 1e9 / hbm_peak, 4)
+    row["workload"] = "decode_k4096_n4096"
+    row["timing"] = "CUDA events over graphs of 36 launches rotating 36 weight copies (300 MB > L2); median of 7"
+    return row
 
 
 # ---------------------------------------------------------------- mixture of experts
@@ -340,7 +468,7 @@ def measure_moe(dev, rank, world, int8_peak, reps=10):
     tops = ops / (ms * 1e-3) / 1e12
     counts = [int(c) for c in np.diff(off)]
     return {"workload": "moe_mixtral_shaped", "tokens": T, "K": K, "N": N, "experts": E, "topk": topk,
-            "group": GROUP, "alpha": pk["alpha"], "rows_per_expert": counts,
+            "group": GROUP, "alpha": pk["alpha"], "rows_per_expert": ",".join(str(c) for c in counts),
             "us_per_layer": round(ms * 1e3, 2), "tops": round(tops, 2), "frac_int8": round(tops / int8_peak, 4),
             "launches_per_layer": 2 + sum(1 for c in counts if c > 0),
             "timing": "CUDA events over graph replays of quantize + gather + per-expert GEMMs; weights > L2"}
@@ -409,12 +537,13 @@ def measure_prefill(dev, rank, world, int8_peak, reps=10):
             tot[i] += ev[i][0].elapsed_time(ev[i][1])
     ms = max_over_ranks([t / reps for t in tot], world, dev)
     del graphs
-    out = []
+    out = {}
     for (K, N, *_), t in zip(layers, ms):
         tops = 2.0 * M * N * K / (t * 1e-3) / 1e12
-        out.append({"M": M, "K": K, "N": N, "us_quantize_plus_gemm": round(t * 1e3, 2), "tops": round(tops, 2),
-                    "frac_int8": round(tops / int8_peak, 4)})
-    return {"workload": "prefill_4096", "group": GROUP, "alpha": 1024, "layers": out,
+        out[f"us_k{K}_n{N}"] = round(t * 1e3, 2)
+        out[f"tops_k{K}_n{N}"] = round(tops, 2)
+        out[f"frac_int8_k{K}_n{N}"] = round(tops / int8_peak, 4)
+    return {"workload": "prefill_4096", "M": M, "group": GROUP, "alpha": 1024, **out,
             "timing": "CUDA events around graph replays of quantize + integer-scale GEMM, the two layers alternating"}
 
 
@@ -439,7 +568,7 @@ def measure_w8a8(dev, rank, world, hbm_peak, int8_peak, reps=7):
     del w
     copies = [pk["w8"], pk["w8"].clone()]
     stream = torch.cuda.current_stream(dev)
-    rows = []
+    rows = {}
     for M in W8A8["M"]:
         x = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
         q, s = bgq.quantize_act_per_token(x)
@@ -472,9 +601,10 @@ def measure_w8a8(dev, rank, world, hbm_peak, int8_peak, reps=7):
         t = ms * 1e-3
         gbs, tops = bytes_ / t / 1e9, ops / t / 1e12
         bound = "hbm" if bytes_ / (hbm_peak * 1e9) >= ops / (int8_peak * 1e12) else "tensor"
-        rows.append({"M": M, "us": round(ms * 1e3, 2), "tops": round(tops, 2), "gbs": round(gbs, 1), "bound": bound,
-                     "frac": round(gbs / hbm_peak if bound == "hbm" else tops / int8_peak, 4)})
-    return {"workload": "w8a8_ffn_up", "K": K, "N": N, "group": GROUP, "alpha": pk["alpha"], "rows": rows,
+        rows[f"us_M{M}"] = round(ms * 1e3, 2)
+        rows[f"frac_M{M}"] = round(gbs / hbm_peak if bound == "hbm" else tops / int8_peak, 4)
+        rows[f"bound_M{M}"] = bound
+    return {"workload": "w8a8_ffn_up", "K": K, "N": N, "group": GROUP, "alpha": pk["alpha"], **rows,
             "timing": "CUDA events over graphs of six launches alternating two 90 MB weight copies"}
 
 
@@ -502,6 +632,7 @@ def measure_asym(dev, rank, world, reps=7):
     zc = bgq.w4_zero_point_term(pk["packed"], pk["S"], group=GROUP, colsum_max=pk["colsum_max"])
     copies = [pk["packed"]] + [pk["packed"].clone() for _ in range(3)]
     stream = torch.cuda.current_stream(dev)
+    rows = {}
 
     def per_launch_ms(call):
         for i in range(3):
@@ -522,7 +653,6 @@ def measure_asym(dev, rank, world, reps=7):
         del gr
         return max_over_ranks([e0.elapsed_time(e1) / (6 * reps)], world, dev)[0]
 
-    rows = []
     for M in ASYM["M"]:
         x = torch.randn((M, K), generator=g, device=dev).add_(1.0).to(torch.bfloat16)
         qa, sa, za = bgq.quantize_act_per_token_asym(x)
@@ -535,9 +665,11 @@ def measure_asym(dev, rank, world, reps=7):
             qa, sa, za, copies[i % 4], pk["S"], zc, ALPHA, group=GROUP, out="f16", y=y, workspace=wsp))
         t_gs = per_launch_ms(lambda i: bgq.w4a8_gemm_intscale(
             qs, ss, copies[i % 4], pk["S"], ALPHA, group=GROUP, out="f16", y=y, workspace=wsp))
-        rows.append({"M": M, "quant_asym_us": round(t_qa * 1e3, 2), "quant_sym_us": round(t_qs * 1e3, 2),
-                     "gemm_asym_us": round(t_ga * 1e3, 2), "gemm_sym_us": round(t_gs * 1e3, 2)})
-    return {"workload": "asym_act_ffn_up", "K": K, "N": N, "group": GROUP, "alpha": ALPHA, "rows": rows,
+        rows[f"quant_asym_us_M{M}"] = round(t_qa * 1e3, 2)
+        rows[f"quant_sym_us_M{M}"] = round(t_qs * 1e3, 2)
+        rows[f"gemm_asym_us_M{M}"] = round(t_ga * 1e3, 2)
+        rows[f"gemm_sym_us_M{M}"] = round(t_gs * 1e3, 2)
+    return {"workload": "asym_act_ffn_up", "K": K, "N": N, "group": GROUP, "alpha": ALPHA, **rows,
             "timing": "CUDA events over graphs of six launches rotating four 45 MB weight copies"}
 
 
@@ -589,7 +721,9 @@ def run_ours(args):
             dist.barrier()
 
     hbm_peak, bf16_peak, peak_src = load_peaks()
-    int8_peak = bf16_peak * INT8_PER_BF16
+    int8_derived = bf16_peak * INT8_PER_BF16
+    probe = measure_int8_peak(dev, world)
+    int8_peak = probe["ss_n256"]  # the measured int8 tensor rate: the large-M roofline's denominator
 
     # ---- inputs (per rank: an independent layer; weak scaling)
     wl = workloads.make_linear(1, K_DIM, N_DIM, x_dtype="bf16", seed=1000 + rank)
@@ -762,6 +896,7 @@ def run_ours(args):
     value = whole_job_tops(world, ops_step, args.steps, total_ms)
     e2e_value = whole_job_tops(world, ops_step, args.steps, e2e_ms)
 
+    per_m = {}
     sweep = []
     for i, M in enumerate(SWEEP):
         g = float(np.mean(g_ms[:, i])) * 1e3  # us
@@ -781,6 +916,13 @@ def run_ours(args):
             "frac_hbm": round(ach_gbs / hbm_peak, 4), "frac_int8": round(ach_tops / int8_peak, 4),
             "is_faster_than_fs": g < f,
         })
+        per_m[f"is_us_M{M}"] = round(g, 2)
+        per_m[f"fs_us_M{M}"] = round(f, 2)
+        per_m[f"quant_us_M{M}"] = round(q, 2)
+        per_m[f"frac_M{M}"] = round(ach_gbs / hbm_peak if bound == "hbm" else ach_tops / int8_peak, 4)
+        per_m[f"bound_M{M}"] = bound
+    per_m["is_faster_than_fs_every_M"] = all(r["is_faster_than_fs"] for r in sweep)
+    per_m["frac_is"] = "fraction of the HBM copy bandwidth (bound hbm) or of the measured int8 tensor rate (tensor)"
     shares = g_ms.mean(axis=0)
     dom = int(np.argmax(shares))
     Md = SWEEP[dom]
@@ -792,9 +934,11 @@ def run_ours(args):
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = measured_traffic(Md)
     roof["kernel"] = f"w4a8_gemm_kernel (integer scale), M={Md} launch"
-    roof["peak_source"] = (f"{peak_src}: HBM copy {hbm_peak} GB/s; int8 = bf16 {bf16_peak} TFLOP/s x "
-                           f"{INT8_PER_BF16} (nominal int8:bf16 ratio)")
+    roof["peak_source"] = (f"int8: measured tcgen05 kind::i8 probe ({int8_peak:.1f} TOPS, 128x256x32 MMAs, "
+                           f"operands in shared memory); HBM: {peak_src} copy {hbm_peak} GB/s")
+    roof["frac_of_derived_int8"] = (roof["achieved"] / int8_derived) if roof["bound"] == "tensor" else None
 
+    decode = measure_decode(dev, rank, world, hbm_peak)
     moe = measure_moe(dev, rank, world, int8_peak)
     prefill = measure_prefill(dev, rank, world, int8_peak)
     w8a8 = measure_w8a8(dev, rank, world, hbm_peak, int8_peak)
@@ -804,9 +948,12 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "i8xi4->i32", "data": "synthetic",
-        "config": config_dict(), "roofline": roof, "sweep": sweep, "clocks": clocks,
+        "config": config_dict(), "per_M": per_m, "roofline": roof, "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * len(SWEEP) * args.steps,
+        "int8_peak": {"measured_tops": round(int8_peak, 1), "tmem_a_n128_tops": round(probe["ts_n128"], 1),
+                      "derived_bf16x2_tops": round(int8_derived, 1)},
+        "decode": decode,
         "moe": moe,
         "prefill": prefill,
         "w8a8": w8a8,

@@ -15,6 +15,7 @@ from ._native import (  # noqa: F401
     pack_w8_groupwise,
     quantize_act_per_token,
     quantize_act_per_token_asym,
+    tensor_i8_peak_probe,
     w4_zero_point_term,
     w4a8_amplifier_search,
     w4a8_gemm_floatscale,
@@ -36,6 +37,7 @@ __all__ = [
     "pack_w8_groupwise",
     "quantize_act_per_token",
     "quantize_act_per_token_asym",
+    "tensor_i8_peak_probe",
     "w4_zero_point_term",
     "w4a8_amplifier_search",
     "w4a8_gemm_floatscale",

@@ -86,6 +86,7 @@ def load(path: str = LIB_PATH):
             "w4a8_moe_workspace_size": ([I32_, P, I64, I64, I32_], I64),
             "w4a8_moe_gemm_intscale": ([P, P, I64, P, P, P, P, I32_, I32_, I64, I64, I32_, P, I32_, P, I64, P],
                                        I32_),
+            "w4a8_tensor_i8_peak_probe": ([I64, I32_, I32_, P, P, P], I32_),
             "w4a8_last_cuda_error": ([I32_], I32_),
             "w4a8_cuda_error_string": ([I32_], ctypes.c_char_p),
         }
@@ -483,6 +484,20 @@ def w4a8_moe_gemm_intscale(q_x, s_a, row_index, offsets, packed, S, alpha: int, 
                                          _ptr(workspace), workspace.numel(), _stream(q_x.device))
     _check("w4a8_moe_gemm_intscale", code)
     return y
+
+
+def tensor_i8_peak_probe(iters: int, n: int = 256, a_in_tmem: bool = False, device=None) -> float:
+    """Launch the int8 tensor-pipe probe on the current stream of `device`
+    (back-to-back 128 x n x 32 MMAs on on-chip operands, one CTA per SM) and
+    return the int8 operations it performs; time it with CUDA events."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    grid = ctypes.c_int32(0)
+    ops = ctypes.c_double(0.0)
+    with torch.cuda.device(device):
+        code = load().w4a8_tensor_i8_peak_probe(int(iters), int(n), 1 if a_in_tmem else 0, ctypes.byref(grid),
+                                                ctypes.byref(ops), _stream(device))
+    _check("w4a8_tensor_i8_peak_probe", code)
+    return float(ops.value)
 
 
 def device_status(clear: bool = True) -> int:

@@ -559,6 +559,19 @@ w4a8_status w4a8_gemm_floatscale(const int8_t* q_x, const float* s_a, const uint
                     workspace, workspace_bytes, stream);
 }
 
+w4a8_status w4a8_tensor_i8_peak_probe(int64_t iters, int32_t n, int32_t a_in_tmem, int32_t* grid_host,
+                                      double* ops_host, void* stream) {
+    if (iters < 1 || iters > (int64_t(1) << 30) || n < 16 || n > 256 || n % 16 != 0) return W4A8_ERR_SHAPE;
+    if (!grid_host || !ops_host) return W4A8_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    w4a8_status st = current_device(dev);
+    if (st != W4A8_OK) return st;
+    W4A8_CUDA_TRY(w4a8::peak::launch(iters, n, a_in_tmem != 0, dev.sms, dev.status, static_cast<cudaStream_t>(stream)));
+    *grid_host = dev.sms;
+    *ops_host = 2.0 * 128.0 * double(n) * 128.0 * double(iters) * double(dev.sms);
+    return W4A8_OK;
+}
+
 int32_t w4a8_last_cuda_error(int32_t clear) {
     const int32_t e = int32_t(t_last_cuda_error);
     if (clear) t_last_cuda_error = cudaSuccess;

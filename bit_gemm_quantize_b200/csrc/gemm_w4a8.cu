@@ -357,11 +357,15 @@ struct Ring {
     }
 };
 
-template <int BT, int PATH, bool W8, bool ZP>
+// G1: the group is one 128-wide K block (group = 128, the method's group
+// size), so every K block ends a group; wide token tiles then drain each group
+// in a loop with no per-stage bookkeeping.
+template <int BT, int PATH, bool W8, bool ZP, bool G1>
 __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH, W8, ZP>::kCtasPerSm)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_y, const std::conditional_t<ZP, ParamsZp, Params> p) {
     using C = Cfg<BT, PATH, W8, ZP>;
+    constexpr bool kLean = G1 && C::kGroupCommit;  // the per-group drain loop below
     constexpr int kAcc = C::kAcc;
     constexpr int kU = C::kUnpackWarps;
     constexpr int SW = C::kSW, SX = C::kSX, SA = C::kSA, SD = C::kSD;
@@ -541,9 +545,9 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 if (j >= st.nkb) break;
-                const bool first = (kin == 0);
-                const bool last = (kin == p.kb_per_group - 1);
-                kin = last ? 0 : kin + 1;
+                const bool first = G1 || (kin == 0);
+                const bool last = G1 || (kin == p.kb_per_group - 1);
+                if constexpr (!G1) kin = last ? 0 : kin + 1;
                 if (first) {
                     if (!mbar_wait_warp(&tempty[rt.idx], rt.phase ^ 1u, abort_flag, p.status)) {
                         ok = false;
@@ -726,6 +730,62 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                     }
                 }
             }
+            if constexpr (kLean) {
+                // One group per K block, each committed to its own accumulator
+                // buffer: wait for the group's MMAs, load this thread's HC
+                // columns of P_g in one TMEM load, hand the buffer back, then
+                // acc += S[g,n] * P_g (or accf += s_g * float(P_g)).  This
+                // column's scale is read from global memory two groups ahead
+                // (a column past N reads column 0's scales: its outputs are
+                // never stored).
+                const uint32_t lane_cols =
+                    tmem_base + (uint32_t(quarter * 32) << 16) + C::kAccCol0 + uint32_t(half * HC);
+                const int32_t n_ld = nvalid ? int32_t(n) : 0;
+                const int32_t nstride = int32_t(p.N);
+                int32_t sidx = sg.g0 * nstride + n_ld;  // element index of the next scale to load (< 2^31)
+                auto ld_scale = [&](int32_t i) -> uint32_t {
+                    if constexpr (PATH == kIntScale)
+                        return uint32_t(int32_t(__ldg(p.S + i)));
+                    else
+                        return __float_as_uint(__ldg(p.s_g + i));
+                };
+                uint32_t s1 = ld_scale(sidx);
+                sidx += nstride;
+                uint32_t s2 = (sg.g0 + 1 < sg.g1) ? ld_scale(sidx) : 0u;
+                sidx += nstride;
+                for (int32_t g = sg.g0; g < sg.g1; ++g) {
+                    const uint32_t sraw = s1;
+                    s1 = s2;
+                    if (g + 2 < sg.g1) s2 = ld_scale(sidx);
+                    sidx += nstride;
+                    if (!mbar_wait_warp(&afull[rt.idx], rt.phase, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint32_t v[HC];
+                    tmem_load<HC>(lane_cols + uint32_t(rt.idx * BT), v);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    __syncwarp();
+                    mbar_arrive_one(&tempty[rt.idx]);
+                    rt.advance(kAcc);
+                    if constexpr (PATH == kIntScale) {
+                        const int32_t s_cur = int32_t(sraw);
+#pragma unroll
+                        for (int q = 0; q < HC; ++q) {
+                            const int32_t pg = C::kX16 ? (int32_t(v[q]) >> 4) : int32_t(v[q]);  // exact
+                            acc[q] += s_cur * pg;
+                        }
+                    } else {
+                        const float f_cur = C::kX16 ? __fmul_rn(__uint_as_float(sraw), 0.0625f)  // P_g was 16 P_g
+                                                    : __uint_as_float(sraw);
+#pragma unroll
+                        for (int q = 0; q < HC; ++q)
+                            accf[q] = __fmaf_rn(f_cur, __int2float_rn(int32_t(v[q])), accf[q]);
+                    }
+                }
+            } else {
             // This column's scales (raw 32 bits) of group g, read straight from
             // global memory two stages before they are used, so that no wait
             // or shared-memory round trip sits between two drains.  Rows past
@@ -882,6 +942,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                     if (!ok) break;
                 }
             }
+            }  // kLean
             if (!ok) break;
 
             // valid token columns of this thread's share (split-tile partials)
@@ -1045,16 +1106,22 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool
     return pl;
 }
 
+template <auto kern, typename P>
+static cudaError_t launch_k(int threads, int smem, const CUtensorMap& tw, const CUtensorMap& tx,
+                            const CUtensorMap& ty, const P& p, cudaStream_t stream) {
+    const cudaError_t e = configure_once<kern>(threads, smem);
+    if (e != cudaSuccess) return e;
+    const LaunchPdl lc(unsigned(p.grid), threads, size_t(smem), stream);
+    return cudaLaunchKernelEx(&lc.cfg, kern, tw, tx, ty, p);
+}
+
 template <int BT, int PATH, bool W8 = false, bool ZP = false>
 static cudaError_t launch_bt(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty,
                              const std::conditional_t<ZP, ParamsZp, Params>& p, cudaStream_t stream) {
     using C = Cfg<BT, PATH, W8, ZP>;
-    auto kern = w4a8_gemm_kernel<BT, PATH, W8, ZP>;
-    const int smem = C::kSmemBytes;
-    const cudaError_t e = configure_once(kern, C::kThreads, smem);
-    if (e != cudaSuccess) return e;
-    const LaunchPdl lc(unsigned(p.grid), C::kThreads, size_t(smem), stream);
-    return cudaLaunchKernelEx(&lc.cfg, kern, tw, tx, ty, p);
+    if (p.kb_per_group == 1)
+        return launch_k<w4a8_gemm_kernel<BT, PATH, W8, ZP, true>>(C::kThreads, C::kSmemBytes, tw, tx, ty, p, stream);
+    return launch_k<w4a8_gemm_kernel<BT, PATH, W8, ZP, false>>(C::kThreads, C::kSmemBytes, tw, tx, ty, p, stream);
 }
 
 cudaError_t launch(const CUtensorMap& tw, const CUtensorMap& tx, const CUtensorMap& ty, const Params& p, int BT, int path,

@@ -11,9 +11,10 @@ namespace w4a8 {
 // The dynamic shared-memory opt-in of a kernel is a per-device function
 // attribute: set it (and check that one CTA fits) once per (kernel, device),
 // the first time the kernel is launched on the device.  Thread-safe; later
-// launches only read the recorded result.
-template <typename Kernel>
-cudaError_t configure_once(Kernel kern, int threads, int smem) {
+// launches only read the recorded result.  The kernel is a template argument,
+// so every kernel has flags of its own.
+template <auto kern>
+cudaError_t configure_once(int threads, int smem) {
     constexpr int kDevs = 64;
     static std::once_flag once[kDevs];
     static cudaError_t result[kDevs];
@@ -77,6 +78,12 @@ struct GatherParams {
 };
 cudaError_t gather(const GatherParams& p, int max_rows, cudaStream_t stream);
 }  // namespace moe
+
+namespace peak {
+// Back-to-back int8 MMAs (128 x n x 32, n % 16 == 0, 16 <= n <= 256) on
+// on-chip operands, iters x 4 per CTA, one CTA per SM of `grid`.
+cudaError_t launch(int64_t iters, int n, bool a_in_tmem, int grid, int* status, cudaStream_t stream);
+}  // namespace peak
 
 namespace pack {
 // Layout of the pack workspace (device bytes).

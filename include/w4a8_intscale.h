@@ -375,6 +375,23 @@ W4A8_API w4a8_status w4a8_gemm_floatscale(const int8_t* q_x, const float* s_a, c
                                  void* stream);
 
 /*
+ * Measurement aid, not a step of the method: the int8 tensor-core rate of this
+ * GPU.  Launches one CTA per SM; each issues iters x 4 back-to-back
+ * tcgen05.mma.kind::i8 of shape 128 x n x 32 (signed int8, int32 accumulator
+ * in TMEM) on operands already on chip: the weight-side operand from shared
+ * memory (a_in_tmem = 0) or from TMEM (a_in_tmem != 0, as the W4A8 GEMM feeds
+ * its unpacked weights), the token-side operand from shared memory.  No loads
+ * from global memory and no epilogue.  Asynchronous on `stream`: time it with
+ * events around the call.
+ * iters      1 .. 2^30; n: 16 .. 256, a multiple of 16; otherwise W4A8_ERR_SHAPE
+ * grid_host  host, written: the CTAs launched (the SM count)
+ * ops_host   host, written: int8 operations of the launch, 2*128*n*128*iters*grid
+ * A wait that runs out sets W4A8_ERR_TIMEOUT in the device status word.
+ */
+W4A8_API w4a8_status w4a8_tensor_i8_peak_probe(int64_t iters, int32_t n, int32_t a_in_tmem, int32_t* grid_host,
+                                              double* ops_host, void* stream);
+
+/*
  * The CUDA runtime error code (cudaError_t) behind the last W4A8_ERR_CUDA that
  * a call of this library returned on the calling thread (0 if none); with
  * clear != 0 the record is reset.  w4a8_cuda_error_string names a code.
