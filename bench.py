@@ -437,15 +437,18 @@ def measure_moe(dev, rank, world, int8_peak, reps=10):
     ri, off = workloads.route_rows(route, E)
     R = int(off[-1])
     ri_d = torch.from_numpy(ri).to(dev)
+    off_d = torch.from_numpy(off).to(dev)
+    wp = bgq.device_pointers(pk["packed"], dev)
+    sp = bgq.device_pointers(pk["S"], dev)
     q = torch.empty((T, K), dtype=torch.int8, device=dev)
     s = torch.empty((T,), dtype=torch.float32, device=dev)
     y = torch.empty((R, N), dtype=torch.float16, device=dev)
-    wsp = bgq.moe_workspace(off, N, K, GROUP, dev)
+    wsp = bgq.grouped_workspace(E, N, K, GROUP, dev)
 
     def layer():
         bgq.quantize_act_per_token(x, q, s)
-        bgq.w4a8_moe_gemm_intscale(q, s, ri_d, off, pk["packed"], pk["S"], pk["alpha"], group=GROUP, out="f16",
-                                   y=y, workspace=wsp)
+        bgq.w4a8_gemm_intscale_grouped(q, s, ri_d, off_d, wp, sp, pk["alpha"], group=GROUP, out="f16", y=y,
+                                       workspace=wsp, N=N)
 
     for _ in range(3):
         layer()
@@ -470,8 +473,9 @@ def measure_moe(dev, rank, world, int8_peak, reps=10):
     return {"workload": "moe_mixtral_shaped", "tokens": T, "K": K, "N": N, "experts": E, "topk": topk,
             "group": GROUP, "alpha": pk["alpha"], "rows_per_expert": ",".join(str(c) for c in counts),
             "us_per_layer": round(ms * 1e3, 2), "tops": round(tops, 2), "frac_int8": round(tops / int8_peak, 4),
-            "launches_per_layer": 2 + sum(1 for c in counts if c > 0),
-            "timing": "CUDA events over graph replays of quantize + gather + per-expert GEMMs; weights > L2"}
+            "launches_per_layer": 3,
+            "timing": "CUDA events over graph replays of quantize + grouped setup + one grouped GEMM over all "
+                      "experts (device routing offsets); weights > L2"}
 
 
 PREFILL = dict(M=4096, shapes=[(4096, 11008), (11008, 4096)])  # (K, N) of the two layers

@@ -9,7 +9,8 @@ from ._native import (  # noqa: F401
     device_status,
     gemm_workspace,
     load,
-    moe_workspace,
+    grouped_workspace,
+    device_pointers,
     pack_moe_experts,
     pack_w4_groupwise,
     pack_w8_groupwise,
@@ -22,7 +23,8 @@ from ._native import (  # noqa: F401
     w4a8_gemm_intscale,
     w4a8_gemm_intscale_asym,
     w4a8_gemm_intscale_static_ws,
-    w4a8_moe_gemm_intscale,
+    w4a8_gemm_intscale_grouped,
+    w4a8_linear_intscale,
     w8a8_gemm_intscale,
 )
 
@@ -31,7 +33,8 @@ __all__ = [
     "device_status",
     "gemm_workspace",
     "load",
-    "moe_workspace",
+    "grouped_workspace",
+    "device_pointers",
     "pack_moe_experts",
     "pack_w4_groupwise",
     "pack_w8_groupwise",
@@ -44,6 +47,7 @@ __all__ = [
     "w4a8_gemm_intscale",
     "w4a8_gemm_intscale_asym",
     "w4a8_gemm_intscale_static_ws",
-    "w4a8_moe_gemm_intscale",
+    "w4a8_gemm_intscale_grouped",
+    "w4a8_linear_intscale",
     "w8a8_gemm_intscale",
 ]

@@ -83,10 +83,12 @@ def load(path: str = LIB_PATH):
             "w4a8_gemm_intscale_static_ws": ([P, P, P, P, I32_, I64, I64, I64, I32_, P, I32_, P], I32_),
             "w4a8_gemm_floatscale": ([P, P, P, P, I64, I64, I64, I32_, P, I32_, P, I64, P], I32_),
             "w4a8_device_status": ([P, I32_], I32_),
-            "w4a8_moe_workspace_size": ([I32_, P, I64, I64, I32_], I64),
-            "w4a8_moe_gemm_intscale": ([P, P, I64, P, P, P, P, I32_, I32_, I64, I64, I32_, P, I32_, P, I64, P],
-                                       I32_),
+            "w4a8_linear_intscale": ([P, I32_, I64, I64, I64, P, P, I32_, I64, I32_, P, I32_, P, P, P, I64, P], I32_),
+            "w4a8_grouped_workspace_size": ([I32_, I64, I64, I32_], I64),
+            "w4a8_gemm_intscale_grouped": ([P, P, I64, P, P, P, P, P, I32_, I32_, I64, I64, I64, I32_, P, I32_, I64,
+                                            P, I64, P], I32_),
             "w4a8_tensor_i8_peak_probe": ([I64, I32_, I32_, P, P, P], I32_),
+            "w4a8_set_wait_limit": ([I64], I64),
             "w4a8_last_cuda_error": ([I32_], I32_),
             "w4a8_cuda_error_string": ([I32_], ctypes.c_char_p),
         }
@@ -338,6 +340,44 @@ def w4a8_gemm_intscale(q_x, s_a, w_packed, S, alpha: int, *, group: int = 128, o
     return y
 
 
+def w4a8_linear_intscale(x, w_packed, S, alpha: int, *, group: int = 128, out: str = "f16",
+                         y: torch.Tensor | None = None, q_x: torch.Tensor | None = None, s_a: torch.Tensor | None = None,
+                         workspace: torch.Tensor | None = None):
+    """y [M, N] = the integer-scale layer from unquantized tokens x [M, K]
+    (fp32 or bf16): per-token quantization and the W4A8 integer-scale GEMM,
+    one kernel when M <= 4.  q_x / s_a receive the token codes and scales when
+    given (allocated here when M > 4, where they are needed)."""
+    _need_cuda("x", x, ndim=2)
+    if x.dtype == torch.float32:
+        dt_x = F32
+    elif x.dtype == torch.bfloat16:
+        dt_x = BF16
+    else:
+        raise ValueError("x must be float32 or bfloat16")
+    _need_cuda("w_packed", w_packed, torch.uint8, 2)
+    _need_cuda("S", S, torch.int16, 2)
+    M, K = x.shape
+    N = w_packed.shape[0]
+    if w_packed.shape[1] * 2 != K:
+        raise ValueError("w_packed must be [N, K/2]")
+    dt, tdt = _OUT[out]
+    if y is None:
+        y = torch.empty((M, N), dtype=tdt, device=x.device)
+    _need_cuda("y", y, tdt, 2)
+    if M > 4 and q_x is None:
+        q_x = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if M > 4 and s_a is None:
+        s_a = torch.empty((M,), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = gemm_workspace(M, N, K, group, 0, x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    code = load().w4a8_linear_intscale(_ptr(x), dt_x, M, K, K, _ptr(w_packed), _ptr(S), int(alpha), N, group,
+                                       _ptr(y), dt, _ptr(q_x), _ptr(s_a), _ptr(workspace), ws_bytes,
+                                       _stream(x.device))
+    _check("w4a8_linear_intscale", code)
+    return y
+
+
 def w4a8_gemm_intscale_asym(q_x, s_a, z_a, w_packed, S, zc, alpha: int, *, group: int = 128, out: str = "f16",
                             y: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
     """y [M, N] = integer-scale W4A8 GEMM of asymmetric token codes: the
@@ -443,46 +483,79 @@ def pack_moe_experts(ws, group: int = 128, alpha: int | None = None):
                 alpha=int(alpha))
 
 
-def moe_workspace(offsets, N: int, K: int, group: int, device) -> torch.Tensor:
-    """A zero-filled workspace for w4a8_moe_gemm_intscale with these row offsets."""
-    off = np.ascontiguousarray(np.asarray(offsets, np.int64))
+_grouped_ws = {}
+
+
+def grouped_workspace(E: int, N: int, K: int, group: int, device) -> torch.Tensor:
+    """A zero-filled workspace for w4a8_gemm_intscale_grouped, reused across
+    calls on the device (calls that may overlap on the GPU need their own)."""
     with torch.cuda.device(device):
-        need = load().w4a8_moe_workspace_size(len(off) - 1, off.ctypes.data_as(ctypes.c_void_p), N, K, group)
+        need = int(load().w4a8_grouped_workspace_size(int(E), int(N), int(K), int(group)))
     if need < 0:
-        raise W4A8Error("w4a8_moe_workspace_size", 1, " (invalid offsets or shape)")
-    return torch.zeros(max(int(need), 16), dtype=torch.uint8, device=device)
+        raise W4A8Error("w4a8_grouped_workspace_size", 1, " (invalid shape or expert count)")
+    key = torch.device(device).index
+    ws = _grouped_ws.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        _grouped_ws[key] = ws
+        _ws_cache[("grouped", key)] = ws  # zeroed with the others after a failure
+    return ws
 
 
-def w4a8_moe_gemm_intscale(q_x, s_a, row_index, offsets, packed, S, alpha: int, *, group: int = 128,
-                           out: str = "f16", y: torch.Tensor | None = None,
-                           workspace: torch.Tensor | None = None, N: int | None = None):
-    """y [R, N]: expert e's integer-scale GEMM over its routed rows
-    row_index[offsets[e]:offsets[e+1]] (offsets: host, E+1 values).  N is taken
-    from the packed weights unless given (needed when every expert is empty)."""
+def device_pointers(tensors, device) -> torch.Tensor:
+    """A device int64 array of the tensors' data pointers (0 for None): the
+    pointer arrays the grouped call reads on the device."""
+    ptrs = [0 if t is None else int(t.data_ptr()) for t in tensors]
+    return torch.tensor(ptrs, dtype=torch.int64).to(device)
+
+
+def w4a8_gemm_intscale_grouped(q_x, s_a, row_index, expert_offsets, packed, S, alpha: int, *, group: int = 128,
+                               out: str = "f16", y: torch.Tensor | None = None, out_row: torch.Tensor | None = None,
+                               y_rows: int | None = None, workspace: torch.Tensor | None = None,
+                               N: int | None = None):
+    """Every expert's integer-scale GEMM over its routed rows in one grouped call.
+
+    row_index [R] int32: the token of each routed row, rows grouped by expert;
+    expert_offsets [E+1] int64 CUDA tensor (device offsets); packed / S: lists
+    of per-expert tensors (None for experts without rows) or int64 CUDA
+    tensors of device pointers; out_row [R] int32 or None: the output row of
+    each routed row (None: row i).  N is taken from the packed weights unless
+    given (needed when pointers are passed)."""
     _need_cuda("q_x", q_x, torch.int8, 2)
     _need_cuda("s_a", s_a, torch.float32, 1)
     _need_cuda("row_index", row_index, torch.int32, 1)
-    off = np.ascontiguousarray(np.asarray(offsets, np.int64))
-    E = len(off) - 1
-    if len(packed) != E or len(S) != E:
-        raise ValueError("one packed weight and one integer-scale tensor per expert")
+    _need_cuda("expert_offsets", expert_offsets, torch.int64, 1)
+    dev = q_x.device
+    E = expert_offsets.numel() - 1
     T, K = q_x.shape
+    R = row_index.numel()
+    if isinstance(packed, torch.Tensor):
+        wp = packed
+    else:
+        if len(packed) != E or len(S) != E:
+            raise ValueError("one packed weight and one integer-scale tensor per expert")
+        if N is None:
+            N = int(next((t.shape[0] for t in packed if t is not None), 0))
+        wp = device_pointers(packed, dev)
+    sp = S if isinstance(S, torch.Tensor) else device_pointers(S, dev)
+    _need_cuda("packed pointers", wp, torch.int64, 1)
+    _need_cuda("S pointers", sp, torch.int64, 1)
     if N is None:
-        N = int(next((p.shape[0] for p in packed if p is not None), 0))
-    R = int(off[-1])
+        raise ValueError("N must be given with pointer arrays")
+    if out_row is not None:
+        _need_cuda("out_row", out_row, torch.int32, 1)
     dt, tdt = _OUT[out]
     if y is None:
-        y = torch.empty((R, N), dtype=tdt, device=q_x.device)
+        rows = R if out_row is None else (int(y_rows) if y_rows is not None else R)
+        y = torch.empty((rows, N), dtype=tdt, device=dev)
     _need_cuda("y", y, tdt, 2)
     if workspace is None:
-        workspace = moe_workspace(off, N, K, group, q_x.device)
-    wp = (ctypes.c_void_p * E)(*[p.data_ptr() if p is not None else 0 for p in packed])
-    sp = (ctypes.c_void_p * E)(*[s.data_ptr() if s is not None else 0 for s in S])
-    code = load().w4a8_moe_gemm_intscale(_ptr(q_x), _ptr(s_a), T, _ptr(row_index),
-                                         off.ctypes.data_as(ctypes.c_void_p), ctypes.cast(wp, ctypes.c_void_p),
-                                         ctypes.cast(sp, ctypes.c_void_p), int(alpha), E, N, K, group, _ptr(y), dt,
-                                         _ptr(workspace), workspace.numel(), _stream(q_x.device))
-    _check("w4a8_moe_gemm_intscale", code)
+        workspace = grouped_workspace(E, N, K, group, dev)
+    code = load().w4a8_gemm_intscale_grouped(_ptr(q_x), _ptr(s_a), T, _ptr(row_index), _ptr(expert_offsets),
+                                             _ptr(out_row), _ptr(wp), _ptr(sp), int(alpha), E, R, N, K, group,
+                                             _ptr(y), dt, y.shape[0], _ptr(workspace), workspace.numel(),
+                                             _stream(dev))
+    _check("w4a8_gemm_intscale_grouped", code)
     return y
 
 

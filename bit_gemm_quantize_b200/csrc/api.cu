@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "w4a8_intscale.h"
@@ -47,6 +48,11 @@ std::mutex g_static_ws_mutex;
 // Device address of the current device's static workspace, looked up once per
 // device (the first call on a device does this set-up).
 w4a8_status static_workspace(void** out);
+
+// How long (SM cycles) a GEMM's pipeline and split-tile waits may last before
+// the kernel gives up with W4A8_ERR_TIMEOUT; w4a8_set_wait_limit changes it.
+constexpr long long kDefaultWaitLimit = 1ll << 31;
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
 // Last CUDA runtime error seen by this thread's library calls.
 thread_local cudaError_t t_last_cuda_error = cudaSuccess;
@@ -142,7 +148,13 @@ w4a8_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int32_t group) {
     if (M < 0 || N <= 0 || K <= 0 || group <= 0) return W4A8_ERR_SHAPE;
     if (N % 8 != 0 || K % 128 != 0 || group % 128 != 0 || K % group != 0) return W4A8_ERR_SHAPE;
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return W4A8_ERR_SHAPE;
+    if ((K / group) * N >= (int64_t(1) << 31)) return W4A8_ERR_SHAPE;  // scale indices are 32-bit
     return W4A8_OK;
+}
+
+// Decode-shaped calls (a few tokens) run on the CUDA cores (gemv_w4a8.cu).
+bool gemv_path(int64_t M, int64_t K, bool w8, bool zp) {
+    return !w8 && !zp && M >= 1 && M <= w4a8::gemv::kMaxM && K <= w4a8::gemv::kMaxK;
 }
 
 w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_t* w_packed, const int16_t* S,
@@ -167,7 +179,27 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
 
     DeviceInfo dev;
     if ((st = current_device(dev)) != W4A8_OK) return st;
-    const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms, w8);
+    if (gemv_path(M, K, w8, zp)) {
+        // decode-shaped: the CUDA-core kernel, no workspace
+        w4a8::gemv::GemvParams g{};
+        g.x = q_x;
+        g.s_a = s_a;
+        g.w = w_packed;
+        g.S = S;
+        g.s_g = s_g;
+        g.y = y;
+        g.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
+                                        : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
+        g.M = int32_t(M);
+        g.N = int32_t(N);
+        g.K = int32_t(K);
+        g.G = int32_t(K / group);
+        g.group = group;
+        g.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
+        W4A8_CUDA_TRY(w4a8::gemv::launch(g, path, w4a8::gemv::kXCodes, dev.sms, static_cast<cudaStream_t>(stream)));
+        return W4A8_OK;
+    }
+    const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms, w8, zp);
     if (pl.W >= (int64_t(1) << 31)) return W4A8_ERR_SHAPE;  // the kernel indexes (tile, group) steps in 32 bits
     int32_t* ws_count = nullptr;
     int32_t* ws_part = nullptr;
@@ -176,6 +208,50 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
         if (!aligned16(workspace)) return W4A8_ERR_ALIGN;
         ws_count = static_cast<int32_t*>(workspace);
         ws_part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + pl.count_bytes);
+    }
+
+    if (pl.wide) {
+        // token tiles of 256 / 192: packed weights one K block (64 B) per box, no
+        // swizzle; token codes BT rows x 128 B, 128-byte swizzle; output boxes of
+        // BT rows (fp16) or 64 rows (4-byte outputs)
+        CUtensorMap tm_w, tm_x, tm_y;
+        if (!make_map_u8(&tm_w, w_packed, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 64, 128,
+                         CU_TENSOR_MAP_SWIZZLE_NONE))
+            return W4A8_ERR_CUDA;
+        if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(M), uint64_t(K), 128, uint32_t(pl.BT),
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4A8_ERR_CUDA;
+        const bool f16 = (y_dtype == W4A8_F16);
+        const CUtensorMapDataType t = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                          : (y_dtype == W4A8_I32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                                                 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+        if (!make_map_2d(&tm_y, t, y, uint64_t(N), uint64_t(M), uint64_t(N) * (f16 ? 2u : 4u), 128,
+                         f16 ? uint32_t(pl.BT) : 64u, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return W4A8_ERR_CUDA;
+        w4a8::gemm::WideParams q{};
+        q.s_a = s_a;
+        q.S = S;
+        q.s_g = s_g;
+        q.y = y;
+        q.ws_part = ws_part;
+        q.ws_count = ws_count;
+        q.status = dev.status;
+        q.M = int32_t(M);
+        q.N = int32_t(N);
+        q.G = int32_t(pl.G);
+        q.kb_per_group = group / 128;
+        q.n_tiles = int32_t(pl.n_tiles);
+        q.m_tiles = int32_t(pl.m_tiles);
+        q.grid = int32_t(pl.grid);
+        q.W = uint32_t(pl.W);
+        q.w_q = uint32_t(pl.W / pl.grid);
+        q.w_r = uint32_t(pl.W % pl.grid);
+        q.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
+        q.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
+                                        : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
+        q.wait_limit = g_wait_limit.load();
+        W4A8_CUDA_TRY(w4a8::gemm::launch_wide(tm_w, tm_x, tm_y, q, path, static_cast<cudaStream_t>(stream)));
+        return W4A8_OK;
     }
 
     CUtensorMap tm_w, tm_x, tm_y;
@@ -218,6 +294,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     p.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
     p.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
                                     : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
+    p.wait_limit = g_wait_limit.load();
     if (zp) {
         w4a8::gemm::ParamsZp pz{};
         static_cast<w4a8::gemm::Params&>(pz) = p;
@@ -230,41 +307,24 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     return W4A8_OK;
 }
 
-// Layout of the mixture-of-experts workspace for host row offsets off[0..E]:
-// [GEMM workspace (counters first)] [gathered codes R x K] [gathered scales,
-// each expert's 16-byte aligned], every part 256-byte aligned.
-struct MoeLayout {
-    int64_t R = 0, max_rows = 0;
-    int64_t gemm_bytes = 0, x_off = 0, s_off = 0, total = 0;
-    int32_t sbase[w4a8::moe::kMaxExperts] = {};
-};
-
 int64_t align256(int64_t v) { return (v + 255) & ~int64_t(255); }
 
-w4a8_status moe_layout(int32_t E, const int64_t* off, int64_t N, int64_t K, int32_t group, const DeviceInfo& dev,
-                       MoeLayout& L) {
-    if (E < 1 || E > w4a8::moe::kMaxExperts || !off) return W4A8_ERR_INVALID_ARG;
-    if (off[0] != 0) return W4A8_ERR_INVALID_ARG;
-    int64_t sfloats = 0;
-    for (int32_t e = 0; e < E; ++e) {
-        const int64_t m = off[e + 1] - off[e];
-        if (m < 0) return W4A8_ERR_INVALID_ARG;
-        L.sbase[e] = int32_t(sfloats);
-        sfloats += (m + 3) & ~int64_t(3);
-        if (m > L.max_rows) L.max_rows = m;
-        if (m > 0) {
-            const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(m, N, K, group, dev.sms);
-            if (pl.W >= (int64_t(1) << 31)) return W4A8_ERR_SHAPE;
-            const int64_t need = plan_splits_tiles(pl) ? pl.ws_bytes : 0;
-            if (need > L.gemm_bytes) L.gemm_bytes = need;
-        }
-    }
-    L.R = off[E];
-    if (L.R > INT32_MAX || sfloats > INT32_MAX) return W4A8_ERR_SHAPE;
-    L.x_off = align256(L.gemm_bytes);
-    L.s_off = L.x_off + align256(L.R * K);
-    L.total = L.s_off + align256(sfloats * 4);
-    return W4A8_OK;
+// Layout of the grouped (mixture-of-experts) workspace: [arrival counters and
+// split-tile partials of the wide kernel] [E weight tensor maps]
+// [schedule: W, W / grid, W % grid, status, m_tiles[E+1], first tile[E+1],
+// first row[E+1]], every part 256-byte aligned.
+struct GroupedLayout {
+    int64_t grid = 0, gemm_bytes = 0, maps_off = 0, sched_off = 0, total = 0;
+};
+
+GroupedLayout grouped_layout(int32_t E, const DeviceInfo& dev) {
+    GroupedLayout L;
+    L.grid = dev.sms;
+    L.gemm_bytes = 4096 + L.grid * 128 * int64_t(w4a8::gemm::wide_token_tile()) * 4;
+    L.maps_off = align256(L.gemm_bytes);
+    L.sched_off = L.maps_off + align256(int64_t(E) * 128);
+    L.total = L.sched_off + align256((4 + 3 * (int64_t(E) + 1)) * 4);
+    return L;
 }
 
 }  // namespace
@@ -448,7 +508,17 @@ int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group,
     DeviceInfo dev;
     if (current_device(dev) != W4A8_OK) return -1;
     const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms, path == 2);
-    return plan_splits_tiles(pl) ? pl.ws_bytes : 0;
+    if (gemv_path(M, K, path == 2, false)) {  // no workspace; the asymmetric GEMM (path 0) runs tiles
+        if (path != 0) return 0;
+        const w4a8::gemm::Plan pn = w4a8::gemm::make_plan(M, N, K, group, dev.sms, false, true);
+        return plan_splits_tiles(pn) ? pn.ws_bytes : 0;
+    }
+    int64_t need = plan_splits_tiles(pl) ? pl.ws_bytes : 0;
+    if (path == 0 && pl.wide) {  // the asymmetric-token GEMM (path 0 too) runs narrow tiles
+        const w4a8::gemm::Plan pn = w4a8::gemm::make_plan(M, N, K, group, dev.sms, false, true);
+        if (plan_splits_tiles(pn) && pn.ws_bytes > need) need = pn.ws_bytes;
+    }
+    return need;
 }
 
 w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, const uint8_t* w_packed, const int16_t* S,
@@ -488,67 +558,127 @@ w4a8_status w4a8_gemm_intscale_static_ws(const int8_t* q_x, const float* s_a, co
                     int64_t(W4A8_STATIC_WORKSPACE_BYTES), stream);
 }
 
-int64_t w4a8_moe_workspace_size(int32_t E, const int64_t* expert_offsets_host, int64_t N, int64_t K,
-                                int32_t group) {
-    if (check_gemm_shape(1, N, K, group) != W4A8_OK) return -1;
-    DeviceInfo dev;
-    if (current_device(dev) != W4A8_OK) return -1;
-    MoeLayout L;
-    if (moe_layout(E, expert_offsets_host, N, K, group, dev, L) != W4A8_OK) return -1;
-    return L.total;
-}
-
-w4a8_status w4a8_moe_gemm_intscale(const int8_t* q_x, const float* s_a, int64_t T, const int32_t* row_index,
-                                   const int64_t* expert_offsets_host, const uint8_t* const* w_packed_host,
-                                   const int16_t* const* S_host, int32_t alpha, int32_t E, int64_t N, int64_t K,
-                                   int32_t group, void* y, int32_t y_dtype, void* workspace,
-                                   int64_t workspace_bytes, void* stream) {
-    w4a8_status st = check_gemm_shape(1, N, K, group);
+w4a8_status w4a8_linear_intscale(const void* x, int32_t x_dtype, int64_t M, int64_t K, int64_t ldx,
+                                 const uint8_t* w_packed, const int16_t* S, int32_t alpha, int64_t N, int32_t group,
+                                 void* y, int32_t y_dtype, int8_t* q_x, float* s_a, void* workspace,
+                                 int64_t workspace_bytes, void* stream) {
+    if (x_dtype != W4A8_F32 && x_dtype != W4A8_BF16) return W4A8_ERR_DTYPE;
+    w4a8_status st = check_gemm_shape(M, N, K, group);
     if (st != W4A8_OK) return st;
-    if (T < 0 || T > INT32_MAX) return W4A8_ERR_SHAPE;
+    if (ldx < K) return W4A8_ERR_SHAPE;
     if (y_dtype != W4A8_F16 && y_dtype != W4A8_F32 && y_dtype != W4A8_I32) return W4A8_ERR_DTYPE;
     if (!is_pow2(alpha) || alpha > (1 << 30)) return W4A8_ERR_INVALID_ARG;
-    if (!expert_offsets_host || !w_packed_host || !S_host) return W4A8_ERR_INVALID_ARG;
+    if (M == 0) return W4A8_OK;
+    if (!x || !w_packed || !S || !y) return W4A8_ERR_INVALID_ARG;
+    const int64_t esz = x_dtype == W4A8_BF16 ? 2 : 4;
+    if (!aligned16(x) || (ldx * esz) % 16 != 0 || !aligned16(w_packed) || !aligned16(S) || !aligned16(y))
+        return W4A8_ERR_ALIGN;
+    if ((q_x && !aligned16(q_x)) || (s_a && !aligned4(s_a))) return W4A8_ERR_ALIGN;
+    if (!gemv_path(M, K, false, false)) {
+        // more tokens: quantize into the caller's buffers, then the GEMM
+        if (!q_x || !s_a) return W4A8_ERR_INVALID_ARG;
+        if (!aligned16(s_a)) return W4A8_ERR_ALIGN;
+        st = quantize_act_per_token(x, x_dtype, M, K, ldx, q_x, s_a, stream);
+        if (st != W4A8_OK) return st;
+        return w4a8_gemm_intscale(q_x, s_a, w_packed, S, alpha, M, N, K, group, y, y_dtype, workspace,
+                                  workspace_bytes, stream);
+    }
     DeviceInfo dev;
     if ((st = current_device(dev)) != W4A8_OK) return st;
-    MoeLayout L;
-    if ((st = moe_layout(E, expert_offsets_host, N, K, group, dev, L)) != W4A8_OK) return st;
-    if (L.R == 0) return W4A8_OK;
-    if (!q_x || !s_a || !row_index || !y || T == 0) return W4A8_ERR_INVALID_ARG;
-    if (!aligned16(q_x) || !aligned16(y) || !aligned16(s_a) || !aligned16(row_index)) return W4A8_ERR_ALIGN;
-    for (int32_t e = 0; e < E; ++e) {
-        if (expert_offsets_host[e + 1] == expert_offsets_host[e]) continue;
-        if (!w_packed_host[e] || !S_host[e]) return W4A8_ERR_INVALID_ARG;
-        if (!aligned16(w_packed_host[e]) || !aligned16(S_host[e])) return W4A8_ERR_ALIGN;
-    }
+    w4a8::gemv::GemvParams g{};
+    g.x = x;
+    g.ldx = ldx;
+    g.w = w_packed;
+    g.S = S;
+    g.y = y;
+    g.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
+                                    : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
+    g.M = int32_t(M);
+    g.N = int32_t(N);
+    g.K = int32_t(K);
+    g.G = int32_t(K / group);
+    g.group = group;
+    g.inv_alpha = std::ldexp(1.0f, -int(std::log2(double(alpha))));
+    g.q_out = q_x;
+    g.s_out = s_a;
+    W4A8_CUDA_TRY(w4a8::gemv::launch(g, w4a8::gemm::kIntScale,
+                                     x_dtype == W4A8_BF16 ? w4a8::gemv::kXBf16 : w4a8::gemv::kXF32, dev.sms,
+                                     static_cast<cudaStream_t>(stream)));
+    return W4A8_OK;
+}
+
+int64_t w4a8_grouped_workspace_size(int32_t E, int64_t N, int64_t K, int32_t group) {
+    if (E < 1 || E > 256 || check_gemm_shape(1, N, K, group) != W4A8_OK) return -1;
+    DeviceInfo dev;
+    if (current_device(dev) != W4A8_OK) return -1;
+    return grouped_layout(E, dev).total;
+}
+
+w4a8_status w4a8_gemm_intscale_grouped(const int8_t* q_x, const float* s_a, int64_t T, const int32_t* row_index,
+                                       const int64_t* expert_offsets, const int32_t* out_row,
+                                       const uint8_t* const* w_packed, const int16_t* const* S, int32_t alpha,
+                                       int32_t E, int64_t R, int64_t N, int64_t K, int32_t group, void* y,
+                                       int32_t y_dtype, int64_t y_rows, void* workspace, int64_t workspace_bytes,
+                                       void* stream) {
+    w4a8_status st = check_gemm_shape(1, N, K, group);
+    if (st != W4A8_OK) return st;
+    if (E < 1 || E > 256) return W4A8_ERR_INVALID_ARG;
+    if (R < 0 || R > INT32_MAX || T < 0 || T > INT32_MAX || y_rows < 0) return W4A8_ERR_SHAPE;
+    if (y_dtype != W4A8_F16 && y_dtype != W4A8_F32 && y_dtype != W4A8_I32) return W4A8_ERR_DTYPE;
+    if (!is_pow2(alpha) || alpha > (1 << 30)) return W4A8_ERR_INVALID_ARG;
+    if (R == 0) return W4A8_OK;
+    if (T == 0 || !out_row && y_rows < R) return W4A8_ERR_SHAPE;
+    if (!q_x || !s_a || !row_index || !expert_offsets || !w_packed || !S || !y) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(q_x) || !aligned16(y) || !aligned4(s_a) || !aligned4(row_index) || (out_row && !aligned4(out_row)) ||
+        (reinterpret_cast<uintptr_t>(expert_offsets) & 7u) != 0 || (reinterpret_cast<uintptr_t>(w_packed) & 7u) != 0 ||
+        (reinterpret_cast<uintptr_t>(S) & 7u) != 0)
+        return W4A8_ERR_ALIGN;
+    DeviceInfo dev;
+    if ((st = current_device(dev)) != W4A8_OK) return st;
+    const GroupedLayout L = grouped_layout(E, dev);
     if (!workspace || workspace_bytes < L.total) return W4A8_ERR_WORKSPACE;
     if (!aligned16(workspace)) return W4A8_ERR_ALIGN;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
 
-    w4a8::moe::GatherParams gp{};
-    gp.q_x = q_x;
-    gp.s_a = s_a;
-    gp.T = T;
-    gp.K = K;
-    gp.row_index = row_index;
-    gp.xg = reinterpret_cast<int8_t*>(ws + L.x_off);
-    gp.sg = reinterpret_cast<float*>(ws + L.s_off);
-    gp.status = dev.status;
-    gp.E = E;
-    for (int32_t e = 0; e <= E; ++e) gp.off[e] = int32_t(expert_offsets_host[e]);
-    for (int32_t e = 0; e < E; ++e) gp.sbase[e] = L.sbase[e];
-    W4A8_CUDA_TRY(w4a8::moe::gather(gp, int(L.max_rows), cs));
-
-    const int64_t ysz = y_dtype == W4A8_F16 ? 2 : 4;
-    for (int32_t e = 0; e < E; ++e) {
-        const int64_t lo = expert_offsets_host[e], m = expert_offsets_host[e + 1] - lo;
-        if (m == 0) continue;
-        st = run_gemm(w4a8::gemm::kIntScale, gp.xg + lo * K, gp.sg + L.sbase[e], w_packed_host[e], S_host[e],
-                      nullptr, alpha, m, N, K, group, static_cast<uint8_t*>(y) + lo * N * ysz, y_dtype,
-                      L.gemm_bytes ? ws : nullptr, L.gemm_bytes, stream);
-        if (st != W4A8_OK) return st;
-    }
+    // tensor maps: a template for the experts' packed weights (its address
+    // is replaced per expert on the device), and the token codes gathered by
+    // row, four at a time (a box one row high)
+    CUtensorMap tm_w, tm_x;
+    if (!make_map_u8(&tm_w, workspace, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+        return W4A8_ERR_CUDA;
+    if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(T), uint64_t(K), 128, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+        return W4A8_ERR_CUDA;
+    w4a8::gemm::WideParams q{};
+    q.s_a = s_a;
+    q.y = y;
+    q.ws_count = reinterpret_cast<int32_t*>(ws);
+    q.ws_part = reinterpret_cast<int32_t*>(ws + 4096);
+    q.status = dev.status;
+    q.M = 0;
+    q.N = int32_t(N);
+    q.G = int32_t(K / group);
+    q.kb_per_group = group / 128;
+    q.n_tiles = int32_t((N + 127) / 128);
+    q.m_tiles = 0;
+    q.grid = int32_t(L.grid);
+    q.inv_alpha = std::ldexp(1.0f, -int(std::log2(double(alpha))));
+    q.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
+                                    : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
+    q.row_index = row_index;
+    q.out_row = out_row;
+    q.moe_scales = reinterpret_cast<const void* const*>(S);
+    q.moe_sched = reinterpret_cast<const int32_t*>(ws + L.sched_off);
+    q.moe_maps = reinterpret_cast<const CUtensorMap*>(ws + L.maps_off);
+    q.E = E;
+    q.moe_T = int32_t(T);
+    q.y_rows = out_row ? y_rows : R;
+    q.wait_limit = g_wait_limit.load();
+    W4A8_CUDA_TRY(w4a8::gemm::launch_wide_moe(tm_w, tm_x, expert_offsets,
+                                              reinterpret_cast<const void* const*>(w_packed), R, q,
+                                              reinterpret_cast<int32_t*>(ws + L.sched_off),
+                                              reinterpret_cast<CUtensorMap*>(ws + L.maps_off),
+                                              static_cast<cudaStream_t>(stream)));
     return W4A8_OK;
 }
 
@@ -570,6 +700,11 @@ w4a8_status w4a8_tensor_i8_peak_probe(int64_t iters, int32_t n, int32_t a_in_tme
     *grid_host = dev.sms;
     *ops_host = 2.0 * 128.0 * double(n) * 128.0 * double(iters) * double(dev.sms);
     return W4A8_OK;
+}
+
+int64_t w4a8_set_wait_limit(int64_t cycles) {
+    const long long v = cycles > 0 ? (long long)cycles : kDefaultWaitLimit;
+    return int64_t(g_wait_limit.exchange(v));
 }
 
 int32_t w4a8_last_cuda_error(int32_t clear) {

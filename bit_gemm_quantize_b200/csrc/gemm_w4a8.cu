@@ -51,6 +51,7 @@
 #include <cstdint>
 #include <type_traits>
 
+#include "gemm_common.cuh"
 #include "gemm_w4a8.h"
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -274,58 +275,6 @@ struct StageIter {
     }
 };
 
-// int4 two's-complement nibbles -> int8, 8 values per 32-bit word.  Byte j
-// of the word holds K position j (low nibble) and j + 4 (high nibble), so the
-// low nibbles give output word 0 (K 0..3) and the high nibbles word 1 (K 4..7)
-// in MMA order with no byte permute.
-// Exact: per byte ((v ^ 8) + 0x78) ^ 0x80 maps nibble v to its sign-extended
-// byte without carries between bytes.
-__device__ __forceinline__ uint2 unpack_int4x8(uint32_t w) {
-    uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
-    uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-    lo = (lo + 0x78787878u) ^ 0x80808080u;
-    hi = (hi + 0x78787878u) ^ 0x80808080u;
-    return make_uint2(lo, hi);
-}
-
-// Scaled: each nibble lands in the high half of its byte, which read as int8
-// is 16 * q exactly.
-__device__ __forceinline__ uint2 unpack_int4x8_x16(uint32_t w) {
-    return make_uint2((w << 4) & 0xF0F0F0F0u, w & 0xF0F0F0F0u);
-}
-
-template <bool X16>
-__device__ __forceinline__ uint2 unpack8(uint32_t w) {
-    if constexpr (X16)
-        return unpack_int4x8_x16(w);
-    else
-        return unpack_int4x8(w);
-}
-
-__device__ __forceinline__ void epi_bar_sync(int threads) {
-    asm volatile("bar.sync 1, %0;" ::"r"(threads) : "memory");
-}
-
-template <int N>
-__device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t (&r)[N]) {
-    if constexpr (N == 8) {
-        tmem_ld8(taddr, r);
-    } else if constexpr (N == 16) {
-        tmem_ld16(taddr, r);
-    } else {
-        static_assert(N == 32, "columns per load");
-        tmem_ld32(taddr, r);
-    }
-}
-
-// Bounded wait without the abort short-cut, for draining copies in flight.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitLimitCycles) break;
-    }
-}
-
 // Output scale of token m: s_a[m] / alpha (exact: 1/alpha is a power of two)
 // for the integer-scale path, s_a[m] for the float-scale path.
 template <int PATH>
@@ -333,29 +282,6 @@ __device__ __forceinline__ float output_scale(const Params& p, int64_t m) {
     return PATH == kIntScale ? __fmul_rn(p.s_a[m], p.inv_alpha) : p.s_a[m];
 }
 
-// Acquire load at GPU scope (the arrival counter of a split tile).
-__device__ __forceinline__ int ld_acquire_gpu(const int* addr) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
-    return v;
-}
-
-// Release add at GPU scope: the CTA's writes ordered before it (by a CTA
-// barrier) become visible to a thread that acquires the counter.
-__device__ __forceinline__ void red_release_gpu_add(int* addr, int v) {
-    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
-}
-
-struct Ring {
-    int idx = 0;
-    uint32_t phase = 0;
-    __device__ __forceinline__ void advance(int n) {
-        if (++idx == n) {
-            idx = 0;
-            phase ^= 1u;
-        }
-    }
-};
 
 // G1: the group is one 128-wide K block (group = 128, the method's group
 // size), so every K block ends a group; wide token tiles then drain each group
@@ -476,10 +402,10 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                 bool free_slot;
                 if constexpr (C::kW8) {
                     // the MMAs of stage pst - SW have read this weight slot
-                    free_slot = pst < SW || mbar_wait_warp(&sdone[rwd.idx], rwd.phase, abort_flag, p.status);
+                    free_slot = pst < SW || mbar_wait_warp(&sdone[rwd.idx], rwd.phase, abort_flag, p.status, p.wait_limit);
                     if (pst >= SW) rwd.advance(SD);
                 } else {
-                    free_slot = mbar_wait_warp(&empty_w[rw.idx], rw.phase ^ 1u, abort_flag, p.status);
+                    free_slot = mbar_wait_warp(&empty_w[rw.idx], rw.phase ^ 1u, abort_flag, p.status, p.wait_limit);
                 }
                 if (!free_slot) {
                     ok = false;
@@ -489,7 +415,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             }
             rw.advance(SW);
             if (pst >= SX) {  // the MMAs of stage pst - SX have read this token slot
-                if (!mbar_wait_warp(&sdone[rxd.idx], rxd.phase, abort_flag, p.status)) {
+                if (!mbar_wait_warp(&sdone[rxd.idx], rxd.phase, abort_flag, p.status, p.wait_limit)) {
                     ok = false;
                     break;
                 }
@@ -532,9 +458,9 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
         const uint32_t w_lo0 = smem_desc_sw128_lo(smem_u32(smem + C::offW));
         while (ok && it.next(st)) {
             // the A operand: the unpacked slot in TMEM, or the int8 weight box itself
-            const bool a_ready = C::kW8 ? mbar_wait_warp(&full_w[rw.idx], rw.phase, abort_flag, p.status)
-                                        : mbar_wait_warp(&full_a[ra.idx], ra.phase, abort_flag, p.status);
-            if (!a_ready || !mbar_wait_warp(&full_x[rx.idx], rx.phase, abort_flag, p.status)) {
+            const bool a_ready = C::kW8 ? mbar_wait_warp(&full_w[rw.idx], rw.phase, abort_flag, p.status, p.wait_limit)
+                                        : mbar_wait_warp(&full_a[ra.idx], ra.phase, abort_flag, p.status, p.wait_limit);
+            if (!a_ready || !mbar_wait_warp(&full_x[rx.idx], rx.phase, abort_flag, p.status, p.wait_limit)) {
                 ok = false;
                 break;
             }
@@ -549,7 +475,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                 const bool last = G1 || (kin == p.kb_per_group - 1);
                 if constexpr (!G1) kin = last ? 0 : kin + 1;
                 if (first) {
-                    if (!mbar_wait_warp(&tempty[rt.idx], rt.phase ^ 1u, abort_flag, p.status)) {
+                    if (!mbar_wait_warp(&tempty[rt.idx], rt.phase ^ 1u, abort_flag, p.status, p.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -579,7 +505,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             if constexpr (!C::kGroupCommit) {
                 // the epilogue waits on stage-done phases: it must have seen the
                 // previous phase of this slot before it is committed again
-                if (!mbar_wait_warp(&sseen[rd.idx], rd.phase ^ 1u, abort_flag, p.status)) {
+                if (!mbar_wait_warp(&sseen[rd.idx], rd.phase ^ 1u, abort_flag, p.status, p.wait_limit)) {
                     ok = false;
                     break;
                 }
@@ -615,7 +541,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
         bool ok = true;
         const uint32_t lane_base = tmem_base + (uint32_t(quarter * 32) << 16);
         while (ok && it.next(st)) {
-            if (!mbar_wait_warp(&full_w[rw.idx], rw.phase, abort_flag, p.status)) {
+            if (!mbar_wait_warp(&full_w[rw.idx], rw.phase, abort_flag, p.status, p.wait_limit)) {
                 ok = false;
                 break;
             }
@@ -629,7 +555,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             __syncwarp();
             mbar_arrive_one(&empty_w[rw.idx]);
             if (ust >= SA) {  // the MMAs of stage ust - SA have read this operand slot
-                if (!mbar_wait_warp(&sdone[rad.idx], rad.phase, abort_flag, p.status)) {
+                if (!mbar_wait_warp(&sdone[rad.idx], rad.phase, abort_flag, p.status, p.wait_limit)) {
                     ok = false;
                     break;
                 }
@@ -758,7 +684,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                     s1 = s2;
                     if (g + 2 < sg.g1) s2 = ld_scale(sidx);
                     sidx += nstride;
-                    if (!mbar_wait_warp(&afull[rt.idx], rt.phase, abort_flag, p.status)) {
+                    if (!mbar_wait_warp(&afull[rt.idx], rt.phase, abort_flag, p.status, p.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -835,7 +761,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                     // Per-stage commits: wait for the stage, then tell the MMA
                     // warp its phase was seen (it waits for that before it
                     // commits the slot again).
-                    if (!mbar_wait_warp(&sdone[rd.idx], rd.phase, abort_flag, p.status)) {
+                    if (!mbar_wait_warp(&sdone[rd.idx], rd.phase, abort_flag, p.status, p.wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -897,8 +823,8 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                 if constexpr (HC <= 16) {
                     // small tiles: both groups' loads in flight before one wait
                     if constexpr (C::kGroupCommit) {
-                        if (!mbar_wait_warp(&afull[gb0], ph0, abort_flag, p.status) ||
-                            (ng == 2 && !mbar_wait_warp(&afull[gb1], ph1, abort_flag, p.status))) {
+                        if (!mbar_wait_warp(&afull[gb0], ph0, abort_flag, p.status, p.wait_limit) ||
+                            (ng == 2 && !mbar_wait_warp(&afull[gb1], ph1, abort_flag, p.status, p.wait_limit))) {
                             ok = false;
                             break;
                         }
@@ -921,7 +847,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                     for (int gi = 0; gi < ng; ++gi) {
                         const uint32_t gb = gi == 0 ? gb0 : gb1;
                         if constexpr (C::kGroupCommit) {
-                            if (!mbar_wait_warp(&afull[gb], gi == 0 ? ph0 : ph1, abort_flag, p.status)) {
+                            if (!mbar_wait_warp(&afull[gb], gi == 0 ? ph0 : ph1, abort_flag, p.status, p.wait_limit)) {
                                 ok = false;
                                 break;
                             }
@@ -988,7 +914,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                     const long long w0 = clock64();
                     int ok_wait = 1;
                     while (ld_acquire_gpu(&p.ws_count[b_first]) < expect) {
-                        if (*abort_flag || clock64() - w0 > kWaitLimitCycles) {
+                        if (*abort_flag || clock64() - w0 > p.wait_limit) {
                             *abort_flag = 1;
                             atomicExch(p.status, kStatusTimeout);
                             ok_wait = 0;
@@ -1089,15 +1015,17 @@ static int token_tile_for(int64_t M) {
     return 128;
 }
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool w8) {
+Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool w8, bool narrow_only) {
     Plan pl{};
-    pl.BT = token_tile_for(M);
+    // more tokens than one 128-token tile: the wide-tile kernel (gemm_wide.cu)
+    pl.wide = !w8 && !narrow_only && M > 128;
+    pl.BT = pl.wide ? wide_token_tile() : token_tile_for(M);
     pl.n_tiles = (N + kTileN - 1) / kTileN;
     pl.m_tiles = (M + pl.BT - 1) / pl.BT;
     pl.G = K / group;
     pl.tiles = pl.n_tiles * pl.m_tiles;
     pl.W = pl.tiles * pl.G;
-    const int64_t slots = int64_t(num_sms) * (w8 ? 1 : W4A8_CTAS_PER_SM(pl.BT));  // resident CTAs
+    const int64_t slots = int64_t(num_sms) * ((w8 || pl.wide) ? 1 : W4A8_CTAS_PER_SM(pl.BT));  // resident CTAs
     pl.grid = pl.W < slots ? pl.W : slots;
     if (pl.grid > kMaxGrid) pl.grid = kMaxGrid;
     const int64_t slot_bytes = int64_t(kTileN) * pl.BT * 4;

@@ -29,6 +29,7 @@ struct Params {
     uint32_t w_q, w_r;   // W / grid, W % grid
     float inv_alpha;     // 1 / alpha (exact, alpha is a power of two)
     int32_t y_dtype;     // OutType
+    long long wait_limit;  // SM cycles a pipeline or split-tile wait may last before it gives up
 };
 
 // Parameters of the kernels for asymmetric token codes (a separate type, so
@@ -38,7 +39,67 @@ struct ParamsZp : Params {
     const int32_t* zc;   // [N] zero-point term zc[n] = sum_g S[g,n] sum_{k in g} q[k,n]
 };
 
+// Parameters of the wide-tile kernel (token tiles of 256; gemm_wide.cu).
+struct WideParams {
+    const float* s_a;    // [M] token scales (MOE: [T], indexed by token)
+    const int16_t* S;    // [G, N] integer group scales (dense integer-scale path)
+    const float* s_g;    // [G, N] float group scales (float-scale path)
+    void* y;             // [M, N] output (MOE: [rows, N], row out_row[i] or i)
+    int32_t* ws_part;    // [grid][128 * 256] partial sums of split tiles
+    int32_t* ws_count;   // [grid] arrival counters, zero between calls
+    int* status;         // device status word
+    int32_t M, N;
+    int32_t G;           // groups along K
+    int32_t kb_per_group;
+    int32_t n_tiles, m_tiles;
+    int32_t grid;
+    uint32_t W, w_q, w_r;  // (tile, group) steps, W / grid, W % grid (dense; MOE: moe_sched)
+    float inv_alpha;
+    int32_t y_dtype;
+    // mixture of experts
+    const int32_t* row_index;      // [R] token of each routed row, rows grouped by expert
+    const int32_t* out_row;        // [R] output row of each routed row, or null (row i)
+    const void* const* moe_scales; // [E] device pointers to each expert's S [G, N]
+    const int32_t* moe_sched;      // W, w_q, w_r, status, then mt[E+1], tstart[E+1], rstart[E+1]
+    const CUtensorMap* moe_maps;   // [E] weight tensor maps
+    int32_t E;
+    int32_t moe_T;                 // tokens: row_index values must lie in [0, T)
+    int64_t y_rows;                // rows of y (MOE): a routed row's output row must be below it
+    long long wait_limit;          // SM cycles a pipeline or split-tile wait may last before it gives up
+};
+
+}  // namespace gemm
+
+namespace gemv {
+// Decode-shaped layers on the CUDA cores (gemv_w4a8.cu): M <= 4 tokens,
+// K <= kMaxK, one CTA per 32 output columns.
+constexpr int kMaxM = 4;
+constexpr int kMaxK = 16384;
+enum XKind { kXCodes = 0, kXBf16 = 1, kXF32 = 2 };
+
+struct GemvParams {
+    const void* x;         // int8 codes [M][K] (kXCodes) or bf16 / fp32 tokens [M][ldx] (quantized here)
+    const float* s_a;      // [M] token scales (kXCodes)
+    int64_t ldx;           // row pitch of x in elements (bf16 / fp32 tokens)
+    const uint8_t* w;      // packed int4 weights [N][K/2]
+    const int16_t* S;      // [G][N] integer scales (integer-scale path)
+    const float* s_g;      // [G][N] float scales (float-scale path)
+    void* y;               // [M][N]
+    int32_t y_dtype;       // gemm::OutType
+    int32_t M, N, K, G, group;
+    float inv_alpha;       // 1 / alpha (integer-scale path)
+    int8_t* q_out;         // optional: the codes the kernel computed [M][K] (fused tokens)
+    float* s_out;          // optional: their scales [M]
+};
+
+int smem_bytes(int mt, int K, int ks);
+cudaError_t launch(const GemvParams& p, int path, int x_kind, int num_sms, cudaStream_t stream);
+}  // namespace gemv
+
+namespace gemm {
+
 struct Plan {
+    bool wide;           // the wide-tile kernel (token tiles of wide_token_tile())
     int BT;              // tokens per tile (MMA N)
     int64_t n_tiles, m_tiles, tiles, G, W, grid;
     int64_t count_bytes;  // bytes of the fixed counter region at the start of the workspace
@@ -46,7 +107,9 @@ struct Plan {
 };
 
 // w8: int8 weight codes (the W8A8 variant); its CTAs run one per SM
-Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool w8 = false);
+// narrow_only: tiles of at most 128 tokens whatever M (the asymmetric-token kernel)
+Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool w8 = false,
+               bool narrow_only = false);
 
 // tm_w: packed weights [N][K/2] u8, box 128 B x 128 rows, 128-byte swizzle
 // tm_x: token codes [M][K] u8, box 128 B x BT rows, 128-byte swizzle
@@ -59,6 +122,22 @@ cudaError_t launch(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUten
 // integer-scale path with int4 weights
 cudaError_t launch_zp(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap& tm_y, const ParamsZp& p,
                       int BT, cudaStream_t stream);
+
+// Wide-tile kernel (token tiles of 256, gemm_wide.cu), integer- or float-scale path.
+// tm_w: packed weights [N][K/2] u8, box 64 B x 128 rows, no swizzle
+// tm_x: token codes [M][K] u8, box 128 B x 256 rows, 128-byte swizzle
+// tm_y: output [M][N], box 128 columns x wide_token_tile() rows (fp16) or 64 rows (4-byte outputs)
+cudaError_t launch_wide(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap& tm_y, const WideParams& p,
+                        int path, cudaStream_t stream);
+// Mixture of experts (integer-scale path): a setup kernel builds the schedule
+// and the per-expert weight maps from device offsets and pointers, then the
+// wide kernel runs over all experts' tiles.  tm_w_template: a weight map of
+// the experts' shape (its address is replaced per expert); tm_x: token codes
+// [T][K] u8, box 128 B x 1 row, 128-byte swizzle (rows gathered four at a time).
+cudaError_t launch_wide_moe(const CUtensorMap& tm_w_template, const CUtensorMap& tm_x, const int64_t* offsets,
+                            const void* const* w_ptrs, int64_t R, const WideParams& p, int32_t* sched,
+                            CUtensorMap* maps, cudaStream_t stream);
+int wide_token_tile();
 
 int token_tile_rows();
 

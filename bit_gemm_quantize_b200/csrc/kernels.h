@@ -60,24 +60,6 @@ cudaError_t launch_asym(const void* x, bool bf16, int64_t M, int64_t K, int64_t 
                         int32_t* z_a, cudaStream_t stream, int num_sms);
 }
 
-namespace moe {
-constexpr int kMaxExperts = 256;
-// Routed-row gather: rows off[e] .. off[e+1]-1 belong to expert e; row i takes
-// token row_index[i]'s codes into xg[i] and its scale into sg[sbase[e] + i - off[e]].
-struct GatherParams {
-    const int8_t* q_x;        // [T, K] token codes
-    const float* s_a;         // [T] token scales
-    int64_t T, K;
-    const int32_t* row_index; // [R] token of each routed row
-    int8_t* xg;               // [R, K] gathered codes
-    float* sg;                // gathered scales, expert e's at float offset sbase[e] (16-byte aligned)
-    int* status;              // device status word (W4A8_ERR_INVALID_ARG for a token index out of range)
-    int32_t E;
-    int32_t off[kMaxExperts + 1];
-    int32_t sbase[kMaxExperts];
-};
-cudaError_t gather(const GatherParams& p, int max_rows, cudaStream_t stream);
-}  // namespace moe
 
 namespace peak {
 // Back-to-back int8 MMAs (128 x n x 32, n % 16 == 0, 16 <= n <= 256) on

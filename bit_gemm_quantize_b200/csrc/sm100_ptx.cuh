@@ -67,14 +67,20 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // so that the whole CTA leaves its loops and reaches the teardown.
 constexpr long long kWaitLimitCycles = 1ll << 31;
 
+// The suspend hint of a bounded wait: 200 us, or less under a shorter limit,
+// so that the limit is checked in time.
+__device__ __forceinline__ uint32_t wait_hint_ns(long long limit) {
+    return limit < 400000ll ? uint32_t(limit / 2) : 200000u;
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+                                          int* status, long long limit = kWaitLimitCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+        if (mbar_try_wait_sleep(bar, parity, wait_hint_ns(limit))) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             atomicExch(status, kStatusTimeout);
             return false;
@@ -88,16 +94,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // costs one poll and one vote; the blocking loop is out of line so that it
 // adds neither instructions nor registers to the caller's fast path.
 static __device__ __noinline__ bool mbar_wait_warp_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                                 int* status) {
+                                                 int* status, long long limit) {
     const long long t0 = clock64();
+    const uint32_t hint = wait_hint_ns(limit);
     while (true) {
-        const bool ok = mbar_try_wait_sleep(bar, parity, 200000u);
+        const bool ok = mbar_try_wait_sleep(bar, parity, hint);
         if (__all_sync(0xffffffffu, ok)) return true;
         int fail = 0;
         if ((threadIdx.x & 31) == 0) {
             if (*abort_flag) {
                 fail = 1;
-            } else if (clock64() - t0 > kWaitLimitCycles) {
+            } else if (clock64() - t0 > limit) {
                 *abort_flag = 1;
                 atomicExch(status, kStatusTimeout);
                 fail = 1;
@@ -108,9 +115,9 @@ static __device__ __noinline__ bool mbar_wait_warp_slow(uint64_t* bar, uint32_t 
 }
 
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                               int* status) {
+                                               int* status, long long limit = kWaitLimitCycles) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-    return mbar_wait_warp_slow(bar, parity, abort_flag, status);
+    return mbar_wait_warp_slow(bar, parity, abort_flag, status, limit);
 }
 
 // ---------------------------------------------------------------- one-lane operations of a converged warp
@@ -182,6 +189,50 @@ __device__ __forceinline__ void tma_load_2d_one(void* dst, const CUtensorMap* ma
         "\n\t}" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
         : "memory");
+}
+
+// Four rows of a 2-D tensor gathered by row index (tile::gather4): the
+// tensor map's box is one row high; rows r0..r3 at column c0 land in four
+// consecutive box-sized rows at dst (with the map's swizzle).  Issued by the
+// calling thread (every active lane issues its own copy).
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int32_t c0, int32_t r0, int32_t r1,
+                                            int32_t r2, int32_t r3, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 1-D bulk copy shared -> global (16-byte aligned addresses, size % 16 == 0),
+// tracked per thread with bulk async-groups like tma_store_2d.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+                 "r"(smem_u32(src)), "r"(bytes)
+                 : "memory");
+}
+
+// Tensor maps built on the device: a copy in shared memory gets a new global
+// base address, then the whole warp copies it to global memory and releases
+// it to the tensor-map proxy; a thread that issues TMA copies with it first
+// acquires it.
+__device__ __forceinline__ void tensormap_replace_address(void* smem_map, const void* gaddr) {
+    asm volatile("tensormap.replace.tile.global_address.shared::cta.b1024.b64 [%0], %1;" ::"r"(smem_u32(smem_map)),
+                 "l"(reinterpret_cast<uint64_t>(gaddr))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tensormap_publish(void* gmem_map, const void* smem_map) {
+    asm volatile(
+        "tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned [%0], [%1], 128;" ::"l"(
+            reinterpret_cast<uint64_t>(gmem_map)),
+        "r"(smem_u32(smem_map))
+        : "memory");
+}
+
+__device__ __forceinline__ void tensormap_acquire(const void* gmem_map) {
+    asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(gmem_map))
+                 : "memory");
 }
 
 // 2-D tiled TMA store from this CTA's shared memory (one thread).  Elements

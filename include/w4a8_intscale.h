@@ -217,6 +217,9 @@ W4A8_API int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32
 /*
  * W4A8 GEMM with integer group scales (the Integer-Scale scheme).
  * (Integer Scale summary §4 / Fig. 3(c); "Quantization" notes 矩阵乘法中的量化计算.)
+ * Kernels by shape: M <= 4 (and K <= 16384) a CUDA-core kernel that streams the
+ * weights (no workspace); M <= 128 the tcgen05 kernel with token tiles of
+ * 16..128; larger M the wide-tile tcgen05 kernel (token tiles of 192).
  *   P_g[m,n] = sum_{k in g} q_x[m,k] q_w[k,n]            (int8 x int4 -> int32, tensor cores)
  *   acc[m,n] = sum_g S[g,n] * P_g[m,n]                    (int32, exact)
  *   y[m,n]   = fl_out(fl32(acc) * fl32(s_a[m] / alpha))   (one conversion per output)
@@ -237,6 +240,27 @@ W4A8_API w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, con
                                const int16_t* S, int32_t alpha, int64_t M, int64_t N, int64_t K,
                                int32_t group, void* y, int32_t y_dtype, void* workspace,
                                int64_t workspace_bytes, void* stream);
+
+/*
+ * The whole integer-scale linear layer from unquantized tokens: per-token
+ * quantization, then the W4A8 integer-scale GEMM (Integer Scale summary,
+ * Fig. 3(c): int8 tokens, int4 weights, integer group scales, one rescale).
+ *   q_x, s_a = quantize_act_per_token(x);  y = w4a8_gemm_intscale(q_x, s_a, ...)
+ * With M <= 4 tokens (and K <= 16384) it is one kernel: every CTA quantizes
+ * the tokens itself (the same codes and scales, bit for bit, as
+ * quantize_act_per_token) and streams its weight columns on the CUDA cores;
+ * with more tokens it is the two calls above, chained on `stream`.
+ * x, x_dtype, M, K, ldx   as quantize_act_per_token (W4A8_F32 or W4A8_BF16)
+ * w_packed, S, alpha, N, group, y, y_dtype, workspace   as w4a8_gemm_intscale
+ * q_x, s_a   device, [M, K] int8 and [M] float32: written with the token codes
+ *            and scales when given (may be NULL when M <= 4); required when
+ *            M > 4 (W4A8_ERR_INVALID_ARG otherwise), s_a then 16-byte aligned
+ * Errors: as quantize_act_per_token and w4a8_gemm_intscale.
+ */
+W4A8_API w4a8_status w4a8_linear_intscale(const void* x, int32_t x_dtype, int64_t M, int64_t K, int64_t ldx,
+                                         const uint8_t* w_packed, const int16_t* S, int32_t alpha, int64_t N,
+                                         int32_t group, void* y, int32_t y_dtype, int8_t* q_x, float* s_a,
+                                         void* workspace, int64_t workspace_bytes, void* stream);
 
 /*
  * Weight-side zero-point term for asymmetric activations.
@@ -323,43 +347,58 @@ W4A8_API w4a8_status w4a8_gemm_intscale_static_ws(const int8_t* q_x, const float
                                                  int32_t group, void* y, int32_t y_dtype, void* stream);
 
 /*
- * Mixture-of-experts layer: one integer-scale W4A8 GEMM per expert over the
- * rows routed to it.  (Integer Scale summary §5.3: the method applied to
- * Mixtral 8x7B; every expert's linear layer is a fine-grained W4A8 GEMM and
- * the amplifier is one per layer, shared by all experts.)
+ * Mixture-of-experts layer in one grouped call: the integer-scale W4A8 GEMM of
+ * every expert over the token rows routed to it.  (Integer Scale summary
+ * §5.3: the method applied to Mixtral 8x7B; every expert's linear layer is a
+ * fine-grained W4A8 GEMM and the amplifier is one per layer, shared by all
+ * experts.)
  *   for every routed row i of expert e (offsets[e] <= i < offsets[e+1]):
- *     y[i, :] = w4a8_gemm_intscale row of token row_index[i] with expert e's
- *               w_packed[e], S[e] and the shared alpha
+ *     y[out_row ? out_row[i] : i, :] = the w4a8_gemm_intscale row of token
+ *         row_index[i] with expert e's w_packed[e], S[e] and the shared alpha
+ * Everything the routing decides is read on the device, so a router kernel
+ * earlier in the stream can produce it without a host round trip: a small
+ * setup kernel turns the offsets into the schedule and each expert's weight
+ * tensor map (in the workspace), then one persistent launch covers every
+ * (expert, tile, group) step.  Token rows are fetched from q_x by index; no
+ * gathered copy is made.
  * q_x, s_a   device, [T, K] int8 and [T] float32: every token quantized once
- *            (quantize_act_per_token); T >= 1 when any row is routed
+ *            (quantize_act_per_token); q_x 16-byte, s_a 4-byte aligned
  * row_index  device, [R] int32: the token of each routed row, rows grouped by
- *            expert (expert 0 first); a token index outside [0, T) makes that
- *            row's output zero and sets the device status word to
- *            W4A8_ERR_INVALID_ARG (read with w4a8_device_status)
- * expert_offsets_host  HOST, [E+1] int64: offsets[0] = 0, non-decreasing,
- *            R = offsets[E] < 2^31; they size the per-expert launches
- * w_packed_host, S_host  HOST arrays of E device pointers: expert e's packed
- *            weights [N, K/2] and integer scales [K/group, N], all packed with
- *            the same alpha (pack each expert's s_g with S = NULL, run
- *            w4a8_amplifier_search over all of them, pack every expert with it);
- *            pointers of experts with no rows may be NULL
- * 1 <= E <= 256; N, K, group as for w4a8_gemm_intscale
- * y          device, [R, N] of y_dtype (W4A8_F16, W4A8_F32, W4A8_I32)
- * workspace  device, >= w4a8_moe_workspace_size(E, offsets, N, K, group) bytes,
- *            zero-filled before its first use; its first 4096 bytes are
- *            counters that every completed call leaves at zero, the rest holds
- *            the gathered rows and partial sums
- * Launches a gather kernel and one GEMM per expert with rows, asynchronously
- * on `stream`.
+ *            expert (expert 0 first).  A token outside [0, T) gives that row
+ *            zero output and sets W4A8_ERR_INVALID_ARG in the device status word
+ * expert_offsets  device, [E+1] int64 (8-byte aligned): offsets[0] = 0,
+ *            non-decreasing, offsets[E] = R; anything else makes the call
+ *            write nothing and set W4A8_ERR_INVALID_ARG in the device status
+ * out_row    device, [R] int32 or NULL: the output row of each routed row, e.g.
+ *            token * top_k + slot to return rows in (token, slot) order; NULL
+ *            writes routed row i to row i.  A row outside [0, y_rows) is not
+ *            written and sets W4A8_ERR_INVALID_ARG in the device status word
+ * w_packed, S  device arrays (8-byte aligned) of E device pointers: expert e's
+ *            packed weights [N, K/2] (16-byte aligned) and integer scales
+ *            [K/group, N] (2-byte aligned), all packed with the same alpha (pack
+ *            each expert's s_g with S = NULL, run w4a8_amplifier_search over all
+ *            of them, pack every expert with it).  Experts with no rows may
+ *            have NULL pointers; a NULL or misaligned pointer of an expert with
+ *            rows makes the call write nothing and set W4A8_ERR_INVALID_ARG
+ * E          1 <= E <= 256; R the routed rows (T * top_k), 0 <= R < 2^31;
+ *            N, K, group as for w4a8_gemm_intscale
+ * y          device, [y_rows, N] of y_dtype (W4A8_F16, W4A8_F32, W4A8_I32),
+ *            16-byte aligned; y_rows >= R when out_row is NULL
+ * workspace  device, >= w4a8_grouped_workspace_size(E, N, K, group) bytes,
+ *            16-byte aligned, zero-filled before its first use; its first 4096
+ *            bytes are counters that every completed call leaves at zero, the
+ *            rest holds partial sums, the tensor maps and the schedule
+ * Asynchronous on `stream`: two launches (setup, then the GEMM), chained with
+ * programmatic dependent launch.
  */
-W4A8_API int64_t w4a8_moe_workspace_size(int32_t E, const int64_t* expert_offsets_host, int64_t N, int64_t K,
-                                         int32_t group);
-W4A8_API w4a8_status w4a8_moe_gemm_intscale(const int8_t* q_x, const float* s_a, int64_t T,
-                                           const int32_t* row_index, const int64_t* expert_offsets_host,
-                                           const uint8_t* const* w_packed_host, const int16_t* const* S_host,
-                                           int32_t alpha, int32_t E, int64_t N, int64_t K, int32_t group,
-                                           void* y, int32_t y_dtype, void* workspace, int64_t workspace_bytes,
-                                           void* stream);
+W4A8_API int64_t w4a8_grouped_workspace_size(int32_t E, int64_t N, int64_t K, int32_t group);
+W4A8_API w4a8_status w4a8_gemm_intscale_grouped(const int8_t* q_x, const float* s_a, int64_t T,
+                                               const int32_t* row_index, const int64_t* expert_offsets,
+                                               const int32_t* out_row, const uint8_t* const* w_packed,
+                                               const int16_t* const* S, int32_t alpha, int32_t E, int64_t R,
+                                               int64_t N, int64_t K, int32_t group, void* y, int32_t y_dtype,
+                                               int64_t y_rows, void* workspace, int64_t workspace_bytes,
+                                               void* stream);
 
 /*
  * W4A8 GEMM with float group scales, the comparison path.
@@ -392,6 +431,20 @@ W4A8_API w4a8_status w4a8_tensor_i8_peak_probe(int64_t iters, int32_t n, int32_t
                                               double* ops_host, void* stream);
 
 /*
+ * How long the GEMMs' waits inside a kernel may last: the pipeline waits
+ * between the roles of a CTA and a split tile's wait for the other CTAs'
+ * partial sums, in SM clock cycles (default 2^31, about one second).  A wait
+ * that runs out makes the kernel leave early (after the copies and MMAs it has
+ * in flight complete) with W4A8_ERR_TIMEOUT in the device status word; the
+ * call's output is then undefined and its workspace must be zeroed again.
+ * cycles <= 0 restores the default.  Applies to launches made after the call,
+ * process-wide.  Returns the previous limit.  A diagnostic and test aid: a
+ * short limit turns a stall (another kernel holding SMs, for instance) into an
+ * error the host can read.
+ */
+W4A8_API int64_t w4a8_set_wait_limit(int64_t cycles);
+
+/*
  * The CUDA runtime error code (cudaError_t) behind the last W4A8_ERR_CUDA that
  * a call of this library returned on the calling thread (0 if none); with
  * clear != 0 the record is reset.  w4a8_cuda_error_string names a code.
@@ -402,8 +455,8 @@ W4A8_API const char* w4a8_cuda_error_string(int32_t code);
 /*
  * Reads (and with clear != 0 resets) the device status word of the current
  * device: 0, or the last device-side error: W4A8_ERR_TIMEOUT (a bounded wait
- * ran out) or W4A8_ERR_INVALID_ARG (a routed row's token index out of range in
- * w4a8_moe_gemm_intscale).  Synchronous.  The word keeps only the last error,
+ * ran out) or W4A8_ERR_INVALID_ARG (bad routing data in
+ * w4a8_gemm_intscale_grouped).  Synchronous.  The word keeps only the last error,
  * so clearing any nonzero status also zeroes the arrival counters of the
  * library's own workspace (w4a8_static_workspace_reset); caller workspaces
  * must be zeroed by the caller.

@@ -241,3 +241,28 @@ def test_failed_gemm_rezeroes_cached_workspaces(lib):
     finally:
         _native._ws_cache.clear()
         _native._ws_cache.update(saved)
+
+
+def test_grouped_argument_checks(lib):
+    def gr(E=4, R=16, T=8, dt=_native.F16, alpha=1024, K=256, q=A, off=A, wp=A, sp=A, out_row=0, y_rows=16, y=A):
+        return lib.w4a8_gemm_intscale_grouped(ctypes.c_void_p(q), ctypes.c_void_p(A), T, ctypes.c_void_p(A),
+                                              ctypes.c_void_p(off), ctypes.c_void_p(out_row), ctypes.c_void_p(wp),
+                                              ctypes.c_void_p(sp), alpha, E, R, 128, K, 128, ctypes.c_void_p(y), dt,
+                                              y_rows, None, 0, None)
+
+    assert gr(E=0) == INVALID
+    assert gr(E=257) == INVALID
+    assert gr(K=200) == SHAPE
+    assert gr(R=-1) == SHAPE
+    assert gr(dt=_native.BF16) == DTYPE
+    assert gr(alpha=6) == INVALID
+    assert gr(R=0) == OK  # nothing routed: a no-op
+    assert gr(T=0) == SHAPE
+    assert gr(y_rows=15) == SHAPE  # rows written in routed order need y_rows >= R
+    assert gr(q=0) == INVALID
+    assert gr(wp=0) == INVALID
+    assert gr(q=U) == ALIGN
+    assert gr(off=A + 4) == ALIGN  # int64 offsets: 8-byte aligned
+    assert gr(sp=A + 4) == ALIGN
+    assert lib.w4a8_grouped_workspace_size(0, 128, 256, 128) == -1
+    assert lib.w4a8_grouped_workspace_size(4, 100, 256, 128) == -1

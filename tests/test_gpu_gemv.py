@@ -1,0 +1,93 @@
+"""The decode-shaped path (M <= 4 tokens, CUDA-core kernel) and the fused
+linear entry point against the oracle: raw int32 accumulators bit-exact,
+token codes and scales bit-exact when the kernel quantizes them itself, fp
+outputs within the tolerance of the other parity tests."""
+import numpy as np
+import pytest
+import torch
+
+import bit_gemm_quantize_b200 as bgq
+import oracle
+from bit_gemm_quantize_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+RTOL = {"f32": 1e-3, "f16": 4e-3}
+
+
+def _close(y, y_ref, out):
+    y = np.asarray(y, np.float64)
+    tau = max(1e-2 * np.sqrt(np.mean(np.square(y_ref))), 1e-30)
+    err = np.abs(y - y_ref) / np.maximum(np.abs(y_ref), tau)
+    assert err.max(initial=0.0) <= RTOL[out], f"max rel err {err.max():.3e}"
+
+
+CASES = [
+    # M, K, N, group: every token count, ragged N (columns past N in the last CTA),
+    # groups of 128 / 256 / 512 and group = K, a K that splits over 16 warps
+    (1, 4096, 4096, 128),
+    (2, 1024, 136, 128),
+    (3, 2048, 1032, 256),
+    (4, 4096, 520, 128),
+    (1, 512, 256, 512),
+    (4, 8192, 264, 128),
+    (2, 16384, 128, 128),
+]
+
+
+@pytest.mark.parametrize("M,K,N,group", CASES)
+def test_gemv_intscale_and_floatscale(M, K, N, group):
+    dev = torch.device("cuda:0")
+    wl = workloads.make_linear(M, K, N, x_dtype="bf16", seed=7 * M + K + N, group=group)
+    q, s = bgq.quantize_act_per_token(torch.from_numpy(wl.x).to(dev).to(torch.bfloat16))
+    pk = bgq.pack_w4_groupwise(torch.from_numpy(wl.w).to(dev), group=group, alpha=1024)
+    ref = oracle.linear_intscale(wl.x, wl.w, group=group, alpha=1024, out="f32")
+    assert bgq.load().w4a8_gemm_workspace_size(M, N, K, group, 1) == 0  # no scratch memory on this path
+    acc = bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], 1024, group=group, out="i32")
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+    for out in ("f32", "f16"):
+        y = bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], 1024, group=group, out=out)
+        _close(y.float().cpu().numpy(), ref["y64"], out)
+    qw, sg = oracle.quantize_groups(wl.w, group)
+    yf_ref = oracle.floatscale(ref["qx"], ref["s_a"], qw, sg, group)
+    for out in ("f32", "f16"):
+        yf = bgq.w4a8_gemm_floatscale(q, s, pk["packed"], pk["s_g"], group=group, out=out)
+        _close(yf.float().cpu().numpy(), yf_ref, out)
+    assert bgq.device_status() == 0
+
+
+@pytest.mark.parametrize("M,x_dtype", [(1, "bf16"), (3, "f32"), (4, "bf16"), (5, "bf16"), (16, "f32")])
+def test_linear_intscale_quantizes_in_the_kernel(M, x_dtype):
+    """Tokens in, outputs out: with M <= 4 one kernel quantizes the tokens
+    itself (codes and scales bit-exact); with more tokens the entry point
+    chains the quantizer and the GEMM."""
+    dev = torch.device("cuda:0")
+    K, N = 4096, 1032
+    wl = workloads.make_linear(M, K, N, x_dtype=x_dtype, seed=90 + M)
+    x = torch.from_numpy(wl.x).to(dev)
+    if x_dtype == "bf16":
+        x = x.to(torch.bfloat16)
+    pk = bgq.pack_w4_groupwise(torch.from_numpy(wl.w).to(dev), group=128, alpha=1024)
+    ref = oracle.linear_intscale(wl.x, wl.w, group=128, alpha=1024, out="f32")
+    q = torch.full((M, K), 99, dtype=torch.int8, device=dev)
+    s = torch.full((M,), -1.0, dtype=torch.float32, device=dev)
+    acc = bgq.w4a8_linear_intscale(x, pk["packed"], pk["S"], 1024, out="i32", q_x=q, s_a=s)
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), ref["qx"])
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), ref["s_a"].view(np.uint32))
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+    y = bgq.w4a8_linear_intscale(x, pk["packed"], pk["S"], 1024, out="f16")
+    _close(y.float().cpu().numpy(), ref["y64"], "f16")
+    assert bgq.device_status() == 0
+
+
+def test_linear_intscale_special_rows():
+    """A zero row (scale 0, codes 0, output 0) beside ordinary rows, fused."""
+    dev = torch.device("cuda:0")
+    wl = workloads.make_linear(3, 1024, 256, x_dtype="f32", seed=5)
+    wl.x[1] = 0.0
+    pk = bgq.pack_w4_groupwise(torch.from_numpy(wl.w).to(dev), group=128, alpha=1024)
+    ref = oracle.linear_intscale(wl.x, wl.w, group=128, alpha=1024, out="f32")
+    acc = bgq.w4a8_linear_intscale(torch.from_numpy(wl.x).to(dev), pk["packed"], pk["S"], 1024, out="i32")
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+    assert not acc[1].any()

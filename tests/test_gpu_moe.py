@@ -1,6 +1,7 @@
-"""Mixture-of-experts path on the GPU against the oracle: routed-row gather and
-one integer-scale GEMM per expert with a shared amplifier (the Integer Scale
-summary's Mixtral results)."""
+"""Mixture-of-experts path on the GPU against the oracle: one grouped call
+(device routing offsets and pointer arrays) runs every expert's integer-scale
+GEMM over its routed rows with a shared amplifier (the Integer Scale summary's
+Mixtral results)."""
 import numpy as np
 import pytest
 import torch
@@ -20,6 +21,13 @@ def _close(y, y_ref, out):
     assert np.all(err <= rtol * np.maximum(np.abs(ref), tau))
 
 
+def _grouped(q, s, ri, off, pk, alpha, out, **kw):
+    dev = q.device
+    return bgq.w4a8_gemm_intscale_grouped(q, s, torch.from_numpy(np.asarray(ri, np.int32)).to(dev),
+                                          torch.from_numpy(np.asarray(off, np.int64)).to(dev), pk["packed"], pk["S"],
+                                          alpha, out=out, **kw)
+
+
 def _run(wl, E, alpha, out="i32", route=None):
     dev = torch.device("cuda:0")
     route = wl.experts if route is None else route
@@ -27,13 +35,13 @@ def _run(wl, E, alpha, out="i32", route=None):
     x = torch.from_numpy(wl.x).to(dev).to(torch.bfloat16)
     q, s = bgq.quantize_act_per_token(x)
     pk = bgq.pack_moe_experts([torch.from_numpy(w).to(dev) for w in wl.w], alpha=alpha)
-    y = bgq.w4a8_moe_gemm_intscale(q, s, torch.from_numpy(ri).to(dev), off, pk["packed"], pk["S"], pk["alpha"],
-                                   out=out)
+    y = _grouped(q, s, ri, off, pk, pk["alpha"], out)
     torch.cuda.synchronize()
     return ri, off, pk, y
 
 
-@pytest.mark.parametrize("T,K,N,E,topk", [(64, 512, 256, 4, 2), (37, 256, 136, 8, 2), (200, 1024, 520, 3, 1)])
+@pytest.mark.parametrize("T,K,N,E,topk", [(64, 512, 256, 4, 2), (37, 256, 136, 8, 2), (200, 1024, 520, 3, 1),
+                                          (700, 512, 384, 2, 1)])
 @pytest.mark.parametrize("alpha", [1024, None])
 def test_moe_parity(T, K, N, E, topk, alpha):
     wl = workloads.make_moe(T, K, N, E, topk=topk, seed=T + E)
@@ -61,9 +69,32 @@ def test_moe_empty_experts_and_single_expert():
     dev = torch.device("cuda:0")
     q = torch.zeros((4, 512), dtype=torch.int8, device=dev)
     s = torch.ones((4,), dtype=torch.float32, device=dev)
-    y = bgq.w4a8_moe_gemm_intscale(q, s, torch.zeros((0,), dtype=torch.int32, device=dev), [0, 0, 0],
-                                   [None, None], [None, None], 1024, N=256)
+    y = bgq.w4a8_gemm_intscale_grouped(q, s, torch.zeros((0,), dtype=torch.int32, device=dev),
+                                       torch.zeros((3,), dtype=torch.int64, device=dev), [None, None], [None, None],
+                                       1024, N=256)
     assert y.shape == (0, 256)
+
+
+def test_moe_output_rows_in_token_slot_order():
+    """out_row = token * top_k + slot returns every token's top-k outputs
+    side by side ([T, top_k, N]) with no gather or permute afterwards."""
+    T, K, N, E, topk = 150, 512, 256, 5, 2
+    wl = workloads.make_moe(T, K, N, E, topk=topk, seed=12)
+    ri, off = workloads.route_rows(wl.experts, E)
+    # the slot of each routed row: position of its expert in the token's routing
+    exp_of_row = np.repeat(np.arange(E), np.diff(off))
+    slot = np.array([int(np.nonzero(wl.experts[t] == e)[0][0]) for t, e in zip(ri, exp_of_row)])
+    out_row = (ri.astype(np.int64) * topk + slot).astype(np.int32)
+    dev = torch.device("cuda:0")
+    q, s = bgq.quantize_act_per_token(torch.from_numpy(wl.x).to(dev).to(torch.bfloat16))
+    pk = bgq.pack_moe_experts([torch.from_numpy(w).to(dev) for w in wl.w], alpha=1024)
+    y = _grouped(q, s, ri, off, pk, 1024, "i32", out_row=torch.from_numpy(out_row).to(dev), y_rows=T * topk)
+    torch.cuda.synchronize()
+    ref = oracle.moe_intscale(wl.x, wl.w, ri, off, alpha=1024)
+    want = np.zeros((T * topk, N), np.int64)
+    want[out_row] = ref["acc"]
+    assert np.array_equal(y.cpu().numpy().astype(np.int64), want)
+    assert bgq.device_status() == 0
 
 
 def test_moe_out_of_range_token_index_is_reported():
@@ -78,8 +109,7 @@ def test_moe_out_of_range_token_index_is_reported():
     q, s = bgq.quantize_act_per_token(x)
     pk = bgq.pack_moe_experts([torch.from_numpy(w).to(dev) for w in wl.w], alpha=1024)
     bgq.device_status(clear=True)
-    acc = bgq.w4a8_moe_gemm_intscale(q, s, torch.from_numpy(ri_bad).to(dev), off, pk["packed"], pk["S"], 1024,
-                                     out="i32")
+    acc = _grouped(q, s, ri_bad, off, pk, 1024, "i32")
     torch.cuda.synchronize()
     assert bgq.device_status(clear=True) == 1
     ref = oracle.moe_intscale(wl.x, wl.w, ri, off, alpha=1024)
@@ -123,9 +153,8 @@ def test_moe_mixtral_full_layer_sampled():
     x = torch.from_numpy(wl.x).to(dev).to(torch.bfloat16)
     q, s = bgq.quantize_act_per_token(x)
     pk = bgq.pack_moe_experts([torch.from_numpy(w).to(dev) for w in wl.w], alpha=None)
-    ri_d = torch.from_numpy(ri).to(dev)
-    acc = bgq.w4a8_moe_gemm_intscale(q, s, ri_d, off, pk["packed"], pk["S"], pk["alpha"], out="i32")
-    y = bgq.w4a8_moe_gemm_intscale(q, s, ri_d, off, pk["packed"], pk["S"], pk["alpha"], out="f16")
+    acc = _grouped(q, s, ri, off, pk, pk["alpha"], "i32")
+    y = _grouped(q, s, ri, off, pk, pk["alpha"], "f16")
     torch.cuda.synchronize()
     assert bgq.device_status() == 0
 
