@@ -405,6 +405,80 @@ def measure_decode(dev, rank, world, hbm_peak, reps=7):
     return row
 
 
+FUSED = dict(K=4096, N=[22016, 4096], M=[1, 4])
+
+
+def measure_fused(dev, rank, world, hbm_peak, reps=7):
+    """Decode with the quantize step fused into the layer's kernel
+    (w4a8_linear_intscale: bf16 tokens in, fp16 outputs out, one launch)
+    against the two-launch pair (quantize_act_per_token, then
+    w4a8_gemm_intscale), per layer, from graphs of back-to-back layers that
+    rotate over enough packed weight copies (>= 300 MB) to stream every layer's
+    weights from HBM.  Inputs drawn on the device as in measure_decode."""
+    import torch
+
+    import bit_gemm_quantize_b200 as bgq
+
+    K = FUSED["K"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(8000 + rank)
+    stream = torch.cuda.current_stream(dev)
+    row = {}
+    for N in FUSED["N"]:
+        w = torch.randn((K, N), generator=g, device=dev)
+        w.mul_(0.02)
+        pk = bgq.pack_w4_groupwise(w, group=GROUP, alpha=ALPHA)
+        del w
+        R = max(6, int((300 << 20) // (N * K // 2)) + 1)
+        copies = [pk["packed"]] + [pk["packed"].clone() for _ in range(R - 1)]
+
+        def per_layer_ms(call):
+            for i in range(3):
+                call(i)
+            torch.cuda.synchronize(dev)
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                for i in range(R):
+                    call(i)
+            gr.replay()
+            ts = []
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                gr.replay()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                ts.append(e0.elapsed_time(e1) / R)
+            del gr
+            return max_over_ranks([float(np.median(ts))], world, dev)[0]
+
+        for M in FUSED["M"]:
+            x = torch.randn((M, K), generator=g, device=dev)
+            cols = torch.randperm(K, generator=g, device=dev)[: max(1, K // 200)]
+            x[:, cols] *= 30.0
+            x = x.to(torch.bfloat16)
+            q = torch.empty((M, K), dtype=torch.int8, device=dev)
+            s = torch.empty((M,), dtype=torch.float32, device=dev)
+            y = torch.empty((M, N), dtype=torch.float16, device=dev)
+            ws = bgq.gemm_workspace(M, N, K, GROUP, 0, dev)
+
+            def pair(i):
+                bgq.quantize_act_per_token(x, q, s)
+                bgq.w4a8_gemm_intscale(q, s, copies[i], pk["S"], ALPHA, group=GROUP, out="f16", y=y, workspace=ws)
+
+            t_f = per_layer_ms(lambda i: bgq.w4a8_linear_intscale(x, copies[i], pk["S"], ALPHA, group=GROUP,
+                                                                  out="f16", y=y, workspace=ws))
+            t_p = per_layer_ms(pair)
+            b = N * K // 2 + 2 * (K // GROUP) * N + 2 * M * K + 2 * M * N
+            row[f"fused_us_n{N}_M{M}"] = round(t_f * 1e3, 2)
+            row[f"pair_us_n{N}_M{M}"] = round(t_p * 1e3, 2)
+            row[f"fused_frac_hbm_n{N}_M{M}"] = round(b / (t_f * 1e-3) / 1e9 / hbm_peak, 4)
+        del copies
+    row["workload"] = "decode_fused_quantize_k4096"
+    row["timing"] = "CUDA events over graphs of back-to-back layers rotating >= 300 MB of weight copies; median of 7"
+    return row
+
+
 # ---------------------------------------------------------------- mixture of experts
 
 MOE = dict(tokens=2048, K=4096, N=14336, experts=8, topk=2)
@@ -943,6 +1017,7 @@ def run_ours(args):
     roof["frac_of_derived_int8"] = (roof["achieved"] / int8_derived) if roof["bound"] == "tensor" else None
 
     decode = measure_decode(dev, rank, world, hbm_peak)
+    fused = measure_fused(dev, rank, world, hbm_peak)
     moe = measure_moe(dev, rank, world, int8_peak)
     prefill = measure_prefill(dev, rank, world, int8_peak)
     w8a8 = measure_w8a8(dev, rank, world, hbm_peak, int8_peak)
@@ -958,6 +1033,7 @@ def run_ours(args):
         "int8_peak": {"measured_tops": round(int8_peak, 1), "tmem_a_n128_tops": round(probe["ts_n128"], 1),
                       "derived_bf16x2_tops": round(int8_derived, 1)},
         "decode": decode,
+        "fused": fused,
         "moe": moe,
         "prefill": prefill,
         "w8a8": w8a8,

@@ -345,8 +345,9 @@ def w4a8_linear_intscale(x, w_packed, S, alpha: int, *, group: int = 128, out: s
                          workspace: torch.Tensor | None = None):
     """y [M, N] = the integer-scale layer from unquantized tokens x [M, K]
     (fp32 or bf16): per-token quantization and the W4A8 integer-scale GEMM,
-    one kernel when M <= 4.  q_x / s_a receive the token codes and scales when
-    given (allocated here when M > 4, where they are needed)."""
+    one kernel when M <= 4 (and 256 <= K <= 16384).  q_x / s_a receive the
+    token codes and scales when given (allocated here otherwise, where the
+    quantizer and the GEMM run as two kernels)."""
     _need_cuda("x", x, ndim=2)
     if x.dtype == torch.float32:
         dt_x = F32
@@ -364,9 +365,10 @@ def w4a8_linear_intscale(x, w_packed, S, alpha: int, *, group: int = 128, out: s
     if y is None:
         y = torch.empty((M, N), dtype=tdt, device=x.device)
     _need_cuda("y", y, tdt, 2)
-    if M > 4 and q_x is None:
+    two_kernels = M > 4 or K < 256 or K > 16384
+    if two_kernels and q_x is None:
         q_x = torch.empty((M, K), dtype=torch.int8, device=x.device)
-    if M > 4 and s_a is None:
+    if two_kernels and s_a is None:
         s_a = torch.empty((M,), dtype=torch.float32, device=x.device)
     if workspace is None:
         workspace = gemm_workspace(M, N, K, group, 0, x.device)

@@ -152,9 +152,24 @@ w4a8_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int32_t group) {
     return W4A8_OK;
 }
 
-// Decode-shaped calls (a few tokens) run on the CUDA cores (gemv_w4a8.cu).
-bool gemv_path(int64_t M, int64_t K, bool w8, bool zp) {
-    return !w8 && !zp && M >= 1 && M <= w4a8::gemv::kMaxM && K <= w4a8::gemv::kMaxK;
+// Decode-shaped calls (a few tokens) run on the CUDA cores (gemv_w4a8.cu):
+// one or two tokens always; three or four while the packed weights take at
+// most 32 MB (measured: past that the tensor-core tiles, which do a quarter of
+// the instructions per weight byte, are faster at four tokens).
+bool gemv_fits(int64_t M, int64_t K, bool w8, bool zp) {
+    return !w8 && !zp && M >= 1 && M <= w4a8::gemv::kMaxM && K >= w4a8::gemv::kMinK && K <= w4a8::gemv::kMaxK;
+}
+bool gemv_path(int64_t M, int64_t N, int64_t K, bool w8, bool zp) {
+    return gemv_fits(M, K, w8, zp) && (M <= 2 || N * (K / 2) <= (int64_t(32) << 20));
+}
+
+// The decode kernel's weight map for M tokens: [N][K/2] bytes, boxes of 32 rows
+// x box_bytes(M) (one or two 128-wide K blocks of 32 columns), swizzled by the
+// box width.
+bool gemv_weight_map(CUtensorMap* m, const uint8_t* w_packed, int64_t N, int64_t K, int64_t M) {
+    const int box = w4a8::gemv::box_bytes(int(M));
+    return make_map_u8(m, w_packed, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), uint32_t(box), 32,
+                       box == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_t* w_packed, const int16_t* S,
@@ -179,7 +194,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
 
     DeviceInfo dev;
     if ((st = current_device(dev)) != W4A8_OK) return st;
-    if (gemv_path(M, K, w8, zp)) {
+    if (gemv_path(M, N, K, w8, zp)) {
         // decode-shaped: the CUDA-core kernel, no workspace
         w4a8::gemv::GemvParams g{};
         g.x = q_x;
@@ -196,7 +211,12 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
         g.G = int32_t(K / group);
         g.group = group;
         g.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
-        W4A8_CUDA_TRY(w4a8::gemv::launch(g, path, w4a8::gemv::kXCodes, dev.sms, static_cast<cudaStream_t>(stream)));
+        g.status = dev.status;
+        g.wait_limit = g_wait_limit.load();
+        CUtensorMap tm;
+        if (!gemv_weight_map(&tm, w_packed, N, K, M)) return W4A8_ERR_CUDA;
+        W4A8_CUDA_TRY(
+            w4a8::gemv::launch(tm, g, path, w4a8::gemv::kXCodes, dev.sms, static_cast<cudaStream_t>(stream)));
         return W4A8_OK;
     }
     const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms, w8, zp);
@@ -211,9 +231,9 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     }
 
     if (pl.wide) {
-        // token tiles of 256 / 192: packed weights one K block (64 B) per box, no
+        // wide token tiles: packed weights one K block (64 B) per box, no
         // swizzle; token codes BT rows x 128 B, 128-byte swizzle; output boxes of
-        // BT rows (fp16) or 64 rows (4-byte outputs)
+        // BT rows (fp16) or one worker group's rows (4-byte outputs)
         CUtensorMap tm_w, tm_x, tm_y;
         if (!make_map_u8(&tm_w, w_packed, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 64, 128,
                          CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -226,7 +246,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
                                           : (y_dtype == W4A8_I32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
                                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
         if (!make_map_2d(&tm_y, t, y, uint64_t(N), uint64_t(M), uint64_t(N) * (f16 ? 2u : 4u), 128,
-                         f16 ? uint32_t(pl.BT) : 64u, CU_TENSOR_MAP_SWIZZLE_NONE))
+                         f16 ? uint32_t(pl.BT) : uint32_t(w4a8::gemm::wide_tail_rows()), CU_TENSOR_MAP_SWIZZLE_NONE))
             return W4A8_ERR_CUDA;
         w4a8::gemm::WideParams q{};
         q.s_a = s_a;
@@ -508,7 +528,7 @@ int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group,
     DeviceInfo dev;
     if (current_device(dev) != W4A8_OK) return -1;
     const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms, path == 2);
-    if (gemv_path(M, K, path == 2, false)) {  // no workspace; the asymmetric GEMM (path 0) runs tiles
+    if (gemv_path(M, N, K, path == 2, false)) {  // no workspace; the asymmetric GEMM (path 0) runs tiles
         if (path != 0) return 0;
         const w4a8::gemm::Plan pn = w4a8::gemm::make_plan(M, N, K, group, dev.sms, false, true);
         return plan_splits_tiles(pn) ? pn.ws_bytes : 0;
@@ -574,7 +594,7 @@ w4a8_status w4a8_linear_intscale(const void* x, int32_t x_dtype, int64_t M, int6
     if (!aligned16(x) || (ldx * esz) % 16 != 0 || !aligned16(w_packed) || !aligned16(S) || !aligned16(y))
         return W4A8_ERR_ALIGN;
     if ((q_x && !aligned16(q_x)) || (s_a && !aligned4(s_a))) return W4A8_ERR_ALIGN;
-    if (!gemv_path(M, K, false, false)) {
+    if (!gemv_fits(M, K, false, false)) {
         // more tokens: quantize into the caller's buffers, then the GEMM
         if (!q_x || !s_a) return W4A8_ERR_INVALID_ARG;
         if (!aligned16(s_a)) return W4A8_ERR_ALIGN;
@@ -601,7 +621,11 @@ w4a8_status w4a8_linear_intscale(const void* x, int32_t x_dtype, int64_t M, int6
     g.inv_alpha = std::ldexp(1.0f, -int(std::log2(double(alpha))));
     g.q_out = q_x;
     g.s_out = s_a;
-    W4A8_CUDA_TRY(w4a8::gemv::launch(g, w4a8::gemm::kIntScale,
+    g.status = dev.status;
+    g.wait_limit = g_wait_limit.load();
+    CUtensorMap tm;
+    if (!gemv_weight_map(&tm, w_packed, N, K, M)) return W4A8_ERR_CUDA;
+    W4A8_CUDA_TRY(w4a8::gemv::launch(tm, g, w4a8::gemm::kIntScale,
                                      x_dtype == W4A8_BF16 ? w4a8::gemv::kXBf16 : w4a8::gemv::kXF32, dev.sms,
                                      static_cast<cudaStream_t>(stream)));
     return W4A8_OK;

@@ -1017,8 +1017,10 @@ static int token_tile_for(int64_t M) {
 
 Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool w8, bool narrow_only) {
     Plan pl{};
-    // more tokens than one 128-token tile: the wide-tile kernel (gemm_wide.cu)
-    pl.wide = !w8 && !narrow_only && M > 128;
+    // dense GEMMs run the tiles of this kernel at every M (measured faster
+    // than the wide-tile kernel, which serves the grouped expert call)
+    (void)narrow_only;
+    pl.wide = false;
     pl.BT = pl.wide ? wide_token_tile() : token_tile_for(M);
     pl.n_tiles = (N + kTileN - 1) / kTileN;
     pl.m_tiles = (M + pl.BT - 1) / pl.BT;

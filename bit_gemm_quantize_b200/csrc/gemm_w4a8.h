@@ -72,9 +72,18 @@ struct WideParams {
 
 namespace gemv {
 // Decode-shaped layers on the CUDA cores (gemv_w4a8.cu): M <= 4 tokens,
-// K <= kMaxK, one CTA per 32 output columns.
+// K <= kMaxK, one CTA per 32 output columns, K split over its warps.
 constexpr int kMaxM = 4;
+constexpr int kMinK = 256;
 constexpr int kMaxK = 16384;
+#ifndef W4A8_GEMV_BOX_M4
+#define W4A8_GEMV_BOX_M4 64
+#endif
+// The weight box of the kernel for M tokens: box_bytes(M) x 32 rows (two
+// 128-wide K blocks per box for one or two tokens; for three or four, where
+// the kernel does four times the arithmetic per byte, the smaller box lets
+// more warps share the SM).
+constexpr int box_bytes(int M) { return M <= 2 ? 128 : W4A8_GEMV_BOX_M4; }
 enum XKind { kXCodes = 0, kXBf16 = 1, kXF32 = 2 };
 
 struct GemvParams {
@@ -90,10 +99,15 @@ struct GemvParams {
     float inv_alpha;       // 1 / alpha (integer-scale path)
     int8_t* q_out;         // optional: the codes the kernel computed [M][K] (fused tokens)
     float* s_out;          // optional: their scales [M]
+    int* status;           // device status word (a ring wait that runs out)
+    long long wait_limit;  // SM cycles a ring wait may last
+    int32_t stages;        // ring slots per warp (set by the launcher)
 };
 
-int smem_bytes(int mt, int K, int ks);
-cudaError_t launch(const GemvParams& p, int path, int x_kind, int num_sms, cudaStream_t stream);
+int smem_bytes(int mt, int K, int ks, int stages, int sub);
+// tm_w: packed weights [N][K/2] u8, box box_bytes(M) x 32 rows, swizzled by the box width
+cudaError_t launch(const CUtensorMap& tm_w, const GemvParams& p, int path, int x_kind, int num_sms,
+                   cudaStream_t stream);
 }  // namespace gemv
 
 namespace gemm {
@@ -126,7 +140,7 @@ cudaError_t launch_zp(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CU
 // Wide-tile kernel (token tiles of 256, gemm_wide.cu), integer- or float-scale path.
 // tm_w: packed weights [N][K/2] u8, box 64 B x 128 rows, no swizzle
 // tm_x: token codes [M][K] u8, box 128 B x 256 rows, 128-byte swizzle
-// tm_y: output [M][N], box 128 columns x wide_token_tile() rows (fp16) or 64 rows (4-byte outputs)
+// tm_y: output [M][N], box 128 columns x wide_token_tile() rows (fp16) or wide_tail_rows() (4-byte outputs)
 cudaError_t launch_wide(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap& tm_y, const WideParams& p,
                         int path, cudaStream_t stream);
 // Mixture of experts (integer-scale path): a setup kernel builds the schedule
@@ -138,6 +152,7 @@ cudaError_t launch_wide_moe(const CUtensorMap& tm_w_template, const CUtensorMap&
                             const void* const* w_ptrs, int64_t R, const WideParams& p, int32_t* sched,
                             CUtensorMap* maps, cudaStream_t stream);
 int wide_token_tile();
+int wide_tail_rows();  // output rows per tail pass of 4-byte outputs
 
 int token_tile_rows();
 

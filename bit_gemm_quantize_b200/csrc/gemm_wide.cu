@@ -58,10 +58,13 @@ namespace wide {
 #endif
 constexpr int kTileN = 128;                       // weight columns per tile (MMA M)
 constexpr int kBT = W4A8_WIDE_BT;                 // tokens per tile (MMA N): 192 or 256
-constexpr int kWorkers = kBT / 16;                // warps 2.., one per 32 lanes x 64 token columns
+#ifndef W4A8_WIDE_WORKERS
+#define W4A8_WIDE_WORKERS 12
+#endif
+constexpr int kWorkers = W4A8_WIDE_WORKERS;       // warps 2.., each 32 lanes x kHC token columns
 constexpr int kWorkerThreads = 32 * kWorkers;
 constexpr int kThreads = 32 * (2 + kWorkers);
-constexpr int kHC = kBT / (kWorkers / 4);         // accumulator columns per worker thread (64)
+constexpr int kHC = kBT / (kWorkers / 4);         // accumulator columns per worker thread
 #ifndef W4A8_WIDE_DRAIN_COLS
 #define W4A8_WIDE_DRAIN_COLS 16
 #endif
@@ -70,7 +73,7 @@ constexpr int SW = 4, SA = 2, SX = (kBT == 256 ? 3 : 4), SD = 8, kAcc = 2;
 constexpr int kWBytes = kTileN * 64;              // packed weights of one K block
 constexpr int kABytes = kTileN * 128;             // unpacked operand of one K block
 constexpr int kXBytes = kBT * 128;                // token codes of one K block
-constexpr int kYBytes = kBT * kTileN * 2;         // output staging: all rows as fp16, or 64 rows of 4-byte words
+constexpr int kYBytes = kBT * kTileN * 2;         // output staging: all rows as fp16, or kHC rows of 4-byte words
 constexpr int offW = 0;
 constexpr int offA = offW + SW * kWBytes;
 constexpr int offX = offA + SA * kABytes;
@@ -83,7 +86,7 @@ constexpr int offMisc = offBar + kBars * 8;
 constexpr int kSmemBytes = offMisc + 64 + 1024;  // + slack to align the base to 1024
 static_assert(offA % 1024 == 0 && offX % 1024 == 0 && offY % 1024 == 0, "swizzle atoms and TMA sources");
 static_assert(kSmemBytes <= 232448, "shared memory");
-static_assert(kHC == 64 && kTileN * kHC * 4 <= kYBytes, "output staging");
+static_assert(kHC % 16 == 0 && kBT % kHC == 0 && kTileN * kHC * 4 <= kYBytes, "output staging");
 static_assert(2 * kBT <= 512 && kWorkers % 4 == 0, "TMEM: two accumulator buffers of kBT columns");
 
 // Step range of CTA b from the (W, w_q, w_r) of the call: [start(b),
@@ -660,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             epi_bar_sync(kWorkerThreads);
             const int esz = p.y_dtype == kOutF16 ? 2 : 4;
-            const int rows = esz == 2 ? kBT : kHC;  // rows per pass: all, or one worker group's 64
+            const int rows = esz == 2 ? kBT : kHC;  // rows per pass: all, or one worker group's kHC
             const int passes = kBT / rows;
             for (int pass = 0; pass < passes; ++pass) {
                 const int tok0 = pass * rows;  // first token of this pass
@@ -848,6 +851,8 @@ cudaError_t launch_wide_moe(const CUtensorMap& tm_w_template, const CUtensorMap&
 }
 
 int wide_token_tile() { return wide::kBT; }
+
+int wide_tail_rows() { return wide::kHC; }
 
 }  // namespace gemm
 }  // namespace w4a8

@@ -10,13 +10,18 @@
 // and §3.2 / Fig. 3(b) (the float-scale comparison path); "Quantization"
 // notes, Symmetric Quantization (the token codes).
 //
-// Layout: a CTA owns 32 consecutive output columns n (lane = column) and
-// splits K over its warps.  Every lane streams its column's packed weights,
-// 64 bytes (one group of 128 K) at a time with four 16-byte loads; the int4
-// codes become 16 * q in int8 lanes (three integer ops per 8 weights) and
-// dp4a multiplies them with the token codes, which sit in shared memory and
-// are read by all lanes at once (broadcast).  Per group and token:
-//   P_g = (sum of dp4a) >> 4            (exact: every product is 16 q x)
+// Layout: a CTA owns 32 consecutive output columns (lane = column) and splits
+// K over its warps.  Each warp streams its share of the 32 columns with TMA:
+// one box of 32 rows x 128 bytes (two 128-wide K blocks of every column) per
+// stage into a ring of shared-memory slots (128-byte swizzle, so the lanes'
+// 16-byte reads of their own rows are conflict-free); the rings fill the
+// SMs' shared memory, which is what keeps enough bytes in flight.
+// A lane unpacks its column's int4 codes to 16 * q in int8 lanes (three
+// integer ops per 8 weights) and dp4a multiplies them with the token codes,
+// kept in shared memory and read by all lanes at once (broadcast).  Per
+// 128-wide K block and token:
+//   P = (sum of dp4a) >> 4              (exact: every product is 16 q x)
+// and per group, after its last block:
 //   acc += S[g,n] * P_g                 (integer scale: one IMAD)
 //   accf += s_g[g,n] * float(P_g)       (float scale: one I2F and one FMA)
 // The warps' partial sums are added in a fixed order through shared memory,
@@ -41,31 +46,82 @@
 namespace w4a8 {
 namespace gemv {
 
-constexpr int kCols = 32;  // output columns per CTA (one per lane)
+#ifndef W4A8_GEMV_INTERLEAVE
+#define W4A8_GEMV_INTERLEAVE 1
+#endif
 
-// Shared memory of a CTA: the token codes [mt][K], their output scales, and
-// the warps' partial sums [ks][mt][32].
-int smem_bytes(int mt, int K, int ks) { return mt * K + 16 + ks * mt * kCols * 4; }
+constexpr int kCols = 32;              // output columns per CTA (one per lane)
+// A stage is SUB 128-wide K blocks of the CTA's 32 columns: one box of 32 rows
+// x 64 SUB bytes, 64 SUB * 32 bytes of shared memory.
+constexpr int stage_bytes(int sub) { return kCols * 64 * sub; }
+constexpr int kMaxStages = 16;
+constexpr int kSmemCap = 225 * 1024;  // dynamic shared memory a CTA may take (the rest: static, alignment)
 
-// x: the tokens, either their int8 codes (MT rows used of M) or bf16 / fp32 values
-template <int MT, int PATH, typename XT>
-__global__ void __launch_bounds__(512) gemv_kernel(const GemvParams p) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int K = p.K;
-    int8_t* codes = reinterpret_cast<int8_t*>(smem);                                   // [MT][K]
-    float* scl = reinterpret_cast<float*>(smem + MT * K);                              // [MT] output scales
-    int32_t* red = reinterpret_cast<int32_t*>(smem + MT * K + 16);                     // [ks][MT][32]
-    float* redf = reinterpret_cast<float*>(red);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// Shared memory of a CTA with ks warps and rings of `stages` slots: the token
+// codes [mt][K], the rings [ks][stages][2 KB], one mbarrier per slot, the
+// partial sums [ks][mt][32], the tokens' output scales.
+int smem_bytes(int mt, int K, int ks, int stages, int sub) {
+    return ((mt * K + 1023) / 1024) * 1024 + ks * stages * stage_bytes(sub) + ks * stages * 8 + ks * mt * kCols * 4 +
+           16;
+}
+
+template <int MT, int PATH, typename XT, int kSub>
+__global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p) {
+    constexpr int kStage = stage_bytes(kSub);
+    constexpr int kBoxBytes = 64 * kSub;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int K = p.K, N = p.N;
     const int ks = blockDim.x >> 5;
-    const int nthreads = blockDim.x;
-    if (threadIdx.x == 0) griddep_launch_dependents();
+    const int nst = p.stages;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int8_t* codes = reinterpret_cast<int8_t*>(smem);                                      // [MT][K]
+    uint8_t* rings = smem + ((MT * K + 1023) / 1024) * 1024;                              // [ks][nst][kStage]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(rings + ks * nst * kStage);              // [ks][nst]
+    int32_t* red = reinterpret_cast<int32_t*>(bars + ks * nst);                           // [ks][MT][32]
+    float* redf = reinterpret_cast<float*>(red);
+    float* scl = reinterpret_cast<float*>(red + ks * MT * kCols);                         // [MT]
+    __shared__ float wmax[16];
+    __shared__ int abort_s;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < ks * nst; ++i) mbar_init(&bars[i], 1);
+        abort_s = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tm_w);
+        griddep_launch_dependents();
+    }
+    __syncthreads();  // barriers initialized
+
+    // this warp's stages (kSub K blocks of the CTA's 32 columns each); the
+    // first stages' boxes go out before anything else (packed weights are never
+    // written by a kernel that lets its successor start early)
+    const int n0 = blockIdx.x * kCols;
+    const int kbpg = p.group >> 7;  // 128-wide K blocks per group
+    const int nkbt = K >> 7;
+    const int nstt = (nkbt + kSub - 1) / kSub;  // stages of the whole K
+#if W4A8_GEMV_INTERLEAVE
+    // warp w takes stages w, w + ks, w + 2 ks, ...: at any time the CTA's
+    // warps read neighbouring pieces of each column
+    const int s0 = warp, sstep = ks, nkb = (nstt - warp + ks - 1) / ks;
+#else
+    // warp w takes a contiguous run of stages
+    const int s0 = (warp * nstt) / ks, sstep = 1, nkb = ((warp + 1) * nstt) / ks - s0;
+#endif
+    uint8_t* ring = rings + warp * nst * kStage;
+    uint64_t* wbar = bars + warp * nst;
+    int issued = 0;
+    auto issue = [&](int j, int slot) {  // this warp's stage j (stage s0 + j sstep), into ring slot `slot`
+        issued = j + 1;
+        mbar_arrive_expect_tx_one(&wbar[slot], uint32_t(kStage));
+        tma_load_2d_one(ring + slot * kStage, &tm_w, (s0 + j * sstep) * kBoxBytes, n0, &wbar[slot]);
+    };
+    for (int j = 0; j < nst && j < nkb; ++j) issue(j, j);
     griddep_wait();  // the tokens may be the previous kernel's output, y its input
 
     // ---- the token codes of rows 0..MT-1 (rows past M: zero codes, scale 0)
     constexpr bool kFused = !std::is_same<XT, int8_t>::value;
+    const int nthreads = blockDim.x;
     if constexpr (kFused) {
-        __shared__ float wmax[16];
         for (int m = 0; m < MT; ++m) {
             const bool live = m < p.M;
             const XT* row = reinterpret_cast<const XT*>(p.x) + int64_t(m) * p.ldx;
@@ -117,92 +173,118 @@ __global__ void __launch_bounds__(512) gemv_kernel(const GemvParams p) {
             *reinterpret_cast<uint4*>(codes + m * K + cc * 16) = v;
         }
         if (threadIdx.x < MT) {
-            const float s = threadIdx.x < p.M ? p.s_a[threadIdx.x] : 0.0f;
+            const float s = int(threadIdx.x) < p.M ? p.s_a[threadIdx.x] : 0.0f;
             scl[threadIdx.x] = PATH == gemm::kIntScale ? __fmul_rn(s, p.inv_alpha) : s;
         }
     }
     __syncthreads();
 
-    // ---- this warp's groups of this lane's column
-    const int n = blockIdx.x * kCols + lane;
-    const bool nvalid = n < p.N;
-    const int n_ld = nvalid ? n : 0;  // a column past N reads column 0 (never stored)
-    const int G = p.G;
-    const int gpw = G / ks;           // groups per warp (ks divides G)
-    const int g0 = warp * gpw;
-    const int kbpg = p.group >> 7;    // 128-wide K blocks per group
-    const uint8_t* wrow = p.w + int64_t(n_ld) * (K / 2);
-    int32_t acc[MT];
+    // ---- the stages: lane = column n0 + lane, its row of the box
+    const int n = n0 + lane;
+    const bool nvalid = n < N;
+    const int n_ld = nvalid ? n : 0;  // a column past N: its row of the box reads as zero, its scale as column 0's
+    // 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3) (64-byte
+    // swizzle of 64-byte rows) or c ^ (r & 7) (128-byte swizzle)
+    const int sw = kSub == 1 ? (lane >> 1) & 3 : lane & 7;
+    int32_t acc[MT], pg[MT];
     float accf[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
         acc[m] = 0;
+        pg[m] = 0;
         accf[m] = 0.0f;
     }
-    // loads of the first K block, then one block ahead
-    const int kb0 = g0 * kbpg, kb1 = (g0 + gpw) * kbpg;
-    uint4 cur[4], nxt[4];
+    // the scales of stage jj's K blocks, loaded two stages ahead (0 past the
+    // last block)
+    auto ld_scales = [&](int jj, uint32_t (&sc)[kSub]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) cur[i] = __ldg(reinterpret_cast<const uint4*>(wrow + kb0 * 64) + i);
-    int32_t pg[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) pg[m] = 0;
-    // this column's scales, loaded two groups ahead of their use
-    auto ld_scale = [&](int g) -> uint32_t {
-        if (g >= g0 + gpw) return 0u;
-        const int64_t si = int64_t(g) * p.N + n_ld;
-        if constexpr (PATH == gemm::kIntScale)
-            return uint32_t(int32_t(__ldg(p.S + si)));
-        else
-            return __float_as_uint(__ldg(p.s_g + si));
-    };
-    uint32_t sc0 = ld_scale(g0), sc1 = ld_scale(g0 + 1);
-    int g_cur = g0;
-    for (int kb = kb0; kb < kb1; ++kb) {
-        if (kb + 1 < kb1) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) nxt[i] = __ldg(reinterpret_cast<const uint4*>(wrow + (kb + 1) * 64) + i);
-        }
-        // 128 weights: 16 packed words -> 32 words of four 16 q each, K order
-        uint32_t wq[32];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint2 a = gemm::unpack_int4x8_x16(cur[i].x), b = gemm::unpack_int4x8_x16(cur[i].y);
-            const uint2 c = gemm::unpack_int4x8_x16(cur[i].z), d = gemm::unpack_int4x8_x16(cur[i].w);
-            wq[8 * i + 0] = a.x; wq[8 * i + 1] = a.y; wq[8 * i + 2] = b.x; wq[8 * i + 3] = b.y;
-            wq[8 * i + 4] = c.x; wq[8 * i + 5] = c.y; wq[8 * i + 6] = d.x; wq[8 * i + 7] = d.y;
-        }
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            const uint4* xr = reinterpret_cast<const uint4*>(codes + m * K + kb * 128);
-            int32_t s = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {  // 16 token codes per shared-memory load (all lanes read the same)
-                const uint4 x4 = xr[j];
-                s = __dp4a(int(wq[4 * j + 0]), int(x4.x), s);
-                s = __dp4a(int(wq[4 * j + 1]), int(x4.y), s);
-                s = __dp4a(int(wq[4 * j + 2]), int(x4.z), s);
-                s = __dp4a(int(wq[4 * j + 3]), int(x4.w), s);
+        for (int u = 0; u < kSub; ++u) {
+            const int kb = (s0 + jj * sstep) * kSub + u;
+            sc[u] = 0u;
+            if (jj < nkb && kb < nkbt) {
+                const int64_t si = int64_t(kb / kbpg) * N + n_ld;
+                if constexpr (PATH == gemm::kIntScale)
+                    sc[u] = uint32_t(int32_t(__ldg(p.S + si)));
+                else
+                    sc[u] = __float_as_uint(__ldg(p.s_g + si));
             }
-            pg[m] += s;
         }
-        if ((kb + 1) % kbpg == 0) {  // the group ends: apply its scale
-            const uint32_t sraw = sc0;
-            sc0 = sc1;
-            sc1 = ld_scale(g_cur + 2);
-            ++g_cur;
+    };
+    uint32_t sc0[kSub], sc1[kSub], sc2[kSub];
+    ld_scales(0, sc0);
+    ld_scales(1, sc1);
+    bool ok = true;
+    int j = 0, slot = 0;
+    uint32_t phase = 0;
+    for (; j < nkb; ++j) {
+        if (!mbar_wait_warp(&wbar[slot], phase, &abort_s, p.status, p.wait_limit)) {
+            ok = false;
+            break;
+        }
+        ld_scales(j + 2, sc2);
+        const uint8_t* row = ring + slot * kStage + lane * kBoxBytes;
+        const int kbs = (s0 + j * sstep) * kSub;
+#pragma unroll
+        for (int u = 0; u < kSub; ++u) {
+            const int kb = kbs + u;
+            if (kSub > 1 && kb >= nkbt) break;  // the last stage of a K that is not a whole number of stages
+            // the block's 128 weights of this column as 16 q in int8 lanes,
+            // unpacked once for all tokens
+            uint32_t wq[32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4*>(row + (((4 * u + c) ^ sw) << 4));
+                const uint32_t pk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const uint2 e = gemm::unpack_int4x8_x16(pk[h]);
+                    wq[8 * c + 2 * h] = e.x;
+                    wq[8 * c + 2 * h + 1] = e.y;
+                }
+            }
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
-                const int32_t P = pg[m] >> 4;  // exact: 16 P_g
-                if constexpr (PATH == gemm::kIntScale)
-                    acc[m] += int32_t(sraw) * P;
-                else
-                    accf[m] = __fmaf_rn(__uint_as_float(sraw), __int2float_rn(P), accf[m]);
-                pg[m] = 0;
+                const uint4* xr = reinterpret_cast<const uint4*>(codes + m * K + kb * 128);
+                int32_t t0 = 0, t1 = 0, t2 = 0, t3 = 0;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {  // 16 weights against 16 token codes (one broadcast load)
+                    const uint4 x = xr[c];
+                    t0 = __dp4a(int(wq[4 * c]), int(x.x), t0);
+                    t1 = __dp4a(int(wq[4 * c + 1]), int(x.y), t1);
+                    t2 = __dp4a(int(wq[4 * c + 2]), int(x.z), t2);
+                    t3 = __dp4a(int(wq[4 * c + 3]), int(x.w), t3);
+                }
+                pg[m] += (t0 + t1) + (t2 + t3);
+            }
+            // the group ends, or this warp's run of it: apply the group's
+            // scale to the part summed so far (S times a partial sum is still
+            // exact)
+            if ((kb + 1) % kbpg == 0 || u == kSub - 1 || kb + 1 == nkbt) {
+#pragma unroll
+                for (int m = 0; m < MT; ++m) {
+                    const int32_t P = pg[m] >> 4;  // exact: every product is 16 q x
+                    if constexpr (PATH == gemm::kIntScale)
+                        acc[m] += int32_t(sc0[u]) * P;
+                    else
+                        accf[m] = __fmaf_rn(__uint_as_float(sc0[u]), __int2float_rn(P), accf[m]);
+                    pg[m] = 0;
+                }
             }
         }
+        __syncwarp();  // every lane has used its row of the slot: refill it
+        if (j + nst < nkb) issue(j + nst, slot);
+        if (++slot == nst) {
+            slot = 0;
+            phase ^= 1u;
+        }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
+        for (int u = 0; u < kSub; ++u) {
+            sc0[u] = sc1[u];
+            sc1[u] = sc2[u];
+        }
+    }
+    if (!ok && lane == 0) {  // after a timeout, let the boxes in flight (stages j..issued-1) land
+        for (int jj = j; jj < issued; ++jj) gemm::drain_wait(&wbar[jj % nst], uint32_t((jj / nst) & 1));
     }
 
     // ---- the warps' partial sums, added in warp order, and the output
@@ -214,8 +296,7 @@ __global__ void __launch_bounds__(512) gemv_kernel(const GemvParams p) {
             redf[(warp * MT + m) * kCols + lane] = accf[m];
     }
     __syncthreads();
-    if (warp < MT && warp < p.M && nvalid) {
-        const int m = warp;
+    for (int m = warp; m < MT && m < p.M && nvalid; m += ks) {
         int32_t a = 0;
         float af = 0.0f;
         for (int w = 0; w < ks; ++w) {
@@ -225,7 +306,7 @@ __global__ void __launch_bounds__(512) gemv_kernel(const GemvParams p) {
                 af = __fadd_rn(af, redf[(w * MT + m) * kCols + lane]);
         }
         const float v = __fmul_rn(PATH == gemm::kIntScale ? __int2float_rn(a) : af, scl[m]);
-        const int64_t o = int64_t(m) * p.N + n;
+        const int64_t o = int64_t(m) * N + n;
         if (p.y_dtype == gemm::kOutI32)
             reinterpret_cast<int32_t*>(p.y)[o] = a;
         else if (p.y_dtype == gemm::kOutF16)
@@ -235,50 +316,97 @@ __global__ void __launch_bounds__(512) gemv_kernel(const GemvParams p) {
     }
 }
 
+// The launch shape: enough CTAs per SM that the grid is one wave, the most
+// warps per CTA (the K split: at most 16, at most one per stage, about 24
+// warps per SM) and rings as deep as the shared memory left to each
+// CTA allows.
+template <auto kern>
+static int regs_of() {  // registers a thread of `kern` uses (read once)
+    static const int regs = [] {
+        cudaFuncAttributes a{};
+        return cudaFuncGetAttributes(&a, kern) == cudaSuccess ? a.numRegs : 255;
+    }();
+    return regs;
+}
+
+// CTAs of `threads` threads and `smem` bytes one SM holds at once (SM limits:
+// 2048 threads, 32 CTAs, 64 K registers allocated per warp in units of 256,
+// 228 KB of shared memory with 1 KB reserved per CTA).
+static int resident(int regs, int threads, int smem) {
+    const int warps = threads / 32;
+    const int warp_regs = ((regs * 32 + 255) / 256) * 256;
+    int occ = 2048 / threads;
+    occ = occ < 32 ? occ : 32;
+    const int by_regs = 65536 / (warp_regs * warps);
+    const int by_smem = (228 * 1024) / (smem + 1024);
+    occ = occ < by_regs ? occ : by_regs;
+    return occ < by_smem ? occ : by_smem;
+}
+
+template <auto kern>
+static void shape(const GemvParams& p, int mt, int sub, int num_sms, int& ks, int& stages, int& smem) {
+    const int64_t blocks = (p.N + kCols - 1) / kCols;
+    const int nkb_total = (p.K / 128 + sub - 1) / sub;  // stages of the whole K
+    // CTAs each SM holds: the whole grid at once if the shared memory allows,
+    // else fewer (more waves)
+    for (int per_sm = int((blocks + num_sms - 1) / num_sms);; --per_sm) {
+        ks = 24 / per_sm;
+        ks = ks > 16 ? 16 : (ks < 1 ? 1 : ks);
+        ks = ks > nkb_total ? nkb_total : ks;
+        for (; ks >= 1; --ks) {
+            const int fixed = smem_bytes(mt, p.K, ks, 0, sub) + 1024;  // + alignment slack
+            int cap = (228 * 1024) / per_sm - 2048;               // 1 KB reserved per CTA, 1 KB static
+            cap = cap < kSmemCap ? cap : kSmemCap;
+            const int nkb = (nkb_total + ks - 1) / ks;
+            stages = (cap - fixed) / (ks * (stage_bytes(sub) + 8));
+            stages = stages > kMaxStages ? kMaxStages : stages;
+            stages = stages > nkb ? nkb : stages;
+            if (stages < 2 && stages < nkb) continue;  // a ring needs two slots to overlap
+            smem = smem_bytes(mt, p.K, ks, stages, sub) + 1024;
+            if (resident(regs_of<kern>(), 32 * ks, smem) >= per_sm) return;
+        }
+        if (per_sm == 1) break;
+    }
+    // one warp, one slot (always fits: the token codes take at most 64 KB)
+    ks = 1;
+    stages = 1;
+    smem = smem_bytes(mt, p.K, 1, 1, sub) + 1024;
+}
+
 template <int MT, int PATH, typename XT>
-static cudaError_t launch_t(const GemvParams& p, int ks, cudaStream_t stream) {
-    constexpr auto kern = gemv_kernel<MT, PATH, XT>;
-    const int smem = smem_bytes(MT, p.K, ks);
-    const cudaError_t e = configure_once<kern>(32 * ks, smem_bytes(MT, kMaxK, 16));
+static cudaError_t launch_t(const CUtensorMap& tm_w, const GemvParams& p, int num_sms, cudaStream_t stream) {
+    constexpr int sub = box_bytes(MT) / 64;
+    constexpr auto kern = gemv_kernel<MT, PATH, XT, sub>;
+    cudaError_t e = configure_once<kern>(512, kSmemCap);
     if (e != cudaSuccess) return e;
+    int ks = 1, stages = 1, smem = 0;
+    shape<kern>(p, MT, sub, num_sms, ks, stages, smem);
+    GemvParams q = p;
+    q.stages = stages;
     const unsigned grid = unsigned((p.N + kCols - 1) / kCols);
     const LaunchPdl lc(grid, unsigned(32 * ks), size_t(smem), stream);
-    return cudaLaunchKernelEx(&lc.cfg, kern, p);
+    return cudaLaunchKernelEx(&lc.cfg, kern, tm_w, q);
 }
 
 template <int PATH, typename XT>
-static cudaError_t launch_path(const GemvParams& p, int ks, cudaStream_t stream) {
+static cudaError_t launch_path(const CUtensorMap& tm_w, const GemvParams& p, int num_sms, cudaStream_t stream) {
     switch (p.M) {
-        case 1: return launch_t<1, PATH, XT>(p, ks, stream);
-        case 2: return launch_t<2, PATH, XT>(p, ks, stream);
-        default: return launch_t<4, PATH, XT>(p, ks, stream);
+        case 1: return launch_t<1, PATH, XT>(tm_w, p, num_sms, stream);
+        case 2: return launch_t<2, PATH, XT>(tm_w, p, num_sms, stream);
+        default: return launch_t<4, PATH, XT>(tm_w, p, num_sms, stream);
     }
 }
 
-}  // namespace gemv
-
-namespace gemv {
-
-// Warps per CTA: enough CTAs x warps to keep every SM streaming (about 32
-// warps per SM, each with two 2 KB K blocks of loads in flight), at most 16,
-// and a divisor of the group count.
-int warps_for(int64_t N, int64_t G, int num_sms) {
-    const int64_t blocks = (N + kCols - 1) / kCols;
-    int ks = 1;
-    while (ks < 16 && blocks * ks < int64_t(num_sms) * 32 && G % (2 * ks) == 0) ks *= 2;
-    return ks;
-}
-
-cudaError_t launch(const GemvParams& p, int path, int x_kind, int num_sms, cudaStream_t stream) {
-    const int ks = warps_for(p.N, p.G, num_sms);
+cudaError_t launch(const CUtensorMap& tm_w, const GemvParams& p, int path, int x_kind, int num_sms,
+                   cudaStream_t stream) {
     if (path == gemm::kIntScale) {
-        if (x_kind == kXCodes) return launch_path<gemm::kIntScale, int8_t>(p, ks, stream);
-        if (x_kind == kXBf16) return launch_path<gemm::kIntScale, __nv_bfloat16>(p, ks, stream);
-        return launch_path<gemm::kIntScale, float>(p, ks, stream);
+        if (x_kind == kXCodes) return launch_path<gemm::kIntScale, int8_t>(tm_w, p, num_sms, stream);
+        if (x_kind == kXBf16) return launch_path<gemm::kIntScale, __nv_bfloat16>(tm_w, p, num_sms, stream);
+        return launch_path<gemm::kIntScale, float>(tm_w, p, num_sms, stream);
     }
-    if (x_kind == kXCodes) return launch_path<gemm::kFloatScale, int8_t>(p, ks, stream);
-    if (x_kind == kXBf16) return launch_path<gemm::kFloatScale, __nv_bfloat16>(p, ks, stream);
-    return launch_path<gemm::kFloatScale, float>(p, ks, stream);
+    if (x_kind == kXCodes) return launch_path<gemm::kFloatScale, int8_t>(tm_w, p, num_sms, stream);
+    if (x_kind == kXBf16) return launch_path<gemm::kFloatScale, __nv_bfloat16>(tm_w, p, num_sms, stream);
+    return launch_path<gemm::kFloatScale, float>(tm_w, p, num_sms, stream);
 }
 
 }  // namespace gemv

@@ -91,9 +91,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // Warp-wide form.  Every lane polls (one warp instruction per poll) and the
 // lanes vote, so the warp stays converged, leaves together and a timeout
 // never splits it.  The common case, a phase that has already completed,
-// costs one poll and one vote; the blocking loop is out of line so that it
-// adds neither instructions nor registers to the caller's fast path.
-static __device__ __noinline__ bool mbar_wait_warp_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+// costs one poll and one vote.  (The blocking loop is inlined too: measured
+// faster than a call, which spills the caller's live registers around it.)
+static __device__ __forceinline__ bool mbar_wait_warp_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                                  int* status, long long limit) {
     const long long t0 = clock64();
     const uint32_t hint = wait_hint_ns(limit);

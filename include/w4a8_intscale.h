@@ -217,9 +217,9 @@ W4A8_API int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32
 /*
  * W4A8 GEMM with integer group scales (the Integer-Scale scheme).
  * (Integer Scale summary §4 / Fig. 3(c); "Quantization" notes 矩阵乘法中的量化计算.)
- * Kernels by shape: M <= 4 (and K <= 16384) a CUDA-core kernel that streams the
- * weights (no workspace); M <= 128 the tcgen05 kernel with token tiles of
- * 16..128; larger M the wide-tile tcgen05 kernel (token tiles of 192).
+ * Kernels by shape (256 <= K <= 16384 for the first): M <= 2, or M <= 4 with
+ * at most 32 MB of packed weights, a CUDA-core kernel that streams the weights
+ * (no workspace); otherwise the tcgen05 kernel with token tiles of 16..128.
  *   P_g[m,n] = sum_{k in g} q_x[m,k] q_w[k,n]            (int8 x int4 -> int32, tensor cores)
  *   acc[m,n] = sum_g S[g,n] * P_g[m,n]                    (int32, exact)
  *   y[m,n]   = fl_out(fl32(acc) * fl32(s_a[m] / alpha))   (one conversion per output)
@@ -246,15 +246,15 @@ W4A8_API w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, con
  * quantization, then the W4A8 integer-scale GEMM (Integer Scale summary,
  * Fig. 3(c): int8 tokens, int4 weights, integer group scales, one rescale).
  *   q_x, s_a = quantize_act_per_token(x);  y = w4a8_gemm_intscale(q_x, s_a, ...)
- * With M <= 4 tokens (and K <= 16384) it is one kernel: every CTA quantizes
- * the tokens itself (the same codes and scales, bit for bit, as
- * quantize_act_per_token) and streams its weight columns on the CUDA cores;
- * with more tokens it is the two calls above, chained on `stream`.
+ * With M <= 4 tokens (and 256 <= K <= 16384) it is one kernel:
+ * every CTA quantizes the tokens itself (the same codes and scales, bit for
+ * bit, as quantize_act_per_token) and streams its weight columns on the CUDA
+ * cores; otherwise it is the two calls above, chained on `stream`.
  * x, x_dtype, M, K, ldx   as quantize_act_per_token (W4A8_F32 or W4A8_BF16)
  * w_packed, S, alpha, N, group, y, y_dtype, workspace   as w4a8_gemm_intscale
  * q_x, s_a   device, [M, K] int8 and [M] float32: written with the token codes
- *            and scales when given (may be NULL when M <= 4); required when
- *            M > 4 (W4A8_ERR_INVALID_ARG otherwise), s_a then 16-byte aligned
+ *            and scales when given (may be NULL on the one-kernel path);
+ *            required otherwise (W4A8_ERR_INVALID_ARG), s_a then 16-byte aligned
  * Errors: as quantize_act_per_token and w4a8_gemm_intscale.
  */
 W4A8_API w4a8_status w4a8_linear_intscale(const void* x, int32_t x_dtype, int64_t M, int64_t K, int64_t ldx,

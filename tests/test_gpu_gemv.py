@@ -23,15 +23,25 @@ def _close(y, y_ref, out):
 
 
 CASES = [
-    # M, K, N, group: every token count, ragged N (columns past N in the last CTA),
-    # groups of 128 / 256 / 512 and group = K, a K that splits over 16 warps
+    # M, K, N, group: every token count; ragged N (a CTA's last columns past N
+    # read zero-filled rows); groups of 128 .. 4096 (one to 32 128-wide blocks
+    # per group); K split over 1 .. 16 warps, rings of 1 .. 16 slots; group = K
+    # (per channel); a K that is not a power of two (9 and 86 groups); the
+    # largest K of the path; the FFN gate/up shape
     (1, 4096, 4096, 128),
     (2, 1024, 136, 128),
     (3, 2048, 1032, 256),
     (4, 4096, 520, 128),
-    (1, 512, 256, 512),
-    (4, 8192, 264, 128),
-    (2, 16384, 128, 128),
+    (1, 1024, 256, 512),
+    (2, 8192, 128, 1024),
+    (3, 4096, 264, 2048),
+    (4, 4096, 392, 4096),
+    (4, 1152, 8, 128),
+    (2, 11008, 520, 128),
+    (3, 16384, 136, 512),
+    (1, 16384, 40, 16384),
+    (1, 8192, 22016, 128),
+    (4, 4096, 22016, 128),
 ]
 
 

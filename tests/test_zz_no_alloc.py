@@ -25,10 +25,11 @@ def _inputs(M, K, N, seed):
 
 # token tiles 16, 32 and 64, with stream-K partitions that cut tiles (so the
 # workspace is used; M = 48 takes the 64-token tile, the widest whose plans fit
-# the 8 MiB array), one that cuts none, and a single token (the decode kernel,
-# which needs no workspace at all)
+# the 8 MiB array), one that cuts none, and a single token (the decode kernel
+# needs no workspace; the size reported for it covers the asymmetric-token
+# GEMM, which runs tiles even for one token)
 @pytest.mark.parametrize("M,K,N,cuts", [(8, 4096, 2048, True), (16, 2048, 1024, True), (32, 4096, 2048, True),
-                                        (48, 4096, 2048, True), (16, 128, 256, False), (1, 4096, 2048, False)])
+                                        (48, 4096, 2048, True), (16, 128, 256, False), (1, 4096, 2048, True)])
 @pytest.mark.parametrize("out", ["i32", "f16"])
 def test_static_workspace_matches_caller_workspace(M, K, N, cuts, out):
     need = bgq.load().w4a8_gemm_workspace_size(M, N, K, 128, 0)
