@@ -42,7 +42,7 @@ PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 INT8_PER_BF16 = 2.0
 
 
-CASE_OPS = ["quant", "gemm_is", "gemm_fs", "gemm_w8", "gemm_asym"]
+CASE_OPS = ["quant", "gemm_is", "gemm_fs", "gemm_w8", "gemm_asym", "moe"]
 
 
 def parse():
@@ -75,6 +75,19 @@ def run_case(a):
     import bit_gemm_quantize_b200 as bgq
 
     dev = torch.device("cuda:0")
+    if a.case == "moe":  # the mixture-of-experts layer of the benchmark (routed quantize + grouped call)
+        layer = moe_layer(dev, 3000)[0]["routed"]
+        layer()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(a.reps):
+            layer()
+        e1.record()
+        torch.cuda.synchronize()
+        st = bgq.device_status()
+        print(f"moe: {e0.elapsed_time(e1) / a.reps * 1e3:.2f} us per layer (device status {st})")
+        return 0 if st == 0 else 1
     wl = workloads.make_linear(a.M, a.K, a.N if a.case != "quant" else 8, x_dtype="bf16", seed=7,
                                group=a.group)
     xs = wl.x + 1.0 if a.case == "gemm_asym" else wl.x
@@ -405,7 +418,7 @@ def measure_decode(dev, rank, world, hbm_peak, reps=7):
     return row
 
 
-FUSED = dict(K=4096, N=[22016, 4096], M=[1, 4])
+FUSED = dict(K=4096, N=[22016, 4096], M=[1])
 
 
 def measure_fused(dev, rank, world, hbm_peak, reps=7):
@@ -495,9 +508,54 @@ def measure_moe(dev, rank, world, int8_peak, reps=10):
 
     import bit_gemm_quantize_b200 as bgq
 
+    layers, meta = moe_layer(dev, 3000 + rank)
+    T, K, N, E, topk = MOE["tokens"], MOE["K"], MOE["N"], MOE["experts"], MOE["topk"]
+    R, off, alpha = meta["R"], meta["off"], meta["alpha"]
+    stream = torch.cuda.current_stream(dev)
+
+    def layer_ms(layer):
+        for _ in range(3):
+            layer()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layer()
+        graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        del graph
+        return max_over_ranks([e0.elapsed_time(e1) / reps], world, dev)[0]
+
+    ms = layer_ms(layers["routed"])
+    ms_g = layer_ms(layers["gather"])
+    ops = 2.0 * R * N * K
+    tops = ops / (ms * 1e-3) / 1e12
+    counts = [int(c) for c in np.diff(off)]
+    return {"workload": "moe_mixtral_shaped", "tokens": T, "K": K, "N": N, "experts": E, "topk": topk,
+            "group": GROUP, "alpha": alpha, "rows_per_expert": ",".join(str(c) for c in counts),
+            "us_per_layer": round(ms * 1e3, 2), "tops": round(tops, 2), "frac_int8": round(tops / int8_peak, 4),
+            "us_per_layer_row_gather": round(ms_g * 1e3, 2), "launches_per_layer": 3,
+            "timing": "CUDA events over graph replays of one layer: the tokens quantized in routed order "
+                      "(quantize_act_routed), the grouped setup and one grouped GEMM over all experts reading "
+                      "whole-tile row blocks (device routing offsets); row_gather: tokens quantized once, rows "
+                      "gathered by index inside the GEMM; weights > L2"}
+
+
+def moe_layer(dev, seed):
+    """Inputs of the Mixtral-shaped layer and a closure that runs it once
+    (quantize, then the grouped call over all experts)."""
+    import torch
+
+    import bit_gemm_quantize_b200 as bgq
+
     T, K, N, E, topk = MOE["tokens"], MOE["K"], MOE["N"], MOE["experts"], MOE["topk"]
     g = torch.Generator(device=dev)
-    g.manual_seed(3000 + rank)
+    g.manual_seed(seed)
     ws = []
     for _ in range(E):
         w = torch.randn((K, N), generator=g, device=dev)
@@ -519,37 +577,20 @@ def measure_moe(dev, rank, world, int8_peak, reps=10):
     y = torch.empty((R, N), dtype=torch.float16, device=dev)
     wsp = bgq.grouped_workspace(E, N, K, GROUP, dev)
 
-    def layer():
+    q_r = torch.empty((R, K), dtype=torch.int8, device=dev)
+    s_r = torch.empty((R,), dtype=torch.float32, device=dev)
+
+    def gather():
         bgq.quantize_act_per_token(x, q, s)
         bgq.w4a8_gemm_intscale_grouped(q, s, ri_d, off_d, wp, sp, pk["alpha"], group=GROUP, out="f16", y=y,
                                        workspace=wsp, N=N)
 
-    for _ in range(3):
-        layer()
-    torch.cuda.synchronize(dev)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        layer()
-    graph.replay()
-    stream = torch.cuda.current_stream(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for _ in range(reps):
-        graph.replay()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = max_over_ranks([e0.elapsed_time(e1) / reps], world, dev)[0]
-    del graph
-    ops = 2.0 * R * N * K
-    tops = ops / (ms * 1e-3) / 1e12
-    counts = [int(c) for c in np.diff(off)]
-    return {"workload": "moe_mixtral_shaped", "tokens": T, "K": K, "N": N, "experts": E, "topk": topk,
-            "group": GROUP, "alpha": pk["alpha"], "rows_per_expert": ",".join(str(c) for c in counts),
-            "us_per_layer": round(ms * 1e3, 2), "tops": round(tops, 2), "frac_int8": round(tops / int8_peak, 4),
-            "launches_per_layer": 3,
-            "timing": "CUDA events over graph replays of quantize + grouped setup + one grouped GEMM over all "
-                      "experts (device routing offsets); weights > L2"}
+    def routed():
+        bgq.quantize_act_routed(x, ri_d, q_r, s_r)
+        bgq.w4a8_gemm_intscale_grouped(q_r, s_r, None, off_d, wp, sp, pk["alpha"], group=GROUP, out="f16", y=y,
+                                       workspace=wsp, N=N)
+
+    return {"routed": routed, "gather": gather}, {"R": R, "off": off, "alpha": pk["alpha"]}
 
 
 PREFILL = dict(M=4096, shapes=[(4096, 11008), (11008, 4096)])  # (K, N) of the two layers
@@ -880,10 +921,12 @@ def run_ours(args):
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_push("timed_step")  # lets a profiler select the timed launches alone
     start.record(stream)
     for _ in range(args.steps):
         step_graph.replay()
     stop.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize(dev)
     barrier()
     clocks = sampler.stop()
@@ -1050,18 +1093,26 @@ def run_ours(args):
 
 # DRAM bytes (read + write) per launch of the integer-scale GEMM, from one
 # ncu capture of `bench.py --case gemm_is --M <M>`, valid for the kernel source
-# it was taken with (first 16 hex digits of its SHA-256).
-MEASURED_TRAFFIC = {1024: (56.385536e6 + 19.70176e6, "e11cabb5d4346aad")}
+# it was taken with (first 16 hex digits of the SHA-256 of the files below).
+MEASURED_TRAFFIC = {1024: (56.37504e6 + 19.445248e6, "27ed1dc887d58bcc")}
+GEMM_SOURCES = ("gemm_w4a8.cu", "gemm_w4a8.h", "gemm_common.cuh", "sm100_ptx.cuh")
+
+
+def gemm_source_digest():
+    h = hashlib.sha256()
+    base = os.path.join(os.path.dirname(os.path.abspath(__file__)), "bit_gemm_quantize_b200", "csrc")
+    for name in GEMM_SOURCES:
+        with open(os.path.join(base, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def measured_traffic(M):
     rec = MEASURED_TRAFFIC.get(M)
     if rec is None:
         return None
-    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "bit_gemm_quantize_b200", "csrc", "gemm_w4a8.cu")
     try:
-        with open(src, "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+        digest = gemm_source_digest()
     except OSError:
         return None
     return rec[0] if digest == rec[1] else None

@@ -16,6 +16,7 @@ from ._native import (  # noqa: F401
     pack_w8_groupwise,
     quantize_act_per_token,
     quantize_act_per_token_asym,
+    quantize_act_routed,
     tensor_i8_peak_probe,
     w4_zero_point_term,
     w4a8_amplifier_search,
@@ -40,6 +41,7 @@ __all__ = [
     "pack_w8_groupwise",
     "quantize_act_per_token",
     "quantize_act_per_token_asym",
+    "quantize_act_routed",
     "tensor_i8_peak_probe",
     "w4_zero_point_term",
     "w4a8_amplifier_search",

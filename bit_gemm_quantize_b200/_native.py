@@ -69,6 +69,7 @@ def load(path: str = LIB_PATH):
         sigs = {
             "w4a8_status_string": ([I32_], ctypes.c_char_p),
             "quantize_act_per_token": ([P, I32_, I64, I64, I64, P, P, P], I32_),
+            "quantize_act_routed": ([P, I32_, I64, I64, I64, P, I64, P, P, P], I32_),
             "quantize_act_per_token_asym": ([P, I32_, I64, I64, I64, P, P, P, P], I32_),
             "w4_zero_point_term": ([P, P, I64, I64, I32_, I32_, I64, P, P], I32_),
             "w4a8_static_workspace_reset": ([], I32_),
@@ -197,6 +198,32 @@ def quantize_act_per_token(x: torch.Tensor, q_x: torch.Tensor | None = None, s_a
     code = load().quantize_act_per_token(_ptr(x), dt, M, K, K, _ptr(q_x), _ptr(s_a), _stream(x.device))
     _check("quantize_act_per_token", code)
     return q_x, s_a
+
+
+def quantize_act_routed(x: torch.Tensor, row_index: torch.Tensor, q_r: torch.Tensor | None = None,
+                        s_r: torch.Tensor | None = None):
+    """Per-token int8 codes and scales of x [T, K] in routed order: row i is
+    token row_index[i] ([R] int32 on the device)."""
+    _need_cuda("x", x, ndim=2)
+    if x.dtype == torch.float32:
+        dt = F32
+    elif x.dtype == torch.bfloat16:
+        dt = BF16
+    else:
+        raise ValueError("x must be float32 or bfloat16")
+    _need_cuda("row_index", row_index, torch.int32, 1)
+    T, K = x.shape
+    R = row_index.shape[0]
+    if q_r is None:
+        q_r = torch.empty((R, K), dtype=torch.int8, device=x.device)
+    if s_r is None:
+        s_r = torch.empty((R,), dtype=torch.float32, device=x.device)
+    _need_cuda("q_r", q_r, torch.int8, 2)
+    _need_cuda("s_r", s_r, torch.float32, 1)
+    code = load().quantize_act_routed(_ptr(x), dt, T, K, K, _ptr(row_index), R, _ptr(q_r), _ptr(s_r),
+                                      _stream(x.device))
+    _check("quantize_act_routed", code)
+    return q_r, s_r
 
 
 def w4a8_amplifier_search(scales: torch.Tensor) -> int:
@@ -345,9 +372,9 @@ def w4a8_linear_intscale(x, w_packed, S, alpha: int, *, group: int = 128, out: s
                          workspace: torch.Tensor | None = None):
     """y [M, N] = the integer-scale layer from unquantized tokens x [M, K]
     (fp32 or bf16): per-token quantization and the W4A8 integer-scale GEMM,
-    one kernel when M <= 4 (and 256 <= K <= 16384).  q_x / s_a receive the
-    token codes and scales when given (allocated here otherwise, where the
-    quantizer and the GEMM run as two kernels)."""
+    one kernel for M = 1 (256 <= K <= 16384).  q_x / s_a receive the token
+    codes and scales when given (allocated here where the quantizer and the
+    GEMM run as two kernels)."""
     _need_cuda("x", x, ndim=2)
     if x.dtype == torch.float32:
         dt_x = F32
@@ -365,7 +392,9 @@ def w4a8_linear_intscale(x, w_packed, S, alpha: int, *, group: int = 128, out: s
     if y is None:
         y = torch.empty((M, N), dtype=tdt, device=x.device)
     _need_cuda("y", y, tdt, 2)
-    two_kernels = M > 4 or K < 256 or K > 16384
+    # buffers for the two-kernel route: more than one token (faster as two
+    # kernels from two up), or K outside the decode kernel's range
+    two_kernels = M > 1 or K < 256 or K > 16384
     if two_kernels and q_x is None:
         q_x = torch.empty((M, K), dtype=torch.int8, device=x.device)
     if two_kernels and s_a is None:
@@ -517,7 +546,8 @@ def w4a8_gemm_intscale_grouped(q_x, s_a, row_index, expert_offsets, packed, S, a
                                N: int | None = None):
     """Every expert's integer-scale GEMM over its routed rows in one grouped call.
 
-    row_index [R] int32: the token of each routed row, rows grouped by expert;
+    row_index [R] int32: the token of each routed row, rows grouped by expert,
+    or None when q_x / s_a are the routed rows themselves (quantize_act_routed);
     expert_offsets [E+1] int64 CUDA tensor (device offsets); packed / S: lists
     of per-expert tensors (None for experts without rows) or int64 CUDA
     tensors of device pointers; out_row [R] int32 or None: the output row of
@@ -525,12 +555,13 @@ def w4a8_gemm_intscale_grouped(q_x, s_a, row_index, expert_offsets, packed, S, a
     given (needed when pointers are passed)."""
     _need_cuda("q_x", q_x, torch.int8, 2)
     _need_cuda("s_a", s_a, torch.float32, 1)
-    _need_cuda("row_index", row_index, torch.int32, 1)
+    if row_index is not None:
+        _need_cuda("row_index", row_index, torch.int32, 1)
     _need_cuda("expert_offsets", expert_offsets, torch.int64, 1)
     dev = q_x.device
     E = expert_offsets.numel() - 1
     T, K = q_x.shape
-    R = row_index.numel()
+    R = row_index.numel() if row_index is not None else T
     if isinstance(packed, torch.Tensor):
         wp = packed
     else:

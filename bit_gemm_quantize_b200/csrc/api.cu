@@ -384,6 +384,24 @@ w4a8_status quantize_act_per_token(const void* x, int32_t x_dtype, int64_t M, in
     return W4A8_OK;
 }
 
+w4a8_status quantize_act_routed(const void* x, int32_t x_dtype, int64_t T, int64_t K, int64_t ldx,
+                                const int32_t* row_index, int64_t R, int8_t* q_r, float* s_r, void* stream) {
+    if (x_dtype != W4A8_F32 && x_dtype != W4A8_BF16) return W4A8_ERR_DTYPE;
+    if (R < 0 || T < 0 || K <= 0 || K % 16 != 0 || ldx < K) return W4A8_ERR_SHAPE;
+    if (R == 0) return W4A8_OK;
+    if (T < 1) return W4A8_ERR_SHAPE;
+    if (!x || !row_index || !q_r || !s_r) return W4A8_ERR_INVALID_ARG;
+    const int64_t esz = x_dtype == W4A8_BF16 ? 2 : 4;
+    if (!aligned16(x) || !aligned16(q_r) || (ldx * esz) % 16 != 0) return W4A8_ERR_ALIGN;
+    if (!aligned4(s_r) || !aligned4(row_index)) return W4A8_ERR_ALIGN;
+    DeviceInfo dev;
+    w4a8_status st = current_device(dev);
+    if (st != W4A8_OK) return st;
+    W4A8_CUDA_TRY(w4a8::quant::launch(x, x_dtype == W4A8_BF16, R, K, ldx, q_r, s_r, dev.status,
+                                      static_cast<cudaStream_t>(stream), dev.sms, row_index, T));
+    return W4A8_OK;
+}
+
 w4a8_status quantize_act_per_token_asym(const void* x, int32_t x_dtype, int64_t M, int64_t K, int64_t ldx,
                                         int8_t* q_x, float* s_a, int32_t* z_a, void* stream) {
     if (x_dtype != W4A8_F32 && x_dtype != W4A8_BF16) return W4A8_ERR_DTYPE;
@@ -594,8 +612,13 @@ w4a8_status w4a8_linear_intscale(const void* x, int32_t x_dtype, int64_t M, int6
     if (!aligned16(x) || (ldx * esz) % 16 != 0 || !aligned16(w_packed) || !aligned16(S) || !aligned16(y))
         return W4A8_ERR_ALIGN;
     if ((q_x && !aligned16(q_x)) || (s_a && !aligned4(s_a))) return W4A8_ERR_ALIGN;
-    if (!gemv_fits(M, K, false, false)) {
-        // more tokens: quantize into the caller's buffers, then the GEMM
+    // One kernel for a single token on the decode path, and for up to four
+    // when the caller gave no buffers; otherwise quantize into the caller's
+    // buffers, then the GEMM (measured faster from two tokens up: the
+    // quantizer overlaps the decode kernel's weight prefetch, while the one
+    // kernel quantizes every row again in each CTA).
+    const bool fused = gemv_fits(M, K, false, false) && (!(q_x && s_a) || (M == 1 && gemv_path(M, N, K, false, false)));
+    if (!fused) {
         if (!q_x || !s_a) return W4A8_ERR_INVALID_ARG;
         if (!aligned16(s_a)) return W4A8_ERR_ALIGN;
         st = quantize_act_per_token(x, x_dtype, M, K, ldx, q_x, s_a, stream);
@@ -652,8 +675,10 @@ w4a8_status w4a8_gemm_intscale_grouped(const int8_t* q_x, const float* s_a, int6
     if (!is_pow2(alpha) || alpha > (1 << 30)) return W4A8_ERR_INVALID_ARG;
     if (R == 0) return W4A8_OK;
     if (T == 0 || !out_row && y_rows < R) return W4A8_ERR_SHAPE;
-    if (!q_x || !s_a || !row_index || !expert_offsets || !w_packed || !S || !y) return W4A8_ERR_INVALID_ARG;
-    if (!aligned16(q_x) || !aligned16(y) || !aligned4(s_a) || !aligned4(row_index) || (out_row && !aligned4(out_row)) ||
+    if (!row_index && T < R) return W4A8_ERR_SHAPE;  // the routed rows themselves
+    if (!q_x || !s_a || !expert_offsets || !w_packed || !S || !y) return W4A8_ERR_INVALID_ARG;
+    if (!aligned16(q_x) || !aligned16(y) || !aligned4(s_a) || (row_index && !aligned4(row_index)) ||
+        (out_row && !aligned4(out_row)) ||
         (reinterpret_cast<uintptr_t>(expert_offsets) & 7u) != 0 || (reinterpret_cast<uintptr_t>(w_packed) & 7u) != 0 ||
         (reinterpret_cast<uintptr_t>(S) & 7u) != 0)
         return W4A8_ERR_ALIGN;
@@ -665,13 +690,15 @@ w4a8_status w4a8_gemm_intscale_grouped(const int8_t* q_x, const float* s_a, int6
     uint8_t* ws = static_cast<uint8_t*>(workspace);
 
     // tensor maps: a template for the experts' packed weights (its address
-    // is replaced per expert on the device), and the token codes gathered by
-    // row, four at a time (a box one row high)
+    // is replaced per expert on the device), and the token codes: gathered by
+    // row, four at a time (a box one row high), or, with no row index, whole
+    // tiles of consecutive routed rows
     CUtensorMap tm_w, tm_x;
     if (!make_map_u8(&tm_w, workspace, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
         return W4A8_ERR_CUDA;
-    if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(T), uint64_t(K), 128, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+    const uint32_t x_box_rows = row_index ? 1u : uint32_t(w4a8::gemm::wide_token_tile());
+    if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(T), uint64_t(K), 128, x_box_rows, CU_TENSOR_MAP_SWIZZLE_128B))
         return W4A8_ERR_CUDA;
     w4a8::gemm::WideParams q{};
     q.s_a = s_a;

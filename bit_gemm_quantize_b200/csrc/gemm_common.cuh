@@ -48,8 +48,10 @@ __device__ __forceinline__ void tmem_load(uint32_t taddr, uint32_t (&r)[N]) {
     } else if constexpr (N == 16) {
         tmem_ld16(taddr, r);
     } else {
-        static_assert(N == 32, "columns per load");
-        tmem_ld32(taddr, r);
+        static_assert(N % 32 == 0, "columns per load");
+#pragma unroll
+        for (int i = 0; i < N / 32; ++i)
+            tmem_ld32(taddr + uint32_t(32 * i), *reinterpret_cast<uint32_t(*)[32]>(&r[32 * i]));
     }
 }
 

@@ -57,7 +57,7 @@ struct WideParams {
     float inv_alpha;
     int32_t y_dtype;
     // mixture of experts
-    const int32_t* row_index;      // [R] token of each routed row, rows grouped by expert
+    const int32_t* row_index;      // [R] token of each routed row, rows grouped by expert (NULL: q_x row i)
     const int32_t* out_row;        // [R] output row of each routed row, or null (row i)
     const void* const* moe_scales; // [E] device pointers to each expert's S [G, N]
     const int32_t* moe_sched;      // W, w_q, w_r, status, then mt[E+1], tstart[E+1], rstart[E+1]

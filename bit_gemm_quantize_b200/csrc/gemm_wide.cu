@@ -316,8 +316,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             rw = Ring{};
             griddep_wait();  // the token codes may be the previous kernel's output
         }
-        // token rows of the current tile (MOE: gathered by routed row)
+        // token rows of the current tile (MOE: gathered by routed row, or,
+        // with no row index, the tile's first routed row of q_x)
         int32_t trow[8];
+        int32_t xrow0 = 0;
         WStageIter<MOE> it(p, range, b);
         WStage st;
         bool ok = true;
@@ -332,8 +334,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const Sched sc = sched_of(p);
                     const int32_t r0 = sc.rstart[st.e] + st.m_tile * kBT;
                     const int32_t r1 = sc.rstart[st.e + 1];
+                    xrow0 = r0;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
+                    for (int q = 0; q < 8 && p.row_index; ++q) {
                         // lane l gathers rows 4l..4l+3 and 128+4l..128+4l+3 (those
                         // below kBT); rows past the expert's last take token 0
                         // (never stored)
@@ -362,12 +365,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t* xdst = smem + offX + rx.idx * kXBytes;
             mbar_arrive_expect_tx_one(&full_x[rx.idx], uint32_t(kXBytes));
             if constexpr (MOE) {
-                __syncwarp();
-                tma_gather4(xdst + 4 * lane * 128, &tm_x, st.kb * 128, trow[0], trow[1], trow[2], trow[3],
-                            &full_x[rx.idx]);
-                if (128 + 4 * lane < kBT)
-                    tma_gather4(xdst + (128 + 4 * lane) * 128, &tm_x, st.kb * 128, trow[4], trow[5], trow[6],
-                                trow[7], &full_x[rx.idx]);
+                if (p.row_index) {
+                    __syncwarp();
+                    tma_gather4(xdst + 4 * lane * 128, &tm_x, st.kb * 128, trow[0], trow[1], trow[2], trow[3],
+                                &full_x[rx.idx]);
+                    if (128 + 4 * lane < kBT)
+                        tma_gather4(xdst + (128 + 4 * lane) * 128, &tm_x, st.kb * 128, trow[4], trow[5], trow[6],
+                                    trow[7], &full_x[rx.idx]);
+                } else {
+                    // the routed rows are q_x's rows: one box of the tile's kBT
+                    // rows (rows past the expert's last are never stored; past
+                    // the last row of q_x they read as zero)
+                    tma_load_2d_one(xdst, &tm_x, st.kb * 128, xrow0, &full_x[rx.idx]);
+                }
             } else {
                 tma_load_2d_one(xdst, &tm_x, st.kb * 128, st.m_tile * kBT, &full_x[rx.idx]);
             }
@@ -522,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int32_t tok;
                 bool tok_ok = true;
                 if constexpr (MOE) {
-                    tok = p.row_index[rbase + t];
+                    tok = p.row_index ? p.row_index[rbase + t] : rbase + t;
                     tok_ok = tok >= 0 && tok < p.moe_T;
                     if (!tok_ok) atomicExch(p.status, 1);  // W4A8_ERR_INVALID_ARG: the row's outputs are zero
                 } else {

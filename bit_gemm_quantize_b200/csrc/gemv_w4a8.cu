@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUten
     int32_t* red = reinterpret_cast<int32_t*>(bars + ks * nst);                           // [ks][MT][32]
     float* redf = reinterpret_cast<float*>(red);
     float* scl = reinterpret_cast<float*>(red + ks * MT * kCols);                         // [MT]
-    __shared__ float wmax[16];
+    __shared__ float wmax[16 * MT];
     __shared__ int abort_s;
     if (threadIdx.x == 0) {
         for (int i = 0; i < ks * nst; ++i) mbar_init(&bars[i], 1);
@@ -122,24 +122,32 @@ __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUten
     constexpr bool kFused = !std::is_same<XT, int8_t>::value;
     const int nthreads = blockDim.x;
     if constexpr (kFused) {
+        // every row's absolute maximum at once (all rows' loads in flight),
+        // one block-wide exchange, then every row's codes
+        float a[MT];
+#pragma unroll
         for (int m = 0; m < MT; ++m) {
-            const bool live = m < p.M;
-            const XT* row = reinterpret_cast<const XT*>(p.x) + int64_t(m) * p.ldx;
-            float a = 0.0f;
-            if (live) {
+            a[m] = 0.0f;
+            if (m < p.M) {
+                const XT* row = reinterpret_cast<const XT*>(p.x) + int64_t(m) * p.ldx;
                 for (int c = threadIdx.x; c < K / 16; c += nthreads) {
                     float v[16];
                     quant::load16<XT>(row + c * 16, v);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
+                    for (int i = 0; i < 16; ++i) a[m] = fmaxf(a[m], fabsf(v[i]));
                 }
             }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-            if (lane == 0) wmax[warp] = a;
-            __syncthreads();
+            for (int o = 16; o > 0; o >>= 1) a[m] = fmaxf(a[m], __shfl_xor_sync(0xffffffffu, a[m], o));
+            if (lane == 0) wmax[warp * MT + m] = a[m];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const bool live = m < p.M;
+            const XT* row = reinterpret_cast<const XT*>(p.x) + int64_t(m) * p.ldx;
             float amax = 0.0f;
-            for (int w = 0; w < ks; ++w) amax = fmaxf(amax, wmax[w]);
+            for (int w = 0; w < ks; ++w) amax = fmaxf(amax, wmax[w * MT + m]);
             const float s = (amax == 0.0f) ? 0.0f : __fdiv_rn(amax, 127.0f);
             const bool zero = (s == 0.0f);
             const bool exact_only = s < 1e-30f;
@@ -162,7 +170,6 @@ __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUten
                 scl[m] = PATH == gemm::kIntScale ? __fmul_rn(s, p.inv_alpha) : s;
                 if (live && blockIdx.x == 0 && p.s_out) p.s_out[m] = s;
             }
-            __syncthreads();  // wmax is reused by the next row
         }
     } else {
         const int8_t* q = reinterpret_cast<const int8_t*>(p.x);

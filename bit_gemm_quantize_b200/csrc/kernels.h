@@ -53,8 +53,11 @@ struct LaunchPdl {
 };
 
 namespace quant {
+// rows: NULL (row m of x gives row m of q) or [M] source rows (row m of q is
+// row rows[m] of x, which has T_src rows; a source outside [0, T_src) gives
+// zero codes and scale and sets W4A8_ERR_INVALID_ARG in *status)
 cudaError_t launch(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a,
-                   int* status, cudaStream_t stream, int num_sms);
+                   int* status, cudaStream_t stream, int num_sms, const int32_t* rows = nullptr, int64_t T_src = 0);
 // asymmetric codes in [-128, 127] with a zero point z_a[m] per row
 cudaError_t launch_asym(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a,
                         int32_t* z_a, cudaStream_t stream, int num_sms);

@@ -70,11 +70,27 @@ __device__ __forceinline__ float row_absmax(const T* row, int64_t K, float* red)
     return block_max(a, red);
 }
 
+// Source row of output row `row`: the row itself, or rows[row] when the
+// caller routes rows (then `ok` says whether it lies in [0, T_src); an
+// invalid source reads row 0 and its outputs are zeroed).
+__device__ __forceinline__ int64_t source_row(const int32_t* rows, int64_t row, int64_t T_src, bool& ok) {
+    if (rows == nullptr) {
+        ok = true;
+        return row;
+    }
+    const int64_t t = rows[row];
+    ok = t >= 0 && t < T_src;
+    return ok ? t : 0;
+}
+
+constexpr int kStatusInvalidArg = 1;  // W4A8_ERR_INVALID_ARG
+
 // Row staged in shared memory by a bulk async copy; two buffers.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) quant_rows_staged(const T* __restrict__ x, int64_t M, int64_t K,
                                                               int64_t ldx, int8_t* __restrict__ q,
-                                                              float* __restrict__ s_a, int* status) {
+                                                              float* __restrict__ s_a, int* status,
+                                                              const int32_t* __restrict__ rows, int64_t T_src) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t row_bytes = uint32_t(K * sizeof(T));
     const uint32_t buf_bytes = (row_bytes + 127u) & ~127u;
@@ -96,9 +112,11 @@ __global__ void __launch_bounds__(kThreads) quant_rows_staged(const T* __restric
 
     int64_t row = blockIdx.x;
     bool inflight[2] = {false, false};  // meaningful in thread 0, which issues the copies
+    bool ok_src = true;
     if (threadIdx.x == 0 && row < M) {
+        const int64_t src = source_row(rows, row, T_src, ok_src);
         mbar_arrive_expect_tx(&bars[0], row_bytes);
-        bulk_load(buf[0], x + row * ldx, row_bytes, &bars[0]);
+        bulk_load(buf[0], x + src * ldx, row_bytes, &bars[0]);
         inflight[0] = true;
     }
     uint32_t phase[2] = {0u, 0u};
@@ -106,16 +124,21 @@ __global__ void __launch_bounds__(kThreads) quant_rows_staged(const T* __restric
     for (; row < M; row += gridDim.x) {
         const int64_t next = row + gridDim.x;
         if (threadIdx.x == 0 && next < M) {  // prefetch the next row into the other buffer
+            const int64_t src = source_row(rows, next, T_src, ok_src);
             mbar_arrive_expect_tx(&bars[st ^ 1], row_bytes);
-            bulk_load(buf[st ^ 1], x + next * ldx, row_bytes, &bars[st ^ 1]);
+            bulk_load(buf[st ^ 1], x + src * ldx, row_bytes, &bars[st ^ 1]);
             inflight[st ^ 1] = true;
         }
         if (!mbar_wait(&bars[st], phase[st], abort_flag, status)) break;
         inflight[st] = false;
         phase[st] ^= 1u;
+        source_row(rows, row, T_src, ok_src);
         const float a = row_absmax<T>(buf[st], K, red);
-        const float s = (a == 0.0f) ? 0.0f : __fdiv_rn(a, 127.0f);
-        if (threadIdx.x == 0) s_a[row] = s;
+        const float s = (a == 0.0f || !ok_src) ? 0.0f : __fdiv_rn(a, 127.0f);
+        if (threadIdx.x == 0) {
+            s_a[row] = s;
+            if (!ok_src) atomicExch(status, kStatusInvalidArg);
+        }
         quantize_row<T>(buf[st], K, s, q + row * K);
         __syncthreads();  // buffer and reduction scratch are free again
         st ^= 1;
@@ -135,15 +158,20 @@ __global__ void __launch_bounds__(kThreads) quant_rows_staged(const T* __restric
 template <typename T>
 __global__ void __launch_bounds__(kThreads) quant_rows_direct(const T* __restrict__ x, int64_t M, int64_t K,
                                                               int64_t ldx, int8_t* __restrict__ q,
-                                                              float* __restrict__ s_a) {
+                                                              float* __restrict__ s_a, int* status,
+                                                              const int32_t* __restrict__ rows, int64_t T_src) {
     __shared__ float red[kWarps];
     if (threadIdx.x == 0) griddep_launch_dependents();
     griddep_wait();  // x may be the previous kernel's output, q and s_a its input
     for (int64_t row = blockIdx.x; row < M; row += gridDim.x) {
-        const T* r = x + row * ldx;
+        bool ok_src = true;
+        const T* r = x + source_row(rows, row, T_src, ok_src) * ldx;
         const float a = row_absmax<T>(r, K, red);
-        const float s = (a == 0.0f) ? 0.0f : __fdiv_rn(a, 127.0f);
-        if (threadIdx.x == 0) s_a[row] = s;
+        const float s = (a == 0.0f || !ok_src) ? 0.0f : __fdiv_rn(a, 127.0f);
+        if (threadIdx.x == 0) {
+            s_a[row] = s;
+            if (!ok_src) atomicExch(status, kStatusInvalidArg);
+        }
         quantize_row<T>(r, K, s, q + row * K);
         __syncthreads();
     }
@@ -268,7 +296,7 @@ static cudaError_t staged_blocks_per_sm(K kern, size_t smem, int* per_sm) {
 
 template <typename T>
 static cudaError_t launch_t(const T* x, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a, int* status,
-                            cudaStream_t stream, int num_sms) {
+                            cudaStream_t stream, int num_sms, const int32_t* rows, int64_t T_src) {
     const uint32_t row_bytes = uint32_t(K * sizeof(T));
     const uint32_t buf_bytes = (row_bytes + 127u) & ~127u;
     const size_t smem = 2 * size_t(buf_bytes) + 2 * sizeof(uint64_t) + kWarps * sizeof(float) + 16;
@@ -279,7 +307,7 @@ static cudaError_t launch_t(const T* x, int64_t M, int64_t K, int64_t ldx, int8_
         if (e != cudaSuccess) return e;
         const int64_t grid = M < int64_t(num_sms) * per_sm ? M : int64_t(num_sms) * per_sm;
         const LaunchPdl lc(unsigned(grid), kThreads, smem, stream);
-        return cudaLaunchKernelEx(&lc.cfg, kern, x, M, K, ldx, q, s_a, status);
+        return cudaLaunchKernelEx(&lc.cfg, kern, x, M, K, ldx, q, s_a, status, rows, T_src);
     }
     auto kern = quant_rows_direct<T>;
     int per_sm = 0;
@@ -288,15 +316,15 @@ static cudaError_t launch_t(const T* x, int64_t M, int64_t K, int64_t ldx, int8_
     if (per_sm < 1) per_sm = 1;
     const int64_t grid = M < int64_t(num_sms) * per_sm ? M : int64_t(num_sms) * per_sm;
     const LaunchPdl lc(unsigned(grid), kThreads, 0, stream);
-    return cudaLaunchKernelEx(&lc.cfg, kern, x, M, K, ldx, q, s_a);
+    return cudaLaunchKernelEx(&lc.cfg, kern, x, M, K, ldx, q, s_a, status, rows, T_src);
 }
 
 cudaError_t launch(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a,
-                   int* status, cudaStream_t stream, int num_sms) {
+                   int* status, cudaStream_t stream, int num_sms, const int32_t* rows, int64_t T_src) {
     if (bf16)
         return launch_t<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(x), M, K, ldx, q, s_a, status, stream,
-                                       num_sms);
-    return launch_t<float>(static_cast<const float*>(x), M, K, ldx, q, s_a, status, stream, num_sms);
+                                       num_sms, rows, T_src);
+    return launch_t<float>(static_cast<const float*>(x), M, K, ldx, q, s_a, status, stream, num_sms, rows, T_src);
 }
 
 cudaError_t launch_asym(const void* x, bool bf16, int64_t M, int64_t K, int64_t ldx, int8_t* q, float* s_a,

@@ -41,6 +41,9 @@ CASES = [
     (3, 16384, 136, 512),
     (1, 16384, 40, 16384),
     (1, 8192, 22016, 128),
+    (2, 4096, 22016, 128),
+    (4, 4096, 8192, 128),
+    # four tokens and 45 MB of weights: past the decode kernel's size rule (tiles)
     (4, 4096, 22016, 128),
 ]
 
@@ -52,7 +55,8 @@ def test_gemv_intscale_and_floatscale(M, K, N, group):
     q, s = bgq.quantize_act_per_token(torch.from_numpy(wl.x).to(dev).to(torch.bfloat16))
     pk = bgq.pack_w4_groupwise(torch.from_numpy(wl.w).to(dev), group=group, alpha=1024)
     ref = oracle.linear_intscale(wl.x, wl.w, group=group, alpha=1024, out="f32")
-    assert bgq.load().w4a8_gemm_workspace_size(M, N, K, group, 1) == 0  # no scratch memory on this path
+    if M <= 2 or N * K // 2 <= 32 << 20:  # the decode kernel takes no scratch memory
+        assert bgq.load().w4a8_gemm_workspace_size(M, N, K, group, 1) == 0
     acc = bgq.w4a8_gemm_intscale(q, s, pk["packed"], pk["S"], 1024, group=group, out="i32")
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
     for out in ("f32", "f16"):
@@ -68,9 +72,9 @@ def test_gemv_intscale_and_floatscale(M, K, N, group):
 
 @pytest.mark.parametrize("M,x_dtype", [(1, "bf16"), (3, "f32"), (4, "bf16"), (5, "bf16"), (16, "f32")])
 def test_linear_intscale_quantizes_in_the_kernel(M, x_dtype):
-    """Tokens in, outputs out: with M <= 4 one kernel quantizes the tokens
-    itself (codes and scales bit-exact); with more tokens the entry point
-    chains the quantizer and the GEMM."""
+    """Tokens in, outputs out: with one token one kernel quantizes the token
+    itself (codes and scale bit-exact); with more tokens and the code buffers
+    given, the entry point chains the quantizer and the GEMM."""
     dev = torch.device("cuda:0")
     K, N = 4096, 1032
     wl = workloads.make_linear(M, K, N, x_dtype=x_dtype, seed=90 + M)
@@ -101,3 +105,33 @@ def test_linear_intscale_special_rows():
     acc = bgq.w4a8_linear_intscale(torch.from_numpy(wl.x).to(dev), pk["packed"], pk["S"], 1024, out="i32")
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
     assert not acc[1].any()
+
+
+@pytest.mark.parametrize("M,K,N,x_dtype", [(3, 4096, 1032, "f32"), (4, 2048, 520, "bf16"), (2, 1152, 264, "f32")])
+def test_linear_intscale_one_kernel_without_buffers(M, K, N, x_dtype):
+    """Through the C entry point with no code / scale buffers: with up to four
+    tokens the one-kernel route runs (it quantizes the tokens in every CTA);
+    raw accumulators bit-exact, fp16 outputs within tolerance."""
+    import ctypes
+
+    dev = torch.device("cuda:0")
+    wl = workloads.make_linear(M, K, N, x_dtype=x_dtype, seed=300 + M)
+    x = torch.from_numpy(wl.x).to(dev)
+    if x_dtype == "bf16":
+        x = x.to(torch.bfloat16)
+    pk = bgq.pack_w4_groupwise(torch.from_numpy(wl.w).to(dev), group=128, alpha=1024)
+    ref = oracle.linear_intscale(wl.x, wl.w, group=128, alpha=1024, out="f32")
+    lib = bgq.load()
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    x_dt = 2 if x_dtype == "bf16" else 0
+    for out, dt, tdt in (("i32", 3, torch.int32), ("f16", 1, torch.float16)):
+        y = torch.empty((M, N), dtype=tdt, device=dev)
+        code = lib.w4a8_linear_intscale(x.data_ptr(), x_dt, M, K, K, pk["packed"].data_ptr(), pk["S"].data_ptr(),
+                                        1024, N, 128, y.data_ptr(), dt, None, None, None, 0, stream)
+        assert code == 0
+        torch.cuda.synchronize()
+        if out == "i32":
+            assert np.array_equal(y.cpu().numpy().astype(np.int64), ref["acc"])
+        else:
+            _close(y.float().cpu().numpy(), ref["y64"], "f16")
+    assert bgq.device_status() == 0

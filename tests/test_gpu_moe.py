@@ -28,14 +28,22 @@ def _grouped(q, s, ri, off, pk, alpha, out, **kw):
                                           alpha, out=out, **kw)
 
 
-def _run(wl, E, alpha, out="i32", route=None):
+def _run(wl, E, alpha, out="i32", route=None, routed=False):
+    """routed: quantize the tokens in routed order and hand the grouped call
+    those rows with no row index (whole-tile reads); otherwise quantize every
+    token once and let the call gather rows by index."""
     dev = torch.device("cuda:0")
     route = wl.experts if route is None else route
     ri, off = workloads.route_rows(route, E)
     x = torch.from_numpy(wl.x).to(dev).to(torch.bfloat16)
-    q, s = bgq.quantize_act_per_token(x)
     pk = bgq.pack_moe_experts([torch.from_numpy(w).to(dev) for w in wl.w], alpha=alpha)
-    y = _grouped(q, s, ri, off, pk, pk["alpha"], out)
+    if routed:
+        q, s = bgq.quantize_act_routed(x, torch.from_numpy(ri.astype(np.int32)).to(dev))
+        y = bgq.w4a8_gemm_intscale_grouped(q, s, None, torch.from_numpy(np.asarray(off, np.int64)).to(dev),
+                                           pk["packed"], pk["S"], pk["alpha"], out=out)
+    else:
+        q, s = bgq.quantize_act_per_token(x)
+        y = _grouped(q, s, ri, off, pk, pk["alpha"], out)
     torch.cuda.synchronize()
     return ri, off, pk, y
 
@@ -43,9 +51,10 @@ def _run(wl, E, alpha, out="i32", route=None):
 @pytest.mark.parametrize("T,K,N,E,topk", [(64, 512, 256, 4, 2), (37, 256, 136, 8, 2), (200, 1024, 520, 3, 1),
                                           (700, 512, 384, 2, 1)])
 @pytest.mark.parametrize("alpha", [1024, None])
-def test_moe_parity(T, K, N, E, topk, alpha):
+@pytest.mark.parametrize("routed", [False, True])
+def test_moe_parity(T, K, N, E, topk, alpha, routed):
     wl = workloads.make_moe(T, K, N, E, topk=topk, seed=T + E)
-    ri, off, pk, acc = _run(wl, E, alpha, "i32")
+    ri, off, pk, acc = _run(wl, E, alpha, "i32", routed=routed)
     ref = oracle.moe_intscale(wl.x, wl.w, ri, off, alpha=alpha, out="f32")
     assert pk["alpha"] == ref["alpha"]
     for e in range(E):
@@ -53,9 +62,48 @@ def test_moe_parity(T, K, N, E, topk, alpha):
         assert np.array_equal(pk["S"][e].cpu().numpy(), ref["S"][e])
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
     for out in ("f32", "f16"):
-        _, _, _, y = _run(wl, E, alpha, out)
+        _, _, _, y = _run(wl, E, alpha, out, routed=routed)
         _close(y.float().cpu().numpy(), ref["y64"], out)
     assert bgq.device_status() == 0
+
+
+@pytest.mark.parametrize("T,K,x_dtype", [(50, 4096, "bf16"), (33, 16384, "f32"), (5, 256, "f32")])
+def test_routed_quantize_matches_per_token_codes(T, K, x_dtype):
+    """Row i of the routed quantization is token row_index[i]'s codes and
+    scale, bit for bit (the oracle's per-token quantization, gathered);
+    tokens repeat, skip and come in any order."""
+    dev = torch.device("cuda:0")
+    wl = workloads.make_linear(T, K, 8, x_dtype=x_dtype, seed=T)
+    qx, s_a = oracle.quantize_act_per_token(wl.x)
+    rng = np.random.default_rng(T)
+    ri = rng.integers(0, T, 3 * T).astype(np.int32)
+    x = torch.from_numpy(wl.x).to(dev)
+    if x_dtype == "bf16":
+        x = x.to(torch.bfloat16)
+    q, s = bgq.quantize_act_routed(x, torch.from_numpy(ri).to(dev))
+    torch.cuda.synchronize()
+    assert np.array_equal(q.cpu().numpy(), qx[ri])
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_a[ri].view(np.uint32))
+    assert bgq.device_status() == 0
+
+
+def test_routed_quantize_out_of_range_token():
+    """A routed row naming a token outside [0, T) gets zero codes and scale,
+    and the device status word reports W4A8_ERR_INVALID_ARG (1)."""
+    dev = torch.device("cuda:0")
+    wl = workloads.make_linear(8, 512, 8, x_dtype="f32", seed=3)
+    qx, s_a = oracle.quantize_act_per_token(wl.x)
+    ri = np.array([2, -1, 7, 8, 0], np.int32)
+    bgq.device_status(clear=True)
+    q, s = bgq.quantize_act_routed(torch.from_numpy(wl.x).to(dev), torch.from_numpy(ri).to(dev))
+    torch.cuda.synchronize()
+    assert bgq.device_status(clear=True) == 1
+    qh, sh = q.cpu().numpy(), s.cpu().numpy()
+    for i, t in enumerate(ri):
+        if 0 <= t < 8:
+            assert np.array_equal(qh[i], qx[t]) and sh[i] == s_a[t]
+        else:
+            assert not qh[i].any() and sh[i] == 0.0
 
 
 def test_moe_empty_experts_and_single_expert():
@@ -65,6 +113,8 @@ def test_moe_empty_experts_and_single_expert():
     ref = oracle.moe_intscale(wl.x, wl.w, ri, off, alpha=1024)
     assert list(np.diff(off)) == [0, 0, 0, 48, 0]
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+    _, _, _, acc_r = _run(wl, 5, 1024, "i32", route, routed=True)
+    assert np.array_equal(acc_r.cpu().numpy().astype(np.int64), ref["acc"])
     # no routed rows at all: nothing to do
     dev = torch.device("cuda:0")
     q = torch.zeros((4, 512), dtype=torch.int8, device=dev)
@@ -155,8 +205,14 @@ def test_moe_mixtral_full_layer_sampled():
     pk = bgq.pack_moe_experts([torch.from_numpy(w).to(dev) for w in wl.w], alpha=None)
     acc = _grouped(q, s, ri, off, pk, pk["alpha"], "i32")
     y = _grouped(q, s, ri, off, pk, pk["alpha"], "f16")
+    # the routed rows quantized in routed order, read as whole tiles
+    ri_d = torch.from_numpy(ri.astype(np.int32)).to(dev)
+    q_r, s_r = bgq.quantize_act_routed(x, ri_d)
+    acc_r = bgq.w4a8_gemm_intscale_grouped(q_r, s_r, None, torch.from_numpy(np.asarray(off, np.int64)).to(dev),
+                                           pk["packed"], pk["S"], pk["alpha"], out="i32")
     torch.cuda.synchronize()
     assert bgq.device_status() == 0
+    assert torch.equal(acc_r, acc)
 
     qx, s_a = oracle.quantize_act_per_token(wl.x)
     assert np.array_equal(q.cpu().numpy(), qx)
