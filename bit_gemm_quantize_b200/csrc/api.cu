@@ -689,16 +689,55 @@ w4a8_status w4a8_gemm_intscale_grouped(const int8_t* q_x, const float* s_a, int6
     if (!aligned16(workspace)) return W4A8_ERR_ALIGN;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
 
-    // tensor maps: a template for the experts' packed weights (its address
-    // is replaced per expert on the device), and the token codes: gathered by
-    // row, four at a time (a box one row high), or, with no row index, whole
-    // tiles of consecutive routed rows
+    const float inv_alpha = std::ldexp(1.0f, -int(std::log2(double(alpha))));
+    const int32_t y_kind = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
+                                               : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
+    if (!row_index) {
+        // routed-order codes: the tiles of w4a8_gemm_intscale (token tile 128),
+        // each tile's rows read as one box.  Tensor maps: a template for the
+        // experts' packed weights (its address is replaced per expert on the
+        // device) and the codes [T][K].
+        CUtensorMap tm_w, tm_x;
+        if (!make_map_u8(&tm_w, workspace, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2),
+                         uint32_t(w4a8::gemm::weight_box_bytes()), 128, CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4A8_ERR_CUDA;
+        if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(T), uint64_t(K), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+            return W4A8_ERR_CUDA;
+        w4a8::gemm::ParamsGr g{};
+        g.s_a = s_a;
+        g.y = y;
+        g.ws_count = reinterpret_cast<int32_t*>(ws);
+        g.ws_part = reinterpret_cast<int32_t*>(ws + 4096);
+        g.status = dev.status;
+        g.M = 0;
+        g.N = N;
+        g.G = K / group;
+        g.kb_per_group = group / 128;
+        g.grid = L.grid;
+        g.inv_alpha = inv_alpha;
+        g.y_dtype = y_kind;
+        g.wait_limit = g_wait_limit.load();
+        g.grp_sched = reinterpret_cast<const int32_t*>(ws + L.sched_off);
+        g.grp_maps = reinterpret_cast<const CUtensorMap*>(ws + L.maps_off);
+        g.grp_scales = reinterpret_cast<const void* const*>(S);
+        g.out_row = out_row;
+        g.y_rows = out_row ? y_rows : R;
+        g.E = E;
+        g.n_tiles = int32_t((N + 127) / 128);
+        W4A8_CUDA_TRY(w4a8::gemm::launch_grouped(tm_w, tm_x, expert_offsets,
+                                                 reinterpret_cast<const void* const*>(w_packed), R, g,
+                                                 reinterpret_cast<int32_t*>(ws + L.sched_off),
+                                                 reinterpret_cast<CUtensorMap*>(ws + L.maps_off),
+                                                 static_cast<cudaStream_t>(stream)));
+        return W4A8_OK;
+    }
+    // rows gathered by index: the wide-tile kernel, four rows per copy (a box
+    // one row high).  Tensor maps: the experts' weight template and the codes.
     CUtensorMap tm_w, tm_x;
     if (!make_map_u8(&tm_w, workspace, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 64, 128,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
         return W4A8_ERR_CUDA;
-    const uint32_t x_box_rows = row_index ? 1u : uint32_t(w4a8::gemm::wide_token_tile());
-    if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(T), uint64_t(K), 128, x_box_rows, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(T), uint64_t(K), 128, 1, CU_TENSOR_MAP_SWIZZLE_128B))
         return W4A8_ERR_CUDA;
     w4a8::gemm::WideParams q{};
     q.s_a = s_a;
@@ -713,9 +752,8 @@ w4a8_status w4a8_gemm_intscale_grouped(const int8_t* q_x, const float* s_a, int6
     q.n_tiles = int32_t((N + 127) / 128);
     q.m_tiles = 0;
     q.grid = int32_t(L.grid);
-    q.inv_alpha = std::ldexp(1.0f, -int(std::log2(double(alpha))));
-    q.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
-                                    : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
+    q.inv_alpha = inv_alpha;
+    q.y_dtype = y_kind;
     q.row_index = row_index;
     q.out_row = out_row;
     q.moe_scales = reinterpret_cast<const void* const*>(S);

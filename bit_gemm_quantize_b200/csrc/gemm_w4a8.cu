@@ -187,45 +187,100 @@ struct Cfg {
 // is 32-bit: a 64-bit division is a long software sequence on the GPU.
 struct Segment {
     uint32_t tile;
+    int32_t e;  // expert (grouped calls)
     int32_t n_tile, m_tile;
     int32_t g0, g1;
     uint32_t first;  // flattened index of the segment's first step
 };
 
+// The stream-K partition of a call's (tile, group) steps over its CTAs:
+// W steps, W / grid and W % grid, and the CTAs that take ranges (a grouped
+// call reads all four from its schedule, written on the device).
+struct Part {
+    uint32_t W, w_q, w_r, grid;
+};
+
+template <bool GR, typename P>
+__device__ __forceinline__ Part part_of(const P& p) {
+    if constexpr (GR)
+        return Part{uint32_t(p.grp_sched[0]), uint32_t(p.grp_sched[1]), uint32_t(p.grp_sched[2]),
+                    uint32_t(p.grp_sched[3])};
+    else
+        return Part{uint32_t(p.W), p.w_q, p.w_r, uint32_t(p.grid)};
+}
+
 // First step of CTA b's range: floor(b * W / grid) = b * (W / grid) + floor(b * (W % grid) / grid).
-__device__ __forceinline__ uint32_t range_start(uint32_t b, const Params& p) {
-    return b * p.w_q + (b * p.w_r) / uint32_t(p.grid);
+// CTAs at or past `grid` (a grouped call launches one per SM and may have
+// fewer steps than that) get the empty range [W, W).
+__device__ __forceinline__ uint32_t range_start(uint32_t b, const Part& pt) {
+    const uint32_t c = b < pt.grid ? b : pt.grid;
+    return c * pt.w_q + (c * pt.w_r) / pt.grid;
 }
 
 // CTA whose range holds step i: the largest b with range_start(b) <= i, from
 // a floating-point estimate corrected with exact starts.
-__device__ __forceinline__ uint32_t range_owner(uint32_t i, const Params& p) {
-    const uint32_t grid = uint32_t(p.grid);
-    uint32_t o = uint32_t((double(i) + 1.0) * double(grid) / double(p.W));
+__device__ __forceinline__ uint32_t range_owner(uint32_t i, const Part& pt) {
+    const uint32_t grid = pt.grid;
+    uint32_t o = uint32_t((double(i) + 1.0) * double(grid) / double(pt.W));
     if (o >= grid) o = grid - 1;
-    while (o > 0 && range_start(o, p) > i) --o;
-    while (o + 1 < grid && range_start(o + 1, p) <= i) ++o;
+    while (o > 0 && range_start(o, pt) > i) --o;
+    while (o + 1 < grid && range_start(o + 1, pt) <= i) ++o;
     return o;
 }
 
+// Per-expert schedule of a grouped call, after the partition in its
+// workspace: m_tiles[E+1], first tile[E+1] and first routed row[E+1].
+struct GrSched {
+    const int32_t* mt;
+    const int32_t* tstart;
+    const int32_t* rstart;
+};
+
+template <typename P>
+__device__ __forceinline__ GrSched grsched_of(const P& p) {
+    const int32_t* base = p.grp_sched + 4;
+    return GrSched{base, base + (p.E + 1), base + 2 * (p.E + 1)};
+}
+
 // Iterates the segments of CTA `b`.  The divisions happen once, at the start
-// of the range; afterwards the tile coordinates advance incrementally.
+// of the range; afterwards the tile coordinates advance incrementally.  A
+// grouped call orders its tiles expert by expert (then by weight-column tile,
+// then by token tile), each expert with its own count of token tiles.
+template <bool GR>
 struct SegmentIter {
     uint32_t i, end, tile;
     int32_t G, g, n_tile, m_tile, m_tiles;
-    __device__ SegmentIter(const Params& p, uint32_t b) {
+    int32_t e, n_tiles, E;  // grouped calls
+    GrSched sc;
+    template <typename P>
+    __device__ SegmentIter(const P& p, const Part& pt, uint32_t b) {
         G = int32_t(p.G);
-        m_tiles = int32_t(p.m_tiles);
-        i = range_start(b, p);
-        end = range_start(b + 1, p);
+        i = range_start(b, pt);
+        end = range_start(b + 1, pt);
         tile = i / uint32_t(G);
         g = int32_t(i - tile * uint32_t(G));
-        n_tile = int32_t(tile / uint32_t(m_tiles));
-        m_tile = int32_t(tile - uint32_t(n_tile) * uint32_t(m_tiles));
+        e = 0;
+        uint32_t local = tile;
+        if constexpr (GR) {
+            sc = grsched_of(p);
+            E = p.E;
+            n_tiles = p.n_tiles;
+            m_tiles = 1;
+            if (i < end) {
+                while (e + 1 < E && uint32_t(sc.tstart[e + 1]) <= tile) ++e;
+                local = tile - uint32_t(sc.tstart[e]);
+                m_tiles = sc.mt[e];
+            }
+        } else {
+            m_tiles = int32_t(p.m_tiles);
+        }
+        n_tile = int32_t(local / uint32_t(m_tiles));
+        m_tile = int32_t(local - uint32_t(n_tile) * uint32_t(m_tiles));
     }
     __device__ bool next(Segment& s) {
         if (i >= end) return false;
         s.tile = tile;
+        s.e = e;
         s.n_tile = n_tile;
         s.m_tile = m_tile;
         s.g0 = g;
@@ -238,7 +293,19 @@ struct SegmentIter {
             ++tile;
             if (++m_tile == m_tiles) {
                 m_tile = 0;
-                ++n_tile;
+                if constexpr (GR) {
+                    if (++n_tile == n_tiles) {
+                        n_tile = 0;
+                        if (i < end) {  // the next expert with rows
+                            do {
+                                ++e;
+                            } while (e + 1 < E && sc.mt[e] == 0);
+                            m_tiles = sc.mt[e];
+                        }
+                    }
+                } else {
+                    ++n_tile;
+                }
             }
         } else {
             g = s.g1;
@@ -249,26 +316,31 @@ struct SegmentIter {
 
 // One pipeline stage: up to two consecutive 128-wide K blocks of one segment.
 struct Stage {
+    int32_t e;    // expert (grouped calls)
     int32_t n_tile, m_tile;
     int32_t kb;   // first K block (global index along K)
     int32_t nkb;  // 1 or 2
 };
 
+template <bool GR>
 struct StageIter {
-    SegmentIter seg;
+    SegmentIter<GR> seg;
     int32_t kbpg;
-    int32_t n_tile = 0, m_tile = 0;
+    int32_t e = 0, n_tile = 0, m_tile = 0;
     int32_t kb = 0, kb_end = 0;
-    __device__ StageIter(const Params& p, uint32_t b) : seg(p, b), kbpg(p.kb_per_group) {}
+    template <typename P>
+    __device__ StageIter(const P& p, const Part& pt, uint32_t b) : seg(p, pt, b), kbpg(p.kb_per_group) {}
     __device__ bool next(Stage& st) {
         while (kb >= kb_end) {
             Segment s;
             if (!seg.next(s)) return false;
+            e = s.e;
             n_tile = s.n_tile;
             m_tile = s.m_tile;
             kb = s.g0 * kbpg;
             kb_end = s.g1 * kbpg;
         }
+        st.e = e;
         st.n_tile = n_tile;
         st.m_tile = m_tile;
         st.kb = kb;
@@ -289,10 +361,14 @@ __device__ __forceinline__ float output_scale(const Params& p, int64_t m) {
 // G1: the group is one 128-wide K block (group = 128, the method's group
 // size), so every K block ends a group; wide token tiles then drain each group
 // in a loop with no per-stage bookkeeping.
-template <int BT, int PATH, bool W8, bool ZP, bool G1>
+// GR: a grouped (mixture-of-experts) call: tiles expert by expert from a
+// schedule in the workspace, each expert's weights through its own tensor
+// map, token rows as blocks of routed-order codes, outputs one row at a time.
+template <int BT, int PATH, bool W8, bool ZP, bool G1, bool GR = false>
 __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH, W8, ZP>::kCtasPerSm)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-                     const __grid_constant__ CUtensorMap tm_y, const std::conditional_t<ZP, ParamsZp, Params> p) {
+                     const __grid_constant__ CUtensorMap tm_y,
+                     const std::conditional_t<ZP, ParamsZp, std::conditional_t<GR, ParamsGr, Params>> p) {
     using C = Cfg<BT, PATH, W8, ZP>;
     constexpr bool kLean = G1 && C::kGroupCommit;  // the per-group drain loop below
     constexpr int kAcc = C::kAcc;
@@ -350,6 +426,9 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
     // The next kernel in the stream may be scheduled now; it cannot share an
     // SM with this CTA (shared memory), so its CTAs start where ours finish.
     if (threadIdx.x == 0) griddep_launch_dependents();
+    // a grouped call's schedule and weight maps come from the setup kernel
+    if constexpr (GR) griddep_wait();
+    const Part pt = part_of<GR>(p);
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
@@ -365,19 +444,30 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
         Ring rwd;          // int8 weights: stage-done slot of the stage whose weight slot is reused (SW back)
         int32_t pst = 0;   // stages issued so far
         uint32_t w_issued = 0u, w_par = 0u, x_issued = 0u, x_par = 0u;  // per slot: copy issued / its parity
+        // the weights' tensor map: one per expert in a grouped call (fetched
+        // to the tensor-map proxy when the expert changes)
+        const CUtensorMap* wmap = &tm_w;
+        int32_t wmap_e = -1;
         auto issue_w = [&](const Stage& st, const Ring& slot) {
+            if constexpr (GR) {
+                if (st.e != wmap_e) {
+                    wmap = p.grp_maps + st.e;
+                    wmap_e = st.e;
+                    tensormap_acquire(wmap);
+                }
+            }
             if constexpr (C::kW8) {
                 // int8 weights: one 128-row x 128 B box per K block
                 uint8_t* dst = smem + C::offW + slot.idx * C::kWBytes;
                 mbar_arrive_expect_tx_one(&full_w[slot.idx], uint32_t(st.nkb * kTileN * kBlockK));
-                tma_load_2d_one(dst, &tm_w, st.kb * kBlockK, st.n_tile * kTileN, &full_w[slot.idx]);
+                tma_load_2d_one(dst, wmap, st.kb * kBlockK, st.n_tile * kTileN, &full_w[slot.idx]);
                 if (st.nkb == 2)
-                    tma_load_2d_one(dst + kTileN * kBlockK, &tm_w, (st.kb + 1) * kBlockK, st.n_tile * kTileN,
+                    tma_load_2d_one(dst + kTileN * kBlockK, wmap, (st.kb + 1) * kBlockK, st.n_tile * kTileN,
                                     &full_w[slot.idx]);
             } else {
                 // one 128 x 128 B box = two K blocks (a lone last block over-reads 64 B per row: harmless)
                 mbar_arrive_expect_tx_one(&full_w[slot.idx], C::kWBytes);
-                tma_load_2d_one(smem + C::offW + slot.idx * C::kWBytes, &tm_w, st.kb * (kBlockK / 2),
+                tma_load_2d_one(smem + C::offW + slot.idx * C::kWBytes, wmap, st.kb * (kBlockK / 2),
                                 st.n_tile * kTileN, &full_w[slot.idx]);
             }
             w_issued |= 1u << slot.idx;
@@ -385,7 +475,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
         };
         int32_t prefetched = 0;  // leading stages whose weights were requested before the wait
         {
-            StageIter it(p, b);
+            StageIter<GR> it(p, pt, b);
             Stage st;
             while (prefetched < (W4A8_PREFETCH(C::kCtasPerSm) < SW ? W4A8_PREFETCH(C::kCtasPerSm) : SW) &&
                    it.next(st)) {
@@ -395,12 +485,15 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             }
         }
         rw = Ring{};
-        griddep_wait();  // the token codes may be the previous kernel's output
-        StageIter it(p, b);
+        wmap_e = -1;
+        if constexpr (!GR) griddep_wait();  // the token codes may be the previous kernel's output
+        StageIter<GR> it(p, pt, b);
         Stage st;
         bool ok = true;
         while (ok && it.next(st)) {
-            const int32_t m0 = st.m_tile * BT;
+            // first token row of the tile (a grouped call: of the expert's routed rows)
+            int32_t m0 = st.m_tile * BT;
+            if constexpr (GR) m0 += grsched_of(p).rstart[st.e];
             if (pst >= prefetched) {
                 bool free_slot;
                 if constexpr (C::kW8) {
@@ -453,7 +546,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
         constexpr uint32_t idesc = idesc_i8(kTileN, BT);
         Ring rx, ra, rt, rd;
         Ring rw;  // int8 weights: the weight slot (the MMA's A operand in shared memory)
-        StageIter it(p, b);
+        StageIter<GR> it(p, pt, b);
         Stage st;
         bool ok = true;
         int32_t kin = 0;  // position of the next K block inside its group (segments start on group boundaries)
@@ -539,7 +632,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
         Ring rw, ra;
         Ring rad;          // stage-done slot of the stage whose operand slot is reused (SA stages back)
         int32_t ust = 0;   // stages unpacked so far
-        StageIter it(p, b);
+        StageIter<GR> it(p, pt, b);
         Stage st;
         bool ok = true;
         const uint32_t lane_base = tmem_base + (uint32_t(quarter * 32) << 16);
@@ -604,14 +697,25 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
         const int half = ew >> 2;      // which part of the BT columns
         const int r = quarter * 32 + lane;
         Ring rt, rd;
-        SegmentIter it(p, b);
+        SegmentIter<GR> it(p, pt, b);
         Segment sg;
         bool ok = true;
         const int32_t kbpg = p.kb_per_group;
         const int32_t G = int32_t(p.G);
         while (ok && it.next(sg)) {
             const int64_t n0 = int64_t(sg.n_tile) * kTileN;
-            const int64_t m0 = int64_t(sg.m_tile) * BT + half * HC;
+            // the tile's first token row and the end of its rows (a grouped
+            // call: the expert's routed rows) and the group scales to use
+            int64_t mbase = int64_t(sg.m_tile) * BT;
+            int64_t mend = p.M;
+            const int16_t* S_g = p.S;
+            if constexpr (GR) {
+                const GrSched gs = grsched_of(p);
+                mbase += gs.rstart[sg.e];
+                mend = gs.rstart[sg.e + 1];
+                S_g = static_cast<const int16_t*>(p.grp_scales[sg.e]);
+            }
+            const int64_t m0 = mbase + half * HC;
             const int64_t n = n0 + r;
             const bool nvalid = n < p.N;
             // output scale of token (tile start + this thread's index among the
@@ -621,10 +725,10 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             int32_t zc_n = 0;     // zero-point term of this thread's column (ZP)
             {
                 const int te = ew * 32 + lane;
-                const int64_t mt = int64_t(sg.m_tile) * BT + te;
-                if (te < BT && mt < p.M) sa_pref = output_scale<PATH>(p, mt);
+                const int64_t mt = mbase + te;
+                if (te < BT && mt < mend) sa_pref = output_scale<PATH>(p, mt);
                 if constexpr (ZP) {
-                    if (te < BT && mt < p.M) z_pref = p.z_a[mt];
+                    if (te < BT && mt < mend) z_pref = p.z_a[mt];
                     if (nvalid) zc_n = p.zc[n];
                 }
             }
@@ -645,13 +749,13 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             if constexpr (C::kEarlyCombine) {
                 if (sg.g0 == 0 && sg.g1 < int32_t(p.G)) {
                     const uint32_t t0 = sg.tile * uint32_t(p.G);
-                    const uint32_t b_last = range_owner(t0 + uint32_t(p.G) - 1u, p);
+                    const uint32_t b_last = range_owner(t0 + uint32_t(p.G) - 1u, pt);
                     if (ew == 0 && lane == 0)
                         misc[3] = (b_last == b + 1 && ld_acquire_gpu(&p.ws_count[b]) >= 1) ? 1u : 0u;
                     epi_bar_sync(kEpiWarps * 32);
                     early = misc[3] != 0u;  // the same for every epilogue thread
                     if (early) {
-                        const int nv = p.M - m0 >= HC ? HC : (p.M - m0 > 0 ? int(p.M - m0) : 0);
+                        const int nv = mend - m0 >= HC ? HC : (mend - m0 > 0 ? int(mend - m0) : 0);
                         const int32_t* cp = p.ws_part + int64_t(b + 1) * (int64_t(kTileN) * BT) +
                                             int64_t(half * HC) * kTileN + r;
 #pragma unroll
@@ -674,7 +778,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                 int32_t sidx = sg.g0 * nstride + n_ld;  // element index of the next scale to load (< 2^31)
                 auto ld_scale = [&](int32_t i) -> uint32_t {
                     if constexpr (PATH == kIntScale)
-                        return uint32_t(int32_t(__ldg(p.S + i)));
+                        return uint32_t(int32_t(__ldg(S_g + i)));
                     else
                         return __float_as_uint(__ldg(p.s_g + i));
                 };
@@ -723,7 +827,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                 if (g >= G || !nvalid) return 0u;
                 const int64_t idx = int64_t(g) * int32_t(p.N) + n;  // N < 2^31 (checked on the host)
                 if constexpr (PATH == kIntScale)
-                    return uint32_t(int32_t(__ldg(p.S + idx)));
+                    return uint32_t(int32_t(__ldg(S_g + idx)));
                 else
                     return __float_as_uint(__ldg(p.s_g + idx));
             };
@@ -875,7 +979,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             if (!ok) break;
 
             // valid token columns of this thread's share (split-tile partials)
-            const int nv = p.M - m0 >= HC ? HC : (p.M - m0 > 0 ? int(p.M - m0) : 0);
+            const int nv = mend - m0 >= HC ? HC : (mend - m0 > 0 ? int(mend - m0) : 0);
             const bool whole = (sg.g0 == 0 && sg.g1 == p.G);
             if (!whole) {
                 // ---- split tile.  The tile's first contributor b_first covers the
@@ -888,8 +992,8 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                 // arrivals, adds the partials to its own, which never leave registers,
                 // writes y and re-zeroes the counter.
                 const uint32_t t0 = sg.tile * uint32_t(p.G);
-                const uint32_t b_first = range_owner(t0, p);
-                const uint32_t b_last = range_owner(t0 + uint32_t(p.G) - 1u, p);
+                const uint32_t b_first = range_owner(t0, pt);
+                const uint32_t b_last = range_owner(t0 + uint32_t(p.G) - 1u, pt);
                 const int64_t slot_elems = int64_t(kTileN) * BT;
                 if (b != b_first) {
                     int32_t* part = p.ws_part + int64_t(b) * slot_elems + int64_t(half * HC) * kTileN + r;
@@ -954,7 +1058,9 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             // memory as [BT tokens][128 columns], stored by one TMA tensor store
             // (which leaves out rows past M and columns past N).
             const bool leader = (ew == 0 && lane == 0);
-            if (leader) bulk_wait_read_all();  // the previous tile's store has read the staging buffer
+            // the previous tile's stores have read the staging buffer (a
+            // grouped call's stores come from every lane of the first warp)
+            if (GR ? ew == 0 : leader) bulk_wait_read_all();
             epi_bar_sync(kEpiWarps * 32);
             float* sa_tile = reinterpret_cast<float*>(smem + C::offSA);
             if (ew * 32 + lane < BT) sa_tile[ew * 32 + lane] = sa_pref;
@@ -993,12 +1099,34 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             }
             fence_proxy_async_smem();  // the staged outputs, visible to the TMA unit
             epi_bar_sync(kEpiWarps * 32);
-            if (leader) {
+            if constexpr (GR) {
+                // one bulk copy per routed row of the tile, to row i or out_row[i]
+                // (rows past the expert's last belong to the next expert: not stored)
+                if (ew == 0) {
+                    const int esz = p.y_dtype == kOutF16 ? 2 : 4;
+                    const int64_t cols = p.N - n0 < kTileN ? p.N - n0 : kTileN;
+                    const int rows = mend - mbase < BT ? int(mend - mbase) : BT;
+                    for (int t = lane; t < rows; t += 32) {
+                        int64_t orow = mbase + t;
+                        if (p.out_row != nullptr) {
+                            orow = p.out_row[orow];
+                            if (orow < 0 || orow >= p.y_rows) {
+                                atomicExch(p.status, kStatusInvalidArg);
+                                continue;
+                            }
+                        }
+                        bulk_store(static_cast<uint8_t*>(p.y) + (orow * p.N + n0) * esz,
+                                   smem + C::offY + int64_t(t) * kTileN * esz, uint32_t(cols * esz));
+                    }
+                    bulk_commit_group();
+                }
+            } else if (leader) {
                 tma_store_2d(&tm_y, smem + C::offY, int32_t(n0), sg.m_tile * BT);
                 bulk_commit_group();
             }
         }
-        if (ew == 0 && lane == 0) bulk_wait_read_all();  // shared memory stays until the stores have read it
+        // shared memory stays until the stores have read it
+        if (GR ? ew == 0 : (ew == 0 && lane == 0)) bulk_wait_read_all();
     }
 
     tc_fence_before();
@@ -1091,6 +1219,22 @@ cudaError_t launch_zp(const CUtensorMap& tw, const CUtensorMap& tx, const CUtens
         case 64: return launch_bt<64, kIntScale, false, true>(tw, tx, ty, p, stream);
         default: return launch_bt<128, kIntScale, false, true>(tw, tx, ty, p, stream);
     }
+}
+
+cudaError_t launch_grouped(const CUtensorMap& tm_w_template, const CUtensorMap& tm_x, const int64_t* offsets,
+                           const void* const* w_ptrs, int64_t R, const ParamsGr& p, int32_t* sched,
+                           CUtensorMap* maps, cudaStream_t stream) {
+    cudaError_t e = launch_grouped_setup(tm_w_template, offsets, w_ptrs, p.grp_scales, p.E, R, 128, p.n_tiles,
+                                         int32_t(p.G), int32_t(p.grid), sched, maps, p.status, stream);
+    if (e != cudaSuccess) return e;
+    using C = Cfg<128, kIntScale, false, false>;
+    // tm_y is not read by a grouped call (its rows are stored one by one)
+    if (p.kb_per_group == 1)
+        return launch_k<w4a8_gemm_kernel<128, kIntScale, false, false, true, true>>(C::kThreads, C::kSmemBytes,
+                                                                                    tm_w_template, tm_x, tm_x, p,
+                                                                                    stream);
+    return launch_k<w4a8_gemm_kernel<128, kIntScale, false, false, false, true>>(C::kThreads, C::kSmemBytes,
+                                                                                 tm_w_template, tm_x, tm_x, p, stream);
 }
 
 int token_tile_rows() { return kTileN; }

@@ -39,6 +39,19 @@ struct ParamsZp : Params {
     const int32_t* zc;   // [N] zero-point term zc[n] = sum_g S[g,n] sum_{k in g} q[k,n]
 };
 
+// Parameters of a grouped (mixture-of-experts) call on the tiles of
+// gemm_w4a8.cu: the token rows are routed-order codes (row i = routed row i),
+// the partition and the per-expert schedule come from the workspace.
+struct ParamsGr : Params {
+    const int32_t* grp_sched;       // W, W / g, W % g, g, then m_tiles[E+1], first tile[E+1], first row[E+1]
+    const CUtensorMap* grp_maps;    // [E] weight tensor maps (built by the setup kernel)
+    const void* const* grp_scales;  // [E] device pointers to each expert's S [G, N]
+    const int32_t* out_row;         // [R] output row of each routed row, or null (row i)
+    int64_t y_rows;                 // rows of y: an output row must lie below it
+    int32_t E;
+    int32_t n_tiles;
+};
+
 // Parameters of the wide-tile kernel (token tiles of 256; gemm_wide.cu).
 struct WideParams {
     const float* s_a;    // [M] token scales (MOE: [T], indexed by token)
@@ -57,7 +70,7 @@ struct WideParams {
     float inv_alpha;
     int32_t y_dtype;
     // mixture of experts
-    const int32_t* row_index;      // [R] token of each routed row, rows grouped by expert (NULL: q_x row i)
+    const int32_t* row_index;      // [R] token of each routed row, rows grouped by expert
     const int32_t* out_row;        // [R] output row of each routed row, or null (row i)
     const void* const* moe_scales; // [E] device pointers to each expert's S [G, N]
     const int32_t* moe_sched;      // W, w_q, w_r, status, then mt[E+1], tstart[E+1], rstart[E+1]
@@ -148,6 +161,19 @@ cudaError_t launch_wide(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const 
 // wide kernel runs over all experts' tiles.  tm_w_template: a weight map of
 // the experts' shape (its address is replaced per expert); tm_x: token codes
 // [T][K] u8, box 128 B x 1 row, 128-byte swizzle (rows gathered four at a time).
+// A grouped call on the tiles of gemm_w4a8.cu (token tile 128): the setup
+// kernel, then the GEMM, chained with programmatic dependent launch.
+// tm_w_template: a packed-weight map of the tiles' box (128 rows x 128 B,
+// 128-byte swizzle) whose address the setup kernel replaces per expert;
+// tm_x: the routed-order codes [R][K], box 128 rows x 128 B.
+cudaError_t launch_grouped(const CUtensorMap& tm_w_template, const CUtensorMap& tm_x, const int64_t* offsets,
+                           const void* const* w_ptrs, int64_t R, const ParamsGr& p, int32_t* sched,
+                           CUtensorMap* maps, cudaStream_t stream);
+// The setup kernel of a grouped call (gemm_wide.cu), for token tiles of `bt`.
+cudaError_t launch_grouped_setup(const CUtensorMap& tm_w_template, const int64_t* offsets, const void* const* w_ptrs,
+                                 const void* const* s_ptrs, int32_t E, int64_t R, int32_t bt, int32_t n_tiles,
+                                 int32_t G, int32_t grid, int32_t* sched, CUtensorMap* maps, int* status,
+                                 cudaStream_t stream);
 cudaError_t launch_wide_moe(const CUtensorMap& tm_w_template, const CUtensorMap& tm_x, const int64_t* offsets,
                             const void* const* w_ptrs, int64_t R, const WideParams& p, int32_t* sched,
                             CUtensorMap* maps, cudaStream_t stream);

@@ -316,10 +316,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             rw = Ring{};
             griddep_wait();  // the token codes may be the previous kernel's output
         }
-        // token rows of the current tile (MOE: gathered by routed row, or,
-        // with no row index, the tile's first routed row of q_x)
+        // token rows of the current tile (MOE: gathered by routed row)
         int32_t trow[8];
-        int32_t xrow0 = 0;
         WStageIter<MOE> it(p, range, b);
         WStage st;
         bool ok = true;
@@ -334,9 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const Sched sc = sched_of(p);
                     const int32_t r0 = sc.rstart[st.e] + st.m_tile * kBT;
                     const int32_t r1 = sc.rstart[st.e + 1];
-                    xrow0 = r0;
 #pragma unroll
-                    for (int q = 0; q < 8 && p.row_index; ++q) {
+                    for (int q = 0; q < 8; ++q) {
                         // lane l gathers rows 4l..4l+3 and 128+4l..128+4l+3 (those
                         // below kBT); rows past the expert's last take token 0
                         // (never stored)
@@ -365,19 +362,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t* xdst = smem + offX + rx.idx * kXBytes;
             mbar_arrive_expect_tx_one(&full_x[rx.idx], uint32_t(kXBytes));
             if constexpr (MOE) {
-                if (p.row_index) {
-                    __syncwarp();
-                    tma_gather4(xdst + 4 * lane * 128, &tm_x, st.kb * 128, trow[0], trow[1], trow[2], trow[3],
-                                &full_x[rx.idx]);
-                    if (128 + 4 * lane < kBT)
-                        tma_gather4(xdst + (128 + 4 * lane) * 128, &tm_x, st.kb * 128, trow[4], trow[5], trow[6],
-                                    trow[7], &full_x[rx.idx]);
-                } else {
-                    // the routed rows are q_x's rows: one box of the tile's kBT
-                    // rows (rows past the expert's last are never stored; past
-                    // the last row of q_x they read as zero)
-                    tma_load_2d_one(xdst, &tm_x, st.kb * 128, xrow0, &full_x[rx.idx]);
-                }
+                __syncwarp();
+                tma_gather4(xdst + 4 * lane * 128, &tm_x, st.kb * 128, trow[0], trow[1], trow[2], trow[3],
+                            &full_x[rx.idx]);
+                if (128 + 4 * lane < kBT)
+                    tma_gather4(xdst + (128 + 4 * lane) * 128, &tm_x, st.kb * 128, trow[4], trow[5], trow[6],
+                                trow[7], &full_x[rx.idx]);
             } else {
                 tma_load_2d_one(xdst, &tm_x, st.kb * 128, st.m_tile * kBT, &full_x[rx.idx]);
             }
@@ -532,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int32_t tok;
                 bool tok_ok = true;
                 if constexpr (MOE) {
-                    tok = p.row_index ? p.row_index[rbase + t] : rbase + t;
+                    tok = p.row_index[rbase + t];
                     tok_ok = tok >= 0 && tok < p.moe_T;
                     if (!tok_ok) atomicExch(p.status, 1);  // W4A8_ERR_INVALID_ARG: the row's outputs are zero
                 } else {
@@ -761,8 +751,8 @@ namespace wide {
 __global__ void __launch_bounds__(256) moe_setup_kernel(const __grid_constant__ CUtensorMap tmpl,
                                                         const int64_t* offsets, const void* const* w_ptrs,
                                                         const void* const* s_ptrs, int32_t E, int64_t R,
-                                                        int32_t n_tiles, int32_t G, int32_t grid, int32_t* sched,
-                                                        CUtensorMap* maps, int* status) {
+                                                        int32_t bt, int32_t n_tiles, int32_t G, int32_t grid,
+                                                        int32_t* sched, CUtensorMap* maps, int* status) {
     __shared__ alignas(128) uint8_t smap[8][128];
     __shared__ int bad_s;
     griddep_wait();  // the offsets and pointers may be the previous kernel's output
@@ -786,7 +776,7 @@ __global__ void __launch_bounds__(256) moe_setup_kernel(const __grid_constant__ 
                 bad = 1;
                 break;
             }
-            const int64_t mte = (m + kBT - 1) / kBT;
+            const int64_t mte = (m + bt - 1) / bt;
             mt[e] = int32_t(mte);
             tstart[e] = int32_t(tiles);
             rstart[e] = int32_t(offsets[e]);
@@ -848,15 +838,21 @@ cudaError_t launch_wide(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const 
                              : wide::launch_t<kFloatScale, false>(tm_w, tm_x, tm_y, p, stream);
 }
 
+cudaError_t launch_grouped_setup(const CUtensorMap& tm_w_template, const int64_t* offsets, const void* const* w_ptrs,
+                                 const void* const* s_ptrs, int32_t E, int64_t R, int32_t bt, int32_t n_tiles,
+                                 int32_t G, int32_t grid, int32_t* sched, CUtensorMap* maps, int* status,
+                                 cudaStream_t stream) {
+    const LaunchPdl lc(1u, 256, 0, stream);
+    return cudaLaunchKernelEx(&lc.cfg, wide::moe_setup_kernel, tm_w_template, offsets, w_ptrs, s_ptrs, E, R, bt,
+                              n_tiles, G, grid, sched, maps, status);
+}
+
 cudaError_t launch_wide_moe(const CUtensorMap& tm_w_template, const CUtensorMap& tm_x, const int64_t* offsets,
                             const void* const* w_ptrs, int64_t R, const WideParams& p, int32_t* sched,
                             CUtensorMap* maps, cudaStream_t stream) {
-    {
-        const LaunchPdl lc(1u, 256, 0, stream);
-        const cudaError_t e = cudaLaunchKernelEx(&lc.cfg, wide::moe_setup_kernel, tm_w_template, offsets, w_ptrs,
-                                                 p.moe_scales, p.E, R, p.n_tiles, p.G, p.grid, sched, maps, p.status);
-        if (e != cudaSuccess) return e;
-    }
+    const cudaError_t e = launch_grouped_setup(tm_w_template, offsets, w_ptrs, p.moe_scales, p.E, R, wide::kBT,
+                                               p.n_tiles, p.G, p.grid, sched, maps, p.status, stream);
+    if (e != cudaSuccess) return e;
     return wide::launch_t<kIntScale, true>(tm_w_template, tm_x, tm_w_template, p, stream);
 }
 

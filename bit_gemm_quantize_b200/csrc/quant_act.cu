@@ -83,8 +83,6 @@ __device__ __forceinline__ int64_t source_row(const int32_t* rows, int64_t row, 
     return ok ? t : 0;
 }
 
-constexpr int kStatusInvalidArg = 1;  // W4A8_ERR_INVALID_ARG
-
 // Row staged in shared memory by a bulk async copy; two buffers.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) quant_rows_staged(const T* __restrict__ x, int64_t M, int64_t K,
