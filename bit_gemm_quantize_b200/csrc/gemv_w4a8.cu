@@ -157,9 +157,12 @@ __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUten
                 if (live && !zero) {
                     float v[16];
                     quant::load16<XT>(row + c * 16, v);
+                    uint32_t cb[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        packed[i >> 2] |= (uint32_t(quant::code_i8(v[i], s, rcp, exact_only)) & 0xFFu) << (8 * (i & 3));
+                    for (int i = 0; i < 16; ++i) cb[i] = quant::code_i8_byte(v[i], s, rcp, exact_only);
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        packed[w] = quant::pack4_low_bytes(cb[4 * w], cb[4 * w + 1], cb[4 * w + 2], cb[4 * w + 3]);
                 }
                 const uint4 q4 = make_uint4(packed[0], packed[1], packed[2], packed[3]);
                 *reinterpret_cast<uint4*>(codes + m * K + c * 16) = q4;

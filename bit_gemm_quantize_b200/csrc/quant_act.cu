@@ -50,9 +50,12 @@ __device__ __forceinline__ void quantize_row(const T* row, int64_t K, float s, i
         if (!zero) {
             float v[16];
             load16<T>(row + c * 16, v);
+            uint32_t cb[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                packed[i >> 2] |= (uint32_t(code_i8(v[i], s, rcp, exact_only)) & 0xFFu) << (8 * (i & 3));
+            for (int i = 0; i < 16; ++i) cb[i] = code_i8_byte(v[i], s, rcp, exact_only);
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                packed[w] = pack4_low_bytes(cb[4 * w], cb[4 * w + 1], cb[4 * w + 2], cb[4 * w + 3]);
         }
         *reinterpret_cast<uint4*>(qrow + c * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }

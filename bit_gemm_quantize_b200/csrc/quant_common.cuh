@@ -59,5 +59,25 @@ __device__ __forceinline__ int code_i8(float x, float s, float rcp, bool exact_o
     return int(r);
 }
 
+// The same code, returned in the low byte of a 32-bit word (the other bytes
+// are unspecified), with the rounding done by adding 1.5 * 2^23: for |t| <
+// 2^22 the sum's round-to-nearest-even drops t's fraction exactly as rint
+// does, and its low mantissa bits are the integer in two's complement.  No
+// clamp on the fast path: s = fl32(max|x| / 127) and the product's error
+// keep |t| below 127.5, so the code already lies in [-127, 127].
+__device__ __forceinline__ uint32_t code_i8_byte(float x, float s, float rcp, bool exact_only) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    const float t = __fmul_rn(x, rcp);
+    const float m = __fadd_rn(t, kMagic);
+    const float r = __fsub_rn(m, kMagic);
+    if (!exact_only && fabsf(__fsub_rn(t, r)) <= 0.49993896484375f) return __float_as_uint(m);
+    return uint32_t(code_i8(x, s, rcp, exact_only));
+}
+
+// Four codes (low bytes of a, b, c, d) as one word: byte 0 = a, ..., byte 3 = d.
+__device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
 }  // namespace quant
 }  // namespace w4a8
