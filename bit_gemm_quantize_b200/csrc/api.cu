@@ -219,7 +219,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
             w4a8::gemv::launch(tm, g, path, w4a8::gemv::kXCodes, dev.sms, static_cast<cudaStream_t>(stream)));
         return W4A8_OK;
     }
-    const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms, w8, zp);
+    const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms, w8);
     if (pl.W >= (int64_t(1) << 31)) return W4A8_ERR_SHAPE;  // the kernel indexes (tile, group) steps in 32 bits
     int32_t* ws_count = nullptr;
     int32_t* ws_part = nullptr;
@@ -228,50 +228,6 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
         if (!aligned16(workspace)) return W4A8_ERR_ALIGN;
         ws_count = static_cast<int32_t*>(workspace);
         ws_part = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + pl.count_bytes);
-    }
-
-    if (pl.wide) {
-        // wide token tiles: packed weights one K block (64 B) per box, no
-        // swizzle; token codes BT rows x 128 B, 128-byte swizzle; output boxes of
-        // BT rows (fp16) or one worker group's rows (4-byte outputs)
-        CUtensorMap tm_w, tm_x, tm_y;
-        if (!make_map_u8(&tm_w, w_packed, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 64, 128,
-                         CU_TENSOR_MAP_SWIZZLE_NONE))
-            return W4A8_ERR_CUDA;
-        if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(M), uint64_t(K), 128, uint32_t(pl.BT),
-                         CU_TENSOR_MAP_SWIZZLE_128B))
-            return W4A8_ERR_CUDA;
-        const bool f16 = (y_dtype == W4A8_F16);
-        const CUtensorMapDataType t = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
-                                          : (y_dtype == W4A8_I32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
-                                                                 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
-        if (!make_map_2d(&tm_y, t, y, uint64_t(N), uint64_t(M), uint64_t(N) * (f16 ? 2u : 4u), 128,
-                         f16 ? uint32_t(pl.BT) : uint32_t(w4a8::gemm::wide_tail_rows()), CU_TENSOR_MAP_SWIZZLE_NONE))
-            return W4A8_ERR_CUDA;
-        w4a8::gemm::WideParams q{};
-        q.s_a = s_a;
-        q.S = S;
-        q.s_g = s_g;
-        q.y = y;
-        q.ws_part = ws_part;
-        q.ws_count = ws_count;
-        q.status = dev.status;
-        q.M = int32_t(M);
-        q.N = int32_t(N);
-        q.G = int32_t(pl.G);
-        q.kb_per_group = group / 128;
-        q.n_tiles = int32_t(pl.n_tiles);
-        q.m_tiles = int32_t(pl.m_tiles);
-        q.grid = int32_t(pl.grid);
-        q.W = uint32_t(pl.W);
-        q.w_q = uint32_t(pl.W / pl.grid);
-        q.w_r = uint32_t(pl.W % pl.grid);
-        q.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
-        q.y_dtype = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
-                                        : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
-        q.wait_limit = g_wait_limit.load();
-        W4A8_CUDA_TRY(w4a8::gemm::launch_wide(tm_w, tm_x, tm_y, q, path, static_cast<cudaStream_t>(stream)));
-        return W4A8_OK;
     }
 
     CUtensorMap tm_w, tm_x, tm_y;
@@ -330,7 +286,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
 int64_t align256(int64_t v) { return (v + 255) & ~int64_t(255); }
 
 // Layout of the grouped (mixture-of-experts) workspace: [arrival counters and
-// split-tile partials of the wide kernel] [E weight tensor maps]
+// split-tile partials of the tiles] [E weight tensor maps]
 // [schedule: W, W / grid, W % grid, status, m_tiles[E+1], first tile[E+1],
 // first row[E+1]], every part 256-byte aligned.
 struct GroupedLayout {
@@ -340,7 +296,7 @@ struct GroupedLayout {
 GroupedLayout grouped_layout(int32_t E, const DeviceInfo& dev) {
     GroupedLayout L;
     L.grid = dev.sms;
-    L.gemm_bytes = 4096 + L.grid * 128 * int64_t(w4a8::gemm::wide_token_tile()) * 4;
+    L.gemm_bytes = 4096 + L.grid * 128 * 128 * 4;  // counters, then one 128 x 128 int32 partial per CTA
     L.maps_off = align256(L.gemm_bytes);
     L.sched_off = L.maps_off + align256(int64_t(E) * 128);
     L.total = L.sched_off + align256((4 + 3 * (int64_t(E) + 1)) * 4);
@@ -546,17 +502,10 @@ int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32_t group,
     DeviceInfo dev;
     if (current_device(dev) != W4A8_OK) return -1;
     const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms, path == 2);
-    if (gemv_path(M, N, K, path == 2, false)) {  // no workspace; the asymmetric GEMM (path 0) runs tiles
-        if (path != 0) return 0;
-        const w4a8::gemm::Plan pn = w4a8::gemm::make_plan(M, N, K, group, dev.sms, false, true);
-        return plan_splits_tiles(pn) ? pn.ws_bytes : 0;
-    }
-    int64_t need = plan_splits_tiles(pl) ? pl.ws_bytes : 0;
-    if (path == 0 && pl.wide) {  // the asymmetric-token GEMM (path 0 too) runs narrow tiles
-        const w4a8::gemm::Plan pn = w4a8::gemm::make_plan(M, N, K, group, dev.sms, false, true);
-        if (plan_splits_tiles(pn) && pn.ws_bytes > need) need = pn.ws_bytes;
-    }
-    return need;
+    // the decode kernel takes no workspace; the asymmetric-token GEMM (path 0
+    // too) always runs the tiles, so path 0 returns their size
+    if (gemv_path(M, N, K, path == 2, false) && path != 0) return 0;
+    return plan_splits_tiles(pl) ? pl.ws_bytes : 0;
 }
 
 w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, const uint8_t* w_packed, const int16_t* S,
@@ -692,82 +641,46 @@ w4a8_status w4a8_gemm_intscale_grouped(const int8_t* q_x, const float* s_a, int6
     const float inv_alpha = std::ldexp(1.0f, -int(std::log2(double(alpha))));
     const int32_t y_kind = y_dtype == W4A8_F16 ? w4a8::gemm::kOutF16
                                                : (y_dtype == W4A8_I32 ? w4a8::gemm::kOutI32 : w4a8::gemm::kOutF32);
-    if (!row_index) {
-        // routed-order codes: the tiles of w4a8_gemm_intscale (token tile 128),
-        // each tile's rows read as one box.  Tensor maps: a template for the
-        // experts' packed weights (its address is replaced per expert on the
-        // device) and the codes [T][K].
-        CUtensorMap tm_w, tm_x;
-        if (!make_map_u8(&tm_w, workspace, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2),
-                         uint32_t(w4a8::gemm::weight_box_bytes()), 128, CU_TENSOR_MAP_SWIZZLE_128B))
-            return W4A8_ERR_CUDA;
-        if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(T), uint64_t(K), 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
-            return W4A8_ERR_CUDA;
-        w4a8::gemm::ParamsGr g{};
-        g.s_a = s_a;
-        g.y = y;
-        g.ws_count = reinterpret_cast<int32_t*>(ws);
-        g.ws_part = reinterpret_cast<int32_t*>(ws + 4096);
-        g.status = dev.status;
-        g.M = 0;
-        g.N = N;
-        g.G = K / group;
-        g.kb_per_group = group / 128;
-        g.grid = L.grid;
-        g.inv_alpha = inv_alpha;
-        g.y_dtype = y_kind;
-        g.wait_limit = g_wait_limit.load();
-        g.grp_sched = reinterpret_cast<const int32_t*>(ws + L.sched_off);
-        g.grp_maps = reinterpret_cast<const CUtensorMap*>(ws + L.maps_off);
-        g.grp_scales = reinterpret_cast<const void* const*>(S);
-        g.out_row = out_row;
-        g.y_rows = out_row ? y_rows : R;
-        g.E = E;
-        g.n_tiles = int32_t((N + 127) / 128);
-        W4A8_CUDA_TRY(w4a8::gemm::launch_grouped(tm_w, tm_x, expert_offsets,
-                                                 reinterpret_cast<const void* const*>(w_packed), R, g,
-                                                 reinterpret_cast<int32_t*>(ws + L.sched_off),
-                                                 reinterpret_cast<CUtensorMap*>(ws + L.maps_off),
-                                                 static_cast<cudaStream_t>(stream)));
-        return W4A8_OK;
-    }
-    // rows gathered by index: the wide-tile kernel, four rows per copy (a box
-    // one row high).  Tensor maps: the experts' weight template and the codes.
+    // The tiles of w4a8_gemm_intscale (token tile 128) in grouped mode.
+    // Tensor maps: a template for the experts' packed weights (its address is
+    // replaced per expert on the device), and the codes [T][K]: boxes of 128
+    // rows for routed-order codes, one row high for rows gathered by index
+    // (four rows per copy).
     CUtensorMap tm_w, tm_x;
-    if (!make_map_u8(&tm_w, workspace, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), 64, 128,
-                     CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!make_map_u8(&tm_w, workspace, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2),
+                     uint32_t(w4a8::gemm::weight_box_bytes()), 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return W4A8_ERR_CUDA;
-    if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(T), uint64_t(K), 128, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_map_u8(&tm_x, q_x, uint64_t(K), uint64_t(T), uint64_t(K), 128, row_index ? 1u : 128u,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
         return W4A8_ERR_CUDA;
-    w4a8::gemm::WideParams q{};
-    q.s_a = s_a;
-    q.y = y;
-    q.ws_count = reinterpret_cast<int32_t*>(ws);
-    q.ws_part = reinterpret_cast<int32_t*>(ws + 4096);
-    q.status = dev.status;
-    q.M = 0;
-    q.N = int32_t(N);
-    q.G = int32_t(K / group);
-    q.kb_per_group = group / 128;
-    q.n_tiles = int32_t((N + 127) / 128);
-    q.m_tiles = 0;
-    q.grid = int32_t(L.grid);
-    q.inv_alpha = inv_alpha;
-    q.y_dtype = y_kind;
-    q.row_index = row_index;
-    q.out_row = out_row;
-    q.moe_scales = reinterpret_cast<const void* const*>(S);
-    q.moe_sched = reinterpret_cast<const int32_t*>(ws + L.sched_off);
-    q.moe_maps = reinterpret_cast<const CUtensorMap*>(ws + L.maps_off);
-    q.E = E;
-    q.moe_T = int32_t(T);
-    q.y_rows = out_row ? y_rows : R;
-    q.wait_limit = g_wait_limit.load();
-    W4A8_CUDA_TRY(w4a8::gemm::launch_wide_moe(tm_w, tm_x, expert_offsets,
-                                              reinterpret_cast<const void* const*>(w_packed), R, q,
-                                              reinterpret_cast<int32_t*>(ws + L.sched_off),
-                                              reinterpret_cast<CUtensorMap*>(ws + L.maps_off),
-                                              static_cast<cudaStream_t>(stream)));
+    w4a8::gemm::ParamsGr g{};
+    g.s_a = s_a;
+    g.y = y;
+    g.ws_count = reinterpret_cast<int32_t*>(ws);
+    g.ws_part = reinterpret_cast<int32_t*>(ws + 4096);
+    g.status = dev.status;
+    g.M = 0;
+    g.N = N;
+    g.G = K / group;
+    g.kb_per_group = group / 128;
+    g.grid = L.grid;
+    g.inv_alpha = inv_alpha;
+    g.y_dtype = y_kind;
+    g.wait_limit = g_wait_limit.load();
+    g.grp_sched = reinterpret_cast<const int32_t*>(ws + L.sched_off);
+    g.grp_maps = reinterpret_cast<const CUtensorMap*>(ws + L.maps_off);
+    g.grp_scales = reinterpret_cast<const void* const*>(S);
+    g.out_row = out_row;
+    g.row_index = row_index;
+    g.y_rows = out_row ? y_rows : R;
+    g.E = E;
+    g.n_tiles = int32_t((N + 127) / 128);
+    g.T = int32_t(T);
+    W4A8_CUDA_TRY(w4a8::gemm::launch_grouped(tm_w, tm_x, expert_offsets,
+                                             reinterpret_cast<const void* const*>(w_packed), R, g,
+                                             reinterpret_cast<int32_t*>(ws + L.sched_off),
+                                             reinterpret_cast<CUtensorMap*>(ws + L.maps_off),
+                                             static_cast<cudaStream_t>(stream)));
     return W4A8_OK;
 }
 

@@ -363,8 +363,9 @@ __device__ __forceinline__ float output_scale(const Params& p, int64_t m) {
 // in a loop with no per-stage bookkeeping.
 // GR: a grouped (mixture-of-experts) call: tiles expert by expert from a
 // schedule in the workspace, each expert's weights through its own tensor
-// map, token rows as blocks of routed-order codes, outputs one row at a time.
-template <int BT, int PATH, bool W8, bool ZP, bool G1, bool GR = false>
+// map, outputs one row at a time; token rows as blocks of routed-order codes,
+// or (GATHER) gathered from q_x by a row index.
+template <int BT, int PATH, bool W8, bool ZP, bool G1, bool GR = false, bool GATHER = false>
 __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH, W8, ZP>::kCtasPerSm)
     w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                      const __grid_constant__ CUtensorMap tm_y,
@@ -490,10 +491,31 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
         StageIter<GR> it(p, pt, b);
         Stage st;
         bool ok = true;
+        // a grouped call with a row index: the tokens of the tile's routed rows
+        // 4 lane .. 4 lane + 3, gathered four rows per copy (rows past the
+        // expert's last, and indices outside [0, T), read token 0: their
+        // outputs are not stored or are zeroed)
+        int32_t trow[4] = {0, 0, 0, 0};
+        int32_t t_e = -1, t_n = -1, t_m = -1;
         while (ok && it.next(st)) {
             // first token row of the tile (a grouped call: of the expert's routed rows)
             int32_t m0 = st.m_tile * BT;
-            if constexpr (GR) m0 += grsched_of(p).rstart[st.e];
+            if constexpr (GR) {
+                const GrSched gs = grsched_of(p);
+                m0 += gs.rstart[st.e];
+                if (GATHER && (st.e != t_e || st.n_tile != t_n || st.m_tile != t_m)) {
+                    t_e = st.e;
+                    t_n = st.n_tile;
+                    t_m = st.m_tile;
+                    const int32_t rend = gs.rstart[st.e + 1];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int32_t r = m0 + 4 * lane + q;
+                        const int32_t tk = r < rend ? p.row_index[r] : 0;
+                        trow[q] = (tk >= 0 && tk < p.T) ? tk : 0;
+                    }
+                }
+            }
             if (pst >= prefetched) {
                 bool free_slot;
                 if constexpr (C::kW8) {
@@ -518,10 +540,20 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                 rxd.advance(SD);
             }
             mbar_arrive_expect_tx_one(&full_x[rx.idx], uint32_t(st.nkb * BT * kBlockK));
-            tma_load_2d_one(smem + C::offX + rx.idx * C::kXBytes, &tm_x, st.kb * kBlockK, m0, &full_x[rx.idx]);
-            if (st.nkb == 2)
-                tma_load_2d_one(smem + C::offX + rx.idx * C::kXBytes + BT * kBlockK, &tm_x, (st.kb + 1) * kBlockK,
-                                m0, &full_x[rx.idx]);
+            if constexpr (GATHER) {
+                // every lane gathers its four rows of each K block (box one row high)
+                __syncwarp();
+                uint8_t* xdst = smem + C::offX + rx.idx * C::kXBytes + 4 * lane * kBlockK;
+                tma_gather4(xdst, &tm_x, st.kb * kBlockK, trow[0], trow[1], trow[2], trow[3], &full_x[rx.idx]);
+                if (st.nkb == 2)
+                    tma_gather4(xdst + BT * kBlockK, &tm_x, (st.kb + 1) * kBlockK, trow[0], trow[1], trow[2],
+                                trow[3], &full_x[rx.idx]);
+            } else {
+                tma_load_2d_one(smem + C::offX + rx.idx * C::kXBytes, &tm_x, st.kb * kBlockK, m0, &full_x[rx.idx]);
+                if (st.nkb == 2)
+                    tma_load_2d_one(smem + C::offX + rx.idx * C::kXBytes + BT * kBlockK, &tm_x,
+                                    (st.kb + 1) * kBlockK, m0, &full_x[rx.idx]);
+            }
             x_issued |= 1u << rx.idx;
             x_par = (x_par & ~(1u << rx.idx)) | (rx.phase << rx.idx);
             rx.advance(SX);
@@ -726,7 +758,23 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             {
                 const int te = ew * 32 + lane;
                 const int64_t mt = mbase + te;
-                if (te < BT && mt < mend) sa_pref = output_scale<PATH>(p, mt);
+                if constexpr (GR) {
+                    // a grouped call: the scale of the routed row (routed-order
+                    // codes) or of its token (a row index); a token outside
+                    // [0, T) marks the row (NaN scale): its outputs are zeroed
+                    if (te < BT && mt < mend) {
+                        int64_t tok = mt;
+                        if constexpr (GATHER) tok = p.row_index[mt];
+                        if (tok >= 0 && tok < p.T) {
+                            sa_pref = output_scale<PATH>(p, tok);
+                        } else {
+                            sa_pref = __int_as_float(0x7fc00000);
+                            atomicExch(p.status, kStatusInvalidArg);
+                        }
+                    }
+                } else {
+                    if (te < BT && mt < mend) sa_pref = output_scale<PATH>(p, mt);
+                }
                 if constexpr (ZP) {
                     if (te < BT && mt < mend) z_pref = p.z_a[mt];
                     if (nvalid) zc_n = p.zc[n];
@@ -1080,6 +1128,16 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             {
                 const int base = half * HC * kTileN + r;  // element index of (token half*HC, column r)
                 const float* sa = sa_tile + half * HC;
+                if constexpr (GR) {
+                    // rows marked invalid (NaN scale) are written as zeros
+#pragma unroll
+                    for (int j = 0; j < HC; ++j) {
+                        if (sa[j] != sa[j]) {
+                            acc[j] = 0;
+                            accf[j] = 0.0f;
+                        }
+                    }
+                }
                 if (p.y_dtype == kOutI32) {
                     int32_t* yo = reinterpret_cast<int32_t*>(smem + C::offY) + base;
 #pragma unroll
@@ -1089,12 +1147,13 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
 #pragma unroll
                     for (int j = 0; j < HC; ++j)
                         yo[j * kTileN] = __float2half_rn(
-                            __fmul_rn(PATH == kIntScale ? __int2float_rn(acc[j]) : accf[j], sa[j]));
+                            __fmul_rn(PATH == kIntScale ? __int2float_rn(acc[j]) : accf[j], GR && sa[j] != sa[j] ? 0.0f : sa[j]));
                 } else {
                     float* yo = reinterpret_cast<float*>(smem + C::offY) + base;
 #pragma unroll
                     for (int j = 0; j < HC; ++j)
-                        yo[j * kTileN] = __fmul_rn(PATH == kIntScale ? __int2float_rn(acc[j]) : accf[j], sa[j]);
+                        yo[j * kTileN] = __fmul_rn(PATH == kIntScale ? __int2float_rn(acc[j]) : accf[j],
+                                                   GR && sa[j] != sa[j] ? 0.0f : sa[j]);
                 }
             }
             fence_proxy_async_smem();  // the staged outputs, visible to the TMA unit
@@ -1146,19 +1205,15 @@ static int token_tile_for(int64_t M) {
     return 128;
 }
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool w8, bool narrow_only) {
+Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool w8) {
     Plan pl{};
-    // dense GEMMs run the tiles of this kernel at every M (measured faster
-    // than the wide-tile kernel, which serves the grouped expert call)
-    (void)narrow_only;
-    pl.wide = false;
-    pl.BT = pl.wide ? wide_token_tile() : token_tile_for(M);
+    pl.BT = token_tile_for(M);
     pl.n_tiles = (N + kTileN - 1) / kTileN;
     pl.m_tiles = (M + pl.BT - 1) / pl.BT;
     pl.G = K / group;
     pl.tiles = pl.n_tiles * pl.m_tiles;
     pl.W = pl.tiles * pl.G;
-    const int64_t slots = int64_t(num_sms) * ((w8 || pl.wide) ? 1 : W4A8_CTAS_PER_SM(pl.BT));  // resident CTAs
+    const int64_t slots = int64_t(num_sms) * (w8 ? 1 : W4A8_CTAS_PER_SM(pl.BT));  // resident CTAs
     pl.grid = pl.W < slots ? pl.W : slots;
     if (pl.grid > kMaxGrid) pl.grid = kMaxGrid;
     const int64_t slot_bytes = int64_t(kTileN) * pl.BT * 4;
@@ -1229,7 +1284,15 @@ cudaError_t launch_grouped(const CUtensorMap& tm_w_template, const CUtensorMap& 
     if (e != cudaSuccess) return e;
     using C = Cfg<128, kIntScale, false, false>;
     // tm_y is not read by a grouped call (its rows are stored one by one)
-    if (p.kb_per_group == 1)
+    const bool g1 = p.kb_per_group == 1;
+    if (p.row_index != nullptr) {
+        if (g1)
+            return launch_k<w4a8_gemm_kernel<128, kIntScale, false, false, true, true, true>>(
+                C::kThreads, C::kSmemBytes, tm_w_template, tm_x, tm_x, p, stream);
+        return launch_k<w4a8_gemm_kernel<128, kIntScale, false, false, false, true, true>>(
+            C::kThreads, C::kSmemBytes, tm_w_template, tm_x, tm_x, p, stream);
+    }
+    if (g1)
         return launch_k<w4a8_gemm_kernel<128, kIntScale, false, false, true, true>>(C::kThreads, C::kSmemBytes,
                                                                                     tm_w_template, tm_x, tm_x, p,
                                                                                     stream);

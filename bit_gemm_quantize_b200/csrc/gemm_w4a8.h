@@ -47,39 +47,13 @@ struct ParamsGr : Params {
     const CUtensorMap* grp_maps;    // [E] weight tensor maps (built by the setup kernel)
     const void* const* grp_scales;  // [E] device pointers to each expert's S [G, N]
     const int32_t* out_row;         // [R] output row of each routed row, or null (row i)
+    const int32_t* row_index;       // [R] token of each routed row (rows gathered from q_x), or null (row i of q_x)
     int64_t y_rows;                 // rows of y: an output row must lie below it
     int32_t E;
     int32_t n_tiles;
+    int32_t T;                      // rows of q_x / s_a: a token index must lie in [0, T)
 };
 
-// Parameters of the wide-tile kernel (token tiles of 256; gemm_wide.cu).
-struct WideParams {
-    const float* s_a;    // [M] token scales (MOE: [T], indexed by token)
-    const int16_t* S;    // [G, N] integer group scales (dense integer-scale path)
-    const float* s_g;    // [G, N] float group scales (float-scale path)
-    void* y;             // [M, N] output (MOE: [rows, N], row out_row[i] or i)
-    int32_t* ws_part;    // [grid][128 * 256] partial sums of split tiles
-    int32_t* ws_count;   // [grid] arrival counters, zero between calls
-    int* status;         // device status word
-    int32_t M, N;
-    int32_t G;           // groups along K
-    int32_t kb_per_group;
-    int32_t n_tiles, m_tiles;
-    int32_t grid;
-    uint32_t W, w_q, w_r;  // (tile, group) steps, W / grid, W % grid (dense; MOE: moe_sched)
-    float inv_alpha;
-    int32_t y_dtype;
-    // mixture of experts
-    const int32_t* row_index;      // [R] token of each routed row, rows grouped by expert
-    const int32_t* out_row;        // [R] output row of each routed row, or null (row i)
-    const void* const* moe_scales; // [E] device pointers to each expert's S [G, N]
-    const int32_t* moe_sched;      // W, w_q, w_r, status, then mt[E+1], tstart[E+1], rstart[E+1]
-    const CUtensorMap* moe_maps;   // [E] weight tensor maps
-    int32_t E;
-    int32_t moe_T;                 // tokens: row_index values must lie in [0, T)
-    int64_t y_rows;                // rows of y (MOE): a routed row's output row must be below it
-    long long wait_limit;          // SM cycles a pipeline or split-tile wait may last before it gives up
-};
 
 }  // namespace gemm
 
@@ -126,7 +100,6 @@ cudaError_t launch(const CUtensorMap& tm_w, const GemvParams& p, int path, int x
 namespace gemm {
 
 struct Plan {
-    bool wide;           // the wide-tile kernel (token tiles of wide_token_tile())
     int BT;              // tokens per tile (MMA N)
     int64_t n_tiles, m_tiles, tiles, G, W, grid;
     int64_t count_bytes;  // bytes of the fixed counter region at the start of the workspace
@@ -134,9 +107,7 @@ struct Plan {
 };
 
 // w8: int8 weight codes (the W8A8 variant); its CTAs run one per SM
-// narrow_only: tiles of at most 128 tokens whatever M (the asymmetric-token kernel)
-Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool w8 = false,
-               bool narrow_only = false);
+Plan make_plan(int64_t M, int64_t N, int64_t K, int32_t group, int num_sms, bool w8 = false);
 
 // tm_w: packed weights [N][K/2] u8, box 128 B x 128 rows, 128-byte swizzle
 // tm_x: token codes [M][K] u8, box 128 B x BT rows, 128-byte swizzle
@@ -150,35 +121,20 @@ cudaError_t launch(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUten
 cudaError_t launch_zp(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap& tm_y, const ParamsZp& p,
                       int BT, cudaStream_t stream);
 
-// Wide-tile kernel (token tiles of 256, gemm_wide.cu), integer- or float-scale path.
-// tm_w: packed weights [N][K/2] u8, box 64 B x 128 rows, no swizzle
-// tm_x: token codes [M][K] u8, box 128 B x 256 rows, 128-byte swizzle
-// tm_y: output [M][N], box 128 columns x wide_token_tile() rows (fp16) or wide_tail_rows() (4-byte outputs)
-cudaError_t launch_wide(const CUtensorMap& tm_w, const CUtensorMap& tm_x, const CUtensorMap& tm_y, const WideParams& p,
-                        int path, cudaStream_t stream);
-// Mixture of experts (integer-scale path): a setup kernel builds the schedule
-// and the per-expert weight maps from device offsets and pointers, then the
-// wide kernel runs over all experts' tiles.  tm_w_template: a weight map of
-// the experts' shape (its address is replaced per expert); tm_x: token codes
-// [T][K] u8, box 128 B x 1 row, 128-byte swizzle (rows gathered four at a time).
 // A grouped call on the tiles of gemm_w4a8.cu (token tile 128): the setup
 // kernel, then the GEMM, chained with programmatic dependent launch.
 // tm_w_template: a packed-weight map of the tiles' box (128 rows x 128 B,
 // 128-byte swizzle) whose address the setup kernel replaces per expert;
-// tm_x: the routed-order codes [R][K], box 128 rows x 128 B.
+// tm_x: the codes [T][K], box 128 B x 128 rows (routed-order codes) or
+// 128 B x 1 row (rows gathered by p.row_index, four per copy).
 cudaError_t launch_grouped(const CUtensorMap& tm_w_template, const CUtensorMap& tm_x, const int64_t* offsets,
                            const void* const* w_ptrs, int64_t R, const ParamsGr& p, int32_t* sched,
                            CUtensorMap* maps, cudaStream_t stream);
-// The setup kernel of a grouped call (gemm_wide.cu), for token tiles of `bt`.
+// The setup kernel of a grouped call (grouped_setup.cu), for token tiles of `bt`.
 cudaError_t launch_grouped_setup(const CUtensorMap& tm_w_template, const int64_t* offsets, const void* const* w_ptrs,
                                  const void* const* s_ptrs, int32_t E, int64_t R, int32_t bt, int32_t n_tiles,
                                  int32_t G, int32_t grid, int32_t* sched, CUtensorMap* maps, int* status,
                                  cudaStream_t stream);
-cudaError_t launch_wide_moe(const CUtensorMap& tm_w_template, const CUtensorMap& tm_x, const int64_t* offsets,
-                            const void* const* w_ptrs, int64_t R, const WideParams& p, int32_t* sched,
-                            CUtensorMap* maps, cudaStream_t stream);
-int wide_token_tile();
-int wide_tail_rows();  // output rows per tail pass of 4-byte outputs
 
 int token_tile_rows();
 

@@ -379,11 +379,13 @@ W4A8_API w4a8_status w4a8_gemm_intscale_static_ws(const int8_t* q_x, const float
  * Everything the routing decides is read on the device, so a router kernel
  * earlier in the stream can produce it without a host round trip: a small
  * setup kernel turns the offsets into the schedule and each expert's weight
- * tensor map (in the workspace), then one persistent launch covers every
- * (expert, tile, group) step.  Token rows are fetched from q_x by index (no
- * gathered copy is made), or, with row_index NULL, q_x holds the routed rows
- * themselves (quantize_act_routed) and each tile's rows are read as one block
- * (measured about a third less time on a Mixtral-shaped layer).
+ * tensor map (in the workspace), then one persistent launch of the
+ * w4a8_gemm_intscale tiles covers every (expert, tile, group) step.  Token
+ * rows are gathered from q_x by index, four rows per copy (no gathered copy
+ * is made), or, with row_index NULL, q_x holds the routed rows themselves
+ * (quantize_act_routed) and each tile's rows are read as one block (measured
+ * about half the time on a Mixtral-shaped layer: the four-row copies bound
+ * the gathered form).
  * q_x, s_a   device, [T, K] int8 and [T] float32: every token quantized once
  *            (quantize_act_per_token), or, with row_index NULL, the routed rows
  *            (T >= R; quantize_act_routed); q_x 16-byte, s_a 4-byte aligned
