@@ -758,13 +758,12 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             {
                 const int te = ew * 32 + lane;
                 const int64_t mt = mbase + te;
-                if constexpr (GR) {
-                    // a grouped call: the scale of the routed row (routed-order
-                    // codes) or of its token (a row index); a token outside
-                    // [0, T) marks the row (NaN scale): its outputs are zeroed
+                if constexpr (GATHER) {
+                    // rows gathered by index: the scale of the row's token; a
+                    // token outside [0, T) marks the row (NaN scale): its
+                    // outputs are zeroed
                     if (te < BT && mt < mend) {
-                        int64_t tok = mt;
-                        if constexpr (GATHER) tok = p.row_index[mt];
+                        const int64_t tok = p.row_index[mt];
                         if (tok >= 0 && tok < p.T) {
                             sa_pref = output_scale<PATH>(p, tok);
                         } else {
@@ -1128,7 +1127,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             {
                 const int base = half * HC * kTileN + r;  // element index of (token half*HC, column r)
                 const float* sa = sa_tile + half * HC;
-                if constexpr (GR) {
+                if constexpr (GATHER) {
                     // rows marked invalid (NaN scale) are written as zeros
 #pragma unroll
                     for (int j = 0; j < HC; ++j) {
@@ -1147,13 +1146,13 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
 #pragma unroll
                     for (int j = 0; j < HC; ++j)
                         yo[j * kTileN] = __float2half_rn(
-                            __fmul_rn(PATH == kIntScale ? __int2float_rn(acc[j]) : accf[j], GR && sa[j] != sa[j] ? 0.0f : sa[j]));
+                            __fmul_rn(PATH == kIntScale ? __int2float_rn(acc[j]) : accf[j], GATHER && sa[j] != sa[j] ? 0.0f : sa[j]));
                 } else {
                     float* yo = reinterpret_cast<float*>(smem + C::offY) + base;
 #pragma unroll
                     for (int j = 0; j < HC; ++j)
                         yo[j * kTileN] = __fmul_rn(PATH == kIntScale ? __int2float_rn(acc[j]) : accf[j],
-                                                   GR && sa[j] != sa[j] ? 0.0f : sa[j]);
+                                                   GATHER && sa[j] != sa[j] ? 0.0f : sa[j]);
                 }
             }
             fence_proxy_async_smem();  // the staged outputs, visible to the TMA unit
