@@ -1094,7 +1094,7 @@ def run_ours(args):
 # DRAM bytes (read + write) per launch of the integer-scale GEMM, from one
 # ncu capture of `bench.py --case gemm_is --M <M>`, valid for the kernel source
 # it was taken with (first 16 hex digits of the SHA-256 of the files below).
-MEASURED_TRAFFIC = {1024: (55.277824e6 + 16.712704e6, "d49d23f51ef9a3dd")}
+MEASURED_TRAFFIC = {1024: (55.618304e6 + 18.213376e6, "9506e380e14de685")}
 GEMM_SOURCES = ("gemm_w4a8.cu", "gemm_w4a8.h", "gemm_common.cuh", "sm100_ptx.cuh")
 
 

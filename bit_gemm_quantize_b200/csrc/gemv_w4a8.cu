@@ -46,6 +46,9 @@
 namespace w4a8 {
 namespace gemv {
 
+#ifndef W4A8_GEMV_WARPS_PER_SM
+#define W4A8_GEMV_WARPS_PER_SM 24  // target warps per SM of the launch shape
+#endif
 #ifndef W4A8_GEMV_INTERLEAVE
 #define W4A8_GEMV_INTERLEAVE 1
 #endif
@@ -360,7 +363,7 @@ static void shape(const GemvParams& p, int mt, int sub, int num_sms, int& ks, in
     // CTAs each SM holds: the whole grid at once if the shared memory allows,
     // else fewer (more waves)
     for (int per_sm = int((blocks + num_sms - 1) / num_sms);; --per_sm) {
-        ks = 24 / per_sm;
+        ks = W4A8_GEMV_WARPS_PER_SM / per_sm;
         ks = ks > 16 ? 16 : (ks < 1 ? 1 : ks);
         ks = ks > nkb_total ? nkb_total : ks;
         for (; ks >= 1; --ks) {
