@@ -813,7 +813,7 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             if constexpr (kLean) {
                 // One group per K block, each committed to its own accumulator
                 // buffer: wait for the group's MMAs, load this thread's HC
-                // columns of P_g in one TMEM load, hand the buffer back, then
+                // columns of P_g, hand the buffer back, and add
                 // acc += S[g,n] * P_g (or accf += s_g * float(P_g)).  This
                 // column's scale is read from global memory two groups ahead
                 // (a column past N reads column 0's scales: its outputs are
@@ -843,26 +843,36 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                         break;
                     }
                     tc_fence_after();
-                    uint32_t v[HC];
-                    tmem_load<HC>(lane_cols + uint32_t(rt.idx * BT), v);
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    __syncwarp();
-                    mbar_arrive_one(&tempty[rt.idx]);
-                    rt.advance(kAcc);
-                    if constexpr (PATH == kIntScale) {
-                        const int32_t s_cur = int32_t(sraw);
+                    // in two halves (load, multiply-add, load, multiply-add):
+                    // the two epilogue warps of an SM sub-partition then drift
+                    // apart, one loading while the other multiplies (measured
+                    // 3% faster at M = 1024 than one load of all HC columns)
+                    constexpr int H = HC / 2;
 #pragma unroll
-                        for (int q = 0; q < HC; ++q) {
-                            const int32_t pg = C::kX16 ? (int32_t(v[q]) >> 4) : int32_t(v[q]);  // exact
-                            acc[q] += s_cur * pg;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t v[H];
+                        tmem_load<H>(lane_cols + uint32_t(rt.idx * BT + hh * H), v);
+                        tmem_wait_ld();
+                        if (hh == 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            mbar_arrive_one(&tempty[rt.idx]);
+                            rt.advance(kAcc);
                         }
-                    } else {
-                        const float f_cur = C::kX16 ? __fmul_rn(__uint_as_float(sraw), 0.0625f)  // P_g was 16 P_g
-                                                    : __uint_as_float(sraw);
+                        if constexpr (PATH == kIntScale) {
+                            const int32_t s_cur = int32_t(sraw);
 #pragma unroll
-                        for (int q = 0; q < HC; ++q)
-                            accf[q] = __fmaf_rn(f_cur, __int2float_rn(int32_t(v[q])), accf[q]);
+                            for (int q = 0; q < H; ++q) {
+                                const int32_t pg = C::kX16 ? (int32_t(v[q]) >> 4) : int32_t(v[q]);  // exact
+                                acc[hh * H + q] += s_cur * pg;
+                            }
+                        } else {
+                            const float f_cur = C::kX16 ? __fmul_rn(__uint_as_float(sraw), 0.0625f)
+                                                        : __uint_as_float(sraw);
+#pragma unroll
+                            for (int q = 0; q < H; ++q)
+                                accf[hh * H + q] = __fmaf_rn(f_cur, __int2float_rn(int32_t(v[q])), accf[hh * H + q]);
+                        }
                     }
                 }
             } else {
