@@ -157,7 +157,8 @@ w4a8_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int32_t group) {
 // most 32 MB (measured: past that the tensor-core tiles, which do a quarter of
 // the instructions per weight byte, are faster at four tokens).
 bool gemv_fits(int64_t M, int64_t K, bool w8, bool zp) {
-    return !w8 && !zp && M >= 1 && M <= w4a8::gemv::kMaxM && K >= w4a8::gemv::kMinK && K <= w4a8::gemv::kMaxK;
+    (void)zp;  // asymmetric token codes: the kernel subtracts z[m] * zc[n] from each accumulator
+    return !w8 && M >= 1 && M <= w4a8::gemv::kMaxM && K >= w4a8::gemv::kMinK && K <= w4a8::gemv::kMaxK;
 }
 bool gemv_path(int64_t M, int64_t N, int64_t K, bool w8, bool zp) {
     return gemv_fits(M, K, w8, zp) && (M <= 2 || N * (K / 2) <= (int64_t(32) << 20));
@@ -213,6 +214,10 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
         g.inv_alpha = path == w4a8::gemm::kIntScale ? std::ldexp(1.0f, -int(std::log2(double(alpha)))) : 1.0f;
         g.status = dev.status;
         g.wait_limit = g_wait_limit.load();
+        if (zp) {
+            g.z_a = z_a;
+            g.zc = zc;
+        }
         CUtensorMap tm;
         if (!gemv_weight_map(&tm, w_packed, N, K, M)) return W4A8_ERR_CUDA;
         W4A8_CUDA_TRY(

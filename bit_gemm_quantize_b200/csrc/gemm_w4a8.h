@@ -89,6 +89,8 @@ struct GemvParams {
     int* status;           // device status word (a ring wait that runs out)
     long long wait_limit;  // SM cycles a ring wait may last
     int32_t stages;        // ring slots per warp (set by the launcher)
+    const int32_t* z_a;    // asymmetric token codes: [M] zero points (with zc; integer-scale path), or null
+    const int32_t* zc;     // [N] zero-point term of each column
 };
 
 int smem_bytes(int mt, int K, int ks, int stages, int sub);

@@ -318,6 +318,11 @@ __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUten
             else
                 af = __fadd_rn(af, redf[(w * MT + m) * kCols + lane]);
         }
+        if constexpr (PATH == gemm::kIntScale) {
+            // asymmetric token codes: acc - z[m] * zc[n] in two's-complement
+            // arithmetic (the terms may wrap; the difference fits in 32 bits)
+            if (p.zc != nullptr) a = int32_t(uint32_t(a) - uint32_t(p.z_a[m]) * uint32_t(p.zc[n]));
+        }
         const float v = __fmul_rn(PATH == gemm::kIntScale ? __int2float_rn(a) : af, scl[m]);
         const int64_t o = int64_t(m) * N + n;
         if (p.y_dtype == gemm::kOutI32)

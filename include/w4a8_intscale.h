@@ -313,8 +313,10 @@ W4A8_API w4a8_status w4_zero_point_term(const uint8_t* w_packed, const int16_t* 
  *   acc[m,n] = sum_g S[g,n] * sum_{k in g} (q_x[m,k] - z_a[m]) q_w[k,n]
  *            = (the w4a8_gemm_intscale accumulator) - z_a[m] * zc[n]
  *   y[m,n]   = fl_out(fl32(acc) * fl32(s_a[m] / alpha))
- * The subtraction happens once per output, in the tile's final pass, in
- * two's-complement int32 arithmetic: the intermediate terms may wrap, the
+ * The subtraction happens once per output, in the final pass (of the tile,
+ * or of the decode kernel, which takes the same shapes as in
+ * w4a8_gemm_intscale), in two's-complement int32 arithmetic: the
+ * intermediate terms may wrap, the
  * result is exact when acc itself fits in int32, which holds when
  * 255*qw*group*max_n sum_g |S[g,n]| < 2^31 (255 = the widest |q_x - z_a|;
  * qw = 7, or 8 for codes in the full range [-8, 7]); w4_zero_point_term

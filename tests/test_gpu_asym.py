@@ -92,8 +92,14 @@ def test_zero_point_term_bitexact(K, N, qmin):
 
 
 ASYM_CASES = [
-    # M, K, N, offset: token tiles 16, 32, 64 and 128, ragged M and N, split tiles
+    # M, K, N, offset: the decode kernel (one to four tokens, its zero-point
+    # correction in the output step), token tiles 16, 32, 64 and 128, ragged M
+    # and N, split tiles
     (1, 256, 128, 1.0),
+    (2, 4096, 1032, 0.5),
+    (3, 1152, 264, -0.75),
+    (4, 2048, 520, 2.0),
+    (1, 4096, 22016, 1.0),
     (5, 1024, 264, 0.5),
     (16, 4096, 1024, 2.0),
     (33, 1024, 256, -1.0),
