@@ -153,23 +153,26 @@ w4a8_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int32_t group) {
 }
 
 // Decode-shaped calls (a few tokens) run on the CUDA cores (gemv_w4a8.cu):
-// one or two tokens always; three or four while the packed weights take at
-// most 32 MB (measured: past that the tensor-core tiles, which do a quarter of
-// the instructions per weight byte, are faster at four tokens).
+// one or two tokens always; three or four while the weights take at most
+// 32 MB (measured with 4-bit weights: past that the tensor-core tiles, which
+// do a quarter of the instructions per weight byte, are faster at four
+// tokens).  8-bit weight codes (w8) take the same kernel without the unpack.
 bool gemv_fits(int64_t M, int64_t K, bool w8, bool zp) {
     (void)zp;  // asymmetric token codes: the kernel subtracts z[m] * zc[n] from each accumulator
-    return !w8 && M >= 1 && M <= w4a8::gemv::kMaxM && K >= w4a8::gemv::kMinK && K <= w4a8::gemv::kMaxK;
+    (void)w8;
+    return M >= 1 && M <= w4a8::gemv::kMaxM && K >= w4a8::gemv::kMinK && K <= w4a8::gemv::kMaxK;
 }
 bool gemv_path(int64_t M, int64_t N, int64_t K, bool w8, bool zp) {
-    return gemv_fits(M, K, w8, zp) && (M <= 2 || N * (K / 2) <= (int64_t(32) << 20));
+    return gemv_fits(M, K, w8, zp) && (M <= 2 || N * (w8 ? K : K / 2) <= (int64_t(32) << 20));
 }
 
-// The decode kernel's weight map for M tokens: [N][K/2] bytes, boxes of 32 rows
-// x box_bytes(M) (one or two 128-wide K blocks of 32 columns), swizzled by the
-// box width.
-bool gemv_weight_map(CUtensorMap* m, const uint8_t* w_packed, int64_t N, int64_t K, int64_t M) {
-    const int box = w4a8::gemv::box_bytes(int(M));
-    return make_map_u8(m, w_packed, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2), uint32_t(box), 32,
+// The decode kernel's weight map for M tokens: [N][K/2] bytes (4-bit) or
+// [N][K] bytes (w8), boxes of 32 rows x box_bytes(M, w8) (one or two 128-wide
+// K blocks of 32 columns), swizzled by the box width.
+bool gemv_weight_map(CUtensorMap* m, const uint8_t* w_packed, int64_t N, int64_t K, int64_t M, bool w8 = false) {
+    const int box = w4a8::gemv::box_bytes(int(M), w8);
+    const uint64_t row = uint64_t(w8 ? K : K / 2);
+    return make_map_u8(m, w_packed, row, uint64_t(N), row, uint32_t(box), 32,
                        box == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -219,9 +222,12 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
             g.zc = zc;
         }
         CUtensorMap tm;
-        if (!gemv_weight_map(&tm, w_packed, N, K, M)) return W4A8_ERR_CUDA;
-        W4A8_CUDA_TRY(
-            w4a8::gemv::launch(tm, g, path, w4a8::gemv::kXCodes, dev.sms, static_cast<cudaStream_t>(stream)));
+        if (!gemv_weight_map(&tm, w_packed, N, K, M, w8)) return W4A8_ERR_CUDA;
+        if (w8)
+            W4A8_CUDA_TRY(w4a8::gemv::launch_w8(tm, g, dev.sms, static_cast<cudaStream_t>(stream)));
+        else
+            W4A8_CUDA_TRY(
+                w4a8::gemv::launch(tm, g, path, w4a8::gemv::kXCodes, dev.sms, static_cast<cudaStream_t>(stream)));
         return W4A8_OK;
     }
     const w4a8::gemm::Plan pl = w4a8::gemm::make_plan(M, N, K, group, dev.sms, w8);

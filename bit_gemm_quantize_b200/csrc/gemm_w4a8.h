@@ -70,14 +70,14 @@ constexpr int kMaxK = 16384;
 // 128-wide K blocks per box for one or two tokens; for three or four, where
 // the kernel does four times the arithmetic per byte, the smaller box lets
 // more warps share the SM).
-constexpr int box_bytes(int M) { return M <= 2 ? 128 : W4A8_GEMV_BOX_M4; }
+constexpr int box_bytes(int M, bool w8 = false) { return (M <= 2 || w8) ? 128 : W4A8_GEMV_BOX_M4; }
 enum XKind { kXCodes = 0, kXBf16 = 1, kXF32 = 2 };
 
 struct GemvParams {
     const void* x;         // int8 codes [M][K] (kXCodes) or bf16 / fp32 tokens [M][ldx] (quantized here)
     const float* s_a;      // [M] token scales (kXCodes)
     int64_t ldx;           // row pitch of x in elements (bf16 / fp32 tokens)
-    const uint8_t* w;      // packed int4 weights [N][K/2]
+    const uint8_t* w;      // packed int4 weights [N][K/2] (or 8-bit codes [N][K])
     const int16_t* S;      // [G][N] integer scales (integer-scale path)
     const float* s_g;      // [G][N] float scales (float-scale path)
     void* y;               // [M][N]
@@ -97,6 +97,9 @@ int smem_bytes(int mt, int K, int ks, int stages, int sub);
 // tm_w: packed weights [N][K/2] u8, box box_bytes(M) x 32 rows, swizzled by the box width
 cudaError_t launch(const CUtensorMap& tm_w, const GemvParams& p, int path, int x_kind, int num_sms,
                    cudaStream_t stream);
+// 8-bit weight codes (the W8A8 variant, integer scale, int8 token codes):
+// tm_w: w8 [N][K] int8, box 128 B x 32 rows, 128-byte swizzle
+cudaError_t launch_w8(const CUtensorMap& tm_w, const GemvParams& p, int num_sms, cudaStream_t stream);
 }  // namespace gemv
 
 namespace gemm {

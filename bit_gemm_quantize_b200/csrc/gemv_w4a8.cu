@@ -68,10 +68,14 @@ int smem_bytes(int mt, int K, int ks, int stages, int sub) {
            16;
 }
 
-template <int MT, int PATH, typename XT, int kSub>
+// W8: 8-bit weight codes [N][K] (the W8A8 variant): a 128-byte box is one
+// 128-wide K block, used as it lands (no unpack, no shift of P).
+template <int MT, int PATH, typename XT, int kSub, bool W8 = false>
 __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvParams p) {
     constexpr int kStage = stage_bytes(kSub);
     constexpr int kBoxBytes = 64 * kSub;
+    constexpr int kKB = W8 ? kSub / 2 : kSub;  // 128-wide K blocks per stage
+    static_assert(!W8 || (kSub == 2 && PATH == gemm::kIntScale && std::is_same<XT, int8_t>::value), "W8 form");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int K = p.K, N = p.N;
@@ -101,7 +105,7 @@ __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUten
     const int n0 = blockIdx.x * kCols;
     const int kbpg = p.group >> 7;  // 128-wide K blocks per group
     const int nkbt = K >> 7;
-    const int nstt = (nkbt + kSub - 1) / kSub;  // stages of the whole K
+    const int nstt = (nkbt + kKB - 1) / kKB;  // stages of the whole K
 #if W4A8_GEMV_INTERLEAVE
     // warp w takes stages w, w + ks, w + 2 ks, ...: at any time the CTA's
     // warps read neighbouring pieces of each column
@@ -209,10 +213,10 @@ __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUten
     }
     // the scales of stage jj's K blocks, loaded two stages ahead (0 past the
     // last block)
-    auto ld_scales = [&](int jj, uint32_t (&sc)[kSub]) {
+    auto ld_scales = [&](int jj, uint32_t (&sc)[kKB]) {
 #pragma unroll
-        for (int u = 0; u < kSub; ++u) {
-            const int kb = (s0 + jj * sstep) * kSub + u;
+        for (int u = 0; u < kKB; ++u) {
+            const int kb = (s0 + jj * sstep) * kKB + u;
             sc[u] = 0u;
             if (jj < nkb && kb < nkbt) {
                 const int64_t si = int64_t(kb / kbpg) * N + n_ld;
@@ -223,7 +227,7 @@ __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUten
             }
         }
     };
-    uint32_t sc0[kSub], sc1[kSub], sc2[kSub];
+    uint32_t sc0[kKB], sc1[kKB], sc2[kKB];
     ld_scales(0, sc0);
     ld_scales(1, sc1);
     bool ok = true;
@@ -236,23 +240,34 @@ __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUten
         }
         ld_scales(j + 2, sc2);
         const uint8_t* row = ring + slot * kStage + lane * kBoxBytes;
-        const int kbs = (s0 + j * sstep) * kSub;
+        const int kbs = (s0 + j * sstep) * kKB;
 #pragma unroll
-        for (int u = 0; u < kSub; ++u) {
+        for (int u = 0; u < kKB; ++u) {
             const int kb = kbs + u;
-            if (kSub > 1 && kb >= nkbt) break;  // the last stage of a K that is not a whole number of stages
-            // the block's 128 weights of this column as 16 q in int8 lanes,
-            // unpacked once for all tokens
+            if (kKB > 1 && kb >= nkbt) break;  // the last stage of a K that is not a whole number of stages
+            // the block's 128 weights of this column in int8 lanes (as 16 q,
+            // unpacked once for all tokens, or the 8-bit codes as they are)
             uint32_t wq[32];
+            if constexpr (W8) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4*>(row + (((4 * u + c) ^ sw) << 4));
-                const uint32_t pk[4] = {v.x, v.y, v.z, v.w};
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(row + ((c ^ sw) << 4));
+                    wq[4 * c] = v.x;
+                    wq[4 * c + 1] = v.y;
+                    wq[4 * c + 2] = v.z;
+                    wq[4 * c + 3] = v.w;
+                }
+            } else {
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const uint2 e = gemm::unpack_int4x8_x16(pk[h]);
-                    wq[8 * c + 2 * h] = e.x;
-                    wq[8 * c + 2 * h + 1] = e.y;
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(row + (((4 * u + c) ^ sw) << 4));
+                    const uint32_t pk[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const uint2 e = gemm::unpack_int4x8_x16(pk[h]);
+                        wq[8 * c + 2 * h] = e.x;
+                        wq[8 * c + 2 * h + 1] = e.y;
+                    }
                 }
             }
 #pragma unroll
@@ -272,10 +287,10 @@ __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUten
             // the group ends, or this warp's run of it: apply the group's
             // scale to the part summed so far (S times a partial sum is still
             // exact)
-            if ((kb + 1) % kbpg == 0 || u == kSub - 1 || kb + 1 == nkbt) {
+            if ((kb + 1) % kbpg == 0 || u == kKB - 1 || kb + 1 == nkbt) {
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
-                    const int32_t P = pg[m] >> 4;  // exact: every product is 16 q x
+                    const int32_t P = W8 ? pg[m] : pg[m] >> 4;  // exact: every 4-bit product is 16 q x
                     if constexpr (PATH == gemm::kIntScale)
                         acc[m] += int32_t(sc0[u]) * P;
                     else
@@ -291,7 +306,7 @@ __global__ void __launch_bounds__(512) gemv_kernel(const __grid_constant__ CUten
             phase ^= 1u;
         }
 #pragma unroll
-        for (int u = 0; u < kSub; ++u) {
+        for (int u = 0; u < kKB; ++u) {
             sc0[u] = sc1[u];
             sc1[u] = sc2[u];
         }
@@ -362,9 +377,10 @@ static int resident(int regs, int threads, int smem) {
 }
 
 template <auto kern>
-static void shape(const GemvParams& p, int mt, int sub, int num_sms, int& ks, int& stages, int& smem) {
+static void shape(const GemvParams& p, int mt, int sub, int kb_per_stage, int num_sms, int& ks, int& stages,
+                  int& smem) {
     const int64_t blocks = (p.N + kCols - 1) / kCols;
-    const int nkb_total = (p.K / 128 + sub - 1) / sub;  // stages of the whole K
+    const int nkb_total = (p.K / 128 + kb_per_stage - 1) / kb_per_stage;  // stages of the whole K
     // CTAs each SM holds: the whole grid at once if the shared memory allows,
     // else fewer (more waves)
     for (int per_sm = int((blocks + num_sms - 1) / num_sms);; --per_sm) {
@@ -391,14 +407,14 @@ static void shape(const GemvParams& p, int mt, int sub, int num_sms, int& ks, in
     smem = smem_bytes(mt, p.K, 1, 1, sub) + 1024;
 }
 
-template <int MT, int PATH, typename XT>
+template <int MT, int PATH, typename XT, bool W8 = false>
 static cudaError_t launch_t(const CUtensorMap& tm_w, const GemvParams& p, int num_sms, cudaStream_t stream) {
-    constexpr int sub = box_bytes(MT) / 64;
-    constexpr auto kern = gemv_kernel<MT, PATH, XT, sub>;
+    constexpr int sub = box_bytes(MT, W8) / 64;
+    constexpr auto kern = gemv_kernel<MT, PATH, XT, sub, W8>;
     cudaError_t e = configure_once<kern>(512, kSmemCap);
     if (e != cudaSuccess) return e;
     int ks = 1, stages = 1, smem = 0;
-    shape<kern>(p, MT, sub, num_sms, ks, stages, smem);
+    shape<kern>(p, MT, sub, W8 ? sub / 2 : sub, num_sms, ks, stages, smem);
     GemvParams q = p;
     q.stages = stages;
     const unsigned grid = unsigned((p.N + kCols - 1) / kCols);
@@ -406,13 +422,17 @@ static cudaError_t launch_t(const CUtensorMap& tm_w, const GemvParams& p, int nu
     return cudaLaunchKernelEx(&lc.cfg, kern, tm_w, q);
 }
 
-template <int PATH, typename XT>
+template <int PATH, typename XT, bool W8 = false>
 static cudaError_t launch_path(const CUtensorMap& tm_w, const GemvParams& p, int num_sms, cudaStream_t stream) {
     switch (p.M) {
-        case 1: return launch_t<1, PATH, XT>(tm_w, p, num_sms, stream);
-        case 2: return launch_t<2, PATH, XT>(tm_w, p, num_sms, stream);
-        default: return launch_t<4, PATH, XT>(tm_w, p, num_sms, stream);
+        case 1: return launch_t<1, PATH, XT, W8>(tm_w, p, num_sms, stream);
+        case 2: return launch_t<2, PATH, XT, W8>(tm_w, p, num_sms, stream);
+        default: return launch_t<4, PATH, XT, W8>(tm_w, p, num_sms, stream);
     }
+}
+
+cudaError_t launch_w8(const CUtensorMap& tm_w, const GemvParams& p, int num_sms, cudaStream_t stream) {
+    return launch_path<gemm::kIntScale, int8_t, true>(tm_w, p, num_sms, stream);
 }
 
 cudaError_t launch(const CUtensorMap& tm_w, const GemvParams& p, int path, int x_kind, int num_sms,

@@ -339,7 +339,9 @@ W4A8_API w4a8_status w4a8_gemm_intscale_asym(const int8_t* q_x, const float* s_a
  * P_g[m,n] = sum_{k in g} q_x[m,k] * w8[n,k]; y = acc * s_a[m] / alpha.
  * Arguments, precondition (now 127*127*group*max_n sum_g |S[g,n]| < 2^31),
  * workspace (w4a8_gemm_workspace_size with path 2), output and errors as in
- * w4a8_gemm_intscale.
+ * w4a8_gemm_intscale.  One or two tokens (three or four while w8 takes at
+ * most 32 MB), 256 <= K <= 16384, run the CUDA-core decode kernel on the
+ * 8-bit codes as stored, with no workspace; other shapes run the tiles.
  */
 W4A8_API w4a8_status w8a8_gemm_intscale(const int8_t* q_x, const float* s_a, const int8_t* w8, const int16_t* S,
                                int32_t alpha, int64_t M, int64_t N, int64_t K, int32_t group, void* y,

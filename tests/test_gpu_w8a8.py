@@ -78,6 +78,40 @@ def test_w8a8_gemm_parity(M, K, N):
     assert bgq.device_status() == 0
 
 
+# One to four tokens take the CUDA-core decode kernel (8-bit codes straight
+# from the ring, no unpack): ragged N, K with an odd number of 128-wide blocks,
+# the largest K, groups wider than a block, and four tokens on either side of
+# the weight-size rule that sends them to the tiles.
+W8_DECODE_CASES = [
+    # M, K, N, group
+    (1, 11008, 4096, 128),
+    (2, 1152, 264, 128),
+    (3, 4096, 1032, 256),
+    (4, 2048, 520, 512),
+    (2, 16384, 256, 128),
+    (4, 4096, 8192, 128),
+    (4, 4096, 8200, 128),
+]
+
+
+@pytest.mark.parametrize("M,K,N,group", W8_DECODE_CASES)
+def test_w8a8_decode_parity(M, K, N, group):
+    dev = _dev()
+    wl = workloads.make_linear(M, K, N, x_dtype="bf16", seed=7 * M + K + N)
+    x = torch.from_numpy(np.ascontiguousarray(wl.x)).to(dev).to(torch.bfloat16)
+    q, s = bgq.quantize_act_per_token(x)
+    pk = bgq.pack_w8_groupwise(torch.from_numpy(wl.w).to(dev), group=group, alpha=None)
+    ref = oracle.linear_intscale(wl.x, wl.w, group=group, alpha=None, out="f32", wbits=8)
+    assert pk["alpha"] == ref["alpha"]
+    if M <= 2 or N * K <= 32 << 20:  # the decode kernel: no workspace
+        assert bgq.gemm_workspace(M, N, K, group, 2, dev) is None
+    acc = bgq.w8a8_gemm_intscale(q, s, pk["w8"], pk["S"], pk["alpha"], group=group, out="i32")
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), ref["acc"])
+    y = bgq.w8a8_gemm_intscale(q, s, pk["w8"], pk["S"], pk["alpha"], group=group, out="f32")
+    _assert_close_f16(y.cpu().numpy(), ref["y64"])
+    assert bgq.device_status() == 0
+
+
 def test_w8a8_matches_dense_integer_product():
     # acc = qx @ (S * q) as one dense integer matmul, at a size with many split tiles
     dev = _dev()
