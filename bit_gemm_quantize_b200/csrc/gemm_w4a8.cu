@@ -171,14 +171,26 @@ struct Cfg {
     static constexpr int offY = offX + kSX * kXBytes;
     static constexpr int offSA = offY + kYBytes;
     static constexpr int offZ = offSA + BT * 4;                     // the tile's zero points (ZP)
-    static constexpr int offBar = offZ + (ZP ? BT * 4 : 0);
+    // integer scales of each weight slot's two K blocks (int16 [2][128]),
+    // copied with the packed box, for folding them into the operand: 128-token
+    // tiles only (narrow tiles accumulate a segment faster in several buffers,
+    // measured), and not on the asymmetric-token path (no room beside its zero
+    // points)
+    static constexpr bool kScaleRing = PATH == kIntScale && !W8 && !ZP && BT == 128;
+    static constexpr int kSSlotBytes = 2 * kTileN * 2;
+    static constexpr int offS = offZ + (ZP ? BT * 4 : 0);
+    static constexpr int offBar = offS + (kScaleRing ? kSW * kSSlotBytes : 0);
     static_assert(!ZP || PATH == kIntScale, "zero points are applied on the integer-scale path");
-    static constexpr int kBars = 2 * kSW + kSX + kSA + 2 * kSD + 2 * kAcc + 1;
+    static constexpr int kBars = 2 * kSW + kSX + kSA + 2 * kSD + 2 * kAcc + 2;
     static constexpr int offMisc = offBar + kBars * 8;
-    static constexpr int kSmemBytes = offMisc + 64 + 1024;  // + slack to align the base to 1024
+    // + up to 1024 bytes of slack to align the base to 1024 (the base of
+    // dynamic shared memory is 1024-aligned when nothing precedes it; the
+    // kernel checks that the slack it has covers the misalignment it sees)
+    static constexpr int kSmemBytes = offMisc + 64 + 1024 <= 227 * 1024 ? offMisc + 64 + 1024 : 227 * 1024;
+    static constexpr int kSlack = kSmemBytes - (offMisc + 64);
     static_assert(kXBytes % 2048 == 0, "token stage must hold whole 8-row swizzle atoms per k-block");
     static_assert(offY % 128 == 0, "TMA store source alignment");
-    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+    static_assert(kSlack >= 0, "shared memory");
     static_assert(kCtasPerSm == 1 || kSmemBytes * kCtasPerSm <= 227 * 1024, "shared memory for two CTAs per SM");
 };
 
@@ -320,6 +332,7 @@ struct Stage {
     int32_t n_tile, m_tile;
     int32_t kb;   // first K block (global index along K)
     int32_t nkb;  // 1 or 2
+    bool seg_first, seg_last;  // the stage opens / closes its segment
 };
 
 template <bool GR>
@@ -331,6 +344,7 @@ struct StageIter {
     template <typename P>
     __device__ StageIter(const P& p, const Part& pt, uint32_t b) : seg(p, pt, b), kbpg(p.kb_per_group) {}
     __device__ bool next(Stage& st) {
+        st.seg_first = false;
         while (kb >= kb_end) {
             Segment s;
             if (!seg.next(s)) return false;
@@ -339,6 +353,7 @@ struct StageIter {
             m_tile = s.m_tile;
             kb = s.g0 * kbpg;
             kb_end = s.g1 * kbpg;
+            st.seg_first = true;
         }
         st.e = e;
         st.n_tile = n_tile;
@@ -346,9 +361,49 @@ struct StageIter {
         st.kb = kb;
         st.nkb = (kb_end - kb) >= 2 ? 2 : 1;
         kb += st.nkb;
+        st.seg_last = kb >= kb_end;
         return true;
     }
 };
+
+// Folded integer scales.  When every integer scale S[g,n] a CTA meets lies in
+// [0, 16], S * q fits in int8 for every 4-bit code q in [-8, 7] (-8 * 16 =
+// -128, 7 * 16 = 112), so the unpack can write the operand S[g,n] * q[k,n]
+// instead of q: the MMAs then sum S * q * x over the whole segment in the
+// TMEM accumulator, which is the same integer as sum_g S[g,n] * P_g, and the
+// per-group drain disappears (one accumulator read per tile instead of one
+// per group).  This needs the scales to be integers: a float scale cannot be
+// folded into an int8 operand exactly.
+// Scales above kFoldMaxS (or negative) keep a CTA on the per-group drain:
+// S * q fits in int8 for every 4-bit code q in [-8, 7] up to S = 16.
+constexpr int kFoldMaxS = 16;
+
+// The largest of 8 int16 scales read as unsigned 16-bit values.
+__device__ __forceinline__ uint32_t scales_max_u16(uint4 v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t m = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0xFFFFu, w[i] >> 16));
+    return m;
+}
+
+// The CTA's choice, read by every role once the epilogue warps' scan of its
+// scales is complete (misc[4]: some scale out of range).
+__device__ __forceinline__ bool fold_decision(const uint32_t* misc) {
+    return *reinterpret_cast<const volatile uint32_t*>(&misc[4]) == 0u;
+}
+
+// S * q for 8 packed codes (low nibbles: K 0-3, high nibbles: K 4-7), as int8
+// bytes.  The offset code u = q + 8 in [0, 15] sits alone in its byte, so
+// u * S <= 240 and u * S + 128 - 8 S = S * q + 128 lies in [0, 240] for
+// 0 <= S <= 16: one multiply-add per 4 bytes with no carry between bytes
+// (k1 = (128 - 8 S) in every byte), and XOR 0x80 turns each byte from
+// excess-128 into two's complement.
+__device__ __forceinline__ uint2 unpack8_folded(uint32_t w, uint32_t s, uint32_t k1) {
+    const uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
+    const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+    return make_uint2((lo * s + k1) ^ 0x80808080u, (hi * s + k1) ^ 0x80808080u);
+}
 
 // Output scale of token m: s_a[m] / alpha (exact: 1/alpha is a power of two)
 // for the integer-scale path, s_a[m] for the float-scale path.
@@ -377,7 +432,15 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
     constexpr int SW = C::kSW, SX = C::kSX, SA = C::kSA, SD = C::kSD;
     constexpr int kEpiWarps = C::kEpiWarps;
     constexpr int HC = BT / (kEpiWarps / 4);  // columns per epilogue thread
-    extern __shared__ uint8_t smem_raw[];
+    // integer scales on 4-bit weights may be folded into the unpacked operand
+    constexpr bool kFoldable = C::kScaleRing;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    if (((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u) > uint32_t(C::kSlack)) {
+        // the layout would not fit behind the aligned base: refuse (no
+        // barrier, TMEM or copy has been touched yet)
+        if (threadIdx.x == 0) atomicExch(p.status, kStatusAlign);
+        return;
+    }
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::offBar);
     uint64_t* full_w = bars;              // W box landed (TMA transaction count)
@@ -389,7 +452,10 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
     uint64_t* tempty = sseen + SD;        // epilogue has read a TMEM accumulator buffer
     uint64_t* afull = tempty + kAcc;      // a group's MMAs into an accumulator buffer are complete
     uint64_t* mma_done = afull + kAcc;
-    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::offMisc);  // [0] tmem base [1] abort [2] last
+    uint64_t* fold_ready = mma_done + 1;  // the epilogue warps have checked the CTA's scales (misc[4])
+    // [0] tmem base [1] abort [2] last [3] early combine [4] nonzero: some
+    // scale of the CTA's steps cannot be folded
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::offMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
     const int warp = threadIdx.x >> 5;
@@ -411,8 +477,10 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             mbar_init(&afull[s], 1);
         }
         mbar_init(&mma_done[0], 1);
+        mbar_init(fold_ready, kEpiWarps);
         misc[1] = 0;
         misc[2] = 0;
+        misc[4] = 0;
         fence_mbar_init();
         prefetch_tensormap(&tm_w);
         prefetch_tensormap(&tm_x);
@@ -467,9 +535,33 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                                     &full_w[slot.idx]);
             } else {
                 // one 128 x 128 B box = two K blocks (a lone last block over-reads 64 B per row: harmless)
-                mbar_arrive_expect_tx_one(&full_w[slot.idx], C::kWBytes);
+                // and, for folding, the K blocks' rows of integer scales of the
+                // tile's columns (columns < N; a 16-byte aligned array only:
+                // otherwise the scales are not folded and not read here)
+                uint32_t s_bytes = 0u;
+                const int16_t* Sx = nullptr;
+                if constexpr (C::kScaleRing) {
+                    Sx = p.S;
+                    if constexpr (GR) Sx = static_cast<const int16_t*>(p.grp_scales[st.e]);
+                    const int64_t n0 = int64_t(st.n_tile) * kTileN;
+                    const int64_t cols = p.N - n0 < kTileN ? p.N - n0 : kTileN;
+                    if ((reinterpret_cast<uintptr_t>(Sx) & 15u) == 0) s_bytes = uint32_t(cols * 2);
+                }
+                mbar_arrive_expect_tx_one(&full_w[slot.idx], C::kWBytes + uint32_t(st.nkb) * s_bytes);
                 tma_load_2d_one(smem + C::offW + slot.idx * C::kWBytes, wmap, st.kb * (kBlockK / 2),
                                 st.n_tile * kTileN, &full_w[slot.idx]);
+                if constexpr (C::kScaleRing) {
+                    if (s_bytes != 0u && lane == 0) {
+                        const int32_t kbpg = p.kb_per_group;
+                        for (int j = 0; j < st.nkb; ++j) {
+                            const int32_t g = kbpg == 1 ? st.kb + j : (st.kb + j) / kbpg;
+                            bulk_load(smem + C::offS + slot.idx * C::kSSlotBytes + j * (kTileN * 2),
+                                      Sx + int64_t(g) * p.N + int64_t(st.n_tile) * kTileN, s_bytes,
+                                      &full_w[slot.idx]);
+                        }
+                    }
+                    __syncwarp();
+                }
             }
             w_issued |= 1u << slot.idx;
             w_par = (w_par & ~(1u << slot.idx)) | (slot.phase << slot.idx);
@@ -584,6 +676,13 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
         int32_t kin = 0;  // position of the next K block inside its group (segments start on group boundaries)
         const uint32_t x_lo0 = smem_desc_sw128_lo(smem_u32(smem + C::offX));
         const uint32_t w_lo0 = smem_desc_sw128_lo(smem_u32(smem + C::offW));
+        // folded scales: one accumulator buffer per segment (its first MMA
+        // overwrites, its last K block commits), no per-group commits
+        bool fold = false;
+        if constexpr (kFoldable) {
+            ok = mbar_wait_warp(fold_ready, 0u, abort_flag, p.status, p.wait_limit);
+            fold = fold_decision(misc);
+        }
         while (ok && it.next(st)) {
             // the A operand: the unpacked slot in TMEM, or the int8 weight box itself
             const bool a_ready = C::kW8 ? mbar_wait_warp(&full_w[rw.idx], rw.phase, abort_flag, p.status, p.wait_limit)
@@ -599,9 +698,9 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 if (j >= st.nkb) break;
-                const bool first = G1 || (kin == 0);
-                const bool last = G1 || (kin == p.kb_per_group - 1);
-                if constexpr (!G1) kin = last ? 0 : kin + 1;
+                const bool first = fold ? (st.seg_first && j == 0) : (G1 || (kin == 0));
+                const bool last = fold ? (st.seg_last && j == st.nkb - 1) : (G1 || (kin == p.kb_per_group - 1));
+                if constexpr (!G1) kin = (last || fold) ? 0 : kin + 1;
                 if (first) {
                     if (!mbar_wait_warp(&tempty[rt.idx], rt.phase ^ 1u, abort_flag, p.status, p.wait_limit)) {
                         ok = false;
@@ -625,12 +724,12 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                                           (first && k == 0) ? 0u : 1u);
                 }
                 if (last) {
-                    if constexpr (C::kGroupCommit) mma_commit_one(&afull[rt.idx]);
+                    if (C::kGroupCommit || fold) mma_commit_one(&afull[rt.idx]);
                     rt.advance(kAcc);
                 }
             }
             if (!ok) break;
-            if constexpr (!C::kGroupCommit) {
+            if (!C::kGroupCommit && !fold) {
                 // the epilogue waits on stage-done phases: it must have seen the
                 // previous phase of this slot before it is committed again
                 if (!mbar_wait_warp(&sseen[rd.idx], rd.phase ^ 1u, abort_flag, p.status, p.wait_limit)) {
@@ -668,6 +767,11 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
         Stage st;
         bool ok = true;
         const uint32_t lane_base = tmem_base + (uint32_t(quarter * 32) << 16);
+        bool fold = false;
+        if constexpr (kFoldable) {
+            ok = mbar_wait_warp(fold_ready, 0u, abort_flag, p.status, p.wait_limit);
+            fold = fold_decision(misc);
+        }
         while (ok && it.next(st)) {
             if (!mbar_wait_warp(&full_w[rw.idx], rw.phase, abort_flag, p.status, p.wait_limit)) {
                 ok = false;
@@ -678,6 +782,16 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
 #pragma unroll
             for (int c = 0; c < 8; ++c)
                 if (c < 4 * st.nkb) v[c] = *reinterpret_cast<const uint4*>(wrow + ((c ^ sw) << 4));
+            // folding: this row's integer scales of the stage's K blocks, copied
+            // with the box (a column past N: 0, its weights read as zero)
+            uint32_t sk0 = 0u, sk1 = 0u;
+            if constexpr (C::kScaleRing) {
+                if (fold && int64_t(st.n_tile) * kTileN + r < p.N) {
+                    const int16_t* srow = reinterpret_cast<const int16_t*>(smem + C::offS + rw.idx * C::kSSlotBytes);
+                    sk0 = uint32_t(int32_t(srow[r]));
+                    sk1 = uint32_t(int32_t(srow[kTileN + r]));
+                }
+            }
             // the packed box may be refilled once every warp has read it (the
             // arrive releases this thread's loads above)
             __syncwarp();
@@ -696,11 +810,23 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
             for (int j = 0; j < 2; ++j) {
                 if (j < st.nkb) {
                     uint32_t o[32];
+                    const uint32_t fs = j == 0 ? sk0 : sk1;
+                    const uint32_t k1 = (128u - 8u * fs) * 0x01010101u;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const uint4 w = v[4 * j + c];
-                        const uint2 o0 = unpack8<C::kX16>(w.x), o1 = unpack8<C::kX16>(w.y);
-                        const uint2 o2 = unpack8<C::kX16>(w.z), o3 = unpack8<C::kX16>(w.w);
+                        uint2 o0, o1, o2, o3;
+                        if (fold) {
+                            o0 = unpack8_folded(w.x, fs, k1);
+                            o1 = unpack8_folded(w.y, fs, k1);
+                            o2 = unpack8_folded(w.z, fs, k1);
+                            o3 = unpack8_folded(w.w, fs, k1);
+                        } else {
+                            o0 = unpack8<C::kX16>(w.x);
+                            o1 = unpack8<C::kX16>(w.y);
+                            o2 = unpack8<C::kX16>(w.z);
+                            o3 = unpack8<C::kX16>(w.w);
+                        }
                         o[8 * c + 0] = o0.x;
                         o[8 * c + 1] = o0.y;
                         o[8 * c + 2] = o1.x;
@@ -723,15 +849,62 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
       }
     } else {
         // ---------------------------------------------------------- epilogue
-        griddep_wait();  // s_a, y and the workspace may be in use by the previous kernel
         const int ew = warp - C::kFirstEpiWarp;
+        bool fold = false;
+        bool fold_seen = true;  // false: the wait for the other warps' checks gave up
+        if constexpr (kFoldable) {
+            // Does this CTA fold its scales?  Every S[g, n] of its steps (the
+            // group rows of its segments, 128 columns each) must lie in
+            // [0, kFoldMaxS].  Scales are written by the weight packing, never
+            // by a kernel that lets its successor start early, so this runs
+            // before waiting for the previous kernel, like the first weight
+            // copies.  A scale array that is not 16-byte aligned (grouped calls
+            // take any even address) is not folded.
+            const int nthr = kEpiWarps * 32;
+            const int t = ew * 32 + lane;
+            SegmentIter<GR> si(p, pt, b);
+            Segment s2;
+            bool bad = false;
+            int32_t base = 0;  // steps of the earlier segments, modulo nthr
+            const int64_t N = p.N;
+            while (si.next(s2)) {
+                const int16_t* Sx = p.S;
+                if constexpr (GR) Sx = static_cast<const int16_t*>(p.grp_scales[s2.e]);
+                if ((reinterpret_cast<uintptr_t>(Sx) & 15u) != 0) bad = true;
+                const int64_t n0 = int64_t(s2.n_tile) * kTileN;
+                const int32_t steps = s2.g1 - s2.g0;
+                int32_t c = t - base;
+                if (c < 0) c += nthr;
+                if (!bad) {
+                    for (; c < steps; c += nthr) {
+                        const int16_t* row = Sx + int64_t(s2.g0 + c) * N + n0;
+                        uint32_t mx = 0u;
+#pragma unroll
+                        for (int q = 0; q < kTileN / 8; ++q) {
+                            if (n0 + 8 * q < N) {
+                                const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + 8 * q));
+                                mx = max(mx, scales_max_u16(v));  // a negative scale reads as >= 2^15
+                            }
+                        }
+                        if (mx > uint32_t(kFoldMaxS)) bad = true;
+                    }
+                }
+                base = (base + steps) % nthr;
+            }
+            if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&misc[4], 1u);
+            __syncwarp();
+            mbar_arrive_one(fold_ready);  // lane 0 (the elected lane) made the update above
+            fold_seen = mbar_wait_warp(fold_ready, 0u, abort_flag, p.status, p.wait_limit);
+            fold = fold_decision(misc);
+        }
+        griddep_wait();  // s_a, y and the workspace may be in use by the previous kernel
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int half = ew >> 2;      // which part of the BT columns
         const int r = quarter * 32 + lane;
         Ring rt, rd;
         SegmentIter<GR> it(p, pt, b);
         Segment sg;
-        bool ok = true;
+        bool ok = fold_seen;
         const int32_t kbpg = p.kb_per_group;
         const int32_t G = int32_t(p.G);
         while (ok && it.next(sg)) {
@@ -810,7 +983,31 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                     }
                 }
             }
-            if constexpr (kLean) {
+            if (fold) {
+                // Folded scales: the segment's MMAs summed S * q * x into one
+                // buffer, committed after its last K block: that is the
+                // segment's accumulator, read once.
+                if (!mbar_wait_warp(&afull[rt.idx], rt.phase, abort_flag, p.status, p.wait_limit)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t lane_cols =
+                    tmem_base + (uint32_t(quarter * 32) << 16) + C::kAccCol0 + uint32_t(rt.idx * BT + half * HC);
+                constexpr int CH = HC < 32 ? HC : 32;
+#pragma unroll
+                for (int c0 = 0; c0 < HC; c0 += CH) {
+                    uint32_t v[CH];
+                    tmem_load<CH>(lane_cols + uint32_t(c0), v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q = 0; q < CH; ++q) acc[c0 + q] = int32_t(v[q]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                mbar_arrive_one(&tempty[rt.idx]);
+                rt.advance(kAcc);
+            } else if constexpr (kLean) {
                 // One group per K block, each committed to its own accumulator
                 // buffer: wait for the group's MMAs, load this thread's HC
                 // columns of P_g, hand the buffer back, and add

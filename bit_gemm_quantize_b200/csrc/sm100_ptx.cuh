@@ -11,6 +11,7 @@ namespace w4a8 {
 
 constexpr int kStatusTimeout = 8;  // mirrors W4A8_ERR_TIMEOUT
 constexpr int kStatusInvalidArg = 1;  // mirrors W4A8_ERR_INVALID_ARG
+constexpr int kStatusAlign = 3;  // mirrors W4A8_ERR_ALIGN
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
