@@ -31,7 +31,10 @@
  *    means nothing was launched.  No C++ exception crosses the ABI.
  *  - Kernels bound every wait; a wait that runs out (about one second) makes
  *    the kernel return early and records W4A8_ERR_TIMEOUT in a device status
- *    word that w4a8_device_status() reads.
+ *    word that w4a8_device_status() reads.  The tcgen05 GEMM kernels also
+ *    record W4A8_ERR_ALIGN there, and return at once, if the device's
+ *    dynamic shared memory does not start 1024-byte aligned (their layout
+ *    needs it; not seen on B200).
  *  - The GEMMs run a persistent grid of at most one CTA per resident slot
  *    (SMs x CTAs per SM) and split the (tile, group) steps into one range per
  *    CTA.  A tile cut by two ranges is finished by one of its CTAs, which
@@ -253,6 +256,10 @@ W4A8_API int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32
  *            NULL when that size is 0), zero-filled, see above
  * Precondition (established by pack_w4_groupwise): the worst-case accumulator
  * 127*7*group*max_n sum_g |S[g,n]| stays below 2^31.
+ * With 128-token tiles, a CTA whose scales S[g,n] all lie in [0, 16] writes
+ * S*q (exact in int8 for every 4-bit code) as the MMA operand and sums the
+ * whole K in one accumulator: the same acc, with no per-group multiply.
+ * This needs S 16-byte aligned (checked above).
  */
 W4A8_API w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, const uint8_t* w_packed,
                                const int16_t* S, int32_t alpha, int64_t M, int64_t N, int64_t K,
