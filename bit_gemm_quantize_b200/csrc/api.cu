@@ -264,6 +264,7 @@ w4a8_status run_gemm(int path, const int8_t* q_x, const float* s_a, const uint8_
     w4a8::gemm::Params p{};
     p.s_a = s_a;
     p.S = S;
+    p.wq = w8 ? nullptr : w_packed;
     p.s_g = s_g;
     p.y = y;
     p.ws_part = ws_part;

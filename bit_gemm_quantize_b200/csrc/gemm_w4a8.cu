@@ -375,8 +375,19 @@ struct StageIter {
 // per group).  This needs the scales to be integers: a float scale cannot be
 // folded into an int8 operand exactly.
 // Scales above kFoldMaxS (or negative) keep a CTA on the per-group drain:
-// S * q fits in int8 for every 4-bit code q in [-8, 7] up to S = 16.
+// S * q fits in int8 for every 4-bit code q in [-8, 7] up to S = 16, and up
+// to S = kFoldMaxS7 for a group whose codes avoid -8 (codes in [-7, 7], the
+// default packing).
 constexpr int kFoldMaxS = 16;
+constexpr int kFoldMaxS7 = 18;
+
+// Whether any of 8 packed codes is -8 (nibble 1000): bit 3 set and bits 0-2
+// clear (adding 7 to the low three bits sets bit 3 unless they are zero; no
+// carry leaves a nibble).
+__device__ __forceinline__ bool has_code_minus8(uint32_t w) {
+    const uint32_t low_nonzero = ((w & 0x77777777u) + 0x77777777u) & 0x88888888u;
+    return (w & 0x88888888u & ~low_nonzero) != 0u;
+}
 
 // The largest of 8 int16 scales read as unsigned 16-bit values.
 __device__ __forceinline__ uint32_t scales_max_u16(uint4 v) {
@@ -394,11 +405,12 @@ __device__ __forceinline__ bool fold_decision(const uint32_t* misc) {
 }
 
 // S * q for 8 packed codes (low nibbles: K 0-3, high nibbles: K 4-7), as int8
-// bytes.  The offset code u = q + 8 in [0, 15] sits alone in its byte, so
-// u * S <= 240 and u * S + 128 - 8 S = S * q + 128 lies in [0, 240] for
-// 0 <= S <= 16: one multiply-add per 4 bytes with no carry between bytes
-// (k1 = (128 - 8 S) in every byte), and XOR 0x80 turns each byte from
-// excess-128 into two's complement.
+// bytes.  With the offset code u = q + 8 in [0, 15] in each byte, the 32-bit
+// word * S + (128 - 8 S) * 0x01010101 equals sum_i (S * q_i + 128) * 256^i
+// exactly (mod 2^32, k1 wrapping for S > 16): when every S * q_i lies in
+// [-128, 127] each coefficient is a byte in [0, 255], so the result's bytes
+// are S * q_i + 128 (any carries of the intermediate product cancel), and
+// XOR 0x80 turns each byte from excess-128 into two's complement.
 __device__ __forceinline__ uint2 unpack8_folded(uint32_t w, uint32_t s, uint32_t k1) {
     const uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
     const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
@@ -855,7 +867,10 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
         if constexpr (kFoldable) {
             // Does this CTA fold its scales?  Every S[g, n] of its steps (the
             // group rows of its segments, 128 columns each) must lie in
-            // [0, kFoldMaxS].  Scales are written by the weight packing, never
+            // [0, kFoldMaxS], or in [0, kFoldMaxS7] with no code -8 in the
+            // group (read from the packed codes of those few columns; a
+            // grouped call does not pass them and folds only up to 16).
+            // Scales are written by the weight packing, never
             // by a kernel that lets its successor start early, so this runs
             // before waiting for the previous kernel, like the first weight
             // copies.  A scale array that is not 16-byte aligned (grouped calls
@@ -877,16 +892,41 @@ __global__ void __launch_bounds__(Cfg<BT, PATH, W8, ZP>::kThreads, Cfg<BT, PATH,
                 if (c < 0) c += nthr;
                 if (!bad) {
                     for (; c < steps; c += nthr) {
-                        const int16_t* row = Sx + int64_t(s2.g0 + c) * N + n0;
+                        const int32_t g = s2.g0 + c;
+                        const int16_t* row = Sx + int64_t(g) * N + n0;
+                        uint4 sv[kTileN / 8];
                         uint32_t mx = 0u;
 #pragma unroll
                         for (int q = 0; q < kTileN / 8; ++q) {
-                            if (n0 + 8 * q < N) {
-                                const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + 8 * q));
-                                mx = max(mx, scales_max_u16(v));  // a negative scale reads as >= 2^15
+                            sv[q] = make_uint4(0u, 0u, 0u, 0u);
+                            if (n0 + 8 * q < N) sv[q] = __ldg(reinterpret_cast<const uint4*>(row + 8 * q));
+                        }
+#pragma unroll
+                        for (int q = 0; q < kTileN / 8; ++q)
+                            mx = max(mx, scales_max_u16(sv[q]));  // a negative scale reads as >= 2^15
+                        if (mx > uint32_t(kFoldMaxS7) || (mx > uint32_t(kFoldMaxS) && (GR || p.wq == nullptr))) {
+                            bad = true;
+                        } else if (mx > uint32_t(kFoldMaxS)) {
+                            // scales of 17 or 18: their groups must hold no code -8
+                            const int64_t half_k = int64_t(p.G) * p.kb_per_group * (kBlockK / 2);  // K / 2
+                            const int32_t gbytes = p.kb_per_group * (kBlockK / 2);                  // group / 2
+                            for (int q = 0; q < kTileN / 8 && !bad; ++q) {
+                                const uint32_t w4[4] = {sv[q].x, sv[q].y, sv[q].z, sv[q].w};
+                                for (int e = 0; e < 8 && !bad; ++e) {
+                                    const uint32_t sval = (w4[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+                                    if (sval <= uint32_t(kFoldMaxS)) continue;
+                                    const uint8_t* cp = p.wq + (n0 + 8 * q + e) * half_k + int64_t(g) * gbytes;
+                                    for (int o = 0; o < gbytes; o += 16) {
+                                        const uint4 cw = __ldg(reinterpret_cast<const uint4*>(cp + o));
+                                        if (has_code_minus8(cw.x) || has_code_minus8(cw.y) || has_code_minus8(cw.z) ||
+                                            has_code_minus8(cw.w)) {
+                                            bad = true;
+                                            break;
+                                        }
+                                    }
+                                }
                             }
                         }
-                        if (mx > uint32_t(kFoldMaxS)) bad = true;
                     }
                 }
                 base = (base + steps) % nthr;

@@ -15,6 +15,7 @@ enum OutType { kOutF32 = 0, kOutF16 = 1, kOutI32 = 3 };
 struct Params {
     const float* s_a;    // [M] token scales
     const int16_t* S;    // [G, N] integer group scales (integer-scale path)
+    const uint8_t* wq;   // [N, K/2] packed codes, read when a scale of 17 or 18 may be folded (null: never)
     const float* s_g;    // [G, N] float group scales (float-scale path)
     void* y;             // [M, N] output
     int32_t* ws_part;    // [grid][128 * BT] partial sums of split tiles (one per contributing CTA)

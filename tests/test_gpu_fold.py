@@ -1,9 +1,9 @@
 """Integer scales folded into the unpacked weight operand.
 
 A CTA of the tile kernel (128-token tiles) whose integer scales all lie in
-[0, 16] writes S * q as the MMA operand (then in int8 for every 4-bit code)
-and accumulates the whole segment in TMEM; any other CTA drains each group
-and multiplies by S.  The sum is the same integer either way, so every case
+[0, 16] (or in [0, 18] for groups without the code -8) writes S * q as the
+MMA operand (then in int8) and accumulates the whole segment in TMEM; any
+other CTA drains each group and multiplies by S.  The sum is the same integer either way, so every case
 here is bit-exact against the oracle's accumulators.
 
 The weights are built so that quantizing them gives chosen codes and scales
@@ -97,17 +97,18 @@ def test_folded_scales_bitexact(M, K, N, group, full_range):
 
 @pytest.mark.parametrize("M,K,N,group", [(8, 1024, 1032, 128), (300, 2048, 776, 256), (1024, 4096, 1024, 128)])
 def test_folded_and_drained_ctas_mixed(M, K, N, group):
-    """Columns 256..383 carry scales of 17 to 200: the CTAs that meet them
-    drain every group, the others fold; tiles split between the two kinds
-    combine."""
+    """Columns 256..383 carry scales of 17 to 200 in groups that all hold the
+    code -8: the CTAs that meet them drain every group, the others fold;
+    tiles split between the two kinds combine."""
     _check(M, K, N, group, True, seed=5 * M + N, band=(256, 384))
 
 
-@pytest.mark.parametrize("M,K,N", [(130, 1024, 520), (1024, 4096, 2048)])
-@pytest.mark.parametrize("big", [17, 40, 200])
+@pytest.mark.parametrize("M,K,N", [(130, 1024, 520), (512, 2048, 1024)])
+@pytest.mark.parametrize("big", [17, 18, 40, 200])
 def test_a_few_scales_above_16(M, K, N, big):
-    """A few groups with one scale above 16: the CTAs that meet them drain,
-    the others fold."""
+    """A few groups with one scale above 16 and codes in [-7, 7]: scales of
+    17 and 18 still fold (S * q stays in int8 without the code -8); the CTAs
+    that meet a larger one drain, the others fold."""
     dev = _dev()
     rng = np.random.default_rng(big + M)
     group = 128
