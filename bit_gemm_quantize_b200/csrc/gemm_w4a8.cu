@@ -25,6 +25,11 @@
 //   accf += s_g * float(P_g)); after the tile's last group y = acc * s_a[m]
 //   / alpha (or accf * s_a[m]), staged in shared memory and written by one
 //   TMA tensor store.
+// Folded integer scales (128-token tiles, when every scale the CTA meets is
+// small enough for S * q to stay in int8): the unpack writes S[g,n] * q
+// instead of q (the stage's scale rows travel with the packed box), the MMAs
+// sum the whole segment in one TMEM buffer, and the epilogue reads it once:
+// the same integer acc with no per-group drain.
 // Keeping the unpacked operand in TMEM instead of shared memory saves two of
 // its passes through the shared-memory port (the unpack's store and the MMA's
 // read, 64 KB per stage), which bound small-token-tile MMAs at about 40
