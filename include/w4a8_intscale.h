@@ -256,10 +256,10 @@ W4A8_API int64_t w4a8_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int32
  *            NULL when that size is 0), zero-filled, see above
  * Precondition (established by pack_w4_groupwise): the worst-case accumulator
  * 127*7*group*max_n sum_g |S[g,n]| stays below 2^31.
- * With 128-token tiles, a CTA whose scales S[g,n] all lie in [0, 16] writes
- * S*q (exact in int8 for every 4-bit code) as the MMA operand and sums the
- * whole K in one accumulator: the same acc, with no per-group multiply.
- * This needs S 16-byte aligned (checked above).
+ * With 128-token tiles, a CTA whose scales S[g,n] all lie in [0, 16] (or
+ * reach 17 or 18 only in groups without the code -8) writes S*q (then exact
+ * in int8) as the MMA operand and sums the whole K in one accumulator: the
+ * same acc, with no per-group multiply.
  */
 W4A8_API w4a8_status w4a8_gemm_intscale(const int8_t* q_x, const float* s_a, const uint8_t* w_packed,
                                const int16_t* S, int32_t alpha, int64_t M, int64_t N, int64_t K,
